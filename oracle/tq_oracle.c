@@ -1,0 +1,854 @@
+/*
+ * tq_oracle.c -- plain, slow CPU reference for TurboQuant-style KV-cache
+ * compression, compressed-cache decode attention and compressed top-k search.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, imports or
+ * runs this file; only the tests, the package's smoke check and the CPU
+ * baseline of the benchmark do.  It shares no code with the CUDA library.
+ *
+ * Everything is computed in double precision.  Where a floating-point value
+ * decides an integer (a quantiser code, a sign bit) the decision is taken in
+ * the precision stated beside it, which is also the precision the GPU path
+ * uses for that decision.
+ *
+ * Sources (web pages on the subject; sections as titled on each page):
+ *  [TQ]   "TurboQuant" summary and discussion, de.news.hada.io topic 27867:
+ *         "Funktionsweise von TurboQuant" (random rotation, then a standard
+ *         per-coordinate quantiser; then 1-bit QJL on the residual),
+ *         "QJL: Eine 1-Bit-Methode ohne Overhead" (JL transform, sign bits,
+ *         estimator pairing a full-precision query with 1-bit data),
+ *         the discussion's note that Lloyd-Max boundaries/reconstruction
+ *         values are used after the rotation, and "Leistung bei der
+ *         Vektorsuche" (inner-product search, top-k).
+ *  [EXP]  "Die KV-Cache-Optimierung von Google erklaert", chatgpz.de:
+ *         "Stufe 1: Die zufaellige Rotation", "Stufe 2: ... (quantisierte JL)"
+ *         (unbiased estimator).
+ *  [MON]  "Monarch v3: NES-inspiriertes KV-Paging", openclawradar.com:
+ *         "Wie es funktioniert" (hot full-precision window, cold compressed
+ *         region) and "Vereinfachte Decode-Schleife" (hot and cold scores,
+ *         softmax, aggregation).
+ *
+ * Readings taken where the pages are silent (each also listed in the design doc):
+ *  - rotation: dense Haar-orthogonal matrix = Q of a QR factorisation of a
+ *    Gaussian matrix with diag(R) made positive;
+ *  - quantiser: Lloyd-Max for the exact marginal of one coordinate of a
+ *    uniform point on the unit sphere of R^d; a vector is normalised by its
+ *    stored fp16 norm; sign-magnitude codes;
+ *  - QJL: S has iid standard-normal entries rounded to fp16; estimator
+ *    <q,r> ~ sqrt(pi/2)/m * |r| * <S q, sign(S r)>;
+ *  - attention: one softmax over hot and cold tokens on every step.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define OR_API __attribute__((visibility("default")))
+
+/* ------------------------------------------------------------------------ */
+/* Random numbers: SplitMix64 (Steele, Lea & Flood, OOPSLA 2014) giving     */
+/* 53-bit uniforms, and the Box-Muller transform (1958) using both outputs. */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+  uint64_t state;
+  int have_spare;
+  double spare;
+} or_rng;
+
+static void rng_seed(or_rng* g, uint64_t seed) {
+  g->state = seed;
+  g->have_spare = 0;
+  g->spare = 0.0;
+}
+
+static uint64_t rng_u64(or_rng* g) {
+  g->state += 0x9E3779B97F4A7C15ULL;
+  uint64_t z = g->state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+static double rng_uniform(or_rng* g) { /* in [0, 1) */
+  return (double)(rng_u64(g) >> 11) * 0x1.0p-53;
+}
+
+static double rng_normal(or_rng* g) {
+  if (g->have_spare) {
+    g->have_spare = 0;
+    return g->spare;
+  }
+  double u1 = 1.0 - rng_uniform(g); /* (0, 1]: log is finite */
+  double u2 = rng_uniform(g);
+  double rad = sqrt(-2.0 * log(u1));
+  double ang = 2.0 * M_PI * u2;
+  g->spare = rad * sin(ang);
+  g->have_spare = 1;
+  return rad * cos(ang);
+}
+
+OR_API void or_normals(uint64_t seed, int64_t count, double* out) {
+  or_rng g;
+  rng_seed(&g, seed);
+  for (int64_t i = 0; i < count; ++i) out[i] = rng_normal(&g);
+}
+
+OR_API void or_uniforms(uint64_t seed, int64_t count, double* out) {
+  or_rng g;
+  rng_seed(&g, seed);
+  for (int64_t i = 0; i < count; ++i) out[i] = rng_uniform(&g);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Rounding to fp32 and fp16 (round to nearest, ties to even).              */
+/* ------------------------------------------------------------------------ */
+static double round_f32(double x) { return (double)(float)x; }
+
+OR_API double or_round_f16(double x) {
+  if (x == 0.0 || !isfinite(x)) return x;
+  double a = fabs(x);
+  if (a >= 65520.0) return copysign(INFINITY, x); /* beyond max + half ulp */
+  int e;
+  frexp(a, &e); /* a = f * 2^e, f in [0.5, 1) */
+  int lead = e - 1; /* a in [2^lead, 2^(lead+1)) */
+  if (lead < -14) lead = -14; /* subnormal range: fixed spacing 2^-24 */
+  double ulp = ldexp(1.0, lead - 10);
+  double q = nearbyint(a / ulp); /* exact quotient; default mode = ties-even */
+  return copysign(q * ulp, x);
+}
+
+/* bit pattern of a value that is already exactly representable in fp16 */
+static uint16_t f16_bits(double v) {
+  uint16_t sign = signbit(v) ? 0x8000u : 0u;
+  double a = fabs(v);
+  if (a == 0.0) return sign;
+  if (isinf(a)) return (uint16_t)(sign | 0x7C00u);
+  if (isnan(a)) return 0x7E00u;
+  if (a < 0x1.0p-14) { /* subnormal: a = mant * 2^-24 */
+    return (uint16_t)(sign | (uint16_t)(a * 0x1.0p24));
+  }
+  int e;
+  double f = frexp(a, &e); /* a = f*2^e, f in [0.5,1) -> 1.m * 2^(e-1) */
+  int biased = (e - 1) + 15;
+  uint16_t mant = (uint16_t)((f * 2.0 - 1.0) * 1024.0);
+  return (uint16_t)(sign | (uint16_t)(biased << 10) | mant);
+}
+
+static double f16_value(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int ex = (h >> 10) & 0x1F;
+  int mant = h & 0x3FF;
+  double v;
+  if (ex == 0)
+    v = ldexp((double)mant, -24);
+  else if (ex == 31)
+    v = mant ? NAN : INFINITY;
+  else
+    v = ldexp(1.0 + mant / 1024.0, ex - 15);
+  return sign ? -v : v;
+}
+
+OR_API uint16_t or_f16_bits(double v) { return f16_bits(or_round_f16(v)); }
+OR_API double or_f16_value(uint16_t h) { return f16_value(h); }
+
+/* ------------------------------------------------------------------------ */
+/* Random rotation [TQ "Funktionsweise", EXP "Stufe 1"]:                    */
+/* G (d x d, filled row by row from the normal stream 2*seed) = Q R by      */
+/* Householder reflections; Pi = Q diag(sign(R_ii)).  x_rot = Pi x.         */
+/* ------------------------------------------------------------------------ */
+OR_API int or_rotation(int d, uint64_t seed, double* pi /* d*d row-major */) {
+  double* a = (double*)malloc(sizeof(double) * d * d); /* becomes R */
+  double* q = (double*)malloc(sizeof(double) * d * d); /* accumulates Q */
+  double* v = (double*)malloc(sizeof(double) * d);
+  if (!a || !q || !v) {
+    free(a); free(q); free(v);
+    return -1;
+  }
+  or_rng g;
+  rng_seed(&g, 2ULL * seed);
+  for (int i = 0; i < d * d; ++i) a[i] = rng_normal(&g);
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) q[i * d + j] = (i == j) ? 1.0 : 0.0;
+
+  for (int k = 0; k < d - 1; ++k) {
+    /* Householder vector for column k, rows k..d-1 */
+    double norm = 0.0;
+    for (int i = k; i < d; ++i) norm += a[i * d + k] * a[i * d + k];
+    norm = sqrt(norm);
+    if (norm == 0.0) continue;
+    double alpha = (a[k * d + k] > 0.0) ? -norm : norm;
+    for (int i = 0; i < d; ++i) v[i] = 0.0;
+    for (int i = k; i < d; ++i) v[i] = a[i * d + k];
+    v[k] -= alpha;
+    double vv = 0.0;
+    for (int i = k; i < d; ++i) vv += v[i] * v[i];
+    if (vv == 0.0) continue;
+    /* A <- H A, H = I - 2 v v^T / (v^T v) */
+    for (int j = 0; j < d; ++j) {
+      double dot = 0.0;
+      for (int i = k; i < d; ++i) dot += v[i] * a[i * d + j];
+      double f = 2.0 * dot / vv;
+      for (int i = k; i < d; ++i) a[i * d + j] -= f * v[i];
+    }
+    /* Q <- Q H */
+    for (int i = 0; i < d; ++i) {
+      double dot = 0.0;
+      for (int j = k; j < d; ++j) dot += q[i * d + j] * v[j];
+      double f = 2.0 * dot / vv;
+      for (int j = k; j < d; ++j) q[i * d + j] -= f * v[j];
+    }
+  }
+  /* Pi = Q diag(sign(R_jj)) */
+  for (int j = 0; j < d; ++j) {
+    double s = (a[j * d + j] < 0.0) ? -1.0 : 1.0;
+    for (int i = 0; i < d; ++i) pi[i * d + j] = q[i * d + j] * s;
+  }
+  free(a); free(q); free(v);
+  return 0;
+}
+
+/* QJL matrix S (m x d): normal stream 2*seed+1, row-major, each entry
+ * rounded to the nearest fp16 value [TQ "QJL"; rounding is a reading]. */
+OR_API void or_qjl_matrix(int m, int d, uint64_t seed, double* s) {
+  or_rng g;
+  rng_seed(&g, 2ULL * seed + 1ULL);
+  for (int i = 0; i < m * d; ++i) s[i] = or_round_f16(rng_normal(&g));
+}
+
+/* ------------------------------------------------------------------------ */
+/* Lloyd-Max codebook for the coordinate marginal of a uniform unit vector  */
+/* [TQ discussion: Lloyd-Max boundaries and reconstruction values after the */
+/* rotation].  f(x) = C_d (1-x^2)^((d-3)/2) on [-1, 1],                     */
+/* C_d = Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2)).                            */
+/* ------------------------------------------------------------------------ */
+#define GL_N 24
+static double gl_x[GL_N], gl_w[GL_N];
+static int gl_ready = 0;
+
+/* Gauss-Legendre nodes: roots of P_n by Newton's method, w = 2/((1-x^2)P_n'^2) */
+static void gl_init(void) {
+  if (gl_ready) return;
+  int n = GL_N;
+  for (int i = 0; i < n; ++i) {
+    double x = cos(M_PI * (i + 0.75) / (n + 0.5));
+    double dp = 0.0;
+    for (int it = 0; it < 100; ++it) {
+      double p0 = 1.0, p1 = x;
+      for (int k = 2; k <= n; ++k) {
+        double p2 = ((2.0 * k - 1.0) * x * p1 - (k - 1.0) * p0) / k;
+        p0 = p1;
+        p1 = p2;
+      }
+      dp = n * (x * p1 - p0) / (x * x - 1.0);
+      double dx = p1 / dp;
+      x -= dx;
+      if (fabs(dx) < 1e-16) break;
+    }
+    /* recompute derivative at the converged node */
+    double p0 = 1.0, p1 = x;
+    for (int k = 2; k <= n; ++k) {
+      double p2 = ((2.0 * k - 1.0) * x * p1 - (k - 1.0) * p0) / k;
+      p0 = p1;
+      p1 = p2;
+    }
+    dp = n * (x * p1 - p0) / (x * x - 1.0);
+    gl_x[i] = x;
+    gl_w[i] = 2.0 / ((1.0 - x * x) * dp * dp);
+  }
+  gl_ready = 1;
+}
+
+/* C_d = r(d)/sqrt(pi) with r(d) = Gamma(d/2)/Gamma((d-1)/2), from
+ * r(2) = 1/sqrt(pi), r(3) = sqrt(pi)/2 and r(d+2) = r(d) d/(d-1). */
+static double sphere_cd(int d) {
+  double r = (d % 2 == 0) ? 1.0 / sqrt(M_PI) : sqrt(M_PI) / 2.0;
+  for (int k = (d % 2 == 0) ? 2 : 3; k < d; k += 2) r *= (double)k / (double)(k - 1);
+  return r / sqrt(M_PI);
+}
+
+static double sphere_pdf(int d, double cd, double x) {
+  double t = 1.0 - x * x;
+  if (t <= 0.0) return 0.0;
+  return cd * pow(t, 0.5 * (d - 3));
+}
+
+static double gl_panel(int d, double cd, double a, double b) {
+  double h = 0.5 * (b - a), c = 0.5 * (a + b), s = 0.0;
+  for (int i = 0; i < GL_N; ++i) s += gl_w[i] * sphere_pdf(d, cd, c + h * gl_x[i]);
+  return s * h;
+}
+
+/* probability mass of [a, b] under the sphere marginal: composite
+ * Gauss-Legendre on panels no wider than a quarter of the density's scale
+ * 1/sqrt(d); the range where the density is below ~1e-300 is skipped. */
+OR_API double or_sphere_mass(int d, double a, double b) {
+  gl_init();
+  double cd = sphere_cd(d);
+  double xmax = (d > 3) ? sqrt(1500.0 / (d - 3)) : 1.0;
+  if (xmax > 1.0) xmax = 1.0;
+  if (a < -xmax) a = -xmax;
+  if (b > xmax) b = xmax;
+  if (b <= a) return 0.0;
+  double h = fmin(1.0 / 64.0, 0.25 / sqrt((double)d));
+  int panels = (int)ceil((b - a) / h);
+  double total = 0.0;
+  for (int i = 0; i < panels; ++i) {
+    double lo = a + (b - a) * i / panels, hi = a + (b - a) * (i + 1) / panels;
+    total += gl_panel(d, cd, lo, hi);
+  }
+  return total;
+}
+
+/* first moment of [a, b] in closed form: int x f(x) dx */
+OR_API double or_sphere_first_moment(int d, double a, double b) {
+  double cd = sphere_cd(d);
+  double e = 0.5 * (d - 1);
+  return cd * (pow(1.0 - a * a, e) - pow(1.0 - b * b, e)) / (d - 1);
+}
+
+/*
+ * Lloyd-Max on the positive half (the density is symmetric, so the
+ * quantiser is too: levels +-c[k]).  L = 2^(bits-1) positive levels;
+ * positive boundaries t[k] = (c[k] + c[k+1]) / 2, k < L-1; the cell of c[0]
+ * is [0, t[0]], that of c[L-1] is [t[L-2], 1].  Start: quantiles of the
+ * normal approximation N(0, 1/d); iterate centroid/boundary updates until
+ * max |delta c| < 1e-15 (at most max_iter rounds).  Returns iterations used.
+ */
+static double norm_quantile(double p) { /* bisection on the normal CDF */
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 200; ++i) {
+    double mid = 0.5 * (lo + hi);
+    if (0.5 * erfc(-mid / sqrt(2.0)) < p) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+OR_API int or_lloyd_max(int d, int bits, int max_iter, double* c /* L */, double* t /* L-1 */,
+                        double* mse_out) {
+  int L = 1 << (bits - 1);
+  for (int k = 0; k < L; ++k)
+    c[k] = norm_quantile((L + k + 0.5) / (2.0 * L)) / sqrt((double)d);
+  int it = 0;
+  for (; it < max_iter; ++it) {
+    for (int k = 0; k + 1 < L; ++k) t[k] = 0.5 * (c[k] + c[k + 1]);
+    double delta = 0.0;
+    for (int k = 0; k < L; ++k) {
+      double a = (k == 0) ? 0.0 : t[k - 1];
+      double b = (k == L - 1) ? 1.0 : t[k];
+      double nc = or_sphere_first_moment(d, a, b) / or_sphere_mass(d, a, b);
+      delta = fmax(delta, fabs(nc - c[k]));
+      c[k] = nc;
+    }
+    if (delta < 1e-15) { ++it; break; }
+  }
+  for (int k = 0; k + 1 < L; ++k) t[k] = 0.5 * (c[k] + c[k + 1]);
+  if (mse_out) {
+    /* E[(X - Q(X))^2] = E[X^2] - sum over both signs of P(cell) c^2, valid
+     * at a centroid fixed point; E[X^2] = 1/d for a unit-sphere coordinate */
+    double s = 0.0;
+    for (int k = 0; k < L; ++k) {
+      double a = (k == 0) ? 0.0 : t[k - 1];
+      double b = (k == L - 1) ? 1.0 : t[k];
+      s += 2.0 * or_sphere_mass(d, a, b) * c[k] * c[k];
+    }
+    *mse_out = 1.0 / d - s;
+  }
+  return it;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Page format (storage layout of the cold tier; 128 token slots per page). */
+/* Sections in order, each starting on a 16-byte boundary:                  */
+/*   KC key codes    128 x d/4 bytes   (2-bit codes: sign and magnitude)    */
+/*   QS QJL signs    128 x m/8 bytes                                        */
+/*   VC value codes  64 pairs x d bytes (4-bit codes; values pages only)    */
+/*   KN key norm     128 x fp16                                             */
+/*   KG residual norm 128 x fp16                                            */
+/*   VN value norm   128 x fp16        (values pages only)                  */
+/* Key code word w (little-endian u32, w < d/16) of a token holds           */
+/* coordinates j = 16w + 8h + r (h in {0,1}, r = 2i + e < 8): sign bit at   */
+/* 16h + 15 - 4i - e, magnitude bit at 16h + 13 - 4i - e.                   */
+/* QJL word w (w < m/32) holds sketch index i = 32w + 16h + r (r < 16) at   */
+/* bit 16h + 15 - r.  Value codes: token pair p = slot/2; byte j of the     */
+/* pair's block holds code(2p, j) in its low nibble and code(2p+1, j) in    */
+/* its high nibble; a code is sign<<3 | magnitude index (0..7).             */
+/* ------------------------------------------------------------------------ */
+#define PAGE_TOKENS 128
+
+typedef struct {
+  size_t kc, qs, vc, kn, kg, vn, bytes;
+} or_layout;
+
+static size_t up16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+static or_layout layout_of(int d, int m, int with_values) {
+  or_layout L;
+  size_t off = 0;
+  L.kc = off; off = up16(off + (size_t)PAGE_TOKENS * d / 4);
+  L.qs = off; off = up16(off + (size_t)PAGE_TOKENS * m / 8);
+  if (with_values) { L.vc = off; off = up16(off + (size_t)PAGE_TOKENS * d / 2); }
+  else L.vc = 0;
+  L.kn = off; off = up16(off + 2 * PAGE_TOKENS);
+  L.kg = off; off = up16(off + 2 * PAGE_TOKENS);
+  if (with_values) { L.vn = off; off = up16(off + 2 * PAGE_TOKENS); }
+  else L.vn = 0;
+  L.bytes = off;
+  return L;
+}
+
+OR_API size_t or_page_layout(int d, int m, int with_values, size_t* offs /* 6 or NULL */) {
+  or_layout L = layout_of(d, m, with_values);
+  if (offs) {
+    offs[0] = L.kc; offs[1] = L.qs; offs[2] = L.vc;
+    offs[3] = L.kn; offs[4] = L.kg; offs[5] = L.vn;
+  }
+  return L.bytes;
+}
+
+static uint32_t rd32(const uint8_t* p) {
+  return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
+}
+static void wr32(uint8_t* p, uint32_t v) {
+  p[0] = (uint8_t)v; p[1] = (uint8_t)(v >> 8); p[2] = (uint8_t)(v >> 16); p[3] = (uint8_t)(v >> 24);
+}
+static uint16_t rd16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+static void wr16(uint8_t* p, uint16_t v) { p[0] = (uint8_t)v; p[1] = (uint8_t)(v >> 8); }
+
+static int kc_sign_bit(int j) { /* position inside word j/16 */
+  int h = (j % 16) / 8, r = j % 8, i = r / 2, e = r % 2;
+  return 16 * h + 15 - 4 * i - e;
+}
+static int kc_mag_bit(int j) { return kc_sign_bit(j) - 2; }
+static int qs_bit(int i) { /* position inside word i/32 */
+  int h = (i % 32) / 16, r = i % 16;
+  return 16 * h + 15 - r;
+}
+
+/* write one key record into token slot `slot` of page `pg` */
+OR_API void or_pack_key(uint8_t* pg, int d, int m, int with_values, int slot,
+                        const int32_t* sign, const int32_t* mag, const int32_t* qbits,
+                        double n, double gamma) {
+  or_layout L = layout_of(d, m, with_values);
+  uint8_t* kc = pg + L.kc + (size_t)slot * (d / 4);
+  for (int w = 0; w < d / 16; ++w) {
+    uint32_t word = 0;
+    for (int j = 16 * w; j < 16 * w + 16; ++j) {
+      if (sign[j]) word |= 1u << kc_sign_bit(j);
+      if (mag[j]) word |= 1u << kc_mag_bit(j);
+    }
+    wr32(kc + 4 * w, word);
+  }
+  uint8_t* qs = pg + L.qs + (size_t)slot * (m / 8);
+  for (int w = 0; w < m / 32; ++w) {
+    uint32_t word = 0;
+    for (int i = 32 * w; i < 32 * w + 32; ++i)
+      if (qbits[i]) word |= 1u << qs_bit(i);
+    wr32(qs + 4 * w, word);
+  }
+  wr16(pg + L.kn + 2 * slot, f16_bits(or_round_f16(n)));
+  wr16(pg + L.kg + 2 * slot, f16_bits(or_round_f16(gamma)));
+}
+
+OR_API void or_unpack_key(const uint8_t* pg, int d, int m, int with_values, int slot,
+                          int32_t* sign, int32_t* mag, int32_t* qbits, double* n, double* gamma) {
+  or_layout L = layout_of(d, m, with_values);
+  const uint8_t* kc = pg + L.kc + (size_t)slot * (d / 4);
+  for (int j = 0; j < d; ++j) {
+    uint32_t word = rd32(kc + 4 * (j / 16));
+    sign[j] = (word >> kc_sign_bit(j)) & 1u;
+    mag[j] = (word >> kc_mag_bit(j)) & 1u;
+  }
+  const uint8_t* qs = pg + L.qs + (size_t)slot * (m / 8);
+  for (int i = 0; i < m; ++i) qbits[i] = (rd32(qs + 4 * (i / 32)) >> qs_bit(i)) & 1u;
+  *n = f16_value(rd16(pg + L.kn + 2 * slot));
+  *gamma = f16_value(rd16(pg + L.kg + 2 * slot));
+}
+
+/* value record: code = sign<<3 | magnitude index */
+OR_API void or_pack_value(uint8_t* pg, int d, int m, int slot, const int32_t* code, double n) {
+  or_layout L = layout_of(d, m, 1);
+  uint8_t* vc = pg + L.vc + (size_t)(slot / 2) * d;
+  int hi = slot & 1;
+  for (int j = 0; j < d; ++j) {
+    uint8_t b = vc[j];
+    uint8_t c = (uint8_t)(code[j] & 0xF);
+    b = hi ? (uint8_t)((b & 0x0F) | (c << 4)) : (uint8_t)((b & 0xF0) | c);
+    vc[j] = b;
+  }
+  wr16(pg + L.vn + 2 * slot, f16_bits(or_round_f16(n)));
+}
+
+OR_API void or_unpack_value(const uint8_t* pg, int d, int m, int slot, int32_t* code, double* n) {
+  or_layout L = layout_of(d, m, 1);
+  const uint8_t* vc = pg + L.vc + (size_t)(slot / 2) * d;
+  for (int j = 0; j < d; ++j) code[j] = (slot & 1) ? (vc[j] >> 4) : (vc[j] & 0xF);
+  *n = f16_value(rd16(pg + L.vn + 2 * slot));
+}
+
+/* batched forms: record v goes to page page_id[v], slot slot[v].
+ * key arrays: sign/mag [N*d], qbits [N*m], n, gamma [N];
+ * value arrays (with_values): vcode [N*d], vn [N]; may be NULL for keys-only. */
+OR_API void or_pack_batch(uint8_t* pool, size_t page_bytes, int d, int m, int with_values,
+                          int64_t N, const int32_t* page_id, const int32_t* slot,
+                          const int32_t* sign, const int32_t* mag, const int32_t* qbits,
+                          const double* n, const double* gamma, const int32_t* vcode,
+                          const double* vn) {
+  for (int64_t v = 0; v < N; ++v) {
+    uint8_t* pg = pool + (size_t)page_id[v] * page_bytes;
+    or_pack_key(pg, d, m, with_values, slot[v], sign + (size_t)v * d, mag + (size_t)v * d,
+                qbits + (size_t)v * m, n[v], gamma[v]);
+    if (with_values && vcode) or_pack_value(pg, d, m, slot[v], vcode + (size_t)v * d, vn[v]);
+  }
+}
+
+OR_API void or_unpack_batch(const uint8_t* pool, size_t page_bytes, int d, int m,
+                            int with_values, int64_t N, const int32_t* page_id,
+                            const int32_t* slot, int32_t* sign, int32_t* mag, int32_t* qbits,
+                            double* n, double* gamma, int32_t* vcode, double* vn) {
+  for (int64_t v = 0; v < N; ++v) {
+    const uint8_t* pg = pool + (size_t)page_id[v] * page_bytes;
+    or_unpack_key(pg, d, m, with_values, slot[v], sign + (size_t)v * d, mag + (size_t)v * d,
+                  qbits + (size_t)v * m, n + v, gamma + v);
+    if (with_values && vcode) or_unpack_value(pg, d, m, slot[v], vcode + (size_t)v * d, vn + v);
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Encoding one vector [TQ "Funktionsweise" steps 1 and 2; EXP "Stufe 1/2"] */
+/* ------------------------------------------------------------------------ */
+/*
+ * x_rot: the rotated vector as fp32 values (Pi x rounded to fp32, or the
+ * caller's pre-rotated input); xnorm: the Euclidean norm of the vector.
+ * n = fp16(xnorm).  Per coordinate, in fp32: T_k = fp32(n * t_k);
+ * sign = [x_rot_j < 0]; magnitude index = #{k : |x_rot_j| >= T_k}.
+ * Reconstruction c_hat_j = (+-) c[idx] in the normalised domain.
+ * Keys only: residual r = x_rot / n - c_hat (double); gamma = fp16(|r|);
+ * QJL bit i = [(S r)_i < 0] (double).
+ */
+static void encode_one(int d, int m, const double* S, const double* cpos, const double* tpos, int L,
+                       const double* x_rot, double xnorm, int is_key, int32_t* sign, int32_t* mag,
+                       int32_t* qbits, double* n_out, double* gamma_out, double* r_scratch) {
+  double n = or_round_f16(xnorm);
+  *n_out = n;
+  if (gamma_out) *gamma_out = 0.0;
+  if (n == 0.0 || !isfinite(n)) {
+    for (int j = 0; j < d; ++j) { sign[j] = 0; mag[j] = 0; }
+    if (is_key) for (int i = 0; i < m; ++i) qbits[i] = 0;
+    return;
+  }
+  float nf = (float)n;
+  for (int j = 0; j < d; ++j) {
+    float xj = (float)x_rot[j];
+    sign[j] = (xj < 0.0f) ? 1 : 0;
+    float ax = fabsf(xj);
+    int idx = 0;
+    for (int k = 0; k + 1 < L; ++k) {
+      float thr = nf * (float)tpos[k]; /* one fp32 product, rounded */
+      if (ax >= thr) idx = k + 1;
+    }
+    mag[j] = idx;
+  }
+  if (!is_key) return;
+  double rr = 0.0;
+  for (int j = 0; j < d; ++j) {
+    double ch = (sign[j] ? -1.0 : 1.0) * cpos[mag[j]];
+    r_scratch[j] = x_rot[j] / n - ch;
+    rr += r_scratch[j] * r_scratch[j];
+  }
+  *gamma_out = or_round_f16(sqrt(rr));
+  for (int i = 0; i < m; ++i) {
+    double p = 0.0;
+    for (int j = 0; j < d; ++j) p += S[(size_t)i * d + j] * r_scratch[j];
+    qbits[i] = (p < 0.0) ? 1 : 0;
+  }
+}
+
+/*
+ * Encode N vectors.  rotated = 0: x is the raw input (values exactly as
+ * stored, e.g. bf16 widened), x_rot = fp32(Pi x) and xnorm = |x|.
+ * rotated = 1: x already holds fp32 rotated values; xnorm = |x|.
+ * Outputs: sign/mag [N*d], qbits [N*m] (keys), n [N], gamma [N] (keys),
+ * xrot_out [N*d] (the fp32 rotated values used, may be NULL).
+ */
+OR_API void or_encode(int d, int m, const double* pi, const double* S, const double* cpos,
+                      const double* tpos, int L, const double* x, int64_t N, int rotated,
+                      int is_key, int32_t* sign, int32_t* mag, int32_t* qbits, double* n,
+                      double* gamma, double* xrot_out, int threads) {
+#ifdef _OPENMP
+  if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel
+#endif
+  {
+    double* xr = (double*)malloc(sizeof(double) * d);
+    double* rs = (double*)malloc(sizeof(double) * d);
+#ifdef _OPENMP
+#pragma omp for schedule(static)
+#endif
+    for (int64_t v = 0; v < N; ++v) {
+      const double* xv = x + (size_t)v * d;
+      double ss = 0.0;
+      for (int j = 0; j < d; ++j) ss += xv[j] * xv[j];
+      for (int j = 0; j < d; ++j) {
+        if (rotated) {
+          xr[j] = round_f32(xv[j]);
+        } else {
+          double acc = 0.0;
+          for (int k = 0; k < d; ++k) acc += pi[(size_t)j * d + k] * xv[k];
+          xr[j] = round_f32(acc);
+        }
+      }
+      if (xrot_out) memcpy(xrot_out + (size_t)v * d, xr, sizeof(double) * d);
+      encode_one(d, m, S, cpos, tpos, L, xr, sqrt(ss), is_key, sign + (size_t)v * d,
+                 mag + (size_t)v * d, is_key ? qbits + (size_t)v * m : NULL, n + v,
+                 is_key ? gamma + v : NULL, rs);
+    }
+    free(xr);
+    free(rs);
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Estimators [TQ "QJL", EXP "Stufe 2"].                                     */
+/* ------------------------------------------------------------------------ */
+/* <q, r> ~ sqrt(pi/2)/m * gamma * sum_i (S q)_i * (1 - 2 bit_i) */
+OR_API double or_qjl_estimate(int m, const double* sq /* S q, m */, const int32_t* qbits,
+                              double gamma) {
+  double acc = 0.0;
+  for (int i = 0; i < m; ++i) acc += qbits[i] ? -sq[i] : sq[i];
+  return sqrt(M_PI / 2.0) / m * gamma * acc;
+}
+
+/* Monte-Carlo check helper: for trial t, S_t = or_qjl_matrix(seed0 + t);
+ * returns the sample mean and (unbiased) sample variance of the estimate of
+ * <q, r> with the exact |r| as gamma. */
+OR_API void or_qjl_montecarlo(int d, int m, const double* q, const double* r, int64_t trials,
+                              uint64_t seed0, double* mean, double* var) {
+  double* S = (double*)malloc(sizeof(double) * m * d);
+  double* sq = (double*)malloc(sizeof(double) * m);
+  int32_t* bits = (int32_t*)malloc(sizeof(int32_t) * m);
+  double rn = 0.0;
+  for (int j = 0; j < d; ++j) rn += r[j] * r[j];
+  rn = sqrt(rn);
+  double s1 = 0.0, s2 = 0.0;
+  for (int64_t t = 0; t < trials; ++t) {
+    or_qjl_matrix(m, d, seed0 + (uint64_t)t, S);
+    for (int i = 0; i < m; ++i) {
+      double a = 0.0, b = 0.0;
+      for (int j = 0; j < d; ++j) {
+        a += S[(size_t)i * d + j] * q[j];
+        b += S[(size_t)i * d + j] * r[j];
+      }
+      sq[i] = a;
+      bits[i] = (b < 0.0) ? 1 : 0;
+    }
+    double e = or_qjl_estimate(m, sq, bits, rn);
+    s1 += e;
+    s2 += e * e;
+  }
+  *mean = s1 / trials;
+  *var = (s2 - s1 * s1 / trials) / (trials - 1);
+  free(S); free(sq); free(bits);
+}
+
+/* estimated score of a stored key against a query (scale applied):
+ * n * ( <q_rot, c_hat> + sqrt(pi/2)/m * gamma * <S q_rot, 1-2 bits> ) * scale */
+static double key_score(int d, int m, const double* qrot, const double* sq, const double* cpos,
+                        const int32_t* sign, const int32_t* mag, const int32_t* qbits, double n,
+                        double gamma, double scale) {
+  double ip = 0.0;
+  for (int j = 0; j < d; ++j) ip += qrot[j] * (sign[j] ? -cpos[mag[j]] : cpos[mag[j]]);
+  return n * (ip + or_qjl_estimate(m, sq, qbits, gamma)) * scale;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention over one (batch, kv head) group [MON "Vereinfachte      */
+/* Decode-Schleife": hot scores, cold scores, softmax, aggregation].         */
+/* One softmax over cold tokens (estimated scores, reconstructed values      */
+/* v_hat = n_v Pi^T c_hat_v) followed by hot tokens (exact fp16 keys and     */
+/* values).  Two-pass softmax.  q: [G, d]; out: [G, d].                      */
+/* ------------------------------------------------------------------------ */
+OR_API int or_attention_group(int d, int m, const double* pi, const double* S,
+                              const double* kcpos, const double* vcpos, int G,
+                              const double* q, double scale, const double* k_hot,
+                              const double* v_hot, int hot_len, const uint8_t* pool,
+                              size_t page_bytes, const int32_t* pages, int cold_len,
+                              double* out) {
+  int nt = cold_len + hot_len;
+  double* logits = (double*)malloc(sizeof(double) * (size_t)G * (nt > 0 ? nt : 1));
+  double* vals = (double*)malloc(sizeof(double) * (size_t)(nt > 0 ? nt : 1) * d);
+  double* qrot = (double*)malloc(sizeof(double) * (size_t)G * d);
+  double* sq = (double*)malloc(sizeof(double) * (size_t)G * m);
+  int32_t* sign = (int32_t*)malloc(sizeof(int32_t) * d);
+  int32_t* mag = (int32_t*)malloc(sizeof(int32_t) * d);
+  int32_t* qb = (int32_t*)malloc(sizeof(int32_t) * m);
+  int32_t* vcode = (int32_t*)malloc(sizeof(int32_t) * d);
+  double* chat = (double*)malloc(sizeof(double) * d);
+  if (!logits || !vals || !qrot || !sq || !sign || !mag || !qb || !vcode || !chat) return -1;
+
+  for (int h = 0; h < G; ++h) {
+    for (int j = 0; j < d; ++j) {
+      double a = 0.0;
+      for (int k = 0; k < d; ++k) a += pi[(size_t)j * d + k] * q[(size_t)h * d + k];
+      qrot[(size_t)h * d + j] = a;
+    }
+    for (int i = 0; i < m; ++i) {
+      double a = 0.0;
+      for (int j = 0; j < d; ++j) a += S[(size_t)i * d + j] * qrot[(size_t)h * d + j];
+      sq[(size_t)h * m + i] = a;
+    }
+  }
+  for (int t = 0; t < cold_len; ++t) {
+    const uint8_t* pg = pool + (size_t)pages[t / PAGE_TOKENS] * page_bytes;
+    int slot = t % PAGE_TOKENS;
+    double n, gamma, nv;
+    or_unpack_key(pg, d, m, 1, slot, sign, mag, qb, &n, &gamma);
+    for (int h = 0; h < G; ++h)
+      logits[(size_t)h * nt + t] = key_score(d, m, qrot + (size_t)h * d, sq + (size_t)h * m,
+                                             kcpos, sign, mag, qb, n, gamma, scale);
+    or_unpack_value(pg, d, m, slot, vcode, &nv);
+    for (int j = 0; j < d; ++j) {
+      int c = vcode[j];
+      chat[j] = ((c >> 3) ? -1.0 : 1.0) * vcpos[c & 7];
+    }
+    for (int k = 0; k < d; ++k) { /* v_hat = n_v * Pi^T c_hat */
+      double a = 0.0;
+      for (int j = 0; j < d; ++j) a += pi[(size_t)j * d + k] * chat[j];
+      vals[(size_t)t * d + k] = nv * a;
+    }
+  }
+  for (int t = 0; t < hot_len; ++t) {
+    for (int h = 0; h < G; ++h) {
+      double a = 0.0;
+      for (int j = 0; j < d; ++j) a += q[(size_t)h * d + j] * k_hot[(size_t)t * d + j];
+      logits[(size_t)h * nt + cold_len + t] = a * scale;
+    }
+    memcpy(vals + (size_t)(cold_len + t) * d, v_hot + (size_t)t * d, sizeof(double) * d);
+  }
+  for (int h = 0; h < G; ++h) {
+    double* o = out + (size_t)h * d;
+    for (int j = 0; j < d; ++j) o[j] = 0.0;
+    if (nt == 0) continue; /* no tokens: output defined as zero */
+    double mx = -INFINITY;
+    for (int t = 0; t < nt; ++t) mx = fmax(mx, logits[(size_t)h * nt + t]);
+    double den = 0.0;
+    for (int t = 0; t < nt; ++t) den += exp(logits[(size_t)h * nt + t] - mx);
+    for (int t = 0; t < nt; ++t) {
+      double p = exp(logits[(size_t)h * nt + t] - mx) / den;
+      for (int j = 0; j < d; ++j) o[j] += p * vals[(size_t)t * d + j];
+    }
+  }
+  free(logits); free(vals); free(qrot); free(sq);
+  free(sign); free(mag); free(qb); free(vcode); free(chat);
+  return 0;
+}
+
+/*
+ * Batched driver: groups listed in sel (pairs b, kv_head); the q heads of
+ * kv head h are h*G .. h*G+G-1 (contiguous grouping).  Layouts:
+ * q [B, Hq, d]; k_hot, v_hot [B, Hkv, W, d]; page_table [B, Hkv, max_pages];
+ * out [nsel, G, d].
+ */
+OR_API int or_attention(int d, int m, const double* pi, const double* S, const double* kcpos,
+                        const double* vcpos, int B, int Hq, int Hkv, const double* q,
+                        double scale, const double* k_hot, const double* v_hot, int W,
+                        const int32_t* hot_len, const uint8_t* pool, size_t page_bytes,
+                        const int32_t* page_table, int max_pages, const int32_t* cold_len,
+                        const int32_t* sel, int nsel, double* out, int threads) {
+  int G = Hq / Hkv;
+  int err = 0;
+#ifdef _OPENMP
+  if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic) reduction(| : err)
+#endif
+  for (int s = 0; s < nsel; ++s) {
+    int b = sel[2 * s], h = sel[2 * s + 1];
+    const double* kh = k_hot ? k_hot + ((size_t)b * Hkv + h) * (size_t)W * d : NULL;
+    const double* vh = v_hot ? v_hot + ((size_t)b * Hkv + h) * (size_t)W * d : NULL;
+    int hl = hot_len ? hot_len[b] : 0;
+    int cl = cold_len ? cold_len[b] : 0;
+    err |= or_attention_group(d, m, pi, S, kcpos, vcpos, G, q + ((size_t)b * Hq + (size_t)h * G) * d,
+                              scale, kh, vh, hl, pool, page_bytes,
+                              page_table + ((size_t)b * Hkv + h) * max_pages, cl,
+                              out + (size_t)s * G * d);
+  }
+  return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Compressed top-k search [TQ "Leistung bei der Vektorsuche"].             */
+/* Score of DB vector i: n_i ( <q_rot, c_hat_i> + sqrt(pi/2)/m gamma_i      */
+/* <S q_rot, 1-2 bits_i> ), scale 1.  Result: the k largest, ties to the    */
+/* lower id.  DB vector i sits in keys-only page i/128, slot i%128.          */
+/* ------------------------------------------------------------------------ */
+static int better(double sa, int32_t ia, double sb, int32_t ib) {
+  return (sa > sb) || (sa == sb && ia < ib);
+}
+
+OR_API void or_topk(int d, int m, const double* pi, const double* S, const double* kcpos,
+                    const double* queries, int Q, const uint8_t* db, size_t page_bytes, int64_t N,
+                    int k, int32_t* out_ids, double* out_scores, int threads) {
+#ifdef _OPENMP
+  if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel
+#endif
+  {
+    double* qrot = (double*)malloc(sizeof(double) * d);
+    double* sq = (double*)malloc(sizeof(double) * m);
+    int32_t* sign = (int32_t*)malloc(sizeof(int32_t) * d);
+    int32_t* mag = (int32_t*)malloc(sizeof(int32_t) * d);
+    int32_t* qb = (int32_t*)malloc(sizeof(int32_t) * m);
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic)
+#endif
+    for (int qi = 0; qi < Q; ++qi) {
+      const double* qv = queries + (size_t)qi * d;
+      for (int j = 0; j < d; ++j) {
+        double a = 0.0;
+        for (int kk = 0; kk < d; ++kk) a += pi[(size_t)j * d + kk] * qv[kk];
+        qrot[j] = a;
+      }
+      for (int i = 0; i < m; ++i) {
+        double a = 0.0;
+        for (int j = 0; j < d; ++j) a += S[(size_t)i * d + j] * qrot[j];
+        sq[i] = a;
+      }
+      int32_t* ids = out_ids + (size_t)qi * k;
+      double* sc = out_scores + (size_t)qi * k;
+      int filled = 0;
+      for (int64_t v = 0; v < N; ++v) {
+        double n, gamma;
+        or_unpack_key(db + (size_t)(v / PAGE_TOKENS) * page_bytes, d, m, 0,
+                      (int)(v % PAGE_TOKENS), sign, mag, qb, &n, &gamma);
+        double s = key_score(d, m, qrot, sq, kcpos, sign, mag, qb, n, gamma, 1.0);
+        int32_t id = (int32_t)v;
+        /* keep the list sorted best-first: insertion into k slots */
+        if (filled < k) {
+          int pos = filled++;
+          while (pos > 0 && better(s, id, sc[pos - 1], ids[pos - 1])) {
+            sc[pos] = sc[pos - 1]; ids[pos] = ids[pos - 1]; --pos;
+          }
+          sc[pos] = s; ids[pos] = id;
+        } else if (better(s, id, sc[k - 1], ids[k - 1])) {
+          int pos = k - 1;
+          while (pos > 0 && better(s, id, sc[pos - 1], ids[pos - 1])) {
+            sc[pos] = sc[pos - 1]; ids[pos] = ids[pos - 1]; --pos;
+          }
+          sc[pos] = s; ids[pos] = id;
+        }
+      }
+      for (int i = filled; i < k; ++i) { ids[i] = -1; sc[i] = -INFINITY; }
+    }
+    free(qrot); free(sq); free(sign); free(mag); free(qb);
+  }
+}
+
+OR_API int or_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
