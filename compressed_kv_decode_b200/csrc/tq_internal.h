@@ -1,0 +1,82 @@
+// Internal declarations shared by the host-side files of libtq.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+struct HostTables {
+  std::vector<float> rot;    // [d*d] row-major, x_rot = rot x
+  std::vector<float> qjl;    // [m*d] row-major, fp16-valued
+  std::vector<float> key_c;  // positive levels
+  std::vector<float> key_t;  // positive boundaries
+  std::vector<float> val_c;
+  std::vector<float> val_t;
+};
+
+bool config_valid(const tq_config& c);
+bool config_supported(const tq_config& c);
+bool generate_tables(const tq_config& cfg, HostTables& out);
+
+// Small per-context constants passed to kernels by value.
+struct Codebook {
+  float key_c[2];
+  float key_t[1];
+  float val_c[8];
+  float val_t[7];
+};
+
+// Device tables owned by a context.
+struct DeviceTables {
+  const float* rot;          // [d*d] fp32
+  const float* qjl;          // [m*d] fp32 (fp16 values)
+  const uint16_t* qjl_h;     // [m*d] fp16 bits
+  const uint16_t* rot_bf_hi; // [d*d] bf16 bits of rot
+  const uint16_t* rot_bf_lo; // [d*d] bf16 bits of rot - bf16(rot)
+  const uint16_t* rot_h_hi;  // [d*d] fp16 bits of rot
+  const uint16_t* rot_h_lo;  // [d*d] fp16 bits of rot - fp16(rot)
+  int* err;                  // device error word (first error wins)
+};
+
+}  // namespace tq
+
+struct tq_ctx {
+  tq_config cfg;
+  int device;
+  int num_sms;
+  tq::HostTables host;
+  tq::Codebook cb;
+  tq::DeviceTables dev;
+  void* dev_block;  // single allocation holding every device table
+};
+
+namespace tq {
+
+// Page layout (bytes) for head dim d, sketch dim m.
+struct PageLayout {
+  size_t kc, qs, vc, kn, kg, vn, bytes;
+};
+PageLayout page_layout(int d, int m, bool with_values);
+
+// Launchers (defined in the .cu files).  Return a tq_status.
+int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq, int Hkv,
+                  float scale, const void* k_hot, const void* v_hot, int W_max,
+                  const int32_t* hot_len, const uint8_t* pool, int64_t pool_pages,
+                  const int32_t* page_table, int max_pages, const int32_t* cold_len, float* out,
+                  void* ws, size_t ws_bytes, void* stream);
+size_t decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max);
+
+int launch_compress(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype, int flags,
+                    int B, int Hkv, int n_new, uint8_t* pool, int64_t pool_pages,
+                    const int32_t* page_table, int max_pages, int32_t* cold_len, void* stream);
+
+int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* db, int64_t N,
+                int k, int32_t* out_ids, float* out_scores, void* ws, size_t ws_bytes,
+                void* stream);
+size_t topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k);
+
+}  // namespace tq

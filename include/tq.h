@@ -1,0 +1,223 @@
+/*
+ * tq.h -- C ABI of libtq: TurboQuant-style compressed KV cache and decode
+ * attention over it, for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (web pages on the subject; sections as titled):
+ *  - "TurboQuant" summary, de.news.hada.io topic 27867, section "Funktionsweise
+ *    von TurboQuant": a vector is randomly rotated, each coordinate goes
+ *    through a standard scalar quantiser, and the residual error is encoded
+ *    with 1-bit QJL; section "QJL: Eine 1-Bit-Methode ohne Overhead": a
+ *    Johnson-Lindenstrauss projection reduced to sign bits and an estimator
+ *    that pairs a full-precision query with those bits; the discussion
+ *    thread: Lloyd-Max boundaries and reconstruction values after rotation.
+ *  - "Monarch v3: NES-inspiriertes KV-Paging", openclawradar.com, sections
+ *    "Wie es funktioniert" and "Vereinfachte Decode-Schleife": recent tokens
+ *    stay at full precision in a hot window, older ones are compressed into a
+ *    cold region, and each decode step scores hot and cold tokens and takes
+ *    one softmax over them.
+ *  - The same summary, section "Leistung bei der Vektorsuche": the codec also
+ *    serves inner-product vector search (top-k).
+ *
+ * Conventions for every call:
+ *  - Device pointers are CUDA device addresses on the device that was current
+ *    when the context was created; host pointers are marked "host".
+ *  - Streams are cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls that take a stream only enqueue work and never synchronise.
+ *  - Argument errors are found on the host, before any launch, and return
+ *    TQ_ERR_INVALID_ARG (or TQ_ERR_UNSUPPORTED for valid but unimplemented
+ *    shapes).  A failed launch returns TQ_ERR_CUDA.  Errors found on the
+ *    device (a page id outside the pool, a length beyond capacity, a wait
+ *    that timed out) are recorded in the context's device error word, the
+ *    offending work is skipped, and tq_get_error() reports the first one.
+ *  - The library allocates device memory only in tq_init_codebook (its
+ *    constant tables and error word) and frees it in tq_destroy.  All other
+ *    buffers (page pool, page tables, lengths, hot window, outputs,
+ *    workspace) are owned by the caller.
+ *  - No C++ exception crosses this boundary.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Version of the cold-page storage format below. */
+#define TQ_LAYOUT_VERSION 1
+/* Token slots per cold page. */
+#define TQ_PAGE_TOKENS 128
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,
+  TQ_ERR_UNSUPPORTED = 2,
+  TQ_ERR_CUDA = 3,
+  TQ_ERR_OOM = 4,
+  TQ_ERR_CAPACITY = 5, /* device: a sequence outgrew its page table or pool */
+  TQ_ERR_TIMEOUT = 6   /* device: a bounded wait on a copy ran out */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_F16 = 1, TQ_BF16 = 2 } tq_dtype;
+
+/* Codec configuration.  Supported: head_dim 64 or 128, key_bits 2 (1-bit
+ * magnitude index + sign), qjl_dim == head_dim, value_bits 4 (3-bit
+ * magnitude index + sign), page_tokens 128.  seed selects the rotation and
+ * the QJL matrix. */
+typedef struct {
+  int head_dim;
+  int key_bits;
+  int qjl_dim;
+  int value_bits;
+  int page_tokens;
+  uint64_t seed;
+} tq_config;
+
+typedef struct tq_ctx tq_ctx; /* opaque; immutable after creation */
+
+/*
+ * Host-only generation of the codec tables ("Funktionsweise von TurboQuant"
+ * and its discussion), no device needed.  All outputs are host arrays:
+ *  rot   [d*d]  row-major Haar rotation Pi (x_rot = Pi x), fp32.  Pi is the Q
+ *               factor of the QR factorisation of a d x d matrix of standard
+ *               normal draws (SplitMix64 stream seeded 2*seed, 53-bit
+ *               uniforms, Box-Muller with both outputs, filled row by row),
+ *               with the signs of its columns chosen so that diag(R) > 0.
+ *  qjl   [m*d]  QJL matrix S, row-major: standard normal draws of stream
+ *               2*seed+1, each rounded to the nearest fp16 value.
+ *  key_c [2^(key_bits-1)], key_t [2^(key_bits-1)-1]: positive Lloyd-Max
+ *               levels and boundaries for one coordinate of a uniform point
+ *               on the unit sphere of R^d (levels are +-key_c), fp32.
+ *  val_c, val_t: the same at value_bits.
+ * Any output may be NULL.  Cost: a fraction of a second (fp64 solves).
+ */
+tq_status tq_generate_params(const tq_config* cfg, float* rot, float* qjl, float* key_c,
+                             float* key_t, float* val_c, float* val_t);
+
+/* Generate the tables (as tq_generate_params) and upload them to the current
+ * device.  *out receives the context; release it with tq_destroy. */
+tq_status tq_init_codebook(const tq_config* cfg, tq_ctx** out);
+
+/* Copy the context's tables to host arrays (same layouts as
+ * tq_generate_params; NULL outputs are skipped). */
+tq_status tq_get_params(const tq_ctx* ctx, float* rot, float* qjl, float* key_c, float* key_t,
+                        float* val_c, float* val_t);
+
+/*
+ * Bytes of one cold page (TQ_PAGE_TOKENS token slots).  with_values = 1: key
+ * and value records (15104 B at d=128, 7936 B at d=64); 0: keys only, as used
+ * by a search database (6656 B, 3584 B).  Layout, sections in this order,
+ * each starting on a 16-byte boundary:
+ *   KC  key codes        128 x d/4 B
+ *   QS  QJL sign bits    128 x m/8 B
+ *   VC  value codes      64 x d B      (values pages only)
+ *   KN  key norm n       128 x fp16
+ *   KG  residual norm    128 x fp16
+ *   VN  value norm       128 x fp16    (values pages only)
+ * Key code word w (u32, little endian, w < d/16) of a token holds coordinates
+ * j = 16w + 8h + 2i + e (h, e in {0,1}, i < 4) with the sign bit at
+ * 16h + 15 - 4i - e and the magnitude bit at 16h + 13 - 4i - e.  QJL word w
+ * (w < m/32) holds sketch index 32w + 16h + r (r < 16) at bit 16h + 15 - r;
+ * a set bit means (S r)_i < 0.  Value codes come in token pairs: the byte of
+ * coordinate j in pair p holds code(2p, j) in its low nibble and
+ * code(2p+1, j) in its high nibble; a code is sign << 3 | magnitude index.
+ * The pair's d-byte block is cut in 8 chunks of d/8 bytes and chunk g
+ * (coordinates g*d/8 ...) is stored at chunk position (g + 2*(p mod 4)) mod 8,
+ * so that four consecutive pairs read chunk-wise hit distinct shared-memory
+ * banks.  Coordinates are those of the rotated domain.
+ */
+size_t tq_page_bytes(const tq_ctx* ctx, int with_values);
+
+/* Input flag for tq_compress_append: k and v already hold Pi x in fp32 (the
+ * rotation folded into the projection that produced them). */
+#define TQ_INPUT_ROTATED 1
+
+/*
+ * Compress n_new new tokens per (batch, kv head) and append them to the cold
+ * pages ("Funktionsweise von TurboQuant"; eviction from the hot window into
+ * the cold region as in Monarch's "Wie es funktioniert").
+ *  k, v        device, [B, Hkv, n_new, d], dtype `dtype` (F16 or BF16; F32
+ *              only with TQ_INPUT_ROTATED).  v = NULL writes keys-only pages.
+ *  page_pool   device, 16-byte aligned, pool_pages pages of
+ *              tq_page_bytes(ctx, v != NULL) bytes each.
+ *  page_table  device int32 [B, Hkv, max_pages]: pool page of each logical
+ *              page; token position t of (b, h) lives in page
+ *              page_table[b, h, t / 128], slot t % 128.
+ *  cold_len    device int32 [B]: tokens already stored per sequence (equal
+ *              for all kv heads).  The new tokens take positions
+ *              cold_len[b] .. cold_len[b] + n_new - 1; cold_len is advanced by
+ *              n_new on the stream after the writes.
+ * Per vector: n = fp16(|x|); codes from x_rot = Pi x against thresholds
+ * fp32(n * t_k); keys also store gamma = fp16(|x_rot/n - c_hat|) and the
+ * signs of S (x_rot/n - c_hat).  Device errors: a position beyond
+ * max_pages*128 or a page id outside [0, pool_pages) -> TQ_ERR_CAPACITY and
+ * that token is not written.
+ */
+tq_status tq_compress_append(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,
+                             int flags, int B, int Hkv, int n_new, uint8_t* page_pool,
+                             int64_t pool_pages, const int32_t* page_table, int max_pages,
+                             int32_t* cold_len, void* stream);
+
+/* Workspace bytes tq_decode_attention needs for these maxima. */
+size_t tq_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max);
+
+/*
+ * One decode step of attention over a hot fp16 window and cold compressed
+ * pages, one softmax over both ("Vereinfachte Decode-Schleife"; the cold
+ * scores use the QJL estimator of "QJL: Eine 1-Bit-Methode ohne Overhead"):
+ *   cold score  n * (<Pi q, c_hat> + sqrt(pi/2)/m * gamma * <S Pi q, 1 - 2 bits>) * scale
+ *   cold value  n_v * Pi^T c_hat_v
+ *   hot score   <q, k> * scale, hot value v (exact)
+ *  q          device [B, Hq, d], q_dtype F32, F16 or BF16.  Query head h
+ *             attends with kv head h / (Hq / Hkv).
+ *  scale      softmax scale; 0 selects 1/sqrt(d).
+ *  k_hot, v_hot device fp16 [B, Hkv, W_max, d]; hot_len device int32 [B]
+ *             (0 <= hot_len <= W_max).  May be NULL when W_max == 0.
+ *  page_pool, pool_pages, page_table, max_pages, cold_len: as in
+ *             tq_compress_append (values pages); cold_len is only read.
+ *  out        device fp32 [B, Hq, d]; a sequence with no tokens gets zeros.
+ *  workspace  device, ws_bytes >= tq_workspace_bytes(ctx, B, Hq, Hkv,
+ *             max_pages, W_max), 256-byte aligned; contents are scratch.
+ * Supported: Hq % Hkv == 0 with Hq / Hkv in {1, 2, 4, 8}.
+ */
+tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                              int Hkv, float scale, const void* k_hot, const void* v_hot,
+                              int W_max, const int32_t* hot_len, const uint8_t* page_pool,
+                              int64_t pool_pages, const int32_t* page_table, int max_pages,
+                              const int32_t* cold_len, float* out, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+/* Workspace bytes tq_score_topk needs. */
+size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k);
+
+/*
+ * Compressed inner-product search ("Leistung bei der Vektorsuche"): the
+ * estimated inner product of every query with every database vector (the
+ * cold score above with scale 1), then the k best per query, ties to the
+ * lower id.
+ *  queries   device fp32 [Q, d].
+ *  db_pages  device keys-only pages; vector i sits in page i / 128, slot
+ *            i % 128 (pages written by tq_compress_append with v = NULL).
+ *  out_ids   device int32 [Q, k]; out_scores device fp32 [Q, k], best first.
+ *            When N < k the tail holds id -1 and score -inf.
+ *  workspace device, ws_bytes >= tq_topk_workspace_bytes(ctx, Q, N, k).
+ * Supported: 1 <= k <= 32.
+ */
+tq_status tq_score_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* db_pages,
+                        int64_t N, int k, int32_t* out_ids, float* out_scores, void* workspace,
+                        size_t ws_bytes, void* stream);
+
+/* Read and clear the context's device error word.  Synchronises with the
+ * device; call it after the work of interest has completed. */
+tq_status tq_get_error(const tq_ctx* ctx);
+
+const char* tq_status_string(tq_status s);
+
+void tq_destroy(tq_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TQ_H */

@@ -372,9 +372,11 @@ OR_API int or_lloyd_max(int d, int bits, int max_iter, double* c /* L */, double
 /* coordinates j = 16w + 8h + r (h in {0,1}, r = 2i + e < 8): sign bit at   */
 /* 16h + 15 - 4i - e, magnitude bit at 16h + 13 - 4i - e.                   */
 /* QJL word w (w < m/32) holds sketch index i = 32w + 16h + r (r < 16) at   */
-/* bit 16h + 15 - r.  Value codes: token pair p = slot/2; byte j of the     */
-/* pair's block holds code(2p, j) in its low nibble and code(2p+1, j) in    */
-/* its high nibble; a code is sign<<3 | magnitude index (0..7).             */
+/* bit 16h + 15 - r.  Value codes: token pair p = slot/2; the byte of       */
+/* coordinate j holds code(2p, j) in its low nibble and code(2p+1, j) in    */
+/* its high nibble; a code is sign<<3 | magnitude index (0..7).  The pair's */
+/* d-byte block is cut in 8 chunks of d/8 bytes; chunk g (coordinates       */
+/* g*d/8 ...) is stored at chunk position (g + 2*(p mod 4)) mod 8.          */
 /* ------------------------------------------------------------------------ */
 #define PAGE_TOKENS 128
 
@@ -427,6 +429,12 @@ static int qs_bit(int i) { /* position inside word i/32 */
   return 16 * h + 15 - r;
 }
 
+/* offset of coordinate j's byte inside the value block of token pair p */
+static int vc_pos(int d, int p, int j) {
+  int chunk = d / 8;
+  return ((j / chunk + 2 * (p % 4)) % 8) * chunk + j % chunk;
+}
+
 /* write one key record into token slot `slot` of page `pg` */
 OR_API void or_pack_key(uint8_t* pg, int d, int m, int with_values, int slot,
                         const int32_t* sign, const int32_t* mag, const int32_t* qbits,
@@ -470,21 +478,25 @@ OR_API void or_unpack_key(const uint8_t* pg, int d, int m, int with_values, int 
 /* value record: code = sign<<3 | magnitude index */
 OR_API void or_pack_value(uint8_t* pg, int d, int m, int slot, const int32_t* code, double n) {
   or_layout L = layout_of(d, m, 1);
-  uint8_t* vc = pg + L.vc + (size_t)(slot / 2) * d;
+  int p = slot / 2;
+  uint8_t* vc = pg + L.vc + (size_t)p * d;
   int hi = slot & 1;
   for (int j = 0; j < d; ++j) {
-    uint8_t b = vc[j];
+    uint8_t* bp = vc + vc_pos(d, p, j);
     uint8_t c = (uint8_t)(code[j] & 0xF);
-    b = hi ? (uint8_t)((b & 0x0F) | (c << 4)) : (uint8_t)((b & 0xF0) | c);
-    vc[j] = b;
+    *bp = hi ? (uint8_t)((*bp & 0x0F) | (c << 4)) : (uint8_t)((*bp & 0xF0) | c);
   }
   wr16(pg + L.vn + 2 * slot, f16_bits(or_round_f16(n)));
 }
 
 OR_API void or_unpack_value(const uint8_t* pg, int d, int m, int slot, int32_t* code, double* n) {
   or_layout L = layout_of(d, m, 1);
-  const uint8_t* vc = pg + L.vc + (size_t)(slot / 2) * d;
-  for (int j = 0; j < d; ++j) code[j] = (slot & 1) ? (vc[j] >> 4) : (vc[j] & 0xF);
+  int p = slot / 2;
+  const uint8_t* vc = pg + L.vc + (size_t)p * d;
+  for (int j = 0; j < d; ++j) {
+    uint8_t b = vc[vc_pos(d, p, j)];
+    code[j] = (slot & 1) ? (b >> 4) : (b & 0xF);
+  }
   *n = f16_value(rd16(pg + L.vn + 2 * slot));
 }
 

@@ -57,7 +57,8 @@ def test_golden_format_examples(O):
     word = lambda off: int.from_bytes(pool[off:off + 4].tobytes(), "little")
     assert word(offs["kc"]) == int(g["key"]["word0"], 16)
     assert word(offs["qs"]) == int(g["qjl"]["word0"], 16)
-    assert pool[offs["vc"] + 1 * d + cj] == int(g["value"]["byte"], 16)
+    assert pool[offs["vc"] + 1 * d + int(g["value"]["offset"])] == int(g["value"]["byte"], 16)
+    assert np.count_nonzero(pool[offs["vc"]:offs["kn"]]) == 1
 
 
 @pytest.mark.parametrize("d,m", D_M)
@@ -90,6 +91,27 @@ def test_every_bit_position_by_inverse_map(O, d, m):
             O.pack(pool, nbytes, d, m, True, [0], [slot], rec)
             sec = pool[offs["qs"]:offs["vc"]].view(np.uint32).reshape(128, m // 32)
             assert np.count_nonzero(sec) == 1 and sec[slot, w] == (1 << b)
+
+
+@pytest.mark.parametrize("d,m", D_M)
+def test_value_byte_positions(O, d, m):
+    """Each (pair, coordinate) lands on its own byte; chunks rotate by two
+    positions per pair within a group of four pairs."""
+    nbytes, offs = O.page_layout(d, m, True)
+    chunk = d // 8
+    for p in range(6):
+        seen = set()
+        for j in range(d):
+            pool = np.zeros(nbytes, np.uint8)
+            rec = _empty_records(1, d, m)
+            rec["vcode"][0, j] = 0x9
+            O.pack(pool, nbytes, d, m, True, [0], [2 * p + 1], rec)
+            blk = pool[offs["vc"] + p * d: offs["vc"] + (p + 1) * d]
+            (pos,) = np.nonzero(blk)
+            assert len(pos) == 1 and blk[pos[0]] == 0x90
+            assert pos[0] // chunk == (j // chunk + 2 * (p % 4)) % 8 and pos[0] % chunk == j % chunk
+            seen.add(int(pos[0]))
+        assert len(seen) == d
 
 
 @pytest.mark.parametrize("d,m", D_M)
