@@ -1,0 +1,360 @@
+#!/usr/bin/env python
+"""Benchmark of compressed-KV decode attention on B200.
+
+Metric: KV tokens*heads per second of tq_decode_attention on the
+Llama-3-8B-shaped 32K-context decode (batch 16, 32 q / 8 kv heads,
+head_dim 128, 1024 hot fp16 tokens + 31744 cold tokens at 3-bit keys /
+4-bit values), with achieved HBM GB/s of the split-K attention kernel
+against the measured copy bandwidth.  A step is one decode call over the
+whole cache: query prep, split-K attention over hot and cold tokens,
+cross-split combine.  The cold pages are written by tq_compress_append from
+seeded synthetic K, V (N(0,1), 8 outlier channels x8 per kv head).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tq|reference]
+
+N > 1 runs under torchrun, one rank per GPU; every rank decodes its own
+batch (weak scaling, no data-path collective); the time is the maximum
+over ranks.  --impl reference times the CPU oracle on a bounded sample of
+the same workload.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "llama3_8b_32k"
+METRIC = "compressed-KV decode attention: KV tokens·heads/s and achieved HBM GB/s vs peak"
+UNIT = "KV tokens*heads/s"
+COLD_RECORD_BYTES = 118   # per cold token per kv head (d=128): 52 B key + 66 B value
+HOT_RECORD_BYTES = 512    # per hot token per kv head: fp16 K and V
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def kernel_traffic(kernel, source):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    with open(os.path.join(ROOT, source), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if rec.get("src_sha") == sha else None
+
+
+class ClockSampler:
+    """SM clock and throttle reasons read through NVML while the timed region runs."""
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv is not None:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# workload on the device
+# ---------------------------------------------------------------------------
+def build_state(torch, tq, W, rank):
+    cfg = W.DECODE[WORKLOAD]
+    B, Hq, Hkv, d = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"]
+    cold, hot = cfg["cold"], cfg["hot"]
+    dev = torch.device("cuda")
+    ctx = tq.Context(d, seed=0)
+    max_pages = cold // 128
+    n_pages = B * Hkv * max_pages
+    page_bytes = ctx.page_bytes(True)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    pool = torch.empty((n_pages, page_bytes), dtype=torch.uint8, device=dev)
+    table = torch.randperm(n_pages, generator=gen, device=dev).to(torch.int32).view(B, Hkv, max_pages)
+    cold_len = torch.zeros(B, dtype=torch.int32, device=dev)
+    chans = torch.stack([torch.randperm(d, generator=gen, device=dev)[:cfg["n_out"]] for _ in range(Hkv)])
+    scale = torch.ones(Hkv, d, device=dev)
+    scale.scatter_(1, chans, cfg["factor"])
+
+    def kv(n):
+        x = torch.randn((B, Hkv, n, d), generator=gen, device=dev) * scale[None, :, None, :]
+        return x.to(torch.bfloat16)
+
+    chunk = 2048
+    for t0 in range(0, cold, chunk):
+        n = min(chunk, cold - t0)
+        tq.tq_compress_append(ctx.handle, kv(n), kv(n), pool, table, cold_len)
+    torch.cuda.synchronize()
+    ctx.check()
+    k_hot = kv(hot).to(torch.float16)
+    v_hot = kv(hot).to(torch.float16)
+    hot_len = torch.full((B,), hot, dtype=torch.int32, device=dev)
+    q = torch.randn((B, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    ws = ctx.workspace(B, Hq, Hkv, max_pages, hot)
+    st = dict(ctx=ctx, pool=pool, table=table, cold_len=cold_len, k_hot=k_hot, v_hot=v_hot,
+              hot_len=hot_len, q=q, out=out, ws=ws, B=B, Hq=Hq, Hkv=Hkv, d=d, cold=cold, hot=hot)
+    return st
+
+
+def decode(tq, st, q=None, out=None):
+    tq.tq_decode_attention(st["ctx"].handle, st["q"] if q is None else q, st["k_hot"],
+                           st["v_hot"], st["hot_len"], st["pool"], st["table"], st["cold_len"],
+                           st["out"] if out is None else out, st["ws"], st["Hkv"])
+
+
+def reduce_max(torch, x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_baseline(sample_groups=None):
+    """The oracle, as it stands, on a bounded sample of the workload: a few
+    (batch, kv head) groups of the 32K decode with random cold records."""
+    import oracle as O
+    from compressed_kv_decode_b200 import workloads as W
+    cfg = W.DECODE[WORKLOAD]
+    d, G = cfg["d"], cfg["Hq"] // cfg["Hkv"]
+    cores = os.cpu_count() or 1
+    n = sample_groups or max(1, min(cfg["B"] * cfg["Hkv"], cores))
+    P = O.Params(d, seed=0)
+    nbytes, offs = O.page_layout(d, d, True)
+    max_pages = cfg["cold"] // 128
+    table = np.arange(n * max_pages, dtype=np.int32).reshape(n, 1, max_pages)
+    pool = W.random_page_bytes(7, n * max_pages, nbytes, offs)
+    rng = np.random.default_rng(8)
+    k_hot = rng.standard_normal((n, 1, cfg["hot"], d)).astype(np.float16).astype(np.float64)
+    v_hot = rng.standard_normal((n, 1, cfg["hot"], d)).astype(np.float16).astype(np.float64)
+    q = W.queries(13, n, G, d, "bfloat16")
+    lens_c = np.full(n, cfg["cold"], np.int32)
+    lens_h = np.full(n, cfg["hot"], np.int32)
+    threads = O.max_threads()
+    t0 = time.perf_counter()
+    O.attention(P, q, 1, 1.0 / math.sqrt(d), k_hot, v_hot, lens_h, pool.reshape(-1), nbytes,
+                table, lens_c, threads=threads)
+    dt = time.perf_counter() - t0
+    units = n * (cfg["cold"] + cfg["hot"])
+    return {"value": units / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": "%d of %d (batch, kv head) groups of the 32K decode (%d tokens each), "
+                      "random cold records, %.2f s" % (n, cfg["B"] * cfg["Hkv"],
+                                                       cfg["cold"] + cfg["hot"], dt)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    steps = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline()
+        if i >= args.warmup:
+            steps.append(r)
+    vals = [s["value"] for s in steps]
+    value = statistics.mean(vals)
+    cb = dict(steps[-1])
+    cb["value"] = value
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "ms_per_step": None, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import compressed_kv_decode_b200 as tq
+    from compressed_kv_decode_b200 import workloads as W
+    torch.cuda.set_device(local_rank)
+    st = build_state(torch, tq, W, rank)
+    ctx = st["ctx"]
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        decode(tq, st)
+    torch.cuda.synchronize()
+    ctx.check()
+
+    # device-resident inputs: K decode calls bracketed by barrier + sync
+    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            tq.tq_set_profile_events(ctx.handle, ev_k[i][0], ev_k[i][1])
+            decode(tq, st)
+        e1.record(stream)
+        e1.synchronize()
+    tq.tq_set_profile_events(ctx.handle, None, None)
+    torch.cuda.synchronize()
+    barrier(world)
+    ctx.check()
+    ms_total = reduce_max(torch, e0.elapsed_time(e1), world)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_k)
+
+    # end to end: q from pinned host memory, output back to pinned host memory
+    q_host = st["q"].cpu().pin_memory()
+    out_host = torch.empty(st["out"].shape, dtype=torch.float32).pin_memory()
+    q_dev = torch.empty_like(st["q"])
+    for _ in range(3):
+        q_dev.copy_(q_host, non_blocking=True)
+        decode(tq, st, q=q_dev)
+        out_host.copy_(st["out"], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        q_dev.copy_(q_host, non_blocking=True)
+        decode(tq, st, q=q_dev)
+        out_host.copy_(st["out"], non_blocking=True)
+    f1.record(stream)
+    f1.synchronize()
+    barrier(world)
+    e2e_ms = reduce_max(torch, f0.elapsed_time(f1), world)
+    ctx.check()
+
+    units_per_step = st["B"] * st["Hkv"] * (st["cold"] + st["hot"])
+    value = units_per_step * world * args.steps / (ms_total / 1e3)
+    e2e_value = units_per_step * world * args.steps / (e2e_ms / 1e3)
+    peaks, peak_kind = measured_peaks()
+    algo_bytes = (st["B"] * st["Hkv"] * (st["cold"] * COLD_RECORD_BYTES + st["hot"] * HOT_RECORD_BYTES)
+                  + st["table"].numel() * 4)
+    achieved = algo_bytes / (attn_ms / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    if rank != 0:
+        return
+    cb = cpu_baseline() if world == 1 else None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16/fp32 (3-bit keys, 4-bit values)",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": st["B"] * world, "kv_heads": st["Hkv"],
+                   "q_heads": st["Hq"], "head_dim": st["d"], "hot_tokens": st["hot"],
+                   "cold_tokens": st["cold"], "parallelism": "dp%d" % world,
+                   "l2": "inputs larger than L2 (%.0f MB per step)" % (algo_bytes / 1e6)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_kind + " hbm_gbs",
+                     "kernel": "attn_kernel", "kernel_ms": attn_ms,
+                     "algorithmic_bytes_per_launch": algo_bytes,
+                     "traffic": kernel_traffic("attn_kernel_llama3_8b_32k",
+                                               "compressed_kv_decode_b200/csrc/tq_decode.cu")},
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": st["q"].numel() * st["q"].element_size(),
+                "d2h_bytes_per_step": st["out"].numel() * 4},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": cb,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local_rank = dist_env()
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,258 @@
+"""Python binding of libtq (TurboQuant-style compressed KV cache and decode
+attention for B200).  Argument marshalling only: every step of the hot path
+runs in the CUDA kernels behind the C ABI declared in ``include/tq.h``.
+
+The functions keep the C names.  Device buffers are torch CUDA tensors
+(passed by data pointer); the stream is torch's current CUDA stream unless
+one is given.  There is no CPU fallback: if ``libtq.so`` is missing or the
+device is absent the calls raise.
+"""
+import ctypes as C
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA = 0, 1, 2, 3
+TQ_ERR_OOM, TQ_ERR_CAPACITY, TQ_ERR_TIMEOUT = 4, 5, 6
+TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
+TQ_INPUT_ROTATED = 1
+TQ_PAGE_TOKENS = 128
+
+
+class TQError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+
+
+class tq_config(C.Structure):
+    _fields_ = [("head_dim", C.c_int), ("key_bits", C.c_int), ("qjl_dim", C.c_int),
+                ("value_bits", C.c_int), ("page_tokens", C.c_int), ("seed", C.c_uint64)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libtq.so (building it first when the sources are newer)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH) or os.environ.get("TQ_REBUILD"):
+            from . import build as _build
+            _build.build()
+        L = C.CDLL(LIB_PATH)
+        vp, i32p, f32p, u8p = C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p
+        L.tq_generate_params.argtypes = [C.POINTER(tq_config)] + [C.c_void_p] * 6
+        L.tq_generate_params.restype = C.c_int
+        L.tq_init_codebook.argtypes = [C.POINTER(tq_config), C.POINTER(C.c_void_p)]
+        L.tq_init_codebook.restype = C.c_int
+        L.tq_get_params.argtypes = [vp] + [C.c_void_p] * 6
+        L.tq_get_params.restype = C.c_int
+        L.tq_page_bytes.argtypes = [vp, C.c_int]
+        L.tq_page_bytes.restype = C.c_size_t
+        L.tq_compress_append.argtypes = [vp, vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                          u8p, C.c_int64, i32p, C.c_int, i32p, vp]
+        L.tq_compress_append.restype = C.c_int
+        L.tq_workspace_bytes.argtypes = [vp, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]
+        L.tq_workspace_bytes.restype = C.c_size_t
+        L.tq_decode_attention.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float,
+                                          vp, vp, C.c_int, i32p, u8p, C.c_int64, i32p, C.c_int,
+                                          i32p, f32p, vp, C.c_size_t, vp]
+        L.tq_decode_attention.restype = C.c_int
+        L.tq_topk_workspace_bytes.argtypes = [vp, C.c_int, C.c_int64, C.c_int]
+        L.tq_topk_workspace_bytes.restype = C.c_size_t
+        L.tq_score_topk.argtypes = [vp, f32p, C.c_int, u8p, C.c_int64, C.c_int, i32p, f32p, vp,
+                                    C.c_size_t, vp]
+        L.tq_score_topk.restype = C.c_int
+        L.tq_set_profile_events.argtypes = [vp, vp, vp]
+        L.tq_set_profile_events.restype = C.c_int
+        L.tq_get_error.argtypes = [vp]
+        L.tq_get_error.restype = C.c_int
+        L.tq_status_string.argtypes = [C.c_int]
+        L.tq_status_string.restype = C.c_char_p
+        L.tq_destroy.argtypes = [vp]
+        L.tq_destroy.restype = None
+        _lib = L
+    return _lib
+
+
+def status_string(s):
+    return lib().tq_status_string(int(s)).decode()
+
+
+def _check(status, what):
+    if status != TQ_OK:
+        raise TQError(status, what)
+
+
+def make_config(head_dim=128, seed=0, key_bits=2, value_bits=4, qjl_dim=None):
+    return tq_config(head_dim, key_bits, head_dim if qjl_dim is None else qjl_dim, value_bits,
+                     TQ_PAGE_TOKENS, seed)
+
+
+def _ptr(t):
+    """Device (or host) address of a torch tensor / numpy array; None -> NULL."""
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _dtype_code(t):
+    import torch
+    return {torch.float32: TQ_F32, torch.float16: TQ_F16, torch.bfloat16: TQ_BF16}[t.dtype]
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _require_cuda(*tensors):
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise ValueError("device tensor expected")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("contiguous tensor expected")
+
+
+# ---------------------------------------------------------------------------
+# C entry points, same names
+# ---------------------------------------------------------------------------
+def tq_generate_params(cfg):
+    """Host-only table generation (no device needed).  Returns numpy arrays."""
+    d, m = cfg.head_dim, cfg.qjl_dim
+    out = dict(rot=np.empty((d, d), np.float32), qjl=np.empty((m, d), np.float32),
+               key_c=np.empty(1 << (cfg.key_bits - 1), np.float32),
+               key_t=np.empty(max((1 << (cfg.key_bits - 1)) - 1, 1), np.float32),
+               val_c=np.empty(1 << (cfg.value_bits - 1), np.float32),
+               val_t=np.empty(max((1 << (cfg.value_bits - 1)) - 1, 1), np.float32))
+    _check(lib().tq_generate_params(C.byref(cfg), *[_ptr(out[k]) for k in
+                                                    ("rot", "qjl", "key_c", "key_t", "val_c", "val_t")]),
+           "tq_generate_params")
+    out["key_t"] = out["key_t"][: (1 << (cfg.key_bits - 1)) - 1]
+    out["val_t"] = out["val_t"][: (1 << (cfg.value_bits - 1)) - 1]
+    return out
+
+
+def tq_init_codebook(cfg):
+    h = C.c_void_p()
+    _check(lib().tq_init_codebook(C.byref(cfg), C.byref(h)), "tq_init_codebook")
+    return h
+
+
+def tq_get_params(ctx, cfg):
+    d, m = cfg.head_dim, cfg.qjl_dim
+    out = dict(rot=np.empty((d, d), np.float32), qjl=np.empty((m, d), np.float32),
+               key_c=np.empty(2, np.float32), key_t=np.empty(1, np.float32),
+               val_c=np.empty(8, np.float32), val_t=np.empty(7, np.float32))
+    _check(lib().tq_get_params(ctx, *[_ptr(out[k]) for k in
+                                      ("rot", "qjl", "key_c", "key_t", "val_c", "val_t")]),
+           "tq_get_params")
+    return out
+
+
+def tq_page_bytes(ctx, with_values=True):
+    return int(lib().tq_page_bytes(ctx, 1 if with_values else 0))
+
+
+def tq_compress_append(ctx, k, v, page_pool, page_table, cold_len, rotated=False, stream=None):
+    """k, v: [B, Hkv, n_new, d] CUDA tensors (fp16/bf16, or fp32 when rotated);
+    v may be None (keys-only pages).  page_pool: uint8 [pool_pages, page_bytes];
+    page_table: int32 [B, Hkv, max_pages]; cold_len: int32 [B] (advanced)."""
+    _require_cuda(k, v, page_pool, page_table, cold_len)
+    B, Hkv, n_new, _ = k.shape
+    _check(lib().tq_compress_append(
+        ctx, _ptr(k), _ptr(v), _dtype_code(k), TQ_INPUT_ROTATED if rotated else 0, B, Hkv, n_new,
+        _ptr(page_pool), page_pool.shape[0], _ptr(page_table), page_table.shape[-1],
+        _ptr(cold_len), _stream(stream)), "tq_compress_append")
+
+
+def tq_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max):
+    return int(lib().tq_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max))
+
+
+def tq_decode_attention(ctx, q, k_hot, v_hot, hot_len, page_pool, page_table, cold_len, out,
+                        workspace, Hkv, scale=0.0, stream=None):
+    """q: [B, Hq, d]; k_hot, v_hot: fp16 [B, Hkv, W_max, d] or None; hot_len,
+    cold_len: int32 [B]; page_pool uint8 [pool_pages, page_bytes]; page_table
+    int32 [B, Hkv, max_pages]; out fp32 [B, Hq, d]; workspace uint8 CUDA tensor."""
+    _require_cuda(q, k_hot, v_hot, hot_len, page_pool, page_table, cold_len, out, workspace)
+    B, Hq, _ = q.shape
+    W_max = 0 if k_hot is None else k_hot.shape[2]
+    max_pages = 0 if page_table is None else page_table.shape[-1]
+    pool_pages = 0 if page_pool is None else page_pool.shape[0]
+    _check(lib().tq_decode_attention(
+        ctx, _ptr(q), _dtype_code(q), B, Hq, Hkv, float(scale), _ptr(k_hot), _ptr(v_hot), W_max,
+        _ptr(hot_len), _ptr(page_pool), pool_pages, _ptr(page_table), max_pages, _ptr(cold_len),
+        _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "tq_decode_attention")
+
+
+def tq_topk_workspace_bytes(ctx, Q, N, k):
+    return int(lib().tq_topk_workspace_bytes(ctx, Q, N, k))
+
+
+def tq_score_topk(ctx, queries, db_pages, N, k, out_ids, out_scores, workspace, stream=None):
+    _require_cuda(queries, db_pages, out_ids, out_scores, workspace)
+    _check(lib().tq_score_topk(
+        ctx, _ptr(queries), queries.shape[0], _ptr(db_pages), int(N), int(k), _ptr(out_ids),
+        _ptr(out_scores), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "tq_score_topk")
+
+
+def tq_set_profile_events(ctx, ev_start, ev_stop):
+    """ev_start/ev_stop: torch.cuda.Event(enable_timing=True) or None."""
+    a = None if ev_start is None else C.c_void_p(ev_start.cuda_event)
+    b = None if ev_stop is None else C.c_void_p(ev_stop.cuda_event)
+    _check(lib().tq_set_profile_events(ctx, a, b), "tq_set_profile_events")
+
+
+def tq_get_error(ctx):
+    return int(lib().tq_get_error(ctx))
+
+
+def tq_destroy(ctx):
+    lib().tq_destroy(ctx)
+
+
+# ---------------------------------------------------------------------------
+# convenience wrapper owning a context
+# ---------------------------------------------------------------------------
+class Context:
+    def __init__(self, head_dim=128, seed=0):
+        self.cfg = make_config(head_dim, seed)
+        self.handle = tq_init_codebook(self.cfg)
+        self.d = head_dim
+
+    def params(self):
+        return tq_get_params(self.handle, self.cfg)
+
+    def page_bytes(self, with_values=True):
+        return tq_page_bytes(self.handle, with_values)
+
+    def workspace(self, B, Hq, Hkv, max_pages, W_max, device="cuda"):
+        import torch
+        n = tq_workspace_bytes(self.handle, B, Hq, Hkv, max_pages, W_max)
+        return torch.empty(n, dtype=torch.uint8, device=device)
+
+    def check(self):
+        s = tq_get_error(self.handle)
+        if s != TQ_OK:
+            raise TQError(s, "device")
+
+    def close(self):
+        if self.handle is not None:
+            tq_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

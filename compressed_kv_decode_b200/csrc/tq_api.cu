@@ -1,0 +1,275 @@
+// C ABI entry points of libtq: argument validation, context lifetime, table
+// upload, and dispatch to the kernel launchers.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "tq_internal.h"
+
+namespace tq {
+
+PageLayout page_layout(int d, int m, bool with_values) {
+  auto up16 = [](size_t x) { return (x + 15) & ~static_cast<size_t>(15); };
+  const size_t P = TQ_PAGE_TOKENS;
+  PageLayout L{};
+  size_t off = 0;
+  L.kc = off;
+  off = up16(off + P * d / 4);
+  L.qs = off;
+  off = up16(off + P * m / 8);
+  if (with_values) {
+    L.vc = off;
+    off = up16(off + P * d / 2);
+  }
+  L.kn = off;
+  off = up16(off + 2 * P);
+  L.kg = off;
+  off = up16(off + 2 * P);
+  if (with_values) {
+    L.vn = off;
+    off = up16(off + 2 * P);
+  }
+  L.bytes = off;
+  return L;
+}
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+float bf16_value(uint16_t b) { return __bfloat162float(__ushort_as_bfloat16(b)); }
+uint16_t f16_bits(float x) { return __half_as_ushort(__float2half_rn(x)); }
+float f16_value(uint16_t b) { return __half2float(__ushort_as_half(b)); }
+
+}  // namespace
+}  // namespace tq
+
+extern "C" {
+
+const char* tq_status_string(tq_status s) {
+  switch (s) {
+    case TQ_OK: return "ok";
+    case TQ_ERR_INVALID_ARG: return "invalid argument";
+    case TQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TQ_ERR_CUDA: return "CUDA error";
+    case TQ_ERR_OOM: return "out of device memory";
+    case TQ_ERR_CAPACITY: return "capacity exceeded (page table, pool or window)";
+    case TQ_ERR_TIMEOUT: return "bounded wait timed out";
+  }
+  return "unknown status";
+}
+
+tq_status tq_generate_params(const tq_config* cfg, float* rot, float* qjl, float* key_c,
+                             float* key_t, float* val_c, float* val_t) {
+  if (!cfg || !tq::config_valid(*cfg)) return TQ_ERR_INVALID_ARG;
+  tq::HostTables t;
+  if (!tq::generate_tables(*cfg, t)) return TQ_ERR_INVALID_ARG;
+  auto put = [](float* dst, const std::vector<float>& src) {
+    if (dst && !src.empty()) std::memcpy(dst, src.data(), src.size() * sizeof(float));
+  };
+  put(rot, t.rot);
+  put(qjl, t.qjl);
+  put(key_c, t.key_c);
+  put(key_t, t.key_t);
+  put(val_c, t.val_c);
+  put(val_t, t.val_t);
+  return TQ_OK;
+}
+
+tq_status tq_init_codebook(const tq_config* cfg, tq_ctx** out) {
+  if (!cfg || !out) return TQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!tq::config_valid(*cfg)) return TQ_ERR_INVALID_ARG;
+  if (!tq::config_supported(*cfg)) return TQ_ERR_UNSUPPORTED;
+  tq_ctx* ctx = new (std::nothrow) tq_ctx();
+  if (!ctx) return TQ_ERR_OOM;
+  ctx->cfg = *cfg;
+  if (!tq::generate_tables(*cfg, ctx->host)) {
+    delete ctx;
+    return TQ_ERR_INVALID_ARG;
+  }
+  if (cudaGetDevice(&ctx->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device) !=
+          cudaSuccess) {
+    delete ctx;
+    return TQ_ERR_CUDA;
+  }
+  const int d = cfg->head_dim, m = cfg->qjl_dim;
+  const tq::HostTables& h = ctx->host;
+  std::memset(&ctx->cb, 0, sizeof(ctx->cb));
+  for (size_t i = 0; i < h.key_c.size() && i < 2; ++i) ctx->cb.key_c[i] = h.key_c[i];
+  for (size_t i = 0; i < h.key_t.size() && i < 1; ++i) ctx->cb.key_t[i] = h.key_t[i];
+  for (size_t i = 0; i < h.val_c.size() && i < 8; ++i) ctx->cb.val_c[i] = h.val_c[i];
+  for (size_t i = 0; i < h.val_t.size() && i < 7; ++i) ctx->cb.val_t[i] = h.val_t[i];
+
+  // one device block: rot f32 | qjl f32 | qjl f16 | rot bf16 hi, lo | rot f16 hi, lo | err
+  const size_t dd = static_cast<size_t>(d) * d, md = static_cast<size_t>(m) * d;
+  auto a256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  size_t off_rot = 0, off_qjl = a256(off_rot + dd * 4), off_qjlh = a256(off_qjl + md * 4);
+  size_t off_bh = a256(off_qjlh + md * 2), off_bl = a256(off_bh + dd * 2);
+  size_t off_hh = a256(off_bl + dd * 2), off_hl = a256(off_hh + dd * 2);
+  size_t off_err = a256(off_hl + dd * 2), total = a256(off_err + 256);
+  std::vector<uint8_t> img(total, 0);
+  std::memcpy(img.data() + off_rot, h.rot.data(), dd * 4);
+  std::memcpy(img.data() + off_qjl, h.qjl.data(), md * 4);
+  uint16_t* qh = reinterpret_cast<uint16_t*>(img.data() + off_qjlh);
+  for (size_t i = 0; i < md; ++i) qh[i] = tq::f16_bits(h.qjl[i]);
+  uint16_t* bh = reinterpret_cast<uint16_t*>(img.data() + off_bh);
+  uint16_t* bl = reinterpret_cast<uint16_t*>(img.data() + off_bl);
+  uint16_t* hh = reinterpret_cast<uint16_t*>(img.data() + off_hh);
+  uint16_t* hl = reinterpret_cast<uint16_t*>(img.data() + off_hl);
+  for (size_t i = 0; i < dd; ++i) {
+    const float x = h.rot[i];
+    bh[i] = tq::bf16_bits(x);
+    bl[i] = tq::bf16_bits(x - tq::bf16_value(bh[i]));
+    hh[i] = tq::f16_bits(x);
+    hl[i] = tq::f16_bits(x - tq::f16_value(hh[i]));
+  }
+  void* blk = nullptr;
+  if (cudaMalloc(&blk, total) != cudaSuccess) {
+    delete ctx;
+    return TQ_ERR_OOM;
+  }
+  if (cudaMemcpy(blk, img.data(), total, cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(blk);
+    delete ctx;
+    return TQ_ERR_CUDA;
+  }
+  uint8_t* b = static_cast<uint8_t*>(blk);
+  ctx->dev_block = blk;
+  ctx->dev.rot = reinterpret_cast<const float*>(b + off_rot);
+  ctx->dev.qjl = reinterpret_cast<const float*>(b + off_qjl);
+  ctx->dev.qjl_h = reinterpret_cast<const uint16_t*>(b + off_qjlh);
+  ctx->dev.rot_bf_hi = reinterpret_cast<const uint16_t*>(b + off_bh);
+  ctx->dev.rot_bf_lo = reinterpret_cast<const uint16_t*>(b + off_bl);
+  ctx->dev.rot_h_hi = reinterpret_cast<const uint16_t*>(b + off_hh);
+  ctx->dev.rot_h_lo = reinterpret_cast<const uint16_t*>(b + off_hl);
+  ctx->dev.err = reinterpret_cast<int*>(b + off_err);
+  *out = ctx;
+  return TQ_OK;
+}
+
+tq_status tq_get_params(const tq_ctx* ctx, float* rot, float* qjl, float* key_c, float* key_t,
+                        float* val_c, float* val_t) {
+  if (!ctx) return TQ_ERR_INVALID_ARG;
+  auto put = [](float* dst, const std::vector<float>& src) {
+    if (dst && !src.empty()) std::memcpy(dst, src.data(), src.size() * sizeof(float));
+  };
+  put(rot, ctx->host.rot);
+  put(qjl, ctx->host.qjl);
+  put(key_c, ctx->host.key_c);
+  put(key_t, ctx->host.key_t);
+  put(val_c, ctx->host.val_c);
+  put(val_t, ctx->host.val_t);
+  return TQ_OK;
+}
+
+size_t tq_page_bytes(const tq_ctx* ctx, int with_values) {
+  if (!ctx) return 0;
+  return tq::page_layout(ctx->cfg.head_dim, ctx->cfg.qjl_dim, with_values != 0).bytes;
+}
+
+tq_status tq_compress_append(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,
+                             int flags, int B, int Hkv, int n_new, uint8_t* page_pool,
+                             int64_t pool_pages, const int32_t* page_table, int max_pages,
+                             int32_t* cold_len, void* stream) {
+  if (!ctx || !k || !page_pool || !page_table || !cold_len) return TQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || n_new < 0 || max_pages <= 0 || pool_pages <= 0)
+    return TQ_ERR_INVALID_ARG;
+  if (dtype != TQ_F32 && dtype != TQ_F16 && dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if ((flags & ~TQ_INPUT_ROTATED) != 0) return TQ_ERR_INVALID_ARG;
+  const bool rotated = (flags & TQ_INPUT_ROTATED) != 0;
+  if (rotated != (dtype == TQ_F32)) return TQ_ERR_UNSUPPORTED;
+  if (!tq::aligned(page_pool, 16) || !tq::aligned(k, 16) || (v && !tq::aligned(v, 16)))
+    return TQ_ERR_INVALID_ARG;
+  if (n_new == 0) return TQ_OK;
+  return static_cast<tq_status>(tq::launch_compress(ctx, k, v, dtype, flags, B, Hkv, n_new,
+                                                    page_pool, pool_pages, page_table, max_pages,
+                                                    cold_len, stream));
+}
+
+size_t tq_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max) {
+  if (!ctx) return 0;
+  return tq::decode_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max);
+}
+
+tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                              int Hkv, float scale, const void* k_hot, const void* v_hot,
+                              int W_max, const int32_t* hot_len, const uint8_t* page_pool,
+                              int64_t pool_pages, const int32_t* page_table, int max_pages,
+                              const int32_t* cold_len, float* out, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  if (!ctx || !q || !out || !workspace) return TQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || W_max < 0 || max_pages < 0)
+    return TQ_ERR_INVALID_ARG;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_ERR_UNSUPPORTED;
+  if (W_max > 0 && (!k_hot || !v_hot || !hot_len)) return TQ_ERR_INVALID_ARG;
+  if (W_max > 0 && (!tq::aligned(k_hot, 16) || !tq::aligned(v_hot, 16))) return TQ_ERR_INVALID_ARG;
+  if (max_pages > 0 && (!page_pool || !page_table || !cold_len || pool_pages <= 0))
+    return TQ_ERR_INVALID_ARG;
+  if (page_pool && !tq::aligned(page_pool, 16)) return TQ_ERR_INVALID_ARG;
+  if (!tq::aligned(workspace, 256)) return TQ_ERR_INVALID_ARG;
+  const size_t need = tq::decode_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max);
+  if (need == 0 || ws_bytes < need) return TQ_ERR_INVALID_ARG;
+  return static_cast<tq_status>(tq::launch_decode(
+      ctx, q, q_dtype, B, Hq, Hkv, scale, W_max > 0 ? k_hot : nullptr,
+      W_max > 0 ? v_hot : nullptr, W_max, W_max > 0 ? hot_len : nullptr,
+      max_pages > 0 ? page_pool : nullptr, pool_pages, max_pages > 0 ? page_table : nullptr,
+      max_pages, max_pages > 0 ? cold_len : nullptr, out, workspace, ws_bytes, stream));
+}
+
+size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k) {
+  if (!ctx || Q <= 0 || N <= 0 || k <= 0) return 0;
+  return tq::topk_workspace_bytes(ctx, Q, N, k);
+}
+
+tq_status tq_score_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* db_pages,
+                        int64_t N, int k, int32_t* out_ids, float* out_scores, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  if (!ctx || !queries || !db_pages || !out_ids || !out_scores || !workspace)
+    return TQ_ERR_INVALID_ARG;
+  if (Q <= 0 || N <= 0 || k <= 0) return TQ_ERR_INVALID_ARG;
+  if (k > 32) return TQ_ERR_UNSUPPORTED;
+  if (!tq::aligned(db_pages, 16) || !tq::aligned(queries, 16) || !tq::aligned(workspace, 256))
+    return TQ_ERR_INVALID_ARG;
+  const size_t need = tq::topk_workspace_bytes(ctx, Q, N, k);
+  if (need == 0 || ws_bytes < need) return TQ_ERR_INVALID_ARG;
+  return static_cast<tq_status>(tq::launch_topk(ctx, queries, Q, db_pages, N, k, out_ids,
+                                                out_scores, workspace, ws_bytes, stream));
+}
+
+tq_status tq_set_profile_events(tq_ctx* ctx, void* ev_start, void* ev_stop) {
+  if (!ctx || ((ev_start == nullptr) != (ev_stop == nullptr))) return TQ_ERR_INVALID_ARG;
+  ctx->prof_start = ev_start;
+  ctx->prof_stop = ev_stop;
+  return TQ_OK;
+}
+
+tq_status tq_get_error(const tq_ctx* ctx) {
+  if (!ctx) return TQ_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaMemcpy(&v, ctx->dev.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(ctx->dev.err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return TQ_ERR_CUDA;
+  }
+  return static_cast<tq_status>(v);
+}
+
+void tq_destroy(tq_ctx* ctx) {
+  if (!ctx) return;
+  if (ctx->dev_block) cudaFree(ctx->dev_block);
+  delete ctx;
+}
+
+}  // extern "C"

@@ -1,0 +1,961 @@
+// Decode attention over a hot fp16 window and cold compressed pages, one
+// softmax over both ("Monarch v3: NES-inspiriertes KV-Paging", sections "Wie es
+// funktioniert" and "Vereinfachte Decode-Schleife"); cold scores use the
+// TurboQuant key estimator with the 1-bit QJL correction ("TurboQuant"
+// summary, sections "Funktionsweise von TurboQuant" and "QJL: Eine 1-Bit-
+// Methode ohne Overhead").
+//
+// Three launches:
+//  1. prep      one CTA per (batch, kv head): q_rot = Pi q, q_s = S q_rot, the
+//               constants of the estimator folded in, split into fp16 hi/lo
+//               and laid out as the tensor-core B fragments each lane needs;
+//               one extra CTA builds the work schedule (units per segment,
+//               prefix sums, partial-record slots).
+//  2. attention persistent warps, each owning a contiguous range of work
+//               units (64 cold tokens or 16 hot tokens).  A warp streams its
+//               units through a private ring of shared-memory slots filled by
+//               1-D bulk copies (TMA) completing on mbarriers, unpacks the
+//               codes into fp16 tensor-core fragments in registers, scores
+//               them with m16n8k16 MMAs (tokens on M, q heads x {hi, lo} on N),
+//               keeps an online softmax and accumulates P.V with MMAs (cold
+//               values in the rotated domain).  It writes one partial
+//               (m, l, o) per segment it touched.
+//  3. combine   per (batch, kv head): log-sum-exp merge of the cold partials,
+//               o_cold = Pi^T o_rot, merge with the hot partials, divide.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "tq_device.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+namespace dec {
+
+constexpr int NW = 8;         // warps per attention CTA
+constexpr int COLD_TOK = 64;  // tokens per cold unit (half a page)
+constexpr int HOT_TOK = 16;   // tokens per hot unit
+constexpr float NEG_INF = -__builtin_huge_valf();
+
+template <int D, int G>
+struct Cfg {
+  static constexpr int KS = D / 16;              // k-steps per key plane (and QJL, m = D)
+  static constexpr int NT = (2 * G + 7) / 8;     // score n-tiles: G heads x {hi, lo}
+  static constexpr int RC = 3 * KS * NT * 2;     // cold B-fragment registers per lane
+  static constexpr int RH = KS * NT * 2;         // hot B-fragment registers per lane
+  static constexpr int WPT = D / 64;             // key code words per lane per token
+  static constexpr int WV = D / 32;              // value words per lane per token pair
+  static constexpr int KC_B = COLD_TOK * D / 4;  // bytes of one unit's sections
+  static constexpr int QS_B = COLD_TOK * D / 8;
+  static constexpr int VC_B = COLD_TOK / 2 * D;
+  static constexpr int OFF_QS = KC_B;
+  static constexpr int OFF_VC = OFF_QS + QS_B;
+  static constexpr int OFF_KN = OFF_VC + VC_B;
+  static constexpr int OFF_KG = OFF_KN + 2 * COLD_TOK;
+  static constexpr int OFF_VN = OFF_KG + 2 * COLD_TOK;
+  static constexpr int COLD_B = OFF_VN + 2 * COLD_TOK;
+  static constexpr int HROW = 2 * D + 16;  // padded hot row: conflict-free ldmatrix
+  static constexpr int HOT_B = 2 * HOT_TOK * HROW;
+  static constexpr int SLOT = ((COLD_B > HOT_B ? COLD_B : HOT_B) + 127) / 128 * 128;
+  static constexpr int NSLOT = (D == 128) ? 3 : 4;
+  static constexpr int PBUF = COLD_TOK * 16;  // fp16 P' tile [64 tokens][8 heads]
+  static constexpr int SMEM = NW * (NSLOT * SLOT + PBUF) + NW * NSLOT * 8;
+};
+
+struct Work {
+  int* sched;         // [4 + 2 (S+1) + S]: U, unit_off, slot_off, seg_len
+  uint32_t* frag_c;   // [BH][RC][32]
+  uint32_t* frag_h;   // [BH][RH][32]
+  float* desc;        // [BH][2][8] descale per (domain, head)
+  float* part;        // [(Wtot + S)][G][D + 2]
+};
+
+struct Params {
+  const void* q;
+  int q_dtype;
+  int B, Hq, Hkv, max_pages, W_max;
+  float sl;  // softmax scale * log2(e)
+  const __half* k_hot;
+  const __half* v_hot;
+  const int32_t* hot_len;
+  const uint8_t* pool;
+  long long pool_pages;
+  long long page_bytes;
+  int off_kc, off_qs, off_vc, off_kn, off_kg, off_vn;
+  const int32_t* page_table;
+  const int32_t* cold_len;
+  float* out;
+  const float* rot;
+  const float* qjl;
+  float kc0, kc1, alpha;
+  float vc[8];
+  int* err;
+  Work w;
+  int S;     // segments = 2 * B * Hkv
+  int Wtot;  // attention warps
+};
+
+__device__ __forceinline__ int* unit_off(const Params& p) { return p.w.sched + 4; }
+__device__ __forceinline__ int* slot_off(const Params& p) { return p.w.sched + 4 + p.S + 1; }
+__device__ __forceinline__ int* seg_len(const Params& p) { return p.w.sched + 4 + 2 * (p.S + 1); }
+
+// largest warp index whose range starts at or before unit u
+__device__ __forceinline__ int warp_of(long long u, long long U, long long W) {
+  return static_cast<int>(((u + 1) * W - 1) / U);
+}
+
+// ---------------------------------------------------------------------------
+// 1. prep
+// ---------------------------------------------------------------------------
+__device__ int block_exclusive_scan(int v, int* scratch /* >= 32 ints */, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = (lane < nw) ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < nw) scratch[lane] = s;
+  }
+  __syncthreads();
+  int before = (warp > 0) ? scratch[warp - 1] : 0;
+  total = scratch[nw - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+__device__ void build_schedule(const Params& p) {
+  __shared__ int scratch[32];
+  __shared__ int carry_s;
+  const int S = p.S;
+  int* uoff = unit_off(p);
+  int* soff = slot_off(p);
+  int* slen = seg_len(p);
+  if (threadIdx.x == 0) carry_s = 0;
+  __syncthreads();
+  for (int base = 0; base < S; base += blockDim.x) {
+    const int sg = base + threadIdx.x;
+    int units = 0;
+    if (sg < S) {
+      const int bh = sg >> 1, b = bh / p.Hkv;
+      int len;
+      if ((sg & 1) == 0) {
+        len = p.cold_len ? p.cold_len[b] : 0;
+        const int cap = p.max_pages * TQ_PAGE_TOKENS;
+        if (len < 0 || len > cap) {
+          report(p.err, TQ_ERR_CAPACITY);
+          len = len < 0 ? 0 : cap;
+        }
+        units = (len + COLD_TOK - 1) / COLD_TOK;
+      } else {
+        len = p.hot_len ? p.hot_len[b] : 0;
+        if (len < 0 || len > p.W_max) {
+          report(p.err, TQ_ERR_CAPACITY);
+          len = len < 0 ? 0 : p.W_max;
+        }
+        units = (len + HOT_TOK - 1) / HOT_TOK;
+      }
+      slen[sg] = len;
+    }
+    int total;
+    const int ex = block_exclusive_scan(units, scratch, total);
+    if (sg < S) uoff[sg] = carry_s + ex;
+    __syncthreads();
+    if (threadIdx.x == 0) carry_s += total;
+    __syncthreads();
+  }
+  const int U = carry_s;
+  // spread the units over min(Wtot, U) warps so that every one of them owns
+  // at least one unit: the warps touching a segment are then consecutive and
+  // each writes a partial record
+  const int Weff = U < p.Wtot ? U : p.Wtot;
+  if (threadIdx.x == 0) {
+    uoff[S] = U;
+    p.w.sched[0] = U;
+    p.w.sched[1] = Weff;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) carry_s = 0;
+  __syncthreads();
+  for (int base = 0; base < S; base += blockDim.x) {
+    const int sg = base + threadIdx.x;
+    int nwarps = 0;
+    if (sg < S) {
+      const int a = uoff[sg], e = uoff[sg + 1];
+      if (e > a) nwarps = warp_of(e - 1, U, Weff) - warp_of(a, U, Weff) + 1;
+    }
+    int total;
+    const int ex = block_exclusive_scan(nwarps, scratch, total);
+    if (sg < S) soff[sg] = carry_s + ex;
+    __syncthreads();
+    if (threadIdx.x == 0) carry_s += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) soff[S] = carry_s;
+}
+
+__device__ __forceinline__ uint32_t pack_split(float xlo, float xhi, int part) {
+  uint16_t h0, l0, h1, l1;
+  split_f16(xlo, h0, l0);
+  split_f16(xhi, h1, l1);
+  return part == 0 ? (static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16))
+                   : (static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16));
+}
+
+// scale factor 2^E putting max|w| in [128, 256): keeps the fp16 lo parts normal
+__device__ __forceinline__ float prescale_for(float mx) {
+  if (!(mx > 0.0f) || !isfinite(mx)) return 1.0f;
+  int e;
+  frexpf(mx, &e);  // mx = f * 2^e, f in [0.5, 1)
+  return ldexpf(1.0f, 8 - e);
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(128) prep_kernel(Params p) {
+  using C = Cfg<D, G>;
+  const int BH = p.B * p.Hkv;
+  if (blockIdx.x == BH) {
+    build_schedule(p);
+    return;
+  }
+  const int bh = blockIdx.x, b = bh / p.Hkv, kvh = bh % p.Hkv;
+  __shared__ float sq[G][D], sqr[G][D], sqs[G][D];
+  __shared__ unsigned smax[2][G];
+  __shared__ float sfac[2][G];
+  const int tid = threadIdx.x;
+  if (tid < 2 * G) smax[tid / G][tid % G] = 0u;
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    const int g = i / D, j = i % D;
+    sq[g][j] = load_as_float(p.q, (static_cast<size_t>(b) * p.Hq + kvh * G + g) * D + j,
+                             static_cast<tq_dtype>(p.q_dtype));
+  }
+  __syncthreads();
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    const int g = i / D, j = i % D;
+    const float4* row = reinterpret_cast<const float4*>(p.rot + static_cast<size_t>(j) * D);
+    float a = 0.0f;
+#pragma unroll 4
+    for (int k4 = 0; k4 < D / 4; ++k4) {
+      float4 r = row[k4];
+      a = fmaf(r.x, sq[g][4 * k4], a);
+      a = fmaf(r.y, sq[g][4 * k4 + 1], a);
+      a = fmaf(r.z, sq[g][4 * k4 + 2], a);
+      a = fmaf(r.w, sq[g][4 * k4 + 3], a);
+    }
+    sqr[g][j] = a;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    const int g = i / D, r = i % D;
+    const float4* row = reinterpret_cast<const float4*>(p.qjl + static_cast<size_t>(r) * D);
+    float a = 0.0f;
+#pragma unroll 4
+    for (int k4 = 0; k4 < D / 4; ++k4) {
+      float4 s = row[k4];
+      a = fmaf(s.x, sqr[g][4 * k4], a);
+      a = fmaf(s.y, sqr[g][4 * k4 + 1], a);
+      a = fmaf(s.z, sqr[g][4 * k4 + 2], a);
+      a = fmaf(s.w, sqr[g][4 * k4 + 3], a);
+    }
+    sqs[g][r] = a;
+  }
+  __syncthreads();
+  const float w1c = p.sl * p.kc0, w2c = p.sl * 128.0f * (p.kc1 - p.kc0), w3c = p.sl * p.alpha;
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    const int g = i / D, j = i % D;
+    float mc = fmaxf(fmaxf(fabsf(w1c * sqr[g][j]), fabsf(w2c * sqr[g][j])), fabsf(w3c * sqs[g][j]));
+    float mh = fabsf(p.sl * sq[g][j]);
+    atomicMax(&smax[0][g], __float_as_uint(mc));
+    atomicMax(&smax[1][g], __float_as_uint(mh));
+  }
+  __syncthreads();
+  if (tid < 2 * G) {
+    const int dom = tid / G, g = tid % G;
+    const float f = prescale_for(__uint_as_float(smax[dom][g]));
+    sfac[dom][g] = f;
+    p.w.desc[(static_cast<size_t>(bh) * 2 + dom) * 8 + g] = 1.0f / f;
+  }
+  __syncthreads();
+  // cold fragments: r = (pk * NT + nt) * 2 + reg; lane = 4 g' + c'
+  for (int idx = tid; idx < C::RC * 32; idx += blockDim.x) {
+    const int r = idx >> 5, lane = idx & 31;
+    const int reg = r & 1, nt = (r >> 1) % C::NT, pk = (r >> 1) / C::NT;
+    const int gc = lane >> 2, cc = lane & 3;
+    const int h = nt * 4 + (gc >> 1), part = gc & 1;
+    uint32_t val = 0u;
+    if (h < G) {
+      const float f = sfac[0][h];
+      if (pk < 2 * C::KS) {
+        const int s = pk % C::KS;
+        const float wc = f * ((pk < C::KS) ? w1c : w2c);
+        const int P = cc * (D / 8) + 2 * s + reg;
+        const int jlo = 16 * (P >> 3) + (P & 7);
+        val = pack_split(wc * sqr[h][jlo], wc * sqr[h][jlo + 8], part);
+      } else {
+        const int s = pk - 2 * C::KS;
+        const float wc = f * w3c;
+        const int P = cc * (D / 8) + 2 * s + reg;
+        const int ilo = 32 * (P >> 4) + (P & 15);
+        val = pack_split(wc * sqs[h][ilo], wc * sqs[h][ilo + 16], part);
+      }
+    }
+    p.w.frag_c[(static_cast<size_t>(bh) * C::RC + r) * 32 + lane] = val;
+  }
+  // hot fragments: natural coordinate order, k = 16 s + 2 c' (+1), + 8 for reg 1
+  for (int idx = tid; idx < C::RH * 32; idx += blockDim.x) {
+    const int r = idx >> 5, lane = idx & 31;
+    const int reg = r & 1, nt = (r >> 1) % C::NT, s = (r >> 1) / C::NT;
+    const int gc = lane >> 2, cc = lane & 3;
+    const int h = nt * 4 + (gc >> 1), part = gc & 1;
+    uint32_t val = 0u;
+    if (h < G) {
+      const float wc = sfac[1][h] * p.sl;
+      const int k0 = 16 * s + 2 * cc + 8 * reg;
+      val = pack_split(wc * sq[h][k0], wc * sq[h][k0 + 1], part);
+    }
+    p.w.frag_h[(static_cast<size_t>(bh) * C::RH + r) * 32 + lane] = val;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. attention
+// ---------------------------------------------------------------------------
+template <int D, int G>
+__device__ __forceinline__ void issue_unit(const Params& p, int sg, int lu, int len, uint8_t* dst,
+                                           uint32_t bar, int lane) {
+  using C = Cfg<D, G>;
+  const int bh = sg >> 1;
+  const uint32_t d0 = smem_u32(dst);
+  if ((sg & 1) == 0) {
+    const int page = p.page_table[static_cast<size_t>(bh) * p.max_pages + (lu >> 1)];
+    const bool ok = page >= 0 && page < p.pool_pages;
+    if (!ok) {
+      if (lane == 0) {
+        report(p.err, TQ_ERR_CAPACITY);
+        mbar_arrive_expect_tx(bar, 0);
+      }
+      __syncwarp();
+      return;
+    }
+    const int half = lu & 1;
+    const uint8_t* base = p.pool + static_cast<size_t>(page) * p.page_bytes;
+    if (lane == 0) mbar_arrive_expect_tx(bar, C::COLD_B);
+    __syncwarp();
+    if (lane == 0) bulk_g2s(d0, base + p.off_kc + half * C::KC_B, C::KC_B, bar);
+    if (lane == 1) bulk_g2s(d0 + C::OFF_QS, base + p.off_qs + half * C::QS_B, C::QS_B, bar);
+    if (lane == 2) bulk_g2s(d0 + C::OFF_VC, base + p.off_vc + half * C::VC_B, C::VC_B, bar);
+    if (lane == 3) bulk_g2s(d0 + C::OFF_KN, base + p.off_kn + half * 2 * COLD_TOK, 2 * COLD_TOK, bar);
+    if (lane == 4) bulk_g2s(d0 + C::OFF_KG, base + p.off_kg + half * 2 * COLD_TOK, 2 * COLD_TOK, bar);
+    if (lane == 5) bulk_g2s(d0 + C::OFF_VN, base + p.off_vn + half * 2 * COLD_TOK, 2 * COLD_TOK, bar);
+  } else {
+    const int t0 = lu * HOT_TOK;
+    const int rows = min(HOT_TOK, len - t0);
+    if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * 2u * (2u * D));
+    __syncwarp();
+    const int r = lane & 15, isv = lane >> 4;
+    if (r < rows) {
+      const __half* src = (isv ? p.v_hot : p.k_hot) +
+                          (static_cast<size_t>(bh) * p.W_max + t0 + r) * D;
+      bulk_g2s(d0 + isv * HOT_TOK * C::HROW + r * C::HROW, src, 2 * D, bar);
+    }
+  }
+}
+
+// 8 value nibbles of a word (4 coordinates x 2 tokens) -> 4 half2 (token
+// even in the low half), through an fp16 table of the 8 magnitudes
+__device__ __forceinline__ void dequant_values(uint32_t x, uint32_t tl0, uint32_t tl1,
+                                               uint32_t th0, uint32_t th1, uint32_t (&h)[4]) {
+  const uint32_t x4 = x << 4;
+  const uint32_t s01 = x & 0x7777u;
+  const uint32_t s23 = (x >> 16) & 0x7777u;
+  const uint32_t lo01 = prmt(tl0, tl1, s01), hi01 = prmt(th0, th1, s01);
+  const uint32_t lo23 = prmt(tl0, tl1, s23), hi23 = prmt(th0, th1, s23);
+  // sign bits of the 8 nibbles as 0x00 / 0xFF bytes (prmt sign replication)
+  const uint32_t m01 = prmt(x, x4, 0x9D8Cu), m23 = prmt(x, x4, 0xBFAEu);
+  const uint32_t hs01 = hi01 | (m01 & 0x80808080u), hs23 = hi23 | (m23 & 0x80808080u);
+  h[0] = prmt(lo01, hs01, 0x5140u);
+  h[1] = prmt(lo01, hs01, 0x7362u);
+  h[2] = prmt(lo23, hs23, 0x5140u);
+  h[3] = prmt(lo23, hs23, 0x7362u);
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
+  using C = Cfg<D, G>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  uint8_t* slots = smem + warp * (C::NSLOT * C::SLOT);
+  uint8_t* pbuf = smem + NW * C::NSLOT * C::SLOT + warp * C::PBUF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NW * (C::NSLOT * C::SLOT + C::PBUF)) +
+                   warp * C::NSLOT;
+
+  const int* sched = p.w.sched;
+  const int U = sched[0];
+  const int* uoff = sched + 4;
+  const int* soff = uoff + p.S + 1;
+  const int* slen = soff + p.S + 1;
+  const int Weff = sched[1];
+  const int gw = blockIdx.x * NW + warp;
+  if (U <= 0 || gw >= Weff) return;
+  const int u0 = static_cast<int>(static_cast<long long>(gw) * U / Weff);
+  const int u1 = static_cast<int>(static_cast<long long>(gw + 1) * U / Weff);
+  if (u0 >= u1) return;
+
+  if (lane < C::NSLOT) mbar_init(smem_u32(&bars[lane]), 1);
+  mbar_init_fence();
+  // P' tile: columns of absent heads stay zero
+  for (int i = lane; i < C::PBUF / 4; i += 32) reinterpret_cast<uint32_t*>(pbuf)[i] = 0u;
+  __syncwarp();
+
+  // segment containing u0 (largest sg with uoff[sg] <= u0)
+  int lo = 0, hi = p.S - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (uoff[mid] <= u0) lo = mid; else hi = mid - 1;
+  }
+  // issue cursor
+  int isg = lo, ilu = u0 - uoff[lo];
+  int iu = u0;
+  auto issue_next = [&](int slot) {
+    while (uoff[isg + 1] <= iu) { ++isg; ilu = 0; }
+    issue_unit<D, G>(p, isg, ilu, slen[isg], slots + slot * C::SLOT, smem_u32(&bars[slot]), lane);
+    ++iu;
+    ++ilu;
+  };
+  for (int s = 0; s < C::NSLOT && iu < u1; ++s) issue_next(s);
+
+  // value dequant tables: low and high bytes of fp16(val_c[k])
+  uint32_t tl0 = 0, tl1 = 0, th0 = 0, th1 = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t hb = __half_as_ushort(__float2half_rn(p.vc[k]));
+    if (k < 4) {
+      tl0 |= (hb & 0xFFu) << (8 * k);
+      th0 |= (hb >> 8) << (8 * k);
+    } else {
+      tl1 |= (hb & 0xFFu) << (8 * (k - 4));
+      th1 |= (hb >> 8) << (8 * (k - 4));
+    }
+  }
+
+  // consume cursor
+  int sg = lo, lu = u0 - uoff[lo];
+  uint32_t bfr[C::RC];
+  float dsc[C::NT];
+  float mrun[C::NT], lrun[C::NT];
+  float oacc[C::KS][4];
+  auto load_segment = [&]() {
+    const int bh = sg >> 1, dom = sg & 1;
+    if (dom == 0) {
+#pragma unroll
+      for (int r = 0; r < C::RC; ++r)
+        bfr[r] = p.w.frag_c[(static_cast<size_t>(bh) * C::RC + r) * 32 + lane];
+    } else {
+#pragma unroll
+      for (int r = 0; r < C::RH; ++r)
+        bfr[r] = p.w.frag_h[(static_cast<size_t>(bh) * C::RH + r) * 32 + lane];
+    }
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt) {
+      const int h = c + 4 * nt;
+      dsc[nt] = (h < G) ? p.w.desc[(static_cast<size_t>(bh) * 2 + dom) * 8 + h] : 0.0f;
+      mrun[nt] = NEG_INF;
+      lrun[nt] = 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < C::KS; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.0f;
+  };
+  load_segment();
+
+  // online-softmax update for scores sv (log2 domain); returns nothing, rescales oacc
+  auto softmax_update = [&](float* sv, int count_per_nt) {
+    float alpha[C::NT];
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt) {
+      float mx = NEG_INF;
+      for (int i = 0; i < count_per_nt; ++i) mx = fmaxf(mx, sv[nt * count_per_nt + i]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float mnew = fmaxf(mrun[nt], mx);
+      float ps = 0.0f;
+      if (mnew == NEG_INF) {
+        alpha[nt] = 1.0f;
+        for (int i = 0; i < count_per_nt; ++i) sv[nt * count_per_nt + i] = 0.0f;
+      } else {
+        alpha[nt] = exp2f(mrun[nt] - mnew);
+        for (int i = 0; i < count_per_nt; ++i) {
+          const float e = exp2f(sv[nt * count_per_nt + i] - mnew);
+          sv[nt * count_per_nt + i] = e;
+          ps += e;
+        }
+      }
+      mrun[nt] = mnew;
+      lrun[nt] = lrun[nt] * alpha[nt] + ps;
+    }
+    // accumulator columns 2c, 2c+1 hold heads 2c and 2c+1
+    const int hA = 2 * c, hB = 2 * c + 1;
+    const int srcA = (lane & ~3) | (hA & 3), srcB = (lane & ~3) | (hB & 3);
+    float aA = __shfl_sync(0xffffffffu, alpha[0], srcA);
+    float aB = __shfl_sync(0xffffffffu, alpha[0], srcB);
+    if (C::NT > 1) {
+      const float a1A = __shfl_sync(0xffffffffu, alpha[C::NT > 1 ? 1 : 0], srcA);
+      const float a1B = __shfl_sync(0xffffffffu, alpha[C::NT > 1 ? 1 : 0], srcB);
+      if (hA >= 4) aA = a1A;
+      if (hB >= 4) aB = a1B;
+    }
+#pragma unroll
+    for (int i = 0; i < C::KS; ++i) {
+      oacc[i][0] *= aA;
+      oacc[i][1] *= aB;
+      oacc[i][2] *= aA;
+      oacc[i][3] *= aB;
+    }
+  };
+
+  auto flush_segment = [&]() {
+    const int bh = sg >> 1, dom = sg & 1;
+    float lt[C::NT];
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt) {
+      float l = lrun[nt];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      lt[nt] = l;
+    }
+    const int first = warp_of(uoff[sg], U, Weff);
+    float* rec = p.w.part + static_cast<size_t>(soff[sg] + (gw - first)) * G * (D + 2);
+    if (g == 0) {
+#pragma unroll
+      for (int nt = 0; nt < C::NT; ++nt) {
+        const int h = c + 4 * nt;
+        if (h < G) {
+          rec[h] = mrun[nt];
+          rec[G + h] = lt[nt];
+        }
+      }
+    }
+    float* o = rec + 2 * G;
+#pragma unroll
+    for (int i = 0; i < C::KS; ++i) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int h = 2 * c + (e & 1);
+        int coord;
+        if (dom == 0)
+          coord = g * (D / 8) + 4 * (i >> 1) + 2 * (i & 1) + (e >> 1);
+        else
+          coord = 16 * i + g + 8 * (e >> 1);
+        if (h < G) o[h * D + coord] = oacc[i][e];
+      }
+    }
+    (void)bh;
+  };
+
+  const uint32_t pb_addr = smem_u32(pbuf);
+  for (int u = u0, k = 0; u < u1; ++u, ++k) {
+    const int slot = k % C::NSLOT;
+    const uint32_t parity = static_cast<uint32_t>(k / C::NSLOT) & 1u;
+    uint8_t* sb = slots + slot * C::SLOT;
+    if (!mbar_wait_bounded(smem_u32(&bars[slot]), parity)) {
+      if (lane == 0) report(p.err, TQ_ERR_TIMEOUT);
+      // let copies already in flight land before the CTA can exit
+      for (int s = 0; s < C::NSLOT; ++s)
+        mbar_wait_bounded(smem_u32(&bars[s]), static_cast<uint32_t>((k + s) / C::NSLOT) & 1u);
+      return;
+    }
+    const int bh = sg >> 1;
+    const int len = slen[sg];
+    if ((sg & 1) == 0) {
+      // ---------------- cold unit: 64 tokens ----------------
+      const int page = p.page_table[static_cast<size_t>(bh) * p.max_pages + (lu >> 1)];
+      const int nv = (page >= 0 && page < p.pool_pages) ? min(COLD_TOK, len - lu * COLD_TOK) : 0;
+      float sv[C::NT * 8];
+      const __half* kn = reinterpret_cast<const __half*>(sb + C::OFF_KN);
+      const uint16_t* kg = reinterpret_cast<const uint16_t*>(sb + C::OFF_KG);
+      const __half* vn = reinterpret_cast<const __half*>(sb + C::OFF_VN);
+      const int qword = (c * (D / 8)) >> 4, qsb = (c * (D / 8)) & 15;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        const int t0 = 16 * mt + g, t1 = t0 + 8;
+        uint32_t kw0[C::WPT], kw1[C::WPT];
+#pragma unroll
+        for (int w = 0; w < C::WPT; ++w) {
+          kw0[w] = *reinterpret_cast<const uint32_t*>(sb + t0 * (D / 4) + 4 * (c * C::WPT + w));
+          kw1[w] = *reinterpret_cast<const uint32_t*>(sb + t1 * (D / 4) + 4 * (c * C::WPT + w));
+        }
+        const uint32_t qw0 = *reinterpret_cast<const uint32_t*>(sb + C::OFF_QS + t0 * (D / 8) + 4 * qword);
+        const uint32_t qw1 = *reinterpret_cast<const uint32_t*>(sb + C::OFF_QS + t1 * (D / 8) + 4 * qword);
+        const uint32_t gg0 = static_cast<uint32_t>(kg[t0]) * 0x10001u;
+        const uint32_t gg1 = static_cast<uint32_t>(kg[t1]) * 0x10001u;
+        float acc[C::NT][4];
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+#pragma unroll
+        for (int s = 0; s < C::KS; ++s) {
+          const int w = s >> 2, sh = 4 * (s & 3);
+          const uint32_t x0a = kw0[w] << sh, x0b = kw0[w] << (sh + 1);
+          const uint32_t x1a = kw1[w] << sh, x1b = kw1[w] << (sh + 1);
+          const uint32_t a0 = (x0a & 0x80008000u) | 0x3C003C00u, a1 = (x1a & 0x80008000u) | 0x3C003C00u;
+          const uint32_t a2 = (x0b & 0x80008000u) | 0x3C003C00u, a3 = (x1b & 0x80008000u) | 0x3C003C00u;
+          const uint32_t m0 = x0a & 0xA000A000u, m1 = x1a & 0xA000A000u;
+          const uint32_t m2 = x0b & 0xA000A000u, m3 = x1b & 0xA000A000u;
+#pragma unroll
+          for (int nt = 0; nt < C::NT; ++nt) {
+            mma_f16(acc[nt], a0, a1, a2, a3, bfr[(s * C::NT + nt) * 2], bfr[(s * C::NT + nt) * 2 + 1]);
+            mma_f16(acc[nt], m0, m1, m2, m3, bfr[((C::KS + s) * C::NT + nt) * 2],
+                    bfr[((C::KS + s) * C::NT + nt) * 2 + 1]);
+          }
+        }
+#pragma unroll
+        for (int s = 0; s < C::KS; ++s) {
+          const int sh = qsb + 2 * s;
+          const uint32_t a0 = ((qw0 << sh) & 0x80008000u) | gg0;
+          const uint32_t a1 = ((qw1 << sh) & 0x80008000u) | gg1;
+          const uint32_t a2 = ((qw0 << (sh + 1)) & 0x80008000u) | gg0;
+          const uint32_t a3 = ((qw1 << (sh + 1)) & 0x80008000u) | gg1;
+#pragma unroll
+          for (int nt = 0; nt < C::NT; ++nt)
+            mma_f16(acc[nt], a0, a1, a2, a3, bfr[((2 * C::KS + s) * C::NT + nt) * 2],
+                    bfr[((2 * C::KS + s) * C::NT + nt) * 2 + 1]);
+        }
+        const float n0 = __half2float(kn[t0]), n1 = __half2float(kn[t1]);
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt) {
+          const float v0 = (acc[nt][0] + acc[nt][1]) * dsc[nt] * n0;
+          const float v1 = (acc[nt][2] + acc[nt][3]) * dsc[nt] * n1;
+          sv[nt * 8 + 2 * mt] = (t0 < nv) ? v0 : NEG_INF;
+          sv[nt * 8 + 2 * mt + 1] = (t1 < nv) ? v1 : NEG_INF;
+        }
+      }
+      softmax_update(sv, 8);
+      // P' = p * n_v as fp16 into the [64 tokens][8 heads] tile
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        const int t0 = 16 * mt + g, t1 = t0 + 8;
+        const float nv0 = __half2float(vn[t0]), nv1 = __half2float(vn[t1]);
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt) {
+          const int h = c + 4 * nt;
+          if (h < G) {
+            const float p0 = (t0 < nv) ? sv[nt * 8 + 2 * mt] * nv0 : 0.0f;
+            const float p1 = (t1 < nv) ? sv[nt * 8 + 2 * mt + 1] * nv1 : 0.0f;
+            reinterpret_cast<__half*>(pbuf)[t0 * 8 + h] = __float2half_rn(p0);
+            reinterpret_cast<__half*>(pbuf)[t1 * 8 + h] = __float2half_rn(p1);
+          }
+        }
+      }
+      __syncwarp();
+      const uint8_t* vc = sb + C::OFF_VC;
+      const int chunk = (g + 2 * c) & 7;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        uint32_t bp0, bp1;
+        ldsm_x2_t(pb_addr + (16 * mt + (lane & 15)) * 16, bp0, bp1);
+        const int pa = 8 * mt + c, pb2 = pa + 4;
+        const uint8_t* ra = vc + pa * D + chunk * (D / 8);
+        const uint8_t* rb = vc + pb2 * D + chunk * (D / 8);
+        uint32_t xa[C::WV], xb[C::WV];
+        if constexpr (C::WV == 4) {
+          const uint4 va = *reinterpret_cast<const uint4*>(ra);
+          const uint4 vb = *reinterpret_cast<const uint4*>(rb);
+          xa[0] = va.x; xa[1] = va.y; xa[2] = va.z; xa[3] = va.w;
+          xb[0] = vb.x; xb[1] = vb.y; xb[2] = vb.z; xb[3] = vb.w;
+        } else {
+          const uint2 va = *reinterpret_cast<const uint2*>(ra);
+          const uint2 vb = *reinterpret_cast<const uint2*>(rb);
+          xa[0] = va.x; xa[1] = va.y;
+          xb[0] = vb.x; xb[1] = vb.y;
+        }
+#pragma unroll
+        for (int wq = 0; wq < C::WV; ++wq) {
+          uint32_t ha[4], hb[4];
+          dequant_values(xa[wq], tl0, tl1, th0, th1, ha);
+          dequant_values(xb[wq], tl0, tl1, th0, th1, hb);
+          mma_f16(oacc[2 * wq], ha[0], ha[1], hb[0], hb[1], bp0, bp1);
+          mma_f16(oacc[2 * wq + 1], ha[2], ha[3], hb[2], hb[3], bp0, bp1);
+        }
+      }
+    } else {
+      // ---------------- hot unit: 16 tokens ----------------
+      const int nv = min(HOT_TOK, len - lu * HOT_TOK);
+      const uint8_t* kt = sb;
+      uint8_t* vt = sb + HOT_TOK * C::HROW;
+      if (nv < HOT_TOK) {  // rows past the window were not copied: zero them
+        for (int i = lane; i < (HOT_TOK - nv) * (C::HROW / 4); i += 32)
+          reinterpret_cast<uint32_t*>(vt + nv * C::HROW)[i] = 0u;
+        __syncwarp();
+      }
+      float acc[C::NT][4];
+#pragma unroll
+      for (int nt = 0; nt < C::NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+      const uint32_t kt_addr = smem_u32(kt);
+#pragma unroll
+      for (int s = 0; s < C::KS; ++s) {
+        const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int col = 16 * s + (lane >> 4) * 8;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(kt_addr + row * C::HROW + col * 2, a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt)
+          mma_f16(acc[nt], a0, a1, a2, a3, bfr[(s * C::NT + nt) * 2], bfr[(s * C::NT + nt) * 2 + 1]);
+      }
+      float sv[C::NT * 2];
+#pragma unroll
+      for (int nt = 0; nt < C::NT; ++nt) {
+        sv[nt * 2] = (g < nv) ? (acc[nt][0] + acc[nt][1]) * dsc[nt] : NEG_INF;
+        sv[nt * 2 + 1] = (g + 8 < nv) ? (acc[nt][2] + acc[nt][3]) * dsc[nt] : NEG_INF;
+      }
+      softmax_update(sv, 2);
+#pragma unroll
+      for (int nt = 0; nt < C::NT; ++nt) {
+        const int h = c + 4 * nt;
+        if (h < G) {
+          reinterpret_cast<__half*>(pbuf)[g * 8 + h] = __float2half_rn(sv[nt * 2]);
+          reinterpret_cast<__half*>(pbuf)[(g + 8) * 8 + h] = __float2half_rn(sv[nt * 2 + 1]);
+        }
+      }
+      __syncwarp();
+      uint32_t bp0, bp1;
+      ldsm_x2_t(pb_addr + (lane & 15) * 16, bp0, bp1);
+      const uint32_t vt_addr = smem_u32(vt);
+#pragma unroll
+      for (int i = 0; i < C::KS; ++i) {
+        const int mi = lane >> 3;
+        const int tok = (lane & 7) + (mi >> 1) * 8;
+        const int col = 16 * i + (mi & 1) * 8;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(vt_addr + tok * C::HROW + col * 2, a0, a1, a2, a3);
+        mma_f16(oacc[i], a0, a1, a2, a3, bp0, bp1);
+      }
+    }
+    // all lanes are done with this slot: refill it
+    __syncwarp();
+    fence_proxy_async_smem();
+    if (iu < u1) issue_next(slot);
+    ++lu;
+    if (u + 1 == u1 || u + 1 >= uoff[sg + 1]) {
+      flush_segment();
+      if (u + 1 < u1) {
+        ++sg;
+        while (uoff[sg + 1] <= u + 1) ++sg;
+        lu = 0;
+        load_segment();
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. combine
+// ---------------------------------------------------------------------------
+template <int D, int G>
+__global__ void __launch_bounds__(D) combine_kernel(Params p) {
+  const int bh = blockIdx.x, b = bh / p.Hkv, kvh = bh % p.Hkv;
+  const int* sched = p.w.sched;
+  const int* soff = sched + 4 + p.S + 1;
+  const int j = threadIdx.x;
+  __shared__ float so[D];
+  for (int g = 0; g < G; ++g) {
+    float M[2], L[2], O[2];
+    for (int dom = 0; dom < 2; ++dom) {
+      const int sg = 2 * bh + dom;
+      const int a = soff[sg], e = soff[sg + 1];
+      float mx = -__builtin_huge_valf();
+      for (int s = a; s < e; ++s) {
+        const float* rec = p.w.part + static_cast<size_t>(s) * G * (D + 2);
+        if (rec[G + g] > 0.0f) mx = fmaxf(mx, rec[g]);
+      }
+      float l = 0.0f, o = 0.0f;
+      if (mx != -__builtin_huge_valf()) {
+        for (int s = a; s < e; ++s) {
+          const float* rec = p.w.part + static_cast<size_t>(s) * G * (D + 2);
+          const float lw = rec[G + g];
+          if (lw > 0.0f) {
+            const float f = exp2f(rec[g] - mx);
+            l += lw * f;
+            o += rec[2 * G + g * D + j] * f;
+          }
+        }
+      }
+      M[dom] = mx;
+      L[dom] = l;
+      O[dom] = o;
+    }
+    // cold accumulator is in the rotated domain: o_cold = Pi^T o_rot
+    __syncthreads();
+    so[j] = O[0];
+    __syncthreads();
+    float oc = 0.0f;
+    if (L[0] > 0.0f) {
+#pragma unroll 8
+      for (int i = 0; i < D; ++i) oc = fmaf(p.rot[static_cast<size_t>(i) * D + j], so[i], oc);
+    }
+    const float Mx = fmaxf(M[0], M[1]);
+    float res = 0.0f;
+    if (Mx != -__builtin_huge_valf()) {
+      const float fc = (L[0] > 0.0f) ? exp2f(M[0] - Mx) : 0.0f;
+      const float fh = (L[1] > 0.0f) ? exp2f(M[1] - Mx) : 0.0f;
+      const float den = L[0] * fc + L[1] * fh;
+      res = (den > 0.0f) ? (oc * fc + O[1] * fh) / den : 0.0f;
+    }
+    p.out[(static_cast<size_t>(b) * p.Hq + kvh * G + g) * D + j] = res;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct WsLayout {
+  size_t sched, frag_c, frag_h, desc, part, total;
+};
+
+template <int D, int G>
+WsLayout ws_layout(int B, int Hkv, int Wtot) {
+  using C = Cfg<D, G>;
+  const size_t BH = static_cast<size_t>(B) * Hkv, S = 2 * BH;
+  WsLayout L;
+  size_t off = 0;
+  L.sched = off;
+  off = align256(off + sizeof(int) * (4 + 2 * (S + 1) + S));
+  L.frag_c = off;
+  off = align256(off + sizeof(uint32_t) * BH * C::RC * 32);
+  L.frag_h = off;
+  off = align256(off + sizeof(uint32_t) * BH * C::RH * 32);
+  L.desc = off;
+  off = align256(off + sizeof(float) * BH * 16);
+  L.part = off;
+  off = align256(off + sizeof(float) * (static_cast<size_t>(Wtot) + S) * G * (D + 2));
+  L.total = off;
+  return L;
+}
+
+template <int D, int G>
+int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st) {
+  using C = Cfg<D, G>;
+  const int grid = ctx->num_sms;
+  p.Wtot = grid * NW;
+  p.S = 2 * p.B * p.Hkv;
+  const WsLayout L = ws_layout<D, G>(p.B, p.Hkv, p.Wtot);
+  if (ws_bytes < L.total) return TQ_ERR_INVALID_ARG;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  p.w.sched = reinterpret_cast<int*>(base + L.sched);
+  p.w.frag_c = reinterpret_cast<uint32_t*>(base + L.frag_c);
+  p.w.frag_h = reinterpret_cast<uint32_t*>(base + L.frag_h);
+  p.w.desc = reinterpret_cast<float*>(base + L.desc);
+  p.w.part = reinterpret_cast<float*>(base + L.part);
+  static bool attr_set[2][9] = {};
+  bool& set = attr_set[D == 128][G];
+  if (!set) {
+    if (cudaFuncSetAttribute(attn_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    set = true;
+  }
+  prep_kernel<D, G><<<p.B * p.Hkv + 1, 128, 0, st>>>(p);
+  if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
+  attn_kernel<D, G><<<grid, NW * 32, C::SMEM, st>>>(p);
+  if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
+  combine_kernel<D, G><<<p.B * p.Hkv, D, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+}  // namespace dec
+
+size_t decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max) {
+  (void)max_pages;
+  (void)W_max;
+  if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0) return 0;
+  const int G = Hq / Hkv;
+  const int Wtot = ctx->num_sms * dec::NW;
+  // the largest layout over the supported group sizes of this head dim
+  size_t best = 0;
+  auto take = [&](size_t v) { best = v > best ? v : best; };
+  if (ctx->cfg.head_dim == 128) {
+    if (G == 1) take(dec::ws_layout<128, 1>(B, Hkv, Wtot).total);
+    if (G == 2) take(dec::ws_layout<128, 2>(B, Hkv, Wtot).total);
+    if (G == 4) take(dec::ws_layout<128, 4>(B, Hkv, Wtot).total);
+    if (G == 8) take(dec::ws_layout<128, 8>(B, Hkv, Wtot).total);
+  } else {
+    if (G == 1) take(dec::ws_layout<64, 1>(B, Hkv, Wtot).total);
+    if (G == 2) take(dec::ws_layout<64, 2>(B, Hkv, Wtot).total);
+    if (G == 4) take(dec::ws_layout<64, 4>(B, Hkv, Wtot).total);
+    if (G == 8) take(dec::ws_layout<64, 8>(B, Hkv, Wtot).total);
+  }
+  return best;
+}
+
+int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq, int Hkv,
+                  float scale, const void* k_hot, const void* v_hot, int W_max,
+                  const int32_t* hot_len, const uint8_t* pool, int64_t pool_pages,
+                  const int32_t* page_table, int max_pages, const int32_t* cold_len, float* out,
+                  void* ws, size_t ws_bytes, void* stream) {
+  const int d = ctx->cfg.head_dim;
+  const int G = Hq / Hkv;
+  const PageLayout L = page_layout(d, ctx->cfg.qjl_dim, true);
+  dec::Params p{};
+  p.q = q;
+  p.q_dtype = static_cast<int>(q_dtype);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.max_pages = max_pages;
+  p.W_max = W_max;
+  const float sc = (scale == 0.0f) ? 1.0f / std::sqrt(static_cast<float>(d)) : scale;
+  p.sl = sc * 1.4426950408889634f;
+  p.k_hot = static_cast<const __half*>(k_hot);
+  p.v_hot = static_cast<const __half*>(v_hot);
+  p.hot_len = hot_len;
+  p.pool = pool;
+  p.pool_pages = pool_pages;
+  p.page_bytes = static_cast<long long>(L.bytes);
+  p.off_kc = static_cast<int>(L.kc);
+  p.off_qs = static_cast<int>(L.qs);
+  p.off_vc = static_cast<int>(L.vc);
+  p.off_kn = static_cast<int>(L.kn);
+  p.off_kg = static_cast<int>(L.kg);
+  p.off_vn = static_cast<int>(L.vn);
+  p.page_table = page_table;
+  p.cold_len = cold_len;
+  p.out = out;
+  p.rot = ctx->dev.rot;
+  p.qjl = ctx->dev.qjl;
+  p.kc0 = ctx->cb.key_c[0];
+  p.kc1 = ctx->cb.key_c[1];
+  p.alpha = std::sqrt(3.14159265358979323846f / 2.0f) / static_cast<float>(ctx->cfg.qjl_dim);
+  for (int k = 0; k < 8; ++k) p.vc[k] = ctx->cb.val_c[k];
+  p.err = ctx->dev.err;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128) {
+    switch (G) {
+      case 1: return dec::run<128, 1>(ctx, p, ws, ws_bytes, st);
+      case 2: return dec::run<128, 2>(ctx, p, ws, ws_bytes, st);
+      case 4: return dec::run<128, 4>(ctx, p, ws, ws_bytes, st);
+      case 8: return dec::run<128, 8>(ctx, p, ws, ws_bytes, st);
+    }
+  } else if (d == 64) {
+    switch (G) {
+      case 1: return dec::run<64, 1>(ctx, p, ws, ws_bytes, st);
+      case 2: return dec::run<64, 2>(ctx, p, ws, ws_bytes, st);
+      case 4: return dec::run<64, 4>(ctx, p, ws, ws_bytes, st);
+      case 8: return dec::run<64, 8>(ctx, p, ws, ws_bytes, st);
+    }
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+
+}  // namespace tq

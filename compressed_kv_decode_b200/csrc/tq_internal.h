@@ -52,6 +52,8 @@ struct tq_ctx {
   tq::Codebook cb;
   tq::DeviceTables dev;
   void* dev_block;  // single allocation holding every device table
+  void* prof_start; // optional cudaEvent_t pair around the main kernel
+  void* prof_stop;
 };
 
 namespace tq {

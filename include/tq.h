@@ -41,6 +41,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -93,16 +99,16 @@ typedef struct tq_ctx tq_ctx; /* opaque; immutable after creation */
  *  val_c, val_t: the same at value_bits.
  * Any output may be NULL.  Cost: a fraction of a second (fp64 solves).
  */
-tq_status tq_generate_params(const tq_config* cfg, float* rot, float* qjl, float* key_c,
+TQ_API tq_status tq_generate_params(const tq_config* cfg, float* rot, float* qjl, float* key_c,
                              float* key_t, float* val_c, float* val_t);
 
 /* Generate the tables (as tq_generate_params) and upload them to the current
  * device.  *out receives the context; release it with tq_destroy. */
-tq_status tq_init_codebook(const tq_config* cfg, tq_ctx** out);
+TQ_API tq_status tq_init_codebook(const tq_config* cfg, tq_ctx** out);
 
 /* Copy the context's tables to host arrays (same layouts as
  * tq_generate_params; NULL outputs are skipped). */
-tq_status tq_get_params(const tq_ctx* ctx, float* rot, float* qjl, float* key_c, float* key_t,
+TQ_API tq_status tq_get_params(const tq_ctx* ctx, float* rot, float* qjl, float* key_c, float* key_t,
                         float* val_c, float* val_t);
 
 /*
@@ -128,7 +134,7 @@ tq_status tq_get_params(const tq_ctx* ctx, float* rot, float* qjl, float* key_c,
  * so that four consecutive pairs read chunk-wise hit distinct shared-memory
  * banks.  Coordinates are those of the rotated domain.
  */
-size_t tq_page_bytes(const tq_ctx* ctx, int with_values);
+TQ_API size_t tq_page_bytes(const tq_ctx* ctx, int with_values);
 
 /* Input flag for tq_compress_append: k and v already hold Pi x in fp32 (the
  * rotation folded into the projection that produced them). */
@@ -155,13 +161,13 @@ size_t tq_page_bytes(const tq_ctx* ctx, int with_values);
  * max_pages*128 or a page id outside [0, pool_pages) -> TQ_ERR_CAPACITY and
  * that token is not written.
  */
-tq_status tq_compress_append(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,
+TQ_API tq_status tq_compress_append(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,
                              int flags, int B, int Hkv, int n_new, uint8_t* page_pool,
                              int64_t pool_pages, const int32_t* page_table, int max_pages,
                              int32_t* cold_len, void* stream);
 
 /* Workspace bytes tq_decode_attention needs for these maxima. */
-size_t tq_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max);
+TQ_API size_t tq_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max);
 
 /*
  * One decode step of attention over a hot fp16 window and cold compressed
@@ -182,7 +188,7 @@ size_t tq_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pag
  *             max_pages, W_max), 256-byte aligned; contents are scratch.
  * Supported: Hq % Hkv == 0 with Hq / Hkv in {1, 2, 4, 8}.
  */
-tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+TQ_API tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
                               int Hkv, float scale, const void* k_hot, const void* v_hot,
                               int W_max, const int32_t* hot_len, const uint8_t* page_pool,
                               int64_t pool_pages, const int32_t* page_table, int max_pages,
@@ -190,7 +196,7 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype
                               size_t ws_bytes, void* stream);
 
 /* Workspace bytes tq_score_topk needs. */
-size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k);
+TQ_API size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k);
 
 /*
  * Compressed inner-product search ("Leistung bei der Vektorsuche"): the
@@ -205,17 +211,26 @@ size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k);
  *  workspace device, ws_bytes >= tq_topk_workspace_bytes(ctx, Q, N, k).
  * Supported: 1 <= k <= 32.
  */
-tq_status tq_score_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* db_pages,
+TQ_API tq_status tq_score_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* db_pages,
                         int64_t N, int k, int32_t* out_ids, float* out_scores, void* workspace,
                         size_t ws_bytes, void* stream);
 
+/* Profiling hook: when ev_start / ev_stop (cudaEvent_t, passed as void*) are
+ * set, the next calls of tq_decode_attention, tq_compress_append and
+ * tq_score_topk record ev_start on their stream right before the launch of
+ * their main kernel (the split-K attention, the compress, the scorer) and
+ * ev_stop right after it, so a caller can time that kernel alone.  NULL, NULL
+ * switches it off.  Not thread-safe: set it only while no other thread uses
+ * the context. */
+TQ_API tq_status tq_set_profile_events(tq_ctx* ctx, void* ev_start, void* ev_stop);
+
 /* Read and clear the context's device error word.  Synchronises with the
  * device; call it after the work of interest has completed. */
-tq_status tq_get_error(const tq_ctx* ctx);
+TQ_API tq_status tq_get_error(const tq_ctx* ctx);
 
-const char* tq_status_string(tq_status s);
+TQ_API const char* tq_status_string(tq_status s);
 
-void tq_destroy(tq_ctx* ctx);
+TQ_API void tq_destroy(tq_ctx* ctx);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,154 @@
+"""Parity of tq_decode_attention (CUDA, through the C ABI) with the CPU oracle
+on the same seeded inputs and the same oracle-written cold pages.
+Tolerance: |gpu - oracle| <= 2e-3 + 1e-2 |oracle| element-wise (fp32
+accumulation on the GPU, fp64 in the oracle)."""
+import numpy as np
+import pytest
+
+import compressed_kv_decode_b200 as tq
+from compressed_kv_decode_b200 import workloads as W
+
+from decode_cases import assert_close, build, gpu_out, oracle_out
+
+pytestmark = pytest.mark.gpu
+
+_ctx_cache = {}
+_par_cache = {}
+
+
+def ctx_for(d, seed=0):
+    if (d, seed) not in _ctx_cache:
+        _ctx_cache[(d, seed)] = tq.Context(d, seed)
+    return _ctx_cache[(d, seed)]
+
+
+def params_for(O, d, seed=0):
+    if (d, seed) not in _par_cache:
+        _par_cache[(d, seed)] = O.Params(d, seed=seed)
+    return _par_cache[(d, seed)]
+
+
+def check_case(O, c, d, seed=0, what=""):
+    ctx, P = ctx_for(d, seed), params_for(O, d, seed)
+    got = gpu_out(tq, ctx, c)
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_OK
+    ref = oracle_out(O, P, c)
+    for (b, h), r in ref.items():
+        assert_close(got[b, h * c.G:(h + 1) * c.G], r, what="%s group %s" % (what, (b, h)))
+    return got
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_device_tables_match_oracle(O, d):
+    ctx, P = ctx_for(d), params_for(O, d)
+    t = ctx.params()
+    assert np.array_equal(t["qjl"].astype(np.float64), P.S)
+    assert np.abs(t["rot"].astype(np.float64) - P.pi64).max() <= 1e-6
+    assert np.array_equal(t["key_c"], P.kc.astype(np.float32))
+    assert np.array_equal(t["val_c"], P.vc.astype(np.float32))
+
+
+def test_tiny_workload(O):
+    """One head, d=64, 256 cold tokens of iid N(0,1) (seed 0, K, V, q)."""
+    K, V, q = W.tiny_case()
+    P = params_for(O, 64)
+    c = build(O, P, 1, 1, 1, 64, [256], [0], 0, 2, real_groups=[])
+    nbytes = c.page_bytes
+    kr, vr = O.encode(P, K, True), O.encode(P, V, False)
+    rec = dict(sign=kr["sign"], mag=kr["mag"], qbits=kr["qbits"], n=kr["n"], gamma=kr["gamma"],
+               vcode=vr["vcode"], vn=vr["vn"])
+    t = np.arange(256)
+    O.pack(c.pool.reshape(-1), nbytes, 64, 64, True, c.table[0, 0, t // 128], t % 128, rec)
+    c.q, c.groups = q, [(0, 0)]
+    got = check_case(O, c, 64, what="tiny")
+    # quality context: error against exact softmax attention on the raw K, V
+    s = (K @ q[0, 0]) / 8.0
+    p = np.exp(s - s.max())
+    exact = (p / p.sum()) @ V
+    assert np.abs(got[0, 0] - exact).max() < 0.5
+
+
+def test_tinyllama_workload(O):
+    cfg = W.DECODE["tinyllama"]
+    P = params_for(O, 64)
+    c = build(O, P, cfg["B"], cfg["Hq"], cfg["Hkv"], 64, [cfg["cold"]], [cfg["hot"]], cfg["hot"],
+              cfg["cold"] // 128, q_dtype=cfg["q_dtype"], seeds=cfg["seeds"], n_out=cfg["n_out"],
+              factor=cfg["factor"])
+    check_case(O, c, 64, what="tinyllama")
+
+
+@pytest.mark.parametrize("d,G,qdt", [(64, 1, "float32"), (64, 2, "float16"), (64, 8, "bfloat16"),
+                                     (128, 1, "bfloat16"), (128, 2, "float32"), (128, 4, "bfloat16"),
+                                     (128, 8, "float16"), (64, 4, "float32")])
+def test_ragged_lengths(O, d, G, qdt):
+    """Partial pages and units, empty cold or hot parts, unused page-table
+    tail, NaN in hot slots past hot_len, random pool page order."""
+    P = params_for(O, d)
+    Hkv = 2
+    cold = [0, 65, 300, 1, 128, 257]
+    hot = [17, 0, 40, 16, 3, 0]
+    c = build(O, P, len(cold), G * Hkv, Hkv, d, cold, hot, 48, 4, q_dtype=qdt, n_out=3,
+              factor=6.0, seed=d + G)
+    check_case(O, c, d, what="ragged d=%d G=%d" % (d, G))
+
+
+def test_empty_sequence_gives_zeros(O):
+    P = params_for(O, 128)
+    c = build(O, P, 2, 8, 2, 128, [0, 200], [0, 5], 16, 2)
+    got = check_case(O, c, 128, what="empty")
+    assert np.all(got[0] == 0.0)
+
+
+def test_llama3_32k_sampled_groups(O):
+    """Full Llama-3-8B-shaped decode (B=16, 32/8 heads, d=128, 31744 cold +
+    1024 hot) in the launch configuration the benchmark times; oracle on
+    three sampled (batch, kv head) groups, random records elsewhere."""
+    cfg = W.DECODE["llama3_8b_32k"]
+    P = params_for(O, 128)
+    B = cfg["B"]
+    groups = [(0, 0), (7, 3), (15, 7)]
+    c = build(O, P, B, cfg["Hq"], cfg["Hkv"], 128, [cfg["cold"]] * B, [cfg["hot"]] * B,
+              cfg["hot"], cfg["cold"] // 128, q_dtype=cfg["q_dtype"], seeds=cfg["seeds"],
+              n_out=cfg["n_out"], factor=cfg["factor"], real_groups=groups, nan_hot_tail=False)
+    # random hot windows for the groups without oracle data
+    rng = np.random.default_rng(5)
+    for b in range(B):
+        for h in range(cfg["Hkv"]):
+            if (b, h) not in groups:
+                c.k_hot[b, h] = rng.standard_normal((cfg["hot"], 128)).astype(np.float16)
+                c.v_hot[b, h] = rng.standard_normal((cfg["hot"], 128)).astype(np.float16)
+    got = check_case(O, c, 128, what="llama3 32k")
+    assert np.isfinite(got).all()
+
+
+def test_bad_page_id_is_reported_and_skipped(O):
+    P = params_for(O, 64)
+    c = build(O, P, 2, 4, 1, 64, [200, 200], [4, 4], 8, 2)
+    ctx = ctx_for(64)
+    good = oracle_out(O, P, c)
+    table = c.table.copy()
+    table[1, 0, 1] = 10_000  # beyond the pool
+    got = gpu_out(tq, ctx, c, table=table)
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_ERR_CAPACITY
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_OK  # cleared
+    assert_close(got[0], good[(0, 0)], what="unaffected sequence")
+    assert np.isfinite(got[1]).all()
+
+
+def test_cold_len_beyond_table_is_reported(O):
+    P = params_for(O, 64)
+    c = build(O, P, 1, 2, 1, 64, [100], [0], 0, 1)
+    c.cold_len = np.array([300], np.int32)  # table holds one page
+    ctx = ctx_for(64)
+    got = gpu_out(tq, ctx, c)
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_ERR_CAPACITY
+    assert np.isfinite(got).all()
+
+
+def test_repeat_calls_identical(O):
+    P = params_for(O, 128)
+    c = build(O, P, 2, 8, 2, 128, [333, 129], [9, 30], 32, 3, q_dtype="bfloat16")
+    ctx = ctx_for(128)
+    a = gpu_out(tq, ctx, c)
+    b = gpu_out(tq, ctx, c)
+    assert np.array_equal(a, b)
