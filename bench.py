@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per GPU (default: the workload's 16); smaller values only "
+                         "size profiler captures and are not the benchmark line")
     return ap.parse_args()
 
 
@@ -130,9 +133,9 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # workload on the device
 # ---------------------------------------------------------------------------
-def build_state(torch, tq, W, rank):
+def build_state(torch, tq, W, rank, batch=None):
     cfg = W.DECODE[WORKLOAD]
-    B, Hq, Hkv, d = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"]
+    B, Hq, Hkv, d = batch or cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"]
     cold, hot = cfg["cold"], cfg["hot"]
     dev = torch.device("cuda")
     ctx = tq.Context(d, seed=0)
@@ -248,7 +251,7 @@ def run_ours(args, rank, world, local_rank):
     import compressed_kv_decode_b200 as tq
     from compressed_kv_decode_b200 import workloads as W
     torch.cuda.set_device(local_rank)
-    st = build_state(torch, tq, W, rank)
+    st = build_state(torch, tq, W, rank, args.batch)
     ctx = st["ctx"]
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -265,6 +268,10 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(torch.cuda.current_device()) as clk:
         e0.record(stream)
         for i in range(args.steps):
+            # torch only reports events it recorded itself: record both once,
+            # the library re-records them around the attention kernel
+            ev_k[i][0].record(stream)
+            ev_k[i][1].record(stream)
             tq.tq_set_profile_events(ctx.handle, ev_k[i][0], ev_k[i][1])
             decode(tq, st)
         e1.record(stream)
