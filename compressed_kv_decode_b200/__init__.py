@@ -20,6 +20,7 @@ TQ_ERR_OOM, TQ_ERR_CAPACITY, TQ_ERR_TIMEOUT = 4, 5, 6
 TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
 TQ_INPUT_ROTATED = 1
 TQ_PAGE_TOKENS = 128
+TQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class TQError(RuntimeError):
@@ -62,6 +63,10 @@ def lib():
                                           vp, vp, C.c_int, i32p, u8p, C.c_int64, i32p, C.c_int,
                                           i32p, f32p, vp, C.c_size_t, vp]
         L.tq_decode_attention.restype = C.c_int
+        L.tq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int,
+                                                  C.c_float, vp, vp, C.c_int, i32p, u8p, C.c_int64,
+                                                  i32p, C.c_int, i32p, f32p, vp]
+        L.tq_decode_attention_noalloc.restype = C.c_int
         L.tq_topk_workspace_bytes.argtypes = [vp, C.c_int, C.c_int64, C.c_int]
         L.tq_topk_workspace_bytes.restype = C.c_size_t
         L.tq_score_topk.argtypes = [vp, f32p, C.c_int, u8p, C.c_int64, C.c_int, i32p, f32p, vp,
@@ -192,6 +197,24 @@ def tq_decode_attention(ctx, q, k_hot, v_hot, hot_len, page_pool, page_table, co
         _ptr(hot_len), _ptr(page_pool), pool_pages, _ptr(page_table), max_pages, _ptr(cold_len),
         _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)), "tq_decode_attention")
+
+
+def tq_decode_attention_noalloc(ctx, q, k_hot, v_hot, hot_len, page_pool, page_table, cold_len,
+                                out, Hkv, scale=0.0, stream=None):
+    """tq_decode_attention for callers that may not allocate device memory:
+    no workspace argument; the library's fixed scratch array (at most
+    TQ_NOALLOC_SCRATCH_BYTES of workspace) is used instead.  Make the first
+    call on a device before any stream capture; calls that overlap on the GPU
+    race on the shared scratch."""
+    _require_cuda(q, k_hot, v_hot, hot_len, page_pool, page_table, cold_len, out)
+    B, Hq, _ = q.shape
+    W_max = 0 if k_hot is None else k_hot.shape[2]
+    max_pages = 0 if page_table is None else page_table.shape[-1]
+    pool_pages = 0 if page_pool is None else page_pool.shape[0]
+    _check(lib().tq_decode_attention_noalloc(
+        ctx, _ptr(q), _dtype_code(q), B, Hq, Hkv, float(scale), _ptr(k_hot), _ptr(v_hot), W_max,
+        _ptr(hot_len), _ptr(page_pool), pool_pages, _ptr(page_table), max_pages, _ptr(cold_len),
+        _ptr(out), _stream(stream)), "tq_decode_attention_noalloc")
 
 
 def tq_topk_workspace_bytes(ctx, Q, N, k):

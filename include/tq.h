@@ -195,6 +195,38 @@ TQ_API tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype 
                               const int32_t* cold_len, float* out, void* workspace,
                               size_t ws_bytes, void* stream);
 
+/* Largest decode workspace tq_decode_attention_noalloc can serve (8 MiB). */
+#define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * tq_decode_attention without a caller-provided workspace and without any
+ * device allocation.  The pages on the subject have no counterpart of this
+ * call: it exists for callers that are not allowed to allocate device
+ * memory -- for example a plugin inside an inference runtime that owns the
+ * whole device-memory budget, or a serving loop that must never block on the
+ * allocator -- and therefore cannot provide the workspace buffer.
+ *
+ * Arguments and results are those of tq_decode_attention, minus workspace
+ * and ws_bytes.  The scratch space is one fixed array of
+ * TQ_NOALLOC_SCRATCH_BYTES bytes that the library keeps in device memory on
+ * every GPU that loads it, until the process exits.  A problem whose
+ * workspace (tq_workspace_bytes) exceeds that size is rejected with
+ * TQ_ERR_CAPACITY before any launch.
+ *  - The first call on a device looks up the array's device address (a
+ *    synchronous runtime call, once per device); make that first call before
+ *    any stream capture.  The context's device must be the current device.
+ *  - All calls share the one array and it keeps the last call's contents
+ *    (nothing in it needs to start at zero).  Calls that overlap on the GPU,
+ *    from different streams or threads, race on it: serialise them.
+ */
+TQ_API tq_status tq_decode_attention_noalloc(const tq_ctx* ctx, const void* q, tq_dtype q_dtype,
+                                             int B, int Hq, int Hkv, float scale,
+                                             const void* k_hot, const void* v_hot, int W_max,
+                                             const int32_t* hot_len, const uint8_t* page_pool,
+                                             int64_t pool_pages, const int32_t* page_table,
+                                             int max_pages, const int32_t* cold_len, float* out,
+                                             void* stream);
+
 /* Workspace bytes tq_score_topk needs. */
 TQ_API size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k);
 
