@@ -33,7 +33,7 @@
 namespace tq {
 namespace dec {
 
-constexpr int NW = 8;         // warps per attention CTA
+constexpr int NW = 12;        // warps per attention CTA
 constexpr int COLD_TOK = 64;  // tokens per cold unit (half a page)
 constexpr int HOT_TOK = 16;   // tokens per hot unit
 constexpr float NEG_INF = -__builtin_huge_valf();
@@ -58,7 +58,7 @@ struct Cfg {
   static constexpr int HROW = 2 * D + 16;  // padded hot row: conflict-free ldmatrix
   static constexpr int HOT_B = 2 * HOT_TOK * HROW;
   static constexpr int SLOT = ((COLD_B > HOT_B ? COLD_B : HOT_B) + 127) / 128 * 128;
-  static constexpr int NSLOT = (D == 128) ? 3 : 4;
+  static constexpr int NSLOT = (D == 128) ? 2 : 3;
   static constexpr int PBUF = COLD_TOK * 16;  // fp16 P' tile [64 tokens][8 heads]
   static constexpr int SMEM = NW * (NSLOT * SLOT + PBUF) + NW * NSLOT * 8;
 };
@@ -220,8 +220,37 @@ __device__ __forceinline__ float prescale_for(float mx) {
   return ldexpf(1.0f, 8 - e);
 }
 
+// y[g][r] = sum_k M[r][k] x[g][k] for all rows r of a D x D matrix: one warp
+// per row, each lane a float4 of the row (coalesced), reduced by shuffles;
+// every row's load is independent, so the L2 latency overlaps.
 template <int D, int G>
-__global__ void __launch_bounds__(128) prep_kernel(Params p) {
+__device__ __forceinline__ void matvec_rows(const float* __restrict__ M, const float (*x)[D],
+                                            float (*y)[D]) {
+  constexpr int LANES = D / 4;  // lanes holding one row
+  constexpr int ROWS_PER_PASS = 32 / LANES;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int sub = lane / LANES, l4 = lane % LANES;
+#pragma unroll 4
+  for (int r0 = warp * ROWS_PER_PASS; r0 < D; r0 += nw * ROWS_PER_PASS) {
+    const int r = r0 + sub;
+    const float4 m = __ldg(reinterpret_cast<const float4*>(M + static_cast<size_t>(r) * D) + l4);
+    float acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      acc[g] = m.x * x[g][4 * l4] + m.y * x[g][4 * l4 + 1] + m.z * x[g][4 * l4 + 2] +
+               m.w * x[g][4 * l4 + 3];
+#pragma unroll
+      for (int o = LANES / 2; o > 0; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
+    }
+    if (l4 == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) y[g][r] = acc[g];
+    }
+  }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(256) prep_kernel(Params p) {
   using C = Cfg<D, G>;
   const int BH = p.B * p.Hkv;
   if (blockIdx.x == BH) {
@@ -240,35 +269,9 @@ __global__ void __launch_bounds__(128) prep_kernel(Params p) {
                              static_cast<tq_dtype>(p.q_dtype));
   }
   __syncthreads();
-  for (int i = tid; i < G * D; i += blockDim.x) {
-    const int g = i / D, j = i % D;
-    const float4* row = reinterpret_cast<const float4*>(p.rot + static_cast<size_t>(j) * D);
-    float a = 0.0f;
-#pragma unroll 4
-    for (int k4 = 0; k4 < D / 4; ++k4) {
-      float4 r = row[k4];
-      a = fmaf(r.x, sq[g][4 * k4], a);
-      a = fmaf(r.y, sq[g][4 * k4 + 1], a);
-      a = fmaf(r.z, sq[g][4 * k4 + 2], a);
-      a = fmaf(r.w, sq[g][4 * k4 + 3], a);
-    }
-    sqr[g][j] = a;
-  }
+  matvec_rows<D, G>(p.rot, sq, sqr);  // q_rot = Pi q
   __syncthreads();
-  for (int i = tid; i < G * D; i += blockDim.x) {
-    const int g = i / D, r = i % D;
-    const float4* row = reinterpret_cast<const float4*>(p.qjl + static_cast<size_t>(r) * D);
-    float a = 0.0f;
-#pragma unroll 4
-    for (int k4 = 0; k4 < D / 4; ++k4) {
-      float4 s = row[k4];
-      a = fmaf(s.x, sqr[g][4 * k4], a);
-      a = fmaf(s.y, sqr[g][4 * k4 + 1], a);
-      a = fmaf(s.z, sqr[g][4 * k4 + 2], a);
-      a = fmaf(s.w, sqr[g][4 * k4 + 3], a);
-    }
-    sqs[g][r] = a;
-  }
+  matvec_rows<D, G>(p.qjl, sqr, sqs);  // q_s = S q_rot
   __syncthreads();
   const float w1c = p.sl * p.kc0, w2c = p.sl * 128.0f * (p.kc1 - p.kc0), w3c = p.sl * p.alpha;
   for (int i = tid; i < G * D; i += blockDim.x) {
@@ -767,12 +770,14 @@ __global__ void __launch_bounds__(D) combine_kernel(Params p) {
   const int* sched = p.w.sched;
   const int* soff = sched + 4 + p.S + 1;
   const int j = threadIdx.x;
-  __shared__ float so[D];
-  for (int g = 0; g < G; ++g) {
-    float M[2], L[2], O[2];
-    for (int dom = 0; dom < 2; ++dom) {
-      const int sg = 2 * bh + dom;
-      const int a = soff[sg], e = soff[sg + 1];
+  __shared__ float so[G][D];
+  float M[2][G], L[2][G], O[2][G];
+#pragma unroll
+  for (int dom = 0; dom < 2; ++dom) {
+    const int sg = 2 * bh + dom;
+    const int a = soff[sg], e = soff[sg + 1];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
       float mx = -__builtin_huge_valf();
       for (int s = a; s < e; ++s) {
         const float* rec = p.w.part + static_cast<size_t>(s) * G * (D + 2);
@@ -790,26 +795,33 @@ __global__ void __launch_bounds__(D) combine_kernel(Params p) {
           }
         }
       }
-      M[dom] = mx;
-      L[dom] = l;
-      O[dom] = o;
+      M[dom][g] = mx;
+      L[dom][g] = l;
+      O[dom][g] = o;
     }
-    // cold accumulator is in the rotated domain: o_cold = Pi^T o_rot
-    __syncthreads();
-    so[j] = O[0];
-    __syncthreads();
-    float oc = 0.0f;
-    if (L[0] > 0.0f) {
+  }
+  // cold accumulators are in the rotated domain: o_cold = Pi^T o_rot, all heads at once
+#pragma unroll
+  for (int g = 0; g < G; ++g) so[g][j] = O[0][g];
+  __syncthreads();
+  float oc[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) oc[g] = 0.0f;
 #pragma unroll 8
-      for (int i = 0; i < D; ++i) oc = fmaf(p.rot[static_cast<size_t>(i) * D + j], so[i], oc);
-    }
-    const float Mx = fmaxf(M[0], M[1]);
+  for (int i = 0; i < D; ++i) {
+    const float r = __ldg(p.rot + static_cast<size_t>(i) * D + j);
+#pragma unroll
+    for (int g = 0; g < G; ++g) oc[g] = fmaf(r, so[g][i], oc[g]);
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float Mx = fmaxf(M[0][g], M[1][g]);
     float res = 0.0f;
     if (Mx != -__builtin_huge_valf()) {
-      const float fc = (L[0] > 0.0f) ? exp2f(M[0] - Mx) : 0.0f;
-      const float fh = (L[1] > 0.0f) ? exp2f(M[1] - Mx) : 0.0f;
-      const float den = L[0] * fc + L[1] * fh;
-      res = (den > 0.0f) ? (oc * fc + O[1] * fh) / den : 0.0f;
+      const float fc = (L[0][g] > 0.0f) ? exp2f(M[0][g] - Mx) : 0.0f;
+      const float fh = (L[1][g] > 0.0f) ? exp2f(M[1][g] - Mx) : 0.0f;
+      const float den = L[0][g] * fc + L[1][g] * fh;
+      res = (den > 0.0f) ? (oc[g] * fc + O[1][g] * fh) / den : 0.0f;
     }
     p.out[(static_cast<size_t>(b) * p.Hq + kvh * G + g) * D + j] = res;
   }
@@ -866,7 +878,7 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
       return TQ_ERR_CUDA;
     set = true;
   }
-  prep_kernel<D, G><<<p.B * p.Hkv + 1, 128, 0, st>>>(p);
+  prep_kernel<D, G><<<p.B * p.Hkv + 1, 256, 0, st>>>(p);
   if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
   attn_kernel<D, G><<<grid, NW * 32, C::SMEM, st>>>(p);
   if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
