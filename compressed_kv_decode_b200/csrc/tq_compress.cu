@@ -422,6 +422,9 @@ int run(const tq_ctx* ctx, Params& p, cudaStream_t st) {
 int launch_compress(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype, int flags,
                     int B, int Hkv, int n_new, uint8_t* pool, int64_t pool_pages,
                     const int32_t* page_table, int max_pages, int32_t* cold_len, void* stream) {
+  if (!(flags & TQ_INPUT_ROTATED))  // raw 16-bit input: rotation and sketch on tcgen05
+    return launch_compress_tc(ctx, k, v, dtype == TQ_BF16, B, Hkv, n_new, pool, pool_pages,
+                              page_table, max_pages, cold_len, stream);
   const int d = ctx->cfg.head_dim;
   const PageLayout L = page_layout(d, ctx->cfg.qjl_dim, v != nullptr);
   cmp::Params p{};

@@ -1,0 +1,522 @@
+// Compress and append on the 5th-generation tensor cores (tcgen05), for raw
+// fp16 / bf16 inputs ("TurboQuant" summary, de.news.hada.io topic 27867,
+// section "Funktionsweise von TurboQuant": random rotation, per-coordinate
+// quantiser, 1-bit QJL sketch of the residual).
+//
+// Persistent CTAs of 256 threads, one 128-token page tile at a time:
+//   TMA     input tile [128 rows x d] (3-D tensor map over [B*Hkv, n_new, d],
+//           128-byte swizzle; rows outside the sequence arrive as zeros),
+//           double-buffered (keys, values)
+//   MMA     one thread issues tcgen05.mma: x_rot = X (Pi_hi + Pi_lo)^T into
+//           TMEM (M = 128, N = d, K = d, f32 accumulate); later p = R S^T
+//   epilogue all 8 warps: thread = (row, half of the columns); x_rot from TMEM
+//           by tcgen05.ld; norm, codes, residual, sign bits and packing stay
+//           in the thread; the residual is written to shared memory in the
+//           MMA's operand layout for the sketch; records go straight to the page.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "tq_device.cuh"
+#include "tq_internal.h"
+#include "tq_tc.cuh"
+
+namespace tq {
+namespace tc {
+
+bool encode_map_3d(CUtensorMap* map, bool bf16, const void* base, const uint64_t dims[3],
+                   const uint64_t strides_bytes[2], const uint32_t box[3]) {
+  using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return false;
+    fn = reinterpret_cast<EncodeFn>(p);
+  }
+  const cuuint64_t gdim[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t gstr[2] = {strides_bytes[0], strides_bytes[1]};
+  const cuuint32_t bdim[3] = {box[0], box[1], box[2]};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+            const_cast<void*>(base), gdim, gstr, bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+namespace ctc {
+
+constexpr int ROWS = 128;
+constexpr int NTHREADS = 256;
+
+template <int D>
+struct Cfg {
+  static constexpr int HALF = D / 2;          // columns per epilogue thread
+  static constexpr int OPB = D * 128;         // bytes of one 64-column block of a D-row operand
+  static constexpr int OP = (D / 64) * OPB;   // D x D operand (Pi hi, Pi lo, S)
+  static constexpr int XB = ROWS * 128;       // one 64-column block of a 128-row tile
+  static constexpr int XT = (D / 64) * XB;    // 128-row tile
+  static constexpr int OFF_PH = 0;
+  static constexpr int OFF_PL = OFF_PH + OP;
+  static constexpr int OFF_S = OFF_PL + OP;
+  static constexpr int OFF_X0 = OFF_S + OP;
+  static constexpr int OFF_X1 = OFF_X0 + XT;
+  static constexpr int OFF_R = OFF_X1 + XT;
+  static constexpr int OFF_NK = OFF_R + XT;        // float[2][128] key norm^2 halves
+  static constexpr int OFF_NV = OFF_NK + 1024;     // float[2][128] value norm^2 halves
+  static constexpr int OFF_G = OFF_NV + 1024;      // float[2][128] residual norm^2 halves
+  static constexpr int OFF_BAR = OFF_G + 1024;     // 5 mbarriers
+  static constexpr int OFF_TMEM = OFF_BAR + 64;
+  static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t TMEM_COLS = (3 * D <= 256) ? 256 : 512;
+  static constexpr int COL_RK = 0, COL_SK = D, COL_RV = 2 * D;
+};
+
+struct Params {
+  int B, Hkv, n_new;
+  bool has_v;
+  uint8_t* pool;
+  long long pool_pages, page_bytes;
+  int off_kc, off_qs, off_vc, off_kn, off_kg, off_vn;
+  const int32_t* page_table;
+  int max_pages;
+  const int32_t* cold_len;
+  const uint16_t* pi_hi;
+  const uint16_t* pi_lo;
+  const uint16_t* s_h;
+  float kc0, kc1, kt0;
+  float vt[7];
+  int* err;
+  int tiles_per_bh;
+};
+
+struct Tile {
+  int bh, lpage, s_lo, s_hi, page, row0;
+};
+
+// the next tile of this CTA with active slots, starting at index t (uniform)
+__device__ __forceinline__ bool next_tile(const Params& p, int& t, Tile& out) {
+  const int total = p.B * p.Hkv * p.tiles_per_bh;
+  for (; t < total; t += gridDim.x) {
+    const int bh = t / p.tiles_per_bh, ti = t % p.tiles_per_bh;
+    const int cl = p.cold_len[bh / p.Hkv];
+    const int lpage = cl / ROWS + ti;
+    const int s_lo = max(cl, lpage * ROWS) - lpage * ROWS;
+    const int s_hi = min(cl + p.n_new, (lpage + 1) * ROWS) - lpage * ROWS;
+    if (s_lo >= s_hi) continue;
+    out.bh = bh;
+    out.lpage = lpage;
+    out.s_lo = s_lo;
+    out.s_hi = s_hi;
+    out.row0 = lpage * ROWS - cl;
+    out.page = (lpage < p.max_pages) ? p.page_table[static_cast<size_t>(bh) * p.max_pages + lpage] : -1;
+    return true;
+  }
+  return false;
+}
+
+template <int D>
+__device__ __forceinline__ void issue_tile_load(const CUtensorMap* map, uint32_t dst, uint32_t bar,
+                                                const Tile& tl) {
+  using C = Cfg<D>;
+  mbar_arrive_expect_tx(bar, C::XT);
+#pragma unroll
+  for (int kb = 0; kb < D / 64; ++kb) tc::tma_load_3d(dst + kb * C::XB, map, kb * 64, tl.row0, tl.bh, bar);
+}
+
+// x_rot = X (Pi_hi + Pi_lo)^T into TMEM columns [col, col + D)
+template <int D, bool BF>
+__device__ __forceinline__ void issue_rotation(uint32_t tmem, int col, uint32_t x, uint32_t ph,
+                                               uint32_t pl) {
+  using C = Cfg<D>;
+  constexpr uint32_t idesc = tc::idesc_f16(ROWS, D, BF);
+#pragma unroll
+  for (int s = 0; s < D / 16; ++s) {
+    const int kb = s >> 2, w = (s & 3) * 32;
+    const uint64_t a = tc::sdesc_sw128(x + kb * C::XB + w);
+    tc::mma_f16(tmem + col, a, tc::sdesc_sw128(ph + kb * C::OPB + w), idesc, s > 0);
+    tc::mma_f16(tmem + col, a, tc::sdesc_sw128(pl + kb * C::OPB + w), idesc, true);
+  }
+}
+
+// sum of squares of this thread's half row of a 16-bit input tile
+template <int D, bool BF>
+__device__ __forceinline__ float half_row_sumsq(const uint8_t* x, int row, int h) {
+  using C = Cfg<D>;
+  float ss = 0.0f;
+#pragma unroll
+  for (int c = 0; c < C::HALF / 8; ++c) {
+    const int k = h * C::HALF + 8 * c;
+    const uint4 v = *reinterpret_cast<const uint4*>(x + tc::sw128_offset(row, k, ROWS));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float a, b;
+      if constexpr (BF) {
+        a = __uint_as_float(w[i] << 16);
+        b = __uint_as_float(w[i] & 0xFFFF0000u);
+      } else {
+        const __half2 hh = *reinterpret_cast<const __half2*>(&w[i]);
+        a = __low2float(hh);
+        b = __high2float(hh);
+      }
+      ss = fmaf(a, a, fmaf(b, b, ss));
+    }
+  }
+  return ss;
+}
+
+template <int D>
+__device__ __forceinline__ void tmem_load_half(uint32_t taddr, float (&x)[D / 2]) {
+#pragma unroll
+  for (int c = 0; c < D / 2; c += 32) {
+    uint32_t r[32];
+    tc::ld32(taddr + c, r);
+    tc::wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[c + i] = __uint_as_float(r[i]);
+  }
+}
+
+template <int D, bool BF>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    compress_tc_kernel(const __grid_constant__ CUtensorMap mapK,
+                       const __grid_constant__ CUtensorMap mapV, Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled operand atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = 32 * (warp & 3) + lane;  // TMEM lane quarter of this warp
+  const int h = warp >> 2;                 // column half
+  const uint32_t s0 = smem_u32(smem);
+  const uint32_t bar_full0 = s0 + C::OFF_BAR, bar_full1 = bar_full0 + 8;
+  const uint32_t bar_rk = bar_full0 + 16, bar_sk = bar_full0 + 24, bar_rv = bar_full0 + 32;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+  float* nk = reinterpret_cast<float*>(smem + C::OFF_NK);
+  float* nvp = reinterpret_cast<float*>(smem + C::OFF_NV);
+  float* gp = reinterpret_cast<float*>(smem + C::OFF_G);
+
+  // resident operands in the K-major SW128 layout: Pi hi, Pi lo (rows = output
+  // coordinate), S (rows = sketch index); 16-byte chunks
+  for (int i = tid; i < D * (D / 8); i += NTHREADS) {
+    const int r = i / (D / 8), k = (i % (D / 8)) * 8;
+    const uint32_t off = tc::sw128_offset(r, k, D);
+    *reinterpret_cast<uint4*>(smem + C::OFF_PH + off) =
+        *reinterpret_cast<const uint4*>(p.pi_hi + static_cast<size_t>(r) * D + k);
+    *reinterpret_cast<uint4*>(smem + C::OFF_PL + off) =
+        *reinterpret_cast<const uint4*>(p.pi_lo + static_cast<size_t>(r) * D + k);
+    *reinterpret_cast<uint4*>(smem + C::OFF_S + off) =
+        *reinterpret_cast<const uint4*>(p.s_h + static_cast<size_t>(r) * D + k);
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 5; ++i) mbar_init(bar_full0 + 8 * i, 1);
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  fence_proxy_async_smem();  // operand tables visible to the tensor cores
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+
+  int t = blockIdx.x;
+  Tile cur;
+  bool have = next_tile(p, t, cur);
+  if (have && tid == 0) {
+    issue_tile_load<D>(&mapK, s0 + C::OFF_X0, bar_full0, cur);
+    if (p.has_v) issue_tile_load<D>(&mapV, s0 + C::OFF_X1, bar_full1, cur);
+  }
+  bool failed = false;
+  for (uint32_t it = 0; have; ++it) {
+    const uint32_t par = it & 1u;
+    int tn = t + gridDim.x;
+    Tile nxt;
+    const bool have_next = next_tile(p, tn, nxt);
+    const bool page_ok = cur.page >= 0 && cur.page < p.pool_pages;
+    const bool active = row >= cur.s_lo && row < cur.s_hi;
+
+    // ---- keys: rotation ------------------------------------------------
+    if (!mbar_wait_bounded(bar_full0, par)) { failed = true; break; }
+    if (tid == 0) {
+      tc::fence_after_sync();
+      issue_rotation<D, BF>(tmem, C::COL_RK, s0 + C::OFF_X0, s0 + C::OFF_PH, s0 + C::OFF_PL);
+      tc::commit(bar_rk);
+    }
+    nk[h * ROWS + row] = half_row_sumsq<D, BF>(smem + C::OFF_X0, row, h);
+    __syncthreads();
+    if (!mbar_wait_bounded(bar_rk, par)) { failed = true; break; }
+    tc::fence_after_sync();
+    if (tid == 0 && have_next) {
+      fence_proxy_async_smem();
+      issue_tile_load<D>(&mapK, s0 + C::OFF_X0, bar_full0, nxt);
+    }
+    float x[C::HALF];
+    tmem_load_half<D>(t_lane + C::COL_RK + h * C::HALF, x);
+    const float nn = sqrtf(nk[row] + nk[ROWS + row]);
+    const __half nh = __float2half_rn(nn);
+    const float n = __half2float(nh);
+    const float T0 = __fmul_rn(n, p.kt0);
+    const float inv = n > 0.0f ? 1.0f / n : 0.0f;
+    uint32_t kw[C::HALF / 16];
+#pragma unroll
+    for (int w = 0; w < C::HALF / 16; ++w) kw[w] = 0u;
+    float g2 = 0.0f;
+#pragma unroll
+    for (int c8 = 0; c8 < C::HALF / 8; ++c8) {
+      uint32_t rh[4];
+#pragma unroll
+      for (int e2 = 0; e2 < 4; ++e2) {
+        float rr[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = 8 * c8 + 2 * e2 + e;  // column within the half
+          const float v = x[i];
+          const uint32_t sg = (n > 0.0f && v < 0.0f) ? 1u : 0u;
+          const uint32_t mg = (n > 0.0f && fabsf(v) >= T0) ? 1u : 0u;
+          const float cp = mg ? p.kc1 : p.kc0;
+          const float r = (n > 0.0f) ? fmaf(v, inv, (v < 0.0f) ? cp : -cp) : 0.0f;
+          rr[e] = r;
+          g2 = fmaf(r, r, g2);
+          const int j = h * C::HALF + i;  // coordinate
+          const int jj = j & 15, hh = jj >> 3, ii = (jj & 7) >> 1, ee = jj & 1;
+          const int sbit = 16 * hh + 15 - 4 * ii - ee;
+          kw[i >> 4] |= (sg << sbit) | (mg << (sbit - 2));
+        }
+        const __half2 pr = __floats2half2_rn(rr[0], rr[1]);
+        rh[e2] = *reinterpret_cast<const uint32_t*>(&pr);
+      }
+      *reinterpret_cast<uint4*>(smem + C::OFF_R + tc::sw128_offset(row, h * C::HALF + 8 * c8, ROWS)) =
+          make_uint4(rh[0], rh[1], rh[2], rh[3]);
+    }
+    gp[h * ROWS + row] = g2;
+    fence_proxy_async_smem();  // residual tile visible to the tensor cores
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- keys: QJL sketch, values: rotation --------------------------------
+    if (tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t idesc = tc::idesc_f16(ROWS, D, false);
+#pragma unroll
+      for (int s = 0; s < D / 16; ++s) {
+        const int kb = s >> 2, w = (s & 3) * 32;
+        tc::mma_f16(tmem + C::COL_SK, tc::sdesc_sw128(s0 + C::OFF_R + kb * C::XB + w),
+                    tc::sdesc_sw128(s0 + C::OFF_S + kb * C::OPB + w), idesc, s > 0);
+      }
+      tc::commit(bar_sk);
+    }
+    if (p.has_v) {
+      if (!mbar_wait_bounded(bar_full1, par)) { failed = true; break; }
+      if (tid == 0) {
+        tc::fence_after_sync();
+        issue_rotation<D, BF>(tmem, C::COL_RV, s0 + C::OFF_X1, s0 + C::OFF_PH, s0 + C::OFF_PL);
+        tc::commit(bar_rv);
+      }
+      nvp[h * ROWS + row] = half_row_sumsq<D, BF>(smem + C::OFF_X1, row, h);
+    }
+    uint8_t* pg = p.pool + static_cast<size_t>(page_ok ? cur.page : 0) * p.page_bytes;
+    const bool wr = page_ok && active;
+    if (wr) {
+      if constexpr (C::HALF / 16 == 4)
+        *reinterpret_cast<uint4*>(pg + p.off_kc + row * (D / 4) + h * (C::HALF / 4)) =
+            make_uint4(kw[0], kw[1], kw[2], kw[3]);
+      else
+        *reinterpret_cast<uint2*>(pg + p.off_kc + row * (D / 4) + h * (C::HALF / 4)) =
+            make_uint2(kw[0], kw[1]);
+    }
+    if (!mbar_wait_bounded(bar_sk, par)) { failed = true; break; }
+    tc::fence_after_sync();
+    tmem_load_half<D>(t_lane + C::COL_SK + h * C::HALF, x);
+    {
+      uint32_t qw[C::HALF / 32];
+#pragma unroll
+      for (int w = 0; w < C::HALF / 32; ++w) qw[w] = 0u;
+#pragma unroll
+      for (int i = 0; i < C::HALF; ++i) {
+        const int within = i & 31;  // sketch index inside its 32-bit word
+        const int bit = 16 * (within >> 4) + 15 - (within & 15);
+        if (n > 0.0f && x[i] < 0.0f) qw[i >> 5] |= 1u << bit;
+      }
+      if (wr) {
+        if constexpr (C::HALF / 32 == 2)
+          *reinterpret_cast<uint2*>(pg + p.off_qs + row * (D / 8) + h * (C::HALF / 8)) =
+              make_uint2(qw[0], qw[1]);
+        else
+          *reinterpret_cast<uint32_t*>(pg + p.off_qs + row * (D / 8) + h * (C::HALF / 8)) = qw[0];
+      }
+    }
+    __syncthreads();  // residual norm halves and value norm halves complete
+    if (wr && h == 0) {
+      reinterpret_cast<__half*>(pg + p.off_kn)[row] = nh;
+      reinterpret_cast<__half*>(pg + p.off_kg)[row] = __float2half_rn(sqrtf(gp[row] + gp[ROWS + row]));
+    }
+    // ---- values ------------------------------------------------------------
+    if (p.has_v) {
+      if (!mbar_wait_bounded(bar_rv, par)) { failed = true; break; }
+      tc::fence_after_sync();
+      if (tid == 0 && have_next) {
+        fence_proxy_async_smem();
+        issue_tile_load<D>(&mapV, s0 + C::OFF_X1, bar_full1, nxt);
+      }
+      tmem_load_half<D>(t_lane + C::COL_RV + h * C::HALF, x);
+      const __half vh = __float2half_rn(sqrtf(nvp[row] + nvp[ROWS + row]));
+      const float vn = __half2float(vh);
+      float T[7];
+#pragma unroll
+      for (int k = 0; k < 7; ++k) T[k] = __fmul_rn(vn, p.vt[k]);
+      // codes of this row, then the pair partner's (adjacent lane) for the bytes
+      uint32_t cw[C::HALF / 8];  // 8 nibbles per word, column i in nibble i % 8
+#pragma unroll
+      for (int w = 0; w < C::HALF / 8; ++w) cw[w] = 0u;
+#pragma unroll
+      for (int i = 0; i < C::HALF; ++i) {
+        uint32_t mg = 0u;
+#pragma unroll
+        for (int k = 0; k < 7; ++k) mg += (fabsf(x[i]) >= T[k]) ? 1u : 0u;
+        const uint32_t code = (vn > 0.0f) ? (((x[i] < 0.0f) ? 8u : 0u) | mg) : 0u;
+        cw[i >> 3] |= code << (4 * (i & 7));
+      }
+      const bool even = (row & 1) == 0;
+      const bool act_e = active, act_o = __shfl_xor_sync(0xffffffffu, active ? 1 : 0, 1) != 0;
+      uint32_t ow[C::HALF / 8];
+#pragma unroll
+      for (int w = 0; w < C::HALF / 8; ++w) ow[w] = __shfl_xor_sync(0xffffffffu, cw[w], 1);
+      if (page_ok && even && (act_e || act_o)) {
+        const int pr = row >> 1;
+        constexpr int CH = D / 8;  // chunk bytes
+        uint8_t* blk = pg + p.off_vc + pr * D;
+#pragma unroll
+        for (int c = 0; c < C::HALF / CH; ++c) {
+          const int chunk = h * (C::HALF / CH) + c;
+          uint8_t* dst = blk + ((chunk + 2 * (pr & 3)) & 7) * CH;
+          uint32_t bytes[CH / 4];
+#pragma unroll
+          for (int b4 = 0; b4 < CH / 4; ++b4) {
+            uint32_t v = 0u;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              const int i = c * CH + 4 * b4 + b;  // column within the half
+              const uint32_t lo = (cw[i >> 3] >> (4 * (i & 7))) & 0xFu;
+              const uint32_t hi = (ow[i >> 3] >> (4 * (i & 7))) & 0xFu;
+              v |= (lo | (hi << 4)) << (8 * b);
+            }
+            bytes[b4] = v;
+          }
+          if (!(act_e && act_o)) {  // one slot of the pair belongs to an earlier or later call
+            const uint32_t keep = act_e ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+#pragma unroll
+            for (int b4 = 0; b4 < CH / 4; ++b4) {
+              const uint32_t old = reinterpret_cast<const uint32_t*>(dst)[b4];
+              bytes[b4] = (old & keep) | (bytes[b4] & ~keep);
+            }
+          }
+          if constexpr (CH == 16)
+            *reinterpret_cast<uint4*>(dst) = make_uint4(bytes[0], bytes[1], bytes[2], bytes[3]);
+          else
+            *reinterpret_cast<uint2*>(dst) = make_uint2(bytes[0], bytes[1]);
+        }
+      }
+      if (wr && h == 0) reinterpret_cast<__half*>(pg + p.off_vn)[row] = vh;
+    }
+    if (threadIdx.x == 0 && !page_ok) report(p.err, TQ_ERR_CAPACITY);
+    tc::fence_before_sync();
+    __syncthreads();  // TMEM columns and the residual tile are reused by the next tile
+    tc::fence_after_sync();
+    cur = nxt;
+    t = tn;
+    have = have_next;
+  }
+  if (failed && threadIdx.x == 0) report(p.err, TQ_ERR_TIMEOUT);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace ctc
+
+__global__ void advance_cold_len(int32_t* cold_len, int B, int n_new) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) cold_len[b] += n_new;
+}
+
+int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf16, int B, int Hkv,
+                       int n_new, uint8_t* pool, int64_t pool_pages, const int32_t* page_table,
+                       int max_pages, int32_t* cold_len, void* stream) {
+  const int d = ctx->cfg.head_dim;
+  const PageLayout L = page_layout(d, ctx->cfg.qjl_dim, v != nullptr);
+  ctc::Params p{};
+  p.B = B;
+  p.Hkv = Hkv;
+  p.n_new = n_new;
+  p.has_v = v != nullptr;
+  p.pool = pool;
+  p.pool_pages = pool_pages;
+  p.page_bytes = static_cast<long long>(L.bytes);
+  p.off_kc = static_cast<int>(L.kc);
+  p.off_qs = static_cast<int>(L.qs);
+  p.off_vc = static_cast<int>(L.vc);
+  p.off_kn = static_cast<int>(L.kn);
+  p.off_kg = static_cast<int>(L.kg);
+  p.off_vn = static_cast<int>(L.vn);
+  p.page_table = page_table;
+  p.max_pages = max_pages;
+  p.cold_len = cold_len;
+  p.pi_hi = bf16 ? ctx->dev.rot_bf_hi : ctx->dev.rot_h_hi;
+  p.pi_lo = bf16 ? ctx->dev.rot_bf_lo : ctx->dev.rot_h_lo;
+  p.s_h = ctx->dev.qjl_h;
+  p.kc0 = ctx->cb.key_c[0];
+  p.kc1 = ctx->cb.key_c[1];
+  p.kt0 = ctx->cb.key_t[0];
+  for (int i = 0; i < 7; ++i) p.vt[i] = ctx->cb.val_t[i];
+  p.err = ctx->dev.err;
+  p.tiles_per_bh = (n_new + ctc::ROWS - 1) / ctc::ROWS + 1;
+  CUtensorMap mk, mv;
+  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_new),
+                            static_cast<uint64_t>(B) * Hkv};
+  const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(n_new) * d * 2};
+  const uint32_t box[3] = {64, ctc::ROWS, 1};
+  if (!tc::encode_map_3d(&mk, bf16, k, dims, strides, box)) return TQ_ERR_CUDA;
+  if (v) {
+    if (!tc::encode_map_3d(&mv, bf16, v, dims, strides, box)) return TQ_ERR_CUDA;
+  } else {
+    mv = mk;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long tiles = static_cast<long long>(B) * Hkv * p.tiles_per_bh;
+  const int grid = static_cast<int>(tiles < ctx->num_sms ? tiles : ctx->num_sms);
+  auto go = [&](auto kern, int smem) -> int {
+    static bool set[4] = {};
+    const int slot = (d == 128 ? 2 : 0) + (bf16 ? 1 : 0);
+    if (!set[slot]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return TQ_ERR_CUDA;
+      set[slot] = true;
+    }
+    if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
+    kern<<<grid, ctc::NTHREADS, smem, st>>>(mk, mv, p);
+    if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
+    advance_cold_len<<<(B + 127) / 128, 128, 0, st>>>(cold_len, B, n_new);
+    return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  };
+  if (d == 128)
+    return bf16 ? go(ctc::compress_tc_kernel<128, true>, ctc::Cfg<128>::SMEM)
+                : go(ctc::compress_tc_kernel<128, false>, ctc::Cfg<128>::SMEM);
+  return bf16 ? go(ctc::compress_tc_kernel<64, true>, ctc::Cfg<64>::SMEM)
+              : go(ctc::compress_tc_kernel<64, false>, ctc::Cfg<64>::SMEM);
+}
+
+}  // namespace tq

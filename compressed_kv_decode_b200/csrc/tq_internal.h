@@ -76,6 +76,10 @@ int launch_compress(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dt
                     int B, int Hkv, int n_new, uint8_t* pool, int64_t pool_pages,
                     const int32_t* page_table, int max_pages, int32_t* cold_len, void* stream);
 
+int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf16, int B, int Hkv,
+                       int n_new, uint8_t* pool, int64_t pool_pages, const int32_t* page_table,
+                       int max_pages, int32_t* cold_len, void* stream);
+
 int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* db, int64_t N,
                 int k, int32_t* out_ids, float* out_scores, void* ws, size_t ws_bytes,
                 void* stream);

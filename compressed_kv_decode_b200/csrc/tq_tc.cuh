@@ -1,0 +1,119 @@
+// Blackwell (sm_100a) tensor-core helpers: tensor memory (TMEM) allocation,
+// tcgen05.mma issue and completion, TMEM loads, shared-memory matrix
+// descriptors for the canonical K-major 128-byte-swizzled layout, and tiled
+// TMA loads (no multicast).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace tq {
+namespace tc {
+
+// ---- TMEM ---------------------------------------------------------------
+// allocate `ncols` columns (power of two >= 32); the warp must be converged;
+// the TMEM address is written to shared memory at `dst`
+__device__ __forceinline__ void tmem_alloc(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// ---- MMA ----------------------------------------------------------------
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (f16 or bf16 inputs,
+// f32 accumulate); issued by a single thread
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+
+// arrive on an mbarrier once every MMA issued so far by this thread is done
+__device__ __forceinline__ void commit(uint32_t mbar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+      : "memory");
+}
+
+// instruction descriptor, kind::f16: f32 accumulator, both operands K-major
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// shared-memory descriptor: K-major, 128-byte swizzle, atoms of 8 rows x 128 B
+// stacked every 1024 B; `addr` is the shared-state-space byte address of the
+// first element (atoms 1024-byte aligned; +32 B steps move along K)
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr & 0x3FFFFu) >> 4);       // start address
+  d |= static_cast<uint64_t>(1u) << 16;                     // leading byte offset (unused)
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;             // stride byte offset
+  d |= static_cast<uint64_t>(1u) << 46;                     // descriptor version
+  d |= static_cast<uint64_t>(2u) << 61;                     // 128-byte swizzle
+  return d;
+}
+
+// byte offset of element (row, k) of a K-major SW128 tile whose rows hold 64
+// 16-bit elements per 128-byte block; blocks of `rows` rows follow each other
+__host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int k, int rows) {
+  const int kb = k >> 6, kk = k & 63;
+  return static_cast<uint32_t>(kb * rows * 128 + row * 128 + ((((kk >> 3) ^ (row & 7)) & 7) << 4) +
+                               ((kk & 7) << 1));
+}
+
+// ---- TMEM -> registers -----------------------------------------------------
+// 32 consecutive 32-bit columns of this thread's lane
+__device__ __forceinline__ void ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---- TMA ----------------------------------------------------------------
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(mbar)
+      : "memory");
+}
+
+// host: encode a tiled 3-D tensor map (dims innermost first) for 16-bit data
+// with 128-byte swizzle; returns false on failure
+bool encode_map_3d(CUtensorMap* map, bool bf16, const void* base, const uint64_t dims[3],
+                   const uint64_t strides_bytes[2], const uint32_t box[3]);
+
+}  // namespace tc
+}  // namespace tq
