@@ -223,17 +223,26 @@ __device__ __forceinline__ float prescale_for(float mx) {
 // y[g][r] = sum_k M[r][k] x[g][k] for all rows r of a D x D matrix: one warp
 // per row, each lane a float4 of the row (coalesced), reduced by shuffles;
 // every row's load is independent, so the L2 latency overlaps.
+constexpr int PREP_WARPS = 8;
+
 template <int D, int G>
 __device__ __forceinline__ void matvec_rows(const float* __restrict__ M, const float (*x)[D],
                                             float (*y)[D]) {
   constexpr int LANES = D / 4;  // lanes holding one row
   constexpr int ROWS_PER_PASS = 32 / LANES;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  constexpr int PASSES = D / (PREP_WARPS * ROWS_PER_PASS);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / LANES, l4 = lane % LANES;
-#pragma unroll 4
-  for (int r0 = warp * ROWS_PER_PASS; r0 < D; r0 += nw * ROWS_PER_PASS) {
-    const int r = r0 + sub;
-    const float4 m = __ldg(reinterpret_cast<const float4*>(M + static_cast<size_t>(r) * D) + l4);
+  float4 mrow[PASSES];  // every row this lane needs, requested at once
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps) {
+    const int r = (ps * PREP_WARPS + warp) * ROWS_PER_PASS + sub;
+    mrow[ps] = __ldg(reinterpret_cast<const float4*>(M + static_cast<size_t>(r) * D) + l4);
+  }
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps) {
+    const int r = (ps * PREP_WARPS + warp) * ROWS_PER_PASS + sub;
+    const float4 m = mrow[ps];
     float acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -764,12 +773,15 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
 // ---------------------------------------------------------------------------
 // 3. combine
 // ---------------------------------------------------------------------------
+constexpr int MAX_COMBINE_SLOTS = 256;  // partial records staged in shared memory per pass
+
 template <int D, int G>
 __global__ void __launch_bounds__(D) combine_kernel(Params p) {
   const int bh = blockIdx.x, b = bh / p.Hkv, kvh = bh % p.Hkv;
   const int* sched = p.w.sched;
   const int* soff = sched + 4 + p.S + 1;
   const int j = threadIdx.x;
+  __shared__ float sm_m[MAX_COMBINE_SLOTS][G], sm_l[MAX_COMBINE_SLOTS][G];
   __shared__ float so[G][D];
   float M[2][G], L[2][G], O[2][G];
 #pragma unroll
@@ -778,38 +790,62 @@ __global__ void __launch_bounds__(D) combine_kernel(Params p) {
     const int a = soff[sg], e = soff[sg + 1];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float mx = -__builtin_huge_valf();
-      for (int s = a; s < e; ++s) {
-        const float* rec = p.w.part + static_cast<size_t>(s) * G * (D + 2);
-        if (rec[G + g] > 0.0f) mx = fmaxf(mx, rec[g]);
+      M[dom][g] = -__builtin_huge_valf();
+      L[dom][g] = 0.0f;
+      O[dom][g] = 0.0f;
+    }
+    for (int base = a; base < e; base += MAX_COMBINE_SLOTS) {
+      const int n = min(MAX_COMBINE_SLOTS, e - base);
+      __syncthreads();
+      // (m, l) of every slot and head, loaded with independent requests
+      for (int i = j; i < n * G; i += blockDim.x) {
+        const int s = i / G, g = i % G;
+        const float* rec = p.w.part + static_cast<size_t>(base + s) * G * (D + 2);
+        sm_m[s][g] = rec[g];
+        sm_l[s][g] = rec[G + g];
       }
-      float l = 0.0f, o = 0.0f;
-      if (mx != -__builtin_huge_valf()) {
-        for (int s = a; s < e; ++s) {
-          const float* rec = p.w.part + static_cast<size_t>(s) * G * (D + 2);
-          const float lw = rec[G + g];
-          if (lw > 0.0f) {
-            const float f = exp2f(rec[g] - mx);
-            l += lw * f;
-            o += rec[2 * G + g * D + j] * f;
-          }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float mx = M[dom][g];
+        for (int s = 0; s < n; ++s)
+          if (sm_l[s][g] > 0.0f) mx = fmaxf(mx, sm_m[s][g]);
+        const float resc = (M[dom][g] == -__builtin_huge_valf() || mx == -__builtin_huge_valf())
+                               ? 0.0f : exp2f(M[dom][g] - mx);
+        float l = L[dom][g] * resc, o = O[dom][g] * resc;
+#pragma unroll 4
+        for (int s = 0; s < n; ++s) {
+          const float lw = sm_l[s][g];
+          const float f = (lw > 0.0f) ? exp2f(sm_m[s][g] - mx) : 0.0f;
+          l += lw * f;
+          o += p.w.part[static_cast<size_t>(base + s) * G * (D + 2) + 2 * G + g * D + j] * f;
         }
+        M[dom][g] = mx;
+        L[dom][g] = l;
+        O[dom][g] = o;
       }
-      M[dom][g] = mx;
-      L[dom][g] = l;
-      O[dom][g] = o;
     }
   }
-  // cold accumulators are in the rotated domain: o_cold = Pi^T o_rot, all heads at once
+  // cold accumulators are in the rotated domain: o_cold = Pi^T o_rot, all heads at once;
+  // Pi is staged in shared memory with every load of the thread in flight at once
+  extern __shared__ float spi[];  // [D][D]
 #pragma unroll
   for (int g = 0; g < G; ++g) so[g][j] = O[0][g];
+  {
+    constexpr int PER = D * D / 4 / D;  // float4 per thread
+    float4 v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) v[i] = __ldg(reinterpret_cast<const float4*>(p.rot) + i * D + j);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) reinterpret_cast<float4*>(spi)[i * D + j] = v[i];
+  }
   __syncthreads();
   float oc[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) oc[g] = 0.0f;
-#pragma unroll 8
+#pragma unroll 16
   for (int i = 0; i < D; ++i) {
-    const float r = __ldg(p.rot + static_cast<size_t>(i) * D + j);
+    const float r = spi[i * D + j];
 #pragma unroll
     for (int g = 0; g < G; ++g) oc[g] = fmaf(r, so[g][i], oc[g]);
   }
@@ -878,11 +914,19 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
       return TQ_ERR_CUDA;
     set = true;
   }
-  prep_kernel<D, G><<<p.B * p.Hkv + 1, 256, 0, st>>>(p);
+  prep_kernel<D, G><<<p.B * p.Hkv + 1, PREP_WARPS * 32, 0, st>>>(p);
   if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
   attn_kernel<D, G><<<grid, NW * 32, C::SMEM, st>>>(p);
   if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
-  combine_kernel<D, G><<<p.B * p.Hkv, D, 0, st>>>(p);
+  static bool comb_set[2][9] = {};
+  bool& cset = comb_set[D == 128][G];
+  if (!cset) {
+    if (cudaFuncSetAttribute(combine_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             D * D * 4) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    cset = true;
+  }
+  combine_kernel<D, G><<<p.B * p.Hkv, D, D * D * 4, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 

@@ -74,6 +74,24 @@ __device__ __forceinline__ int qjl_index(int s, int kk) {
   return 32 * (P >> 4) + (P & 15) + 16 * e;
 }
 
+// y[r] = sum_k M[r][k] x[k]: one warp per row, float4 per lane, shuffle reduce
+template <int D>
+__device__ __forceinline__ void warp_matvec(const float* __restrict__ M, const float* x, float* y) {
+  constexpr int LANES = D / 4, RPP = 32 / LANES, NW = 4, PASSES = D / (NW * RPP);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sub = lane / LANES, l4 = lane % LANES;
+  float4 m[PASSES];
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps)
+    m[ps] = __ldg(reinterpret_cast<const float4*>(M + static_cast<size_t>((ps * NW + warp) * RPP + sub) * D) + l4);
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps) {
+    float a = m[ps].x * x[4 * l4] + m[ps].y * x[4 * l4 + 1] + m[ps].z * x[4 * l4 + 2] + m[ps].w * x[4 * l4 + 3];
+#pragma unroll
+    for (int o = LANES / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (l4 == 0) y[(ps * NW + warp) * RPP + sub] = a;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) qprep_kernel(Params p) {
   using C = Cfg<D>;
@@ -85,17 +103,9 @@ __global__ void __launch_bounds__(128) qprep_kernel(Params p) {
   if (tid == 0) smax = 0u;
   for (int j = tid; j < D; j += blockDim.x) sq[j] = p.queries[static_cast<size_t>(q) * D + j];
   __syncthreads();
-  for (int j = tid; j < D; j += blockDim.x) {
-    float a = 0.0f;
-    for (int k = 0; k < D; ++k) a = fmaf(p.rot[static_cast<size_t>(j) * D + k], sq[k], a);
-    sr[j] = a;
-  }
+  warp_matvec<D>(p.rot, sq, sr);
   __syncthreads();
-  for (int i = tid; i < D; i += blockDim.x) {
-    float a = 0.0f;
-    for (int j = 0; j < D; ++j) a = fmaf(p.qjl[static_cast<size_t>(i) * D + j], sr[j], a);
-    ss[i] = a;
-  }
+  warp_matvec<D>(p.qjl, sr, ss);
   __syncthreads();
   const float w1 = p.kc0, w2 = 128.0f * (p.kc1 - p.kc0), w3 = p.alpha;
   for (int j = tid; j < D; j += blockDim.x) {
@@ -193,10 +203,32 @@ __global__ void __launch_bounds__(NWARP * 32, 1) score_kernel(Params p) {
       dq[t] = (qq < p.Q) ? p.desc[qq] : 0.0f;
     }
     const long long pg0 = p.pages * sl / p.n_slices, pg1 = p.pages * (sl + 1) / p.n_slices;
-    for (long long grp = pg0 * 4 + warp; grp < pg1 * 4; grp += NWARP) {
+    // the 32 records of step grp; the next step's words are requested before
+    // the current step's contraction so the L2 latency overlaps it
+    uint32_t kw_n[2][2][D / 64], qw_n[2][2];
+    uint16_t gg_n[2][2], nn_n[2][2];
+    auto fetch = [&](long long grp) {
       const long long page = grp >> 2;
       const int slot0 = static_cast<int>(grp & 3) * 32;
       const uint8_t* pgp = p.db + page * p.page_bytes;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int slot = slot0 + 16 * mt + g + 8 * r;
+#pragma unroll
+          for (int w = 0; w < D / 64; ++w)
+            kw_n[mt][r][w] = __ldg(reinterpret_cast<const uint32_t*>(pgp + p.off_kc + slot * (D / 4)) + c * (D / 64) + w);
+          qw_n[mt][r] = __ldg(reinterpret_cast<const uint32_t*>(pgp + p.off_qs + slot * (D / 8)) + qword);
+          gg_n[mt][r] = __ldg(reinterpret_cast<const uint16_t*>(pgp + p.off_kg) + slot);
+          nn_n[mt][r] = __ldg(reinterpret_cast<const uint16_t*>(pgp + p.off_kn) + slot);
+        }
+      }
+    };
+    if (pg0 * 4 + warp < pg1 * 4) fetch(pg0 * 4 + warp);
+    for (long long grp = pg0 * 4 + warp; grp < pg1 * 4; grp += NWARP) {
+      const long long page = grp >> 2;
+      const int slot0 = static_cast<int>(grp & 3) * 32;
       float acc[2][C::NTQ][4];
       uint32_t kw[2][2][D / 64], qw[2][2];
       uint32_t gg[2][2];
@@ -206,18 +238,17 @@ __global__ void __launch_bounds__(NWARP * 32, 1) score_kernel(Params p) {
       for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          const int slot = slot0 + 16 * mt + g + 8 * r;
-          ids[mt][r] = static_cast<int>(page * TQ_PAGE_TOKENS + slot);
+          ids[mt][r] = static_cast<int>(page * TQ_PAGE_TOKENS + slot0 + 16 * mt + g + 8 * r);
 #pragma unroll
-          for (int w = 0; w < D / 64; ++w)
-            kw[mt][r][w] = __ldg(reinterpret_cast<const uint32_t*>(pgp + p.off_kc + slot * (D / 4)) + c * (D / 64) + w);
-          qw[mt][r] = __ldg(reinterpret_cast<const uint32_t*>(pgp + p.off_qs + slot * (D / 8)) + qword);
-          gg[mt][r] = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(pgp + p.off_kg) + slot)) * 0x10001u;
-          nn[mt][r] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const uint16_t*>(pgp + p.off_kn) + slot)));
+          for (int w = 0; w < D / 64; ++w) kw[mt][r][w] = kw_n[mt][r][w];
+          qw[mt][r] = qw_n[mt][r];
+          gg[mt][r] = static_cast<uint32_t>(gg_n[mt][r]) * 0x10001u;
+          nn[mt][r] = __half2float(__ushort_as_half(nn_n[mt][r]));
         }
 #pragma unroll
         for (int t = 0; t < C::NTQ; ++t) acc[mt][t][0] = acc[mt][t][1] = acc[mt][t][2] = acc[mt][t][3] = 0.0f;
       }
+      if (grp + NWARP < pg1 * 4) fetch(grp + NWARP);
       // key planes: k-steps 0..KS-1 (sign) and KS..2KS-1 (magnitude)
 #pragma unroll
       for (int s = 0; s < C::KS; ++s) {
