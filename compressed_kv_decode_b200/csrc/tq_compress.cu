@@ -325,18 +325,14 @@ __global__ void __launch_bounds__(NWARP * 32, 1) compress_kernel(Params p) {
           const uint32_t partner = __shfl_xor_sync(0xffffffffu, packed, 4);
           if ((g & 1) == 0) {
             const int j = 8 * t + 2 * c;
-            const int chunk = D / 8;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
               const int slot = (half ? r1 : r0);
               const int pair = slot >> 1;
               const uint32_t mine = (packed >> (8 * half)) & 0xFFu;   // codes (j, j+1), even slot
               const uint32_t other = (partner >> (8 * half)) & 0xFFu; // codes (j, j+1), odd slot
-              const uint32_t b0 = (mine & 0xFu) | ((other & 0xFu) << 4);
-              const uint32_t b1 = (mine >> 4) | ((other >> 4) << 4);
-              const int pos = ((j / chunk + 2 * (pair & 3)) & 7) * chunk + (j % chunk);
-              *reinterpret_cast<uint16_t*>(stg + C::STG_VC + pair * D + pos) =
-                  static_cast<uint16_t>(b0 | (b1 << 8));
+              stg[C::STG_VC + vc_pos<D>(j, pair)] = static_cast<uint8_t>((mine & 0xFu) | ((other & 0xFu) << 4));
+              stg[C::STG_VC + vc_pos<D>(j + 1, pair)] = static_cast<uint8_t>((mine >> 4) | ((other >> 4) << 4));
             }
           }
         }
@@ -367,27 +363,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) compress_kernel(Params p) {
         if (p.v)
           reinterpret_cast<uint16_t*>(pg + p.off_vn)[i] = reinterpret_cast<const uint16_t*>(stg + C::STG_VN)[i];
       }
-      if (p.v) {
-        // whole pairs with both slots active: 16-byte copies; a pair with one
-        // active slot keeps the other slot's nibble already in the page
-        const int p_lo = (s_lo + 1) >> 1, p_hi = s_hi >> 1;
-        for (int i = tid + p_lo * (D / 16); i < p_hi * (D / 16); i += blockDim.x)
-          reinterpret_cast<uint4*>(pg + p.off_vc)[i] = reinterpret_cast<const uint4*>(stg + C::STG_VC)[i];
-        if (s_lo & 1) {  // pair s_lo/2: only the odd slot (high nibble) is new
-          const int pr = s_lo >> 1;
-          for (int i = tid; i < D; i += blockDim.x) {
-            uint8_t* dst = pg + p.off_vc + pr * D + i;
-            *dst = static_cast<uint8_t>((*dst & 0x0Fu) | (stg[C::STG_VC + pr * D + i] & 0xF0u));
-          }
-        }
-        if ((s_hi & 1) && !((s_lo & 1) && (s_lo >> 1) == (s_hi >> 1))) {
-          const int pr = s_hi >> 1;  // only the even slot (low nibble) is new
-          for (int i = tid; i < D; i += blockDim.x) {
-            uint8_t* dst = pg + p.off_vc + pr * D + i;
-            *dst = static_cast<uint8_t>((*dst & 0xF0u) | (stg[C::STG_VC + pr * D + i] & 0x0Fu));
-          }
-        }
-      }
+      if (p.v) vc_copy_out<D>(stg + C::STG_VC, pg + p.off_vc, s_lo, s_hi, tid, blockDim.x);
     }
     __syncthreads();  // staging reused by the next tile
   }

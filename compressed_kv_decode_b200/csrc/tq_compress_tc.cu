@@ -75,7 +75,8 @@ struct Cfg {
   static constexpr int OFF_NK = OFF_R + XT;        // float[2][128] key norm^2 halves
   static constexpr int OFF_NV = OFF_NK + 1024;     // float[2][128] value norm^2 halves
   static constexpr int OFF_G = OFF_NV + 1024;      // float[2][128] residual norm^2 halves
-  static constexpr int OFF_BAR = OFF_G + 1024;     // 5 mbarriers
+  static constexpr int OFF_VS = OFF_G + 1024;      // value-code section staging (64 D bytes)
+  static constexpr int OFF_BAR = OFF_VS + D * 64;  // 5 mbarriers
   static constexpr int OFF_TMEM = OFF_BAR + 64;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = (3 * D <= 256) ? 256 : 512;
@@ -391,45 +392,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         cw[i >> 3] |= code << (4 * (i & 7));
       }
       const bool even = (row & 1) == 0;
-      const bool act_e = active, act_o = __shfl_xor_sync(0xffffffffu, active ? 1 : 0, 1) != 0;
       uint32_t ow[C::HALF / 8];
 #pragma unroll
       for (int w = 0; w < C::HALF / 8; ++w) ow[w] = __shfl_xor_sync(0xffffffffu, cw[w], 1);
-      if (page_ok && even && (act_e || act_o)) {
+      // even rows place the byte pairs (own code low, partner's high) in the
+      // staged section; the whole section then goes out with 16-byte copies
+      uint8_t* vs = smem + C::OFF_VS;
+      if (even) {
         const int pr = row >> 1;
-        constexpr int CH = D / 8;  // chunk bytes
-        uint8_t* blk = pg + p.off_vc + pr * D;
 #pragma unroll
-        for (int c = 0; c < C::HALF / CH; ++c) {
-          const int chunk = h * (C::HALF / CH) + c;
-          uint8_t* dst = blk + ((chunk + 2 * (pr & 3)) & 7) * CH;
-          uint32_t bytes[CH / 4];
-#pragma unroll
-          for (int b4 = 0; b4 < CH / 4; ++b4) {
-            uint32_t v = 0u;
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-              const int i = c * CH + 4 * b4 + b;  // column within the half
-              const uint32_t lo = (cw[i >> 3] >> (4 * (i & 7))) & 0xFu;
-              const uint32_t hi = (ow[i >> 3] >> (4 * (i & 7))) & 0xFu;
-              v |= (lo | (hi << 4)) << (8 * b);
-            }
-            bytes[b4] = v;
-          }
-          if (!(act_e && act_o)) {  // one slot of the pair belongs to an earlier or later call
-            const uint32_t keep = act_e ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
-#pragma unroll
-            for (int b4 = 0; b4 < CH / 4; ++b4) {
-              const uint32_t old = reinterpret_cast<const uint32_t*>(dst)[b4];
-              bytes[b4] = (old & keep) | (bytes[b4] & ~keep);
-            }
-          }
-          if constexpr (CH == 16)
-            *reinterpret_cast<uint4*>(dst) = make_uint4(bytes[0], bytes[1], bytes[2], bytes[3]);
-          else
-            *reinterpret_cast<uint2*>(dst) = make_uint2(bytes[0], bytes[1]);
+        for (int i = 0; i < C::HALF; ++i) {
+          const uint32_t lo = (cw[i >> 3] >> (4 * (i & 7))) & 0xFu;
+          const uint32_t hi = (ow[i >> 3] >> (4 * (i & 7))) & 0xFu;
+          vs[vc_pos<D>(h * C::HALF + i, pr)] = static_cast<uint8_t>(lo | (hi << 4));
         }
       }
+      __syncthreads();
+      if (page_ok) vc_copy_out<D>(vs, pg + p.off_vc, cur.s_lo, cur.s_hi, tid, NTHREADS);
       if (wr && h == 0) reinterpret_cast<__half*>(pg + p.off_vn)[row] = vh;
     }
     if (threadIdx.x == 0 && !page_ok) report(p.err, TQ_ERR_CAPACITY);

@@ -527,12 +527,15 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
       if (hA >= 4) aA = a1A;
       if (hB >= 4) aB = a1B;
     }
+    // the output only needs rescaling when some head's running max moved
+    if (__any_sync(0xffffffffu, aA != 1.0f || aB != 1.0f)) {
 #pragma unroll
-    for (int i = 0; i < C::KS; ++i) {
-      oacc[i][0] *= aA;
-      oacc[i][1] *= aB;
-      oacc[i][2] *= aA;
-      oacc[i][3] *= aB;
+      for (int i = 0; i < C::KS; ++i) {
+        oacc[i][0] *= aA;
+        oacc[i][1] *= aB;
+        oacc[i][2] *= aA;
+        oacc[i][3] *= aB;
+      }
     }
   };
 
@@ -565,15 +568,12 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int h = 2 * c + (e & 1);
-        int coord;
-        if (dom == 0)
-          coord = g * (D / 8) + 4 * (i >> 1) + 2 * (i & 1) + (e >> 1);
-        else
-          coord = 16 * i + g + 8 * (e >> 1);
+        const int coord = 16 * i + g + 8 * (e >> 1);
         if (h < G) o[h * D + coord] = oacc[i][e];
       }
     }
     (void)bh;
+    (void)dom;
   };
 
   const uint32_t pb_addr = smem_u32(pbuf);
@@ -612,9 +612,12 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         const uint32_t qw1 = *reinterpret_cast<const uint32_t*>(sb + C::OFF_QS + t1 * (D / 8) + 4 * qword);
         const uint32_t gg0 = static_cast<uint32_t>(kg[t0]) * 0x10001u;
         const uint32_t gg1 = static_cast<uint32_t>(kg[t1]) * 0x10001u;
-        float acc[C::NT][4];
+        // three independent accumulation chains (sign, magnitude, QJL planes)
+        float acc[C::NT][4], acm[C::NT][4], acq[C::NT][4];
 #pragma unroll
-        for (int nt = 0; nt < C::NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+        for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[nt][e] = acm[nt][e] = acq[nt][e] = 0.0f;
 #pragma unroll
         for (int s = 0; s < C::KS; ++s) {
           const int w = s >> 2, sh = 4 * (s & 3);
@@ -624,25 +627,24 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
           const uint32_t a2 = (x0b & 0x80008000u) | 0x3C003C00u, a3 = (x1b & 0x80008000u) | 0x3C003C00u;
           const uint32_t m0 = x0a & 0xA000A000u, m1 = x1a & 0xA000A000u;
           const uint32_t m2 = x0b & 0xA000A000u, m3 = x1b & 0xA000A000u;
+          const int sq = qsb + 2 * s;
+          const uint32_t q0 = ((qw0 << sq) & 0x80008000u) | gg0;
+          const uint32_t q1 = ((qw1 << sq) & 0x80008000u) | gg1;
+          const uint32_t q2 = ((qw0 << (sq + 1)) & 0x80008000u) | gg0;
+          const uint32_t q3 = ((qw1 << (sq + 1)) & 0x80008000u) | gg1;
 #pragma unroll
           for (int nt = 0; nt < C::NT; ++nt) {
             mma_f16(acc[nt], a0, a1, a2, a3, bfr[(s * C::NT + nt) * 2], bfr[(s * C::NT + nt) * 2 + 1]);
-            mma_f16(acc[nt], m0, m1, m2, m3, bfr[((C::KS + s) * C::NT + nt) * 2],
+            mma_f16(acm[nt], m0, m1, m2, m3, bfr[((C::KS + s) * C::NT + nt) * 2],
                     bfr[((C::KS + s) * C::NT + nt) * 2 + 1]);
+            mma_f16(acq[nt], q0, q1, q2, q3, bfr[((2 * C::KS + s) * C::NT + nt) * 2],
+                    bfr[((2 * C::KS + s) * C::NT + nt) * 2 + 1]);
           }
         }
 #pragma unroll
-        for (int s = 0; s < C::KS; ++s) {
-          const int sh = qsb + 2 * s;
-          const uint32_t a0 = ((qw0 << sh) & 0x80008000u) | gg0;
-          const uint32_t a1 = ((qw1 << sh) & 0x80008000u) | gg1;
-          const uint32_t a2 = ((qw0 << (sh + 1)) & 0x80008000u) | gg0;
-          const uint32_t a3 = ((qw1 << (sh + 1)) & 0x80008000u) | gg1;
+        for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
-          for (int nt = 0; nt < C::NT; ++nt)
-            mma_f16(acc[nt], a0, a1, a2, a3, bfr[((2 * C::KS + s) * C::NT + nt) * 2],
-                    bfr[((2 * C::KS + s) * C::NT + nt) * 2 + 1]);
-        }
+          for (int e = 0; e < 4; ++e) acc[nt][e] += acm[nt][e] + acq[nt][e];
         const float n0 = __half2float(kn[t0]), n1 = __half2float(kn[t1]);
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt) {
@@ -670,34 +672,25 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         }
       }
       __syncwarp();
+      // value codes: the lane's word for coordinate tile i of a 16-token
+      // block dequantises to its A fragment (coordinates x tokens)
       const uint8_t* vc = sb + C::OFF_VC;
-      const int chunk = (g + 2 * c) & 7;
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
         uint32_t bp0, bp1;
         ldsm_x2_t(pb_addr + (16 * mt + (lane & 15)) * 16, bp0, bp1);
-        const int pa = 8 * mt + c, pb2 = pa + 4;
-        const uint8_t* ra = vc + pa * D + chunk * (D / 8);
-        const uint8_t* rb = vc + pb2 * D + chunk * (D / 8);
-        uint32_t xa[C::WV], xb[C::WV];
-        if constexpr (C::WV == 4) {
-          const uint4 va = *reinterpret_cast<const uint4*>(ra);
-          const uint4 vb = *reinterpret_cast<const uint4*>(rb);
-          xa[0] = va.x; xa[1] = va.y; xa[2] = va.z; xa[3] = va.w;
-          xb[0] = vb.x; xb[1] = vb.y; xb[2] = vb.z; xb[3] = vb.w;
-        } else {
-          const uint2 va = *reinterpret_cast<const uint2*>(ra);
-          const uint2 vb = *reinterpret_cast<const uint2*>(rb);
-          xa[0] = va.x; xa[1] = va.y;
-          xb[0] = vb.x; xb[1] = vb.y;
+        const uint8_t* vb = vc + mt * (8 * D) + lane * 16;
+        uint32_t xw[C::KS];
+#pragma unroll
+        for (int q4 = 0; q4 < C::KS / 4; ++q4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(vb + 512 * q4);
+          xw[4 * q4] = v.x; xw[4 * q4 + 1] = v.y; xw[4 * q4 + 2] = v.z; xw[4 * q4 + 3] = v.w;
         }
 #pragma unroll
-        for (int wq = 0; wq < C::WV; ++wq) {
-          uint32_t ha[4], hb[4];
-          dequant_values(xa[wq], tl0, tl1, th0, th1, ha);
-          dequant_values(xb[wq], tl0, tl1, th0, th1, hb);
-          mma_f16(oacc[2 * wq], ha[0], ha[1], hb[0], hb[1], bp0, bp1);
-          mma_f16(oacc[2 * wq + 1], ha[2], ha[3], hb[2], hb[3], bp0, bp1);
+        for (int i = 0; i < C::KS; ++i) {
+          uint32_t h[4];
+          dequant_values(xw[i], tl0, tl1, th0, th1, h);
+          mma_f16(oacc[i], h[0], h[1], h[2], h[3], bp0, bp1);
         }
       }
     } else {

@@ -149,3 +149,47 @@ __device__ __forceinline__ float load_as_float(const void* p, size_t i, tq_dtype
 }
 
 }  // namespace tq
+
+namespace tq {
+
+// Value-code section of a page: token pair p (slots 2p, 2p+1) of coordinate j
+// is one byte (even slot in the low nibble).  Blocks of 16 tokens (kb) by
+// tiles of 16 coordinates (i): the 32-bit word of lane 4g + c at
+// kb*8D + (i/4)*512 + (4g + c)*16 + (i%4)*4 holds coordinates (g, g+8) x
+// token pairs (c, c+4) of the block -- one m16n8k16 A fragment (rows =
+// coordinates, k = tokens) after dequantisation.
+template <int D>
+__host__ __device__ __forceinline__ int vc_pos(int j, int p) {
+  const int kb = p >> 3, q = p & 7, c = q & 3, th = q >> 2;
+  const int i = j >> 4, g = j & 7, jh = (j >> 3) & 1;
+  return kb * (8 * D) + (i >> 2) * 512 + (4 * g + c) * 16 + (i & 3) * 4 + jh + 2 * th;
+}
+
+// Copy a value-code section staged in shared memory (same layout as the
+// page) to the page, for the active token slots [s_lo, s_hi): 16-byte copies
+// when the whole page is written, else byte copies that keep the nibble of a
+// pair's slot outside the range.
+template <int D>
+__device__ __forceinline__ void vc_copy_out(const uint8_t* stg, uint8_t* dst, int s_lo, int s_hi,
+                                            int tid, int nthr) {
+  if (s_lo == 0 && s_hi == 128) {
+    for (int i = tid; i < D * 4; i += nthr)
+      reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(stg)[i];
+    return;
+  }
+  const int p_lo = s_lo >> 1, p_hi = (s_hi + 1) >> 1, np = p_hi - p_lo;
+  for (int i = tid; i < D * np; i += nthr) {
+    const int j = i / np, p = p_lo + i % np;
+    const int off = vc_pos<D>(j, p);
+    uint8_t b = stg[off];
+    const bool ev = 2 * p >= s_lo && 2 * p < s_hi;
+    const bool od = 2 * p + 1 >= s_lo && 2 * p + 1 < s_hi;
+    if (!(ev && od)) {
+      const uint8_t keep = ev ? 0xF0 : 0x0F;
+      b = static_cast<uint8_t>((dst[off] & keep) | (b & ~keep));
+    }
+    dst[off] = b;
+  }
+}
+
+}  // namespace tq

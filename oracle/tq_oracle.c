@@ -364,7 +364,7 @@ OR_API int or_lloyd_max(int d, int bits, int max_iter, double* c /* L */, double
 /* Sections in order, each starting on a 16-byte boundary:                  */
 /*   KC key codes    128 x d/4 bytes   (2-bit codes: sign and magnitude)    */
 /*   QS QJL signs    128 x m/8 bytes                                        */
-/*   VC value codes  64 pairs x d bytes (4-bit codes; values pages only)    */
+/*   VC value codes  64 x d bytes       (4-bit codes; values pages only)    */
 /*   KN key norm     128 x fp16                                             */
 /*   KG residual norm 128 x fp16                                            */
 /*   VN value norm   128 x fp16        (values pages only)                  */
@@ -372,11 +372,15 @@ OR_API int or_lloyd_max(int d, int bits, int max_iter, double* c /* L */, double
 /* coordinates j = 16w + 8h + r (h in {0,1}, r = 2i + e < 8): sign bit at   */
 /* 16h + 15 - 4i - e, magnitude bit at 16h + 13 - 4i - e.                   */
 /* QJL word w (w < m/32) holds sketch index i = 32w + 16h + r (r < 16) at   */
-/* bit 16h + 15 - r.  Value codes: token pair p = slot/2; the byte of       */
-/* coordinate j holds code(2p, j) in its low nibble and code(2p+1, j) in    */
-/* its high nibble; a code is sign<<3 | magnitude index (0..7).  The pair's */
-/* d-byte block is cut in 8 chunks of d/8 bytes; chunk g (coordinates       */
-/* g*d/8 ...) is stored at chunk position (g + 2*(p mod 4)) mod 8.          */
+/* bit 16h + 15 - r.  Value codes (a code is sign<<3 | magnitude index,      */
+/* 0..7): one byte holds two tokens of one coordinate, the even token in the */
+/* low nibble.  Tokens are grouped in blocks of 16 (kb = slot/16) and        */
+/* coordinates in tiles of 16 (i = j/16); inside a (block, tile) pair, with  */
+/* g = j mod 8, jh = (j mod 16)/8, pair q = (slot mod 16)/2, c = q mod 4,    */
+/* th = q/4, the byte sits at                                               */
+/*   kb*8d + (i/4)*512 + (4g + c)*16 + (i mod 4)*4 + jh + 2*th              */
+/* so that the 32-bit word at (4g + c)*16 + (i mod 4)*4 holds, in its four   */
+/* bytes, coordinates (g, g+8) x token pairs (c, c+4) of the block.          */
 /* ------------------------------------------------------------------------ */
 #define PAGE_TOKENS 128
 
@@ -429,10 +433,13 @@ static int qs_bit(int i) { /* position inside word i/32 */
   return 16 * h + 15 - r;
 }
 
-/* offset of coordinate j's byte inside the value block of token pair p */
-static int vc_pos(int d, int p, int j) {
-  int chunk = d / 8;
-  return ((j / chunk + 2 * (p % 4)) % 8) * chunk + j % chunk;
+/* offset, inside the value-code section, of the byte holding token pair p
+ * (slots 2p, 2p+1) of coordinate j */
+static size_t vc_pos(int d, int p, int j) {
+  int kb = p / 8, q = p % 8, c = q % 4, th = q / 4;
+  int i = j / 16, g = j % 8, jh = (j % 16) / 8;
+  return (size_t)kb * 8 * d + (size_t)(i / 4) * 512 + (size_t)(4 * g + c) * 16 +
+         (size_t)(i % 4) * 4 + (size_t)(jh + 2 * th);
 }
 
 /* write one key record into token slot `slot` of page `pg` */
@@ -479,7 +486,7 @@ OR_API void or_unpack_key(const uint8_t* pg, int d, int m, int with_values, int 
 OR_API void or_pack_value(uint8_t* pg, int d, int m, int slot, const int32_t* code, double n) {
   or_layout L = layout_of(d, m, 1);
   int p = slot / 2;
-  uint8_t* vc = pg + L.vc + (size_t)p * d;
+  uint8_t* vc = pg + L.vc;
   int hi = slot & 1;
   for (int j = 0; j < d; ++j) {
     uint8_t* bp = vc + vc_pos(d, p, j);
@@ -492,7 +499,7 @@ OR_API void or_pack_value(uint8_t* pg, int d, int m, int slot, const int32_t* co
 OR_API void or_unpack_value(const uint8_t* pg, int d, int m, int slot, int32_t* code, double* n) {
   or_layout L = layout_of(d, m, 1);
   int p = slot / 2;
-  const uint8_t* vc = pg + L.vc + (size_t)p * d;
+  const uint8_t* vc = pg + L.vc;
   for (int j = 0; j < d; ++j) {
     uint8_t b = vc[vc_pos(d, p, j)];
     code[j] = (slot & 1) ? (b >> 4) : (b & 0xF);

@@ -43,7 +43,7 @@ def test_golden_format_examples(O):
     d = m = 64
     nbytes, offs = O.page_layout(d, m, True)
     pool = np.zeros(nbytes, np.uint8)
-    rec = _empty_records(4, d, m)
+    rec = _empty_records(6, d, m)
     for j in map(int, g["key"]["sign"].split(",")):
         rec["sign"][0, j] = 1
     for j in map(int, g["key"]["mag"].split(",")):
@@ -53,65 +53,37 @@ def test_golden_format_examples(O):
     cj = int(g["value"]["coord"])
     rec["vcode"][2, cj] = int(g["value"]["slot2"], 16)
     rec["vcode"][3, cj] = int(g["value"]["slot3"], 16)
-    O.pack(pool, nbytes, d, m, True, [0, 0, 0, 0], [0, 1, 2, 3], rec)
+    cj2 = int(g["value2"]["coord"])
+    rec["vcode"][4, cj2] = int(g["value2"]["slot26"], 16)
+    rec["vcode"][5, cj2] = int(g["value2"]["slot27"], 16)
+    O.pack(pool, nbytes, d, m, True, [0] * 6, [0, 1, 2, 3, 26, 27], rec)
     word = lambda off: int.from_bytes(pool[off:off + 4].tobytes(), "little")
     assert word(offs["kc"]) == int(g["key"]["word0"], 16)
     assert word(offs["qs"]) == int(g["qjl"]["word0"], 16)
-    assert pool[offs["vc"] + 1 * d + int(g["value"]["offset"])] == int(g["value"]["byte"], 16)
-    assert np.count_nonzero(pool[offs["vc"]:offs["kn"]]) == 1
-
-
-@pytest.mark.parametrize("d,m", D_M)
-def test_every_bit_position_by_inverse_map(O, d, m):
-    """Set one field at a time and find the single bit it lands on; derive the
-    expected position from the bit's side: bit b of key word w belongs to
-    half h=b//16, nibble slot 3-i=(b%16)//4, nibble bit k=b%4: sign plane if
-    k>=2 (e=3-k) else magnitude plane (e=1-k); coordinate 16w+8h+2i+e."""
-    nbytes, offs = O.page_layout(d, m, True)
-    slot = 5
-    for w in range(d // 16):
-        for b in range(32):
-            h, nb, k = b // 16, (b % 16) // 4, b % 4
-            i = 3 - nb
-            plane = "sign" if k >= 2 else "mag"
-            e = 3 - k if k >= 2 else 1 - k
-            j = 16 * w + 8 * h + 2 * i + e
-            pool = np.zeros(nbytes, np.uint8)
-            rec = _empty_records(1, d, m)
-            rec[plane][0, j] = 1
-            O.pack(pool, nbytes, d, m, True, [0], [slot], rec)
-            sec = pool[offs["kc"]:offs["qs"]].view(np.uint32).reshape(128, d // 16)
-            assert np.count_nonzero(sec) == 1 and sec[slot, w] == (1 << b)
-    for w in range(m // 32):
-        for b in range(32):
-            i = 32 * w + 16 * (b // 16) + (15 - b % 16)
-            pool = np.zeros(nbytes, np.uint8)
-            rec = _empty_records(1, d, m)
-            rec["qbits"][0, i] = 1
-            O.pack(pool, nbytes, d, m, True, [0], [slot], rec)
-            sec = pool[offs["qs"]:offs["vc"]].view(np.uint32).reshape(128, m // 32)
-            assert np.count_nonzero(sec) == 1 and sec[slot, w] == (1 << b)
+    assert pool[offs["vc"] + int(g["value"]["offset"])] == int(g["value"]["byte"], 16)
+    assert pool[offs["vc"] + int(g["value2"]["offset"])] == int(g["value2"]["byte"], 16)
+    assert np.count_nonzero(pool[offs["vc"]:offs["kn"]]) == 2
 
 
 @pytest.mark.parametrize("d,m", D_M)
 def test_value_byte_positions(O, d, m):
-    """Each (pair, coordinate) lands on its own byte; chunks rotate by two
-    positions per pair within a group of four pairs."""
+    """Every (token pair, coordinate) lands on its own byte of the value
+    section (a bijection onto its 64 d bytes), and all bytes of a 16-token
+    block stay inside that block's 8 d bytes."""
     nbytes, offs = O.page_layout(d, m, True)
-    chunk = d // 8
-    for p in range(6):
-        seen = set()
+    seen = set()
+    for p in range(64):
         for j in range(d):
             pool = np.zeros(nbytes, np.uint8)
             rec = _empty_records(1, d, m)
             rec["vcode"][0, j] = 0x9
             O.pack(pool, nbytes, d, m, True, [0], [2 * p + 1], rec)
-            blk = pool[offs["vc"] + p * d: offs["vc"] + (p + 1) * d]
-            (pos,) = np.nonzero(blk)
-            assert len(pos) == 1 and blk[pos[0]] == 0x90
-            assert pos[0] // chunk == (j // chunk + 2 * (p % 4)) % 8 and pos[0] % chunk == j % chunk
+            sec = pool[offs["vc"]: offs["vc"] + 64 * d]
+            (pos,) = np.nonzero(sec)
+            assert len(pos) == 1 and sec[pos[0]] == 0x90
+            assert pos[0] // (8 * d) == p // 8
             seen.add(int(pos[0]))
-        assert len(seen) == d
+    assert len(seen) == 64 * d
 
 
 @pytest.mark.parametrize("d,m", D_M)
