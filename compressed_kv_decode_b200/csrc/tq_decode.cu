@@ -51,16 +51,17 @@ struct Cfg {
   static constexpr int VC_B = COLD_TOK / 2 * D;
   static constexpr int OFF_QS = KC_B;
   static constexpr int OFF_VC = OFF_QS + QS_B;
-  static constexpr int OFF_KN = OFF_VC + VC_B;
-  static constexpr int OFF_KG = OFF_KN + 2 * COLD_TOK;
-  static constexpr int OFF_VN = OFF_KG + 2 * COLD_TOK;
-  static constexpr int COLD_B = OFF_VN + 2 * COLD_TOK;
+  // the page's three norm sections (key, residual, value) are adjacent and
+  // staged whole with one copy
+  static constexpr int OFF_N = OFF_VC + VC_B;
+  static constexpr int NORM_B = 3 * 2 * TQ_PAGE_TOKENS;
+  static constexpr int COLD_B = OFF_N + NORM_B;
   static constexpr int HROW = 2 * D + 16;  // padded hot row: conflict-free ldmatrix
   static constexpr int HOT_B = 2 * HOT_TOK * HROW;
   static constexpr int SLOT = ((COLD_B > HOT_B ? COLD_B : HOT_B) + 127) / 128 * 128;
   static constexpr int NSLOT = (D == 128) ? 2 : 3;
   static constexpr int PBUF = COLD_TOK * 16;  // fp16 P' tile [64 tokens][8 heads]
-  static constexpr int SMEM = NW * (NSLOT * SLOT + PBUF) + NW * NSLOT * 8;
+  static constexpr int SMEM = NW * (NSLOT * SLOT + PBUF) + NW * NSLOT * 8 + NW * NSLOT * 4;
 };
 
 struct Work {
@@ -343,13 +344,12 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
 // 2. attention
 // ---------------------------------------------------------------------------
 template <int D, int G>
-__device__ __forceinline__ void issue_unit(const Params& p, int sg, int lu, int len, uint8_t* dst,
-                                           uint32_t bar, int lane) {
+__device__ __forceinline__ void issue_unit(const Params& p, int sg, int lu, int len, int page,
+                                           uint8_t* dst, uint32_t bar, int lane) {
   using C = Cfg<D, G>;
   const int bh = sg >> 1;
   const uint32_t d0 = smem_u32(dst);
   if ((sg & 1) == 0) {
-    const int page = p.page_table[static_cast<size_t>(bh) * p.max_pages + (lu >> 1)];
     const bool ok = page >= 0 && page < p.pool_pages;
     if (!ok) {
       if (lane == 0) {
@@ -363,12 +363,15 @@ __device__ __forceinline__ void issue_unit(const Params& p, int sg, int lu, int 
     const uint8_t* base = p.pool + static_cast<size_t>(page) * p.page_bytes;
     if (lane == 0) mbar_arrive_expect_tx(bar, C::COLD_B);
     __syncwarp();
-    if (lane == 0) bulk_g2s(d0, base + p.off_kc + half * C::KC_B, C::KC_B, bar);
-    if (lane == 1) bulk_g2s(d0 + C::OFF_QS, base + p.off_qs + half * C::QS_B, C::QS_B, bar);
-    if (lane == 2) bulk_g2s(d0 + C::OFF_VC, base + p.off_vc + half * C::VC_B, C::VC_B, bar);
-    if (lane == 3) bulk_g2s(d0 + C::OFF_KN, base + p.off_kn + half * 2 * COLD_TOK, 2 * COLD_TOK, bar);
-    if (lane == 4) bulk_g2s(d0 + C::OFF_KG, base + p.off_kg + half * 2 * COLD_TOK, 2 * COLD_TOK, bar);
-    if (lane == 5) bulk_g2s(d0 + C::OFF_VN, base + p.off_vn + half * 2 * COLD_TOK, 2 * COLD_TOK, bar);
+    // the four section copies go out as one instruction, one lane each
+    if (lane < 4) {
+      const uint32_t dst = d0 + (lane == 0 ? 0 : lane == 1 ? C::OFF_QS : lane == 2 ? C::OFF_VC : C::OFF_N);
+      const uint8_t* src = base + (lane == 0 ? p.off_kc + half * C::KC_B
+                                   : lane == 1 ? p.off_qs + half * C::QS_B
+                                   : lane == 2 ? p.off_vc + half * C::VC_B : p.off_kn);
+      const uint32_t bytes = lane == 0 ? C::KC_B : lane == 1 ? C::QS_B : lane == 2 ? C::VC_B : C::NORM_B;
+      bulk_g2s(dst, src, bytes, bar);
+    }
   } else {
     const int t0 = lu * HOT_TOK;
     const int rows = min(HOT_TOK, len - t0);
@@ -411,6 +414,9 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
   uint8_t* pbuf = smem + NW * C::NSLOT * C::SLOT + warp * C::PBUF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NW * (C::NSLOT * C::SLOT + C::PBUF)) +
                    warp * C::NSLOT;
+  // page index of the unit staged in each slot (validity of cold pages)
+  int* slot_page = reinterpret_cast<int*>(smem + NW * (C::NSLOT * C::SLOT + C::PBUF) + NW * C::NSLOT * 8) +
+                   warp * C::NSLOT;
 
   const int* sched = p.w.sched;
   const int U = sched[0];
@@ -437,15 +443,33 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
     if (uoff[mid] <= u0) lo = mid; else hi = mid - 1;
   }
   // issue cursor
-  int isg = lo, ilu = u0 - uoff[lo];
+  int isg = lo, ilu = u0 - uoff[lo], iend = uoff[lo + 1];
   int iu = u0;
-  auto issue_next = [&](int slot) {
-    while (uoff[isg + 1] <= iu) { ++isg; ilu = 0; }
-    issue_unit<D, G>(p, isg, ilu, slen[isg], slots + slot * C::SLOT, smem_u32(&bars[slot]), lane);
+  // the next unit to stage: located (and its page looked up) one unit ahead
+  // of its copy, so the page-table load overlaps a unit of compute
+  int nx_sg = 0, nx_lu = 0, nx_len = 0, nx_page = -1;
+  auto prep_next = [&]() {
+    while (iend <= iu) {  // segment ends are read once per segment
+      ++isg;
+      ilu = 0;
+      iend = uoff[isg + 1];
+    }
+    nx_sg = isg;
+    nx_lu = ilu;
+    nx_len = slen[isg];
+    nx_page = ((isg & 1) == 0) ? p.page_table[static_cast<size_t>(isg >> 1) * p.max_pages + (ilu >> 1)] : 0;
+  };
+  auto fire_next = [&](int slot) {
+    if (lane == 0) slot_page[slot] = nx_page;
+    issue_unit<D, G>(p, nx_sg, nx_lu, nx_len, nx_page, slots + slot * C::SLOT, smem_u32(&bars[slot]),
+                     lane);
     ++iu;
     ++ilu;
   };
-  for (int s = 0; s < C::NSLOT && iu < u1; ++s) issue_next(s);
+  for (int s = 0; s < C::NSLOT && iu < u1; ++s) {
+    prep_next();
+    fire_next(s);
+  }
 
   // value dequant tables: low and high bytes of fp16(val_c[k])
   uint32_t tl0 = 0, tl1 = 0, th0 = 0, th1 = 0;
@@ -462,7 +486,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
   }
 
   // consume cursor
-  int sg = lo, lu = u0 - uoff[lo];
+  int sg = lo, lu = u0 - uoff[lo], send = uoff[lo + 1];
   uint32_t bfr[C::RC];
   float dsc[C::NT];
   float mrun[C::NT], lrun[C::NT];
@@ -578,6 +602,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
 
   const uint32_t pb_addr = smem_u32(pbuf);
   for (int u = u0, k = 0; u < u1; ++u, ++k) {
+    if (iu < u1) prep_next();
     const int slot = k % C::NSLOT;
     const uint32_t parity = static_cast<uint32_t>(k / C::NSLOT) & 1u;
     uint8_t* sb = slots + slot * C::SLOT;
@@ -592,12 +617,13 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
     const int len = slen[sg];
     if ((sg & 1) == 0) {
       // ---------------- cold unit: 64 tokens ----------------
-      const int page = p.page_table[static_cast<size_t>(bh) * p.max_pages + (lu >> 1)];
+      const int page = slot_page[slot];
       const int nv = (page >= 0 && page < p.pool_pages) ? min(COLD_TOK, len - lu * COLD_TOK) : 0;
       float sv[C::NT * 8];
-      const __half* kn = reinterpret_cast<const __half*>(sb + C::OFF_KN);
-      const uint16_t* kg = reinterpret_cast<const uint16_t*>(sb + C::OFF_KG);
-      const __half* vn = reinterpret_cast<const __half*>(sb + C::OFF_VN);
+      const int hoff = (lu & 1) * 2 * COLD_TOK;  // this half page's first norm
+      const __half* kn = reinterpret_cast<const __half*>(sb + C::OFF_N + hoff);
+      const uint16_t* kg = reinterpret_cast<const uint16_t*>(sb + C::OFF_N + 2 * TQ_PAGE_TOKENS + hoff);
+      const __half* vn = reinterpret_cast<const __half*>(sb + C::OFF_N + 4 * TQ_PAGE_TOKENS + hoff);
       const int qword = (c * (D / 8)) >> 4, qsb = (c * (D / 8)) & 15;
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
@@ -746,16 +772,17 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         mma_f16(oacc[i], a0, a1, a2, a3, bp0, bp1);
       }
     }
-    // all lanes are done with this slot: refill it
+    // all lanes are done with this slot (every value read from it has been
+    // consumed): refill it
     __syncwarp();
-    fence_proxy_async_smem();
-    if (iu < u1) issue_next(slot);
+    if (iu < u1) fire_next(slot);
     ++lu;
-    if (u + 1 == u1 || u + 1 >= uoff[sg + 1]) {
+    if (u + 1 == u1 || u + 1 >= send) {
       flush_segment();
       if (u + 1 < u1) {
         ++sg;
         while (uoff[sg + 1] <= u + 1) ++sg;
+        send = uoff[sg + 1];
         lu = 0;
         load_segment();
       }
@@ -888,6 +915,8 @@ WsLayout ws_layout(int B, int Hkv, int Wtot) {
 template <int D, int G>
 int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st) {
   using C = Cfg<D, G>;
+  if (p.off_kg != p.off_kn + 2 * TQ_PAGE_TOKENS || p.off_vn != p.off_kg + 2 * TQ_PAGE_TOKENS)
+    return TQ_ERR_UNSUPPORTED;  // norm sections staged with one copy
   const int grid = ctx->num_sms;
   p.Wtot = grid * NW;
   p.S = 2 * p.B * p.Hkv;
