@@ -107,13 +107,14 @@ tq_status tq_init_codebook(const tq_config* cfg, tq_ctx** out) {
   for (size_t i = 0; i < h.val_c.size() && i < 8; ++i) ctx->cb.val_c[i] = h.val_c[i];
   for (size_t i = 0; i < h.val_t.size() && i < 7; ++i) ctx->cb.val_t[i] = h.val_t[i];
 
-  // one device block: rot f32 | qjl f32 | qjl f16 | rot bf16 hi, lo | rot f16 hi, lo | err
+  // one device block: rot f32 | qjl f32 | qjl f16 | rot bf16 hi, lo | rot f16 hi, lo | S Pi f32 | err
   const size_t dd = static_cast<size_t>(d) * d, md = static_cast<size_t>(m) * d;
   auto a256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   size_t off_rot = 0, off_qjl = a256(off_rot + dd * 4), off_qjlh = a256(off_qjl + md * 4);
   size_t off_bh = a256(off_qjlh + md * 2), off_bl = a256(off_bh + dd * 2);
   size_t off_hh = a256(off_bl + dd * 2), off_hl = a256(off_hh + dd * 2);
-  size_t off_err = a256(off_hl + dd * 2), total = a256(off_err + 256);
+  size_t off_sp = a256(off_hl + dd * 2);  // S Pi, fp32 [m][d]
+  size_t off_err = a256(off_sp + md * 4), total = a256(off_err + 256);
   std::vector<uint8_t> img(total, 0);
   std::memcpy(img.data() + off_rot, h.rot.data(), dd * 4);
   std::memcpy(img.data() + off_qjl, h.qjl.data(), md * 4);
@@ -129,6 +130,19 @@ tq_status tq_init_codebook(const tq_config* cfg, tq_ctx** out) {
     bl[i] = tq::bf16_bits(x - tq::bf16_value(bh[i]));
     hh[i] = tq::f16_bits(x);
     hl[i] = tq::f16_bits(x - tq::f16_value(hh[i]));
+  }
+  {
+    // S Pi (fp64 sums, fp32 store): the decode prep forms q_s = S (Pi q) as
+    // (S Pi) q, in the same pass as Pi q
+    float* sp = reinterpret_cast<float*>(img.data() + off_sp);
+    for (int r = 0; r < m; ++r)
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k)
+          acc += static_cast<double>(h.qjl[static_cast<size_t>(r) * d + k]) *
+                 static_cast<double>(h.rot[static_cast<size_t>(k) * d + c]);
+        sp[static_cast<size_t>(r) * d + c] = static_cast<float>(acc);
+      }
   }
   void* blk = nullptr;
   if (cudaMalloc(&blk, total) != cudaSuccess) {
@@ -149,6 +163,7 @@ tq_status tq_init_codebook(const tq_config* cfg, tq_ctx** out) {
   ctx->dev.rot_bf_lo = reinterpret_cast<const uint16_t*>(b + off_bl);
   ctx->dev.rot_h_hi = reinterpret_cast<const uint16_t*>(b + off_hh);
   ctx->dev.rot_h_lo = reinterpret_cast<const uint16_t*>(b + off_hl);
+  ctx->dev.sp = reinterpret_cast<const float*>(b + off_sp);
   ctx->dev.err = reinterpret_cast<int*>(b + off_err);
   *out = ctx;
   return TQ_OK;

@@ -89,6 +89,7 @@ struct Params {
   float* out;
   const float* rot;
   const float* qjl;
+  const float* sp;  // S Pi
   float kc0, kc1, alpha;
   float vc[8];
   int* err;
@@ -105,6 +106,14 @@ __device__ __forceinline__ int* seg_len(const Params& p) { return p.w.sched + 4 
 __device__ __forceinline__ int warp_of(long long u, long long U, long long W) {
   return static_cast<int>(((u + 1) * W - 1) / U);
 }
+
+// Programmatic dependent launch: a kernel lets the next one in the stream be
+// scheduled early (launch_dependents), and the next one waits for this one's
+// completion and memory before touching its results (wait).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // 1. prep
@@ -259,9 +268,48 @@ __device__ __forceinline__ void matvec_rows(const float* __restrict__ M, const f
   }
 }
 
+// y1 = M1 x and y2 = M2 x together: every row load of both is issued first
+template <int D, int G>
+__device__ __forceinline__ void matvec_rows2(const float* __restrict__ M1, const float* __restrict__ M2,
+                                             const float (*x)[D], float (*y1)[D], float (*y2)[D]) {
+  constexpr int LANES = D / 4;
+  constexpr int ROWS_PER_PASS = 32 / LANES;
+  constexpr int PASSES = D / (PREP_WARPS * ROWS_PER_PASS);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / LANES, l4 = lane % LANES;
+  float4 mrow[2][PASSES];
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps) {
+    const int r = (ps * PREP_WARPS + warp) * ROWS_PER_PASS + sub;
+    mrow[0][ps] = __ldg(reinterpret_cast<const float4*>(M1 + static_cast<size_t>(r) * D) + l4);
+    mrow[1][ps] = __ldg(reinterpret_cast<const float4*>(M2 + static_cast<size_t>(r) * D) + l4);
+  }
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int r = (ps * PREP_WARPS + warp) * ROWS_PER_PASS + sub;
+      const float4 m = mrow[w][ps];
+      float acc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        acc[g] = m.x * x[g][4 * l4] + m.y * x[g][4 * l4 + 1] + m.z * x[g][4 * l4 + 2] +
+                 m.w * x[g][4 * l4 + 3];
+#pragma unroll
+        for (int o = LANES / 2; o > 0; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
+      }
+      if (l4 == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) (w == 0 ? y1 : y2)[g][r] = acc[g];
+      }
+    }
+  }
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   using C = Cfg<D, G>;
+  pdl_launch_dependents();
   const int BH = p.B * p.Hkv;
   if (blockIdx.x == BH) {
     build_schedule(p);
@@ -279,9 +327,7 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
                              static_cast<tq_dtype>(p.q_dtype));
   }
   __syncthreads();
-  matvec_rows<D, G>(p.rot, sq, sqr);  // q_rot = Pi q
-  __syncthreads();
-  matvec_rows<D, G>(p.qjl, sqr, sqs);  // q_s = S q_rot
+  matvec_rows2<D, G>(p.rot, p.sp, sq, sqr, sqs);  // q_rot = Pi q, q_s = (S Pi) q
   __syncthreads();
   const float w1c = p.sl * p.kc0, w2c = p.sl * 128.0f * (p.kc1 - p.kc0), w3c = p.sl * p.alpha;
   for (int i = tid; i < G * D; i += blockDim.x) {
@@ -406,6 +452,8 @@ __device__ __forceinline__ void dequant_values(uint32_t x, uint32_t tl0, uint32_
 
 template <int D, int G>
 __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
+  pdl_wait();  // schedule and query operands come from the prep launch
+  pdl_launch_dependents();
   using C = Cfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -798,59 +846,11 @@ constexpr int MAX_COMBINE_SLOTS = 256;  // partial records staged in shared memo
 template <int D, int G>
 __global__ void __launch_bounds__(D) combine_kernel(Params p) {
   const int bh = blockIdx.x, b = bh / p.Hkv, kvh = bh % p.Hkv;
-  const int* sched = p.w.sched;
-  const int* soff = sched + 4 + p.S + 1;
   const int j = threadIdx.x;
-  __shared__ float sm_m[MAX_COMBINE_SLOTS][G], sm_l[MAX_COMBINE_SLOTS][G];
-  __shared__ float so[G][D];
-  float M[2][G], L[2][G], O[2][G];
-#pragma unroll
-  for (int dom = 0; dom < 2; ++dom) {
-    const int sg = 2 * bh + dom;
-    const int a = soff[sg], e = soff[sg + 1];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      M[dom][g] = -__builtin_huge_valf();
-      L[dom][g] = 0.0f;
-      O[dom][g] = 0.0f;
-    }
-    for (int base = a; base < e; base += MAX_COMBINE_SLOTS) {
-      const int n = min(MAX_COMBINE_SLOTS, e - base);
-      __syncthreads();
-      // (m, l) of every slot and head, loaded with independent requests
-      for (int i = j; i < n * G; i += blockDim.x) {
-        const int s = i / G, g = i % G;
-        const float* rec = p.w.part + static_cast<size_t>(base + s) * G * (D + 2);
-        sm_m[s][g] = rec[g];
-        sm_l[s][g] = rec[G + g];
-      }
-      __syncthreads();
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float mx = M[dom][g];
-        for (int s = 0; s < n; ++s)
-          if (sm_l[s][g] > 0.0f) mx = fmaxf(mx, sm_m[s][g]);
-        const float resc = (M[dom][g] == -__builtin_huge_valf() || mx == -__builtin_huge_valf())
-                               ? 0.0f : exp2f(M[dom][g] - mx);
-        float l = L[dom][g] * resc, o = O[dom][g] * resc;
-#pragma unroll 4
-        for (int s = 0; s < n; ++s) {
-          const float lw = sm_l[s][g];
-          const float f = (lw > 0.0f) ? exp2f(sm_m[s][g] - mx) : 0.0f;
-          l += lw * f;
-          o += p.w.part[static_cast<size_t>(base + s) * G * (D + 2) + 2 * G + g * D + j] * f;
-        }
-        M[dom][g] = mx;
-        L[dom][g] = l;
-        O[dom][g] = o;
-      }
-    }
-  }
-  // cold accumulators are in the rotated domain: o_cold = Pi^T o_rot, all heads at once;
-  // Pi is staged in shared memory with every load of the thread in flight at once
+  // Pi does not depend on the attention launch: stage it in shared memory
+  // first, every load of the thread in flight at once, overlapping the tail
+  // of that launch
   extern __shared__ float spi[];  // [D][D]
-#pragma unroll
-  for (int g = 0; g < G; ++g) so[g][j] = O[0][g];
   {
     constexpr int PER = D * D / 4 / D;  // float4 per thread
     float4 v[PER];
@@ -859,6 +859,71 @@ __global__ void __launch_bounds__(D) combine_kernel(Params p) {
 #pragma unroll
     for (int i = 0; i < PER; ++i) reinterpret_cast<float4*>(spi)[i * D + j] = v[i];
   }
+  pdl_wait();  // partial records come from the attention launch
+  const int* sched = p.w.sched;
+  const int* soff = sched + 4 + p.S + 1;
+  __shared__ float sm_m[MAX_COMBINE_SLOTS][G], sm_l[MAX_COMBINE_SLOTS][G];
+  __shared__ float so[G][D];
+  constexpr float NINF = -__builtin_huge_valf();
+  constexpr int RB = G * (D + 2);  // floats per record
+  float M[2][G], L[2][G], O[2][G];
+#pragma unroll
+  for (int dom = 0; dom < 2; ++dom) {
+    const int sg = 2 * bh + dom;
+    const int a = soff[sg], e = soff[sg + 1];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      M[dom][g] = NINF;
+      L[dom][g] = 0.0f;
+      O[dom][g] = 0.0f;
+    }
+    for (int base = a; base < e; base += MAX_COMBINE_SLOTS) {
+      const int n = min(MAX_COMBINE_SLOTS, e - base);
+      __syncthreads();
+      for (int i = j; i < n * G; i += blockDim.x) {
+        const int sl = i / G, g = i % G;
+        const float* rec = p.w.part + static_cast<size_t>(base + sl) * RB;
+        sm_m[sl][g] = rec[g];
+        sm_l[sl][g] = rec[G + g];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float mx = M[dom][g];
+        for (int sl = 0; sl < n; ++sl)
+          if (sm_l[sl][g] > 0.0f) mx = fmaxf(mx, sm_m[sl][g]);
+        const float resc = (M[dom][g] == NINF || mx == NINF) ? 0.0f : exp2f(M[dom][g] - mx);
+        L[dom][g] *= resc;
+        O[dom][g] *= resc;
+        M[dom][g] = mx;
+      }
+      // partial outputs: eight records x every head requested at once
+      for (int s0 = 0; s0 < n; s0 += 8) {
+        float ov[8][G];
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            ov[t][g] = (s0 + t < n) ? p.w.part[static_cast<size_t>(base + s0 + t) * RB + 2 * G + g * D + j]
+                                    : 0.0f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (s0 + t < n) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              const float lw = sm_l[s0 + t][g];
+              const float f = (lw > 0.0f) ? exp2f(sm_m[s0 + t][g] - M[dom][g]) : 0.0f;
+              L[dom][g] += lw * f;
+              O[dom][g] += ov[t][g] * f;
+            }
+          }
+        }
+      }
+    }
+  }
+  // cold accumulators are in the rotated domain: o_cold = Pi^T o_rot, all heads at once
+#pragma unroll
+  for (int g = 0; g < G; ++g) so[g][j] = O[0][g];
   __syncthreads();
   float oc[G];
 #pragma unroll
@@ -873,7 +938,7 @@ __global__ void __launch_bounds__(D) combine_kernel(Params p) {
   for (int g = 0; g < G; ++g) {
     const float Mx = fmaxf(M[0][g], M[1][g]);
     float res = 0.0f;
-    if (Mx != -__builtin_huge_valf()) {
+    if (Mx != NINF) {
       const float fc = (L[0][g] > 0.0f) ? exp2f(M[0][g] - Mx) : 0.0f;
       const float fh = (L[1][g] > 0.0f) ? exp2f(M[1][g] - Mx) : 0.0f;
       const float den = L[0][g] * fc + L[1][g] * fh;
@@ -938,7 +1003,19 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
   }
   prep_kernel<D, G><<<p.B * p.Hkv + 1, PREP_WARPS * 32, 0, st>>>(p);
   if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
-  attn_kernel<D, G><<<grid, NW * 32, C::SMEM, st>>>(p);
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NW * 32);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_kernel<D, G>, p) != cudaSuccess) return TQ_ERR_CUDA;
+  }
   if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
   static bool comb_set[2][9] = {};
   bool& cset = comb_set[D == 128][G];
@@ -948,7 +1025,19 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
       return TQ_ERR_CUDA;
     cset = true;
   }
-  combine_kernel<D, G><<<p.B * p.Hkv, D, D * D * 4, st>>>(p);
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.B * p.Hkv);
+    cfg.blockDim = dim3(D);
+    cfg.dynamicSmemBytes = D * D * 4;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, combine_kernel<D, G>, p) != cudaSuccess) return TQ_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
@@ -1012,6 +1101,7 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
   p.out = out;
   p.rot = ctx->dev.rot;
   p.qjl = ctx->dev.qjl;
+  p.sp = ctx->dev.sp;
   p.kc0 = ctx->cb.key_c[0];
   p.kc1 = ctx->cb.key_c[1];
   p.alpha = std::sqrt(3.14159265358979323846f / 2.0f) / static_cast<float>(ctx->cfg.qjl_dim);

@@ -39,6 +39,7 @@ struct DeviceTables {
   const uint16_t* rot_bf_lo; // [d*d] bf16 bits of rot - bf16(rot)
   const uint16_t* rot_h_hi;  // [d*d] fp16 bits of rot
   const uint16_t* rot_h_lo;  // [d*d] fp16 bits of rot - fp16(rot)
+  const float* sp;           // [m*d] S Pi (fp32)
   int* err;                  // device error word (first error wins)
 };
 
