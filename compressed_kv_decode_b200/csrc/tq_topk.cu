@@ -6,14 +6,19 @@
 //
 // Launches:
 //  1. qprep   per query: q_rot, q_s, estimator constants folded in, per-query
-//             power-of-two prescale, fp16 hi/lo split, stored as the B matrix
-//             of the tensor-core contraction in MMA k-index order.
-//  2. score   persistent CTAs over (query tile of 32, database slice) items.
-//             Each warp unpacks 32 database records at a time straight from
-//             global memory (L2-resident) into exact {0, +-1, +-2^-7, +-gamma}
-//             fp16 fragments and contracts them with the query tile held in
-//             shared memory (m16n8k16 MMAs, fp32 accumulate); a threshold filter
-//             feeds rare insertions into per-warp top-k lists in shared memory.
+//             power-of-two prescale, fp16 hi/lo split, written into the
+//             tensor-core B operand of its 64-query block (K-major, 128-byte
+//             swizzle, rows = query x {hi, lo}).
+//  2. score   persistent CTAs over items = (64-query block, slice of database
+//             pages), one CTA per SM.  The block's B operand stays in shared
+//             memory for the item.  For each 128-record page, eight warps
+//             expand the packed codes into fp16 bit planes in tensor memory
+//             (A, lane = record: sign, sign*magnitude, QJL signs x gamma) while
+//             the previous page's product runs; a control warp issues one
+//             tcgen05.mma chain per page (M = 128 records, N = 64 queries x
+//             {hi, lo}, K = 3d) into a TMEM accumulator.  The eight warps read
+//             the scores back, and a threshold filter feeds rare insertions into
+//             per-warp top-k lists in shared memory.
 //  3. merge   per query: the best k of all per-warp lists.
 #include <cuda_runtime.h>
 
@@ -22,21 +27,41 @@
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
+#include "tq_tc.cuh"
 
 namespace tq {
 namespace tk {
 
-constexpr int NWARP = 8;
-constexpr int QT = 32;  // queries per tile (64 B columns: hi, lo)
+constexpr int NEPI = 8;                    // epilogue warps: (TMEM lane quarter) x (query half)
+constexpr int NTHREADS = (NEPI + 1) * 32;  // + the control warp
+constexpr int QB = 64;                     // queries per block
+constexpr int NROW = 2 * QB;               // B rows: query x {hi, lo}
+constexpr int QH = QB / 2;                 // queries per epilogue warp
+constexpr int PAGE = TQ_PAGE_TOKENS;       // records per tile
+constexpr int SB_LD = QH + 1;              // score staging row (padded)
+constexpr int SB_BYTES = NEPI * 32 * SB_LD * 4;
 constexpr float NEG_INF = -__builtin_huge_valf();
+
+// float <-> unsigned with the same order (for atomicMax on scores)
+__device__ __forceinline__ uint32_t ord_bits(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float unord_bits(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+constexpr uint32_t ORD_NEG_INF = 0x007fffffu;
 
 template <int D>
 struct Cfg {
-  static constexpr int KS = D / 16;
-  static constexpr int KTOT = 3 * D;          // k extent: sign plane, magnitude plane, QJL plane
-  static constexpr int RB = 2 * KTOT + 16;    // padded B row bytes
-  static constexpr int NTQ = 2 * QT / 8;      // n-tiles per query tile
-  static constexpr int SMEM_B = 2 * QT * RB;  // B tile
+  static constexpr int KTOT = 3 * D;              // sign plane, magnitude plane, QJL plane
+  static constexpr int B_BYTES = NROW * KTOT * 2;  // one block's B operand (SW128 image)
+  static constexpr int ACOLS = KTOT / 2;           // TMEM columns of one A buffer
+  static constexpr int COL_A0 = 0, COL_A1 = 192, COL_D = 384;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(ACOLS <= 192, "A buffer");
+  // shared memory (from a 1024-byte aligned base): B | lists | barriers
+  static constexpr int OFF_B = 0;
 };
 
 struct Params {
@@ -48,64 +73,90 @@ struct Params {
   long long page_bytes;
   int off_kc, off_qs, off_kn, off_kg;
   const float* rot;
-  const float* qjl;
+  const float* sp;  // S Pi
   float kc0, kc1, alpha;
-  uint16_t* bmat;    // [Q * 2][KTOT] fp16 bits (rows: query hi, query lo)
-  float* desc;       // [Q] descale
-  float* cand_s;     // [items][NWARP][QT][k]
+  uint16_t* bimg;   // [n_qb][NROW * KTOT] fp16 bits, SW128 image per block
+  float* desc;      // [n_qb * QB] descale
+  uint32_t* gbound;  // [n_qb * QB] best known lower bound of each query's k-th score (ordered bits)
+  float* cand_s;    // [items][NEPI][QH][k]
   int* cand_i;
-  int n_slices;
+  int n_qb, n_slices;
   long long pages;
   int* err;
 };
 
-// coordinate fed by MMA k-index kk (0..15) of key k-step s for lane column c
+// K index k of the A operand (and so of B): plane, and the coordinate
+// (planes 0, 1) or sketch index (plane 2).  A record's A row holds, per plane,
+// two halves of D/4 TMEM columns; column c of a half covers two K elements
+// (low, high 16 bits):
+//   planes 0/1: c = 8 wl + 2 i + e -> coordinate 16 (half*D/32 + wl) + 2 i + e (+ 8 high)
+//   plane 2:    c = 16 wl + r      -> sketch index 32 (half*D/64 + wl) + r (+ 16 high)
 template <int D>
-__device__ __forceinline__ int key_coord(int s, int kk) {
-  const int c = (kk & 7) >> 1, e = kk & 1, reg = kk >> 3;
-  const int P = c * (D / 8) + 2 * s + reg;
-  return 16 * (P >> 3) + (P & 7) + 8 * e;
-}
-
-template <int D>
-__device__ __forceinline__ int qjl_index(int s, int kk) {
-  const int c = (kk & 7) >> 1, e = kk & 1, reg = kk >> 3;
-  const int P = c * (D / 8) + 2 * s + reg;
-  return 32 * (P >> 4) + (P & 15) + 16 * e;
-}
-
-// y[r] = sum_k M[r][k] x[k]: one warp per row, float4 per lane, shuffle reduce
-template <int D>
-__device__ __forceinline__ void warp_matvec(const float* __restrict__ M, const float* x, float* y) {
-  constexpr int LANES = D / 4, RPP = 32 / LANES, NW = 4, PASSES = D / (NW * RPP);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sub = lane / LANES, l4 = lane % LANES;
-  float4 m[PASSES];
-#pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps)
-    m[ps] = __ldg(reinterpret_cast<const float4*>(M + static_cast<size_t>((ps * NW + warp) * RPP + sub) * D) + l4);
-#pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps) {
-    float a = m[ps].x * x[4 * l4] + m[ps].y * x[4 * l4 + 1] + m[ps].z * x[4 * l4 + 2] + m[ps].w * x[4 * l4 + 3];
-#pragma unroll
-    for (int o = LANES / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (l4 == 0) y[(ps * NW + warp) * RPP + sub] = a;
+__host__ __device__ __forceinline__ void k_index(int k, int& plane, int& idx) {
+  const int col = k >> 1, hiword = k & 1;
+  plane = col / (D / 2);
+  const int c = col % (D / 2);
+  const int half = c / (D / 4), l = c % (D / 4);
+  if (plane < 2) {
+    const int wl = l >> 3, i = (l & 7) >> 1, e = l & 1;
+    idx = 16 * (half * (D / 32) + wl) + 2 * i + e + 8 * hiword;
+  } else {
+    const int wl = l >> 4, r = l & 15;
+    idx = 32 * (half * (D / 64) + wl) + r + 16 * hiword;
   }
 }
 
+// y1 = M1 x and y2 = M2 x (D x D, one warp per row group, float4 per lane)
+template <int D>
+__device__ __forceinline__ void warp_matvec2(const float* __restrict__ M1, const float* __restrict__ M2,
+                                             const float* x, float* y1, float* y2) {
+  constexpr int LANES = D / 4, RPP = 32 / LANES, NW = 4, PASSES = D / (NW * RPP);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sub = lane / LANES, l4 = lane % LANES;
+  float4 m[2][PASSES];
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps) {
+    const size_t r = static_cast<size_t>((ps * NW + warp) * RPP + sub);
+    m[0][ps] = __ldg(reinterpret_cast<const float4*>(M1 + r * D) + l4);
+    m[1][ps] = __ldg(reinterpret_cast<const float4*>(M2 + r * D) + l4);
+  }
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) {
+      float a = m[w][ps].x * x[4 * l4] + m[w][ps].y * x[4 * l4 + 1] + m[w][ps].z * x[4 * l4 + 2] +
+                m[w][ps].w * x[4 * l4 + 3];
+#pragma unroll
+      for (int o = LANES / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (l4 == 0) (w == 0 ? y1 : y2)[(ps * NW + warp) * RPP + sub] = a;
+    }
+  }
+}
+
+// one CTA per query slot of the padded blocks; slots past Q write zero rows
 template <int D>
 __global__ void __launch_bounds__(128) qprep_kernel(Params p) {
   using C = Cfg<D>;
-  const int q = blockIdx.x;
+  const int q = blockIdx.x, qb = q / QB, ql = q % QB;
   __shared__ float sq[D], sr[D], ss[D];
   __shared__ unsigned smax;
   __shared__ float sfac;
   const int tid = threadIdx.x;
+  uint8_t* img = reinterpret_cast<uint8_t*>(p.bimg + static_cast<size_t>(qb) * (C::B_BYTES / 2));
+  if (q >= p.Q) {
+    for (int k0 = tid * 8; k0 < C::KTOT; k0 += blockDim.x * 8)
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+        *reinterpret_cast<uint4*>(img + tc::sw128_offset(2 * ql + part, k0, NROW)) = make_uint4(0, 0, 0, 0);
+    if (tid == 0) {
+      p.desc[q] = 0.0f;
+      p.gbound[q] = ORD_NEG_INF;
+    }
+    return;
+  }
   if (tid == 0) smax = 0u;
   for (int j = tid; j < D; j += blockDim.x) sq[j] = p.queries[static_cast<size_t>(q) * D + j];
   __syncthreads();
-  warp_matvec<D>(p.rot, sq, sr);
-  __syncthreads();
-  warp_matvec<D>(p.qjl, sr, ss);
+  warp_matvec2<D>(p.rot, p.sp, sq, sr, ss);  // q_rot = Pi q, q_s = (S Pi) q
   __syncthreads();
   const float w1 = p.kc0, w2 = 128.0f * (p.kc1 - p.kc0), w3 = p.alpha;
   for (int j = tid; j < D; j += blockDim.x) {
@@ -123,19 +174,25 @@ __global__ void __launch_bounds__(128) qprep_kernel(Params p) {
     }
     sfac = f;
     p.desc[q] = 1.0f / f;
+    p.gbound[q] = ORD_NEG_INF;
   }
   __syncthreads();
   const float f = sfac;
-  for (int kk = tid; kk < C::KTOT; kk += blockDim.x) {
-    const int plane = kk / D, s = (kk % D) / 16, ki = kk % 16;
-    float w;
-    if (plane == 0) w = w1 * sr[key_coord<D>(s, ki)];
-    else if (plane == 1) w = w2 * sr[key_coord<D>(s, ki)];
-    else w = w3 * ss[qjl_index<D>(s, ki)];
-    uint16_t hi, lo;
-    split_f16(f * w, hi, lo);
-    p.bmat[(static_cast<size_t>(q) * 2) * C::KTOT + kk] = hi;
-    p.bmat[(static_cast<size_t>(q) * 2 + 1) * C::KTOT + kk] = lo;
+  // 16-byte chunks of 8 K elements, hi and lo rows
+  for (int k0 = tid * 8; k0 < C::KTOT; k0 += blockDim.x * 8) {
+    uint32_t wh[4] = {0u, 0u, 0u, 0u}, wl[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      int plane, idx;
+      k_index<D>(k0 + e, plane, idx);
+      const float w = plane == 0 ? w1 * sr[idx] : plane == 1 ? w2 * sr[idx] : w3 * ss[idx];
+      uint16_t hi, lo;
+      split_f16(f * w, hi, lo);
+      wh[e >> 1] |= static_cast<uint32_t>(hi) << (16 * (e & 1));
+      wl[e >> 1] |= static_cast<uint32_t>(lo) << (16 * (e & 1));
+    }
+    *reinterpret_cast<uint4*>(img + tc::sw128_offset(2 * ql, k0, NROW)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    *reinterpret_cast<uint4*>(img + tc::sw128_offset(2 * ql + 1, k0, NROW)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
   }
 }
 
@@ -143,213 +200,388 @@ __device__ __forceinline__ bool better(float sa, int ia, float sb, int ib) {
   return sa > sb || (sa == sb && ia < ib);
 }
 
-// insert (s, id) into a sorted (best first) list of k entries
-__device__ __forceinline__ void list_insert(float* ls, int* li, int k, float s, int id) {
-  if (!better(s, id, ls[k - 1], li[k - 1])) return;
-  int pos = k - 1;
-  while (pos > 0 && better(s, id, ls[pos - 1], li[pos - 1])) {
-    ls[pos] = ls[pos - 1];
-    li[pos] = li[pos - 1];
-    --pos;
+// Insert (cs, ci) into the sorted (best first) list of k <= 32 entries, the
+// whole warp at once: lane e holds entry e, the rank of the candidate is the
+// number of entries ahead of it, the entries behind it move down one lane.
+// Returns the list's k-th entry afterwards in (ts, ti) (ti < 0x7fffffff once
+// the list is full).
+__device__ __forceinline__ void warp_insert(float* ls, int* li, int k, float cs, int ci, float& ts, int& ti) {
+  const int lane = threadIdx.x & 31;
+  const bool in = lane < k;
+  const float es = in ? ls[lane] : NEG_INF;
+  const int ei = in ? li[lane] : 0x7fffffff;
+  const int pos = __popc(__ballot_sync(0xffffffffu, in && better(es, ei, cs, ci)));
+  const float us = __shfl_up_sync(0xffffffffu, es, 1);
+  const int ui = __shfl_up_sync(0xffffffffu, ei, 1);
+  float ns = es;
+  int ni = ei;
+  if (lane == pos) {
+    ns = cs;
+    ni = ci;
+  } else if (lane > pos) {
+    ns = us;
+    ni = ui;
   }
-  ls[pos] = s;
-  li[pos] = id;
+  if (in && pos < k) {
+    ls[lane] = ns;
+    li[lane] = ni;
+  }
+  ts = __shfl_sync(0xffffffffu, ns, k - 1);
+  ti = __shfl_sync(0xffffffffu, ni, k - 1);
+  __syncwarp();
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N == 32) tc::st32(taddr, r);
+  else if constexpr (N == 16) tc::st16(taddr, r);
+  else tc::st8(taddr, r);
+}
+
+// A row of one record (this thread's half of the coordinates), from its
+// packed words: sign plane (+-1), sign*magnitude plane (+-2^-7), QJL plane
+// (+-gamma).  Key code word w holds coordinates 16 w + 8 h + 2 i + e with the
+// sign bit at 16 h + 15 - 4 i - e and the magnitude bit two below; QJL word
+// w holds sketch index 32 w + 16 h + r at bit 16 h + 15 - r.
+template <int D>
+__device__ __forceinline__ void build_a_row(const uint32_t* kw, const uint32_t* qw, uint32_t gg,
+                                            uint32_t base, int half) {
+  constexpr int NW = D / 32;  // key words of one half
+  uint32_t a[D / 4];
+#pragma unroll
+  for (int wl = 0; wl < NW; ++wl)
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      a[wl * 8 + s] = ((kw[wl] << ((s >> 1) * 4 + (s & 1))) & 0x80008000u) | 0x3C003C00u;
+  tmem_store<D / 4>(base + half * (D / 4), a);
+#pragma unroll
+  for (int wl = 0; wl < NW; ++wl)
+#pragma unroll
+    for (int s = 0; s < 8; ++s) a[wl * 8 + s] = (kw[wl] << ((s >> 1) * 4 + (s & 1))) & 0xA000A000u;
+  tmem_store<D / 4>(base + D / 2 + half * (D / 4), a);
+#pragma unroll
+  for (int wl = 0; wl < D / 64; ++wl)
+#pragma unroll
+    for (int r = 0; r < 16; ++r) a[wl * 16 + r] = ((qw[wl] << r) & 0x80008000u) | gg;
+  tmem_store<D / 4>(base + D + half * (D / 4), a);
+}
+
+// the packed words of one record half, gamma and norm
+template <int D>
+struct Rec {
+  uint32_t kw[D / 32];
+  uint32_t qw[D / 64];
+  uint32_t gg;
+  uint32_t n;
+};
+
+template <int D>
+__device__ __forceinline__ void load_rec(Rec<D>& r, const uint8_t* pg, const Params& p, int slot, int half) {
+  const uint8_t* kp = pg + p.off_kc + slot * (D / 4) + half * (D / 8);
+  const uint8_t* qp = pg + p.off_qs + slot * (D / 8) + half * (D / 16);
+  if constexpr (D == 128) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(kp));
+    r.kw[0] = v.x; r.kw[1] = v.y; r.kw[2] = v.z; r.kw[3] = v.w;
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(qp));
+    r.qw[0] = u.x; r.qw[1] = u.y;
+  } else {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(kp));
+    r.kw[0] = v.x; r.kw[1] = v.y;
+    r.qw[0] = __ldg(reinterpret_cast<const uint32_t*>(qp));
+  }
+  r.gg = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(pg + p.off_kg) + slot)) * 0x10001u;
+  r.n = __ldg(reinterpret_cast<const uint16_t*>(pg + p.off_kn) + slot);
+}
+
+// the pages of slice sl of n_slices over the database
+__device__ __forceinline__ void slice_pages(const Params& p, int item, long long& pg0, long long& pg1) {
+  const int sl = item / p.n_qb;
+  pg0 = p.pages * sl / p.n_slices;
+  pg1 = p.pages * (sl + 1) / p.n_slices;
+}
+
+// CTA tile sequence: the pages of its items, item after item
+struct TileSeq {
+  int item;
+  long long page, end;
+  __device__ __forceinline__ bool start(const Params& p, int items) {
+    item = blockIdx.x;
+    if (item >= items) return false;
+    slice_pages(p, item, page, end);
+    return page < end;
+  }
+  // advance; false at the end of the sequence
+  __device__ __forceinline__ bool next(const Params& p, int items) {
+    if (++page < end) return true;
+    item += gridDim.x;
+    if (item >= items) return false;
+    slice_pages(p, item, page, end);
+    return page < end;
+  }
+};
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 template <int D>
-__global__ void __launch_bounds__(NWARP * 32, 1) score_kernel(Params p) {
+__global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
   using C = Cfg<D>;
-  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int NMMA = C::KTOT / 16;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, c = lane & 3;
-  uint8_t* bt = smem;
-  float* ls_all = reinterpret_cast<float*>(smem + C::SMEM_B);
-  int* li_all = reinterpret_cast<int*>(smem + C::SMEM_B + NWARP * QT * p.k * 4);
-  float* ls = ls_all + warp * QT * p.k;
-  int* li = li_all + warp * QT * p.k;
+  const int k = p.k;
+  float* ls_all = reinterpret_cast<float*>(smem + C::B_BYTES);
+  int* li_all = reinterpret_cast<int*>(smem + C::B_BYTES + NEPI * QH * k * 4);
+  float* sbuf = reinterpret_cast<float*>(smem + C::B_BYTES + NEPI * QH * k * 8);
+  uint8_t* bars = smem + C::B_BYTES + NEPI * QH * k * 8 + SB_BYTES;
+  const uint32_t bar_ab = smem_u32(bars), bar_dfull = bar_ab + 16, bar_dfree = bar_ab + 24;
+  const uint32_t bar_bfull = bar_ab + 32, bar_bfree = bar_ab + 40, bar_drain = bar_ab + 48;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 56);
+  int& s_failed = *reinterpret_cast<int*>(bars + 60);
 
-  const int n_qt = (p.Q + QT - 1) / QT;
-  const int items = n_qt * p.n_slices;
-  const int qword = (c * (D / 8)) >> 4, qsb = (c * (D / 8)) & 15;
-  const uint32_t b_base = smem_u32(bt) + ((lane & 7) + ((lane >> 4) & 1) * 8) * C::RB + ((lane >> 3) & 1) * 16;
+  const int items = p.n_qb * p.n_slices;
+  if (tid == 0) {
+    mbar_init(bar_ab, NEPI);
+    mbar_init(bar_ab + 8, NEPI);
+    mbar_init(bar_dfull, 1);
+    mbar_init(bar_dfree, NEPI);
+    mbar_init(bar_bfull, 1);
+    mbar_init(bar_bfree, 1);
+    mbar_init(bar_drain, 1);
+    s_failed = 0;
+    mbar_init_fence();
+  }
+  if (warp == NEPI) {
+    tc::tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool failed = false;
 
-  for (int item = blockIdx.x; item < items; item += gridDim.x) {
-    const int qt = item % n_qt, sl = item / n_qt;
-    const int q0 = qt * QT;
-    // query tile: rows 2*i (hi) and 2*i+1 (lo) of the B matrix
-    __syncthreads();
-    for (int i = tid; i < 2 * QT * (C::KTOT / 8); i += blockDim.x) {
-      const int row = i / (C::KTOT / 8), ch = i % (C::KTOT / 8);
-      const int qq = q0 + row / 2;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (qq < p.Q)
-        v = reinterpret_cast<const uint4*>(p.bmat + (static_cast<size_t>(q0) * 2 + row) * C::KTOT)[ch];
-      reinterpret_cast<uint4*>(bt + row * C::RB)[ch] = v;
+  if (warp == NEPI) {
+    // ---- control: B operand per item, one MMA chain per page ------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_f16(128, NROW, false);
+      const uint32_t s_b = smem_u32(smem);
+      TileSeq ts;
+      bool more = ts.start(p, items);
+      uint32_t t = 0, nb = 0;
+      bool b_pending = false;
+      auto load_b = [&](int item) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.bimg) + static_cast<size_t>(item % p.n_qb) * C::B_BYTES;
+        mbar_arrive_expect_tx(bar_bfull, C::B_BYTES);
+        for (int off = 0; off < C::B_BYTES; off += 16384)
+          bulk_g2s(s_b + off, src + off, C::B_BYTES - off < 16384 ? C::B_BYTES - off : 16384, bar_bfull);
+        b_pending = true;
+      };
+      if (more) load_b(ts.item);
+      while (more && !failed) {
+        const int item = ts.item;
+        if (!mbar_wait_bounded(bar_bfull, nb & 1)) { failed = true; break; }
+        b_pending = false;
+        do {
+          if (!mbar_wait_bounded(bar_ab + 8 * (t & 1), (t >> 1) & 1)) { failed = true; break; }
+          if (t > 0 && !mbar_wait_bounded(bar_dfree, (t - 1) & 1)) { failed = true; break; }
+          tc::fence_after_sync();
+          const uint32_t a = tmem + (t & 1 ? C::COL_A1 : C::COL_A0);
+#pragma unroll
+          for (int s = 0; s < NMMA; ++s)
+            tc::mma_f16_tmem_a(tmem + C::COL_D, a + 8 * s,
+                               tc::sdesc_sw128(s_b + (s >> 2) * (NROW * 128) + (s & 3) * 32), idesc, s > 0);
+          tc::commit(bar_dfull);
+          ++t;
+          more = ts.next(p, items);
+        } while (more && ts.item == item);
+        if (failed) break;
+        // the B operand is rewritten once this item's products are done
+        tc::commit(bar_bfree);
+        if (!mbar_wait_bounded(bar_bfree, nb & 1)) { failed = true; break; }
+        ++nb;
+        if (more) load_b(ts.item);
+      }
+      if (failed) {
+        // no copy or product may still be in flight when the CTA exits
+        if (b_pending) mbar_wait_bounded(bar_bfull, nb & 1);
+        tc::commit(bar_drain);
+        mbar_wait_bounded(bar_drain, 0);
+        s_failed = 1;
+      }
     }
-    for (int i = lane; i < QT * p.k; i += 32) {
-      ls[i] = NEG_INF;
-      li[i] = 0x7fffffff;
-    }
-    __syncthreads();
-    // thresholds and descales of this lane's queries (n-tile t -> query 4t + c)
-    float thr_s[C::NTQ];
-    int thr_i[C::NTQ];
-    float dq[C::NTQ];
-#pragma unroll
-    for (int t = 0; t < C::NTQ; ++t) {
-      thr_s[t] = NEG_INF;
-      thr_i[t] = 0x7fffffff;
-      const int qq = q0 + 4 * t + c;
-      dq[t] = (qq < p.Q) ? p.desc[qq] : 0.0f;
-    }
-    const long long pg0 = p.pages * sl / p.n_slices, pg1 = p.pages * (sl + 1) / p.n_slices;
-    // the 32 records of step grp; the next step's words are requested before
-    // the current step's contraction so the L2 latency overlaps it
-    uint32_t kw_n[2][2][D / 64], qw_n[2][2];
-    uint16_t gg_n[2][2], nn_n[2][2];
-    auto fetch = [&](long long grp) {
-      const long long page = grp >> 2;
-      const int slot0 = static_cast<int>(grp & 3) * 32;
-      const uint8_t* pgp = p.db + page * p.page_bytes;
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int slot = slot0 + 16 * mt + g + 8 * r;
-#pragma unroll
-          for (int w = 0; w < D / 64; ++w)
-            kw_n[mt][r][w] = __ldg(reinterpret_cast<const uint32_t*>(pgp + p.off_kc + slot * (D / 4)) + c * (D / 64) + w);
-          qw_n[mt][r] = __ldg(reinterpret_cast<const uint32_t*>(pgp + p.off_qs + slot * (D / 8)) + qword);
-          gg_n[mt][r] = __ldg(reinterpret_cast<const uint16_t*>(pgp + p.off_kg) + slot);
-          nn_n[mt][r] = __ldg(reinterpret_cast<const uint16_t*>(pgp + p.off_kn) + slot);
-        }
+    __syncwarp();
+  } else {
+    // ---- eight warps: A planes, scores, lists --------------------------------
+    const int qr = warp & 3, half = warp >> 2;
+    const int row = 32 * qr + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * qr) << 16);
+    float* ls = ls_all + warp * QH * k;
+    int* li = li_all + warp * QH * k;
+    // lists hold scores before the per-query power-of-two descale (the order
+    // is the same); the descale is applied when a list is written out
+    uint32_t qmask = 0u;
+    int list_item = -1;
+    // lane j: the bound on query j's k-th score (ordered bits): the best
+    // k-th score of any list of this query, in any CTA, seen so far; a record
+    // below it cannot be among the query's k best
+    uint32_t bl = ORD_NEG_INF, bl_pf = ORD_NEG_INF;
+    const uint32_t* gb = p.gbound;
+    int q0h = 0;
+    auto flush = [&](int item) {
+      const size_t base = (static_cast<size_t>(item) * NEPI + warp) * QH * k;
+      const float* dq = p.desc + (item % p.n_qb) * QB + QH * half;
+      for (int i = lane; i < QH * k; i += 32) {
+        p.cand_s[base + i] = ls[i] * __ldg(dq + i / k);
+        p.cand_i[base + i] = li[i];
       }
     };
-    if (pg0 * 4 + warp < pg1 * 4) fetch(pg0 * 4 + warp);
-    for (long long grp = pg0 * 4 + warp; grp < pg1 * 4; grp += NWARP) {
-      const long long page = grp >> 2;
-      const int slot0 = static_cast<int>(grp & 3) * 32;
-      float acc[2][C::NTQ][4];
-      uint32_t kw[2][2][D / 64], qw[2][2];
-      uint32_t gg[2][2];
-      float nn[2][2];
-      int ids[2][2];
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          ids[mt][r] = static_cast<int>(page * TQ_PAGE_TOKENS + slot0 + 16 * mt + g + 8 * r);
-#pragma unroll
-          for (int w = 0; w < D / 64; ++w) kw[mt][r][w] = kw_n[mt][r][w];
-          qw[mt][r] = qw_n[mt][r];
-          gg[mt][r] = static_cast<uint32_t>(gg_n[mt][r]) * 0x10001u;
-          nn[mt][r] = __half2float(__ushort_as_half(nn_n[mt][r]));
-        }
-#pragma unroll
-        for (int t = 0; t < C::NTQ; ++t) acc[mt][t][0] = acc[mt][t][1] = acc[mt][t][2] = acc[mt][t][3] = 0.0f;
+    auto reset = [&](int item) {
+      __syncwarp();
+      for (int i = lane; i < QH * k; i += 32) {
+        ls[i] = NEG_INF;
+        li[i] = 0x7fffffff;
       }
-      if (grp + NWARP < pg1 * 4) fetch(grp + NWARP);
-      // key planes: k-steps 0..KS-1 (sign) and KS..2KS-1 (magnitude)
-#pragma unroll
-      for (int s = 0; s < C::KS; ++s) {
-        const int w = s >> 2, sh = 4 * (s & 3);
-        uint32_t a1[2][4], a2[2][4];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          const uint32_t x0a = kw[mt][0][w] << sh, x0b = kw[mt][0][w] << (sh + 1);
-          const uint32_t x1a = kw[mt][1][w] << sh, x1b = kw[mt][1][w] << (sh + 1);
-          a1[mt][0] = (x0a & 0x80008000u) | 0x3C003C00u;
-          a1[mt][1] = (x1a & 0x80008000u) | 0x3C003C00u;
-          a1[mt][2] = (x0b & 0x80008000u) | 0x3C003C00u;
-          a1[mt][3] = (x1b & 0x80008000u) | 0x3C003C00u;
-          a2[mt][0] = x0a & 0xA000A000u;
-          a2[mt][1] = x1a & 0xA000A000u;
-          a2[mt][2] = x0b & 0xA000A000u;
-          a2[mt][3] = x1b & 0xA000A000u;
-        }
-#pragma unroll
-        for (int t = 0; t < C::NTQ; t += 2) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(b_base + t * 8 * C::RB + s * 32, b0, b1, b2, b3);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            mma_f16(acc[mt][t], a1[mt][0], a1[mt][1], a1[mt][2], a1[mt][3], b0, b1);
-            mma_f16(acc[mt][t + 1], a1[mt][0], a1[mt][1], a1[mt][2], a1[mt][3], b2, b3);
-          }
-          ldsm_x4(b_base + t * 8 * C::RB + (C::KS + s) * 32, b0, b1, b2, b3);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            mma_f16(acc[mt][t], a2[mt][0], a2[mt][1], a2[mt][2], a2[mt][3], b0, b1);
-            mma_f16(acc[mt][t + 1], a2[mt][0], a2[mt][1], a2[mt][2], a2[mt][3], b2, b3);
-          }
-        }
+      q0h = (item % p.n_qb) * QB + QH * half;
+      qmask = __ballot_sync(0xffffffffu, q0h + lane < p.Q);
+      bl = __ldcg(gb + q0h + lane);
+      bl_pf = bl;
+      __syncwarp();
+    };
+    // the tile sequence runs one page ahead: tile t+1 is expanded while the
+    // product of tile t runs, and tile t+2's words are in flight meanwhile
+    TileSeq ts;
+    bool have = ts.start(p, items);
+    Rec<D> r;
+    if (have) load_rec<D>(r, p.db + ts.page * p.page_bytes, p, row, half);
+    bool cur = false;
+    uint32_t n_cur = 0u;
+    long long page_cur = 0;
+    int item_cur = 0;
+    uint32_t t = 0;
+    auto build_next = [&](uint32_t buf) {
+      build_a_row<D>(r.kw, r.qw, r.gg, t_lane + (buf ? C::COL_A1 : C::COL_A0), half);
+      tc::wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_ab + 8 * buf);
+    };
+    if (have) {
+      build_next(0u);
+      cur = true;
+      n_cur = r.n;
+      page_cur = ts.page;
+      item_cur = ts.item;
+      have = ts.next(p, items);
+      if (have) load_rec<D>(r, p.db + ts.page * p.page_bytes, p, row, half);
+    }
+    while (cur) {
+      const bool nxt = have;
+      uint32_t n_nxt = 0u;
+      long long page_nxt = 0;
+      int item_nxt = 0;
+      if (nxt) {
+        build_next((t + 1) & 1u);
+        n_nxt = r.n;
+        page_nxt = ts.page;
+        item_nxt = ts.item;
+        have = ts.next(p, items);
+        if (have) load_rec<D>(r, p.db + ts.page * p.page_bytes, p, row, half);
       }
-      // QJL plane: k-steps 2KS .. 3KS-1
-#pragma unroll
-      for (int s = 0; s < C::KS; ++s) {
-        const int sh = qsb + 2 * s;
-        uint32_t a3[2][4];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          a3[mt][0] = ((qw[mt][0] << sh) & 0x80008000u) | gg[mt][0];
-          a3[mt][1] = ((qw[mt][1] << sh) & 0x80008000u) | gg[mt][1];
-          a3[mt][2] = ((qw[mt][0] << (sh + 1)) & 0x80008000u) | gg[mt][0];
-          a3[mt][3] = ((qw[mt][1] << (sh + 1)) & 0x80008000u) | gg[mt][1];
-        }
-#pragma unroll
-        for (int t = 0; t < C::NTQ; t += 2) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(b_base + t * 8 * C::RB + (2 * C::KS + s) * 32, b0, b1, b2, b3);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            mma_f16(acc[mt][t], a3[mt][0], a3[mt][1], a3[mt][2], a3[mt][3], b0, b1);
-            mma_f16(acc[mt][t + 1], a3[mt][0], a3[mt][1], a3[mt][2], a3[mt][3], b2, b3);
-          }
-        }
+      // scores of tile t: 32 queries x {hi, lo} of this warp's half
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_dfull, t & 1u));
+      if (!ok) {
+        failed = true;
+        break;
       }
-      // threshold filter, rare insertions (one candidate at a time per warp)
+      tc::fence_after_sync();
+      uint32_t v0[32], v1[32];
+      tc::ld32(t_lane + C::COL_D + 64 * half, v0);
+      tc::ld32(t_lane + C::COL_D + 64 * half + 32, v1);
+      tc::wait_ld();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_dfree);
+      if (item_cur != list_item) {
+        if (list_item >= 0) flush(list_item);
+        reset(item_cur);
+        list_item = item_cur;
+      }
+      const long long id64 = page_cur * PAGE + row;
+      const bool valid = id64 < p.N;
+      const int id = static_cast<int>(id64);
+      const float nf = __half2float(__ushort_as_half(static_cast<unsigned short>(n_cur)));
+      // bounds published by other lists, fetched one tile ahead
+      bl = max(bl, bl_pf);
+      bl_pf = __ldcg(gb + q0h + lane);
+      float sc[QH];
+      uint32_t cm = 0u;
 #pragma unroll
-      for (int t = 0; t < C::NTQ; ++t) {
+      for (int j = 0; j < QH; ++j) {
+        const uint32_t* v = j < QH / 2 ? v0 : v1;
+        const int c = 2 * (j % (QH / 2));
+        sc[j] = (__uint_as_float(v[c]) + __uint_as_float(v[c + 1])) * nf;
+        const float thr = unord_bits(__shfl_sync(0xffffffffu, bl, j));
+        if (sc[j] >= thr) cm |= 1u << j;
+      }
+      cm = valid ? (cm & qmask) : 0u;
+      const uint32_t anyq = __reduce_or_sync(0xffffffffu, cm);
+      if (anyq) {
+        // rare: the scores go through shared memory so that the insertions
+        // run as a rolled loop over (query, record) candidates
+        float* sb = sbuf + warp * 32 * SB_LD;
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const float s = (acc[mt][t][2 * r] + acc[mt][t][2 * r + 1]) * dq[t] * nn[mt][r];
-            const int id = ids[mt][r];
-            const bool valid = id < p.N && (q0 + 4 * t + c) < p.Q;
-            const bool cand = valid && better(s, id, thr_s[t], thr_i[t]);
-            unsigned mask = __ballot_sync(0xffffffffu, cand);
-            while (mask) {
-              const int src = __ffs(mask) - 1;
-              mask &= mask - 1;
-              const int qc = src & 3;  // query 4t + qc of the tile
-              if (lane == src) list_insert(ls + (4 * t + qc) * p.k, li + (4 * t + qc) * p.k, p.k, s, id);
-              __syncwarp();
-              if (c == qc) {
-                thr_s[t] = ls[(4 * t + qc) * p.k + p.k - 1];
-                thr_i[t] = li[(4 * t + qc) * p.k + p.k - 1];
+        for (int j = 0; j < QH; ++j) sb[lane * SB_LD + j] = sc[j];
+        __syncwarp();
+        const int id0 = id - lane;
+        uint32_t rem = anyq;
+        while (rem) {
+          const int j = __ffs(rem) - 1;
+          rem &= rem - 1;
+          unsigned m = __ballot_sync(0xffffffffu, (cm >> j) & 1u);
+          while (m) {
+            const int src = __ffs(m) - 1;
+            m &= m - 1;
+            float ts;
+            int ti;
+            warp_insert(ls + j * k, li + j * k, k, sb[src * SB_LD + j], id0 + src, ts, ti);
+            if (ti != 0x7fffffff) {
+              const uint32_t ob = ord_bits(ts);
+              if (lane == j && ob > bl) {
+                bl = ob;
+                atomicMax(p.gbound + q0h + j, ob);
               }
             }
           }
         }
+        __syncwarp();
       }
+      ++t;
+      cur = nxt;
+      n_cur = n_nxt;
+      page_cur = page_nxt;
+      item_cur = item_nxt;
     }
-    __syncwarp();
-    // per-warp lists -> global candidates of this item
-    const size_t base = (static_cast<size_t>(item) * NWARP + warp) * QT * p.k;
-    for (int i = lane; i < QT * p.k; i += 32) {
-      p.cand_s[base + i] = ls[i];
-      p.cand_i[base + i] = li[i];
+    if (!failed && list_item >= 0) {
+      __syncwarp();
+      flush(list_item);
     }
+    if (failed && lane == 0) s_failed = 1;
   }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == NEPI) tc::tmem_dealloc(tmem, C::TMEM_COLS);
+  if (tid == 0 && s_failed) report(p.err, TQ_ERR_TIMEOUT);
 }
 
-// per query: the best k among n_slices * NWARP lists of k candidates
+// per query: the best k among n_slices x 4 lists of k candidates (the four
+// warps of its query half, in every slice)
 __global__ void __launch_bounds__(128) merge_kernel(Params p, int32_t* out_ids, float* out_scores) {
   const int q = blockIdx.x;
-  const int qt = q / QT, qi = q % QT;
-  const int n_qt = (p.Q + QT - 1) / QT;
-  const int lists = p.n_slices * NWARP;
+  const int qb = q / QB, ql = q % QB, half = ql / QH, j = ql % QH;
+  const int lists = p.n_slices * 4;
   extern __shared__ uint8_t sm[];
   float* cs = reinterpret_cast<float*>(sm);
   int* ci = reinterpret_cast<int*>(sm + sizeof(float) * lists * p.k);
@@ -358,9 +590,9 @@ __global__ void __launch_bounds__(128) merge_kernel(Params p, int32_t* out_ids, 
   const int total = lists * p.k;
   for (int i = threadIdx.x; i < total; i += blockDim.x) {
     const int l = i / p.k, e = i % p.k;
-    const int sl = l / NWARP, w = l % NWARP;
-    const int item = sl * n_qt + qt;
-    const size_t src = ((static_cast<size_t>(item) * NWARP + w) * QT + qi) * p.k + e;
+    const int sl = l >> 2, w = 4 * half + (l & 3);
+    const int item = sl * p.n_qb + qb;
+    const size_t src = ((static_cast<size_t>(item) * NEPI + w) * QH + j) * p.k + e;
     cs[i] = p.cand_s[src];
     ci[i] = p.cand_i[src];
   }
@@ -411,34 +643,49 @@ __global__ void __launch_bounds__(128) merge_kernel(Params p, int32_t* out_ids, 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct Ws {
-  size_t bmat, desc, cs, ci, total;
+  size_t bimg, desc, gb, cs, ci, total;
 };
 
+// slices of the database per query block: at least four items per SM, and
+// among the counts up to four times that, the one that loads the SMs most
+// evenly (items a multiple of the SM count where one exists); never more
+// slices than pages, so that every item has a page
 inline int n_slices_for(const tq_ctx* ctx, int Q, long long pages) {
-  const int n_qt = (Q + QT - 1) / QT;
-  // enough items to fill every SM several times, slices of at least a few pages
-  long long want = (static_cast<long long>(ctx->num_sms) * 4 + n_qt - 1) / n_qt;
-  if (want < 1) want = 1;
-  if (want > pages) want = pages;
-  return static_cast<int>(want);
+  const long long n_qb = (Q + QB - 1) / QB, sms = ctx->num_sms > 0 ? ctx->num_sms : 1;
+  long long lo = (4 * sms + n_qb - 1) / n_qb;
+  if (lo < 1) lo = 1;
+  long long best = lo;
+  double best_eff = 0.0;
+  for (long long ns = lo; ns <= 4 * lo; ++ns) {
+    const long long items = n_qb * ns, waves = (items + sms - 1) / sms;
+    const double eff = static_cast<double>(items) / static_cast<double>(waves * sms);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = ns;
+    }
+  }
+  if (best > pages) best = pages;
+  return static_cast<int>(best < 1 ? 1 : best);
 }
 
 Ws ws_layout(const tq_ctx* ctx, int Q, long long N, int k) {
   const int d = ctx->cfg.head_dim;
   const long long pages = (N + TQ_PAGE_TOKENS - 1) / TQ_PAGE_TOKENS;
-  const int n_qt = (Q + QT - 1) / QT;
+  const int n_qb = (Q + QB - 1) / QB;
   const int ns = n_slices_for(ctx, Q, pages);
-  const size_t items = static_cast<size_t>(n_qt) * ns;
+  const size_t items = static_cast<size_t>(n_qb) * ns;
   Ws w;
   size_t off = 0;
-  w.bmat = off;
-  off = align256(off + sizeof(uint16_t) * static_cast<size_t>(n_qt) * QT * 2 * 3 * d);
+  w.bimg = off;
+  off = align256(off + sizeof(uint16_t) * static_cast<size_t>(n_qb) * NROW * 3 * d);
   w.desc = off;
-  off = align256(off + sizeof(float) * static_cast<size_t>(n_qt) * QT);
+  off = align256(off + sizeof(float) * static_cast<size_t>(n_qb) * QB);
+  w.gb = off;
+  off = align256(off + sizeof(uint32_t) * static_cast<size_t>(n_qb) * QB);
   w.cs = off;
-  off = align256(off + sizeof(float) * items * NWARP * QT * k);
+  off = align256(off + sizeof(float) * items * NEPI * QH * k);
   w.ci = off;
-  off = align256(off + sizeof(int) * items * NWARP * QT * k);
+  off = align256(off + sizeof(int) * items * NEPI * QH * k);
   w.total = off;
   return w;
 }
@@ -453,6 +700,7 @@ int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* d
                 int k, int32_t* out_ids, float* out_scores, void* ws, size_t ws_bytes,
                 void* stream) {
   const int d = ctx->cfg.head_dim;
+  if (ctx->cfg.qjl_dim != d) return TQ_ERR_UNSUPPORTED;
   const tk::Ws L = tk::ws_layout(ctx, Q, N, k);
   if (ws_bytes < L.total) return TQ_ERR_INVALID_ARG;
   const PageLayout pl = page_layout(d, ctx->cfg.qjl_dim, false);
@@ -468,41 +716,43 @@ int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* d
   p.off_kn = static_cast<int>(pl.kn);
   p.off_kg = static_cast<int>(pl.kg);
   p.rot = ctx->dev.rot;
-  p.qjl = ctx->dev.qjl;
+  p.sp = ctx->dev.sp;
   p.kc0 = ctx->cb.key_c[0];
   p.kc1 = ctx->cb.key_c[1];
   p.alpha = 1.2533141373155001f / static_cast<float>(ctx->cfg.qjl_dim);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  p.bmat = reinterpret_cast<uint16_t*>(base + L.bmat);
+  p.bimg = reinterpret_cast<uint16_t*>(base + L.bimg);
   p.desc = reinterpret_cast<float*>(base + L.desc);
+  p.gbound = reinterpret_cast<uint32_t*>(base + L.gb);
   p.cand_s = reinterpret_cast<float*>(base + L.cs);
   p.cand_i = reinterpret_cast<int*>(base + L.ci);
   p.pages = (N + TQ_PAGE_TOKENS - 1) / TQ_PAGE_TOKENS;
+  p.n_qb = (Q + tk::QB - 1) / tk::QB;
   p.n_slices = tk::n_slices_for(ctx, Q, p.pages);
   p.err = ctx->dev.err;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int n_qt = (Q + tk::QT - 1) / tk::QT;
-  const int items = n_qt * p.n_slices;
+  const int items = p.n_qb * p.n_slices;
   const int grid = items < ctx->num_sms ? items : ctx->num_sms;
-  const size_t merge_smem = static_cast<size_t>(p.n_slices) * tk::NWARP * k * 8;
+  const size_t merge_smem = static_cast<size_t>(p.n_slices) * 4 * k * 8;
   if (merge_smem > 200 * 1024) return TQ_ERR_UNSUPPORTED;
-  // queries of the last partial tile are read as zero rows by the scorer;
-  // the B matrix has room for whole tiles
   auto go = [&](auto dtag) -> int {
     constexpr int D = decltype(dtag)::value;
     using C = tk::Cfg<D>;
-    const size_t smem = C::SMEM_B + static_cast<size_t>(tk::NWARP) * tk::QT * k * 8;
-    static bool set = false;
-    if (!set) {
-      if (cudaFuncSetAttribute(tk::score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               232448) != cudaSuccess)
-        return TQ_ERR_CUDA;
-      set = true;
-    }
+    // B operand | lists | score staging | barriers, from a 1024-byte aligned base; at least
+    // 116 KB so that one CTA (and one 512-column TMEM allocation) sits on an SM
+    size_t smem = 1024 + C::B_BYTES + static_cast<size_t>(tk::NEPI) * tk::QH * k * 8 + tk::SB_BYTES + 64;
+    if (smem < 116 * 1024) smem = 116 * 1024;
     if (smem > 232448) return TQ_ERR_UNSUPPORTED;
-    tk::qprep_kernel<D><<<Q, 128, 0, st>>>(p);
+    static size_t smem_set = 0;
+    if (smem > smem_set) {
+      if (cudaFuncSetAttribute(tk::score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return TQ_ERR_CUDA;
+      smem_set = smem;
+    }
+    tk::qprep_kernel<D><<<p.n_qb * tk::QB, 128, 0, st>>>(p);
     if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
-    tk::score_kernel<D><<<grid, tk::NWARP * 32, smem, st>>>(p);
+    tk::score_kernel<D><<<grid, tk::NTHREADS, smem, st>>>(p);
     if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
     if (merge_smem > 48 * 1024 &&
         cudaFuncSetAttribute(tk::merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
