@@ -7,21 +7,25 @@
 // Launches:
 //  1. qprep   per query: q_rot, q_s, estimator constants folded in, per-query
 //             power-of-two prescale, fp16 hi/lo split, written into the
-//             tensor-core B operand of its 64-query block (K-major, 128-byte
+//             tensor-core B operand of its query block (K-major, 128-byte
 //             swizzle, rows = query x {hi, lo}).
-//  2. score   persistent CTAs over items = (64-query block, slice of database
+//  2. score   persistent CTAs over items = (query block, slice of database
 //             pages), one CTA per SM.  The block's B operand stays in shared
 //             memory for the item.  For each 128-record page, eight warps
-//             expand the packed codes into fp16 bit planes in tensor memory
-//             (A, lane = record: sign, sign*magnitude, QJL signs x gamma) while
-//             the previous page's product runs; a control warp issues one
-//             tcgen05.mma chain per page (M = 128 records, N = 64 queries x
-//             {hi, lo}, K = 3d) into a TMEM accumulator.  The eight warps read
-//             the scores back, and a threshold filter feeds rare insertions into
+//             expand the packed codes into fp16 planes in tensor memory (A,
+//             lane = record): the key plane +-b / +-a for magnitude index 0 / 1
+//             (a / b the fp16 ratio nearest kc1 / kc0; the query side carries
+//             kc0 / b), and the QJL plane +-gamma; meanwhile the previous
+//             page's product runs.  A control warp issues one tcgen05.mma chain
+//             per page (M = 128 records, N = queries x {hi, lo}, K = 2d) into a
+//             TMEM accumulator.  The eight warps read the scores back, and a
+//             filter against a per-query bound shared by all lists (the best
+//             k-th score any list has reached) feeds rare insertions into
 //             per-warp top-k lists in shared memory.
 //  3. merge   per query: the best k of all per-warp lists.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <type_traits>
 
@@ -34,12 +38,10 @@ namespace tk {
 
 constexpr int NEPI = 8;                    // epilogue warps: (TMEM lane quarter) x (query half)
 constexpr int NTHREADS = (NEPI + 1) * 32;  // + the control warp
-constexpr int QB = 64;                     // queries per block
-constexpr int NROW = 2 * QB;               // B rows: query x {hi, lo}
-constexpr int QH = QB / 2;                 // queries per epilogue warp
 constexpr int PAGE = TQ_PAGE_TOKENS;       // records per tile
-constexpr int SB_LD = QH + 1;              // score staging row (padded)
+constexpr int SB_LD = 33;                  // score staging row of 32 queries (padded)
 constexpr int SB_BYTES = NEPI * 32 * SB_LD * 4;
+constexpr int COL_A0 = 0, COL_A1 = 128, COL_D = 256, TMEM_COLS = 512;
 constexpr float NEG_INF = -__builtin_huge_valf();
 
 // float <-> unsigned with the same order (for atomicMax on scores)
@@ -52,16 +54,21 @@ __device__ __forceinline__ float unord_bits(uint32_t u) {
 }
 constexpr uint32_t ORD_NEG_INF = 0x007fffffu;
 
-template <int D>
+// D: head dimension (= sketch size m); QB: queries per block (64 or 128)
+template <int D, int QB>
 struct Cfg {
-  static constexpr int KTOT = 3 * D;              // sign plane, magnitude plane, QJL plane
+  static constexpr int NROW = 2 * QB;              // B rows = MMA N: query x {hi, lo}
+  static constexpr int WQ = QB / 2;                // queries per epilogue warp
+  static constexpr int NPASS = WQ / 32;            // 32-query passes per warp and page
+  static constexpr int KTOT = 2 * D;               // key plane, QJL plane
   static constexpr int B_BYTES = NROW * KTOT * 2;  // one block's B operand (SW128 image)
-  static constexpr int ACOLS = KTOT / 2;           // TMEM columns of one A buffer
-  static constexpr int COL_A0 = 0, COL_A1 = 192, COL_D = 384;
-  static constexpr int TMEM_COLS = 512;
-  static_assert(ACOLS <= 192, "A buffer");
-  // shared memory (from a 1024-byte aligned base): B | lists | barriers
-  static constexpr int OFF_B = 0;
+  static constexpr int NMMA = KTOT / 16;
+  static_assert(KTOT / 2 <= COL_A1 - COL_A0, "A buffer");
+  static_assert(NROW <= TMEM_COLS - COL_D, "accumulator");
+  // shared memory, from a 1024-byte aligned base: B | lists | score staging | barriers
+  static size_t smem_bytes(int k) {
+    return 1024 + static_cast<size_t>(B_BYTES) + static_cast<size_t>(NEPI) * WQ * k * 8 + SB_BYTES + 64;
+  }
 };
 
 struct Params {
@@ -73,31 +80,33 @@ struct Params {
   long long page_bytes;
   int off_kc, off_qs, off_kn, off_kg;
   const float* rot;
-  const float* sp;  // S Pi
-  float kc0, kc1, alpha;
-  uint16_t* bimg;   // [n_qb][NROW * KTOT] fp16 bits, SW128 image per block
-  float* desc;      // [n_qb * QB] descale
-  uint32_t* gbound;  // [n_qb * QB] best known lower bound of each query's k-th score (ordered bits)
-  float* cand_s;    // [items][NEPI][QH][k]
+  const float* sp;     // S Pi
+  float w_key, alpha;  // query weights of the key plane (kc0 / b) and of the QJL plane
+  uint32_t key_b2, key_diff;  // fp16 bits of b in both halves; bits(a) - bits(b)
+  uint16_t* bimg;      // [n_qb][NROW * KTOT] fp16 bits, SW128 image per block
+  float* desc;         // [n_qb * QB] descale
+  uint32_t* gslots;    // [n_qb * QB][k] per query: slot e holds the best score (ordered bits)
+                       // among the scored records with id = e mod k
+  float* cand_s;       // [items][NEPI][WQ][k]
   int* cand_i;
   int n_qb, n_slices;
   long long pages;
   int* err;
 };
 
-// K index k of the A operand (and so of B): plane, and the coordinate
-// (planes 0, 1) or sketch index (plane 2).  A record's A row holds, per plane,
-// two halves of D/4 TMEM columns; column c of a half covers two K elements
-// (low, high 16 bits):
-//   planes 0/1: c = 8 wl + 2 i + e -> coordinate 16 (half*D/32 + wl) + 2 i + e (+ 8 high)
-//   plane 2:    c = 16 wl + r      -> sketch index 32 (half*D/64 + wl) + r (+ 16 high)
+// K index k of the A operand (and so of B): plane (0 key, 1 QJL) and the
+// coordinate or sketch index.  A record's A row holds, per plane, two halves
+// of D/4 TMEM columns; column c of a half covers two K elements (low, high
+// 16 bits):
+//   key plane: c = 8 wl + 2 i + e -> coordinate 16 (half*D/32 + wl) + 2 i + e (+ 8 high)
+//   QJL plane: c = 16 wl + r      -> sketch index 32 (half*D/64 + wl) + r (+ 16 high)
 template <int D>
 __host__ __device__ __forceinline__ void k_index(int k, int& plane, int& idx) {
   const int col = k >> 1, hiword = k & 1;
   plane = col / (D / 2);
   const int c = col % (D / 2);
   const int half = c / (D / 4), l = c % (D / 4);
-  if (plane < 2) {
+  if (plane == 0) {
     const int wl = l >> 3, i = (l & 7) >> 1, e = l & 1;
     idx = 16 * (half * (D / 32) + wl) + 2 * i + e + 8 * hiword;
   } else {
@@ -133,9 +142,9 @@ __device__ __forceinline__ void warp_matvec2(const float* __restrict__ M1, const
 }
 
 // one CTA per query slot of the padded blocks; slots past Q write zero rows
-template <int D>
+template <int D, int QB>
 __global__ void __launch_bounds__(128) qprep_kernel(Params p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, QB>;
   const int q = blockIdx.x, qb = q / QB, ql = q % QB;
   __shared__ float sq[D], sr[D], ss[D];
   __shared__ unsigned smax;
@@ -146,11 +155,9 @@ __global__ void __launch_bounds__(128) qprep_kernel(Params p) {
     for (int k0 = tid * 8; k0 < C::KTOT; k0 += blockDim.x * 8)
 #pragma unroll
       for (int part = 0; part < 2; ++part)
-        *reinterpret_cast<uint4*>(img + tc::sw128_offset(2 * ql + part, k0, NROW)) = make_uint4(0, 0, 0, 0);
-    if (tid == 0) {
-      p.desc[q] = 0.0f;
-      p.gbound[q] = ORD_NEG_INF;
-    }
+        *reinterpret_cast<uint4*>(img + tc::sw128_offset(2 * ql + part, k0, C::NROW)) = make_uint4(0, 0, 0, 0);
+    if (tid == 0) p.desc[q] = 0.0f;
+    for (int e = tid; e < p.k; e += blockDim.x) p.gslots[static_cast<size_t>(q) * p.k + e] = ORD_NEG_INF;
     return;
   }
   if (tid == 0) smax = 0u;
@@ -158,9 +165,9 @@ __global__ void __launch_bounds__(128) qprep_kernel(Params p) {
   __syncthreads();
   warp_matvec2<D>(p.rot, p.sp, sq, sr, ss);  // q_rot = Pi q, q_s = (S Pi) q
   __syncthreads();
-  const float w1 = p.kc0, w2 = 128.0f * (p.kc1 - p.kc0), w3 = p.alpha;
+  const float w1 = p.w_key, w3 = p.alpha;
   for (int j = tid; j < D; j += blockDim.x) {
-    const float m = fmaxf(fmaxf(fabsf(w1 * sr[j]), fabsf(w2 * sr[j])), fabsf(w3 * ss[j]));
+    const float m = fmaxf(fabsf(w1 * sr[j]), fabsf(w3 * ss[j]));
     atomicMax(&smax, __float_as_uint(m));
   }
   __syncthreads();
@@ -174,8 +181,8 @@ __global__ void __launch_bounds__(128) qprep_kernel(Params p) {
     }
     sfac = f;
     p.desc[q] = 1.0f / f;
-    p.gbound[q] = ORD_NEG_INF;
   }
+  for (int e = tid; e < p.k; e += blockDim.x) p.gslots[static_cast<size_t>(q) * p.k + e] = ORD_NEG_INF;
   __syncthreads();
   const float f = sfac;
   // 16-byte chunks of 8 K elements, hi and lo rows
@@ -185,21 +192,20 @@ __global__ void __launch_bounds__(128) qprep_kernel(Params p) {
     for (int e = 0; e < 8; ++e) {
       int plane, idx;
       k_index<D>(k0 + e, plane, idx);
-      const float w = plane == 0 ? w1 * sr[idx] : plane == 1 ? w2 * sr[idx] : w3 * ss[idx];
+      const float w = plane == 0 ? w1 * sr[idx] : w3 * ss[idx];
       uint16_t hi, lo;
       split_f16(f * w, hi, lo);
       wh[e >> 1] |= static_cast<uint32_t>(hi) << (16 * (e & 1));
       wl[e >> 1] |= static_cast<uint32_t>(lo) << (16 * (e & 1));
     }
-    *reinterpret_cast<uint4*>(img + tc::sw128_offset(2 * ql, k0, NROW)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-    *reinterpret_cast<uint4*>(img + tc::sw128_offset(2 * ql + 1, k0, NROW)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+    *reinterpret_cast<uint4*>(img + tc::sw128_offset(2 * ql, k0, C::NROW)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    *reinterpret_cast<uint4*>(img + tc::sw128_offset(2 * ql + 1, k0, C::NROW)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
   }
 }
 
 __device__ __forceinline__ bool better(float sa, int ia, float sb, int ib) {
   return sa > sb || (sa == sb && ia < ib);
 }
-
 // Insert (cs, ci) into the sorted (best first) list of k <= 32 entries, the
 // whole warp at once: lane e holds entry e, the rank of the candidate is the
 // number of entries ahead of it, the entries behind it move down one lane.
@@ -231,6 +237,48 @@ __device__ __forceinline__ void warp_insert(float* ls, int* li, int k, float cs,
   __syncwarp();
 }
 
+// compare-exchange with the lane `mask` away: keep the better (or the worse)
+// of the two entries
+__device__ __forceinline__ void cmpx(float& s, int& i, int mask, bool keep_better) {
+  const float os = __shfl_xor_sync(0xffffffffu, s, mask);
+  const int oi = __shfl_xor_sync(0xffffffffu, i, mask);
+  if (better(os, oi, s, i) == keep_better) {
+    s = os;
+    i = oi;
+  }
+}
+
+// Merge a batch of up to 32 candidates (one per lane; (-inf, 0x7fffffff) for
+// none) into the sorted list of k <= 32 entries: bitonic sort of the batch,
+// elementwise better of the sorted batch and the reversed list (the best 32
+// of both, a bitonic sequence), bitonic merge; the first k are the list.
+// Returns the list's k-th entry in (ts, ti).
+__device__ __forceinline__ void warp_merge_batch(float* ls, int* li, int k, float s, int i, float& ts, int& ti) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1)
+      cmpx(s, i, stride, ((lane & stride) == 0) == ((lane & size) == 0));
+  const float es = lane < k ? ls[lane] : NEG_INF;
+  const int ei = lane < k ? li[lane] : 0x7fffffff;
+  const float rs = __shfl_sync(0xffffffffu, es, 31 - lane);
+  const int ri = __shfl_sync(0xffffffffu, ei, 31 - lane);
+  if (better(rs, ri, s, i)) {
+    s = rs;
+    i = ri;
+  }
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) cmpx(s, i, stride, (lane & stride) == 0);
+  if (lane < k) {
+    ls[lane] = s;
+    li[lane] = i;
+  }
+  ts = __shfl_sync(0xffffffffu, s, k - 1);
+  ti = __shfl_sync(0xffffffffu, i, k - 1);
+  __syncwarp();
+}
+
 template <int N>
 __device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t* r) {
   if constexpr (N == 32) tc::st32(taddr, r);
@@ -239,31 +287,29 @@ __device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t* r) {
 }
 
 // A row of one record (this thread's half of the coordinates), from its
-// packed words: sign plane (+-1), sign*magnitude plane (+-2^-7), QJL plane
-// (+-gamma).  Key code word w holds coordinates 16 w + 8 h + 2 i + e with the
-// sign bit at 16 h + 15 - 4 i - e and the magnitude bit two below; QJL word
-// w holds sketch index 32 w + 16 h + r at bit 16 h + 15 - r.
+// packed words: the key plane (sign, magnitude index -> +-b, +-a) and the QJL
+// plane (+-gamma).  Key code word w holds coordinates 16 w + 8 h + 2 i + e
+// with the sign bit at 16 h + 15 - 4 i - e and the magnitude bit two below;
+// QJL word w holds sketch index 32 w + 16 h + r at bit 16 h + 15 - r.
 template <int D>
 __device__ __forceinline__ void build_a_row(const uint32_t* kw, const uint32_t* qw, uint32_t gg,
-                                            uint32_t base, int half) {
+                                            uint32_t base, int half, uint32_t key_b2, uint32_t key_diff) {
   constexpr int NW = D / 32;  // key words of one half
   uint32_t a[D / 4];
 #pragma unroll
   for (int wl = 0; wl < NW; ++wl)
 #pragma unroll
-    for (int s = 0; s < 8; ++s)
-      a[wl * 8 + s] = ((kw[wl] << ((s >> 1) * 4 + (s & 1))) & 0x80008000u) | 0x3C003C00u;
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t x = kw[wl] << ((s >> 1) * 4 + (s & 1));
+      const uint32_t m = (x >> 13) & 0x00010001u;  // magnitude bits -> bit 0 / bit 16
+      a[wl * 8 + s] = (x & 0x80008000u) | (m * key_diff + key_b2);
+    }
   tmem_store<D / 4>(base + half * (D / 4), a);
-#pragma unroll
-  for (int wl = 0; wl < NW; ++wl)
-#pragma unroll
-    for (int s = 0; s < 8; ++s) a[wl * 8 + s] = (kw[wl] << ((s >> 1) * 4 + (s & 1))) & 0xA000A000u;
-  tmem_store<D / 4>(base + D / 2 + half * (D / 4), a);
 #pragma unroll
   for (int wl = 0; wl < D / 64; ++wl)
 #pragma unroll
     for (int r = 0; r < 16; ++r) a[wl * 16 + r] = ((qw[wl] << r) & 0x80008000u) | gg;
-  tmem_store<D / 4>(base + D + half * (D / 4), a);
+  tmem_store<D / 4>(base + D / 2 + half * (D / 4), a);
 }
 
 // the packed words of one record half, gamma and norm
@@ -324,18 +370,18 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-template <int D>
+template <int D, int QB>
 __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
-  using C = Cfg<D>;
-  constexpr int NMMA = C::KTOT / 16;
+  using C = Cfg<D, QB>;
+  constexpr int WQ = C::WQ;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int k = p.k;
   float* ls_all = reinterpret_cast<float*>(smem + C::B_BYTES);
-  int* li_all = reinterpret_cast<int*>(smem + C::B_BYTES + NEPI * QH * k * 4);
-  float* sbuf = reinterpret_cast<float*>(smem + C::B_BYTES + NEPI * QH * k * 8);
-  uint8_t* bars = smem + C::B_BYTES + NEPI * QH * k * 8 + SB_BYTES;
+  int* li_all = reinterpret_cast<int*>(smem + C::B_BYTES + NEPI * WQ * k * 4);
+  float* sbuf = reinterpret_cast<float*>(smem + C::B_BYTES + NEPI * WQ * k * 8);
+  uint8_t* bars = smem + C::B_BYTES + NEPI * WQ * k * 8 + SB_BYTES;
   const uint32_t bar_ab = smem_u32(bars), bar_dfull = bar_ab + 16, bar_dfree = bar_ab + 24;
   const uint32_t bar_bfull = bar_ab + 32, bar_bfree = bar_ab + 40, bar_drain = bar_ab + 48;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 56);
@@ -354,7 +400,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
     mbar_init_fence();
   }
   if (warp == NEPI) {
-    tc::tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tc::tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
@@ -366,7 +412,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
   if (warp == NEPI) {
     // ---- control: B operand per item, one MMA chain per page ------------------
     if (lane == 0) {
-      constexpr uint32_t idesc = tc::idesc_f16(128, NROW, false);
+      constexpr uint32_t idesc = tc::idesc_f16(128, C::NROW, false);
       const uint32_t s_b = smem_u32(smem);
       TileSeq ts;
       bool more = ts.start(p, items);
@@ -388,11 +434,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
           if (!mbar_wait_bounded(bar_ab + 8 * (t & 1), (t >> 1) & 1)) { failed = true; break; }
           if (t > 0 && !mbar_wait_bounded(bar_dfree, (t - 1) & 1)) { failed = true; break; }
           tc::fence_after_sync();
-          const uint32_t a = tmem + (t & 1 ? C::COL_A1 : C::COL_A0);
+          const uint32_t a = tmem + (t & 1 ? COL_A1 : COL_A0);
 #pragma unroll
-          for (int s = 0; s < NMMA; ++s)
-            tc::mma_f16_tmem_a(tmem + C::COL_D, a + 8 * s,
-                               tc::sdesc_sw128(s_b + (s >> 2) * (NROW * 128) + (s & 3) * 32), idesc, s > 0);
+          for (int s = 0; s < C::NMMA; ++s)
+            tc::mma_f16_tmem_a(tmem + COL_D, a + 8 * s,
+                               tc::sdesc_sw128(s_b + (s >> 2) * (C::NROW * 128) + (s & 3) * 32), idesc, s > 0);
           tc::commit(bar_dfull);
           ++t;
           more = ts.next(p, items);
@@ -418,36 +464,47 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
     const int qr = warp & 3, half = warp >> 2;
     const int row = 32 * qr + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * qr) << 16);
-    float* ls = ls_all + warp * QH * k;
-    int* li = li_all + warp * QH * k;
-    // lists hold scores before the per-query power-of-two descale (the order
-    // is the same); the descale is applied when a list is written out
-    uint32_t qmask = 0u;
-    int list_item = -1;
-    // lane j: the bound on query j's k-th score (ordered bits): the best
-    // k-th score of any list of this query, in any CTA, seen so far; a record
-    // below it cannot be among the query's k best
-    uint32_t bl = ORD_NEG_INF, bl_pf = ORD_NEG_INF;
-    const uint32_t* gb = p.gbound;
-    int q0h = 0;
+    float* ls = ls_all + warp * WQ * k;
+    int* li = li_all + warp * WQ * k;
+    float* sb = sbuf + warp * 32 * SB_LD;
+    // per 32-query pass: valid-query mask, and in lane j a lower bound on
+    // query j's k-th best score (ordered bits), below which a record cannot
+    // be among the k best: the k-th entry of this warp's list, or the least
+    // of the query's k slots (k distinct records' scores).  The slots are
+    // read one per page, one page ahead (sf, slot se); their running minimum
+    // (cmin) becomes a bound when a round of k slots is complete (slots only
+    // grow, so values read at different times still bound the k-th score).
+    uint32_t qmask[C::NPASS], bl[C::NPASS], cmin[C::NPASS], sf[C::NPASS];
+    int list_item = -1, q0h = 0, se = 0;
     auto flush = [&](int item) {
-      const size_t base = (static_cast<size_t>(item) * NEPI + warp) * QH * k;
-      const float* dq = p.desc + (item % p.n_qb) * QB + QH * half;
-      for (int i = lane; i < QH * k; i += 32) {
+      const size_t base = (static_cast<size_t>(item) * NEPI + warp) * WQ * k;
+      const float* dq = p.desc + (item % p.n_qb) * QB + WQ * half;
+      // lists hold scores before the per-query power-of-two descale (the
+      // order is the same); the descale is applied here
+      for (int i = lane; i < WQ * k; i += 32) {
         p.cand_s[base + i] = ls[i] * __ldg(dq + i / k);
         p.cand_i[base + i] = li[i];
       }
     };
     auto reset = [&](int item) {
       __syncwarp();
-      for (int i = lane; i < QH * k; i += 32) {
+      for (int i = lane; i < WQ * k; i += 32) {
         ls[i] = NEG_INF;
         li[i] = 0x7fffffff;
       }
-      q0h = (item % p.n_qb) * QB + QH * half;
-      qmask = __ballot_sync(0xffffffffu, q0h + lane < p.Q);
-      bl = __ldcg(gb + q0h + lane);
-      bl_pf = bl;
+      q0h = (item % p.n_qb) * QB + WQ * half;
+#pragma unroll
+      for (int ps = 0; ps < C::NPASS; ++ps) {
+        qmask[ps] = __ballot_sync(0xffffffffu, q0h + 32 * ps + lane < p.Q);
+        const uint32_t* sl = p.gslots + static_cast<size_t>(q0h + 32 * ps + lane) * k;
+        uint32_t mn = 0xffffffffu;
+#pragma unroll 4
+        for (int e = 0; e < k; ++e) mn = min(mn, __ldcg(sl + e));
+        bl[ps] = mn;
+        cmin[ps] = 0xffffffffu;
+        sf[ps] = __ldcg(sl);
+      }
+      se = 0;
       __syncwarp();
     };
     // the tile sequence runs one page ahead: tile t+1 is expanded while the
@@ -462,7 +519,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
     int item_cur = 0;
     uint32_t t = 0;
     auto build_next = [&](uint32_t buf) {
-      build_a_row<D>(r.kw, r.qw, r.gg, t_lane + (buf ? C::COL_A1 : C::COL_A0), half);
+      build_a_row<D>(r.kw, r.qw, r.gg, t_lane + (buf ? COL_A1 : COL_A0), half, p.key_b2, p.key_diff);
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
@@ -490,20 +547,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
         have = ts.next(p, items);
         if (have) load_rec<D>(r, p.db + ts.page * p.page_bytes, p, row, half);
       }
-      // scores of tile t: 32 queries x {hi, lo} of this warp's half
       const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_dfull, t & 1u));
       if (!ok) {
         failed = true;
         break;
       }
       tc::fence_after_sync();
-      uint32_t v0[32], v1[32];
-      tc::ld32(t_lane + C::COL_D + 64 * half, v0);
-      tc::ld32(t_lane + C::COL_D + 64 * half + 32, v1);
-      tc::wait_ld();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_dfree);
       if (item_cur != list_item) {
         if (list_item >= 0) flush(list_item);
         reset(item_cur);
@@ -511,53 +560,82 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
       }
       const long long id64 = page_cur * PAGE + row;
       const bool valid = id64 < p.N;
-      const int id = static_cast<int>(id64);
+      const int id0 = static_cast<int>(page_cur * PAGE + 32 * qr);
       const float nf = __half2float(__ushort_as_half(static_cast<unsigned short>(n_cur)));
-      // bounds published by other lists, fetched one tile ahead
-      bl = max(bl, bl_pf);
-      bl_pf = __ldcg(gb + q0h + lane);
-      float sc[QH];
-      uint32_t cm = 0u;
+      // scores of this warp's queries (32 per pass) x {hi, lo}; the
+      // accumulator is released as soon as it is read
+      float sc[C::NPASS][32];
 #pragma unroll
-      for (int j = 0; j < QH; ++j) {
-        const uint32_t* v = j < QH / 2 ? v0 : v1;
-        const int c = 2 * (j % (QH / 2));
-        sc[j] = (__uint_as_float(v[c]) + __uint_as_float(v[c + 1])) * nf;
-        const float thr = unord_bits(__shfl_sync(0xffffffffu, bl, j));
-        if (sc[j] >= thr) cm |= 1u << j;
+      for (int ps = 0; ps < C::NPASS; ++ps) {
+        uint32_t v0[32], v1[32];
+        const uint32_t col = COL_D + 2 * WQ * half + 64 * ps;
+        tc::ld32(t_lane + col, v0);
+        tc::ld32(t_lane + col + 32, v1);
+        tc::wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const uint32_t* v = j < 16 ? v0 : v1;
+          const int c = 2 * (j % 16);
+          sc[ps][j] = (__uint_as_float(v[c]) + __uint_as_float(v[c + 1])) * nf;
+        }
       }
-      cm = valid ? (cm & qmask) : 0u;
-      const uint32_t anyq = __reduce_or_sync(0xffffffffu, cm);
-      if (anyq) {
-        // rare: the scores go through shared memory so that the insertions
-        // run as a rolled loop over (query, record) candidates
-        float* sb = sbuf + warp * 32 * SB_LD;
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_dfree);
 #pragma unroll
-        for (int j = 0; j < QH; ++j) sb[lane * SB_LD + j] = sc[j];
-        __syncwarp();
-        const int id0 = id - lane;
-        uint32_t rem = anyq;
-        while (rem) {
-          const int j = __ffs(rem) - 1;
-          rem &= rem - 1;
-          unsigned m = __ballot_sync(0xffffffffu, (cm >> j) & 1u);
-          while (m) {
-            const int src = __ffs(m) - 1;
-            m &= m - 1;
-            float ts;
-            int ti;
-            warp_insert(ls + j * k, li + j * k, k, sb[src * SB_LD + j], id0 + src, ts, ti);
-            if (ti != 0x7fffffff) {
-              const uint32_t ob = ord_bits(ts);
-              if (lane == j && ob > bl) {
-                bl = ob;
-                atomicMax(p.gbound + q0h + j, ob);
+      for (int ps = 0; ps < C::NPASS; ++ps) {
+        // slot se of this lane's query, read one page ago
+        cmin[ps] = min(cmin[ps], sf[ps]);
+        if (se == k - 1) {
+          bl[ps] = max(bl[ps], cmin[ps]);
+          cmin[ps] = 0xffffffffu;
+        }
+        sf[ps] = __ldcg(p.gslots + static_cast<size_t>(q0h + 32 * ps + lane) * k + (se == k - 1 ? 0 : se + 1));
+        const float blf = unord_bits(bl[ps]);
+        uint32_t cm = 0u;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (sc[ps][j] >= __shfl_sync(0xffffffffu, blf, j)) cm |= 1u << j;
+        cm = valid ? (cm & qmask[ps]) : 0u;
+        const uint32_t anyq = __reduce_or_sync(0xffffffffu, cm);
+        if (anyq) {
+          // rare: the scores go through shared memory so that the insertions
+          // run as a rolled loop over (query, record) candidates
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sb[lane * SB_LD + j] = sc[ps][j];
+          __syncwarp();
+          uint32_t rem = anyq;
+          while (rem) {
+            const int j = __ffs(rem) - 1;
+            rem &= rem - 1;
+            const int jq = 32 * ps + j;
+            const bool mine = (cm >> j) & 1u;
+            unsigned m = __ballot_sync(0xffffffffu, mine);
+            // every candidate raises its slot
+            if (mine)
+              atomicMax(p.gslots + static_cast<size_t>(q0h + jq) * k + (id0 + lane) % k,
+                        ord_bits(sb[lane * SB_LD + j]));
+            float ts2 = NEG_INF;
+            int ti = 0x7fffffff;
+            if (__popc(m) >= 6) {
+              warp_merge_batch(ls + jq * k, li + jq * k, k, mine ? sb[lane * SB_LD + j] : NEG_INF,
+                               mine ? id0 + lane : 0x7fffffff, ts2, ti);
+            } else {
+              while (m) {
+                const int src = __ffs(m) - 1;
+                m &= m - 1;
+                warp_insert(ls + jq * k, li + jq * k, k, sb[src * SB_LD + j], id0 + src, ts2, ti);
               }
             }
+            if (ti != 0x7fffffff) {
+              const uint32_t ob = ord_bits(ts2);
+              if (lane == j) bl[ps] = max(bl[ps], ob);
+            }
           }
+          __syncwarp();
         }
-        __syncwarp();
       }
+      se = se == k - 1 ? 0 : se + 1;
       ++t;
       cur = nxt;
       n_cur = n_nxt;
@@ -572,15 +650,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == NEPI) tc::tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == NEPI) tc::tmem_dealloc(tmem, TMEM_COLS);
   if (tid == 0 && s_failed) report(p.err, TQ_ERR_TIMEOUT);
 }
 
 // per query: the best k among n_slices x 4 lists of k candidates (the four
 // warps of its query half, in every slice)
+template <int QB>
 __global__ void __launch_bounds__(128) merge_kernel(Params p, int32_t* out_ids, float* out_scores) {
+  constexpr int WQ = QB / 2;
   const int q = blockIdx.x;
-  const int qb = q / QB, ql = q % QB, half = ql / QH, j = ql % QH;
+  const int qb = q / QB, ql = q % QB, half = ql / WQ, j = ql % WQ;
   const int lists = p.n_slices * 4;
   extern __shared__ uint8_t sm[];
   float* cs = reinterpret_cast<float*>(sm);
@@ -592,7 +672,7 @@ __global__ void __launch_bounds__(128) merge_kernel(Params p, int32_t* out_ids, 
     const int l = i / p.k, e = i % p.k;
     const int sl = l >> 2, w = 4 * half + (l & 3);
     const int item = sl * p.n_qb + qb;
-    const size_t src = ((static_cast<size_t>(item) * NEPI + w) * QH + j) * p.k + e;
+    const size_t src = ((static_cast<size_t>(item) * NEPI + w) * WQ + j) * p.k + e;
     cs[i] = p.cand_s[src];
     ci[i] = p.cand_i[src];
   }
@@ -642,6 +722,10 @@ __global__ void __launch_bounds__(128) merge_kernel(Params p, int32_t* out_ids, 
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// queries per block: 128 (MMA N = 256) while the per-warp lists of 64
+// queries fit in shared memory beside the 2 x 128-row B operand, else 64
+inline int qb_for(int k) { return k <= 16 ? 128 : 64; }
+
 struct Ws {
   size_t bimg, desc, gb, cs, ci, total;
 };
@@ -650,8 +734,8 @@ struct Ws {
 // among the counts up to four times that, the one that loads the SMs most
 // evenly (items a multiple of the SM count where one exists); never more
 // slices than pages, so that every item has a page
-inline int n_slices_for(const tq_ctx* ctx, int Q, long long pages) {
-  const long long n_qb = (Q + QB - 1) / QB, sms = ctx->num_sms > 0 ? ctx->num_sms : 1;
+inline int n_slices_for(const tq_ctx* ctx, int Q, int qb, long long pages) {
+  const long long n_qb = (Q + qb - 1) / qb, sms = ctx->num_sms > 0 ? ctx->num_sms : 1;
   long long lo = (4 * sms + n_qb - 1) / n_qb;
   if (lo < 1) lo = 1;
   long long best = lo;
@@ -669,25 +753,59 @@ inline int n_slices_for(const tq_ctx* ctx, int Q, long long pages) {
 }
 
 Ws ws_layout(const tq_ctx* ctx, int Q, long long N, int k) {
-  const int d = ctx->cfg.head_dim;
+  const int d = ctx->cfg.head_dim, qb = qb_for(k);
   const long long pages = (N + TQ_PAGE_TOKENS - 1) / TQ_PAGE_TOKENS;
-  const int n_qb = (Q + QB - 1) / QB;
-  const int ns = n_slices_for(ctx, Q, pages);
+  const int n_qb = (Q + qb - 1) / qb;
+  const int ns = n_slices_for(ctx, Q, qb, pages);
   const size_t items = static_cast<size_t>(n_qb) * ns;
   Ws w;
   size_t off = 0;
   w.bimg = off;
-  off = align256(off + sizeof(uint16_t) * static_cast<size_t>(n_qb) * NROW * 3 * d);
+  off = align256(off + sizeof(uint16_t) * static_cast<size_t>(n_qb) * (2 * qb) * (2 * d));
   w.desc = off;
-  off = align256(off + sizeof(float) * static_cast<size_t>(n_qb) * QB);
+  off = align256(off + sizeof(float) * static_cast<size_t>(n_qb) * qb);
   w.gb = off;
-  off = align256(off + sizeof(uint32_t) * static_cast<size_t>(n_qb) * QB);
+  off = align256(off + sizeof(uint32_t) * static_cast<size_t>(n_qb) * qb * k);
   w.cs = off;
-  off = align256(off + sizeof(float) * items * NEPI * QH * k);
+  off = align256(off + sizeof(float) * items * NEPI * (qb / 2) * k);
   w.ci = off;
-  off = align256(off + sizeof(int) * items * NEPI * QH * k);
+  off = align256(off + sizeof(int) * items * NEPI * (qb / 2) * k);
   w.total = off;
   return w;
+}
+
+// fp16 bits of a positive value with at most 11 significant bits in the
+// normal range
+inline uint32_t f16_bits_exact(double v) {
+  const int e = static_cast<int>(std::floor(std::log2(v)));
+  const double mant = v / std::ldexp(1.0, e) - 1.0;
+  return (static_cast<uint32_t>(e + 15) << 10) | static_cast<uint32_t>(std::lround(mant * 1024.0));
+}
+
+// the key plane's two magnitudes: fp16 values b (index 0) and a (index 1)
+// whose ratio a / b is the nearest of all ratios of 11-bit integers (times a
+// power of two) to kc1 / kc0; b is scaled into [1, 2).  Returns the
+// relative error of a / b.
+inline double key_plane_values(double kc0, double kc1, double& a, double& b) {
+  const double r = kc1 / kc0;
+  double best = -1.0;
+  a = r;
+  b = 1.0;
+  for (int sh = -3; sh <= 3; ++sh) {
+    const double t = std::ldexp(r, -sh);
+    for (int qd = 1; qd < 2048; ++qd) {
+      const double pn = std::nearbyint(qd * t);
+      if (pn < 1.0 || pn > 2047.0) continue;
+      const double err = std::fabs(std::ldexp(pn / qd, sh) - r);
+      if (best < 0.0 || err < best) {
+        best = err;
+        const double sc = std::ldexp(1.0, -static_cast<int>(std::floor(std::log2(static_cast<double>(qd)))));
+        b = qd * sc;
+        a = std::ldexp(pn, sh) * sc;
+      }
+    }
+  }
+  return best / r;
 }
 
 }  // namespace tk
@@ -704,6 +822,7 @@ int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* d
   const tk::Ws L = tk::ws_layout(ctx, Q, N, k);
   if (ws_bytes < L.total) return TQ_ERR_INVALID_ARG;
   const PageLayout pl = page_layout(d, ctx->cfg.qjl_dim, false);
+  const int qb = tk::qb_for(k);
   tk::Params p{};
   p.queries = queries;
   p.Q = Q;
@@ -717,52 +836,61 @@ int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* d
   p.off_kg = static_cast<int>(pl.kg);
   p.rot = ctx->dev.rot;
   p.sp = ctx->dev.sp;
-  p.kc0 = ctx->cb.key_c[0];
-  p.kc1 = ctx->cb.key_c[1];
+  // the key plane's centroid ratio is carried to better than 2^-19
+  double ka, kb;
+  if (!(tk::key_plane_values(ctx->cb.key_c[0], ctx->cb.key_c[1], ka, kb) <= 0x1p-19))
+    return TQ_ERR_UNSUPPORTED;
+  const uint32_t bits_a = tk::f16_bits_exact(ka), bits_b = tk::f16_bits_exact(kb);
+  if (!(ka > kb) || bits_a >= 0x7C00u) return TQ_ERR_UNSUPPORTED;
+  p.w_key = static_cast<float>(ctx->cb.key_c[0] / kb);
+  p.key_b2 = bits_b * 0x10001u;
+  p.key_diff = bits_a - bits_b;
   p.alpha = 1.2533141373155001f / static_cast<float>(ctx->cfg.qjl_dim);
   uint8_t* base = static_cast<uint8_t*>(ws);
   p.bimg = reinterpret_cast<uint16_t*>(base + L.bimg);
   p.desc = reinterpret_cast<float*>(base + L.desc);
-  p.gbound = reinterpret_cast<uint32_t*>(base + L.gb);
+  p.gslots = reinterpret_cast<uint32_t*>(base + L.gb);
   p.cand_s = reinterpret_cast<float*>(base + L.cs);
   p.cand_i = reinterpret_cast<int*>(base + L.ci);
   p.pages = (N + TQ_PAGE_TOKENS - 1) / TQ_PAGE_TOKENS;
-  p.n_qb = (Q + tk::QB - 1) / tk::QB;
-  p.n_slices = tk::n_slices_for(ctx, Q, p.pages);
+  p.n_qb = (Q + qb - 1) / qb;
+  p.n_slices = tk::n_slices_for(ctx, Q, qb, p.pages);
   p.err = ctx->dev.err;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int items = p.n_qb * p.n_slices;
   const int grid = items < ctx->num_sms ? items : ctx->num_sms;
   const size_t merge_smem = static_cast<size_t>(p.n_slices) * 4 * k * 8;
   if (merge_smem > 200 * 1024) return TQ_ERR_UNSUPPORTED;
-  auto go = [&](auto dtag) -> int {
-    constexpr int D = decltype(dtag)::value;
-    using C = tk::Cfg<D>;
-    // B operand | lists | score staging | barriers, from a 1024-byte aligned base; at least
-    // 116 KB so that one CTA (and one 512-column TMEM allocation) sits on an SM
-    size_t smem = 1024 + C::B_BYTES + static_cast<size_t>(tk::NEPI) * tk::QH * k * 8 + tk::SB_BYTES + 64;
+  auto go = [&](auto dtag, auto qtag) -> int {
+    constexpr int D = decltype(dtag)::value, QB = decltype(qtag)::value;
+    using C = tk::Cfg<D, QB>;
+    // at least 116 KB, so that one CTA (and one 512-column TMEM allocation)
+    // sits on an SM
+    size_t smem = C::smem_bytes(k);
     if (smem < 116 * 1024) smem = 116 * 1024;
     if (smem > 232448) return TQ_ERR_UNSUPPORTED;
     static size_t smem_set = 0;
     if (smem > smem_set) {
-      if (cudaFuncSetAttribute(tk::score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(tk::score_kernel<D, QB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem)) != cudaSuccess)
         return TQ_ERR_CUDA;
       smem_set = smem;
     }
-    tk::qprep_kernel<D><<<p.n_qb * tk::QB, 128, 0, st>>>(p);
+    tk::qprep_kernel<D, QB><<<p.n_qb * QB, 128, 0, st>>>(p);
     if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
-    tk::score_kernel<D><<<grid, tk::NTHREADS, smem, st>>>(p);
+    tk::score_kernel<D, QB><<<grid, tk::NTHREADS, smem, st>>>(p);
     if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
     if (merge_smem > 48 * 1024 &&
-        cudaFuncSetAttribute(tk::merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(tk::merge_kernel<QB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(merge_smem)) != cudaSuccess)
       return TQ_ERR_CUDA;
-    tk::merge_kernel<<<Q, 128, merge_smem, st>>>(p, out_ids, out_scores);
+    tk::merge_kernel<QB><<<Q, 128, merge_smem, st>>>(p, out_ids, out_scores);
     return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
   };
-  if (d == 128) return go(std::integral_constant<int, 128>{});
-  if (d == 64) return go(std::integral_constant<int, 64>{});
+  using I64 = std::integral_constant<int, 64>;
+  using I128 = std::integral_constant<int, 128>;
+  if (d == 128) return qb == 128 ? go(I128{}, I128{}) : go(I128{}, I64{});
+  if (d == 64) return qb == 128 ? go(I64{}, I128{}) : go(I64{}, I64{});
   return TQ_ERR_UNSUPPORTED;
 }
 

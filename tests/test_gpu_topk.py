@@ -1,9 +1,10 @@
 """Parity of tq_score_topk (CUDA, through the C ABI) with the oracle's
 compressed search on the same oracle-written keys-only pages.
 
-Scores: GPU (fp16 hi/lo query planes against exact bit-plane operands, fp32
-accumulation) within a bound derived from that arithmetic of the oracle's
-fp64 scores.  Ids: identical at every rank whose oracle score is separated
+Scores: GPU (fp16 hi/lo query planes against bit-plane operands, fp32
+accumulation; the key plane holds the two centroid magnitudes as fp16 values
+whose ratio is within 2^-19 of kc1/kc0) within a bound derived from that
+arithmetic of the oracle's fp64 scores.  Ids: identical at every rank whose oracle score is separated
 from the other candidates by more than twice that bound; inside a group of
 near-ties the GPU may order equal-within-bound candidates differently."""
 import math
@@ -56,12 +57,14 @@ def gpu_topk(ctx, queries, db, N, k):
 
 def score_bound(P, q, rec_n_max, gamma_max):
     """Bound on |GPU score - exact estimate| for query q: the fp16 hi/lo split
-    leaves 2^-22 relative error per query-plane element; fp32 accumulation of
-    3d terms adds 3d 2^-24 relative to the sum of |terms|."""
+    leaves 2^-22 relative error per query-plane element; the key plane's fp16
+    centroid ratio adds at most 2^-19 relative on the key terms; fp32
+    accumulation of the 2d terms adds 2d 2^-24 relative to the sum of |terms|
+    (3d is used, a margin)."""
     qrot = P.pi32 @ q
     qs = P.S @ qrot
     mag = np.abs(qrot).sum() * P.kc[-1] + P.alpha * gamma_max * np.abs(qs).sum()
-    return rec_n_max * mag * (2.0 ** -20 + 3 * len(q) * 2.0 ** -24) + 1e-12
+    return rec_n_max * mag * (2.0 ** -20 + 2.0 ** -19 + 3 * len(q) * 2.0 ** -24) + 1e-12
 
 
 def check_against_oracle(O, P, ctx, queries, db, rec, N, k, extra=8):
