@@ -91,6 +91,7 @@ struct Params {
   int* cand_i;
   int n_qb, n_slices;
   long long pages;
+  int seed_only;  // a seeding pass: raise the slots only, write no lists
   int* err;
 };
 
@@ -477,6 +478,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
     uint32_t qmask[C::NPASS], bl[C::NPASS], cmin[C::NPASS], sf[C::NPASS];
     int list_item = -1, q0h = 0, se = 0;
     auto flush = [&](int item) {
+      if (p.seed_only) return;
       const size_t base = (static_cast<size_t>(item) * NEPI + warp) * WQ * k;
       const float* dq = p.desc + (item % p.n_qb) * QB + WQ * half;
       // lists hold scores before the per-query power-of-two descale (the
@@ -878,6 +880,16 @@ int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* d
     }
     tk::qprep_kernel<D, QB><<<p.n_qb * QB, 128, 0, st>>>(p);
     if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
+    // seeding pass over the first pages: every query's slots start from the
+    // k best of a sample instead of from nothing, which spares the main
+    // pass most of its early list insertions
+    const long long seed_pages = p.n_slices > 64 ? p.n_slices : 64;
+    if (p.pages >= 8 * seed_pages) {
+      tk::Params ps = p;
+      ps.pages = seed_pages;
+      ps.seed_only = 1;
+      tk::score_kernel<D, QB><<<grid, tk::NTHREADS, smem, st>>>(ps);
+    }
     tk::score_kernel<D, QB><<<grid, tk::NTHREADS, smem, st>>>(p);
     if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
     if (merge_smem > 48 * 1024 &&
