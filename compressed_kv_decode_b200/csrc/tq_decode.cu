@@ -15,8 +15,10 @@
 //               units (64 cold tokens or 16 hot tokens).  A warp streams its
 //               units through a private ring of shared-memory slots filled by
 //               1-D bulk copies (TMA) completing on mbarriers, unpacks the
-//               codes into fp16 tensor-core fragments in registers, scores
-//               them with m16n8k16 MMAs (tokens on M, q heads x {hi, lo} on N),
+//               codes into fp16 tensor-core fragments in registers (the key
+//               code as one plane of +-b / +-a, a / b the fp16 ratio nearest
+//               kc1 / kc0, and the QJL signs as +-gamma), scores them with
+//               m16n8k16 MMAs (tokens on M, q heads x {hi, lo} on N),
 //               keeps an online softmax and accumulates P.V with MMAs (cold
 //               values in the rotated domain).  It writes one partial
 //               (m, l, o) per segment it touched.
@@ -29,6 +31,7 @@
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
+#include "tq_keyplane.h"
 
 namespace tq {
 namespace dec {
@@ -42,7 +45,7 @@ template <int D, int G>
 struct Cfg {
   static constexpr int KS = D / 16;              // k-steps per key plane (and QJL, m = D)
   static constexpr int NT = (2 * G + 7) / 8;     // score n-tiles: G heads x {hi, lo}
-  static constexpr int RC = 3 * KS * NT * 2;     // cold B-fragment registers per lane
+  static constexpr int RC = 2 * KS * NT * 2;     // cold B-fragment registers per lane (key, QJL planes)
   static constexpr int RH = KS * NT * 2;         // hot B-fragment registers per lane
   static constexpr int WPT = D / 64;             // key code words per lane per token
   static constexpr int WV = D / 32;              // value words per lane per token pair
@@ -90,7 +93,8 @@ struct Params {
   const float* rot;
   const float* qjl;
   const float* sp;  // S Pi
-  float kc0, kc1, alpha;
+  float w_key, alpha;          // query weights of the key plane (kc0 / b) and of the QJL plane
+  uint32_t key_b2, key_d7;     // key plane: fp16 b and fp16(2^7 (a - b)), both halves
   float vc[8];
   int* err;
   Work w;
@@ -329,10 +333,10 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   __syncthreads();
   matvec_rows2<D, G>(p.rot, p.sp, sq, sqr, sqs);  // q_rot = Pi q, q_s = (S Pi) q
   __syncthreads();
-  const float w1c = p.sl * p.kc0, w2c = p.sl * 128.0f * (p.kc1 - p.kc0), w3c = p.sl * p.alpha;
+  const float w1c = p.sl * p.w_key, w3c = p.sl * p.alpha;
   for (int i = tid; i < G * D; i += blockDim.x) {
     const int g = i / D, j = i % D;
-    float mc = fmaxf(fmaxf(fabsf(w1c * sqr[g][j]), fabsf(w2c * sqr[g][j])), fabsf(w3c * sqs[g][j]));
+    float mc = fmaxf(fabsf(w1c * sqr[g][j]), fabsf(w3c * sqs[g][j]));
     float mh = fabsf(p.sl * sq[g][j]);
     atomicMax(&smax[0][g], __float_as_uint(mc));
     atomicMax(&smax[1][g], __float_as_uint(mh));
@@ -354,14 +358,14 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
     uint32_t val = 0u;
     if (h < G) {
       const float f = sfac[0][h];
-      if (pk < 2 * C::KS) {
-        const int s = pk % C::KS;
-        const float wc = f * ((pk < C::KS) ? w1c : w2c);
+      if (pk < C::KS) {
+        const int s = pk;
+        const float wc = f * w1c;
         const int P = cc * (D / 8) + 2 * s + reg;
         const int jlo = 16 * (P >> 3) + (P & 7);
         val = pack_split(wc * sqr[h][jlo], wc * sqr[h][jlo + 8], part);
       } else {
-        const int s = pk - 2 * C::KS;
+        const int s = pk - C::KS;
         const float wc = f * w3c;
         const int P = cc * (D / 8) + 2 * s + reg;
         const int ilo = 32 * (P >> 4) + (P & 15);
@@ -686,21 +690,22 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         const uint32_t qw1 = *reinterpret_cast<const uint32_t*>(sb + C::OFF_QS + t1 * (D / 8) + 4 * qword);
         const uint32_t gg0 = static_cast<uint32_t>(kg[t0]) * 0x10001u;
         const uint32_t gg1 = static_cast<uint32_t>(kg[t1]) * 0x10001u;
-        // three independent accumulation chains (sign, magnitude, QJL planes)
-        float acc[C::NT][4], acm[C::NT][4], acq[C::NT][4];
+        // two independent accumulation chains (key plane, QJL plane)
+        float acc[C::NT][4], acq[C::NT][4];
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][e] = acm[nt][e] = acq[nt][e] = 0.0f;
+          for (int e = 0; e < 4; ++e) acc[nt][e] = acq[nt][e] = 0.0f;
 #pragma unroll
         for (int s = 0; s < C::KS; ++s) {
           const int w = s >> 2, sh = 4 * (s & 3);
           const uint32_t x0a = kw0[w] << sh, x0b = kw0[w] << (sh + 1);
           const uint32_t x1a = kw1[w] << sh, x1b = kw1[w] << (sh + 1);
-          const uint32_t a0 = (x0a & 0x80008000u) | 0x3C003C00u, a1 = (x1a & 0x80008000u) | 0x3C003C00u;
-          const uint32_t a2 = (x0b & 0x80008000u) | 0x3C003C00u, a3 = (x1b & 0x80008000u) | 0x3C003C00u;
-          const uint32_t m0 = x0a & 0xA000A000u, m1 = x1a & 0xA000A000u;
-          const uint32_t m2 = x0b & 0xA000A000u, m3 = x1b & 0xA000A000u;
+          // key plane: sign bit at 15 / 31, magnitude bit at 13 / 29 -> +-b or +-a
+          const uint32_t a0 = key_plane_pair(x0a, p.key_d7, p.key_b2);
+          const uint32_t a1 = key_plane_pair(x1a, p.key_d7, p.key_b2);
+          const uint32_t a2 = key_plane_pair(x0b, p.key_d7, p.key_b2);
+          const uint32_t a3 = key_plane_pair(x1b, p.key_d7, p.key_b2);
           const int sq = qsb + 2 * s;
           const uint32_t q0 = ((qw0 << sq) & 0x80008000u) | gg0;
           const uint32_t q1 = ((qw1 << sq) & 0x80008000u) | gg1;
@@ -709,16 +714,14 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
 #pragma unroll
           for (int nt = 0; nt < C::NT; ++nt) {
             mma_f16(acc[nt], a0, a1, a2, a3, bfr[(s * C::NT + nt) * 2], bfr[(s * C::NT + nt) * 2 + 1]);
-            mma_f16(acm[nt], m0, m1, m2, m3, bfr[((C::KS + s) * C::NT + nt) * 2],
+            mma_f16(acq[nt], q0, q1, q2, q3, bfr[((C::KS + s) * C::NT + nt) * 2],
                     bfr[((C::KS + s) * C::NT + nt) * 2 + 1]);
-            mma_f16(acq[nt], q0, q1, q2, q3, bfr[((2 * C::KS + s) * C::NT + nt) * 2],
-                    bfr[((2 * C::KS + s) * C::NT + nt) * 2 + 1]);
           }
         }
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][e] += acm[nt][e] + acq[nt][e];
+          for (int e = 0; e < 4; ++e) acc[nt][e] += acq[nt][e];
         const float n0 = __half2float(kn[t0]), n1 = __half2float(kn[t1]);
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt) {
@@ -1102,8 +1105,11 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
   p.rot = ctx->dev.rot;
   p.qjl = ctx->dev.qjl;
   p.sp = ctx->dev.sp;
-  p.kc0 = ctx->cb.key_c[0];
-  p.kc1 = ctx->cb.key_c[1];
+  KeyPlane kp;
+  if (!key_plane(ctx->cb.key_c[0], ctx->cb.key_c[1], kp)) return TQ_ERR_UNSUPPORTED;
+  p.w_key = static_cast<float>(ctx->cb.key_c[0] / kp.b);
+  p.key_b2 = kp.b2;
+  p.key_d7 = kp.d7;
   p.alpha = std::sqrt(3.14159265358979323846f / 2.0f) / static_cast<float>(ctx->cfg.qjl_dim);
   for (int k = 0; k < 8; ++k) p.vc[k] = ctx->cb.val_c[k];
   p.err = ctx->dev.err;

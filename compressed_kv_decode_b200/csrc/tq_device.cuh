@@ -136,6 +136,21 @@ __device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r
 }
 
 // fp16 hi/lo split of an fp32 value: hi = fp16(x), lo = fp16(x - hi)
+// d = a * b + c on two fp16 lanes (round to nearest even)
+__device__ __forceinline__ uint32_t hfma2_bits(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// key-plane value of two coordinates from a code word shifted so that their
+// sign bits sit at 15 / 31 and magnitude bits at 13 / 29: the masked word is
+// the fp16 pair +-m 2^-7, and one FMA gives +-(b + m (a - b)) exactly
+// (d7 = fp16(2^7 (a - b)) chosen so; b2 = b in both halves)
+__device__ __forceinline__ uint32_t key_plane_pair(uint32_t x, uint32_t d7, uint32_t b2) {
+  return hfma2_bits(x & 0xA000A000u, d7, (x & 0x80008000u) | b2);
+}
+
 __device__ __forceinline__ void split_f16(float x, uint16_t& hi, uint16_t& lo) {
   __half h = __float2half_rn(x);
   hi = __half_as_ushort(h);

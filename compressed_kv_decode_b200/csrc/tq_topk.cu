@@ -31,6 +31,7 @@
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
+#include "tq_keyplane.h"
 #include "tq_tc.cuh"
 
 namespace tq {
@@ -82,7 +83,7 @@ struct Params {
   const float* rot;
   const float* sp;     // S Pi
   float w_key, alpha;  // query weights of the key plane (kc0 / b) and of the QJL plane
-  uint32_t key_b2, key_diff;  // fp16 bits of b in both halves; bits(a) - bits(b)
+  uint32_t key_b2, key_d7;  // fp16 b and fp16(2^7 (a - b)), both halves
   uint16_t* bimg;      // [n_qb][NROW * KTOT] fp16 bits, SW128 image per block
   float* desc;         // [n_qb * QB] descale
   uint32_t* gslots;    // [n_qb * QB][k] per query: slot e holds the best score (ordered bits)
@@ -294,16 +295,14 @@ __device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t* r) {
 // QJL word w holds sketch index 32 w + 16 h + r at bit 16 h + 15 - r.
 template <int D>
 __device__ __forceinline__ void build_a_row(const uint32_t* kw, const uint32_t* qw, uint32_t gg,
-                                            uint32_t base, int half, uint32_t key_b2, uint32_t key_diff) {
+                                            uint32_t base, int half, uint32_t key_b2, uint32_t key_d7) {
   constexpr int NW = D / 32;  // key words of one half
   uint32_t a[D / 4];
 #pragma unroll
   for (int wl = 0; wl < NW; ++wl)
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
-      const uint32_t x = kw[wl] << ((s >> 1) * 4 + (s & 1));
-      const uint32_t m = (x >> 13) & 0x00010001u;  // magnitude bits -> bit 0 / bit 16
-      a[wl * 8 + s] = (x & 0x80008000u) | (m * key_diff + key_b2);
+      a[wl * 8 + s] = key_plane_pair(kw[wl] << ((s >> 1) * 4 + (s & 1)), key_d7, key_b2);
     }
   tmem_store<D / 4>(base + half * (D / 4), a);
 #pragma unroll
@@ -521,7 +520,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {
     int item_cur = 0;
     uint32_t t = 0;
     auto build_next = [&](uint32_t buf) {
-      build_a_row<D>(r.kw, r.qw, r.gg, t_lane + (buf ? COL_A1 : COL_A0), half, p.key_b2, p.key_diff);
+      build_a_row<D>(r.kw, r.qw, r.gg, t_lane + (buf ? COL_A1 : COL_A0), half, p.key_b2, p.key_d7);
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
@@ -776,40 +775,6 @@ Ws ws_layout(const tq_ctx* ctx, int Q, long long N, int k) {
   return w;
 }
 
-// fp16 bits of a positive value with at most 11 significant bits in the
-// normal range
-inline uint32_t f16_bits_exact(double v) {
-  const int e = static_cast<int>(std::floor(std::log2(v)));
-  const double mant = v / std::ldexp(1.0, e) - 1.0;
-  return (static_cast<uint32_t>(e + 15) << 10) | static_cast<uint32_t>(std::lround(mant * 1024.0));
-}
-
-// the key plane's two magnitudes: fp16 values b (index 0) and a (index 1)
-// whose ratio a / b is the nearest of all ratios of 11-bit integers (times a
-// power of two) to kc1 / kc0; b is scaled into [1, 2).  Returns the
-// relative error of a / b.
-inline double key_plane_values(double kc0, double kc1, double& a, double& b) {
-  const double r = kc1 / kc0;
-  double best = -1.0;
-  a = r;
-  b = 1.0;
-  for (int sh = -3; sh <= 3; ++sh) {
-    const double t = std::ldexp(r, -sh);
-    for (int qd = 1; qd < 2048; ++qd) {
-      const double pn = std::nearbyint(qd * t);
-      if (pn < 1.0 || pn > 2047.0) continue;
-      const double err = std::fabs(std::ldexp(pn / qd, sh) - r);
-      if (best < 0.0 || err < best) {
-        best = err;
-        const double sc = std::ldexp(1.0, -static_cast<int>(std::floor(std::log2(static_cast<double>(qd)))));
-        b = qd * sc;
-        a = std::ldexp(pn, sh) * sc;
-      }
-    }
-  }
-  return best / r;
-}
-
 }  // namespace tk
 
 size_t topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k) {
@@ -839,14 +804,11 @@ int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* d
   p.rot = ctx->dev.rot;
   p.sp = ctx->dev.sp;
   // the key plane's centroid ratio is carried to better than 2^-19
-  double ka, kb;
-  if (!(tk::key_plane_values(ctx->cb.key_c[0], ctx->cb.key_c[1], ka, kb) <= 0x1p-19))
-    return TQ_ERR_UNSUPPORTED;
-  const uint32_t bits_a = tk::f16_bits_exact(ka), bits_b = tk::f16_bits_exact(kb);
-  if (!(ka > kb) || bits_a >= 0x7C00u) return TQ_ERR_UNSUPPORTED;
-  p.w_key = static_cast<float>(ctx->cb.key_c[0] / kb);
-  p.key_b2 = bits_b * 0x10001u;
-  p.key_diff = bits_a - bits_b;
+  KeyPlane kp;
+  if (!key_plane(ctx->cb.key_c[0], ctx->cb.key_c[1], kp)) return TQ_ERR_UNSUPPORTED;
+  p.w_key = static_cast<float>(ctx->cb.key_c[0] / kp.b);
+  p.key_b2 = kp.b2;
+  p.key_d7 = kp.d7;
   p.alpha = 1.2533141373155001f / static_cast<float>(ctx->cfg.qjl_dim);
   uint8_t* base = static_cast<uint8_t*>(ws);
   p.bimg = reinterpret_cast<uint16_t*>(base + L.bimg);
