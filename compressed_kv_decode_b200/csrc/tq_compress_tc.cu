@@ -425,6 +425,342 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
+
+// ---------------------------------------------------------------------------
+// Keys only (search databases, key-only appends): the same steps, software
+// pipelined over tiles and warp-specialised.  One warp issues the copies and
+// the tensor-core work (one lane); sixteen warps quantise, a thread owning one
+// row and a quarter of its columns.  The rotation of tile t+1 (two TMEM
+// accumulators) and the sketch of tile t (its residual kept in TMEM as the
+// sketch's A operand, two buffers) run while the sixteen warps quantise;
+// input tiles are double-buffered.  Hand-offs go through mbarriers:
+//   full[b]     input tile b landed (and its tile record published)
+//   rk[b]       rotation of the tile in buffer b done
+//   resfull[b]  tile b quantised: residual in TMEM, input and rotation
+//               buffers free
+//   sk          sketch done;  skfree  sketch accumulator read
+// A tile record ring in shared memory carries each tile's page and row range
+// from the issuing lane to the quantising warps (bh < 0: no further tile).
+// ---------------------------------------------------------------------------
+// sum of squares of this thread's part (quarter) of a row of a 16-bit tile
+template <int D, bool BF>
+__device__ __forceinline__ float part_row_sumsq(const uint8_t* x, int row, int q) {
+  constexpr int PART = D / 4;
+  float ss = 0.0f;
+#pragma unroll
+  for (int c = 0; c < PART / 8; ++c) {
+    const int k = q * PART + 8 * c;
+    const uint4 v = *reinterpret_cast<const uint4*>(x + tc::sw128_offset(row, k, ROWS));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float a, b;
+      if constexpr (BF) {
+        a = __uint_as_float(w[i] << 16);
+        b = __uint_as_float(w[i] & 0xFFFF0000u);
+      } else {
+        const __half2 hh = *reinterpret_cast<const __half2*>(&w[i]);
+        a = __low2float(hh);
+        b = __high2float(hh);
+      }
+      ss = fmaf(a, a, fmaf(b, b, ss));
+    }
+  }
+  return ss;
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_load_part(uint32_t taddr, float (&x)[N]) {
+  uint32_t r[N];
+  if constexpr (N == 32) tc::ld32(taddr, r);
+  else tc::ld16(taddr, r);
+  tc::wait_ld();
+#pragma unroll
+  for (int i = 0; i < N; ++i) x[i] = __uint_as_float(r[i]);
+}
+
+constexpr int KEPI = 16;                    // quantising warps
+constexpr int KTHREADS = (KEPI + 1) * 32;   // + the issuing warp
+constexpr int NPART = 4;                    // column quarters
+
+template <int D>
+struct KCfg {
+  static constexpr int PART = D / NPART;  // columns per thread
+  static constexpr int OPB = D * 128;
+  static constexpr int OP = (D / 64) * OPB;
+  static constexpr int XB = ROWS * 128;
+  static constexpr int XT = (D / 64) * XB;
+  static constexpr int OFF_PH = 0;
+  static constexpr int OFF_PL = OFF_PH + OP;
+  static constexpr int OFF_S = OFF_PL + OP;
+  static constexpr int OFF_X = OFF_S + OP;            // two input tiles
+  static constexpr int OFF_NK = OFF_X + 2 * XT;       // float[2][4][128] key norm^2 parts
+  static constexpr int OFF_G = OFF_NK + 2 * 4 * 512;  // float[2][4][128] residual norm^2 parts
+  static constexpr int OFF_RING = OFF_G + 2 * 4 * 512;  // Tile[4]
+  static constexpr int OFF_BAR = OFF_RING + 128;      // 9 mbarriers
+  static constexpr int OFF_TMEM = OFF_BAR + 128;
+  static constexpr int OFF_FAIL = OFF_TMEM + 4;
+  static constexpr int SMEM = OFF_TMEM + 16 + 1024;   // + alignment slack
+  // TMEM columns: two rotation accumulators, the sketch accumulator, two
+  // fp16 residual buffers (A operand: two K elements per 32-bit column)
+  static constexpr int COL_RK0 = 0, COL_SK = 2 * D, COL_RES0 = 3 * D;
+  static constexpr uint32_t TMEM_COLS = (4 * D <= 256) ? 256 : 512;
+  static_assert(COL_RES0 + D <= static_cast<int>(TMEM_COLS), "TMEM columns");
+  static_assert(sizeof(Tile) * 4 <= 128, "tile ring");
+};
+
+// barrier among the quantising warps (named barrier 1), returning whether any
+// of their threads passed `pred`
+__device__ __forceinline__ bool epi_sync_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(KEPI * 32)
+      : "memory");
+  return r != 0;
+}
+
+template <int D, bool BF>
+__global__ void __maxnreg__(96) compress_keys_kernel(const __grid_constant__ CUtensorMap mapK, Params p) {
+  using C = KCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t s0 = smem_u32(smem);
+  const uint32_t bar_full = s0 + C::OFF_BAR, bar_rk = bar_full + 16, bar_res = bar_full + 32;
+  const uint32_t bar_sk = bar_full + 48, bar_skfree = bar_full + 56, bar_drain = bar_full + 64;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+  int* fail_flag = reinterpret_cast<int*>(smem + C::OFF_FAIL);
+  float* nk = reinterpret_cast<float*>(smem + C::OFF_NK);
+  float* gp = reinterpret_cast<float*>(smem + C::OFF_G);
+  Tile* ring = reinterpret_cast<Tile*>(smem + C::OFF_RING);
+
+  for (int i = tid; i < D * (D / 8); i += KTHREADS) {
+    const int r = i / (D / 8), k = (i % (D / 8)) * 8;
+    const uint32_t off = tc::sw128_offset(r, k, D);
+    *reinterpret_cast<uint4*>(smem + C::OFF_PH + off) =
+        *reinterpret_cast<const uint4*>(p.pi_hi + static_cast<size_t>(r) * D + k);
+    *reinterpret_cast<uint4*>(smem + C::OFF_PL + off) =
+        *reinterpret_cast<const uint4*>(p.pi_lo + static_cast<size_t>(r) * D + k);
+    *reinterpret_cast<uint4*>(smem + C::OFF_S + off) =
+        *reinterpret_cast<const uint4*>(p.s_h + static_cast<size_t>(r) * D + k);
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(bar_full + 8 * i, 1);       // full[2], rk[2]
+    for (int i = 0; i < 2; ++i) mbar_init(bar_res + 8 * i, KEPI);     // resfull[2]
+    mbar_init(bar_sk, 1);
+    mbar_init(bar_skfree, KEPI);
+    mbar_init(bar_drain, 1);
+    *fail_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == KEPI) {
+    tc::tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  if (warp == KEPI) {
+    // ---- copies and tensor-core work, one lane ------------------------------
+    if (lane == 0) {
+      bool failed = false;
+      int tsearch = blockIdx.x;
+      uint32_t loads[2] = {0u, 0u}, landed[2] = {0u, 0u};
+      // publish the record of tile `idx` of this CTA's sequence and start its
+      // copy into buffer `buf`; a missing tile publishes bh = -1
+      auto fetch = [&](uint32_t idx, uint32_t buf) -> bool {
+        Tile tl;
+        const bool ok = next_tile(p, tsearch, tl);
+        if (ok) tsearch += gridDim.x;
+        else tl.bh = -1;
+        ring[idx & 3u] = tl;
+        if (ok) {
+          fence_proxy_async_smem();
+          issue_tile_load<D>(&mapK, s0 + C::OFF_X + buf * C::XT, bar_full + 8 * buf, tl);
+          ++loads[buf];
+        } else {
+          mbar_arrive(bar_full + 8 * buf);  // releases the record
+        }
+        return ok;
+      };
+      auto rotate = [&](uint32_t idx) -> bool {
+        const uint32_t bb = idx & 1u;
+        if (!mbar_wait_bounded(bar_full + 8 * bb, (idx >> 1) & 1u)) return false;
+        ++landed[bb];
+        tc::fence_after_sync();
+        issue_rotation<D, BF>(tmem, C::COL_RK0 + static_cast<int>(bb) * D, s0 + C::OFF_X + bb * C::XT,
+                              s0 + C::OFF_PH, s0 + C::OFF_PL);
+        tc::commit(bar_rk + 8 * bb);
+        return true;
+      };
+      constexpr uint32_t idesc_sk = tc::idesc_f16(ROWS, D, false);
+      bool h_cur = fetch(0, 0);
+      bool h_next = h_cur && fetch(1, 1);
+      if (h_cur && !rotate(0)) failed = true;
+      for (uint32_t it = 0; h_cur && !failed; ++it) {
+        const uint32_t b = it & 1u;
+        if (h_next && !rotate(it + 1)) { failed = true; break; }
+        // tile it quantised: its buffers are free and its residual is ready
+        if (!mbar_wait_bounded(bar_res + 8 * b, (it >> 1) & 1u)) { failed = true; break; }
+        bool h_next2 = false;
+        if (h_next) h_next2 = fetch(it + 2, b);
+        if (it > 0 && !mbar_wait_bounded(bar_skfree, (it - 1) & 1u)) { failed = true; break; }
+        tc::fence_after_sync();
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          const int kb = s >> 2, w = (s & 3) * 32;
+          tc::mma_f16_tmem_a(tmem + C::COL_SK, tmem + C::COL_RES0 + b * (D / 2) + 8 * s,
+                             tc::sdesc_sw128(s0 + C::OFF_S + kb * C::OPB + w), idesc_sk, s > 0);
+        }
+        tc::commit(bar_sk);
+        h_cur = h_next;
+        h_next = h_next2;
+      }
+      // no copy or product may still be in flight when the CTA exits
+      for (int bb = 0; bb < 2; ++bb)
+        for (uint32_t k2 = landed[bb]; k2 < loads[bb]; ++k2) mbar_wait_bounded(bar_full + 8 * bb, k2 & 1u);
+      tc::commit(bar_drain);
+      mbar_wait_bounded(bar_drain, 0);
+      if (failed) *fail_flag = 1;
+    }
+    __syncwarp();
+  } else {
+    // ---- sixteen warps: quantise, then the previous tile's sign bits --------
+    const int row = 32 * (warp & 3) + lane;  // TMEM lane quarter of this warp
+    const int q = warp >> 2;                 // column quarter
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    bool failed = false;
+    Tile cur, prev;
+    bool have_prev = false;
+    float prev_n = 0.0f;
+    for (uint32_t it = 0;; ++it) {
+      const uint32_t b = it & 1u;
+      // the tile's record (released with its copy)
+      if (!mbar_wait_bounded(bar_full + 8 * b, (it >> 1) & 1u)) failed = true;
+      cur = ring[it & 3u];
+      if (epi_sync_or(failed)) {
+        failed = true;
+        break;
+      }
+      const bool have = cur.bh >= 0;
+      if (!have && !have_prev) break;
+      float x[C::PART];
+      float n = 0.0f;
+      if (have) {
+        if (!mbar_wait_bounded(bar_rk + 8 * b, (it >> 1) & 1u)) failed = true;
+        tc::fence_after_sync();
+        nk[(b * NPART + q) * ROWS + row] = part_row_sumsq<D, BF>(smem + C::OFF_X + b * C::XT, row, q);
+        tmem_load_part<C::PART>(t_lane + C::COL_RK0 + b * D + q * C::PART, x);
+      }
+      if (epi_sync_or(failed)) {  // norm parts complete
+        failed = true;
+        break;
+      }
+      if (have) {
+        const bool page_ok = cur.page >= 0 && cur.page < p.pool_pages;
+        const bool wr = page_ok && row >= cur.s_lo && row < cur.s_hi;
+        if (tid == 0 && !page_ok) report(p.err, TQ_ERR_CAPACITY);
+        uint8_t* pg = p.pool + static_cast<size_t>(page_ok ? cur.page : 0) * p.page_bytes;
+        const float* nkb = nk + b * NPART * ROWS;
+        const float nn = sqrtf((nkb[row] + nkb[ROWS + row]) + (nkb[2 * ROWS + row] + nkb[3 * ROWS + row]));
+        const __half nh = __float2half_rn(nn);
+        n = __half2float(nh);
+        const float T0 = __fmul_rn(n, p.kt0);
+        const float inv = n > 0.0f ? 1.0f / n : 0.0f;
+        uint32_t kw[C::PART / 16];
+#pragma unroll
+        for (int w = 0; w < C::PART / 16; ++w) kw[w] = 0u;
+        uint32_t rh[C::PART / 2];
+        float g2 = 0.0f;
+#pragma unroll
+        for (int i2 = 0; i2 < C::PART / 2; ++i2) {
+          float rr[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int i = 2 * i2 + e;  // column within the part (parts are 16-aligned)
+            const float v = x[i];
+            const uint32_t sg = (n > 0.0f && v < 0.0f) ? 1u : 0u;
+            const uint32_t mg = (n > 0.0f && fabsf(v) >= T0) ? 1u : 0u;
+            const float cp = mg ? p.kc1 : p.kc0;
+            const float r = (n > 0.0f) ? fmaf(v, inv, (v < 0.0f) ? cp : -cp) : 0.0f;
+            rr[e] = r;
+            g2 = fmaf(r, r, g2);
+            const int jj = i & 15, hh = jj >> 3, ii = (jj & 7) >> 1, ee = jj & 1;
+            const int sbit = 16 * hh + 15 - 4 * ii - ee;
+            kw[i >> 4] |= (sg << sbit) | (mg << (sbit - 2));
+          }
+          const __half2 pr = __floats2half2_rn(rr[0], rr[1]);
+          rh[i2] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        // residual: fp16, coordinates 2c, 2c+1 in TMEM column c of this buffer
+        if constexpr (C::PART / 2 == 16)
+          tc::st16(t_lane + C::COL_RES0 + b * (D / 2) + q * (C::PART / 2), rh);
+        else
+          tc::st8(t_lane + C::COL_RES0 + b * (D / 2) + q * (C::PART / 2), rh);
+        gp[(b * NPART + q) * ROWS + row] = g2;
+        if (wr) {
+          if constexpr (C::PART / 16 == 2)
+            *reinterpret_cast<uint2*>(pg + p.off_kc + row * (D / 4) + q * (C::PART / 4)) =
+                make_uint2(kw[0], kw[1]);
+          else
+            *reinterpret_cast<uint32_t*>(pg + p.off_kc + row * (D / 4) + q * (C::PART / 4)) = kw[0];
+          if (q == 0) reinterpret_cast<__half*>(pg + p.off_kn)[row] = nh;
+        }
+        tc::wait_st();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_res + 8 * b);
+      }
+      if (have_prev) {
+        if (!mbar_wait_bounded(bar_sk, (it - 1) & 1u)) failed = true;
+        tc::fence_after_sync();
+        tmem_load_part<C::PART>(t_lane + C::COL_SK + q * C::PART, x);
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_skfree);
+        const bool page_ok = prev.page >= 0 && prev.page < p.pool_pages;
+        if (!failed && page_ok && row >= prev.s_lo && row < prev.s_hi) {
+          uint8_t* pgp = p.pool + static_cast<size_t>(prev.page) * p.page_bytes;
+          // sketch index i of the part sits in its 32-bit word at bit
+          // 16 (i / 16 mod 2) + 15 - i mod 16 (a part of 16 fills one half word)
+          uint32_t qw = 0u;
+#pragma unroll
+          for (int i = 0; i < C::PART; ++i) {
+            const int within = i & 31;
+            const int bit = 16 * (within >> 4) + 15 - (within & 15);
+            if (prev_n > 0.0f && x[i] < 0.0f) qw |= 1u << bit;
+          }
+          if constexpr (C::PART == 32)
+            *reinterpret_cast<uint32_t*>(pgp + p.off_qs + row * (D / 8) + q * 4) = qw;
+          else
+            *reinterpret_cast<uint16_t*>(pgp + p.off_qs + row * (D / 8) + q * 2) = static_cast<uint16_t>(qw);
+          if (q == 0) {
+            const float* gpp = gp + (b ^ 1u) * NPART * ROWS;
+            reinterpret_cast<__half*>(pgp + p.off_kg)[row] = __float2half_rn(
+                sqrtf((gpp[row] + gpp[ROWS + row]) + (gpp[2 * ROWS + row] + gpp[3 * ROWS + row])));
+          }
+        }
+      }
+      prev = cur;
+      prev_n = n;
+      have_prev = have;
+      if (!have) break;  // the last tile's sign bits are out
+    }
+    if (failed && lane == 0) *fail_flag = 1;
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == KEPI) tc::tmem_dealloc(tmem, C::TMEM_COLS);
+  if (tid == 0 && *fail_flag) report(p.err, TQ_ERR_TIMEOUT);
+}
+
 }  // namespace ctc
 
 __global__ void advance_cold_len(int32_t* cold_len, int B, int n_new) {
@@ -491,6 +827,28 @@ int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf1
     advance_cold_len<<<(B + 127) / 128, 128, 0, st>>>(cold_len, B, n_new);
     return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
   };
+  if (!v) {
+    // keys only: the software-pipelined kernel
+    auto gok = [&](auto kern, int smem) -> int {
+      static bool set[4] = {};
+      const int slot = (d == 128 ? 2 : 0) + (bf16 ? 1 : 0);
+      if (!set[slot]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+          return TQ_ERR_CUDA;
+        set[slot] = true;
+      }
+      if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
+      kern<<<grid, ctc::KTHREADS, smem, st>>>(mk, p);
+      if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
+      advance_cold_len<<<(B + 127) / 128, 128, 0, st>>>(cold_len, B, n_new);
+      return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+    };
+    if (d == 128)
+      return bf16 ? gok(ctc::compress_keys_kernel<128, true>, ctc::KCfg<128>::SMEM)
+                  : gok(ctc::compress_keys_kernel<128, false>, ctc::KCfg<128>::SMEM);
+    return bf16 ? gok(ctc::compress_keys_kernel<64, true>, ctc::KCfg<64>::SMEM)
+                : gok(ctc::compress_keys_kernel<64, false>, ctc::KCfg<64>::SMEM);
+  }
   if (d == 128)
     return bf16 ? go(ctc::compress_tc_kernel<128, true>, ctc::Cfg<128>::SMEM)
                 : go(ctc::compress_tc_kernel<128, false>, ctc::Cfg<128>::SMEM);

@@ -366,9 +366,6 @@ struct TileSeq {
   }
 };
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 
 template <int D, int QB>
 __global__ void __launch_bounds__(NTHREADS, 1) score_kernel(Params p) {

@@ -194,6 +194,89 @@ def test_keys_only_pages(O):
     assert compare_records(O, P, k[0, 0], rk, got, True, None) == 0
 
 
+def check_sketch_raw(P, rk, got, err):
+    """Residual norm and sketch sign bits of raw-input records against the
+    oracle's, on rows whose norm and codes match: the GPU residual differs
+    from the oracle's by the rotation error err/n plus fp16 rounding, so
+    gamma may differ by that much and a sign bit may flip only where
+    |S r| is within the error that carries through S."""
+    d = P.d
+    nz = rk["n"][:, None]
+    rows = (got["n"] == rk["n"]) & np.all((got["sign"] == rk["sign"]) & (got["mag"] == rk["mag"]), axis=1)
+    rows &= rk["n"] > 0
+    chat = np.where(rk["sign"] == 1, -1.0, 1.0) * P.kc[rk["mag"]]
+    r = np.where(nz > 0, rk["xrot"] / np.where(nz > 0, nz, 1) - chat, 0.0)
+    dr = err / np.where(nz > 0, nz, 1)  # per-element bound on the residual's rotation error
+    gam = np.linalg.norm(r, axis=1)
+    gbound = gam * 2.0 ** -10 + np.linalg.norm(dr, axis=1) + 1e-12
+    assert np.all(~rows | (np.abs(got["gamma"] - rk["gamma"]) <= gbound)), "residual norm"
+    pexact = r @ P.S.T
+    bound = ((dr + np.abs(r) * 2.0 ** -11) @ np.abs(P.S).T) + d * 2.0 ** -23 * (np.abs(r) @ np.abs(P.S).T)
+    flips = (got["qbits"] != rk["qbits"]) & rows[:, None]
+    assert np.all(~flips | (np.abs(pexact) <= bound)), "sketch sign flip away from zero"
+    return int(flips.sum())
+
+
+@pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
+def test_raw_keys_only_many_tiles(O, dtype):
+    """Keys-only appends of raw 16-bit inputs (the software-pipelined tensor-
+    core path): 4 x 8 sequences of 2050 tokens, several page tiles per CTA, a
+    partial last page; records match the oracle within the rotation error."""
+    d = 128
+    P = params_for(O, d)
+    ctx = ctx_for(d)
+    B, Hkv, n = 4, 8, 2050
+    scales = W.compress_scales(21, Hkv, d)
+    x = np.stack([W.compress_data(22 + b, scales, n) for b in range(B)])  # [B, Hkv, n, d]
+    x = W.round_to(x, dtype)
+    pool, table, cl = gpu_append(ctx, [(x, None)], B, Hkv, d, math.ceil(n / 128), with_values=False,
+                                 dtype=dtype, rotated=False)
+    assert np.array_equal(cl, [n] * B)
+    nb = ctx.page_bytes(False)
+    eps = 2.0 ** -8 if dtype == "bfloat16" else 2.0 ** -11
+    flips = sflips = 0
+    for b in range(B):
+        for h in range(Hkv):
+            got = unpack_seq(O, pool, table, b, h, n, d, False, nb)
+            rk = O.encode(P, x[b, h], True)
+            err = (np.abs(x[b, h]) @ np.abs(P.pi32).T) * (eps * eps * 2 + 64 * 2.0 ** -24)
+            flips += compare_records(O, P, x[b, h], rk, got, True, err)
+            sflips += check_sketch_raw(P, rk, got, err)
+    assert sflips <= 0.01 * B * Hkv * n * d
+    print("code differences at decision boundaries: %d, sketch sign flips near zero: %d, of %d"
+          % (flips, sflips, B * Hkv * n * d))
+
+
+def test_raw_keys_only_ragged_appends(O):
+    """Keys-only raw appends of odd lengths split pages across calls; every
+    record matches the oracle's encoding of the whole sequence within the
+    rotation error."""
+    d = 64
+    P = params_for(O, d)
+    ctx = ctx_for(d)
+    B, Hkv = 2, 3
+    sizes = [5, 128, 77, 300, 1, 250]
+    n = sum(sizes)
+    scales = W.compress_scales(23, Hkv, d)
+    x = W.round_to(np.stack([W.compress_data(24 + b, scales, n) for b in range(B)]), "bfloat16")
+    chunks, t = [], 0
+    for sz in sizes:
+        chunks.append((x[:, :, t:t + sz], None))
+        t += sz
+    pool, table, cl = gpu_append(ctx, chunks, B, Hkv, d, math.ceil(n / 128), with_values=False,
+                                 dtype="bfloat16", rotated=False)
+    assert np.array_equal(cl, [n] * B)
+    nb = ctx.page_bytes(False)
+    eps = 2.0 ** -8
+    for b in range(B):
+        for h in range(Hkv):
+            got = unpack_seq(O, pool, table, b, h, n, d, False, nb)
+            rk = O.encode(P, x[b, h], True)
+            err = (np.abs(x[b, h]) @ np.abs(P.pi32).T) * (eps * eps * 2 + 64 * 2.0 ** -24)
+            compare_records(O, P, x[b, h], rk, got, True, err)
+            check_sketch_raw(P, rk, got, err)
+
+
 def test_capacity_error(O):
     ctx = ctx_for(64)
     k = np.random.default_rng(5).standard_normal((1, 1, 300, 64))
