@@ -684,20 +684,28 @@ __global__ void __maxnreg__(96) compress_keys_kernel(const __grid_constant__ CUt
           float rr[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
+            // computed as for n > 0; a zero vector's row is cleared below
             const int i = 2 * i2 + e;  // column within the part (parts are 16-aligned)
             const float v = x[i];
-            const uint32_t sg = (n > 0.0f && v < 0.0f) ? 1u : 0u;
-            const uint32_t mg = (n > 0.0f && fabsf(v) >= T0) ? 1u : 0u;
-            const float cp = mg ? p.kc1 : p.kc0;
-            const float r = (n > 0.0f) ? fmaf(v, inv, (v < 0.0f) ? cp : -cp) : 0.0f;
+            const bool neg = v < 0.0f, big = fabsf(v) >= T0;
+            const float cp = big ? p.kc1 : p.kc0;
+            const float r = fmaf(v, inv, neg ? cp : -cp);
             rr[e] = r;
             g2 = fmaf(r, r, g2);
             const int jj = i & 15, hh = jj >> 3, ii = (jj & 7) >> 1, ee = jj & 1;
             const int sbit = 16 * hh + 15 - 4 * ii - ee;
-            kw[i >> 4] |= (sg << sbit) | (mg << (sbit - 2));
+            if (neg) kw[i >> 4] |= 1u << sbit;
+            if (big) kw[i >> 4] |= 1u << (sbit - 2);
           }
           const __half2 pr = __floats2half2_rn(rr[0], rr[1]);
           rh[i2] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        if (!(n > 0.0f)) {  // zero vector: all codes, residual and its norm are 0
+#pragma unroll
+          for (int w = 0; w < C::PART / 16; ++w) kw[w] = 0u;
+#pragma unroll
+          for (int i2 = 0; i2 < C::PART / 2; ++i2) rh[i2] = 0u;
+          g2 = 0.0f;
         }
         // residual: fp16, coordinates 2c, 2c+1 in TMEM column c of this buffer
         if constexpr (C::PART / 2 == 16)
@@ -735,8 +743,9 @@ __global__ void __maxnreg__(96) compress_keys_kernel(const __grid_constant__ CUt
           for (int i = 0; i < C::PART; ++i) {
             const int within = i & 31;
             const int bit = 16 * (within >> 4) + 15 - (within & 15);
-            if (prev_n > 0.0f && x[i] < 0.0f) qw |= 1u << bit;
+            if (x[i] < 0.0f) qw |= 1u << bit;
           }
+          if (!(prev_n > 0.0f)) qw = 0u;  // zero vector
           if constexpr (C::PART == 32)
             *reinterpret_cast<uint32_t*>(pgp + p.off_qs + row * (D / 8) + q * 4) = qw;
           else

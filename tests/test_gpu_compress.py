@@ -229,6 +229,8 @@ def test_raw_keys_only_many_tiles(O, dtype):
     scales = W.compress_scales(21, Hkv, d)
     x = np.stack([W.compress_data(22 + b, scales, n) for b in range(B)])  # [B, Hkv, n, d]
     x = W.round_to(x, dtype)
+    x[0, 0, 5] = 0.0    # zero vectors: all codes, norms and signs 0
+    x[3, 7, 2049] = 0.0
     pool, table, cl = gpu_append(ctx, [(x, None)], B, Hkv, d, math.ceil(n / 128), with_values=False,
                                  dtype=dtype, rotated=False)
     assert np.array_equal(cl, [n] * B)
@@ -242,6 +244,10 @@ def test_raw_keys_only_many_tiles(O, dtype):
             err = (np.abs(x[b, h]) @ np.abs(P.pi32).T) * (eps * eps * 2 + 64 * 2.0 ** -24)
             flips += compare_records(O, P, x[b, h], rk, got, True, err)
             sflips += check_sketch_raw(P, rk, got, err)
+    for b, h, t in ((0, 0, 5), (3, 7, 2049)):
+        got = unpack_seq(O, pool, table, b, h, n, d, False, nb)
+        for f in ("sign", "mag", "qbits", "n", "gamma"):
+            assert not np.any(got[f][t]), f
     assert sflips <= 0.01 * B * Hkv * n * d
     print("code differences at decision boundaries: %d, sketch sign flips near zero: %d, of %d"
           % (flips, sflips, B * Hkv * n * d))
