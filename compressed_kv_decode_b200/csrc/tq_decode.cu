@@ -31,7 +31,6 @@
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
-#include "tq_keyplane.h"
 
 namespace tq {
 namespace dec {
@@ -45,7 +44,8 @@ template <int D, int G>
 struct Cfg {
   static constexpr int KS = D / 16;              // k-steps per key plane (and QJL, m = D)
   static constexpr int NT = (2 * G + 7) / 8;     // score n-tiles: G heads x {hi, lo}
-  static constexpr int RC = 2 * KS * NT * 2;     // cold B-fragment registers per lane (key, QJL planes)
+  static constexpr int KK = D / 32;              // int8 k-steps per cold plane (m = D)
+  static constexpr int RC = 4 * KK * NT * 2;     // cold B-fragment registers per lane (planes s, m, sm, QJL)
   static constexpr int RH = KS * NT * 2;         // hot B-fragment registers per lane
   static constexpr int WPT = D / 64;             // key code words per lane per token
   static constexpr int WV = D / 32;              // value words per lane per token pair
@@ -67,11 +67,16 @@ struct Cfg {
   static constexpr int SMEM = NW * (NSLOT * SLOT + PBUF) + NW * NSLOT * 8 + NW * NSLOT * 4;
 };
 
+constexpr int DESC_N = 6;
+enum { DS_UK = 0, DS_HOT = 1, DS_CK = 2, DS_UQ = 3, DS_CQ = 4 };
+constexpr float FIX_MAX = 32511.0f;  // 16-bit fixed point whose hi byte stays within int8
+
 struct Work {
   int* sched;         // [4 + 2 (S+1) + S]: U, unit_off, slot_off, seg_len
   uint32_t* frag_c;   // [BH][RC][32]
   uint32_t* frag_h;   // [BH][RH][32]
-  float* desc;        // [BH][2][8] descale per (domain, head)
+  float* desc;        // [BH][DESC_N][8] per head: key unit, hot descale, key constant,
+                      // QJL unit, QJL constant (softmax scale folded in)
   float* part;        // [(Wtot + S)][G][D + 2]
 };
 
@@ -93,8 +98,7 @@ struct Params {
   const float* rot;
   const float* qjl;
   const float* sp;  // S Pi
-  float w_key, alpha;          // query weights of the key plane (kc0 / b) and of the QJL plane
-  uint32_t key_b2, key_d7;     // key plane: fp16 b and fp16(2^7 (a - b)), both halves
+  float kc0, kc1, alpha;       // key centroids, QJL constant sqrt(pi/2)/m
   float vc[8];
   int* err;
   Work w;
@@ -333,43 +337,91 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   __syncthreads();
   matvec_rows2<D, G>(p.rot, p.sp, sq, sqr, sqs);  // q_rot = Pi q, q_s = (S Pi) q
   __syncthreads();
-  const float w1c = p.sl * p.w_key, w3c = p.sl * p.alpha;
+  // Cold keys: four 0/1 operand planes -- sign s, magnitude m, s AND m, QJL
+  // sign b -- against 16-bit fixed-point query weights (int8 hi, lo):
+  //   <q_rot, c_hat> = c0 sum(q_rot) - 2 c0 <q_rot, s> + (c1 - c0) <q_rot, m>
+  //                    - 2 (c1 - c0) <q_rot, s m>
+  //   <q_s, 1 - 2 b> = sum(q_s) - 2 <q_s, b>
+  // One fixed-point unit per head for the three key planes, one for the QJL plane.
+  const float ck0 = p.kc0, dk1 = p.kc1 - p.kc0;
+  __shared__ unsigned smr[G], sms[G];
+  __shared__ float s_uk[G], s_uq[G];
+  if (tid < G) smr[tid] = sms[tid] = 0u;
+  __syncthreads();
   for (int i = tid; i < G * D; i += blockDim.x) {
     const int g = i / D, j = i % D;
-    float mc = fmaxf(fabsf(w1c * sqr[g][j]), fabsf(w3c * sqs[g][j]));
-    float mh = fabsf(p.sl * sq[g][j]);
-    atomicMax(&smax[0][g], __float_as_uint(mc));
-    atomicMax(&smax[1][g], __float_as_uint(mh));
+    atomicMax(&smr[g], __float_as_uint(fabsf(sqr[g][j])));
+    atomicMax(&sms[g], __float_as_uint(fabsf(sqs[g][j])));
+    atomicMax(&smax[1][g], __float_as_uint(fabsf(p.sl * sq[g][j])));
   }
   __syncthreads();
-  if (tid < 2 * G) {
-    const int dom = tid / G, g = tid % G;
-    const float f = prescale_for(__uint_as_float(smax[dom][g]));
-    sfac[dom][g] = f;
-    p.w.desc[(static_cast<size_t>(bh) * 2 + dom) * 8 + g] = 1.0f / f;
+  {
+    // per-head sums (one warp per head, fixed order)
+    const int wp = tid >> 5, ln = tid & 31;
+    if (wp < G) {
+      float a = 0.0f, b2 = 0.0f;
+      for (int j = ln; j < D; j += 32) {
+        a += sqr[wp][j];
+        b2 += sqs[wp][j];
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b2 += __shfl_xor_sync(0xffffffffu, b2, o);
+      }
+      if (ln == 0) {
+        const float mr = __uint_as_float(smr[wp]), ms = __uint_as_float(sms[wp]);
+        const float uk = mr > 0.0f ? 2.0f * fmaxf(ck0, dk1) * mr / FIX_MAX : 1.0f;
+        const float uq = ms > 0.0f ? 2.0f * p.alpha * ms / FIX_MAX : 1.0f;
+        s_uk[wp] = uk;
+        s_uq[wp] = uq;
+        float* ds = p.w.desc + static_cast<size_t>(bh) * DESC_N * 8;
+        ds[DS_UK * 8 + wp] = p.sl * uk;
+        ds[DS_CK * 8 + wp] = p.sl * ck0 * a;
+        ds[DS_UQ * 8 + wp] = p.sl * uq;
+        ds[DS_CQ * 8 + wp] = p.sl * p.alpha * b2;
+        const float f = prescale_for(__uint_as_float(smax[1][wp]));
+        sfac[1][wp] = f;
+        ds[DS_HOT * 8 + wp] = 1.0f / f;
+      }
+    }
   }
   __syncthreads();
-  // cold fragments: r = (pk * NT + nt) * 2 + reg; lane = 4 g' + c'
+  // cold fragments (m16n8k32, B = [k][n], 4 int8 of k per register):
+  // r = ((plane * KK + kappa) * NT + nt) * 2 + reg, lane = 4 g' + c';
+  // k = 4 c' + j (reg 0) or 4 c' + 16 + j (reg 1) of k-step kappa reads, on the
+  // A side, bit position p of byte j of one of lane c''s packed words:
+  //   key planes: word c' WPT + (2 kappa + reg) / 4, sign position
+  //               p = {7, 6, 3, 2}[(2 kappa + reg) % 4] (magnitude: p - 2)
+  //   QJL plane:  word c' / LPW, p = (c' % LPW) 8 / LPW + 2 kappa + reg
+  constexpr int LPW = 4 / C::KK;  // lanes sharing one QJL word
   for (int idx = tid; idx < C::RC * 32; idx += blockDim.x) {
     const int r = idx >> 5, lane = idx & 31;
     const int reg = r & 1, nt = (r >> 1) % C::NT, pk = (r >> 1) / C::NT;
+    const int plane = pk / C::KK, kap = pk % C::KK;
     const int gc = lane >> 2, cc = lane & 3;
     const int h = nt * 4 + (gc >> 1), part = gc & 1;
     uint32_t val = 0u;
     if (h < G) {
-      const float f = sfac[0][h];
-      if (pk < C::KS) {
-        const int s = pk;
-        const float wc = f * w1c;
-        const int P = cc * (D / 8) + 2 * s + reg;
-        const int jlo = 16 * (P >> 3) + (P & 7);
-        val = pack_split(wc * sqr[h][jlo], wc * sqr[h][jlo + 8], part);
-      } else {
-        const int s = pk - C::KS;
-        const float wc = f * w3c;
-        const int P = cc * (D / 8) + 2 * s + reg;
-        const int ilo = 32 * (P >> 4) + (P & 15);
-        val = pack_split(wc * sqs[h][ilo], wc * sqs[h][ilo + 16], part);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float qv;
+        if (plane < 3) {
+          const int gam = 2 * kap + reg;
+          const int ps = (gam & 3) == 0 ? 7 : (gam & 3) == 1 ? 6 : (gam & 3) == 2 ? 3 : 2;
+          const int beta = 8 * j + ps, hh = beta >> 4, rem = 15 - (beta & 15);
+          const int coord = 16 * (cc * C::WPT + (gam >> 2)) + 8 * hh + 2 * (rem >> 2) + (rem & 1);
+          const float w = plane == 0 ? -2.0f * ck0 * sqr[h][coord]
+                        : plane == 1 ? dk1 * sqr[h][coord] : -2.0f * dk1 * sqr[h][coord];
+          qv = w / s_uk[h];
+        } else {
+          const int pq = (cc % LPW) * (8 / LPW) + 2 * kap + reg;
+          const int beta = 8 * j + pq, hh = beta >> 4, rr = 15 - (beta & 15);
+          const int si = 32 * (cc / LPW) + 16 * hh + rr;
+          qv = -2.0f * p.alpha * sqs[h][si] / s_uq[h];
+        }
+        const int q16 = max(-32511, min(32511, __float2int_rn(qv)));
+        const int lo = ((q16 + 128) & 255) - 128, hi = (q16 - lo) >> 8;
+        val |= static_cast<uint32_t>((part == 0 ? hi : lo) & 0xFF) << (8 * j);
       }
     }
     p.w.frag_c[(static_cast<size_t>(bh) * C::RC + r) * 32 + lane] = val;
@@ -434,6 +486,22 @@ __device__ __forceinline__ void issue_unit(const Params& p, int sg, int lu, int 
       bulk_g2s(d0 + isv * HOT_TOK * C::HROW + r * C::HROW, src, 2 * D, bar);
     }
   }
+}
+
+// d += a * b, m16n8k32, a unsigned 8-bit, b signed 8-bit, s32 accumulate
+__device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// bit position, inside each byte of a key code word, of the sign bits read by
+// group gam % 4 (the magnitude bits sit two below)
+__host__ __device__ constexpr int sign_pos(int gam) {
+  return (gam & 3) == 0 ? 7 : (gam & 3) == 1 ? 6 : (gam & 3) == 2 ? 3 : 2;
 }
 
 // 8 value nibbles of a word (4 coordinates x 2 tokens) -> 4 half2 (token
@@ -540,7 +608,8 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
   // consume cursor
   int sg = lo, lu = u0 - uoff[lo], send = uoff[lo + 1];
   uint32_t bfr[C::RC];
-  float dsc[C::NT];
+  float dsc[C::NT];                                   // hot: descale
+  float uk[C::NT], ck[C::NT], uq[C::NT], cq[C::NT];  // cold: fixed-point units and constants
   float mrun[C::NT], lrun[C::NT];
   float oacc[C::KS][4];
   auto load_segment = [&]() {
@@ -554,13 +623,20 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
       for (int r = 0; r < C::RH; ++r)
         bfr[r] = p.w.frag_h[(static_cast<size_t>(bh) * C::RH + r) * 32 + lane];
     }
+    const float* ds = p.w.desc + static_cast<size_t>(bh) * DESC_N * 8;
 #pragma unroll
     for (int nt = 0; nt < C::NT; ++nt) {
       const int h = c + 4 * nt;
-      dsc[nt] = (h < G) ? p.w.desc[(static_cast<size_t>(bh) * 2 + dom) * 8 + h] : 0.0f;
+      const bool in = h < G;
+      dsc[nt] = in ? ds[DS_HOT * 8 + h] : 0.0f;
+      uk[nt] = in ? ds[DS_UK * 8 + h] : 0.0f;
+      ck[nt] = in ? ds[DS_CK * 8 + h] : 0.0f;
+      uq[nt] = in ? ds[DS_UQ * 8 + h] : 0.0f;
+      cq[nt] = in ? ds[DS_CQ * 8 + h] : 0.0f;
       mrun[nt] = NEG_INF;
       lrun[nt] = 0.0f;
     }
+    (void)dom;
 #pragma unroll
     for (int i = 0; i < C::KS; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.0f;
   };
@@ -676,7 +752,10 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
       const __half* kn = reinterpret_cast<const __half*>(sb + C::OFF_N + hoff);
       const uint16_t* kg = reinterpret_cast<const uint16_t*>(sb + C::OFF_N + 2 * TQ_PAGE_TOKENS + hoff);
       const __half* vn = reinterpret_cast<const __half*>(sb + C::OFF_N + 4 * TQ_PAGE_TOKENS + hoff);
-      const int qword = (c * (D / 8)) >> 4, qsb = (c * (D / 8)) & 15;
+      // lane c's QJL word and the first bit position it reads in each byte
+      constexpr int LPW = 4 / C::KK;
+      const int qword = c / LPW, qbase = (c % LPW) * (8 / LPW);
+      constexpr uint32_t M8 = 0x01010101u;
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
         const int t0 = 16 * mt + g, t1 = t0 + 8;
@@ -688,45 +767,54 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         }
         const uint32_t qw0 = *reinterpret_cast<const uint32_t*>(sb + C::OFF_QS + t0 * (D / 8) + 4 * qword);
         const uint32_t qw1 = *reinterpret_cast<const uint32_t*>(sb + C::OFF_QS + t1 * (D / 8) + 4 * qword);
-        const uint32_t gg0 = static_cast<uint32_t>(kg[t0]) * 0x10001u;
-        const uint32_t gg1 = static_cast<uint32_t>(kg[t1]) * 0x10001u;
-        // two independent accumulation chains (key plane, QJL plane)
-        float acc[C::NT][4], acq[C::NT][4];
+        // integer accumulators: key planes (s, m, s m) and the QJL plane
+        int dk[C::NT][4], dq[C::NT][4];
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][e] = acq[nt][e] = 0.0f;
+          for (int e = 0; e < 4; ++e) dk[nt][e] = dq[nt][e] = 0;
 #pragma unroll
-        for (int s = 0; s < C::KS; ++s) {
-          const int w = s >> 2, sh = 4 * (s & 3);
-          const uint32_t x0a = kw0[w] << sh, x0b = kw0[w] << (sh + 1);
-          const uint32_t x1a = kw1[w] << sh, x1b = kw1[w] << (sh + 1);
-          // key plane: sign bit at 15 / 31, magnitude bit at 13 / 29 -> +-b or +-a
-          const uint32_t a0 = key_plane_pair(x0a, p.key_d7, p.key_b2);
-          const uint32_t a1 = key_plane_pair(x1a, p.key_d7, p.key_b2);
-          const uint32_t a2 = key_plane_pair(x0b, p.key_d7, p.key_b2);
-          const uint32_t a3 = key_plane_pair(x1b, p.key_d7, p.key_b2);
-          const int sq = qsb + 2 * s;
-          const uint32_t q0 = ((qw0 << sq) & 0x80008000u) | gg0;
-          const uint32_t q1 = ((qw1 << sq) & 0x80008000u) | gg1;
-          const uint32_t q2 = ((qw0 << (sq + 1)) & 0x80008000u) | gg0;
-          const uint32_t q3 = ((qw1 << (sq + 1)) & 0x80008000u) | gg1;
+        for (int kap = 0; kap < C::KK; ++kap) {
+          // A operands: bit p of every byte of a code word, as 0/1 bytes
+          const int ga = 2 * kap, gb = 2 * kap + 1;
+          const int pa = sign_pos(ga), pb = sign_pos(gb);
+          const uint32_t xa0 = kw0[ga >> 2] >> pa, xa1 = kw1[ga >> 2] >> pa;
+          const uint32_t xb0 = kw0[gb >> 2] >> pb, xb1 = kw1[gb >> 2] >> pb;
+          const uint32_t ya0 = kw0[ga >> 2] >> (pa - 2), ya1 = kw1[ga >> 2] >> (pa - 2);
+          const uint32_t yb0 = kw0[gb >> 2] >> (pb - 2), yb1 = kw1[gb >> 2] >> (pb - 2);
 #pragma unroll
           for (int nt = 0; nt < C::NT; ++nt) {
-            mma_f16(acc[nt], a0, a1, a2, a3, bfr[(s * C::NT + nt) * 2], bfr[(s * C::NT + nt) * 2 + 1]);
-            mma_f16(acq[nt], q0, q1, q2, q3, bfr[((C::KS + s) * C::NT + nt) * 2],
-                    bfr[((C::KS + s) * C::NT + nt) * 2 + 1]);
+            const uint32_t* bs = bfr + ((0 * C::KK + kap) * C::NT + nt) * 2;
+            const uint32_t* bm = bfr + ((1 * C::KK + kap) * C::NT + nt) * 2;
+            const uint32_t* bsm = bfr + ((2 * C::KK + kap) * C::NT + nt) * 2;
+            imma_u8s8(dk[nt], xa0 & M8, xa1 & M8, xb0 & M8, xb1 & M8, bs[0], bs[1]);
+            imma_u8s8(dk[nt], ya0 & M8, ya1 & M8, yb0 & M8, yb1 & M8, bm[0], bm[1]);
+            imma_u8s8(dk[nt], xa0 & ya0 & M8, xa1 & ya1 & M8, xb0 & yb0 & M8, xb1 & yb1 & M8, bsm[0],
+                      bsm[1]);
           }
         }
 #pragma unroll
-        for (int nt = 0; nt < C::NT; ++nt)
+        for (int kap = 0; kap < C::KK; ++kap) {
+          const int pq = qbase + 2 * kap;
+          const uint32_t q0 = (qw0 >> pq) & M8, q1 = (qw1 >> pq) & M8;
+          const uint32_t q2 = (qw0 >> (pq + 1)) & M8, q3 = (qw1 >> (pq + 1)) & M8;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][e] += acq[nt][e];
+          for (int nt = 0; nt < C::NT; ++nt) {
+            const uint32_t* bq = bfr + ((3 * C::KK + kap) * C::NT + nt) * 2;
+            imma_u8s8(dq[nt], q0, q1, q2, q3, bq[0], bq[1]);
+          }
+        }
         const float n0 = __half2float(kn[t0]), n1 = __half2float(kn[t1]);
+        const float gm0 = __half2float(__ushort_as_half(kg[t0])), gm1 = __half2float(__ushort_as_half(kg[t1]));
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt) {
-          const float v0 = (acc[nt][0] + acc[nt][1]) * dsc[nt] * n0;
-          const float v1 = (acc[nt][2] + acc[nt][3]) * dsc[nt] * n1;
+          // columns 2c, 2c+1: the hi and lo bytes of head c's weights
+          const float vk0 = static_cast<float>(dk[nt][0] * 256 + dk[nt][1]);
+          const float vk1 = static_cast<float>(dk[nt][2] * 256 + dk[nt][3]);
+          const float vq0 = static_cast<float>(dq[nt][0] * 256 + dq[nt][1]);
+          const float vq1 = static_cast<float>(dq[nt][2] * 256 + dq[nt][3]);
+          const float v0 = fmaf(gm0, fmaf(uq[nt], vq0, cq[nt]), fmaf(uk[nt], vk0, ck[nt])) * n0;
+          const float v1 = fmaf(gm1, fmaf(uq[nt], vq1, cq[nt]), fmaf(uk[nt], vk1, ck[nt])) * n1;
           sv[nt * 8 + 2 * mt] = (t0 < nv) ? v0 : NEG_INF;
           sv[nt * 8 + 2 * mt + 1] = (t1 < nv) ? v1 : NEG_INF;
         }
@@ -973,7 +1061,7 @@ WsLayout ws_layout(int B, int Hkv, int Wtot) {
   L.frag_h = off;
   off = align256(off + sizeof(uint32_t) * BH * C::RH * 32);
   L.desc = off;
-  off = align256(off + sizeof(float) * BH * 16);
+  off = align256(off + sizeof(float) * BH * DESC_N * 8);
   L.part = off;
   off = align256(off + sizeof(float) * (static_cast<size_t>(Wtot) + S) * G * (D + 2));
   L.total = off;
@@ -1105,11 +1193,8 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
   p.rot = ctx->dev.rot;
   p.qjl = ctx->dev.qjl;
   p.sp = ctx->dev.sp;
-  KeyPlane kp;
-  if (!key_plane(ctx->cb.key_c[0], ctx->cb.key_c[1], kp)) return TQ_ERR_UNSUPPORTED;
-  p.w_key = static_cast<float>(ctx->cb.key_c[0] / kp.b);
-  p.key_b2 = kp.b2;
-  p.key_d7 = kp.d7;
+  p.kc0 = ctx->cb.key_c[0];
+  p.kc1 = ctx->cb.key_c[1];
   p.alpha = std::sqrt(3.14159265358979323846f / 2.0f) / static_cast<float>(ctx->cfg.qjl_dim);
   for (int k = 0; k < 8; ++k) p.vc[k] = ctx->cb.val_c[k];
   p.err = ctx->dev.err;
