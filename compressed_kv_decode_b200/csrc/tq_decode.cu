@@ -238,77 +238,43 @@ __device__ __forceinline__ float prescale_for(float mx) {
   return ldexpf(1.0f, 8 - e);
 }
 
-// y[g][r] = sum_k M[r][k] x[g][k] for all rows r of a D x D matrix: one warp
-// per row, each lane a float4 of the row (coalesced), reduced by shuffles;
-// every row's load is independent, so the L2 latency overlaps.
+// y1[g][r] = sum_k M1[r][k] x[g][k] and y2 = M2 x, for all rows r of two
+// D x D matrices.  Four lanes share a row: lane qq of the four takes the
+// float4 chunks qq, qq + 4, ... of the row (coalesced row reads, conflict-free
+// reads of x), so a row costs its FMAs plus a two-step shuffle reduction.
+// All row loads of a pass are issued before any arithmetic.
 constexpr int PREP_WARPS = 8;
 
 template <int D, int G>
-__device__ __forceinline__ void matvec_rows(const float* __restrict__ M, const float (*x)[D],
-                                            float (*y)[D]) {
-  constexpr int LANES = D / 4;  // lanes holding one row
-  constexpr int ROWS_PER_PASS = 32 / LANES;
-  constexpr int PASSES = D / (PREP_WARPS * ROWS_PER_PASS);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane / LANES, l4 = lane % LANES;
-  float4 mrow[PASSES];  // every row this lane needs, requested at once
-#pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps) {
-    const int r = (ps * PREP_WARPS + warp) * ROWS_PER_PASS + sub;
-    mrow[ps] = __ldg(reinterpret_cast<const float4*>(M + static_cast<size_t>(r) * D) + l4);
-  }
-#pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps) {
-    const int r = (ps * PREP_WARPS + warp) * ROWS_PER_PASS + sub;
-    const float4 m = mrow[ps];
-    float acc[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      acc[g] = m.x * x[g][4 * l4] + m.y * x[g][4 * l4 + 1] + m.z * x[g][4 * l4 + 2] +
-               m.w * x[g][4 * l4 + 3];
-#pragma unroll
-      for (int o = LANES / 2; o > 0; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
-    }
-    if (l4 == 0) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) y[g][r] = acc[g];
-    }
-  }
-}
-
-// y1 = M1 x and y2 = M2 x together: every row load of both is issued first
-template <int D, int G>
 __device__ __forceinline__ void matvec_rows2(const float* __restrict__ M1, const float* __restrict__ M2,
                                              const float (*x)[D], float (*y1)[D], float (*y2)[D]) {
-  constexpr int LANES = D / 4;
-  constexpr int ROWS_PER_PASS = 32 / LANES;
-  constexpr int PASSES = D / (PREP_WARPS * ROWS_PER_PASS);
+  constexpr int CH = D / 16;                             // float4 chunks per lane and row
+  constexpr int ROWS_PER_PASS = PREP_WARPS * 8;          // 8 rows per warp
+  constexpr int PASSES = D / ROWS_PER_PASS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane / LANES, l4 = lane % LANES;
-  float4 mrow[2][PASSES];
-#pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps) {
-    const int r = (ps * PREP_WARPS + warp) * ROWS_PER_PASS + sub;
-    mrow[0][ps] = __ldg(reinterpret_cast<const float4*>(M1 + static_cast<size_t>(r) * D) + l4);
-    mrow[1][ps] = __ldg(reinterpret_cast<const float4*>(M2 + static_cast<size_t>(r) * D) + l4);
-  }
+  const int qq = lane & 3, rsub = lane >> 2;
 #pragma unroll
   for (int w = 0; w < 2; ++w) {
+    const float* M = w == 0 ? M1 : M2;
+    float (*y)[D] = w == 0 ? y1 : y2;
 #pragma unroll
     for (int ps = 0; ps < PASSES; ++ps) {
-      const int r = (ps * PREP_WARPS + warp) * ROWS_PER_PASS + sub;
-      const float4 m = mrow[w][ps];
-      float acc[G];
+      const int r = ps * ROWS_PER_PASS + warp * 8 + rsub;
+      float4 m[CH];
+#pragma unroll
+      for (int i = 0; i < CH; ++i)
+        m[i] = __ldg(reinterpret_cast<const float4*>(M + static_cast<size_t>(r) * D) + qq + 4 * i);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        acc[g] = m.x * x[g][4 * l4] + m.y * x[g][4 * l4 + 1] + m.z * x[g][4 * l4 + 2] +
-                 m.w * x[g][4 * l4 + 3];
+        float acc = 0.0f;
 #pragma unroll
-        for (int o = LANES / 2; o > 0; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
-      }
-      if (l4 == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) (w == 0 ? y1 : y2)[g][r] = acc[g];
+        for (int i = 0; i < CH; ++i) {
+          const float4 xv = reinterpret_cast<const float4*>(x[g])[qq + 4 * i];
+          acc = fmaf(m[i].x, xv.x, fmaf(m[i].y, xv.y, fmaf(m[i].z, xv.z, fmaf(m[i].w, xv.w, acc))));
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (qq == 0) y[g][r] = acc;
       }
     }
   }
@@ -324,7 +290,7 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
     return;
   }
   const int bh = blockIdx.x, b = bh / p.Hkv, kvh = bh % p.Hkv;
-  __shared__ float sq[G][D], sqr[G][D], sqs[G][D];
+  __shared__ __align__(16) float sq[G][D], sqr[G][D], sqs[G][D];
   __shared__ unsigned smax[2][G];
   __shared__ float sfac[2][G];
   const int tid = threadIdx.x;
@@ -345,7 +311,7 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   // One fixed-point unit per head for the three key planes, one for the QJL plane.
   const float ck0 = p.kc0, dk1 = p.kc1 - p.kc0;
   __shared__ unsigned smr[G], sms[G];
-  __shared__ float s_uk[G], s_uq[G];
+  __shared__ float s_uk[G], s_uq[G];  // reciprocals of the fixed-point units
   if (tid < G) smr[tid] = sms[tid] = 0u;
   __syncthreads();
   for (int i = tid; i < G * D; i += blockDim.x) {
@@ -372,8 +338,8 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
         const float mr = __uint_as_float(smr[wp]), ms = __uint_as_float(sms[wp]);
         const float uk = mr > 0.0f ? 2.0f * fmaxf(ck0, dk1) * mr / FIX_MAX : 1.0f;
         const float uq = ms > 0.0f ? 2.0f * p.alpha * ms / FIX_MAX : 1.0f;
-        s_uk[wp] = uk;
-        s_uq[wp] = uq;
+        s_uk[wp] = 1.0f / uk;
+        s_uq[wp] = 1.0f / uq;
         float* ds = p.w.desc + static_cast<size_t>(bh) * DESC_N * 8;
         ds[DS_UK * 8 + wp] = p.sl * uk;
         ds[DS_CK * 8 + wp] = p.sl * ck0 * a;
@@ -412,12 +378,12 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
           const int coord = 16 * (cc * C::WPT + (gam >> 2)) + 8 * hh + 2 * (rem >> 2) + (rem & 1);
           const float w = plane == 0 ? -2.0f * ck0 * sqr[h][coord]
                         : plane == 1 ? dk1 * sqr[h][coord] : -2.0f * dk1 * sqr[h][coord];
-          qv = w / s_uk[h];
+          qv = w * s_uk[h];
         } else {
           const int pq = (cc % LPW) * (8 / LPW) + 2 * kap + reg;
           const int beta = 8 * j + pq, hh = beta >> 4, rr = 15 - (beta & 15);
           const int si = 32 * (cc / LPW) + 16 * hh + rr;
-          qv = -2.0f * p.alpha * sqs[h][si] / s_uq[h];
+          qv = -2.0f * p.alpha * sqs[h][si] * s_uq[h];
         }
         const int q16 = max(-32511, min(32511, __float2int_rn(qv)));
         const int lo = ((q16 + 128) & 255) - 128, hi = (q16 - lo) >> 8;
