@@ -475,8 +475,9 @@ __host__ __device__ constexpr int sign_pos(int gam) {
 __device__ __forceinline__ void dequant_values(uint32_t x, uint32_t tl0, uint32_t tl1,
                                                uint32_t th0, uint32_t th1, uint32_t (&h)[4]) {
   const uint32_t x4 = x << 4;
-  const uint32_t s01 = x & 0x7777u;
-  const uint32_t s23 = (x >> 16) & 0x7777u;
+  // magnitude selectors (prmt reads the low 16 bits of its selector)
+  const uint32_t s01 = x & 0x77777777u;
+  const uint32_t s23 = s01 >> 16;
   const uint32_t lo01 = prmt(tl0, tl1, s01), hi01 = prmt(th0, th1, s01);
   const uint32_t lo23 = prmt(tl0, tl1, s23), hi23 = prmt(th0, th1, s23);
   // sign bits of the 8 nibbles as 0x00 / 0xFF bytes (prmt sign replication)
