@@ -285,24 +285,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float rr[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
+          // computed as for n > 0; a zero vector's row is cleared below
           const int i = 8 * c8 + 2 * e2 + e;  // column within the half
           const float v = x[i];
-          const uint32_t sg = (n > 0.0f && v < 0.0f) ? 1u : 0u;
-          const uint32_t mg = (n > 0.0f && fabsf(v) >= T0) ? 1u : 0u;
-          const float cp = mg ? p.kc1 : p.kc0;
-          const float r = (n > 0.0f) ? fmaf(v, inv, (v < 0.0f) ? cp : -cp) : 0.0f;
+          const bool neg = v < 0.0f, big = fabsf(v) >= T0;
+          const float cp = big ? p.kc1 : p.kc0;
+          const float r = fmaf(v, inv, neg ? cp : -cp);
           rr[e] = r;
           g2 = fmaf(r, r, g2);
-          const int j = h * C::HALF + i;  // coordinate
-          const int jj = j & 15, hh = jj >> 3, ii = (jj & 7) >> 1, ee = jj & 1;
+          const int jj = i & 15, hh = jj >> 3, ii = (jj & 7) >> 1, ee = jj & 1;  // halves are 16-aligned
           const int sbit = 16 * hh + 15 - 4 * ii - ee;
-          kw[i >> 4] |= (sg << sbit) | (mg << (sbit - 2));
+          if (neg) kw[i >> 4] |= 1u << sbit;
+          if (big) kw[i >> 4] |= 1u << (sbit - 2);
         }
-        const __half2 pr = __floats2half2_rn(rr[0], rr[1]);
+        const __half2 pr = __floats2half2_rn(n > 0.0f ? rr[0] : 0.0f, n > 0.0f ? rr[1] : 0.0f);
         rh[e2] = *reinterpret_cast<const uint32_t*>(&pr);
       }
       *reinterpret_cast<uint4*>(smem + C::OFF_R + tc::sw128_offset(row, h * C::HALF + 8 * c8, ROWS)) =
           make_uint4(rh[0], rh[1], rh[2], rh[3]);
+    }
+    if (!(n > 0.0f)) {  // zero vector: all codes and the residual norm are 0
+#pragma unroll
+      for (int w = 0; w < C::HALF / 16; ++w) kw[w] = 0u;
+      g2 = 0.0f;
     }
     gp[h * ROWS + row] = g2;
     fence_proxy_async_smem();  // residual tile visible to the tensor cores
@@ -350,7 +355,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int i = 0; i < C::HALF; ++i) {
         const int within = i & 31;  // sketch index inside its 32-bit word
         const int bit = 16 * (within >> 4) + 15 - (within & 15);
-        if (n > 0.0f && x[i] < 0.0f) qw[i >> 5] |= 1u << bit;
+        if (x[i] < 0.0f) qw[i >> 5] |= 1u << bit;
+      }
+      if (!(n > 0.0f)) {  // zero vector
+#pragma unroll
+        for (int w = 0; w < C::HALF / 32; ++w) qw[w] = 0u;
       }
       if (wr) {
         if constexpr (C::HALF / 32 == 2)
@@ -388,8 +397,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint32_t mg = 0u;
 #pragma unroll
         for (int k = 0; k < 7; ++k) mg += (fabsf(x[i]) >= T[k]) ? 1u : 0u;
-        const uint32_t code = (vn > 0.0f) ? (((x[i] < 0.0f) ? 8u : 0u) | mg) : 0u;
+        const uint32_t code = ((x[i] < 0.0f) ? 8u : 0u) | mg;
         cw[i >> 3] |= code << (4 * (i & 7));
+      }
+      if (!(vn > 0.0f)) {  // zero vector
+#pragma unroll
+        for (int w = 0; w < C::HALF / 8; ++w) cw[w] = 0u;
       }
       const bool even = (row & 1) == 0;
       uint32_t ow[C::HALF / 8];
