@@ -253,10 +253,12 @@ def decode(tq, st, q=None, out=None):
 
 
 def reduce_max(torch, x, world):
+    """The maximum of x over ranks (a time: the slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
