@@ -63,6 +63,11 @@ def lib():
                                    dp, C.c_double, dp, dp, C.c_int, ip, u8, sz, ip, C.c_int, ip,
                                    ip, C.c_int, dp, C.c_int]
         L.or_attention.restype = C.c_int
+        L.or_attention_gated.argtypes = [C.c_int, C.c_int, dp, dp, dp, dp, C.c_int, C.c_int,
+                                         C.c_int, dp, C.c_double, dp, dp, C.c_int, ip, u8, sz, ip,
+                                         C.c_int, ip, ip, C.c_int, C.c_int, C.c_double, ip, dp,
+                                         C.c_int]
+        L.or_attention_gated.restype = C.c_int
         L.or_topk.argtypes = [C.c_int, C.c_int, dp, dp, dp, dp, C.c_int, u8, sz, C.c_int64,
                               C.c_int, ip, dp, C.c_int]
         L.or_max_threads.restype = C.c_int
@@ -271,10 +276,12 @@ def qjl_montecarlo(q, r, trials, seed0):
 # attention and search
 # --------------------------------------------------------------------------
 def attention(params, q, Hkv, scale, k_hot, v_hot, hot_len, pool, page_bytes, page_table,
-              cold_len, groups=None, threads=0):
+              cold_len, groups=None, threads=0, threshold=None):
     """q [B, Hq, d]; k_hot/v_hot [B, Hkv, W, d] or None; hot_len, cold_len [B];
     page_table [B, Hkv, max_pages].  groups: list of (b, kv_head) or None=all.
-    Returns out [len(groups), G, d] (fp64) and the group list."""
+    Returns out [len(groups), G, d] (fp64) and the group list.  With a
+    threshold, a head reads its cold tokens only when its largest raw hot
+    score is below it, and the result is (out, groups, open [len(groups), G])."""
     p = params
     q, qp = _d(q)
     B, Hq, d = q.shape
@@ -300,11 +307,20 @@ def attention(params, q, Hkv, scale, k_hot, v_hot, hot_len, pool, page_bytes, pa
     out = np.empty((len(groups), G, d))
     if pool is None:
         pool = np.zeros(16, np.uint8)
-    rc = lib().or_attention(d, p.m, pip, Sp, kcp, vcp, B, Hq, Hkv, qp, scale, khp, vhp, W, hlp,
-                            _u8(pool), page_bytes, ptp, max_pages, clp, selp, len(groups),
-                            out.ctypes.data_as(C.POINTER(C.c_double)), threads)
+    if threshold is None:
+        rc = lib().or_attention(d, p.m, pip, Sp, kcp, vcp, B, Hq, Hkv, qp, scale, khp, vhp, W,
+                                hlp, _u8(pool), page_bytes, ptp, max_pages, clp, selp,
+                                len(groups), out.ctypes.data_as(C.POINTER(C.c_double)), threads)
+        assert rc == 0
+        return out, groups
+    opened = np.empty((len(groups), G), np.int32)
+    rc = lib().or_attention_gated(d, p.m, pip, Sp, kcp, vcp, B, Hq, Hkv, qp, scale, khp, vhp, W,
+                                  hlp, _u8(pool), page_bytes, ptp, max_pages, clp, selp,
+                                  len(groups), 1, float(threshold),
+                                  opened.ctypes.data_as(C.POINTER(C.c_int32)),
+                                  out.ctypes.data_as(C.POINTER(C.c_double)), threads)
     assert rc == 0
-    return out, groups
+    return out, groups, opened
 
 
 def topk(params, queries, db_pool, page_bytes, N, k, threads=0):

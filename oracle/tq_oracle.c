@@ -689,12 +689,21 @@ static double key_score(int d, int m, const double* qrot, const double* sq, cons
 /* v_hat = n_v Pi^T c_hat_v) followed by hot tokens (exact fp16 keys and     */
 /* values).  Two-pass softmax.  q: [G, d]; out: [G, d].                      */
 /* ------------------------------------------------------------------------ */
+/*
+ * Threshold gate [MON "Vereinfachte Decode-Schleife": the cold pages are
+ * decompressed and scored only if max(scores_hot) < threshold].  Reading: the
+ * test is taken per query head on the raw hot scores <q, k_t> (the product
+ * q @ kv_hot.T as written, no softmax scale); with no hot tokens the maximum
+ * is -inf.  A head whose test fails attends to its hot tokens alone.  With
+ * gated = 0 every head reads the cold tokens.  open (may be NULL) receives
+ * per head 1 if it read the cold tokens, else 0.
+ */
 OR_API int or_attention_group(int d, int m, const double* pi, const double* S,
                               const double* kcpos, const double* vcpos, int G,
                               const double* q, double scale, const double* k_hot,
                               const double* v_hot, int hot_len, const uint8_t* pool,
                               size_t page_bytes, const int32_t* pages, int cold_len,
-                              double* out) {
+                              int gated, double threshold, int32_t* open, double* out) {
   int nt = cold_len + hot_len;
   double* logits = (double*)malloc(sizeof(double) * (size_t)G * (nt > 0 ? nt : 1));
   double* vals = (double*)malloc(sizeof(double) * (size_t)(nt > 0 ? nt : 1) * d);
@@ -749,12 +758,23 @@ OR_API int or_attention_group(int d, int m, const double* pi, const double* S,
   for (int h = 0; h < G; ++h) {
     double* o = out + (size_t)h * d;
     for (int j = 0; j < d; ++j) o[j] = 0.0;
-    if (nt == 0) continue; /* no tokens: output defined as zero */
+    int first = 0; /* first token of the softmax: 0, or cold_len when the gate is shut */
+    if (gated) {
+      double hmax = -INFINITY;
+      for (int t = 0; t < hot_len; ++t) {
+        double a = 0.0;
+        for (int j = 0; j < d; ++j) a += q[(size_t)h * d + j] * k_hot[(size_t)t * d + j];
+        hmax = fmax(hmax, a);
+      }
+      if (!(hmax < threshold)) first = cold_len;
+    }
+    if (open) open[h] = (first == 0) ? 1 : 0;
+    if (nt - first == 0) continue; /* no tokens: output defined as zero */
     double mx = -INFINITY;
-    for (int t = 0; t < nt; ++t) mx = fmax(mx, logits[(size_t)h * nt + t]);
+    for (int t = first; t < nt; ++t) mx = fmax(mx, logits[(size_t)h * nt + t]);
     double den = 0.0;
-    for (int t = 0; t < nt; ++t) den += exp(logits[(size_t)h * nt + t] - mx);
-    for (int t = 0; t < nt; ++t) {
+    for (int t = first; t < nt; ++t) den += exp(logits[(size_t)h * nt + t] - mx);
+    for (int t = first; t < nt; ++t) {
       double p = exp(logits[(size_t)h * nt + t] - mx) / den;
       for (int j = 0; j < d; ++j) o[j] += p * vals[(size_t)t * d + j];
     }
@@ -768,14 +788,17 @@ OR_API int or_attention_group(int d, int m, const double* pi, const double* S,
  * Batched driver: groups listed in sel (pairs b, kv_head); the q heads of
  * kv head h are h*G .. h*G+G-1 (contiguous grouping).  Layouts:
  * q [B, Hq, d]; k_hot, v_hot [B, Hkv, W, d]; page_table [B, Hkv, max_pages];
- * out [nsel, G, d].
+ * out [nsel, G, d]; open (may be NULL) [nsel, G].  gated, threshold: the
+ * threshold gate of or_attention_group.
  */
-OR_API int or_attention(int d, int m, const double* pi, const double* S, const double* kcpos,
-                        const double* vcpos, int B, int Hq, int Hkv, const double* q,
-                        double scale, const double* k_hot, const double* v_hot, int W,
-                        const int32_t* hot_len, const uint8_t* pool, size_t page_bytes,
-                        const int32_t* page_table, int max_pages, const int32_t* cold_len,
-                        const int32_t* sel, int nsel, double* out, int threads) {
+OR_API int or_attention_gated(int d, int m, const double* pi, const double* S,
+                              const double* kcpos, const double* vcpos, int B, int Hq, int Hkv,
+                              const double* q, double scale, const double* k_hot,
+                              const double* v_hot, int W, const int32_t* hot_len,
+                              const uint8_t* pool, size_t page_bytes, const int32_t* page_table,
+                              int max_pages, const int32_t* cold_len, const int32_t* sel, int nsel,
+                              int gated, double threshold, int32_t* open, double* out,
+                              int threads) {
   int G = Hq / Hkv;
   int err = 0;
 #ifdef _OPENMP
@@ -790,10 +813,23 @@ OR_API int or_attention(int d, int m, const double* pi, const double* S, const d
     int cl = cold_len ? cold_len[b] : 0;
     err |= or_attention_group(d, m, pi, S, kcpos, vcpos, G, q + ((size_t)b * Hq + (size_t)h * G) * d,
                               scale, kh, vh, hl, pool, page_bytes,
-                              page_table + ((size_t)b * Hkv + h) * max_pages, cl,
+                              page_table + ((size_t)b * Hkv + h) * max_pages, cl, gated,
+                              threshold, open ? open + (size_t)s * G : NULL,
                               out + (size_t)s * G * d);
   }
   return err;
+}
+
+/* The ungated form: every head reads hot and cold tokens. */
+OR_API int or_attention(int d, int m, const double* pi, const double* S, const double* kcpos,
+                        const double* vcpos, int B, int Hq, int Hkv, const double* q,
+                        double scale, const double* k_hot, const double* v_hot, int W,
+                        const int32_t* hot_len, const uint8_t* pool, size_t page_bytes,
+                        const int32_t* page_table, int max_pages, const int32_t* cold_len,
+                        const int32_t* sel, int nsel, double* out, int threads) {
+  return or_attention_gated(d, m, pi, S, kcpos, vcpos, B, Hq, Hkv, q, scale, k_hot, v_hot, W,
+                            hot_len, pool, page_bytes, page_table, max_pages, cold_len, sel, nsel,
+                            0, 0.0, NULL, out, threads);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -153,3 +153,77 @@ def test_topk_ties_go_to_lower_id(O):
     ids, sc = O.topk(P, rng.standard_normal((2, d)), pool, nbytes, N, 5)
     assert np.array_equal(ids, np.tile(np.arange(5), (2, 1)))
     assert np.all(sc == sc[:, :1])
+
+
+@pytest.mark.parametrize("d,G", [(64, 8), (128, 4)])
+def test_threshold_gate_selects_hot_only_or_hot_and_cold(O, d, G):
+    """Monarch's gate ("Vereinfachte Decode-Schleife"): a head reads its cold
+    tokens only when max_t <q, k_hot_t> is below the threshold.  With exact
+    (zero-residual) records the gated result must be textbook attention over
+    either hot or hot + cold, per head, decided by a numpy matmul of q with
+    the hot keys; the threshold sits between the raw maxima so that both
+    outcomes occur and a scaled-score gate would give a different split."""
+    m = d
+    P = O.Params(d, seed=5)
+    rng = np.random.default_rng(100 + d + G)
+    B, Hkv = 3, 2
+    Hq = G * Hkv
+    max_pages = 3
+    nbytes, _ = O.page_layout(d, m, True)
+    n_pages = B * Hkv * max_pages
+    pool = np.zeros(n_pages * nbytes, np.uint8)
+    table = rng.permutation(n_pages).astype(np.int32).reshape(B, Hkv, max_pages)
+    W = 70
+    k_hot = np.float16(rng.standard_normal((B, Hkv, W, d))).astype(np.float64)
+    v_hot = np.float16(rng.standard_normal((B, Hkv, W, d))).astype(np.float64)
+    q = rng.standard_normal((B, Hq, d))
+    cold_len = np.array([300, 129, 5], np.int32)
+    hot_len = np.array([70, 0, 33], np.int32)
+    recs = {}
+    for b in range(B):
+        for h in range(Hkv):
+            n = int(cold_len[b])
+            rec = _direct_records(rng, n, d, m)
+            t = np.arange(n)
+            O.pack(pool, nbytes, d, m, True, table[b, h, t // 128], t % 128, rec)
+            recs[b, h] = rec
+    scale = 1.0 / math.sqrt(d)
+    hmax = np.full((B, Hq), -np.inf)
+    for b in range(B):
+        for hq in range(Hq):
+            if hot_len[b]:
+                hmax[b, hq] = (k_hot[b, hq // G, :hot_len[b]] @ q[b, hq]).max()
+    finite = np.sort(hmax[np.isfinite(hmax)])
+    thr = 0.5 * (finite[len(finite) // 2 - 1] + finite[len(finite) // 2])
+    out, groups, opened = O.attention(P, q, Hkv, scale, k_hot, v_hot, hot_len, pool, nbytes,
+                                      table, cold_len, threshold=thr)
+    want_open = hmax < thr
+    assert want_open.any() and (~want_open[np.isfinite(hmax)]).any()
+    assert (hmax * scale < thr).sum() != want_open.sum()  # the scale matters for this threshold
+    for gi, (b, h) in enumerate(groups):
+        Kc, Vc = _reconstruct(P, recs[b, h])
+        Kh, Vh = k_hot[b, h, :hot_len[b]], v_hot[b, h, :hot_len[b]]
+        for g in range(G):
+            hq = h * G + g
+            assert opened[gi, g] == int(want_open[b, hq])
+            K = np.concatenate([Kc, Kh]) if want_open[b, hq] else Kh
+            V = np.concatenate([Vc, Vh]) if want_open[b, hq] else Vh
+            ref = np.zeros(d) if len(K) == 0 else _sdpa(q[b, hq][None], K, V, scale)[0]
+            assert np.abs(out[gi, g] - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
+    # +inf opens every head: the ungated result; -inf shuts every head: hot
+    # tokens alone, zeros where there are none
+    ung, _ = O.attention(P, q, Hkv, scale, k_hot, v_hot, hot_len, pool, nbytes, table, cold_len)
+    out_inf, _, op_inf = O.attention(P, q, Hkv, scale, k_hot, v_hot, hot_len, pool, nbytes,
+                                     table, cold_len, threshold=np.inf)
+    assert op_inf.all() and np.array_equal(out_inf, ung)
+    out_ninf, _, op_ninf = O.attention(P, q, Hkv, scale, k_hot, v_hot, hot_len, pool, nbytes,
+                                       table, cold_len, threshold=-np.inf)
+    assert not op_ninf.any()
+    for gi, (b, h) in enumerate(groups):
+        for g in range(G):
+            if hot_len[b] == 0:
+                assert not out_ninf[gi, g].any()
+            else:
+                ref = _sdpa(q[b, h * G + g][None], k_hot[b, h, :hot_len[b]],
+                            v_hot[b, h, :hot_len[b]], scale)[0]
+                assert np.abs(out_ninf[gi, g] - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
