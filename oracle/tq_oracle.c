@@ -696,7 +696,8 @@ static double key_score(int d, int m, const double* qrot, const double* sq, cons
  * q @ kv_hot.T as written, no softmax scale); with no hot tokens the maximum
  * is -inf.  A head whose test fails attends to its hot tokens alone.  With
  * gated = 0 every head reads the cold tokens.  open (may be NULL) receives
- * per head 1 if it read the cold tokens, else 0.
+ * per head the gate's decision: 1 if the head reads its cold tokens (whether
+ * or not there are any), else 0.
  */
 OR_API int or_attention_group(int d, int m, const double* pi, const double* S,
                               const double* kcpos, const double* vcpos, int G,
@@ -758,7 +759,7 @@ OR_API int or_attention_group(int d, int m, const double* pi, const double* S,
   for (int h = 0; h < G; ++h) {
     double* o = out + (size_t)h * d;
     for (int j = 0; j < d; ++j) o[j] = 0.0;
-    int first = 0; /* first token of the softmax: 0, or cold_len when the gate is shut */
+    int is_open = 1;
     if (gated) {
       double hmax = -INFINITY;
       for (int t = 0; t < hot_len; ++t) {
@@ -766,9 +767,10 @@ OR_API int or_attention_group(int d, int m, const double* pi, const double* S,
         for (int j = 0; j < d; ++j) a += q[(size_t)h * d + j] * k_hot[(size_t)t * d + j];
         hmax = fmax(hmax, a);
       }
-      if (!(hmax < threshold)) first = cold_len;
+      is_open = hmax < threshold;
     }
-    if (open) open[h] = (first == 0) ? 1 : 0;
+    if (open) open[h] = is_open; /* the gate's decision, also when there is no cold token */
+    const int first = is_open ? 0 : cold_len; /* first token of the softmax */
     if (nt - first == 0) continue; /* no tokens: output defined as zero */
     double mx = -INFINITY;
     for (int t = first; t < nt; ++t) mx = fmax(mx, logits[(size_t)h * nt + t]);

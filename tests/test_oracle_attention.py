@@ -177,7 +177,7 @@ def test_threshold_gate_selects_hot_only_or_hot_and_cold(O, d, G):
     k_hot = np.float16(rng.standard_normal((B, Hkv, W, d))).astype(np.float64)
     v_hot = np.float16(rng.standard_normal((B, Hkv, W, d))).astype(np.float64)
     q = rng.standard_normal((B, Hq, d))
-    cold_len = np.array([300, 129, 5], np.int32)
+    cold_len = np.array([300, 129, 0], np.int32)
     hot_len = np.array([70, 0, 33], np.int32)
     recs = {}
     for b in range(B):
