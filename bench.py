@@ -133,13 +133,13 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # workload on the device
 # ---------------------------------------------------------------------------
-def build_state(torch, tq, W, rank, batch=None):
-    cfg = W.DECODE[WORKLOAD]
+def build_state(torch, tq, W, rank, batch=None, workload=WORKLOAD):
+    cfg = W.DECODE[workload]
     B, Hq, Hkv, d = batch or cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"]
     cold, hot = cfg["cold"], cfg["hot"]
     dev = torch.device("cuda")
     ctx = tq.Context(d, seed=0)
-    max_pages = cold // 128
+    max_pages = (cold + 127) // 128
     n_pages = B * Hkv * max_pages
     page_bytes = ctx.page_bytes(True)
     gen = torch.Generator(device=dev)
@@ -164,7 +164,7 @@ def build_state(torch, tq, W, rank, batch=None):
     k_hot = kv(hot).to(torch.float16)
     v_hot = kv(hot).to(torch.float16)
     hot_len = torch.full((B,), hot, dtype=torch.int32, device=dev)
-    q = torch.randn((B, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.randn((B, Hq, d), generator=gen, device=dev).to(getattr(torch, cfg["q_dtype"]))
     out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
     ws = ctx.workspace(B, Hq, Hkv, max_pages, hot)
     st = dict(ctx=ctx, pool=pool, table=table, cold_len=cold_len, k_hot=k_hot, v_hot=v_hot,
@@ -244,6 +244,58 @@ def measure_search(torch, tq, reps=3):
     return {"workload": "search_1m (10^6 x 4096 queries, d=128, top-10)",
             "query_vectors_per_s": Q * N / (ms / 1e3), "kernel_ms": ms,
             "achieved_tflops": flops / (ms / 1e3) / 1e12, "algorithmic_flops": flops}
+
+
+def graph_ms(torch, fn, reps=50):
+    """Mean device time of fn (one step) replayed from a CUDA graph."""
+    main = torch.cuda.current_stream()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(main)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        fn()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=cap):
+            fn()
+    main.wait_stream(cap)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(main)
+    for _ in range(reps):
+        g.replay()
+    b.record(main)
+    b.synchronize()
+    del g
+    return a.elapsed_time(b) / reps
+
+
+def gated_decode(tq, st, threshold, used):
+    tq.tq_decode_attention_gated(st["ctx"].handle, st["q"], st["k_hot"], st["v_hot"],
+                                 st["hot_len"], st["pool"], st["table"], st["cold_len"],
+                                 threshold, st["out"], st["ws"], st["Hkv"], cold_used=used)
+
+
+def measure_gated(torch, tq, st, reps=50):
+    """Monarch's threshold gate on a decode state: step time with every head
+    open, every head shut, and the threshold at the median of the per-head
+    raw hot-score maxima (about half the heads read their cold tokens)."""
+    G = st["Hq"] // st["Hkv"]
+    qf = st["q"].float().view(st["B"], st["Hkv"], G, st["d"])
+    hmax = torch.einsum("bhgd,bhtd->bhgt", qf, st["k_hot"].float()).amax(-1).reshape(st["B"], -1)
+    used = torch.empty((st["B"], st["Hq"]), dtype=torch.int32, device=st["q"].device)
+    res = {}
+    for name, thr in (("open", float("inf")), ("median", float(hmax.median())),
+                      ("shut", float("-inf"))):
+        ms = graph_ms(torch, lambda: gated_decode(tq, st, thr, used), reps)
+        u = used.view(st["B"], st["Hkv"], G)
+        res[name] = {"ms_per_step": ms, "threshold": thr,
+                     "heads_reading_cold": float(u.float().mean()),
+                     "groups_reading_cold": float(u.any(-1).float().mean())}
+    res["ungated_ms_per_step"] = graph_ms(torch, lambda: decode(tq, st), reps)
+    st["ctx"].check()
+    return res
 
 
 def decode(tq, st, q=None, out=None):
@@ -416,6 +468,8 @@ def run_ours(args, rank, world, local_rank):
     cb = cpu_baseline() if world == 1 else None
     rows = {}
     if world == 1:
+        rows["gated_decode"] = measure_gated(torch, tq, st)
+        rows["gated_decode"]["workload"] = WORKLOAD + " with Monarch's threshold gate"
         del st, graph
         torch.cuda.empty_cache()
         rows["compress"] = measure_compress(torch, tq)

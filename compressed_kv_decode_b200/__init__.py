@@ -63,6 +63,11 @@ def lib():
                                           vp, vp, C.c_int, i32p, u8p, C.c_int64, i32p, C.c_int,
                                           i32p, f32p, vp, C.c_size_t, vp]
         L.tq_decode_attention.restype = C.c_int
+        L.tq_decode_attention_gated.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int,
+                                                C.c_float, vp, vp, C.c_int, i32p, i32p, u8p,
+                                                C.c_int64, i32p, C.c_int, i32p, C.c_float, i32p,
+                                                f32p, vp, C.c_size_t, vp]
+        L.tq_decode_attention_gated.restype = C.c_int
         L.tq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int,
                                                   C.c_float, vp, vp, C.c_int, i32p, u8p, C.c_int64,
                                                   i32p, C.c_int, i32p, f32p, vp]
@@ -197,6 +202,27 @@ def tq_decode_attention(ctx, q, k_hot, v_hot, hot_len, page_pool, page_table, co
         _ptr(hot_len), _ptr(page_pool), pool_pages, _ptr(page_table), max_pages, _ptr(cold_len),
         _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)), "tq_decode_attention")
+
+
+def tq_decode_attention_gated(ctx, q, k_hot, v_hot, hot_len, page_pool, page_table, cold_len,
+                              threshold, out, workspace, Hkv, scale=0.0, hot_start=None,
+                              cold_used=None, stream=None):
+    """tq_decode_attention with Monarch's threshold gate: a q head reads its
+    cold tokens only when max_t <q, k_hot_t> (raw, fp32) < threshold.
+    hot_start: int32 [B] ring slot of the oldest hot token, or None;
+    cold_used: int32 [B, Hq] out (1 = the head read its cold tokens), or None."""
+    _require_cuda(q, k_hot, v_hot, hot_len, page_pool, page_table, cold_len, out, workspace,
+                  hot_start, cold_used)
+    B, Hq, _ = q.shape
+    W_max = 0 if k_hot is None else k_hot.shape[2]
+    max_pages = 0 if page_table is None else page_table.shape[-1]
+    pool_pages = 0 if page_pool is None else page_pool.shape[0]
+    _check(lib().tq_decode_attention_gated(
+        ctx, _ptr(q), _dtype_code(q), B, Hq, Hkv, float(scale), _ptr(k_hot), _ptr(v_hot), W_max,
+        _ptr(hot_start), _ptr(hot_len), _ptr(page_pool), pool_pages, _ptr(page_table), max_pages,
+        _ptr(cold_len), float(threshold), _ptr(cold_used), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)),
+        "tq_decode_attention_gated")
 
 
 def tq_decode_attention_noalloc(ctx, q, k_hot, v_hot, hot_len, page_pool, page_table, cold_len,

@@ -213,12 +213,14 @@ size_t tq_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pag
   return tq::decode_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max);
 }
 
-tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
-                              int Hkv, float scale, const void* k_hot, const void* v_hot,
-                              int W_max, const int32_t* hot_len, const uint8_t* page_pool,
-                              int64_t pool_pages, const int32_t* page_table, int max_pages,
-                              const int32_t* cold_len, float* out, void* workspace,
-                              size_t ws_bytes, void* stream) {
+namespace {
+
+tq_status decode_common(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                        int Hkv, float scale, const void* k_hot, const void* v_hot, int W_max,
+                        const int32_t* hot_start, const int32_t* hot_len,
+                        const uint8_t* page_pool, int64_t pool_pages, const int32_t* page_table,
+                        int max_pages, const int32_t* cold_len, const tq::DecodeGate* gate,
+                        float* out, void* workspace, size_t ws_bytes, void* stream) {
   if (!ctx || !q || !out || !workspace) return TQ_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || W_max < 0 || max_pages < 0)
     return TQ_ERR_INVALID_ARG;
@@ -232,13 +234,41 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype
     return TQ_ERR_INVALID_ARG;
   if (page_pool && !tq::aligned(page_pool, 16)) return TQ_ERR_INVALID_ARG;
   if (!tq::aligned(workspace, 256)) return TQ_ERR_INVALID_ARG;
+  if (gate && std::isnan(gate->threshold)) return TQ_ERR_INVALID_ARG;
   const size_t need = tq::decode_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max);
   if (need == 0 || ws_bytes < need) return TQ_ERR_INVALID_ARG;
   return static_cast<tq_status>(tq::launch_decode(
       ctx, q, q_dtype, B, Hq, Hkv, scale, W_max > 0 ? k_hot : nullptr,
-      W_max > 0 ? v_hot : nullptr, W_max, W_max > 0 ? hot_len : nullptr,
-      max_pages > 0 ? page_pool : nullptr, pool_pages, max_pages > 0 ? page_table : nullptr,
-      max_pages, max_pages > 0 ? cold_len : nullptr, out, workspace, ws_bytes, stream));
+      W_max > 0 ? v_hot : nullptr, W_max, W_max > 0 ? hot_start : nullptr,
+      W_max > 0 ? hot_len : nullptr, max_pages > 0 ? page_pool : nullptr, pool_pages,
+      max_pages > 0 ? page_table : nullptr, max_pages, max_pages > 0 ? cold_len : nullptr, gate,
+      out, workspace, ws_bytes, stream));
+}
+
+}  // namespace
+
+tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                              int Hkv, float scale, const void* k_hot, const void* v_hot,
+                              int W_max, const int32_t* hot_len, const uint8_t* page_pool,
+                              int64_t pool_pages, const int32_t* page_table, int max_pages,
+                              const int32_t* cold_len, float* out, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  return decode_common(ctx, q, q_dtype, B, Hq, Hkv, scale, k_hot, v_hot, W_max, nullptr, hot_len,
+                       page_pool, pool_pages, page_table, max_pages, cold_len, nullptr, out,
+                       workspace, ws_bytes, stream);
+}
+
+tq_status tq_decode_attention_gated(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B,
+                                    int Hq, int Hkv, float scale, const void* k_hot,
+                                    const void* v_hot, int W_max, const int32_t* hot_start,
+                                    const int32_t* hot_len, const uint8_t* page_pool,
+                                    int64_t pool_pages, const int32_t* page_table, int max_pages,
+                                    const int32_t* cold_len, float threshold, int32_t* cold_used,
+                                    float* out, void* workspace, size_t ws_bytes, void* stream) {
+  const tq::DecodeGate gate{threshold, cold_used};
+  return decode_common(ctx, q, q_dtype, B, Hq, Hkv, scale, k_hot, v_hot, W_max, hot_start,
+                       hot_len, page_pool, pool_pages, page_table, max_pages, cold_len, &gate,
+                       out, workspace, ws_bytes, stream);
 }
 
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k) {

@@ -78,6 +78,8 @@ struct Work {
   float* desc;        // [BH][DESC_N][8] per head: key unit, hot descale, key constant,
                       // QJL unit, QJL constant (softmax scale folded in)
   float* part;        // [(Wtot + S)][G][D + 2]
+  float* gmax;        // [BH][gate_nsplit][G] raw hot-score maxima per slot range (gated form)
+  int* gmask;         // [BH] bit g set: q head g of the group reads its cold tokens
 };
 
 struct Params {
@@ -88,6 +90,7 @@ struct Params {
   const __half* k_hot;
   const __half* v_hot;
   const int32_t* hot_len;
+  const int32_t* hot_start;  // [B] ring slot of the oldest hot token, or null (= 0)
   const uint8_t* pool;
   long long pool_pages;
   long long page_bytes;
@@ -104,6 +107,12 @@ struct Params {
   Work w;
   int S;     // segments = 2 * B * Hkv
   int Wtot;  // attention warps
+  // threshold gate: a q head reads its cold tokens only when its largest raw
+  // hot score <q, k_t> is below gate_thr
+  int gated;
+  float gate_thr;
+  int gate_nsplit;     // hot slot ranges of GATE_TOK slots
+  int32_t* cold_used;  // [B, Hq] out (gated form), or null
 };
 
 __device__ __forceinline__ int* unit_off(const Params& p) { return p.w.sched + 4; }
@@ -122,6 +131,31 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// slot of the ring holding the oldest hot token of sequence b (0 without a ring)
+__device__ __forceinline__ int hot_start_of(const Params& p, int b) {
+  if (!p.hot_start) return 0;
+  const int s = p.hot_start[b];
+  return (s >= 0 && s < p.W_max) ? s : 0;
+}
+
+// ---------------------------------------------------------------------------
+// 0. threshold gate (gated form only)
+// ---------------------------------------------------------------------------
+constexpr int GATE_TOK = 128;  // hot slots per gate CTA (one 16-slot tile per warp)
+
+// bit g set: q head g of group bh reads its cold tokens (after the gate launch)
+__device__ int gate_mask_of(const Params& p, int bh) {
+  const int G = p.Hq / p.Hkv;
+  int mask = 0;
+  for (int g = 0; g < G; ++g) {
+    float m = NEG_INF;
+    for (int s = 0; s < p.gate_nsplit; ++s)
+      m = fmaxf(m, p.w.gmax[(static_cast<size_t>(bh) * p.gate_nsplit + s) * G + g]);
+    if (m < p.gate_thr) mask |= 1 << g;
+  }
+  return mask;
+}
 
 // ---------------------------------------------------------------------------
 // 1. prep
@@ -174,6 +208,11 @@ __device__ void build_schedule(const Params& p) {
           report(p.err, TQ_ERR_CAPACITY);
           len = len < 0 ? 0 : cap;
         }
+        if (p.gated) {
+          const int mask = gate_mask_of(p, bh);
+          p.w.gmask[bh] = mask;
+          if (mask == 0) len = 0;  // no head of the group reads its cold tokens
+        }
         units = (len + COLD_TOK - 1) / COLD_TOK;
       } else {
         len = p.hot_len ? p.hot_len[b] : 0;
@@ -181,6 +220,8 @@ __device__ void build_schedule(const Params& p) {
           report(p.err, TQ_ERR_CAPACITY);
           len = len < 0 ? 0 : p.W_max;
         }
+        if (p.hot_start && p.W_max > 0 && (p.hot_start[b] < 0 || p.hot_start[b] >= p.W_max))
+          report(p.err, TQ_ERR_CAPACITY);
         units = (len + HOT_TOK - 1) / HOT_TOK;
       }
       slen[sg] = len;
@@ -242,35 +283,57 @@ __device__ __forceinline__ float prescale_for(float mx) {
 // D x D matrices.  Four lanes share a row: lane qq of the four takes the
 // float4 chunks qq, qq + 4, ... of the row (coalesced row reads, conflict-free
 // reads of x), so a row costs its FMAs plus a two-step shuffle reduction.
-// All row loads of a pass are issued before any arithmetic.
+// Every row load of both matrices is issued at the start of the kernel,
+// before the query is loaded (the rows do not depend on it).
 constexpr int PREP_WARPS = 8;
 
+template <int D>
+struct MatRows {
+  static constexpr int CH = D / 16;                     // float4 chunks per lane and row
+  static constexpr int ROWS_PER_PASS = PREP_WARPS * 8;  // 8 rows per warp
+  static constexpr int PASSES = D / ROWS_PER_PASS;
+  float4 m[2][PASSES][CH];
+};
+
+// the lane's row chunks of both matrices, loaded before the query is ready
+template <int D>
+__device__ __forceinline__ void matvec_prefetch(const float* __restrict__ M1,
+                                                const float* __restrict__ M2, MatRows<D>& mr) {
+  using R = MatRows<D>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qq = lane & 3, rsub = lane >> 2;
+#pragma unroll
+  for (int w = 0; w < 2; ++w)
+#pragma unroll
+    for (int ps = 0; ps < R::PASSES; ++ps) {
+      const int r = ps * R::ROWS_PER_PASS + warp * 8 + rsub;
+      const float* M = w == 0 ? M1 : M2;
+#pragma unroll
+      for (int i = 0; i < R::CH; ++i)
+        mr.m[w][ps][i] = __ldg(reinterpret_cast<const float4*>(M + static_cast<size_t>(r) * D) + qq + 4 * i);
+    }
+}
+
 template <int D, int G>
-__device__ __forceinline__ void matvec_rows2(const float* __restrict__ M1, const float* __restrict__ M2,
-                                             const float (*x)[D], float (*y1)[D], float (*y2)[D]) {
-  constexpr int CH = D / 16;                             // float4 chunks per lane and row
-  constexpr int ROWS_PER_PASS = PREP_WARPS * 8;          // 8 rows per warp
-  constexpr int PASSES = D / ROWS_PER_PASS;
+__device__ __forceinline__ void matvec_rows2(const MatRows<D>& mr, const float (*x)[D],
+                                             float (*y1)[D], float (*y2)[D]) {
+  using R = MatRows<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qq = lane & 3, rsub = lane >> 2;
 #pragma unroll
   for (int w = 0; w < 2; ++w) {
-    const float* M = w == 0 ? M1 : M2;
     float (*y)[D] = w == 0 ? y1 : y2;
 #pragma unroll
-    for (int ps = 0; ps < PASSES; ++ps) {
-      const int r = ps * ROWS_PER_PASS + warp * 8 + rsub;
-      float4 m[CH];
-#pragma unroll
-      for (int i = 0; i < CH; ++i)
-        m[i] = __ldg(reinterpret_cast<const float4*>(M + static_cast<size_t>(r) * D) + qq + 4 * i);
+    for (int ps = 0; ps < R::PASSES; ++ps) {
+      const int r = ps * R::ROWS_PER_PASS + warp * 8 + rsub;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float acc = 0.0f;
 #pragma unroll
-        for (int i = 0; i < CH; ++i) {
+        for (int i = 0; i < R::CH; ++i) {
           const float4 xv = reinterpret_cast<const float4*>(x[g])[qq + 4 * i];
-          acc = fmaf(m[i].x, xv.x, fmaf(m[i].y, xv.y, fmaf(m[i].z, xv.z, fmaf(m[i].w, xv.w, acc))));
+          const float4 mv = mr.m[w][ps][i];
+          acc = fmaf(mv.x, xv.x, fmaf(mv.y, xv.y, fmaf(mv.z, xv.z, fmaf(mv.w, xv.w, acc))));
         }
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
@@ -286,6 +349,7 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   pdl_launch_dependents();
   const int BH = p.B * p.Hkv;
   if (blockIdx.x == BH) {
+    if (p.gated) pdl_wait();  // the gate launch's maxima
     build_schedule(p);
     return;
   }
@@ -294,6 +358,8 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   __shared__ unsigned smax[2][G];
   __shared__ float sfac[2][G];
   const int tid = threadIdx.x;
+  MatRows<D> mr;
+  matvec_prefetch<D>(p.rot, p.sp, mr);  // Pi and S Pi rows do not wait for the query
   if (tid < 2 * G) smax[tid / G][tid % G] = 0u;
   for (int i = tid; i < G * D; i += blockDim.x) {
     const int g = i / D, j = i % D;
@@ -301,7 +367,7 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
                              static_cast<tq_dtype>(p.q_dtype));
   }
   __syncthreads();
-  matvec_rows2<D, G>(p.rot, p.sp, sq, sqr, sqs);  // q_rot = Pi q, q_s = (S Pi) q
+  matvec_rows2<D, G>(mr, sq, sqr, sqs);  // q_rot = Pi q, q_s = (S Pi) q
   __syncthreads();
   // Cold keys: four 0/1 operand planes -- sign s, magnitude m, s AND m, QJL
   // sign b -- against 16-bit fixed-point query weights (int8 hi, lo):
@@ -409,6 +475,127 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
 }
 
 // ---------------------------------------------------------------------------
+// 0. threshold gate (gated form only), launched before prep
+// ---------------------------------------------------------------------------
+// Largest raw hot score max_t <q_g, k_t> of each q head g of a (batch, kv
+// head) group over one range of GATE_TOK ring slots (-inf where no slot of the
+// range holds a token).  Each warp scores one tile of 16 slots with m16n8k16
+// MMAs: tokens on M, the group's heads x {hi, lo} fp16 parts of the
+// prescaled query on N, fp32 accumulation.  The contraction order inside a
+// k-step is free, so a lane's A fragment is two whole 16-byte chunks of its
+// two rows (k-steps 2i and 2i+1 take the halves of chunk c + 4i) and the B
+// fragment takes the query coordinates of the same chunks.
+template <int D, int G>
+__global__ void __launch_bounds__(256) gate_kernel(Params p) {
+  pdl_launch_dependents();
+  constexpr int NT = (2 * G + 7) / 8;  // n-tiles: G heads x {hi, lo}
+  constexpr int NCH = D / 32;          // 16-byte chunks per lane and row
+  const int split = blockIdx.x, bh = blockIdx.y, b = bh / p.Hkv, kvh = bh % p.Hkv;
+  __shared__ __align__(16) float sq[G][D];
+  __shared__ unsigned smx[G];
+  __shared__ float sf[G];
+  __shared__ float wmax[8][G];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, c = lane & 3;
+  // the warp's two rows per lane: slots s0 (row g) and s0 + 8 (row g + 8).
+  // Every slot below W_max is loaded before the lengths are known (slots
+  // without a token only feed their own rows of the MMA and are masked).
+  const int s0 = split * GATE_TOK + warp * 16 + g;
+  uint4 kr[2][NCH];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int slot = s0 + 8 * h;
+    const uint4* row =
+        reinterpret_cast<const uint4*>(p.k_hot + (static_cast<size_t>(bh) * p.W_max + slot) * D);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+      kr[h][i] = slot < p.W_max ? __ldg(row + c + 4 * i) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  constexpr int QPT = (G * D + 255) / 256;  // query elements per thread
+  float qv[QPT];
+#pragma unroll
+  for (int k = 0; k < QPT; ++k) {
+    const int i = tid + 256 * k;
+    qv[k] = i < G * D ? load_as_float(p.q, (static_cast<size_t>(b) * p.Hq + kvh * G) * D + i,
+                                      static_cast<tq_dtype>(p.q_dtype))
+                      : 0.0f;
+  }
+  int len = p.hot_len[b];
+  len = len < 0 ? 0 : (len > p.W_max ? p.W_max : len);  // the schedule reports the error
+  const int start = hot_start_of(p, b);
+  bool valid[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int slot = s0 + 8 * h;
+    int rel = slot - start;
+    if (rel < 0) rel += p.W_max;
+    valid[h] = slot < p.W_max && rel < len;
+  }
+  if (tid < G) smx[tid] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < QPT; ++k) {
+    const int i = tid + 256 * k;
+    if (i < G * D) {
+      sq[i / D][i % D] = qv[k];
+      atomicMax(&smx[i / D], __float_as_uint(fabsf(qv[k])));
+    }
+  }
+  __syncthreads();
+  if (tid < G) sf[tid] = prescale_for(__uint_as_float(smx[tid]));
+  __syncthreads();
+  // B fragments: column n = lane >> 2 of n-tile nt is head (8 nt + n) / 2, part n % 2
+  uint32_t bfr[NCH][2][NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int n = 8 * nt + g, hh = n >> 1, part = n & 1;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        const int d0 = 8 * (c + 4 * i) + 4 * hs;
+        if (hh < G) {
+          const float f = sf[hh];
+          bfr[i][hs][nt][0] = pack_split(f * sq[hh][d0], f * sq[hh][d0 + 1], part);
+          bfr[i][hs][nt][1] = pack_split(f * sq[hh][d0 + 2], f * sq[hh][d0 + 3], part);
+        } else {
+          bfr[i][hs][nt][0] = bfr[i][hs][nt][1] = 0u;
+        }
+      }
+  }
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NCH; ++i)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      mma_f16(acc[nt], kr[0][i].x, kr[1][i].x, kr[0][i].y, kr[1][i].y, bfr[i][0][nt][0],
+              bfr[i][0][nt][1]);
+      mma_f16(acc[nt], kr[0][i].z, kr[1][i].z, kr[0][i].w, kr[1][i].w, bfr[i][1][nt][0],
+              bfr[i][1][nt][1]);
+    }
+  // lane (g, c) holds, for head c + 4 nt, the hi and lo parts of rows g and g + 8
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float m = NEG_INF;
+    if (valid[0]) m = acc[nt][0] + acc[nt][1];
+    if (valid[1]) m = fmaxf(m, acc[nt][2] + acc[nt][3]);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int hh = c + 4 * nt;
+    if (g == 0 && hh < G) wmax[warp][hh] = m;
+  }
+  __syncthreads();
+  if (tid < G) {
+    float m = NEG_INF;
+    for (int w = 0; w < 8; ++w) m = fmaxf(m, wmax[w][tid]);
+    // undo the power-of-two prescale (exact)
+    p.w.gmax[(static_cast<size_t>(bh) * p.gate_nsplit + split) * G + tid] = m / sf[tid];
+  }
+}
+
+// ---------------------------------------------------------------------------
 // 2. attention
 // ---------------------------------------------------------------------------
 template <int D, int G>
@@ -447,8 +634,10 @@ __device__ __forceinline__ void issue_unit(const Params& p, int sg, int lu, int 
     __syncwarp();
     const int r = lane & 15, isv = lane >> 4;
     if (r < rows) {
+      int slot = t0 + r + hot_start_of(p, bh / p.Hkv);
+      if (slot >= p.W_max) slot -= p.W_max;
       const __half* src = (isv ? p.v_hot : p.k_hot) +
-                          (static_cast<size_t>(bh) * p.W_max + t0 + r) * D;
+                          (static_cast<size_t>(bh) * p.W_max + slot) * D;
       bulk_g2s(d0 + isv * HOT_TOK * C::HROW + r * C::HROW, src, 2 * D, bar);
     }
   }
@@ -899,110 +1088,188 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
 // ---------------------------------------------------------------------------
 // 3. combine
 // ---------------------------------------------------------------------------
-constexpr int MAX_COMBINE_SLOTS = 256;  // partial records staged in shared memory per pass
+constexpr int COMB_THREADS = 256;
+constexpr int COMB_CHUNK = 256;  // records whose weights are staged in shared memory at once
 
+// Shared memory of the combine kernel: Pi, the staged record weights, and the
+// per-slice output sums.
 template <int D, int G>
-__global__ void __launch_bounds__(D) combine_kernel(Params p) {
+struct CombCfg {
+  static constexpr int NSL = COMB_THREADS / D;  // record slices
+  static constexpr int OFF_W = D * D * 4;
+  static constexpr int OFF_S = OFF_W + COMB_CHUNK * G * 4;
+  static constexpr int SMEM = OFF_S + NSL * 2 * G * D * 4;
+};
+
+// max (op 0) or sum (op 1) of v over the threads that share thread index mod G
+template <int G>
+__device__ __forceinline__ float group_reduce(float v, float (*red)[G], int op) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int o = G; o < 32; o <<= 1) {
+    const float w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = op == 0 ? fmaxf(v, w) : v + w;
+  }
+  __syncthreads();
+  if (lane < G) red[warp][lane] = v;
+  __syncthreads();
+  float r = red[0][tid % G];
+  for (int w = 1; w < COMB_THREADS / 32; ++w) r = op == 0 ? fmaxf(r, red[w][tid % G]) : r + red[w][tid % G];
+  return r;
+}
+
+// Per (batch, kv head): log-sum-exp merge of the group's partial records
+// (cold records hold rotated-domain outputs), o_cold = Pi^T o_rot, merge of
+// cold and hot, division by the softmax denominator.  Three passes over the
+// records: per-head maxima; softmax weights (staged in shared memory, one
+// chunk at a time); weighted outputs, NSL slices of records accumulated in
+// parallel with many loads in flight.
+template <int D, int G>
+__global__ void __launch_bounds__(COMB_THREADS) combine_kernel(Params p) {
+  using CC = CombCfg<D, G>;
+  constexpr int NSL = CC::NSL;
+  constexpr int RB = G * (D + 2);  // floats per record
+  constexpr float NINF = -__builtin_huge_valf();
   const int bh = blockIdx.x, b = bh / p.Hkv, kvh = bh % p.Hkv;
-  const int j = threadIdx.x;
-  // Pi does not depend on the attention launch: stage it in shared memory
-  // first, every load of the thread in flight at once, overlapping the tail
-  // of that launch
-  extern __shared__ float spi[];  // [D][D]
+  const int tid = threadIdx.x, sl = tid / D, j = tid % D;
+  extern __shared__ __align__(16) uint8_t csm[];
+  float* spi = reinterpret_cast<float*>(csm);               // [D][D]
+  float* wts = reinterpret_cast<float*>(csm + CC::OFF_W);   // [COMB_CHUNK][G]
+  float* ssum = reinterpret_cast<float*>(csm + CC::OFF_S);  // [NSL][2][G][D]
+  __shared__ float red[COMB_THREADS / 32][G];
+  __shared__ float sM[2][G], sL[2][G];
+  // Pi does not depend on the attention launch: stage it first, overlapping
+  // the tail of that launch
   {
-    constexpr int PER = D * D / 4 / D;  // float4 per thread
-    float4 v[PER];
+    constexpr int PER = D * D / 4 / COMB_THREADS;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) v[i] = __ldg(reinterpret_cast<const float4*>(p.rot) + i * D + j);
-#pragma unroll
-    for (int i = 0; i < PER; ++i) reinterpret_cast<float4*>(spi)[i * D + j] = v[i];
+    for (int i = 0; i < PER; ++i)
+      reinterpret_cast<float4*>(spi)[i * COMB_THREADS + tid] =
+          __ldg(reinterpret_cast<const float4*>(p.rot) + i * COMB_THREADS + tid);
   }
   pdl_wait();  // partial records come from the attention launch
-  const int* sched = p.w.sched;
-  const int* soff = sched + 4 + p.S + 1;
-  __shared__ float sm_m[MAX_COMBINE_SLOTS][G], sm_l[MAX_COMBINE_SLOTS][G];
-  __shared__ float so[G][D];
-  constexpr float NINF = -__builtin_huge_valf();
-  constexpr int RB = G * (D + 2);  // floats per record
-  float M[2][G], L[2][G], O[2][G];
-#pragma unroll
-  for (int dom = 0; dom < 2; ++dom) {
-    const int sg = 2 * bh + dom;
-    const int a = soff[sg], e = soff[sg + 1];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      M[dom][g] = NINF;
-      L[dom][g] = 0.0f;
-      O[dom][g] = 0.0f;
+  const int* soff = p.w.sched + 4 + p.S + 1;
+  const int a0 = soff[2 * bh], a1 = soff[2 * bh + 1], e1 = soff[2 * bh + 2];
+  const int R = e1 - a0;
+  const float* part = p.w.part;
+  // pass 1: per (domain, head) maxima over records that hold tokens; the
+  // thread's head is tid % G throughout (COMB_THREADS is a multiple of G)
+  const int hg = tid % G;
+  float mx0 = NINF, mx1 = NINF;
+  for (int i = tid; i < R * G; i += COMB_THREADS) {
+    const int r = a0 + i / G;
+    const float* rec = part + static_cast<size_t>(r) * RB;
+    const float m = rec[hg], l = rec[G + hg];
+    if (l > 0.0f) {
+      if (r < a1) mx0 = fmaxf(mx0, m);
+      else mx1 = fmaxf(mx1, m);
     }
-    for (int base = a; base < e; base += MAX_COMBINE_SLOTS) {
-      const int n = min(MAX_COMBINE_SLOTS, e - base);
-      __syncthreads();
-      for (int i = j; i < n * G; i += blockDim.x) {
-        const int sl = i / G, g = i % G;
-        const float* rec = p.w.part + static_cast<size_t>(base + sl) * RB;
-        sm_m[sl][g] = rec[g];
-        sm_l[sl][g] = rec[G + g];
-      }
-      __syncthreads();
+  }
+  mx0 = group_reduce<G>(mx0, red, 0);
+  mx1 = group_reduce<G>(mx1, red, 0);
+  if (tid < G) {
+    sM[0][tid] = mx0;
+    sM[1][tid] = mx1;
+  }
+  float O[2][G];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float mx = M[dom][g];
-        for (int sl = 0; sl < n; ++sl)
-          if (sm_l[sl][g] > 0.0f) mx = fmaxf(mx, sm_m[sl][g]);
-        const float resc = (M[dom][g] == NINF || mx == NINF) ? 0.0f : exp2f(M[dom][g] - mx);
-        L[dom][g] *= resc;
-        O[dom][g] *= resc;
-        M[dom][g] = mx;
-      }
-      // partial outputs: eight records x every head requested at once
-      for (int s0 = 0; s0 < n; s0 += 8) {
-        float ov[8][G];
+  for (int d2 = 0; d2 < 2; ++d2)
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
+    for (int g = 0; g < G; ++g) O[d2][g] = 0.0f;
+  float l0 = 0.0f, l1 = 0.0f;
+  for (int base = 0; base < R; base += COMB_CHUNK) {
+    const int n = min(COMB_CHUNK, R - base);
+    __syncthreads();
+    // pass 2: weights exp2(m - M) of this chunk, and the denominators
+    for (int i = tid; i < n * G; i += COMB_THREADS) {
+      const int r = a0 + base + i / G;
+      const float* rec = part + static_cast<size_t>(r) * RB;
+      const float m = rec[hg], l = rec[G + hg];
+      const float M = r < a1 ? mx0 : mx1;
+      const float w = (l > 0.0f) ? exp2f(m - M) : 0.0f;
+      wts[i] = w;
+      if (r < a1) l0 += l * w;
+      else l1 += l * w;
+    }
+    __syncthreads();
+    // pass 3: weighted outputs; slice sl takes records sl, sl + NSL, ...
+    int r = sl;
+    for (; r + 3 * NSL < n; r += 4 * NSL) {
+      float ov[4][G];
 #pragma unroll
-          for (int g = 0; g < G; ++g)
-            ov[t][g] = (s0 + t < n) ? p.w.part[static_cast<size_t>(base + s0 + t) * RB + 2 * G + g * D + j]
-                                    : 0.0f;
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (s0 + t < n) {
+        for (int g = 0; g < G; ++g)
+          ov[u][g] = part[static_cast<size_t>(a0 + base + r + u * NSL) * RB + 2 * G + g * D + j];
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-              const float lw = sm_l[s0 + t][g];
-              const float f = (lw > 0.0f) ? exp2f(sm_m[s0 + t][g] - M[dom][g]) : 0.0f;
-              L[dom][g] += lw * f;
-              O[dom][g] += ov[t][g] * f;
-            }
-          }
+      for (int u = 0; u < 4; ++u) {
+        const int rr = r + u * NSL;
+        const int dom = (a0 + base + rr) < a1 ? 0 : 1;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float w = wts[rr * G + g] * ov[u][g];
+          if (dom == 0) O[0][g] += w;
+          else O[1][g] += w;
         }
       }
     }
-  }
-  // cold accumulators are in the rotated domain: o_cold = Pi^T o_rot, all heads at once
+    for (; r < n; r += NSL) {
+      const int dom = (a0 + base + r) < a1 ? 0 : 1;
 #pragma unroll
-  for (int g = 0; g < G; ++g) so[g][j] = O[0][g];
+      for (int g = 0; g < G; ++g) {
+        const float w = wts[r * G + g] * part[static_cast<size_t>(a0 + base + r) * RB + 2 * G + g * D + j];
+        if (dom == 0) O[0][g] += w;
+        else O[1][g] += w;
+      }
+    }
+  }
+  l0 = group_reduce<G>(l0, red, 1);
+  l1 = group_reduce<G>(l1, red, 1);
+  if (tid < G) {
+    sL[0][tid] = l0;
+    sL[1][tid] = l1;
+  }
+#pragma unroll
+  for (int d2 = 0; d2 < 2; ++d2)
+#pragma unroll
+    for (int g = 0; g < G; ++g) ssum[((sl * 2 + d2) * G + g) * D + j] = O[d2][g];
   __syncthreads();
-  float oc[G];
+  // slice sums; the cold one back into slice 0's rows for the rotation
+  if (sl == 0) {
 #pragma unroll
-  for (int g = 0; g < G; ++g) oc[g] = 0.0f;
-#pragma unroll 16
-  for (int i = 0; i < D; ++i) {
-    const float r = spi[i * D + j];
+    for (int d2 = 0; d2 < 2; ++d2)
 #pragma unroll
-    for (int g = 0; g < G; ++g) oc[g] = fmaf(r, so[g][i], oc[g]);
+      for (int g = 0; g < G; ++g) {
+        float s = O[d2][g];
+#pragma unroll
+        for (int k = 1; k < NSL; ++k) s += ssum[((k * 2 + d2) * G + g) * D + j];
+        ssum[(d2 * G + g) * D + j] = s;
+      }
   }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float Mx = fmaxf(M[0][g], M[1][g]);
+  __syncthreads();
+  int mask = (1 << G) - 1;
+  if (p.gated) mask = p.w.gmask[bh];
+  // o_cold = Pi^T o_rot; thread (sl, j) takes heads g = sl, sl + NSL, ...
+  for (int g = sl; g < G; g += NSL) {
+    const float* so = ssum + g * D;  // cold sums (domain 0)
+    float oc = 0.0f;
+#pragma unroll 16
+    for (int i = 0; i < D; ++i) oc = fmaf(spi[i * D + j], so[i], oc);
+    const float oh = ssum[(G + g) * D + j];
+    const bool open = (mask >> g) & 1;
+    const float Mc = sM[0][g], Mh = sM[1][g];
+    const float Lc = open ? sL[0][g] : 0.0f, Lh = sL[1][g];
+    const float Mx = fmaxf(Lc > 0.0f ? Mc : NINF, Lh > 0.0f ? Mh : NINF);
     float res = 0.0f;
     if (Mx != NINF) {
-      const float fc = (L[0][g] > 0.0f) ? exp2f(M[0][g] - Mx) : 0.0f;
-      const float fh = (L[1][g] > 0.0f) ? exp2f(M[1][g] - Mx) : 0.0f;
-      const float den = L[0][g] * fc + L[1][g] * fh;
-      res = (den > 0.0f) ? (oc[g] * fc + O[1][g] * fh) / den : 0.0f;
+      const float fc = (Lc > 0.0f) ? exp2f(Mc - Mx) : 0.0f;
+      const float fh = (Lh > 0.0f) ? exp2f(Mh - Mx) : 0.0f;
+      const float den = Lc * fc + Lh * fh;
+      res = (den > 0.0f) ? ((fc > 0.0f ? oc * fc : 0.0f) + (fh > 0.0f ? oh * fh : 0.0f)) / den : 0.0f;
     }
     p.out[(static_cast<size_t>(b) * p.Hq + kvh * G + g) * D + j] = res;
+    if (j == 0 && p.gated && p.cold_used)
+      p.cold_used[static_cast<size_t>(b) * p.Hq + kvh * G + g] = open;
   }
 }
 
@@ -1012,11 +1279,13 @@ __global__ void __launch_bounds__(D) combine_kernel(Params p) {
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-  size_t sched, frag_c, frag_h, desc, part, total;
+  size_t sched, frag_c, frag_h, desc, part, gmax, gmask, total;
 };
 
+inline int gate_splits(int W_max) { return (W_max + GATE_TOK - 1) / GATE_TOK; }
+
 template <int D, int G>
-WsLayout ws_layout(int B, int Hkv, int Wtot) {
+WsLayout ws_layout(int B, int Hkv, int Wtot, int W_max) {
   using C = Cfg<D, G>;
   const size_t BH = static_cast<size_t>(B) * Hkv, S = 2 * BH;
   WsLayout L;
@@ -1031,6 +1300,10 @@ WsLayout ws_layout(int B, int Hkv, int Wtot) {
   off = align256(off + sizeof(float) * BH * DESC_N * 8);
   L.part = off;
   off = align256(off + sizeof(float) * (static_cast<size_t>(Wtot) + S) * G * (D + 2));
+  L.gmax = off;
+  off = align256(off + sizeof(float) * BH * gate_splits(W_max) * G);
+  L.gmask = off;
+  off = align256(off + sizeof(int) * BH);
   L.total = off;
   return L;
 }
@@ -1043,7 +1316,7 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
   const int grid = ctx->num_sms;
   p.Wtot = grid * NW;
   p.S = 2 * p.B * p.Hkv;
-  const WsLayout L = ws_layout<D, G>(p.B, p.Hkv, p.Wtot);
+  const WsLayout L = ws_layout<D, G>(p.B, p.Hkv, p.Wtot, p.W_max);
   if (ws_bytes < L.total) return TQ_ERR_INVALID_ARG;
   uint8_t* base = static_cast<uint8_t*>(ws);
   p.w.sched = reinterpret_cast<int*>(base + L.sched);
@@ -1051,6 +1324,9 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
   p.w.frag_h = reinterpret_cast<uint32_t*>(base + L.frag_h);
   p.w.desc = reinterpret_cast<float*>(base + L.desc);
   p.w.part = reinterpret_cast<float*>(base + L.part);
+  p.w.gmax = reinterpret_cast<float*>(base + L.gmax);
+  p.w.gmask = reinterpret_cast<int*>(base + L.gmask);
+  p.gate_nsplit = gate_splits(p.W_max);
   static bool attr_set[2][9] = {};
   bool& set = attr_set[D == 128][G];
   if (!set) {
@@ -1059,7 +1335,22 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
       return TQ_ERR_CUDA;
     set = true;
   }
-  prep_kernel<D, G><<<p.B * p.Hkv + 1, PREP_WARPS * 32, 0, st>>>(p);
+  if (p.gated && p.gate_nsplit > 0) {
+    // gate, then prep overlapping it: only prep's schedule CTA waits for the maxima
+    gate_kernel<D, G><<<dim3(p.gate_nsplit, p.B * p.Hkv), 256, 0, st>>>(p);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.B * p.Hkv + 1);
+    cfg.blockDim = dim3(PREP_WARPS * 32);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, prep_kernel<D, G>, p) != cudaSuccess) return TQ_ERR_CUDA;
+  } else {
+    prep_kernel<D, G><<<p.B * p.Hkv + 1, PREP_WARPS * 32, 0, st>>>(p);
+  }
   if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
   {
     cudaLaunchConfig_t cfg{};
@@ -1079,15 +1370,15 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
   bool& cset = comb_set[D == 128][G];
   if (!cset) {
     if (cudaFuncSetAttribute(combine_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             D * D * 4) != cudaSuccess)
+                             CombCfg<D, G>::SMEM) != cudaSuccess)
       return TQ_ERR_CUDA;
     cset = true;
   }
   {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(p.B * p.Hkv);
-    cfg.blockDim = dim3(D);
-    cfg.dynamicSmemBytes = D * D * 4;
+    cfg.blockDim = dim3(COMB_THREADS);
+    cfg.dynamicSmemBytes = CombCfg<D, G>::SMEM;
     cfg.stream = st;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1103,7 +1394,6 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
 
 size_t decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max) {
   (void)max_pages;
-  (void)W_max;
   if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0) return 0;
   const int G = Hq / Hkv;
   const int Wtot = ctx->num_sms * dec::NW;
@@ -1111,24 +1401,25 @@ size_t decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max
   size_t best = 0;
   auto take = [&](size_t v) { best = v > best ? v : best; };
   if (ctx->cfg.head_dim == 128) {
-    if (G == 1) take(dec::ws_layout<128, 1>(B, Hkv, Wtot).total);
-    if (G == 2) take(dec::ws_layout<128, 2>(B, Hkv, Wtot).total);
-    if (G == 4) take(dec::ws_layout<128, 4>(B, Hkv, Wtot).total);
-    if (G == 8) take(dec::ws_layout<128, 8>(B, Hkv, Wtot).total);
+    if (G == 1) take(dec::ws_layout<128, 1>(B, Hkv, Wtot, W_max).total);
+    if (G == 2) take(dec::ws_layout<128, 2>(B, Hkv, Wtot, W_max).total);
+    if (G == 4) take(dec::ws_layout<128, 4>(B, Hkv, Wtot, W_max).total);
+    if (G == 8) take(dec::ws_layout<128, 8>(B, Hkv, Wtot, W_max).total);
   } else {
-    if (G == 1) take(dec::ws_layout<64, 1>(B, Hkv, Wtot).total);
-    if (G == 2) take(dec::ws_layout<64, 2>(B, Hkv, Wtot).total);
-    if (G == 4) take(dec::ws_layout<64, 4>(B, Hkv, Wtot).total);
-    if (G == 8) take(dec::ws_layout<64, 8>(B, Hkv, Wtot).total);
+    if (G == 1) take(dec::ws_layout<64, 1>(B, Hkv, Wtot, W_max).total);
+    if (G == 2) take(dec::ws_layout<64, 2>(B, Hkv, Wtot, W_max).total);
+    if (G == 4) take(dec::ws_layout<64, 4>(B, Hkv, Wtot, W_max).total);
+    if (G == 8) take(dec::ws_layout<64, 8>(B, Hkv, Wtot, W_max).total);
   }
   return best;
 }
 
 int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq, int Hkv,
                   float scale, const void* k_hot, const void* v_hot, int W_max,
-                  const int32_t* hot_len, const uint8_t* pool, int64_t pool_pages,
-                  const int32_t* page_table, int max_pages, const int32_t* cold_len, float* out,
-                  void* ws, size_t ws_bytes, void* stream) {
+                  const int32_t* hot_start, const int32_t* hot_len, const uint8_t* pool,
+                  int64_t pool_pages, const int32_t* page_table, int max_pages,
+                  const int32_t* cold_len, const DecodeGate* gate, float* out, void* ws,
+                  size_t ws_bytes, void* stream) {
   const int d = ctx->cfg.head_dim;
   const int G = Hq / Hkv;
   const PageLayout L = page_layout(d, ctx->cfg.qjl_dim, true);
@@ -1145,6 +1436,12 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
   p.k_hot = static_cast<const __half*>(k_hot);
   p.v_hot = static_cast<const __half*>(v_hot);
   p.hot_len = hot_len;
+  p.hot_start = hot_start;
+  if (gate) {
+    p.gated = 1;
+    p.gate_thr = gate->threshold;
+    p.cold_used = gate->cold_used;
+  }
   p.pool = pool;
   p.pool_pages = pool_pages;
   p.page_bytes = static_cast<long long>(L.bytes);

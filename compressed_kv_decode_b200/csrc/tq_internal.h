@@ -65,12 +65,21 @@ struct PageLayout {
 };
 PageLayout page_layout(int d, int m, bool with_values);
 
+// Threshold gate of the gated decode: a q head reads its cold tokens only
+// when its largest raw hot score is below threshold; cold_used [B, Hq] (may
+// be null) receives 1 / 0 per head.
+struct DecodeGate {
+  float threshold;
+  int32_t* cold_used;
+};
+
 // Launchers (defined in the .cu files).  Return a tq_status.
 int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq, int Hkv,
                   float scale, const void* k_hot, const void* v_hot, int W_max,
-                  const int32_t* hot_len, const uint8_t* pool, int64_t pool_pages,
-                  const int32_t* page_table, int max_pages, const int32_t* cold_len, float* out,
-                  void* ws, size_t ws_bytes, void* stream);
+                  const int32_t* hot_start, const int32_t* hot_len, const uint8_t* pool,
+                  int64_t pool_pages, const int32_t* page_table, int max_pages,
+                  const int32_t* cold_len, const DecodeGate* gate, float* out, void* ws,
+                  size_t ws_bytes, void* stream);
 size_t decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max);
 
 int launch_compress(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype, int flags,

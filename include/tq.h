@@ -195,6 +195,42 @@ TQ_API tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype 
                               const int32_t* cold_len, float* out, void* workspace,
                               size_t ws_bytes, void* stream);
 
+/*
+ * tq_decode_attention with Monarch's threshold gate and a ring-buffer hot
+ * window ("Vereinfachte Decode-Schleife": the cold pages are decompressed and
+ * scored only if max(scores_hot) < threshold).
+ *  threshold  per query head h of sequence b, the gate is open when
+ *             max_t <q_h, k_t> < threshold, the maximum taken over the hot
+ *             tokens of h's kv head in fp32 on the raw dot products (no
+ *             softmax scale), -inf when there are none.  An open head
+ *             attends to hot and cold tokens exactly as tq_decode_attention;
+ *             a shut head to its hot tokens alone (zeros if it has none).
+ *             +INFINITY opens every head; NaN is rejected.  Where the
+ *             maximum lies within fp32 rounding of the threshold the decision
+ *             may go either way; cold_used reports the one taken.
+ *  cold_used  device int32 [B, Hq] out: the gate's decision per head, 1 when
+ *             the head attends to its cold tokens (whether or not it has
+ *             any), else 0.  May be NULL.
+ *  hot_start  device int32 [B], or NULL for 0: the hot window of sequence b
+ *             is a ring of W_max slots whose logical token i
+ *             (0 <= i < hot_len[b]) sits in slot (hot_start[b] + i) mod
+ *             W_max.  Attention does not depend on token order, so the ring
+ *             only saves the caller from shifting the window when it evicts
+ *             its oldest tokens.  A start outside [0, W_max) is a device
+ *             error (TQ_ERR_CAPACITY) and reads as 0.
+ * The other arguments, the workspace size and the results are those of
+ * tq_decode_attention.  When every head of a (batch, kv head) group is shut,
+ * the group's cold pages are not read at all.
+ */
+TQ_API tq_status tq_decode_attention_gated(const tq_ctx* ctx, const void* q, tq_dtype q_dtype,
+                                           int B, int Hq, int Hkv, float scale,
+                                           const void* k_hot, const void* v_hot, int W_max,
+                                           const int32_t* hot_start, const int32_t* hot_len,
+                                           const uint8_t* page_pool, int64_t pool_pages,
+                                           const int32_t* page_table, int max_pages,
+                                           const int32_t* cold_len, float threshold,
+                                           int32_t* cold_used, float* out, void* workspace,
+                                           size_t ws_bytes, void* stream);
 /* Largest decode workspace tq_decode_attention_noalloc can serve (8 MiB). */
 #define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 
