@@ -133,13 +133,13 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # workload on the device
 # ---------------------------------------------------------------------------
-def build_state(torch, tq, W, rank, batch=None, workload=WORKLOAD):
+def build_state(torch, tq, W, rank, batch=None, workload=WORKLOAD, extra_pages=0):
     cfg = W.DECODE[workload]
     B, Hq, Hkv, d = batch or cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"]
     cold, hot = cfg["cold"], cfg["hot"]
     dev = torch.device("cuda")
     ctx = tq.Context(d, seed=0)
-    max_pages = (cold + 127) // 128
+    max_pages = (cold + 127) // 128 + extra_pages
     n_pages = B * Hkv * max_pages
     page_bytes = ctx.page_bytes(True)
     gen = torch.Generator(device=dev)
@@ -295,6 +295,45 @@ def measure_gated(torch, tq, st, reps=50):
                      "groups_reading_cold": float(u.any(-1).float().mean())}
     res["ungated_ms_per_step"] = graph_ms(torch, lambda: decode(tq, st), reps)
     st["ctx"].check()
+    return res
+
+
+def measure_monarch(torch, tq, W, workload, evict_block, thresholds=(float("inf"), float("-inf")),
+                    steps=256):
+    """Monarch decode steps (append, gated attention, eviction) on a decode
+    workload: the hot ring holds W_max = the workload's hot length slots,
+    window = W_max - E; the timed steps (replayed from a CUDA graph, one step
+    per replay) include every eviction that falls due (one per E steps)."""
+    st = build_state(torch, tq, W, 0, None, workload, extra_pages=(steps + 64) // 128 + 3)
+    ctx, B, Hq, Hkv, d = st["ctx"], st["B"], st["Hq"], st["Hkv"], st["d"]
+    W_max, E = st["hot"], evict_block
+    window = W_max - E
+    dev = st["q"].device
+    k_new = torch.randn((B, Hkv, d), device=dev).half()
+    v_new = torch.randn((B, Hkv, d), device=dev).half()
+    hot_start = torch.zeros(B, dtype=torch.int32, device=dev)
+    ws = torch.empty(tq.tq_monarch_workspace_bytes(ctx.handle, B, Hq, Hkv, st["table"].shape[-1],
+                                                   W_max, E), dtype=torch.uint8, device=dev)
+    used = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+    res = {"workload": workload, "evict_block": E, "window": window, "hot_slots": W_max,
+           "steps": steps}
+    for thr in thresholds:
+        st["hot_len"].fill_(window)
+        hot_start.zero_()
+        st["cold_len"].fill_(st["cold"])
+
+        def step():
+            tq.tq_monarch_step(ctx.handle, st["q"], k_new, v_new, st["k_hot"], st["v_hot"],
+                               hot_start, st["hot_len"], st["pool"], st["table"], st["cold_len"],
+                               thr, window, E, st["out"], ws, Hkv, cold_used=used)
+        ms = graph_ms(torch, step, steps)
+        ctx.check()
+        tokens = B * Hkv * (W_max + st["cold"])
+        res["threshold_%s" % thr] = {"us_per_step": ms * 1e3,
+                                     "kv_tokens_heads_per_s": tokens / (ms / 1e3),
+                                     "heads_reading_cold": float(used.float().mean())}
+    del st
+    torch.cuda.empty_cache()
     return res
 
 
@@ -471,6 +510,10 @@ def run_ours(args, rank, world, local_rank):
         rows["gated_decode"] = measure_gated(torch, tq, st)
         rows["gated_decode"]["workload"] = WORKLOAD + " with Monarch's threshold gate"
         del st, graph
+        torch.cuda.empty_cache()
+        rows["monarch_step"] = [measure_monarch(torch, tq, W, "tinyllama", 128),
+                                measure_monarch(torch, tq, W, "tinyllama", 1),
+                                measure_monarch(torch, tq, W, WORKLOAD, 128)]
         torch.cuda.empty_cache()
         rows["compress"] = measure_compress(torch, tq)
         torch.cuda.empty_cache()

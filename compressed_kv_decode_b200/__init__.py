@@ -68,6 +68,14 @@ def lib():
                                                 C.c_int64, i32p, C.c_int, i32p, C.c_float, i32p,
                                                 f32p, vp, C.c_size_t, vp]
         L.tq_decode_attention_gated.restype = C.c_int
+        L.tq_monarch_workspace_bytes.argtypes = [vp, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                                 C.c_int]
+        L.tq_monarch_workspace_bytes.restype = C.c_size_t
+        L.tq_monarch_step.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float, vp,
+                                      vp, vp, vp, C.c_int, i32p, i32p, u8p, C.c_int64, i32p,
+                                      C.c_int, i32p, C.c_float, C.c_int, C.c_int, i32p, f32p, vp,
+                                      C.c_size_t, vp]
+        L.tq_monarch_step.restype = C.c_int
         L.tq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int,
                                                   C.c_float, vp, vp, C.c_int, i32p, u8p, C.c_int64,
                                                   i32p, C.c_int, i32p, f32p, vp]
@@ -223,6 +231,31 @@ def tq_decode_attention_gated(ctx, q, k_hot, v_hot, hot_len, page_pool, page_tab
         _ptr(cold_len), float(threshold), _ptr(cold_used), _ptr(out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)),
         "tq_decode_attention_gated")
+
+
+def tq_monarch_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max, evict_block):
+    return int(lib().tq_monarch_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max, evict_block))
+
+
+def tq_monarch_step(ctx, q, k_new, v_new, k_hot, v_hot, hot_start, hot_len, page_pool,
+                    page_table, cold_len, threshold, window, evict_block, out, workspace, Hkv,
+                    scale=0.0, cold_used=None, stream=None):
+    """One Monarch decode step: append (k_new, v_new fp16 [B, Hkv, d], or
+    None), gated attention over the hot ring and cold pages, eviction of the
+    oldest evict_block hot tokens of every sequence holding window +
+    evict_block of them.  k_hot, v_hot fp16 [B, Hkv, W_max, d]; hot_start,
+    hot_len, cold_len int32 [B] (all updated on the device)."""
+    _require_cuda(q, k_new, v_new, k_hot, v_hot, hot_start, hot_len, page_pool, page_table,
+                  cold_len, out, workspace, cold_used)
+    B, Hq, _ = q.shape
+    W_max = k_hot.shape[2]
+    _check(lib().tq_monarch_step(
+        ctx, _ptr(q), _dtype_code(q), B, Hq, Hkv, float(scale), _ptr(k_new), _ptr(v_new),
+        _ptr(k_hot), _ptr(v_hot), W_max, _ptr(hot_start), _ptr(hot_len), _ptr(page_pool),
+        page_pool.shape[0], _ptr(page_table), page_table.shape[-1], _ptr(cold_len),
+        float(threshold), int(window), int(evict_block), _ptr(cold_used), _ptr(out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+        "tq_monarch_step")
 
 
 def tq_decode_attention_noalloc(ctx, q, k_hot, v_hot, hot_len, page_pool, page_table, cold_len,

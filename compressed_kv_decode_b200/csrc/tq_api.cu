@@ -271,6 +271,44 @@ tq_status tq_decode_attention_gated(const tq_ctx* ctx, const void* q, tq_dtype q
                        out, workspace, ws_bytes, stream);
 }
 
+size_t tq_monarch_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages,
+                                  int W_max, int evict_block) {
+  if (!ctx) return 0;
+  return tq::monarch_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max, evict_block);
+}
+
+tq_status tq_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                          int Hkv, float scale, const void* k_new, const void* v_new, void* k_hot,
+                          void* v_hot, int W_max, int32_t* hot_start, int32_t* hot_len,
+                          uint8_t* page_pool, int64_t pool_pages, const int32_t* page_table,
+                          int max_pages, int32_t* cold_len, float threshold, int window,
+                          int evict_block, int32_t* cold_used, float* out, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  if (!ctx || !q || !out || !workspace || !k_hot || !v_hot || !hot_start || !hot_len)
+    return TQ_ERR_INVALID_ARG;
+  if (!page_pool || !page_table || !cold_len || pool_pages <= 0 || max_pages <= 0)
+    return TQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return TQ_ERR_INVALID_ARG;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || !std::isfinite(scale) || std::isnan(threshold)) return TQ_ERR_INVALID_ARG;
+  if (window < 0 || evict_block < 1 || W_max < 1 ||
+      static_cast<long long>(window) + evict_block > W_max)
+    return TQ_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return TQ_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_ERR_UNSUPPORTED;
+  if (!tq::aligned(k_hot, 16) || !tq::aligned(v_hot, 16) || !tq::aligned(page_pool, 16) ||
+      !tq::aligned(workspace, 256))
+    return TQ_ERR_INVALID_ARG;
+  if (k_new && (!tq::aligned(k_new, 16) || !tq::aligned(v_new, 16))) return TQ_ERR_INVALID_ARG;
+  const size_t need = tq::monarch_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max, evict_block);
+  if (need == 0 || ws_bytes < need) return TQ_ERR_INVALID_ARG;
+  return static_cast<tq_status>(tq::launch_monarch_step(
+      ctx, q, q_dtype, B, Hq, Hkv, scale, k_new, v_new, k_hot, v_hot, W_max, hot_start, hot_len,
+      page_pool, pool_pages, page_table, max_pages, cold_len, threshold, window, evict_block,
+      cold_used, out, workspace, ws_bytes, stream));
+}
+
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k) {
   if (!ctx || Q <= 0 || N <= 0 || k <= 0) return 0;
   return tq::topk_workspace_bytes(ctx, Q, N, k);

@@ -99,6 +99,7 @@ struct Params {
   float vt[7];
   int* err;
   int tiles_per_bh;
+  const int32_t* n_new_b;  // [B] tokens appended per sequence (eviction), or null: n_new for all
 };
 
 struct Tile {
@@ -111,9 +112,10 @@ __device__ __forceinline__ bool next_tile(const Params& p, int& t, Tile& out) {
   for (; t < total; t += gridDim.x) {
     const int bh = t / p.tiles_per_bh, ti = t % p.tiles_per_bh;
     const int cl = p.cold_len[bh / p.Hkv];
+    const int nn = p.n_new_b ? min(p.n_new_b[bh / p.Hkv], p.n_new) : p.n_new;
     const int lpage = cl / ROWS + ti;
     const int s_lo = max(cl, lpage * ROWS) - lpage * ROWS;
-    const int s_hi = min(cl + p.n_new, (lpage + 1) * ROWS) - lpage * ROWS;
+    const int s_hi = min(cl + nn, (lpage + 1) * ROWS) - lpage * ROWS;
     if (s_lo >= s_hi) continue;
     out.bh = bh;
     out.lpage = lpage;
@@ -208,6 +210,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float* nvp = reinterpret_cast<float*>(smem + C::OFF_NV);
   float* gp = reinterpret_cast<float*>(smem + C::OFF_G);
 
+  {
+    // a CTA without a tile leaves before staging the operand tables (calls
+    // that append to few sequences, such as evictions, launch many idle CTAs)
+    int t0 = blockIdx.x;
+    Tile probe;
+    if (!next_tile(p, t0, probe)) return;
+  }
   // resident operands in the K-major SW128 layout: Pi hi, Pi lo (rows = output
   // coordinate), S (rows = sketch index); 16-byte chunks
   for (int i = tid; i < D * (D / 8); i += NTHREADS) {
@@ -792,7 +801,7 @@ __global__ void advance_cold_len(int32_t* cold_len, int B, int n_new) {
 
 int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf16, int B, int Hkv,
                        int n_new, uint8_t* pool, int64_t pool_pages, const int32_t* page_table,
-                       int max_pages, int32_t* cold_len, void* stream) {
+                       int max_pages, int32_t* cold_len, void* stream, const int32_t* n_new_b) {
   const int d = ctx->cfg.head_dim;
   const PageLayout L = page_layout(d, ctx->cfg.qjl_dim, v != nullptr);
   ctc::Params p{};
@@ -821,6 +830,7 @@ int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf1
   for (int i = 0; i < 7; ++i) p.vt[i] = ctx->cb.val_t[i];
   p.err = ctx->dev.err;
   p.tiles_per_bh = (n_new + ctc::ROWS - 1) / ctc::ROWS + 1;
+  p.n_new_b = n_new_b;
   CUtensorMap mk, mv;
   const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_new),
                             static_cast<uint64_t>(B) * Hkv};
@@ -846,7 +856,8 @@ int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf1
     if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
     kern<<<grid, ctc::NTHREADS, smem, st>>>(mk, mv, p);
     if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
-    advance_cold_len<<<(B + 127) / 128, 128, 0, st>>>(cold_len, B, n_new);
+    // per-sequence counts: the caller advances the lengths
+    if (!n_new_b) advance_cold_len<<<(B + 127) / 128, 128, 0, st>>>(cold_len, B, n_new);
     return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
   };
   if (!v) {
@@ -862,7 +873,7 @@ int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf1
       if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
       kern<<<grid, ctc::KTHREADS, smem, st>>>(mk, p);
       if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
-      advance_cold_len<<<(B + 127) / 128, 128, 0, st>>>(cold_len, B, n_new);
+      if (!n_new_b) advance_cold_len<<<(B + 127) / 128, 128, 0, st>>>(cold_len, B, n_new);
       return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
     };
     if (d == 128)

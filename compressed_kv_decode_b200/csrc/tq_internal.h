@@ -86,9 +86,24 @@ int launch_compress(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dt
                     int B, int Hkv, int n_new, uint8_t* pool, int64_t pool_pages,
                     const int32_t* page_table, int max_pages, int32_t* cold_len, void* stream);
 
+// n_new_b (device [B], may be null): tokens appended per sequence, at most
+// n_new each (the input still holds n_new rows per (batch, kv head)); with it
+// cold_len is left for the caller to advance.
 int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf16, int B, int Hkv,
                        int n_new, uint8_t* pool, int64_t pool_pages, const int32_t* page_table,
-                       int max_pages, int32_t* cold_len, void* stream);
+                       int max_pages, int32_t* cold_len, void* stream,
+                       const int32_t* n_new_b = nullptr);
+
+// One Monarch decode step (append, gated attention, eviction); see tq.h.
+int launch_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq, int Hkv,
+                        float scale, const void* k_new, const void* v_new, void* k_hot,
+                        void* v_hot, int W_max, int32_t* hot_start, int32_t* hot_len,
+                        uint8_t* pool, int64_t pool_pages, const int32_t* page_table,
+                        int max_pages, int32_t* cold_len, float threshold, int window,
+                        int evict_block, int32_t* cold_used, float* out, void* ws,
+                        size_t ws_bytes, void* stream);
+size_t monarch_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages,
+                               int W_max, int evict_block);
 
 int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* db, int64_t N,
                 int k, int32_t* out_ids, float* out_scores, void* ws, size_t ws_bytes,

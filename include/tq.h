@@ -231,6 +231,47 @@ TQ_API tq_status tq_decode_attention_gated(const tq_ctx* ctx, const void* q, tq_
                                            const int32_t* cold_len, float threshold,
                                            int32_t* cold_used, float* out, void* workspace,
                                            size_t ws_bytes, void* stream);
+/* Workspace bytes tq_monarch_step needs. */
+TQ_API size_t tq_monarch_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages,
+                                         int W_max, int evict_block);
+/*
+ * One decode step of Monarch's hot/cold cache ("Monarch v3: NES-inspiriertes
+ * KV-Paging", sections "Wie es funktioniert" and "Vereinfachte
+ * Decode-Schleife"), all on the stream, nothing on the host:
+ *  1. append  k_new, v_new (device fp16 [B, Hkv, d], both NULL to skip): the
+ *             token joins the hot ring of every kv head at slot
+ *             (hot_start[b] + hot_len[b]) mod W_max and hot_len[b] grows by
+ *             one.  A full ring (hot_len == W_max) is a device error
+ *             (TQ_ERR_CAPACITY) and the token is dropped.
+ *  2. attend  tq_decode_attention_gated over the ring (with the new token)
+ *             and the cold pages, threshold and cold_used as there.
+ *  3. evict   every sequence whose hot window now holds at least
+ *             window + evict_block tokens has its oldest evict_block hot
+ *             tokens compressed (tq_compress_append from fp16) and appended to
+ *             its cold pages; hot_start advances by evict_block (mod W_max),
+ *             hot_len shrinks and cold_len grows by it.  evict_block = 1 is
+ *             the loop as written (evict whenever the window is exceeded);
+ *             larger blocks keep between window and window + evict_block - 1
+ *             tokens hot and compress a block at a time.
+ *  k_hot, v_hot  device fp16 [B, Hkv, W_max, d], read and written.
+ *  hot_start, hot_len, cold_len  device int32 [B], read and written.
+ *  page_pool, pool_pages, page_table, max_pages  values pages, as in
+ *             tq_compress_append.
+ *  workspace  device, 256-byte aligned, ws_bytes >=
+ *             tq_monarch_workspace_bytes(ctx, B, Hq, Hkv, max_pages, W_max,
+ *             evict_block).
+ * Requires window >= 0, evict_block >= 1 and window + evict_block <= W_max
+ * (the ring never overflows while hot_len < window + evict_block holds
+ * before a step).
+ */
+TQ_API tq_status tq_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                                 int Hkv, float scale, const void* k_new, const void* v_new,
+                                 void* k_hot, void* v_hot, int W_max, int32_t* hot_start,
+                                 int32_t* hot_len, uint8_t* page_pool, int64_t pool_pages,
+                                 const int32_t* page_table, int max_pages, int32_t* cold_len,
+                                 float threshold, int window, int evict_block,
+                                 int32_t* cold_used, float* out, void* workspace,
+                                 size_t ws_bytes, void* stream);
 /* Largest decode workspace tq_decode_attention_noalloc can serve (8 MiB). */
 #define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 
