@@ -71,6 +71,16 @@ def lib():
         L.or_topk.argtypes = [C.c_int, C.c_int, dp, dp, dp, dp, C.c_int, u8, sz, C.c_int64,
                               C.c_int, ip, dp, C.c_int]
         L.or_max_threads.restype = C.c_int
+        L.or_angle_lloyd_max.argtypes = [C.c_int, C.c_int, C.c_int, dp, dp]
+        L.or_angle_lloyd_max.restype = C.c_int
+        L.or_polar_code_bytes.argtypes = [C.c_int, C.c_int, C.c_int]
+        L.or_polar_code_bytes.restype = sz
+        L.or_polar_encode.argtypes = [C.c_int, C.POINTER(C.c_float), C.c_int64, C.c_int, C.c_int,
+                                      u8, C.POINTER(C.c_uint16)]
+        L.or_polar_decode.argtypes = [C.c_int, u8, C.POINTER(C.c_uint16), C.c_int64, C.c_int,
+                                      C.c_int, dp]
+        L.or_polar_transform.argtypes = [C.c_int, dp, dp, dp]
+        L.or_polar_inverse.argtypes = [C.c_int, C.c_double, dp, dp]
         _lib = L
     return _lib
 
@@ -340,3 +350,121 @@ def topk(params, queries, db_pool, page_bytes, N, k, threads=0):
 
 def max_threads():
     return lib().or_max_threads()
+
+
+# --------------------------------------------------------------------------
+# stage-1 variants: PolarQuant and MSE-only b-bit codes
+# --------------------------------------------------------------------------
+def angle_lloyd_max(k, bits, max_iter=100000):
+    """Lloyd-Max levels and boundaries of the angle between two blocks of k
+    coordinates (density proportional to sin^(k-1)(2 phi) on [0, pi/2])."""
+    c = np.empty(1 << bits)
+    t = np.empty((1 << bits) - 1)
+    it = lib().or_angle_lloyd_max(k, bits, max_iter, c.ctypes.data_as(C.POINTER(C.c_double)),
+                                  t.ctypes.data_as(C.POINTER(C.c_double)))
+    return c, t, it
+
+
+def polar_code_bytes(d, b1, b2):
+    return int(lib().or_polar_code_bytes(d, b1, b2))
+
+
+def polar_encode(x, b1, b2):
+    """x [N, d] rotated vectors (rounded to fp32).  Returns codes uint8
+    [N, polar_code_bytes] and the fp16 bits of the final radii [N]."""
+    x = np.ascontiguousarray(np.asarray(x, np.float32))
+    N, d = x.shape
+    cb = polar_code_bytes(d, b1, b2)
+    codes = np.zeros((N, cb), np.uint8)
+    rad = np.zeros(N, np.uint16)
+    lib().or_polar_encode(d, x.ctypes.data_as(C.POINTER(C.c_float)), N, b1, b2, _u8(codes),
+                          rad.ctypes.data_as(C.POINTER(C.c_uint16)))
+    return codes, rad
+
+
+def polar_decode(codes, rad, d, b1, b2):
+    codes = np.ascontiguousarray(codes, np.uint8)
+    rad = np.ascontiguousarray(rad, np.uint16)
+    N = codes.shape[0]
+    out = np.empty((N, d))
+    lib().or_polar_decode(d, _u8(codes), rad.ctypes.data_as(C.POINTER(C.c_uint16)), N, b1, b2,
+                          out.ctypes.data_as(C.POINTER(C.c_double)))
+    return out
+
+
+def polar_transform(x):
+    """Exact (fp64) transform of one vector: final radius, angles (level 1
+    first, then levels 2, 3, ...)."""
+    x, xp = _d(x)
+    d = x.shape[0]
+    r = C.c_double()
+    ang = np.empty(d - 1)
+    lib().or_polar_transform(d, xp, C.byref(r), ang.ctypes.data_as(C.POINTER(C.c_double)))
+    return r.value, ang
+
+
+def polar_inverse(radius, angles):
+    angles, ap = _d(angles)
+    d = angles.shape[0] + 1
+    out = np.empty(d)
+    lib().or_polar_inverse(d, float(radius), ap, out.ctypes.data_as(C.POINTER(C.c_double)))
+    return out
+
+
+def mse_pack(sign, mag, bits):
+    """MSE-only b-bit codes, one vector per row: code_j = sign << (b-1) | mag
+    in bits [b j, b j + b) of a little-endian bit stream."""
+    sign = np.asarray(sign, np.int64)
+    mag = np.asarray(mag, np.int64)
+    N, d = sign.shape
+    code = (sign << (bits - 1)) | mag
+    out = np.zeros((N, (bits * d + 7) // 8), np.uint8)
+    for j in range(d):
+        for i in range(bits):
+            pos = bits * j + i
+            out[:, pos >> 3] |= (((code[:, j] >> i) & 1) << (pos & 7)).astype(np.uint8)
+    return out
+
+
+def mse_unpack(packed, d, bits):
+    packed = np.asarray(packed, np.uint8)
+    N = packed.shape[0]
+    code = np.zeros((N, d), np.int64)
+    for j in range(d):
+        for i in range(bits):
+            pos = bits * j + i
+            code[:, j] |= ((packed[:, pos >> 3] >> (pos & 7)) & 1).astype(np.int64) << i
+    return code >> (bits - 1), code & ((1 << (bits - 1)) - 1)
+
+
+def mse_encode(params, x_rot, bits):
+    """MSE-only b-bit stage 1 on rotated vectors: the oracle's quantiser with
+    a 2^(b-1)-level Lloyd-Max codebook (no QJL).  Returns packed codes, the
+    fp16 norms and the codebook."""
+    p = params
+    x = np.asarray(x_rot, np.float64).reshape(-1, p.d)
+    c, t, _, _ = lloyd_max(p.d, bits)
+    f32 = lambda a: a.astype(np.float32).astype(np.float64)
+    cpos, tpos = f32(c), f32(t)
+    N = x.shape[0]
+    sign = np.empty((N, p.d), np.int32)
+    mag = np.empty((N, p.d), np.int32)
+    qbits = np.zeros((N, p.m), np.int32)
+    n = np.empty(N)
+    gamma = np.zeros(N)
+    xr = np.empty((N, p.d))
+    x, xp = _d(x)
+    pi, pip = _d(p.pi32)
+    S, Sp = _d(p.S)
+    cp_, cpp = _d(cpos)
+    tp_, tpp = _d(tpos)
+    ptr = lambda a, ty: a.ctypes.data_as(C.POINTER(ty))
+    lib().or_encode(p.d, p.m, pip, Sp, cpp, tpp, len(cpos), xp, N, 1, 0, ptr(sign, C.c_int32),
+                    ptr(mag, C.c_int32), ptr(qbits, C.c_int32), ptr(n, C.c_double),
+                    ptr(gamma, C.c_double), ptr(xr, C.c_double), 0)
+    return mse_pack(sign, mag, bits), n, cpos
+
+
+def mse_decode(packed, n, cpos, d, bits):
+    sign, mag = mse_unpack(packed, d, bits)
+    return np.asarray(n)[:, None] * np.where(sign == 1, -1.0, 1.0) * cpos[mag]

@@ -909,3 +909,242 @@ OR_API int or_max_threads(void) {
   return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------ */
+/* Stage-1 variant: PolarQuant [TQ "PolarQuant: Ein neuer Winkel auf        */
+/* Kompression": pairs of coordinates go to polar form, the radii are       */
+/* paired again and the transform repeats until one radius and a set of     */
+/* angles remain; the angles, whose distribution is known and concentrated, */
+/* are quantised on a fixed grid].                                          */
+/*                                                                           */
+/* Applied to the rotated vector.  Level 1 pairs coordinates (2i, 2i+1):    */
+/* angle theta in [0, 2 pi), uniform for a rotated vector, quantised on     */
+/* 2^b1 equal bins with the bin centres as levels (the Lloyd-Max quantiser  */
+/* of a uniform angle).  Level l >= 2 pairs the radii (r_e, r_o) of two      */
+/* blocks of k = 2^(l-1) coordinates: phi = atan(r_o / r_e) in [0, pi/2]    */
+/* has density proportional to sin^(k-1)(2 phi) (cos^2 phi is Beta(k/2,     */
+/* k/2) for a uniform direction), quantised with its own 2^b2-level          */
+/* Lloyd-Max codebook.  The last radius is stored as fp16.                   */
+/*                                                                           */
+/* Every decision is taken in fp32 exactly as stated here, so that a GPU    */
+/* encoder given the same fp32 inputs takes the same ones: radii            */
+/* sqrtf(fmaf(u, u, v * v)); level 1 reduces (a, b) to the first quadrant   */
+/* by exact swaps and negations and counts the boundaries tan(2 pi j / M)   */
+/* (fp32) with b' >= a' * t; level l counts the boundaries tan(t_j) (fp32)   */
+/* with r_o >= r_e * T (only when r_o > 0).  A zero pair has angle 0.        */
+/* ------------------------------------------------------------------------ */
+
+/* int_a^b phi^order sin^(k-1)(2 phi) dphi, composite Gauss-Legendre */
+static double angle_moment(int k, double a, double b, int order) {
+  gl_init();
+  if (b <= a) return 0.0;
+  int panels = (int)ceil((b - a) / 0.01);
+  double h = (b - a) / panels, s = 0.0;
+  for (int p = 0; p < panels; ++p) {
+    double lo = a + p * h, hh = 0.5 * h, c = lo + hh, ps = 0.0;
+    for (int i = 0; i < GL_N; ++i) {
+      double x = c + hh * gl_x[i];
+      double f = pow(sin(2.0 * x), k - 1);
+      ps += gl_w[i] * (order ? x * f : f);
+    }
+    s += ps * hh;
+  }
+  return s;
+}
+
+/* Lloyd-Max codebook of the level angle for blocks of k coordinates:
+ * 2^bits levels c (increasing) and 2^bits - 1 boundaries t on [0, pi/2]. */
+OR_API int or_angle_lloyd_max(int k, int bits, int max_iter, double* c, double* t) {
+  int L = 1 << bits;
+  for (int j = 0; j < L; ++j) c[j] = (j + 0.5) * (M_PI / 2.0) / L;
+  int it = 0;
+  for (; it < max_iter; ++it) {
+    for (int j = 0; j + 1 < L; ++j) t[j] = 0.5 * (c[j] + c[j + 1]);
+    double delta = 0.0;
+    for (int j = 0; j < L; ++j) {
+      double a = (j == 0) ? 0.0 : t[j - 1];
+      double b = (j == L - 1) ? M_PI / 2.0 : t[j];
+      double nc = angle_moment(k, a, b, 1) / angle_moment(k, a, b, 0);
+      delta = fmax(delta, fabs(nc - c[j]));
+      c[j] = nc;
+    }
+    if (delta < 1e-15) { ++it; break; }
+  }
+  for (int j = 0; j + 1 < L; ++j) t[j] = 0.5 * (c[j] + c[j + 1]);
+  return it;
+}
+
+static int polar_levels(int d) { /* levels >= 2: log2(d) - 1 */
+  int n = 0;
+  for (int v = d / 2; v > 1; v >>= 1) ++n;
+  return n;
+}
+
+static void put_bits(uint8_t* dst, size_t bitpos, int nbits, uint32_t v) {
+  for (int i = 0; i < nbits; ++i)
+    if ((v >> i) & 1u) dst[(bitpos + i) >> 3] |= (uint8_t)(1u << ((bitpos + i) & 7));
+}
+
+static uint32_t get_bits(const uint8_t* src, size_t bitpos, int nbits) {
+  uint32_t v = 0;
+  for (int i = 0; i < nbits; ++i)
+    v |= (uint32_t)((src[(bitpos + i) >> 3] >> ((bitpos + i) & 7)) & 1u) << i;
+  return v;
+}
+
+/* bytes of one vector's angle codes */
+OR_API size_t or_polar_code_bytes(int d, int b1, int b2) {
+  size_t bits = (size_t)b1 * (d / 2) + (size_t)b2 * (d / 2 - 1);
+  return (bits + 7) / 8;
+}
+
+/* level-1 bin of the pair (a, b) among M = 2^b1 equal bins of [0, 2 pi) */
+static int level1_bin(float a, float b, int M, const float* tq /* M/4 - 1 */) {
+  int q;
+  float u, v; /* the pair turned into the first quadrant [0, pi/2) */
+  if (a > 0.0f && b >= 0.0f) { q = 0; u = a; v = b; }
+  else if (a <= 0.0f && b > 0.0f) { q = 1; u = b; v = -a; }
+  else if (a < 0.0f && b <= 0.0f) { q = 2; u = -a; v = -b; }
+  else if (a >= 0.0f && b < 0.0f) { q = 3; u = -b; v = a; }
+  else { return 0; } /* zero pair */
+  int j = 0;
+  for (int i = 0; i < M / 4 - 1; ++i)
+    if (v >= u * tq[i]) j = i + 1;
+  return q * (M / 4) + j;
+}
+
+/* x: N rotated vectors (fp32); codes: N * or_polar_code_bytes bytes
+ * (zeroed here); radius: fp16 bits of the final radius.  b1 >= 2. */
+OR_API void or_polar_encode(int d, const float* x, int64_t N, int b1, int b2, uint8_t* codes,
+                            uint16_t* radius) {
+  int M = 1 << b1, L = 1 << b2, nl = polar_levels(d);
+  size_t cb = or_polar_code_bytes(d, b1, b2);
+  float tq[64];
+  for (int i = 0; i < M / 4 - 1; ++i) tq[i] = (float)tan(2.0 * M_PI * (i + 1) / M);
+  float T[16][16];
+  double c[64], t[64];
+  for (int l = 0; l < nl; ++l) {
+    or_angle_lloyd_max(1 << (l + 1), b2, 100000, c, t);
+    for (int j = 0; j < L - 1; ++j) T[l][j] = (float)tan(t[j]);
+  }
+  float* r = (float*)malloc(sizeof(float) * (d / 2));
+  for (int64_t n = 0; n < N; ++n) {
+    const float* v = x + (size_t)n * d;
+    uint8_t* out = codes + (size_t)n * cb;
+    memset(out, 0, cb);
+    size_t pos = 0;
+    for (int i = 0; i < d / 2; ++i) {
+      float a = v[2 * i], b = v[2 * i + 1];
+      put_bits(out, pos, b1, (uint32_t)level1_bin(a, b, M, tq));
+      pos += b1;
+      r[i] = sqrtf(fmaf(a, a, b * b));
+    }
+    int nodes = d / 2;
+    for (int l = 0; l < nl; ++l) {
+      nodes /= 2;
+      for (int i = 0; i < nodes; ++i) {
+        float re = r[2 * i], ro = r[2 * i + 1];
+        int j = 0;
+        if (ro > 0.0f)
+          for (int s = 0; s < L - 1; ++s)
+            if (ro >= re * T[l][s]) j = s + 1;
+        put_bits(out, pos, b2, (uint32_t)j);
+        pos += b2;
+        r[i] = sqrtf(fmaf(re, re, ro * ro));
+      }
+    }
+    radius[n] = f16_bits(or_round_f16((double)r[0]));
+  }
+  free(r);
+}
+
+/* reconstruction (fp64) from the codes and the fp16 radius */
+OR_API void or_polar_decode(int d, const uint8_t* codes, const uint16_t* radius, int64_t N, int b1,
+                            int b2, double* xhat) {
+  int M = 1 << b1, L = 1 << b2, nl = polar_levels(d);
+  size_t cb = or_polar_code_bytes(d, b1, b2);
+  double cl[16][16], t[64];
+  for (int l = 0; l < nl; ++l) or_angle_lloyd_max(1 << (l + 1), b2, 100000, cl[l], t);
+  double* r = (double*)malloc(sizeof(double) * (d / 2));
+  double* rn = (double*)malloc(sizeof(double) * (d / 2));
+  for (int64_t n = 0; n < N; ++n) {
+    const uint8_t* in = codes + (size_t)n * cb;
+    r[0] = f16_value(radius[n]);
+    /* level-l codes start after the level-1 codes and the lower levels' */
+    size_t base = (size_t)b1 * (d / 2);
+    size_t off[16];
+    int cnt = d / 2;
+    for (int l = 0; l < nl; ++l) {
+      cnt /= 2;
+      off[l] = base;
+      base += (size_t)b2 * cnt;
+    }
+    int nodes = 1;
+    for (int l = nl - 1; l >= 0; --l) {
+      for (int i = 0; i < nodes; ++i) {
+        double phi = cl[l][get_bits(in, off[l] + (size_t)b2 * i, b2)];
+        rn[2 * i] = r[i] * cos(phi);
+        rn[2 * i + 1] = r[i] * sin(phi);
+      }
+      nodes *= 2;
+      memcpy(r, rn, sizeof(double) * nodes);
+    }
+    double* o = xhat + (size_t)n * d;
+    for (int i = 0; i < d / 2; ++i) {
+      double th = 2.0 * M_PI * (get_bits(in, (size_t)b1 * i, b1) + 0.5) / M;
+      o[2 * i] = r[i] * cos(th);
+      o[2 * i + 1] = r[i] * sin(th);
+    }
+  }
+  free(r);
+  free(rn);
+}
+
+/* the exact transform (no quantisation), fp64: final radius and the angles
+ * (level 1 first, then levels 2, 3, ...), and its inverse */
+OR_API void or_polar_transform(int d, const double* x, double* radius, double* angles) {
+  double* r = (double*)malloc(sizeof(double) * (d / 2));
+  int k = 0;
+  for (int i = 0; i < d / 2; ++i) {
+    double th = atan2(x[2 * i + 1], x[2 * i]);
+    angles[k++] = th < 0.0 ? th + 2.0 * M_PI : th;
+    r[i] = hypot(x[2 * i], x[2 * i + 1]);
+  }
+  for (int nodes = d / 4; nodes >= 1; nodes /= 2)
+    for (int i = 0; i < nodes; ++i) {
+      angles[k++] = atan2(r[2 * i + 1], r[2 * i]);
+      r[i] = hypot(r[2 * i], r[2 * i + 1]);
+    }
+  *radius = r[0];
+  free(r);
+}
+
+OR_API void or_polar_inverse(int d, double radius, const double* angles, double* x) {
+  double* r = (double*)malloc(sizeof(double) * d);
+  double* rn = (double*)malloc(sizeof(double) * d);
+  int nl = polar_levels(d);
+  size_t off[16];
+  size_t base = (size_t)(d / 2);
+  int cnt = d / 2;
+  for (int l = 0; l < nl; ++l) {
+    cnt /= 2;
+    off[l] = base;
+    base += cnt;
+  }
+  r[0] = radius;
+  int nodes = 1;
+  for (int l = nl - 1; l >= 0; --l) {
+    for (int i = 0; i < nodes; ++i) {
+      rn[2 * i] = r[i] * cos(angles[off[l] + i]);
+      rn[2 * i + 1] = r[i] * sin(angles[off[l] + i]);
+    }
+    nodes *= 2;
+    memcpy(r, rn, sizeof(double) * nodes);
+  }
+  for (int i = 0; i < d / 2; ++i) {
+    x[2 * i] = r[i] * cos(angles[i]);
+    x[2 * i + 1] = r[i] * sin(angles[i]);
+  }
+  free(r);
+  free(rn);
+}
