@@ -337,6 +337,62 @@ def measure_monarch(torch, tq, W, workload, evict_block, thresholds=(float("inf"
     return res
 
 
+def measure_stage1(torch, tq, N=1 << 20, reps=5):
+    """Stage-1 variants on 2^20 rotated fp32 vectors (d = 128, N(0,1)):
+    encode and decode kernel times (CUDA events, median of reps) with their
+    HBM bytes, and the distortion of encode -> decode (relative MSE, and the
+    RMS inner-product error against 64 random unit queries) on the first
+    65536 vectors."""
+    d = 128
+    ctx = tq.Context(d, seed=0)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(41)
+    x = torch.randn((N, d), generator=gen, device="cuda")
+    q = torch.randn((64, d), generator=gen, device="cuda", dtype=torch.float64)
+    q /= q.norm(dim=1, keepdim=True)
+    xh = torch.empty_like(x)
+    peaks, _ = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    res = []
+    for kind, b1, b2, name in ((tq.TQ_STAGE1_POLAR, 4, 2, "polar b1=4 b2=2"),
+                               (tq.TQ_STAGE1_MSE, 3, 0, "mse b=3"),
+                               (tq.TQ_STAGE1_MSE, 2, 0, "mse b=2"),
+                               (tq.TQ_STAGE1_MSE, 4, 0, "mse b=4")):
+        cb = tq.tq_stage1_code_bytes(ctx.handle, kind, b1, b2)
+        codes = torch.empty((N, cb), dtype=torch.uint8, device="cuda")
+        norms = torch.empty(N, dtype=torch.int16, device="cuda")
+        times = {"encode": [], "decode": []}
+        for i in range(reps + 1):
+            for what in ("encode", "decode"):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                if what == "encode":
+                    tq.tq_stage1_encode(ctx.handle, kind, b1, b2, x, codes, norms)
+                else:
+                    tq.tq_stage1_decode(ctx.handle, kind, b1, b2, codes, norms, xh)
+                b.record()
+                torch.cuda.synchronize()
+                if i > 0:
+                    times[what].append(a.elapsed_time(b))
+        n_s = 65536
+        xs, hs = x[:n_s].double(), xh[:n_s].double()
+        rel = ((hs - xs) ** 2).sum(1) / (xs ** 2).sum(1)
+        ip = (hs - xs) @ q.T
+        row = {"variant": name, "code_bytes_per_vector": cb + 2,
+               "bits_per_coordinate": 8.0 * (cb + 2) / d,
+               "relative_mse": float(rel.mean()), "ip_rms_error": float(ip.pow(2).mean().sqrt())}
+        for what in ("encode", "decode"):
+            ms = statistics.median(times[what])
+            by = N * (d * 4 + cb + 2)
+            row[what + "_ms"] = ms
+            row[what + "_gbs"] = by / (ms / 1e3) / 1e9
+            row[what + "_hbm_frac"] = row[what + "_gbs"] / peak
+        res.append(row)
+        del codes, norms
+    ctx.check()
+    return {"workload": "2^20 rotated N(0,1) vectors, d=128, fp32", "variants": res}
+
+
 def decode(tq, st, q=None, out=None):
     tq.tq_decode_attention(st["ctx"].handle, st["q"] if q is None else q, st["k_hot"],
                            st["v_hot"], st["hot_len"], st["pool"], st["table"], st["cold_len"],
@@ -518,6 +574,8 @@ def run_ours(args, rank, world, local_rank):
         rows["compress"] = measure_compress(torch, tq)
         torch.cuda.empty_cache()
         rows["search"] = measure_search(torch, tq)
+        torch.cuda.empty_cache()
+        rows["stage1"] = measure_stage1(torch, tq)
         peak_tf = float(peaks.get("bf16_tflops", 1590.0))
         rows["compress"]["hbm_frac"] = rows["compress"]["achieved_gbs"] / peak
         rows["compress"]["tensor_frac"] = rows["compress"]["achieved_tflops"] / peak_tf

@@ -76,6 +76,14 @@ def lib():
                                       C.c_int, i32p, C.c_float, C.c_int, C.c_int, i32p, f32p, vp,
                                       C.c_size_t, vp]
         L.tq_monarch_step.restype = C.c_int
+        L.tq_stage1_code_bytes.argtypes = [vp, C.c_int, C.c_int, C.c_int]
+        L.tq_stage1_code_bytes.restype = C.c_size_t
+        L.tq_stage1_encode.argtypes = [vp, C.c_int, C.c_int, C.c_int, f32p, C.c_int64, u8p, vp,
+                                       vp]
+        L.tq_stage1_encode.restype = C.c_int
+        L.tq_stage1_decode.argtypes = [vp, C.c_int, C.c_int, C.c_int, u8p, vp, C.c_int64, f32p,
+                                       vp]
+        L.tq_stage1_decode.restype = C.c_int
         L.tq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int,
                                                   C.c_float, vp, vp, C.c_int, i32p, u8p, C.c_int64,
                                                   i32p, C.c_int, i32p, f32p, vp]
@@ -256,6 +264,29 @@ def tq_monarch_step(ctx, q, k_new, v_new, k_hot, v_hot, hot_start, hot_len, page
         float(threshold), int(window), int(evict_block), _ptr(cold_used), _ptr(out),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
         "tq_monarch_step")
+
+
+TQ_STAGE1_MSE, TQ_STAGE1_POLAR = 0, 1
+
+
+def tq_stage1_code_bytes(ctx, kind, bits1, bits2=0):
+    return int(lib().tq_stage1_code_bytes(ctx, kind, bits1, bits2))
+
+
+def tq_stage1_encode(ctx, kind, bits1, bits2, x_rot, codes, norms, stream=None):
+    """x_rot fp32 [N, d] -> codes uint8 [N, code_bytes], norms fp16-bits
+    (int16 / uint16 tensor) [N]."""
+    _require_cuda(x_rot, codes, norms)
+    _check(lib().tq_stage1_encode(ctx, int(kind), int(bits1), int(bits2), _ptr(x_rot),
+                                  x_rot.shape[0], _ptr(codes), _ptr(norms), _stream(stream)),
+           "tq_stage1_encode")
+
+
+def tq_stage1_decode(ctx, kind, bits1, bits2, codes, norms, x_hat, stream=None):
+    _require_cuda(codes, norms, x_hat)
+    _check(lib().tq_stage1_decode(ctx, int(kind), int(bits1), int(bits2), _ptr(codes),
+                                  _ptr(norms), codes.shape[0], _ptr(x_hat), _stream(stream)),
+           "tq_stage1_decode")
 
 
 def tq_decode_attention_noalloc(ctx, q, k_hot, v_hot, hot_len, page_pool, page_table, cold_len,

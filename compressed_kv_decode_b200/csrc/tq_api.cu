@@ -309,6 +309,29 @@ tq_status tq_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, in
       cold_used, out, workspace, ws_bytes, stream));
 }
 
+size_t tq_stage1_code_bytes(const tq_ctx* ctx, int kind, int bits1, int bits2) {
+  if (!ctx) return 0;
+  return tq::stage1_code_bytes(ctx->cfg.head_dim, kind, bits1, bits2);
+}
+
+tq_status tq_stage1_encode(const tq_ctx* ctx, int kind, int bits1, int bits2, const float* x_rot,
+                           int64_t N, uint8_t* codes, uint16_t* norms, void* stream) {
+  if (!ctx || N < 0 || (N > 0 && (!x_rot || !codes || !norms))) return TQ_ERR_INVALID_ARG;
+  if (N > 0 && !tq::aligned(x_rot, 16)) return TQ_ERR_INVALID_ARG;
+  if (tq::stage1_code_bytes(ctx->cfg.head_dim, kind, bits1, bits2) == 0) return TQ_ERR_UNSUPPORTED;
+  return static_cast<tq_status>(tq::launch_stage1(ctx, kind, bits1, bits2, true, x_rot, nullptr,
+                                                  codes, nullptr, norms, nullptr, N, stream));
+}
+
+tq_status tq_stage1_decode(const tq_ctx* ctx, int kind, int bits1, int bits2, const uint8_t* codes,
+                           const uint16_t* norms, int64_t N, float* x_hat, void* stream) {
+  if (!ctx || N < 0 || (N > 0 && (!x_hat || !codes || !norms))) return TQ_ERR_INVALID_ARG;
+  if (N > 0 && !tq::aligned(x_hat, 16)) return TQ_ERR_INVALID_ARG;
+  if (tq::stage1_code_bytes(ctx->cfg.head_dim, kind, bits1, bits2) == 0) return TQ_ERR_UNSUPPORTED;
+  return static_cast<tq_status>(tq::launch_stage1(ctx, kind, bits1, bits2, false, nullptr, codes,
+                                                  nullptr, norms, nullptr, x_hat, N, stream));
+}
+
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k) {
   if (!ctx || Q <= 0 || N <= 0 || k <= 0) return 0;
   return tq::topk_workspace_bytes(ctx, Q, N, k);

@@ -21,6 +21,11 @@ struct HostTables {
 bool config_valid(const tq_config& c);
 bool config_supported(const tq_config& c);
 bool generate_tables(const tq_config& cfg, HostTables& out);
+// Lloyd-Max codebooks used by the stage-1 variants (fp64 results):
+// positive levels / boundaries of one sphere coordinate at `bits` bits, and
+// the levels / boundaries of the block-pair angle (density sin^(k-1)(2 phi)).
+void sphere_lloyd_max(int d, int bits, std::vector<double>& c, std::vector<double>& t);
+void angle_lloyd_max(int k, int bits, std::vector<double>& c, std::vector<double>& t);
 
 // Small per-context constants passed to kernels by value.
 struct Codebook {
@@ -102,6 +107,10 @@ int launch_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int 
                         int max_pages, int32_t* cold_len, float threshold, int window,
                         int evict_block, int32_t* cold_used, float* out, void* ws,
                         size_t ws_bytes, void* stream);
+size_t stage1_code_bytes(int d, int kind, int b1, int b2);
+int launch_stage1(const tq_ctx* ctx, int kind, int b1, int b2, bool encode, const float* x,
+                  const uint8_t* codes_in, uint8_t* codes_out, const uint16_t* norms_in,
+                  uint16_t* norms_out, float* xhat, long long N, void* stream);
 size_t monarch_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages,
                                int W_max, int evict_block);
 

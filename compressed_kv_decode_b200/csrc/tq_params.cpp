@@ -157,6 +157,57 @@ void lloyd_max(int d, int bits, std::vector<double>& c_out, std::vector<double>&
   t_out.assign(t.begin(), t.end());
 }
 
+// Lloyd-Max levels and boundaries of the angle phi = atan(r_o / r_e) between
+// the radii of two blocks of k coordinates of a uniform direction, density
+// proportional to sin^(k-1)(2 phi) on [0, pi/2]: cell masses and first
+// moments by composite Simpson (double): iterated to a 1e-13 fixed point on a
+// coarse rule, then polished on a rule 16 times finer (Simpson's error falls
+// as the fourth power of the step) to a 1e-14 fixed point.
+double angle_integral(int k, double a, double b, int order, int n /* even */) {
+  const double h = (b - a) / n;
+  double s = 0.0;
+  for (int i = 0; i <= n; ++i) {
+    const double x = a + h * i;
+    const double f = std::pow(std::sin(2.0 * x), k - 1) * (order ? x : 1.0);
+    s += f * ((i == 0 || i == n) ? 1.0 : ((i & 1) ? 4.0 : 2.0));
+  }
+  return s * h / 3.0;
+}
+
+}  // namespace
+
+void angle_lloyd_max(int k, int bits, std::vector<double>& c_out, std::vector<double>& t_out) {
+  const int L = 1 << bits;
+  const double half_pi = 1.5707963267948966192;
+  std::vector<double> c(L), t(L - 1);
+  for (int j = 0; j < L; ++j) c[j] = half_pi * (j + 0.5) / L;
+  for (int phase = 0; phase < 2; ++phase) {
+    const int n = phase == 0 ? 1000 : 16000;
+    const double tol = phase == 0 ? 1e-13 : 1e-14;
+    for (int it = 0; it < 20000; ++it) {
+      for (int j = 0; j + 1 < L; ++j) t[j] = 0.5 * (c[j] + c[j + 1]);
+      double delta = 0.0;
+      for (int j = 0; j < L; ++j) {
+        const double a = (j == 0) ? 0.0 : t[j - 1];
+        const double b = (j == L - 1) ? half_pi : t[j];
+        const double nc = angle_integral(k, a, b, 1, n) / angle_integral(k, a, b, 0, n);
+        delta = std::fmax(delta, std::fabs(nc - c[j]));
+        c[j] = nc;
+      }
+      if (delta < tol) break;
+    }
+  }
+  for (int j = 0; j + 1 < L; ++j) t[j] = 0.5 * (c[j] + c[j + 1]);
+  c_out = c;
+  t_out = t;
+}
+
+void sphere_lloyd_max(int d, int bits, std::vector<double>& c_out, std::vector<double>& t_out) {
+  lloyd_max(d, bits, c_out, t_out);
+}
+
+namespace {
+
 float round_to_half(double x) {
   // nearest fp16 value (ties to even), returned as float
   if (x == 0.0 || !std::isfinite(x)) return static_cast<float>(x);

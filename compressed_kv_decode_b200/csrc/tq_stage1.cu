@@ -1,0 +1,403 @@
+// Stage-1 quantiser variants on rotated vectors ("TurboQuant" summary,
+// de.news.hada.io topic 27867, section "Funktionsweise von TurboQuant": a
+// standard per-coordinate quantiser after the rotation; section "PolarQuant:
+// Ein neuer Winkel auf Kompression": pairs of coordinates to polar form, the
+// radii paired again recursively until one radius and a set of angles
+// remain, the angles quantised on fixed grids).
+//
+//  MSE    b bits per coordinate: sign + (b-1)-bit Lloyd-Max magnitude index of
+//         x_rot / n, n = fp16(|x|); no QJL sketch.  Code of coordinate j in
+//         bits [b j, b j + b) of a little-endian bit stream.
+//  POLAR  level-1 angles of the coordinate pairs on 2^b1 equal bins of
+//         [0, 2 pi), level-l angles (l >= 2) of the block radii with a
+//         2^b2-level Lloyd-Max codebook of their density sin^(k-1)(2 phi),
+//         k = 2^(l-1); the final radius as fp16.  Codes: level 1 first (b1
+//         bits per pair), then level 2, 3, ... (b2 bits per node).
+//
+// One warp per vector, D/32 coordinates per lane (coalesced 8- or 16-byte
+// loads).  Every decision is an fp32 comparison whose operands are formed the
+// same way in the CPU oracle: radii sqrtf(fmaf(u, u, v * v)), level-1 bins by
+// exact turns into the first quadrant and v >= u * tan(boundary), higher
+// levels by r_o >= r_e * tan(boundary), MSE codes by |x_j| >= fp32(n t_k).
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "tq_device.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+namespace s1 {
+
+constexpr int MAX_LEVELS = 6;  // levels >= 2 at d = 128
+constexpr int MAX_B2 = 8;      // 2^3 levels per higher-level angle
+
+struct PolarTables {
+  float tq1[7];              // tan(2 pi j / M), j = 1 .. M/4 - 1 (first-quadrant boundaries)
+  float cos1[32], sin1[32];  // level-1 bin centres
+  float T[MAX_LEVELS][MAX_B2 - 1];  // tan of the level boundaries
+  float cosl[MAX_LEVELS][MAX_B2], sinl[MAX_LEVELS][MAX_B2];
+};
+
+struct MseTables {
+  float c[8];  // positive levels
+  float t[7];  // positive boundaries
+};
+
+__host__ __device__ constexpr int log2i(int v) { return v <= 1 ? 0 : 1 + log2i(v / 2); }
+
+__device__ __forceinline__ void or_bits(uint32_t* words, int pos, int nbits, uint32_t v) {
+  const int w = pos >> 5, o = pos & 31;
+  atomicOr(&words[w], v << o);
+  if (o + nbits > 32) atomicOr(&words[w + 1], v >> (32 - o));
+}
+
+__device__ __forceinline__ uint32_t read_bits(const uint32_t* words, int pos, int nbits) {
+  const int w = pos >> 5, o = pos & 31;
+  uint64_t x = words[w];
+  if (o + nbits > 32) x |= static_cast<uint64_t>(words[w + 1]) << 32;
+  return static_cast<uint32_t>(x >> o) & ((1u << nbits) - 1u);
+}
+
+__device__ __forceinline__ float tree_radius(float u, float v) {
+  return __fsqrt_rn(__fmaf_rn(u, u, __fmul_rn(v, v)));
+}
+
+__device__ __forceinline__ int level1_bin(float a, float b, int M, const PolarTables& tb) {
+  int q;
+  float u, v;
+  if (a > 0.0f && b >= 0.0f) { q = 0; u = a; v = b; }
+  else if (a <= 0.0f && b > 0.0f) { q = 1; u = b; v = -a; }
+  else if (a < 0.0f && b <= 0.0f) { q = 2; u = -a; v = -b; }
+  else if (a >= 0.0f && b < 0.0f) { q = 3; u = -b; v = a; }
+  else return 0;  // zero pair
+  int j = 0;
+  for (int i = 0; i < M / 4 - 1; ++i)
+    if (v >= __fmul_rn(u, tb.tq1[i])) j = i + 1;
+  return q * (M / 4) + j;
+}
+
+constexpr int WARPS = 8;
+constexpr int MAX_CODE_WORDS = 16;  // 64 bytes of codes per vector
+
+template <int D>
+__global__ void __launch_bounds__(WARPS * 32) polar_encode_kernel(const float* __restrict__ x,
+                                                                  long long N, int b1, int b2,
+                                                                  int code_bytes,
+                                                                  uint8_t* __restrict__ codes,
+                                                                  uint16_t* __restrict__ radius,
+                                                                  PolarTables tb) {
+  constexpr int PER = D / 32;     // coordinates per lane
+  constexpr int PAIRS = PER / 2;  // level-1 pairs per lane
+  constexpr int NL = log2i(D) - 1;
+  __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = 1 << b1, L = 1 << b2;
+  for (long long n = static_cast<long long>(blockIdx.x) * WARPS + warp; n < N;
+       n += static_cast<long long>(gridDim.x) * WARPS) {
+    if (lane < MAX_CODE_WORDS) words[warp][lane] = 0u;
+    __syncwarp();
+    float v[PER];
+    if constexpr (PER == 4) {
+      const float4 t = reinterpret_cast<const float4*>(x + n * D)[lane];
+      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else {
+      const float2 t = reinterpret_cast<const float2*>(x + n * D)[lane];
+      v[0] = t.x; v[1] = t.y;
+    }
+    // level 1: the lane's pairs
+    float r[PAIRS];
+#pragma unroll
+    for (int p = 0; p < PAIRS; ++p) {
+      const int i = lane * PAIRS + p;
+      or_bits(words[warp], b1 * i, b1, static_cast<uint32_t>(level1_bin(v[2 * p], v[2 * p + 1], M, tb)));
+      r[p] = tree_radius(v[2 * p], v[2 * p + 1]);
+    }
+    // levels >= 2: node i of a level pairs the radii of nodes 2i, 2i + 1 below
+    int base = b1 * (D / 2);
+    int nodes = D / 2;
+    float rr = r[0];  // the radius of the node this lane holds after in-lane levels
+    int held = lane * PAIRS;  // index (at the current level) of the node held in rr
+    int lvl = 0;
+    if constexpr (PAIRS == 2) {
+      // level 2 pairs the lane's own two radii
+      nodes /= 2;
+      const float re = r[0], ro = r[1];
+      int j = 0;
+      if (ro > 0.0f)
+        for (int s = 0; s < L - 1; ++s)
+          if (ro >= __fmul_rn(re, tb.T[0][s])) j = s + 1;
+      or_bits(words[warp], base + b2 * lane, b2, static_cast<uint32_t>(j));
+      rr = tree_radius(re, ro);
+      held = lane;
+      base += b2 * nodes;
+      lvl = 1;
+    }
+    // remaining levels across lanes: at stride st the node held by lane l
+    // (l a multiple of 2 st) pairs with the one held by lane l + st
+    for (int st = 1; lvl < NL; st *= 2, ++lvl) {
+      nodes /= 2;
+      const float ro = __shfl_down_sync(0xffffffffu, rr, st);
+      const bool owner = (lane % (2 * st)) == 0;
+      if (owner) {
+        const float re = rr;
+        int j = 0;
+        if (ro > 0.0f)
+          for (int s = 0; s < L - 1; ++s)
+            if (ro >= __fmul_rn(re, tb.T[lvl][s])) j = s + 1;
+        const int node = held / 2;
+        or_bits(words[warp], base + b2 * node, b2, static_cast<uint32_t>(j));
+        rr = tree_radius(re, ro);
+        held = node;
+      }
+      base += b2 * nodes;
+    }
+    __syncwarp();
+    uint8_t* dst = codes + n * code_bytes;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(words[warp]);
+    for (int i = lane; i < code_bytes; i += 32) dst[i] = src[i];
+    if (lane == 0) radius[n] = __half_as_ushort(__float2half_rn(rr));
+    __syncwarp();
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(WARPS * 32) polar_decode_kernel(const uint8_t* __restrict__ codes,
+                                                                  const uint16_t* __restrict__ radius,
+                                                                  long long N, int b1, int b2,
+                                                                  int code_bytes,
+                                                                  float* __restrict__ xhat,
+                                                                  PolarTables tb) {
+  constexpr int PER = D / 32;
+  constexpr int PAIRS = PER / 2;
+  constexpr int NL = log2i(D) - 1;
+  __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (long long n = static_cast<long long>(blockIdx.x) * WARPS + warp; n < N;
+       n += static_cast<long long>(gridDim.x) * WARPS) {
+    if (lane < MAX_CODE_WORDS) words[warp][lane] = 0u;
+    __syncwarp();
+    uint8_t* wb = reinterpret_cast<uint8_t*>(words[warp]);
+    for (int i = lane; i < code_bytes; i += 32) wb[i] = codes[n * code_bytes + i];
+    __syncwarp();
+    // section offsets of the levels >= 2
+    int off[NL];
+    {
+      int base = b1 * (D / 2), cnt = D / 2;
+#pragma unroll
+      for (int l = 0; l < NL; ++l) {
+        cnt /= 2;
+        off[l] = base;
+        base += b2 * cnt;
+      }
+    }
+    const float R = __half2float(__ushort_as_half(radius[n]));
+    float out[PER];
+#pragma unroll
+    for (int p = 0; p < PAIRS; ++p) {
+      const int i = lane * PAIRS + p;  // level-1 pair index
+      float r = R;
+      // walk from the top level down to the pair: at level l (0 = level 2)
+      // the pair lies under node i >> (l + 1), in child (i >> l) & 1
+#pragma unroll
+      for (int l = NL - 1; l >= 0; --l) {
+        const int node = i >> (l + 1), child = (i >> l) & 1;
+        const int j = static_cast<int>(read_bits(words[warp], off[l] + b2 * node, b2));
+        r = __fmul_rn(r, child ? tb.sinl[l][j] : tb.cosl[l][j]);
+      }
+      const int k = static_cast<int>(read_bits(words[warp], b1 * i, b1));
+      out[2 * p] = __fmul_rn(r, tb.cos1[k]);
+      out[2 * p + 1] = __fmul_rn(r, tb.sin1[k]);
+    }
+    if constexpr (PER == 4)
+      reinterpret_cast<float4*>(xhat + n * D)[lane] = make_float4(out[0], out[1], out[2], out[3]);
+    else
+      reinterpret_cast<float2*>(xhat + n * D)[lane] = make_float2(out[0], out[1]);
+    __syncwarp();
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(WARPS * 32) mse_encode_kernel(const float* __restrict__ x,
+                                                                long long N, int bits,
+                                                                int code_bytes,
+                                                                uint8_t* __restrict__ codes,
+                                                                uint16_t* __restrict__ norms,
+                                                                MseTables tb) {
+  constexpr int PER = D / 32;
+  __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int L = 1 << (bits - 1);
+  for (long long n = static_cast<long long>(blockIdx.x) * WARPS + warp; n < N;
+       n += static_cast<long long>(gridDim.x) * WARPS) {
+    if (lane < MAX_CODE_WORDS) words[warp][lane] = 0u;
+    __syncwarp();
+    float v[PER];
+    if constexpr (PER == 4) {
+      const float4 t = reinterpret_cast<const float4*>(x + n * D)[lane];
+      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else {
+      const float2 t = reinterpret_cast<const float2*>(x + n * D)[lane];
+      v[0] = t.x; v[1] = t.y;
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) ss = fmaf(v[e], v[e], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const __half nh = __float2half_rn(sqrtf(ss));
+    const float nf = __half2float(nh);
+    const bool degenerate = !(nf > 0.0f) || isinf(nf);  // zero or overflowing norm: all codes 0
+#pragma unroll
+    for (int e = 0; e < PER && !degenerate; ++e) {
+      const float a = fabsf(v[e]);
+      int k = 0;
+      for (int s = 0; s < L - 1; ++s)
+        if (a >= __fmul_rn(nf, tb.t[s])) k = s + 1;
+      const uint32_t sgn = (v[e] < 0.0f) ? 1u : 0u;
+      const uint32_t code = (sgn << (bits - 1)) | static_cast<uint32_t>(k);
+      or_bits(words[warp], bits * (lane * PER + e), bits, code);
+    }
+    __syncwarp();
+    uint8_t* dst = codes + n * code_bytes;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(words[warp]);
+    for (int i = lane; i < code_bytes; i += 32) dst[i] = src[i];
+    if (lane == 0) norms[n] = __half_as_ushort(nh);
+    __syncwarp();
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(WARPS * 32) mse_decode_kernel(const uint8_t* __restrict__ codes,
+                                                                const uint16_t* __restrict__ norms,
+                                                                long long N, int bits,
+                                                                int code_bytes,
+                                                                float* __restrict__ xhat,
+                                                                MseTables tb) {
+  constexpr int PER = D / 32;
+  __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (long long n = static_cast<long long>(blockIdx.x) * WARPS + warp; n < N;
+       n += static_cast<long long>(gridDim.x) * WARPS) {
+    if (lane < MAX_CODE_WORDS) words[warp][lane] = 0u;
+    __syncwarp();
+    uint8_t* wb = reinterpret_cast<uint8_t*>(words[warp]);
+    for (int i = lane; i < code_bytes; i += 32) wb[i] = codes[n * code_bytes + i];
+    __syncwarp();
+    const float nf = __half2float(__ushort_as_half(norms[n]));
+    float out[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const uint32_t code = read_bits(words[warp], bits * (lane * PER + e), bits);
+      const float c = tb.c[code & ((1u << (bits - 1)) - 1u)];
+      out[e] = __fmul_rn(nf, (code >> (bits - 1)) ? -c : c);
+    }
+    if constexpr (PER == 4)
+      reinterpret_cast<float4*>(xhat + n * D)[lane] = make_float4(out[0], out[1], out[2], out[3]);
+    else
+      reinterpret_cast<float2*>(xhat + n * D)[lane] = make_float2(out[0], out[1]);
+    __syncwarp();
+  }
+}
+
+// host tables, computed once per (kind, d, b1, b2) and kept for the process
+std::mutex g_mu;
+std::map<std::tuple<int, int, int>, PolarTables> g_polar;
+std::map<std::pair<int, int>, MseTables> g_mse;
+
+PolarTables polar_tables(int d, int b1, int b2) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  const auto key = std::make_tuple(d, b1, b2);
+  auto it = g_polar.find(key);
+  if (it != g_polar.end()) return it->second;
+  PolarTables tb{};
+  const int M = 1 << b1, L = 1 << b2;
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int i = 0; i < M / 4 - 1; ++i) tb.tq1[i] = static_cast<float>(std::tan(two_pi * (i + 1) / M));
+  for (int j = 0; j < M; ++j) {
+    tb.cos1[j] = static_cast<float>(std::cos(two_pi * (j + 0.5) / M));
+    tb.sin1[j] = static_cast<float>(std::sin(two_pi * (j + 0.5) / M));
+  }
+  const int nl = log2i(d) - 1;
+  for (int l = 0; l < nl; ++l) {
+    std::vector<double> c, t;
+    angle_lloyd_max(1 << (l + 1), b2, c, t);
+    for (int s = 0; s < L - 1; ++s) tb.T[l][s] = static_cast<float>(std::tan(t[s]));
+    for (int j = 0; j < L; ++j) {
+      tb.cosl[l][j] = static_cast<float>(std::cos(c[j]));
+      tb.sinl[l][j] = static_cast<float>(std::sin(c[j]));
+    }
+  }
+  g_polar[key] = tb;
+  return tb;
+}
+
+MseTables mse_tables(int d, int bits) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  const auto key = std::make_pair(d, bits);
+  auto it = g_mse.find(key);
+  if (it != g_mse.end()) return it->second;
+  MseTables tb{};
+  std::vector<double> c, t;
+  sphere_lloyd_max(d, bits, c, t);
+  for (size_t i = 0; i < c.size(); ++i) tb.c[i] = static_cast<float>(c[i]);
+  for (size_t i = 0; i < t.size(); ++i) tb.t[i] = static_cast<float>(t[i]);
+  g_mse[key] = tb;
+  return tb;
+}
+
+}  // namespace s1
+
+size_t stage1_code_bytes(int d, int kind, int b1, int b2) {
+  if (d != 64 && d != 128) return 0;
+  if (kind == TQ_STAGE1_MSE) {
+    if (b1 < 2 || b1 > 4) return 0;
+    return (static_cast<size_t>(b1) * d + 7) / 8;
+  }
+  if (kind == TQ_STAGE1_POLAR) {
+    if (b1 < 2 || b1 > 5 || b2 < 1 || b2 > 3) return 0;
+    return (static_cast<size_t>(b1) * (d / 2) + static_cast<size_t>(b2) * (d / 2 - 1) + 7) / 8;
+  }
+  return 0;
+}
+
+int launch_stage1(const tq_ctx* ctx, int kind, int b1, int b2, bool encode, const float* x,
+                  const uint8_t* codes_in, uint8_t* codes_out, const uint16_t* norms_in,
+                  uint16_t* norms_out, float* xhat, long long N, void* stream) {
+  const int d = ctx->cfg.head_dim;
+  const int cb = static_cast<int>(stage1_code_bytes(d, kind, b1, b2));
+  if (cb == 0) return TQ_ERR_UNSUPPORTED;
+  if (N == 0) return TQ_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long blocks_needed = (N + s1::WARPS - 1) / s1::WARPS;
+  const int grid = static_cast<int>(blocks_needed < 16LL * ctx->num_sms ? blocks_needed : 16LL * ctx->num_sms);
+  const int threads = s1::WARPS * 32;
+  if (kind == TQ_STAGE1_POLAR) {
+    const s1::PolarTables tb = s1::polar_tables(d, b1, b2);
+    if (encode) {
+      if (d == 128) s1::polar_encode_kernel<128><<<grid, threads, 0, st>>>(x, N, b1, b2, cb, codes_out, norms_out, tb);
+      else s1::polar_encode_kernel<64><<<grid, threads, 0, st>>>(x, N, b1, b2, cb, codes_out, norms_out, tb);
+    } else {
+      if (d == 128) s1::polar_decode_kernel<128><<<grid, threads, 0, st>>>(codes_in, norms_in, N, b1, b2, cb, xhat, tb);
+      else s1::polar_decode_kernel<64><<<grid, threads, 0, st>>>(codes_in, norms_in, N, b1, b2, cb, xhat, tb);
+    }
+  } else {
+    const s1::MseTables tb = s1::mse_tables(d, b1);
+    if (encode) {
+      if (d == 128) s1::mse_encode_kernel<128><<<grid, threads, 0, st>>>(x, N, b1, cb, codes_out, norms_out, tb);
+      else s1::mse_encode_kernel<64><<<grid, threads, 0, st>>>(x, N, b1, cb, codes_out, norms_out, tb);
+    } else {
+      if (d == 128) s1::mse_decode_kernel<128><<<grid, threads, 0, st>>>(codes_in, norms_in, N, b1, cb, xhat, tb);
+      else s1::mse_decode_kernel<64><<<grid, threads, 0, st>>>(codes_in, norms_in, N, b1, cb, xhat, tb);
+    }
+  }
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+}  // namespace tq

@@ -324,6 +324,47 @@ TQ_API tq_status tq_score_topk(const tq_ctx* ctx, const float* queries, int Q, c
                         int64_t N, int k, int32_t* out_ids, float* out_scores, void* workspace,
                         size_t ws_bytes, void* stream);
 
+/*
+ * Stage-1 quantiser variants on rotated vectors, for comparing distortion
+ * ("Funktionsweise von TurboQuant": a standard per-coordinate quantiser after
+ * the rotation; "PolarQuant: Ein neuer Winkel auf Kompression": coordinate
+ * pairs to polar form, radii paired again recursively until one radius and a
+ * set of angles remain, angles quantised on fixed grids).  Neither variant
+ * carries the QJL sketch.
+ *  TQ_STAGE1_MSE    bits1 = b in 2..4 (bits2 unused): per coordinate the
+ *                   sign and a (b-1)-bit Lloyd-Max magnitude index of
+ *                   x_rot / n (levels of one coordinate of a uniform point on
+ *                   the sphere, as the key and value codebooks), decided as
+ *                   |x_rot,j| >= fp32(n * t_k); n = fp16(|x_rot|).  Code of
+ *                   coordinate j = sign << (b-1) | index, in bits
+ *                   [b j, b j + b) of a little-endian bit stream.
+ *  TQ_STAGE1_POLAR  bits1 = b1 in 2..5, bits2 = b2 in 1..3: level 1 pairs
+ *                   coordinates (2i, 2i+1), angle in [0, 2 pi) on 2^b1 equal
+ *                   bins (reconstructed at the bin centre); level l >= 2 pairs
+ *                   the radii of blocks of k = 2^(l-1) coordinates, angle
+ *                   atan(r_o / r_e) in [0, pi/2] with the 2^b2-level Lloyd-Max
+ *                   codebook of its density, proportional to sin^(k-1)(2 phi);
+ *                   the final radius is stored as fp16 in norms.  Radii are
+ *                   sqrtf(fmaf(u, u, v * v)) in fp32; a level-1 pair is turned
+ *                   into the first quadrant by exact swaps and negations and
+ *                   its bin counts the boundaries with v >= u * fp32(tan); a
+ *                   higher level counts r_o >= r_e * fp32(tan(boundary)) when
+ *                   r_o > 0; a zero pair has angle 0.  Codes: level 1 (b1 bits
+ *                   per pair, pair order), then level 2, 3, ... (b2 bits per
+ *                   node, node order), one little-endian bit stream.
+ *  x_rot   device fp32 [N, d] rotated vectors, 16-byte aligned.
+ *  codes   device uint8 [N, tq_stage1_code_bytes(...)]; norms device fp16 [N].
+ *  x_hat   device fp32 [N, d] reconstruction in the rotated domain.
+ * Unsupported bit counts give TQ_ERR_UNSUPPORTED (and a code size of 0).
+ */
+typedef enum { TQ_STAGE1_MSE = 0, TQ_STAGE1_POLAR = 1 } tq_stage1_kind;
+TQ_API size_t tq_stage1_code_bytes(const tq_ctx* ctx, int kind, int bits1, int bits2);
+TQ_API tq_status tq_stage1_encode(const tq_ctx* ctx, int kind, int bits1, int bits2,
+                                  const float* x_rot, int64_t N, uint8_t* codes,
+                                  uint16_t* norms, void* stream);
+TQ_API tq_status tq_stage1_decode(const tq_ctx* ctx, int kind, int bits1, int bits2,
+                                  const uint8_t* codes, const uint16_t* norms, int64_t N,
+                                  float* x_hat, void* stream);
 /* Profiling hook: when ev_start / ev_stop (cudaEvent_t, passed as void*) are
  * set, the next calls of tq_decode_attention, tq_compress_append and
  * tq_score_topk record ev_start on their stream right before the launch of
