@@ -84,6 +84,12 @@ def lib():
         L.tq_stage1_decode.argtypes = [vp, C.c_int, C.c_int, C.c_int, u8p, vp, C.c_int64, f32p,
                                        vp]
         L.tq_stage1_decode.restype = C.c_int
+        L.tq_tensor_cache_workspace_bytes.argtypes = [vp, C.c_int, C.c_int, C.c_int, C.c_int]
+        L.tq_tensor_cache_workspace_bytes.restype = C.c_size_t
+        L.tq_tensor_cache_step.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float,
+                                           vp, vp, vp, vp, C.c_int, i32p, i32p, f32p, f32p, f32p,
+                                           f32p, f32p, vp, C.c_size_t, vp]
+        L.tq_tensor_cache_step.restype = C.c_int
         L.tq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int,
                                                   C.c_float, vp, vp, C.c_int, i32p, u8p, C.c_int64,
                                                   i32p, C.c_int, i32p, f32p, vp]
@@ -264,6 +270,26 @@ def tq_monarch_step(ctx, q, k_new, v_new, k_hot, v_hot, hot_start, hot_len, page
         float(threshold), int(window), int(evict_block), _ptr(cold_used), _ptr(out),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
         "tq_monarch_step")
+
+
+def tq_tensor_cache_workspace_bytes(ctx, B, Hq, Hkv, W):
+    return int(lib().tq_tensor_cache_workspace_bytes(ctx, B, Hq, Hkv, W))
+
+
+def tq_tensor_cache_step(ctx, q, k_new, v_new, k_ring, v_ring, ring_start, ring_len, A, lam, eta,
+                         gate, out, workspace, Hkv, scale=0.0, stream=None):
+    """One Tensor Cache step: the token enters the fp16 ring (evicting the
+    oldest into A when full), then y = softmax attention over the ring +
+    sigmoid(gate) * (q A).  k_ring, v_ring [B, Hkv, W, d]; A fp32 [B, Hkv, d, d];
+    lam, eta fp32 [Hkv]; gate fp32 [Hq]."""
+    _require_cuda(q, k_new, v_new, k_ring, v_ring, ring_start, ring_len, A, lam, eta, gate, out,
+                  workspace)
+    B, Hq, _ = q.shape
+    _check(lib().tq_tensor_cache_step(
+        ctx, _ptr(q), _dtype_code(q), B, Hq, Hkv, float(scale), _ptr(k_new), _ptr(v_new),
+        _ptr(k_ring), _ptr(v_ring), k_ring.shape[2], _ptr(ring_start), _ptr(ring_len), _ptr(A),
+        _ptr(lam), _ptr(eta), _ptr(gate), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "tq_tensor_cache_step")
 
 
 TQ_STAGE1_MSE, TQ_STAGE1_POLAR = 0, 1

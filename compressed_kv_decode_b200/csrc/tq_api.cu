@@ -309,6 +309,34 @@ tq_status tq_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, in
       cold_used, out, workspace, ws_bytes, stream));
 }
 
+size_t tq_tensor_cache_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int W) {
+  if (!ctx || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || W <= 0) return 0;
+  return tq::tensor_cache_workspace_bytes(ctx, B, Hq, Hkv, W);
+}
+
+tq_status tq_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                               int Hkv, float scale, const void* k_new, const void* v_new,
+                               void* k_ring, void* v_ring, int W, int32_t* ring_start,
+                               int32_t* ring_len, float* A, const float* lambda,
+                               const float* eta, const float* gate, float* out,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  if (!ctx || !q || !k_new || !v_new || !k_ring || !v_ring || !ring_start || !ring_len || !A ||
+      !lambda || !eta || !gate || !out || !workspace)
+    return TQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || W <= 0) return TQ_ERR_INVALID_ARG;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_ERR_UNSUPPORTED;
+  if (!tq::aligned(k_ring, 16) || !tq::aligned(v_ring, 16) || !tq::aligned(workspace, 256))
+    return TQ_ERR_INVALID_ARG;
+  const size_t need = tq::tensor_cache_workspace_bytes(ctx, B, Hq, Hkv, W);
+  if (need == 0 || ws_bytes < need) return TQ_ERR_INVALID_ARG;
+  return static_cast<tq_status>(tq::launch_tensor_cache_step(
+      ctx, q, q_dtype, B, Hq, Hkv, scale, k_new, v_new, k_ring, v_ring, W, ring_start, ring_len,
+      A, lambda, eta, gate, out, workspace, ws_bytes, stream));
+}
+
 size_t tq_stage1_code_bytes(const tq_ctx* ctx, int kind, int bits1, int bits2) {
   if (!ctx) return 0;
   return tq::stage1_code_bytes(ctx->cfg.head_dim, kind, bits1, bits2);
@@ -317,7 +345,7 @@ size_t tq_stage1_code_bytes(const tq_ctx* ctx, int kind, int bits1, int bits2) {
 tq_status tq_stage1_encode(const tq_ctx* ctx, int kind, int bits1, int bits2, const float* x_rot,
                            int64_t N, uint8_t* codes, uint16_t* norms, void* stream) {
   if (!ctx || N < 0 || (N > 0 && (!x_rot || !codes || !norms))) return TQ_ERR_INVALID_ARG;
-  if (N > 0 && !tq::aligned(x_rot, 16)) return TQ_ERR_INVALID_ARG;
+  if (N > 0 && (!tq::aligned(x_rot, 16) || !tq::aligned(codes, 4))) return TQ_ERR_INVALID_ARG;
   if (tq::stage1_code_bytes(ctx->cfg.head_dim, kind, bits1, bits2) == 0) return TQ_ERR_UNSUPPORTED;
   return static_cast<tq_status>(tq::launch_stage1(ctx, kind, bits1, bits2, true, x_rot, nullptr,
                                                   codes, nullptr, norms, nullptr, N, stream));
@@ -326,7 +354,7 @@ tq_status tq_stage1_encode(const tq_ctx* ctx, int kind, int bits1, int bits2, co
 tq_status tq_stage1_decode(const tq_ctx* ctx, int kind, int bits1, int bits2, const uint8_t* codes,
                            const uint16_t* norms, int64_t N, float* x_hat, void* stream) {
   if (!ctx || N < 0 || (N > 0 && (!x_hat || !codes || !norms))) return TQ_ERR_INVALID_ARG;
-  if (N > 0 && !tq::aligned(x_hat, 16)) return TQ_ERR_INVALID_ARG;
+  if (N > 0 && (!tq::aligned(x_hat, 16) || !tq::aligned(codes, 4))) return TQ_ERR_INVALID_ARG;
   if (tq::stage1_code_bytes(ctx->cfg.head_dim, kind, bits1, bits2) == 0) return TQ_ERR_UNSUPPORTED;
   return static_cast<tq_status>(tq::launch_stage1(ctx, kind, bits1, bits2, false, nullptr, codes,
                                                   nullptr, norms, nullptr, x_hat, N, stream));

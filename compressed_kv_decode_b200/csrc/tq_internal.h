@@ -107,6 +107,13 @@ int launch_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int 
                         int max_pages, int32_t* cold_len, float threshold, int window,
                         int evict_block, int32_t* cold_used, float* out, void* ws,
                         size_t ws_bytes, void* stream);
+size_t tensor_cache_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int W);
+int launch_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                             int Hkv, float scale, const void* k_new, const void* v_new,
+                             void* k_ring, void* v_ring, int W, int32_t* ring_start,
+                             int32_t* ring_len, float* A, const float* lambda, const float* eta,
+                             const float* gate, float* out, void* ws, size_t ws_bytes,
+                             void* stream);
 size_t stage1_code_bytes(int d, int kind, int b1, int b2);
 int launch_stage1(const tq_ctx* ctx, int kind, int b1, int b2, bool encode, const float* x,
                   const uint8_t* codes_in, uint8_t* codes_out, const uint16_t* norms_in,

@@ -15,7 +15,9 @@
 //         bits per pair), then level 2, 3, ... (b2 bits per node).
 //
 // One warp per vector, D/32 coordinates per lane (coalesced 8- or 16-byte
-// loads).  Every decision is an fp32 comparison whose operands are formed the
+// loads); a record's codes are a whole number of 32-bit words, assembled
+// across lanes with shuffles (level-1 and MSE codes) or shared-memory ORs
+// (the polar levels >= 2) and moved as words.  Every decision is an fp32 comparison whose operands are formed the
 // same way in the CPU oracle: radii sqrtf(fmaf(u, u, v * v)), level-1 bins by
 // exact turns into the first quadrant and v >= u * tan(boundary), higher
 // levels by r_o >= r_e * tan(boundary), MSE codes by |x_j| >= fp32(n t_k).
@@ -65,6 +67,23 @@ __device__ __forceinline__ uint32_t read_bits(const uint32_t* words, int pos, in
   return static_cast<uint32_t>(x >> o) & ((1u << nbits) - 1u);
 }
 
+// Lane l holds v (bpl bits) destined for bits [bpl l, bpl l + bpl) of a
+// stream of bpl words; returns word `lane` of it (lanes >= bpl get 0).  Each
+// word gathers the few lanes that overlap it with shuffles.
+__device__ __forceinline__ uint32_t assemble_words(uint32_t v, int bpl, int lane) {
+  const int lo_bit = 32 * lane;
+  const int l0 = lo_bit / bpl;
+  const int K = (32 + bpl - 1) / bpl + 1;  // warp-uniform
+  uint32_t word = 0u;
+  for (int k = 0; k < K; ++k) {
+    const int src = l0 + k;
+    const uint32_t vs = __shfl_sync(0xffffffffu, v, src < 32 ? src : 31);
+    const int sh = bpl * src - lo_bit;
+    if (lane < bpl && src < 32 && sh < 32) word |= sh >= 0 ? (vs << sh) : (vs >> (-sh));
+  }
+  return word;
+}
+
 __device__ __forceinline__ float tree_radius(float u, float v) {
   return __fsqrt_rn(__fmaf_rn(u, u, __fmul_rn(v, v)));
 }
@@ -84,7 +103,25 @@ __device__ __forceinline__ int level1_bin(float a, float b, int M, const PolarTa
 }
 
 constexpr int WARPS = 8;
+constexpr int VPW = 4;              // vectors per warp and iteration, all loads issued first
 constexpr int MAX_CODE_WORDS = 16;  // 64 bytes of codes per vector
+
+template <int PER>
+__device__ __forceinline__ void load_row(const float* x, long long n, long long N, int lane,
+                                         float (&v)[PER]) {
+  if (n >= N) {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) v[e] = 0.0f;
+    return;
+  }
+  if constexpr (PER == 4) {
+    const float4 t = reinterpret_cast<const float4*>(x + n * (32 * PER))[lane];
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else {
+    const float2 t = reinterpret_cast<const float2*>(x + n * (32 * PER))[lane];
+    v[0] = t.x; v[1] = t.y;
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(WARPS * 32) polar_encode_kernel(const float* __restrict__ x,
@@ -159,9 +196,8 @@ __global__ void __launch_bounds__(WARPS * 32) polar_encode_kernel(const float* _
       base += b2 * nodes;
     }
     __syncwarp();
-    uint8_t* dst = codes + n * code_bytes;
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(words[warp]);
-    for (int i = lane; i < code_bytes; i += 32) dst[i] = src[i];
+    if (lane < code_bytes / 4)
+      reinterpret_cast<uint32_t*>(codes + n * code_bytes)[lane] = words[warp][lane];
     if (lane == 0) radius[n] = __half_as_ushort(__float2half_rn(rr));
     __syncwarp();
   }
@@ -178,13 +214,29 @@ __global__ void __launch_bounds__(WARPS * 32) polar_decode_kernel(const uint8_t*
   constexpr int PAIRS = PER / 2;
   constexpr int NL = log2i(D) - 1;
   __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
+  // the tables are read with per-lane indices: from shared memory, not the
+  // kernel parameters (whose reads serialise over distinct addresses)
+  __shared__ PolarTables st;
+  for (int i = threadIdx.x; i < static_cast<int>(sizeof(PolarTables) / 4); i += blockDim.x)
+    reinterpret_cast<float*>(&st)[i] = reinterpret_cast<const float*>(&tb)[i];
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (long long n = static_cast<long long>(blockIdx.x) * WARPS + warp; n < N;
-       n += static_cast<long long>(gridDim.x) * WARPS) {
-    if (lane < MAX_CODE_WORDS) words[warp][lane] = 0u;
-    __syncwarp();
-    uint8_t* wb = reinterpret_cast<uint8_t*>(words[warp]);
-    for (int i = lane; i < code_bytes; i += 32) wb[i] = codes[n * code_bytes + i];
+  const int nw = code_bytes / 4;
+  for (long long n0 = (static_cast<long long>(blockIdx.x) * WARPS + warp) * VPW; n0 < N;
+       n0 += static_cast<long long>(gridDim.x) * WARPS * VPW) {
+  uint32_t cw[VPW];
+  float rad[VPW];
+#pragma unroll
+  for (int u = 0; u < VPW; ++u) {
+    const bool ok = n0 + u < N;
+    cw[u] = (ok && lane < nw) ? reinterpret_cast<const uint32_t*>(codes + (n0 + u) * code_bytes)[lane] : 0u;
+    rad[u] = ok ? __half2float(__ushort_as_half(radius[n0 + u])) : 0.0f;
+  }
+#pragma unroll
+  for (int u = 0; u < VPW; ++u) {
+    if (n0 + u >= N) break;
+    const long long n = n0 + u;
+    if (lane < MAX_CODE_WORDS) words[warp][lane] = lane < nw ? cw[u] : 0u;
     __syncwarp();
     // section offsets of the levels >= 2
     int off[NL];
@@ -197,7 +249,7 @@ __global__ void __launch_bounds__(WARPS * 32) polar_decode_kernel(const uint8_t*
         base += b2 * cnt;
       }
     }
-    const float R = __half2float(__ushort_as_half(radius[n]));
+    const float R = rad[u];
     float out[PER];
 #pragma unroll
     for (int p = 0; p < PAIRS; ++p) {
@@ -209,17 +261,18 @@ __global__ void __launch_bounds__(WARPS * 32) polar_decode_kernel(const uint8_t*
       for (int l = NL - 1; l >= 0; --l) {
         const int node = i >> (l + 1), child = (i >> l) & 1;
         const int j = static_cast<int>(read_bits(words[warp], off[l] + b2 * node, b2));
-        r = __fmul_rn(r, child ? tb.sinl[l][j] : tb.cosl[l][j]);
+        r = __fmul_rn(r, child ? st.sinl[l][j] : st.cosl[l][j]);
       }
       const int k = static_cast<int>(read_bits(words[warp], b1 * i, b1));
-      out[2 * p] = __fmul_rn(r, tb.cos1[k]);
-      out[2 * p + 1] = __fmul_rn(r, tb.sin1[k]);
+      out[2 * p] = __fmul_rn(r, st.cos1[k]);
+      out[2 * p + 1] = __fmul_rn(r, st.sin1[k]);
     }
     if constexpr (PER == 4)
       reinterpret_cast<float4*>(xhat + n * D)[lane] = make_float4(out[0], out[1], out[2], out[3]);
     else
       reinterpret_cast<float2*>(xhat + n * D)[lane] = make_float2(out[0], out[1]);
     __syncwarp();
+  }
   }
 }
 
@@ -231,21 +284,20 @@ __global__ void __launch_bounds__(WARPS * 32) mse_encode_kernel(const float* __r
                                                                 uint16_t* __restrict__ norms,
                                                                 MseTables tb) {
   constexpr int PER = D / 32;
-  __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = 1 << (bits - 1);
-  for (long long n = static_cast<long long>(blockIdx.x) * WARPS + warp; n < N;
-       n += static_cast<long long>(gridDim.x) * WARPS) {
-    if (lane < MAX_CODE_WORDS) words[warp][lane] = 0u;
-    __syncwarp();
+  for (long long n0 = (static_cast<long long>(blockIdx.x) * WARPS + warp) * VPW; n0 < N;
+       n0 += static_cast<long long>(gridDim.x) * WARPS * VPW) {
+  float vin[VPW][PER];
+#pragma unroll
+  for (int u = 0; u < VPW; ++u) load_row<PER>(x, n0 + u, N, lane, vin[u]);
+#pragma unroll
+  for (int u = 0; u < VPW; ++u) {
+    const long long n = n0 + u;
+    if (n >= N) break;
     float v[PER];
-    if constexpr (PER == 4) {
-      const float4 t = reinterpret_cast<const float4*>(x + n * D)[lane];
-      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-    } else {
-      const float2 t = reinterpret_cast<const float2*>(x + n * D)[lane];
-      v[0] = t.x; v[1] = t.y;
-    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) v[e] = vin[u][e];
     float ss = 0.0f;
 #pragma unroll
     for (int e = 0; e < PER; ++e) ss = fmaf(v[e], v[e], ss);
@@ -254,22 +306,22 @@ __global__ void __launch_bounds__(WARPS * 32) mse_encode_kernel(const float* __r
     const __half nh = __float2half_rn(sqrtf(ss));
     const float nf = __half2float(nh);
     const bool degenerate = !(nf > 0.0f) || isinf(nf);  // zero or overflowing norm: all codes 0
+    uint32_t mine = 0u;  // the lane's PER codes, contiguous
 #pragma unroll
-    for (int e = 0; e < PER && !degenerate; ++e) {
+    for (int e = 0; e < PER; ++e) {
       const float a = fabsf(v[e]);
       int k = 0;
-      for (int s = 0; s < L - 1; ++s)
-        if (a >= __fmul_rn(nf, tb.t[s])) k = s + 1;
+#pragma unroll
+      for (int s = 0; s < 7; ++s)  // constant indices: the table stays in registers
+        if (s < L - 1 && a >= __fmul_rn(nf, tb.t[s])) k = s + 1;
       const uint32_t sgn = (v[e] < 0.0f) ? 1u : 0u;
-      const uint32_t code = (sgn << (bits - 1)) | static_cast<uint32_t>(k);
-      or_bits(words[warp], bits * (lane * PER + e), bits, code);
+      const uint32_t code = degenerate ? 0u : ((sgn << (bits - 1)) | static_cast<uint32_t>(k));
+      mine |= code << (bits * e);
     }
-    __syncwarp();
-    uint8_t* dst = codes + n * code_bytes;
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(words[warp]);
-    for (int i = lane; i < code_bytes; i += 32) dst[i] = src[i];
+    const uint32_t w = assemble_words(mine, PER * bits, lane);  // PER bits words = the record
+    if (lane < PER * bits) reinterpret_cast<uint32_t*>(codes + n * code_bytes)[lane] = w;
     if (lane == 0) norms[n] = __half_as_ushort(nh);
-    __syncwarp();
+  }
   }
 }
 
@@ -283,19 +335,33 @@ __global__ void __launch_bounds__(WARPS * 32) mse_decode_kernel(const uint8_t* _
   constexpr int PER = D / 32;
   __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (long long n = static_cast<long long>(blockIdx.x) * WARPS + warp; n < N;
-       n += static_cast<long long>(gridDim.x) * WARPS) {
-    if (lane < MAX_CODE_WORDS) words[warp][lane] = 0u;
+  const int nw = code_bytes / 4;
+  for (long long n0 = (static_cast<long long>(blockIdx.x) * WARPS + warp) * VPW; n0 < N;
+       n0 += static_cast<long long>(gridDim.x) * WARPS * VPW) {
+  uint32_t cw[VPW];
+  float nrm[VPW];
+#pragma unroll
+  for (int u = 0; u < VPW; ++u) {
+    const bool ok = n0 + u < N;
+    cw[u] = (ok && lane < nw) ? reinterpret_cast<const uint32_t*>(codes + (n0 + u) * code_bytes)[lane] : 0u;
+    nrm[u] = ok ? __half2float(__ushort_as_half(norms[n0 + u])) : 0.0f;
+  }
+#pragma unroll
+  for (int u = 0; u < VPW; ++u) {
+    if (n0 + u >= N) break;
+    const long long n = n0 + u;
+    if (lane < MAX_CODE_WORDS) words[warp][lane] = lane < nw ? cw[u] : 0u;
     __syncwarp();
-    uint8_t* wb = reinterpret_cast<uint8_t*>(words[warp]);
-    for (int i = lane; i < code_bytes; i += 32) wb[i] = codes[n * code_bytes + i];
-    __syncwarp();
-    const float nf = __half2float(__ushort_as_half(norms[n]));
+    const float nf = nrm[u];
     float out[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
       const uint32_t code = read_bits(words[warp], bits * (lane * PER + e), bits);
-      const float c = tb.c[code & ((1u << (bits - 1)) - 1u)];
+      const uint32_t mi = code & ((1u << (bits - 1)) - 1u);
+      float c = tb.c[0];
+#pragma unroll
+      for (int k = 1; k < 8; ++k)  // select with constant indices (no local copy of the table)
+        if (mi == static_cast<uint32_t>(k)) c = tb.c[k];
       out[e] = __fmul_rn(nf, (code >> (bits - 1)) ? -c : c);
     }
     if constexpr (PER == 4)
@@ -303,6 +369,7 @@ __global__ void __launch_bounds__(WARPS * 32) mse_decode_kernel(const uint8_t* _
     else
       reinterpret_cast<float2*>(xhat + n * D)[lane] = make_float2(out[0], out[1]);
     __syncwarp();
+  }
   }
 }
 
@@ -375,7 +442,7 @@ int launch_stage1(const tq_ctx* ctx, int kind, int b1, int b2, bool encode, cons
   if (cb == 0) return TQ_ERR_UNSUPPORTED;
   if (N == 0) return TQ_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long blocks_needed = (N + s1::WARPS - 1) / s1::WARPS;
+  const long long blocks_needed = (N + s1::WARPS * s1::VPW - 1) / (s1::WARPS * s1::VPW);
   const int grid = static_cast<int>(blocks_needed < 16LL * ctx->num_sms ? blocks_needed : 16LL * ctx->num_sms);
   const int threads = s1::WARPS * 32;
   if (kind == TQ_STAGE1_POLAR) {

@@ -1,0 +1,192 @@
+// One decode step of Tensor Cache's two-level state ("Tensor Cache:
+// Eviction-conditioned Associative Memory for Transformers", gist.science,
+// section "Methodik: Tensor Cache (TC)"): an fp16 ring of the last W tokens
+// read with exact softmax attention (L1), and a d x d outer-product matrix A
+// per kv head written only by the ring's evictions (L2),
+//   A <- lambda A + eta (k (x) v),   r = q A,   y = y_local + sigmoid(g) r.
+//
+// Launches, all on the caller's stream:
+//   update   one CTA per (sequence, kv head): the step's token enters the
+//            ring; when the ring is full the token it overwrites is first
+//            written into A; then r = q A (the updated A) for the group's
+//            query heads.  One pass over A: read, update, write, and the
+//            partial products of the read.  The new ring start and length go
+//            to the workspace (the caller's arrays are read by every head).
+//   decode   the split-K attention over the ring alone (prep, attention,
+//            combine), with the ring start and length of this step
+//   fuse     y += sigmoid(g) r; the new ring start and length written back
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "tq_device.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+namespace tcache {
+
+template <int D, int G>
+__global__ void __launch_bounds__(256) update_kernel(const void* q, int q_dtype, int Hq, int Hkv,
+                                                     const __half* __restrict__ k_new,
+                                                     const __half* __restrict__ v_new,
+                                                     __half* k_ring, __half* v_ring, int W,
+                                                     const int32_t* ring_start,
+                                                     const int32_t* ring_len, float* A,
+                                                     const float* lambda, const float* eta,
+                                                     float* r_out, int32_t* new_start,
+                                                     int32_t* new_len, int* err) {
+  constexpr int NR = 256 / D;  // row phases
+  const int bh = blockIdx.x, b = bh / Hkv, kvh = bh % Hkv;
+  const int tid = threadIdx.x, j = tid % D, rp = tid / D;
+  __shared__ float sk[D], sv[D];
+  __shared__ float sq[G][D];
+  __shared__ float part[NR][G][D];
+  const int len = ring_len[b], start = ring_start[b];
+  const bool ok = len >= 0 && len <= W && start >= 0 && start < W;
+  if (!ok) {
+    if (tid == 0) report(err, TQ_ERR_CAPACITY);
+    if (tid == 0 && kvh == 0) {
+      new_start[b] = 0;
+      new_len[b] = 0;
+    }
+    for (int i = tid; i < G * D; i += blockDim.x)
+      r_out[(static_cast<size_t>(b) * Hq + kvh * G + i / D) * D + i % D] = 0.0f;
+    return;
+  }
+  const bool evict = len == W;
+  int slot = evict ? start : start + len;
+  if (slot >= W) slot -= W;
+  const size_t row = (static_cast<size_t>(bh) * W + slot) * D;
+  if (tid < D) {
+    sk[tid] = evict ? __half2float(k_ring[row + tid]) : 0.0f;
+    sv[tid] = evict ? __half2float(v_ring[row + tid]) : 0.0f;
+  }
+  for (int i = tid; i < G * D; i += blockDim.x)
+    sq[i / D][i % D] = load_as_float(q, (static_cast<size_t>(b) * Hq + kvh * G) * D + i,
+                                     static_cast<tq_dtype>(q_dtype));
+  __syncthreads();  // the evicted row is read before the new token overwrites it
+  if (tid < D) {
+    k_ring[row + tid] = k_new[static_cast<size_t>(bh) * D + tid];
+    v_ring[row + tid] = v_new[static_cast<size_t>(bh) * D + tid];
+  }
+  if (tid == 0 && kvh == 0) {
+    new_start[b] = evict ? (start + 1 == W ? 0 : start + 1) : start;
+    new_len[b] = evict ? W : len + 1;
+  }
+  // A[i][j], i = key coordinate: this thread takes column j, rows rp, rp + NR, ...
+  float* Ab = A + static_cast<size_t>(bh) * D * D;
+  const float lam = lambda[kvh], et = eta[kvh];
+  const float evj = evict ? et * sv[j] : 0.0f;
+  float acc[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) acc[g] = 0.0f;
+#pragma unroll 4
+  for (int i = rp; i < D; i += NR) {
+    float a = Ab[static_cast<size_t>(i) * D + j];
+    if (evict) {
+      a = fmaf(lam, a, evj * sk[i]);
+      Ab[static_cast<size_t>(i) * D + j] = a;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = fmaf(sq[g][i], a, acc[g]);
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) part[rp][g][j] = acc[g];
+  __syncthreads();
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    const int g = i / D, jj = i % D;
+    float s = 0.0f;
+#pragma unroll
+    for (int k = 0; k < NR; ++k) s += part[k][g][jj];
+    r_out[(static_cast<size_t>(b) * Hq + kvh * G + g) * D + jj] = s;
+  }
+}
+
+__global__ void fuse_kernel(float* out, const float* r, const float* gate, int B, int Hq, int D,
+                            const int32_t* new_start, const int32_t* new_len, int32_t* ring_start,
+                            int32_t* ring_len) {
+  const long long n = static_cast<long long>(B) * Hq * D;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int hq = static_cast<int>((i / D) % Hq);
+    const float s = 1.0f / (1.0f + expf(-gate[hq]));
+    out[i] = fmaf(s, r[i], out[i]);
+  }
+  if (blockIdx.x == 0)
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+      ring_start[b] = new_start[b];
+      ring_len[b] = new_len[b];
+    }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace tcache
+
+size_t tensor_cache_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int W) {
+  const size_t dec = decode_workspace_bytes(ctx, B, Hq, Hkv, 0, W);
+  if (dec == 0) return 0;
+  return tcache::align256(dec) +
+         tcache::align256(sizeof(float) * static_cast<size_t>(B) * Hq * ctx->cfg.head_dim) +
+         2 * tcache::align256(sizeof(int32_t) * B);
+}
+
+int launch_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                             int Hkv, float scale, const void* k_new, const void* v_new,
+                             void* k_ring, void* v_ring, int W, int32_t* ring_start,
+                             int32_t* ring_len, float* A, const float* lambda, const float* eta,
+                             const float* gate, float* out, void* ws, size_t ws_bytes,
+                             void* stream) {
+  (void)ws_bytes;
+  const int d = ctx->cfg.head_dim;
+  const int G = Hq / Hkv;
+  const size_t dec = decode_workspace_bytes(ctx, B, Hq, Hkv, 0, W);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* r = reinterpret_cast<float*>(base + tcache::align256(dec));
+  int32_t* ns = reinterpret_cast<int32_t*>(
+      reinterpret_cast<uint8_t*>(r) + tcache::align256(sizeof(float) * static_cast<size_t>(B) * Hq * d));
+  int32_t* nl = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ns) +
+                                           tcache::align256(sizeof(int32_t) * B));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __half* kn = static_cast<const __half*>(k_new);
+  const __half* vn = static_cast<const __half*>(v_new);
+  __half* kr = static_cast<__half*>(k_ring);
+  __half* vr = static_cast<__half*>(v_ring);
+  const int qd = static_cast<int>(q_dtype);
+#define TQ_TC_LAUNCH(DD, GG)                                                                      \
+  tcache::update_kernel<DD, GG><<<B * Hkv, 256, 0, st>>>(q, qd, Hq, Hkv, kn, vn, kr, vr, W,       \
+                                                        ring_start, ring_len, A, lambda, eta, r,  \
+                                                        ns, nl, ctx->dev.err)
+  if (d == 128) {
+    switch (G) {
+      case 1: TQ_TC_LAUNCH(128, 1); break;
+      case 2: TQ_TC_LAUNCH(128, 2); break;
+      case 4: TQ_TC_LAUNCH(128, 4); break;
+      case 8: TQ_TC_LAUNCH(128, 8); break;
+      default: return TQ_ERR_UNSUPPORTED;
+    }
+  } else if (d == 64) {
+    switch (G) {
+      case 1: TQ_TC_LAUNCH(64, 1); break;
+      case 2: TQ_TC_LAUNCH(64, 2); break;
+      case 4: TQ_TC_LAUNCH(64, 4); break;
+      case 8: TQ_TC_LAUNCH(64, 8); break;
+      default: return TQ_ERR_UNSUPPORTED;
+    }
+  } else {
+    return TQ_ERR_UNSUPPORTED;
+  }
+#undef TQ_TC_LAUNCH
+  if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
+  const int rc = launch_decode(ctx, q, q_dtype, B, Hq, Hkv, scale, k_ring, v_ring, W, ns, nl,
+                               nullptr, 0, nullptr, 0, nullptr, nullptr, out, ws, dec, stream);
+  if (rc != TQ_OK) return rc;
+  const long long n = static_cast<long long>(B) * Hq * d;
+  const int blocks = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+  tcache::fuse_kernel<<<blocks, 256, 0, st>>>(out, r, gate, B, Hq, d, ns, nl, ring_start, ring_len);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+}  // namespace tq

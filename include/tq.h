@@ -324,6 +324,39 @@ TQ_API tq_status tq_score_topk(const tq_ctx* ctx, const float* queries, int Q, c
                         int64_t N, int k, int32_t* out_ids, float* out_scores, void* workspace,
                         size_t ws_bytes, void* stream);
 
+/* Workspace bytes tq_tensor_cache_step needs. */
+TQ_API size_t tq_tensor_cache_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int W);
+/*
+ * One decode step of Tensor Cache's two-level state ("Tensor Cache:
+ * Eviction-conditioned Associative Memory for Transformers", section
+ * "Methodik: Tensor Cache (TC)"):
+ *  L1  an fp16 ring of the last W tokens per (batch, kv head), attended with
+ *      exact softmax (scale as tq_decode_attention);
+ *  L2  a d x d fp32 matrix A per (batch, kv head), written only by the ring's
+ *      evictions: A <- lambda A + eta (k (x) v), i.e. A[i][j] += eta k_i v_j
+ *      after scaling by lambda;
+ *  read r = q A (r_j = sum_i q_i A[i][j], q unscaled) with the A of the query
+ *      head's kv head; output y = y_local + sigmoid(g) r.
+ * Order: the step's token (k_new, v_new: device fp16 [B, Hkv, d]) enters the
+ * ring; when the ring already holds W tokens, the token it overwrites (the
+ * oldest) is first written into A.  Then attention over the ring and the read
+ * of A, so every token is in exactly one level.
+ *  k_ring, v_ring  device fp16 [B, Hkv, W, d]; ring_start, ring_len device
+ *                  int32 [B] (logical token i at slot (start + i) mod W),
+ *                  updated on the device.
+ *  A               device fp32 [B, Hkv, d, d], updated in place.
+ *  lambda, eta     device fp32 [Hkv]; gate device fp32 [Hq] (g before the
+ *                  sigmoid).
+ *  out             device fp32 [B, Hq, d].
+ * A ring length outside [0, W] or start outside [0, W) is a device error
+ * (TQ_ERR_CAPACITY); that sequence's state restarts empty.
+ */
+TQ_API tq_status tq_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B,
+                                      int Hq, int Hkv, float scale, const void* k_new,
+                                      const void* v_new, void* k_ring, void* v_ring, int W,
+                                      int32_t* ring_start, int32_t* ring_len, float* A,
+                                      const float* lambda, const float* eta, const float* gate,
+                                      float* out, void* workspace, size_t ws_bytes, void* stream);
 /*
  * Stage-1 quantiser variants on rotated vectors, for comparing distortion
  * ("Funktionsweise von TurboQuant": a standard per-coordinate quantiser after
@@ -353,7 +386,8 @@ TQ_API tq_status tq_score_topk(const tq_ctx* ctx, const float* queries, int Q, c
  *                   per pair, pair order), then level 2, 3, ... (b2 bits per
  *                   node, node order), one little-endian bit stream.
  *  x_rot   device fp32 [N, d] rotated vectors, 16-byte aligned.
- *  codes   device uint8 [N, tq_stage1_code_bytes(...)]; norms device fp16 [N].
+ *  codes   device uint8 [N, tq_stage1_code_bytes(...)], 4-byte aligned (a
+ *          record is a whole number of 32-bit words); norms device fp16 [N].
  *  x_hat   device fp32 [N, d] reconstruction in the rotated domain.
  * Unsupported bit counts give TQ_ERR_UNSUPPORTED (and a code size of 0).
  */
