@@ -337,6 +337,43 @@ def measure_monarch(torch, tq, W, workload, evict_block, thresholds=(float("inf"
     return res
 
 
+def measure_tensor_cache(torch, tq, W, workload, steps=256):
+    """Tensor Cache steps on a decode workload's shapes: the fp16 ring holds
+    the workload's hot length W (full, so every step evicts one token per kv
+    head into A), no cold pages; each step replayed from a CUDA graph."""
+    cfg = W.DECODE[workload]
+    B, Hq, Hkv, d, Wr = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], cfg["hot"]
+    ctx = tq.Context(d, seed=0)
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(51)
+    k_ring = torch.randn((B, Hkv, Wr, d), generator=gen, device=dev).half()
+    v_ring = torch.randn((B, Hkv, Wr, d), generator=gen, device=dev).half()
+    A = torch.randn((B, Hkv, d, d), generator=gen, device=dev) * 0.01
+    lam = torch.full((Hkv,), 0.95, device=dev)
+    eta = torch.full((Hkv,), 0.1, device=dev)
+    gate = torch.zeros(Hq, device=dev)
+    q = torch.randn((B, Hq, d), generator=gen, device=dev).to(getattr(torch, cfg["q_dtype"]))
+    k_new = torch.randn((B, Hkv, d), generator=gen, device=dev).half()
+    v_new = torch.randn((B, Hkv, d), generator=gen, device=dev).half()
+    rs = torch.zeros(B, dtype=torch.int32, device=dev)
+    rl = torch.full((B,), Wr, dtype=torch.int32, device=dev)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.tq_tensor_cache_workspace_bytes(ctx.handle, B, Hq, Hkv, Wr),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        tq.tq_tensor_cache_step(ctx.handle, q, k_new, v_new, k_ring, v_ring, rs, rl, A, lam, eta,
+                                gate, out, ws, Hkv)
+    ms = graph_ms(torch, step, steps)
+    ctx.check()
+    # bytes per step: the ring once (fp16 K and V), A read and written, q, out
+    by = B * Hkv * (Wr * 4 * d + 8 * d * d) + B * Hq * d * 6
+    return {"workload": workload + " shapes, fp16 ring of %d + d x d fp32 memory" % Wr,
+            "us_per_step": ms * 1e3, "bytes_per_step": by,
+            "achieved_gbs": by / (ms / 1e3) / 1e9}
+
+
 def measure_stage1(torch, tq, N=1 << 20, reps=5):
     """Stage-1 variants on 2^20 rotated fp32 vectors (d = 128, N(0,1)):
     encode and decode kernel times (CUDA events, median of reps) with their
@@ -566,6 +603,9 @@ def run_ours(args, rank, world, local_rank):
         rows["gated_decode"] = measure_gated(torch, tq, st)
         rows["gated_decode"]["workload"] = WORKLOAD + " with Monarch's threshold gate"
         del st, graph
+        torch.cuda.empty_cache()
+        rows["tensor_cache_step"] = [measure_tensor_cache(torch, tq, W, "tinyllama"),
+                                     measure_tensor_cache(torch, tq, W, WORKLOAD)]
         torch.cuda.empty_cache()
         rows["monarch_step"] = [measure_monarch(torch, tq, W, "tinyllama", 128),
                                 measure_monarch(torch, tq, W, "tinyllama", 1),
