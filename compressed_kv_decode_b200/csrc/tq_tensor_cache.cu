@@ -75,16 +75,25 @@ __global__ void __launch_bounds__(256) update_kernel(const void* q, int q_dtype,
     new_start[b] = evict ? (start + 1 == W ? 0 : start + 1) : start;
     new_len[b] = evict ? W : len + 1;
   }
-  // A[i][j], i = key coordinate: this thread takes column j, rows rp, rp + NR, ...
+  // A[i][j], i = key coordinate: this thread takes column j, rows rp, rp + NR,
+  // ...; all of its D / NR values are loaded before any arithmetic (the
+  // kernel has one CTA per group, so memory parallelism comes from here)
+  constexpr int RPT = D / NR;  // rows per thread
   float* Ab = A + static_cast<size_t>(bh) * D * D;
+  float av[RPT];
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) av[m] = Ab[static_cast<size_t>(rp + NR * m) * D + j];
+  // a barrier keeps the compiler from sinking the loads past the stores below
+  __syncthreads();
   const float lam = lambda[kvh], et = eta[kvh];
   const float evj = evict ? et * sv[j] : 0.0f;
   float acc[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) acc[g] = 0.0f;
-#pragma unroll 4
-  for (int i = rp; i < D; i += NR) {
-    float a = Ab[static_cast<size_t>(i) * D + j];
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) {
+    const int i = rp + NR * m;
+    float a = av[m];
     if (evict) {
       a = fmaf(lam, a, evj * sk[i]);
       Ab[static_cast<size_t>(i) * D + j] = a;
