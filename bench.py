@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--batch", type=int, default=None,
                     help="sequences per GPU (default: the workload's 16); smaller values only "
                          "size profiler captures and are not the benchmark line")
+    ap.add_argument("--only", default=None,
+                    choices=["gated", "monarch", "tensor_cache", "stage1"],
+                    help="run one extra row alone and print it (sized for profiler captures; "
+                         "not the benchmark line)")
     return ap.parse_args()
 
 
@@ -646,9 +650,29 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_only(args):
+    """One extra row alone, for profiler captures of its kernels."""
+    import torch
+    import compressed_kv_decode_b200 as tq
+    from compressed_kv_decode_b200 import workloads as W
+    if args.only == "gated":
+        st = build_state(torch, tq, W, 0, args.batch)
+        res = measure_gated(torch, tq, st, reps=args.steps)
+    elif args.only == "monarch":
+        res = measure_monarch(torch, tq, W, "tinyllama", 128, steps=args.steps)
+    elif args.only == "tensor_cache":
+        res = measure_tensor_cache(torch, tq, W, WORKLOAD, steps=args.steps)
+    else:
+        res = measure_stage1(torch, tq, reps=max(1, args.steps))
+    print(json.dumps({"only": args.only, "row": res}), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local_rank = dist_env()
+    if args.only:
+        run_only(args)
+        return
     if world > 1:
         import torch
         import torch.distributed as dist

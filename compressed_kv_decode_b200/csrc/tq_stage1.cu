@@ -276,16 +276,15 @@ __global__ void __launch_bounds__(WARPS * 32) polar_decode_kernel(const uint8_t*
   }
 }
 
-template <int D>
+template <int D, int BITS>
 __global__ void __launch_bounds__(WARPS * 32) mse_encode_kernel(const float* __restrict__ x,
-                                                                long long N, int bits,
-                                                                int code_bytes,
+                                                                long long N, int code_bytes,
                                                                 uint8_t* __restrict__ codes,
                                                                 uint16_t* __restrict__ norms,
                                                                 MseTables tb) {
   constexpr int PER = D / 32;
+  constexpr int bits = BITS, L = 1 << (BITS - 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int L = 1 << (bits - 1);
   for (long long n0 = (static_cast<long long>(blockIdx.x) * WARPS + warp) * VPW; n0 < N;
        n0 += static_cast<long long>(gridDim.x) * WARPS * VPW) {
   float vin[VPW][PER];
@@ -312,8 +311,8 @@ __global__ void __launch_bounds__(WARPS * 32) mse_encode_kernel(const float* __r
       const float a = fabsf(v[e]);
       int k = 0;
 #pragma unroll
-      for (int s = 0; s < 7; ++s)  // constant indices: the table stays in registers
-        if (s < L - 1 && a >= __fmul_rn(nf, tb.t[s])) k = s + 1;
+      for (int s = 0; s < L - 1; ++s)
+        if (a >= __fmul_rn(nf, tb.t[s])) k = s + 1;
       const uint32_t sgn = (v[e] < 0.0f) ? 1u : 0u;
       const uint32_t code = degenerate ? 0u : ((sgn << (bits - 1)) | static_cast<uint32_t>(k));
       mine |= code << (bits * e);
@@ -325,17 +324,21 @@ __global__ void __launch_bounds__(WARPS * 32) mse_encode_kernel(const float* __r
   }
 }
 
-template <int D>
+template <int D, int BITS>
 __global__ void __launch_bounds__(WARPS * 32) mse_decode_kernel(const uint8_t* __restrict__ codes,
                                                                 const uint16_t* __restrict__ norms,
-                                                                long long N, int bits,
-                                                                int code_bytes,
+                                                                long long N, int code_bytes,
                                                                 float* __restrict__ xhat,
                                                                 MseTables tb) {
   constexpr int PER = D / 32;
-  __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
+  constexpr int BPL = PER * BITS;  // code bits per lane; the record is BPL words
+  constexpr uint32_t MMASK = (1u << (BITS - 1)) - 1u;
+  __shared__ float sc[8];  // levels, read with per-lane indices
+  if (threadIdx.x < 8) sc[threadIdx.x] = tb.c[threadIdx.x];
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = code_bytes / 4;
+  const int lo_bit = BPL * lane, w0 = lo_bit >> 5, w1 = (lo_bit + BPL - 1) >> 5, sh = lo_bit & 31;
   for (long long n0 = (static_cast<long long>(blockIdx.x) * WARPS + warp) * VPW; n0 < N;
        n0 += static_cast<long long>(gridDim.x) * WARPS * VPW) {
   uint32_t cw[VPW];
@@ -350,25 +353,23 @@ __global__ void __launch_bounds__(WARPS * 32) mse_decode_kernel(const uint8_t* _
   for (int u = 0; u < VPW; ++u) {
     if (n0 + u >= N) break;
     const long long n = n0 + u;
-    if (lane < MAX_CODE_WORDS) words[warp][lane] = lane < nw ? cw[u] : 0u;
-    __syncwarp();
+    // the lane's BPL code bits from the (at most two) words holding them
+    const uint32_t lo = __shfl_sync(0xffffffffu, cw[u], w0);
+    const uint32_t hi = __shfl_sync(0xffffffffu, cw[u], w1);
+    const uint32_t mine =
+        static_cast<uint32_t>(((static_cast<uint64_t>(hi) << 32) | lo) >> sh);
     const float nf = nrm[u];
     float out[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
-      const uint32_t code = read_bits(words[warp], bits * (lane * PER + e), bits);
-      const uint32_t mi = code & ((1u << (bits - 1)) - 1u);
-      float c = tb.c[0];
-#pragma unroll
-      for (int k = 1; k < 8; ++k)  // select with constant indices (no local copy of the table)
-        if (mi == static_cast<uint32_t>(k)) c = tb.c[k];
-      out[e] = __fmul_rn(nf, (code >> (bits - 1)) ? -c : c);
+      const uint32_t code = (mine >> (BITS * e)) & ((1u << BITS) - 1u);
+      const float c = sc[code & MMASK];
+      out[e] = __fmul_rn(nf, (code >> (BITS - 1)) ? -c : c);
     }
     if constexpr (PER == 4)
       reinterpret_cast<float4*>(xhat + n * D)[lane] = make_float4(out[0], out[1], out[2], out[3]);
     else
       reinterpret_cast<float2*>(xhat + n * D)[lane] = make_float2(out[0], out[1]);
-    __syncwarp();
   }
   }
 }
@@ -456,13 +457,23 @@ int launch_stage1(const tq_ctx* ctx, int kind, int b1, int b2, bool encode, cons
     }
   } else {
     const s1::MseTables tb = s1::mse_tables(d, b1);
-    if (encode) {
-      if (d == 128) s1::mse_encode_kernel<128><<<grid, threads, 0, st>>>(x, N, b1, cb, codes_out, norms_out, tb);
-      else s1::mse_encode_kernel<64><<<grid, threads, 0, st>>>(x, N, b1, cb, codes_out, norms_out, tb);
+#define TQ_S1_MSE(DD, BB)                                                                          \
+  do {                                                                                             \
+    if (encode)                                                                                    \
+      s1::mse_encode_kernel<DD, BB><<<grid, threads, 0, st>>>(x, N, cb, codes_out, norms_out, tb); \
+    else                                                                                           \
+      s1::mse_decode_kernel<DD, BB><<<grid, threads, 0, st>>>(codes_in, norms_in, N, cb, xhat, tb); \
+  } while (0)
+    if (d == 128) {
+      if (b1 == 2) TQ_S1_MSE(128, 2);
+      else if (b1 == 3) TQ_S1_MSE(128, 3);
+      else TQ_S1_MSE(128, 4);
     } else {
-      if (d == 128) s1::mse_decode_kernel<128><<<grid, threads, 0, st>>>(codes_in, norms_in, N, b1, cb, xhat, tb);
-      else s1::mse_decode_kernel<64><<<grid, threads, 0, st>>>(codes_in, norms_in, N, b1, cb, xhat, tb);
+      if (b1 == 2) TQ_S1_MSE(64, 2);
+      else if (b1 == 3) TQ_S1_MSE(64, 3);
+      else TQ_S1_MSE(64, 4);
     }
+#undef TQ_S1_MSE
   }
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
