@@ -380,11 +380,22 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   __shared__ float s_uk[G], s_uq[G];  // reciprocals of the fixed-point units
   if (tid < G) smr[tid] = sms[tid] = 0u;
   __syncthreads();
+  // per-head maxima: the 32 lanes of a warp share one head (D >= 32), so a
+  // warp reduction leaves one shared-memory atomic per warp and quantity
   for (int i = tid; i < G * D; i += blockDim.x) {
     const int g = i / D, j = i % D;
-    atomicMax(&smr[g], __float_as_uint(fabsf(sqr[g][j])));
-    atomicMax(&sms[g], __float_as_uint(fabsf(sqs[g][j])));
-    atomicMax(&smax[1][g], __float_as_uint(fabsf(p.sl * sq[g][j])));
+    float a = fabsf(sqr[g][j]), c = fabsf(sqs[g][j]), e = fabsf(p.sl * sq[g][j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
+      e = fmaxf(e, __shfl_xor_sync(0xffffffffu, e, o));
+    }
+    if ((tid & 31) == 0) {
+      atomicMax(&smr[g], __float_as_uint(a));
+      atomicMax(&sms[g], __float_as_uint(c));
+      atomicMax(&smax[1][g], __float_as_uint(e));
+    }
   }
   __syncthreads();
   {
