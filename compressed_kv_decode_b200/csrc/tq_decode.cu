@@ -142,7 +142,8 @@ __device__ __forceinline__ int hot_start_of(const Params& p, int b) {
 // ---------------------------------------------------------------------------
 // 0. threshold gate (gated form only)
 // ---------------------------------------------------------------------------
-constexpr int GATE_TOK = 128;  // hot slots per gate CTA (one 16-slot tile per warp)
+constexpr int GATE_TOK = 256;   // hot slots per gate CTA
+constexpr int GATE_TILES = 2;   // 16-slot tiles per warp (8 warps)
 
 // bit g set: q head g of group bh reads its cold tokens (after the gate launch)
 __device__ int gate_mask_of(const Params& p, int bh) {
@@ -490,7 +491,7 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
 // ---------------------------------------------------------------------------
 // Largest raw hot score max_t <q_g, k_t> of each q head g of a (batch, kv
 // head) group over one range of GATE_TOK ring slots (-inf where no slot of the
-// range holds a token).  Each warp scores one tile of 16 slots with m16n8k16
+// range holds a token).  Each warp scores GATE_TILES tiles of 16 slots with m16n8k16
 // MMAs: tokens on M, the group's heads x {hi, lo} fp16 parts of the
 // prescaled query on N, fp32 accumulation.  The contraction order inside a
 // k-step is free, so a lane's A fragment is two whole 16-byte chunks of its
@@ -508,20 +509,22 @@ __global__ void __launch_bounds__(256) gate_kernel(Params p) {
   __shared__ float wmax[8][G];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, c = lane & 3;
-  // the warp's two rows per lane: slots s0 (row g) and s0 + 8 (row g + 8).
-  // Every slot below W_max is loaded before the lengths are known (slots
-  // without a token only feed their own rows of the MMA and are masked).
-  const int s0 = split * GATE_TOK + warp * 16 + g;
-  uint4 kr[2][NCH];
+  // the warp's tiles (tile tt covers 16 slots from (tt * 8 + warp) * 16); per
+  // tile two rows per lane: row g and row g + 8 of the tile.  Every slot below
+  // W_max is loaded before the lengths are known (slots without a token only
+  // feed their own rows of the MMA and are masked).
+  uint4 kr[GATE_TILES][2][NCH];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int slot = s0 + 8 * h;
-    const uint4* row =
-        reinterpret_cast<const uint4*>(p.k_hot + (static_cast<size_t>(bh) * p.W_max + slot) * D);
+  for (int tt = 0; tt < GATE_TILES; ++tt)
 #pragma unroll
-    for (int i = 0; i < NCH; ++i)
-      kr[h][i] = slot < p.W_max ? __ldg(row + c + 4 * i) : make_uint4(0u, 0u, 0u, 0u);
-  }
+    for (int h = 0; h < 2; ++h) {
+      const int slot = split * GATE_TOK + (tt * 8 + warp) * 16 + g + 8 * h;
+      const uint4* row =
+          reinterpret_cast<const uint4*>(p.k_hot + (static_cast<size_t>(bh) * p.W_max + slot) * D);
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+        kr[tt][h][i] = slot < p.W_max ? __ldg(row + c + 4 * i) : make_uint4(0u, 0u, 0u, 0u);
+    }
   constexpr int QPT = (G * D + 255) / 256;  // query elements per thread
   float qv[QPT];
 #pragma unroll
@@ -534,14 +537,16 @@ __global__ void __launch_bounds__(256) gate_kernel(Params p) {
   int len = p.hot_len[b];
   len = len < 0 ? 0 : (len > p.W_max ? p.W_max : len);  // the schedule reports the error
   const int start = hot_start_of(p, b);
-  bool valid[2];
+  bool valid[GATE_TILES][2];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int slot = s0 + 8 * h;
-    int rel = slot - start;
-    if (rel < 0) rel += p.W_max;
-    valid[h] = slot < p.W_max && rel < len;
-  }
+  for (int tt = 0; tt < GATE_TILES; ++tt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int slot = split * GATE_TOK + (tt * 8 + warp) * 16 + g + 8 * h;
+      int rel = slot - start;
+      if (rel < 0) rel += p.W_max;
+      valid[tt][h] = slot < p.W_max && rel < len;
+    }
   if (tid < G) smx[tid] = 0u;
   __syncthreads();
 #pragma unroll
@@ -574,24 +579,33 @@ __global__ void __launch_bounds__(256) gate_kernel(Params p) {
         }
       }
   }
-  float acc[NT][4];
+  float mx[NT];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+  for (int nt = 0; nt < NT; ++nt) mx[nt] = NEG_INF;
 #pragma unroll
-  for (int i = 0; i < NCH; ++i)
+  for (int tt = 0; tt < GATE_TILES; ++tt) {
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_f16(acc[nt], kr[tt][0][i].x, kr[tt][1][i].x, kr[tt][0][i].y, kr[tt][1][i].y,
+                bfr[i][0][nt][0], bfr[i][0][nt][1]);
+        mma_f16(acc[nt], kr[tt][0][i].z, kr[tt][1][i].z, kr[tt][0][i].w, kr[tt][1][i].w,
+                bfr[i][1][nt][0], bfr[i][1][nt][1]);
+      }
+    // lane (g, c) holds, for head c + 4 nt, the hi and lo parts of rows g and g + 8
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      mma_f16(acc[nt], kr[0][i].x, kr[1][i].x, kr[0][i].y, kr[1][i].y, bfr[i][0][nt][0],
-              bfr[i][0][nt][1]);
-      mma_f16(acc[nt], kr[0][i].z, kr[1][i].z, kr[0][i].w, kr[1][i].w, bfr[i][1][nt][0],
-              bfr[i][1][nt][1]);
+      if (valid[tt][0]) mx[nt] = fmaxf(mx[nt], acc[nt][0] + acc[nt][1]);
+      if (valid[tt][1]) mx[nt] = fmaxf(mx[nt], acc[nt][2] + acc[nt][3]);
     }
-  // lane (g, c) holds, for head c + 4 nt, the hi and lo parts of rows g and g + 8
+  }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    float m = NEG_INF;
-    if (valid[0]) m = acc[nt][0] + acc[nt][1];
-    if (valid[1]) m = fmaxf(m, acc[nt][2] + acc[nt][3]);
+    float m = mx[nt];
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const int hh = c + 4 * nt;
