@@ -123,9 +123,9 @@ __device__ __forceinline__ void load_row(const float* x, long long n, long long 
   }
 }
 
-template <int D>
+template <int D, int B1, int B2>
 __global__ void __launch_bounds__(WARPS * 32) polar_encode_kernel(const float* __restrict__ x,
-                                                                  long long N, int b1, int b2,
+                                                                  long long N,
                                                                   int code_bytes,
                                                                   uint8_t* __restrict__ codes,
                                                                   uint16_t* __restrict__ radius,
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(WARPS * 32) polar_encode_kernel(const float* _
   constexpr int NL = log2i(D) - 1;
   __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int M = 1 << b1, L = 1 << b2;
+  constexpr int b1 = B1, b2 = B2, M = 1 << B1, L = 1 << B2;
   for (long long n = static_cast<long long>(blockIdx.x) * WARPS + warp; n < N;
        n += static_cast<long long>(gridDim.x) * WARPS) {
     if (lane < MAX_CODE_WORDS) words[warp][lane] = 0u;
@@ -148,14 +148,16 @@ __global__ void __launch_bounds__(WARPS * 32) polar_encode_kernel(const float* _
       const float2 t = reinterpret_cast<const float2*>(x + n * D)[lane];
       v[0] = t.x; v[1] = t.y;
     }
-    // level 1: the lane's pairs
+    // level 1: the lane's pairs, contiguous bits, assembled across lanes
     float r[PAIRS];
+    uint32_t mine = 0u;
 #pragma unroll
     for (int p = 0; p < PAIRS; ++p) {
-      const int i = lane * PAIRS + p;
-      or_bits(words[warp], b1 * i, b1, static_cast<uint32_t>(level1_bin(v[2 * p], v[2 * p + 1], M, tb)));
+      mine |= static_cast<uint32_t>(level1_bin(v[2 * p], v[2 * p + 1], M, tb)) << (b1 * p);
       r[p] = tree_radius(v[2 * p], v[2 * p + 1]);
     }
+    const uint32_t w1 = assemble_words(mine, PAIRS * b1, lane);  // words 0 .. PAIRS b1 - 1
+    uint32_t w2 = 0u;  // (d = 128) the level-2 words, held by lanes 0 .. b2 - 1
     // levels >= 2: node i of a level pairs the radii of nodes 2i, 2i + 1 below
     int base = b1 * (D / 2);
     int nodes = D / 2;
@@ -168,9 +170,10 @@ __global__ void __launch_bounds__(WARPS * 32) polar_encode_kernel(const float* _
       const float re = r[0], ro = r[1];
       int j = 0;
       if (ro > 0.0f)
+#pragma unroll
         for (int s = 0; s < L - 1; ++s)
           if (ro >= __fmul_rn(re, tb.T[0][s])) j = s + 1;
-      or_bits(words[warp], base + b2 * lane, b2, static_cast<uint32_t>(j));
+      w2 = assemble_words(static_cast<uint32_t>(j), b2, lane);  // one code per lane
       rr = tree_radius(re, ro);
       held = lane;
       base += b2 * nodes;
@@ -186,6 +189,7 @@ __global__ void __launch_bounds__(WARPS * 32) polar_encode_kernel(const float* _
         const float re = rr;
         int j = 0;
         if (ro > 0.0f)
+#pragma unroll
           for (int s = 0; s < L - 1; ++s)
             if (ro >= __fmul_rn(re, tb.T[lvl][s])) j = s + 1;
         const int node = held / 2;
@@ -196,23 +200,28 @@ __global__ void __launch_bounds__(WARPS * 32) polar_encode_kernel(const float* _
       base += b2 * nodes;
     }
     __syncwarp();
+    // words: level 1 from w1, (d = 128) level 2 from w2, the rest from shared memory
+    constexpr int n1 = PAIRS * b1, n2 = (PAIRS == 2) ? b2 : 0;
+    const uint32_t w2l = __shfl_sync(0xffffffffu, w2, (lane - n1) & 31);
     if (lane < code_bytes / 4)
-      reinterpret_cast<uint32_t*>(codes + n * code_bytes)[lane] = words[warp][lane];
+      reinterpret_cast<uint32_t*>(codes + n * code_bytes)[lane] =
+          lane < n1 ? w1 : (lane < n1 + n2 ? w2l : words[warp][lane]);
     if (lane == 0) radius[n] = __half_as_ushort(__float2half_rn(rr));
     __syncwarp();
   }
 }
 
-template <int D>
+template <int D, int B1, int B2>
 __global__ void __launch_bounds__(WARPS * 32) polar_decode_kernel(const uint8_t* __restrict__ codes,
                                                                   const uint16_t* __restrict__ radius,
-                                                                  long long N, int b1, int b2,
+                                                                  long long N,
                                                                   int code_bytes,
                                                                   float* __restrict__ xhat,
                                                                   PolarTables tb) {
   constexpr int PER = D / 32;
   constexpr int PAIRS = PER / 2;
   constexpr int NL = log2i(D) - 1;
+  constexpr int b1 = B1, b2 = B2;
   __shared__ uint32_t words[WARPS][MAX_CODE_WORDS];
   // the tables are read with per-lane indices: from shared memory, not the
   // kernel parameters (whose reads serialise over distinct addresses)
@@ -448,13 +457,33 @@ int launch_stage1(const tq_ctx* ctx, int kind, int b1, int b2, bool encode, cons
   const int threads = s1::WARPS * 32;
   if (kind == TQ_STAGE1_POLAR) {
     const s1::PolarTables tb = s1::polar_tables(d, b1, b2);
-    if (encode) {
-      if (d == 128) s1::polar_encode_kernel<128><<<grid, threads, 0, st>>>(x, N, b1, b2, cb, codes_out, norms_out, tb);
-      else s1::polar_encode_kernel<64><<<grid, threads, 0, st>>>(x, N, b1, b2, cb, codes_out, norms_out, tb);
-    } else {
-      if (d == 128) s1::polar_decode_kernel<128><<<grid, threads, 0, st>>>(codes_in, norms_in, N, b1, b2, cb, xhat, tb);
-      else s1::polar_decode_kernel<64><<<grid, threads, 0, st>>>(codes_in, norms_in, N, b1, b2, cb, xhat, tb);
-    }
+#define TQ_S1_POLAR(DD, BB1, BB2)                                                                  \
+  do {                                                                                             \
+    if (encode)                                                                                    \
+      s1::polar_encode_kernel<DD, BB1, BB2><<<grid, threads, 0, st>>>(x, N, cb, codes_out,          \
+                                                                      norms_out, tb);               \
+    else                                                                                           \
+      s1::polar_decode_kernel<DD, BB1, BB2><<<grid, threads, 0, st>>>(codes_in, norms_in, N, cb,    \
+                                                                      xhat, tb);                    \
+  } while (0)
+#define TQ_S1_POLAR_B2(DD, BB1)                 \
+  do {                                          \
+    if (b2 == 1) TQ_S1_POLAR(DD, BB1, 1);       \
+    else if (b2 == 2) TQ_S1_POLAR(DD, BB1, 2);  \
+    else TQ_S1_POLAR(DD, BB1, 3);               \
+  } while (0)
+#define TQ_S1_POLAR_D(DD)                       \
+  do {                                          \
+    if (b1 == 2) TQ_S1_POLAR_B2(DD, 2);         \
+    else if (b1 == 3) TQ_S1_POLAR_B2(DD, 3);    \
+    else if (b1 == 4) TQ_S1_POLAR_B2(DD, 4);    \
+    else TQ_S1_POLAR_B2(DD, 5);                 \
+  } while (0)
+    if (d == 128) TQ_S1_POLAR_D(128);
+    else TQ_S1_POLAR_D(64);
+#undef TQ_S1_POLAR_D
+#undef TQ_S1_POLAR_B2
+#undef TQ_S1_POLAR
   } else {
     const s1::MseTables tb = s1::mse_tables(d, b1);
 #define TQ_S1_MSE(DD, BB)                                                                          \
