@@ -113,6 +113,7 @@ struct Params {
   float gate_thr;
   int gate_nsplit;     // hot slot ranges of GATE_TOK slots
   int32_t* cold_used;  // [B, Hq] out (gated form), or null
+  DecodeFuse fuse;     // combine epilogue (fuse.r null: none)
 };
 
 __device__ __forceinline__ int* unit_off(const Params& p) { return p.w.sched + 4; }
@@ -1292,9 +1293,18 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(Params p) {
       const float den = Lc * fc + Lh * fh;
       res = (den > 0.0f) ? ((fc > 0.0f ? oc * fc : 0.0f) + (fh > 0.0f ? oh * fh : 0.0f)) / den : 0.0f;
     }
-    p.out[(static_cast<size_t>(b) * p.Hq + kvh * G + g) * D + j] = res;
+    const size_t oi = (static_cast<size_t>(b) * p.Hq + kvh * G + g) * D + j;
+    if (p.fuse.r) {  // out += sigmoid(gate) r
+      const float sg = 1.0f / (1.0f + expf(-p.fuse.gate[kvh * G + g]));
+      res = fmaf(sg, p.fuse.r[oi], res);
+    }
+    p.out[oi] = res;
     if (j == 0 && p.gated && p.cold_used)
       p.cold_used[static_cast<size_t>(b) * p.Hq + kvh * G + g] = open;
+  }
+  if (p.fuse.r && kvh == 0 && tid == 0) {
+    p.fuse.dst_start[b] = p.fuse.src_start[b];
+    p.fuse.dst_len[b] = p.fuse.src_len[b];
   }
 }
 
@@ -1444,7 +1454,7 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
                   const int32_t* hot_start, const int32_t* hot_len, const uint8_t* pool,
                   int64_t pool_pages, const int32_t* page_table, int max_pages,
                   const int32_t* cold_len, const DecodeGate* gate, float* out, void* ws,
-                  size_t ws_bytes, void* stream) {
+                  size_t ws_bytes, void* stream, const DecodeFuse* fuse) {
   const int d = ctx->cfg.head_dim;
   const int G = Hq / Hkv;
   const PageLayout L = page_layout(d, ctx->cfg.qjl_dim, true);
@@ -1462,6 +1472,7 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
   p.v_hot = static_cast<const __half*>(v_hot);
   p.hot_len = hot_len;
   p.hot_start = hot_start;
+  if (fuse) p.fuse = *fuse;
   if (gate) {
     p.gated = 1;
     p.gate_thr = gate->threshold;

@@ -78,13 +78,25 @@ struct DecodeGate {
   int32_t* cold_used;
 };
 
+// Optional epilogue of the decode's combine: out += sigmoid(gate[h]) r (the
+// Tensor Cache memory read), and the ring start and length of the step copied
+// back to the caller's arrays.
+struct DecodeFuse {
+  const float* r;         // [B, Hq, D]
+  const float* gate;      // [Hq]
+  const int32_t* src_start;
+  const int32_t* src_len;  // [B]
+  int32_t* dst_start;
+  int32_t* dst_len;  // [B]
+};
+
 // Launchers (defined in the .cu files).  Return a tq_status.
 int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq, int Hkv,
                   float scale, const void* k_hot, const void* v_hot, int W_max,
                   const int32_t* hot_start, const int32_t* hot_len, const uint8_t* pool,
                   int64_t pool_pages, const int32_t* page_table, int max_pages,
                   const int32_t* cold_len, const DecodeGate* gate, float* out, void* ws,
-                  size_t ws_bytes, void* stream);
+                  size_t ws_bytes, void* stream, const DecodeFuse* fuse = nullptr);
 size_t decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max);
 
 int launch_compress(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype, int flags,

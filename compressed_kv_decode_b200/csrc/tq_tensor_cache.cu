@@ -13,8 +13,9 @@
 //            partial products of the read.  The new ring start and length go
 //            to the workspace (the caller's arrays are read by every head).
 //   decode   the split-K attention over the ring alone (prep, attention,
-//            combine), with the ring start and length of this step
-//   fuse     y += sigmoid(g) r; the new ring start and length written back
+//            combine), with the ring start and length of this step; the
+//            combine's epilogue adds sigmoid(g) r and writes the new ring
+//            start and length back
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -113,23 +114,6 @@ __global__ void __launch_bounds__(256) update_kernel(const void* q, int q_dtype,
   }
 }
 
-__global__ void fuse_kernel(float* out, const float* r, const float* gate, int B, int Hq, int D,
-                            const int32_t* new_start, const int32_t* new_len, int32_t* ring_start,
-                            int32_t* ring_len) {
-  const long long n = static_cast<long long>(B) * Hq * D;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int hq = static_cast<int>((i / D) % Hq);
-    const float s = 1.0f / (1.0f + expf(-gate[hq]));
-    out[i] = fmaf(s, r[i], out[i]);
-  }
-  if (blockIdx.x == 0)
-    for (int b = threadIdx.x; b < B; b += blockDim.x) {
-      ring_start[b] = new_start[b];
-      ring_len[b] = new_len[b];
-    }
-}
-
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 }  // namespace tcache
@@ -189,13 +173,10 @@ int launch_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype,
   }
 #undef TQ_TC_LAUNCH
   if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
-  const int rc = launch_decode(ctx, q, q_dtype, B, Hq, Hkv, scale, k_ring, v_ring, W, ns, nl,
-                               nullptr, 0, nullptr, 0, nullptr, nullptr, out, ws, dec, stream);
-  if (rc != TQ_OK) return rc;
-  const long long n = static_cast<long long>(B) * Hq * d;
-  const int blocks = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
-  tcache::fuse_kernel<<<blocks, 256, 0, st>>>(out, r, gate, B, Hq, d, ns, nl, ring_start, ring_len);
-  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  // the combine adds sigmoid(g) r and writes the ring start and length back
+  const DecodeFuse fz{r, gate, ns, nl, ring_start, ring_len};
+  return launch_decode(ctx, q, q_dtype, B, Hq, Hkv, scale, k_ring, v_ring, W, ns, nl, nullptr, 0,
+                       nullptr, 0, nullptr, nullptr, out, ws, dec, stream, &fz);
 }
 
 }  // namespace tq
