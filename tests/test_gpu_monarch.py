@@ -186,3 +186,58 @@ def run_case(O, d, G, window, E, steps, mode, seed, cold0=(150, 0), hot0=None, s
 def test_monarch_steps_match_oracle(O, d, G, window, E, mode):
     steps = 40 if E < 128 else 140
     run_case(O, d, G, window, E, steps, mode, seed=d + G + E)
+
+
+def test_full_ring_is_reported_and_token_dropped(O):
+    """A ring already holding W_max tokens cannot take the step's token: the
+    append reports TQ_ERR_CAPACITY and leaves the ring and lengths as they
+    were; the rest of the step still runs on the stored state."""
+    import torch
+    d, G, window, E = 64, 2, 6, 2
+    ctx = ctx_for(d)
+    B, Hkv = 1, 1
+    Hq, W_max = G * Hkv, window + E
+    dev = "cuda"
+    k_hot = torch.randn((B, Hkv, W_max, d), device=dev).half()
+    v_hot = torch.randn((B, Hkv, W_max, d), device=dev).half()
+    k0 = k_hot.clone()
+    hs = torch.tensor([3], dtype=torch.int32, device=dev)
+    hl = torch.tensor([W_max], dtype=torch.int32, device=dev)
+    cl = torch.zeros(1, dtype=torch.int32, device=dev)
+    nbytes = ctx.page_bytes(True)
+    pool = torch.zeros((4, nbytes), dtype=torch.uint8, device=dev)
+    tbl = torch.arange(2, dtype=torch.int32, device=dev).view(1, 1, 2)
+    out = torch.empty((B, Hq, d), device=dev)
+    ws = torch.empty(tq.tq_monarch_workspace_bytes(ctx.handle, B, Hq, Hkv, 2, W_max, E),
+                     dtype=torch.uint8, device=dev)
+    q = torch.randn((B, Hq, d), device=dev)
+    kn = torch.randn((B, Hkv, d), device=dev).half()
+    tq.tq_monarch_step(ctx.handle, q, kn, kn, k_hot, v_hot, hs, hl, pool, tbl, cl, float("inf"),
+                       window, E, out, ws, Hkv)
+    torch.cuda.synchronize()
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_ERR_CAPACITY
+    # the stored window was full: the step then evicted its E oldest tokens
+    assert int(hl.item()) == W_max - E and int(cl.item()) == E
+    assert int(hs.item()) == (3 + E) % W_max
+    assert torch.equal(k_hot, k0)  # the dropped token was not written
+    assert torch.isfinite(out).all()
+
+
+def test_invalid_window_arguments_rejected():
+    import torch
+    ctx = ctx_for(64)
+    dev = "cuda"
+    B, Hkv, d = 1, 1, 64
+    k_hot = torch.zeros((B, Hkv, 8, d), device=dev).half()
+    z = torch.zeros(1, dtype=torch.int32, device=dev)
+    pool = torch.zeros((2, ctx.page_bytes(True)), dtype=torch.uint8, device=dev)
+    tbl = torch.zeros((1, 1, 2), dtype=torch.int32, device=dev)
+    out = torch.empty((B, 1, d), device=dev)
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device=dev)
+    q = torch.zeros((B, 1, d), device=dev)
+    with pytest.raises(tq.TQError):  # window + E > W_max
+        tq.tq_monarch_step(ctx.handle, q, None, None, k_hot, k_hot, z, z, pool, tbl, z,
+                           float("inf"), 7, 2, out, ws, Hkv)
+    with pytest.raises(tq.TQError):  # E = 0
+        tq.tq_monarch_step(ctx.handle, q, None, None, k_hot, k_hot, z, z, pool, tbl, z,
+                           float("inf"), 4, 0, out, ws, Hkv)

@@ -108,3 +108,21 @@ def test_unsupported_bits_rejected():
     assert tq.tq_stage1_code_bytes(ctx.handle, tq.TQ_STAGE1_MSE, 5, 0) == 0
     assert tq.tq_stage1_code_bytes(ctx.handle, tq.TQ_STAGE1_POLAR, 4, 2) == 48
     assert tq.tq_stage1_code_bytes(ctx.handle, tq.TQ_STAGE1_MSE, 3, 0) == 48
+
+
+def test_empty_batch_and_unsupported_calls():
+    import torch
+    ctx = ctx_for(128)
+    x = torch.zeros((0, 128), device="cuda")
+    codes = torch.zeros((0, 48), dtype=torch.uint8, device="cuda")
+    norms = torch.zeros(0, dtype=torch.int16, device="cuda")
+    tq.tq_stage1_encode(ctx.handle, tq.TQ_STAGE1_POLAR, 4, 2, x, codes, norms)  # N = 0: no-op
+    x1 = torch.zeros((1, 128), device="cuda")
+    c1 = torch.zeros((1, 64), dtype=torch.uint8, device="cuda")
+    n1 = torch.zeros(1, dtype=torch.int16, device="cuda")
+    with pytest.raises(tq.TQError):
+        tq.tq_stage1_encode(ctx.handle, tq.TQ_STAGE1_POLAR, 6, 2, x1, c1, n1)
+    with pytest.raises(tq.TQError):
+        tq.tq_stage1_encode(ctx.handle, tq.TQ_STAGE1_MSE, 1, 0, x1, c1, n1)
+    torch.cuda.synchronize()
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_OK

@@ -97,3 +97,29 @@ def test_tensor_cache_steps_match_oracle(O, d, G, W, qdt):
                 assert np.array_equal(kg[b, h, (exp_start[b] + i) % W], k)
     Ag = A.cpu().numpy().astype(np.float64)
     assert np.abs(Ag - tc.A).max() <= 1e-5 * np.abs(tc.A).max()
+
+
+def test_invalid_ring_state_is_reported_and_reset(O):
+    import torch
+    d, Hkv, G, W = 64, 1, 2, 4
+    ctx = ctx_for(d)
+    dev = "cuda"
+    B = 2
+    kr = torch.zeros((B, Hkv, W, d), device=dev).half()
+    rs = torch.tensor([0, 0], dtype=torch.int32, device=dev)
+    rl = torch.tensor([W + 3, 1], dtype=torch.int32, device=dev)  # sequence 0 is corrupt
+    A = torch.zeros((B, Hkv, d, d), device=dev)
+    lam = torch.ones(Hkv, device=dev)
+    eta = torch.ones(Hkv, device=dev)
+    gate = torch.zeros(Hkv * G, device=dev)
+    out = torch.empty((B, Hkv * G, d), device=dev)
+    ws = torch.empty(tq.tq_tensor_cache_workspace_bytes(ctx.handle, B, Hkv * G, Hkv, W),
+                     dtype=torch.uint8, device=dev)
+    q = torch.randn((B, Hkv * G, d), device=dev)
+    kn = torch.randn((B, Hkv, d), device=dev).half()
+    tq.tq_tensor_cache_step(ctx.handle, q, kn, kn, kr, kr.clone(), rs, rl, A, lam, eta, gate, out,
+                            ws, Hkv)
+    torch.cuda.synchronize()
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_ERR_CAPACITY
+    assert rl.cpu().tolist() == [0, 2] and rs.cpu().tolist() == [0, 0]
+    assert torch.isfinite(out).all() and not out[0].any()
