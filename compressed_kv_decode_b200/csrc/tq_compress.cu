@@ -377,13 +377,8 @@ __global__ void advance_kernel(int32_t* cold_len, int B, int n_new) {
 template <int D, int IN>
 int run(const tq_ctx* ctx, Params& p, cudaStream_t st) {
   using C = Cfg<D>;
-  static bool set = false;
-  if (!set) {
-    if (cudaFuncSetAttribute(compress_kernel<D, IN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM) != cudaSuccess)
-      return TQ_ERR_CUDA;
-    set = true;
-  }
+  static SmemAttr attr;
+  if (!raise_smem_limit(compress_kernel<D, IN>, C::SMEM, attr)) return TQ_ERR_CUDA;
   const long long tiles = static_cast<long long>(p.B) * p.Hkv * p.tiles_per_bh;
   const int grid = static_cast<int>(tiles < ctx->num_sms ? tiles : ctx->num_sms);
   if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);

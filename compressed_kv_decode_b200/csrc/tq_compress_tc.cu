@@ -846,13 +846,11 @@ int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf1
   const long long tiles = static_cast<long long>(B) * Hkv * p.tiles_per_bh;
   const int grid = static_cast<int>(tiles < ctx->num_sms ? tiles : ctx->num_sms);
   auto go = [&](auto kern, int smem) -> int {
-    static bool set[4] = {};
+    // one record per kernel: every instantiation has the same function-pointer
+    // type, so they are told apart by head dim and input type
+    static SmemAttr attr[4];
     const int slot = (d == 128 ? 2 : 0) + (bf16 ? 1 : 0);
-    if (!set[slot]) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return TQ_ERR_CUDA;
-      set[slot] = true;
-    }
+    if (!raise_smem_limit(kern, smem, attr[slot])) return TQ_ERR_CUDA;
     if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
     kern<<<grid, ctc::NTHREADS, smem, st>>>(mk, mv, p);
     if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
@@ -863,13 +861,9 @@ int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf1
   if (!v) {
     // keys only: the software-pipelined kernel
     auto gok = [&](auto kern, int smem) -> int {
-      static bool set[4] = {};
+      static SmemAttr attr[4];  // per head dim and input type, as above
       const int slot = (d == 128 ? 2 : 0) + (bf16 ? 1 : 0);
-      if (!set[slot]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-          return TQ_ERR_CUDA;
-        set[slot] = true;
-      }
+      if (!raise_smem_limit(kern, smem, attr[slot])) return TQ_ERR_CUDA;
       if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
       kern<<<grid, ctc::KTHREADS, smem, st>>>(mk, p);
       if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);

@@ -1362,14 +1362,8 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
   p.w.gmax = reinterpret_cast<float*>(base + L.gmax);
   p.w.gmask = reinterpret_cast<int*>(base + L.gmask);
   p.gate_nsplit = gate_splits(p.W_max);
-  static bool attr_set[2][9] = {};
-  bool& set = attr_set[D == 128][G];
-  if (!set) {
-    if (cudaFuncSetAttribute(attn_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM) != cudaSuccess)
-      return TQ_ERR_CUDA;
-    set = true;
-  }
+  static SmemAttr attn_attr;
+  if (!raise_smem_limit(attn_kernel<D, G>, C::SMEM, attn_attr)) return TQ_ERR_CUDA;
   if (p.gated && p.gate_nsplit > 0) {
     // gate, then prep overlapping it: only prep's schedule CTA waits for the maxima
     gate_kernel<D, G><<<dim3(p.gate_nsplit, p.B * p.Hkv), 256, 0, st>>>(p);
@@ -1401,14 +1395,8 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
     if (cudaLaunchKernelEx(&cfg, attn_kernel<D, G>, p) != cudaSuccess) return TQ_ERR_CUDA;
   }
   if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
-  static bool comb_set[2][9] = {};
-  bool& cset = comb_set[D == 128][G];
-  if (!cset) {
-    if (cudaFuncSetAttribute(combine_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CombCfg<D, G>::SMEM) != cudaSuccess)
-      return TQ_ERR_CUDA;
-    cset = true;
-  }
+  static SmemAttr comb_attr;
+  if (!raise_smem_limit(combine_kernel<D, G>, CombCfg<D, G>::SMEM, comb_attr)) return TQ_ERR_CUDA;
   {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(p.B * p.Hkv);

@@ -1,6 +1,9 @@
 // Internal declarations shared by the host-side files of libtq.
 #pragma once
 
+#include <cuda_runtime.h>
+
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <vector>
@@ -8,6 +11,30 @@
 #include "../../include/tq.h"
 
 namespace tq {
+
+// The dynamic shared-memory limit already raised for one kernel, per device
+// (zero-initialised as a static; safe to share between threads).
+struct SmemAttr {
+  std::atomic<int> bytes[64];
+};
+
+// Raise `kernel`'s dynamic shared-memory limit to at least `bytes` on the
+// current device, once per device and size.
+template <typename K>
+inline bool raise_smem_limit(K kernel, int bytes, SmemAttr& st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::atomic<int>* slot = (dev >= 0 && dev < 64) ? &st.bytes[dev] : nullptr;
+  if (slot && slot->load(std::memory_order_acquire) >= bytes) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  if (slot) {
+    int cur = slot->load(std::memory_order_relaxed);
+    while (cur < bytes && !slot->compare_exchange_weak(cur, bytes, std::memory_order_release)) {
+    }
+  }
+  return true;
+}
 
 struct HostTables {
   std::vector<float> rot;    // [d*d] row-major, x_rot = rot x

@@ -830,13 +830,9 @@ int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* d
     size_t smem = C::smem_bytes(k);
     if (smem < 116 * 1024) smem = 116 * 1024;
     if (smem > 232448) return TQ_ERR_UNSUPPORTED;
-    static size_t smem_set = 0;
-    if (smem > smem_set) {
-      if (cudaFuncSetAttribute(tk::score_kernel<D, QB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
-        return TQ_ERR_CUDA;
-      smem_set = smem;
-    }
+    static SmemAttr score_attr;  // one per kernel instantiation; grows with k
+    if (!raise_smem_limit(tk::score_kernel<D, QB>, static_cast<int>(smem), score_attr))
+      return TQ_ERR_CUDA;
     tk::qprep_kernel<D, QB><<<p.n_qb * QB, 128, 0, st>>>(p);
     if (ctx->prof_start) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_start), st);
     // seeding pass over the first pages: every query's slots start from the
@@ -851,9 +847,9 @@ int launch_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* d
     }
     tk::score_kernel<D, QB><<<grid, tk::NTHREADS, smem, st>>>(p);
     if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
+    static SmemAttr merge_attr;
     if (merge_smem > 48 * 1024 &&
-        cudaFuncSetAttribute(tk::merge_kernel<QB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(merge_smem)) != cudaSuccess)
+        !raise_smem_limit(tk::merge_kernel<QB>, static_cast<int>(merge_smem), merge_attr))
       return TQ_ERR_CUDA;
     tk::merge_kernel<QB><<<Q, 128, merge_smem, st>>>(p, out_ids, out_scores);
     return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
