@@ -28,7 +28,7 @@
  *         region) and "Vereinfachte Decode-Schleife" (hot and cold scores,
  *         softmax, aggregation).
  *
- * Readings taken where the pages are silent (each also listed in the design doc):
+ * Readings taken where the pages are silent:
  *  - rotation: dense Haar-orthogonal matrix = Q of a QR factorisation of a
  *    Gaussian matrix with diag(R) made positive;
  *  - quantiser: Lloyd-Max for the exact marginal of one coordinate of a
