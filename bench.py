@@ -49,7 +49,7 @@ def parse():
                     help="sequences per GPU (default: the workload's 16); smaller values only "
                          "size profiler captures and are not the benchmark line")
     ap.add_argument("--only", default=None,
-                    choices=["gated", "monarch", "tensor_cache", "stage1"],
+                    choices=["gated", "monarch", "tensor_cache", "stage1", "self_index"],
                     help="run one extra row alone and print it (sized for profiler captures; "
                          "not the benchmark line)")
     return ap.parse_args()
@@ -378,6 +378,47 @@ def measure_tensor_cache(torch, tq, W, workload, steps=256):
             "achieved_gbs": by / (ms / 1e3) / 1e9}
 
 
+def measure_self_index(torch, tq, reps=3):
+    """Self-Indexing index build and LUT scores on the 32K decode's key
+    shapes (16 x 8 kv heads x 32768 fp16 keys, d = 128, 32 query heads):
+    kernel times (CUDA events, median of reps) and HBM GB/s over keys read +
+    codes and centroids written (build), codes read + scores written
+    (scores)."""
+    B, Hkv, Hq, T, d = 16, 8, 32, 32768, 128
+    ctx = tq.Context(d, seed=0)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(61)
+    k = torch.randn((B, Hkv, T, d), generator=gen, device="cuda").half()
+    q = torch.randn((B, Hq, d), generator=gen, device="cuda").to(torch.bfloat16)
+    mu = torch.empty((B, Hkv, d), device="cuda")
+    codes = torch.empty((B, Hkv, T, d // 4), dtype=torch.uint8, device="cuda")
+    cent = torch.empty((B, Hkv, d // 4, 16, 4), device="cuda")
+    scores = torch.empty((B, Hq, T), device="cuda")
+    tb, ts = [], []
+    for i in range(reps + 1):
+        for which, lst in (("build", tb), ("scores", ts)):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            if which == "build":
+                tq.tq_self_index_build(ctx.handle, k, mu, codes, cent)
+            else:
+                tq.tq_self_index_scores(ctx.handle, q, codes, cent, scores, Hkv)
+            b.record()
+            torch.cuda.synchronize()
+            if i > 0:
+                lst.append(a.elapsed_time(b))
+    ctx.check()
+    mb, ms = statistics.median(tb), statistics.median(ts)
+    by_b = B * Hkv * T * (2 * d + d // 4)
+    by_s = B * Hq * T * (d // 4 + 4)
+    peak = float(measured_peaks()[0]["hbm_gbs"])
+    return {"workload": "16 x 8 kv heads x 32768 fp16 keys, d=128; 32 query heads",
+            "build_ms": mb, "build_gbs": by_b / (mb / 1e3) / 1e9,
+            "build_hbm_frac": by_b / (mb / 1e3) / 1e9 / peak,
+            "scores_ms": ms, "scores_gbs": by_s / (ms / 1e3) / 1e9,
+            "scores_hbm_frac": by_s / (ms / 1e3) / 1e9 / peak}
+
+
 def measure_stage1(torch, tq, N=1 << 20, reps=5):
     """Stage-1 variants on 2^20 rotated fp32 vectors (d = 128, N(0,1)):
     encode and decode kernel times (CUDA events, median of reps) with their
@@ -620,6 +661,8 @@ def run_ours(args, rank, world, local_rank):
         rows["search"] = measure_search(torch, tq)
         torch.cuda.empty_cache()
         rows["stage1"] = measure_stage1(torch, tq)
+        torch.cuda.empty_cache()
+        rows["self_index"] = measure_self_index(torch, tq)
         peak_tf = float(peaks.get("bf16_tflops", 1590.0))
         rows["compress"]["hbm_frac"] = rows["compress"]["achieved_gbs"] / peak
         rows["compress"]["tensor_frac"] = rows["compress"]["achieved_tflops"] / peak_tf
@@ -662,6 +705,8 @@ def run_only(args):
         res = measure_monarch(torch, tq, W, "tinyllama", 128, steps=args.steps)
     elif args.only == "tensor_cache":
         res = measure_tensor_cache(torch, tq, W, WORKLOAD, steps=args.steps)
+    elif args.only == "self_index":
+        res = measure_self_index(torch, tq, reps=max(1, args.steps))
     else:
         res = measure_stage1(torch, tq, reps=max(1, args.steps))
     print(json.dumps({"only": args.only, "row": res}), flush=True)

@@ -90,6 +90,11 @@ def lib():
                                            vp, vp, vp, vp, C.c_int, i32p, i32p, f32p, f32p, f32p,
                                            f32p, f32p, vp, C.c_size_t, vp]
         L.tq_tensor_cache_step.restype = C.c_int
+        L.tq_self_index_build.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, f32p, u8p, f32p, vp]
+        L.tq_self_index_build.restype = C.c_int
+        L.tq_self_index_scores.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, u8p,
+                                           f32p, f32p, vp]
+        L.tq_self_index_scores.restype = C.c_int
         L.tq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int,
                                                   C.c_float, vp, vp, C.c_int, i32p, u8p, C.c_int64,
                                                   i32p, C.c_int, i32p, f32p, vp]
@@ -290,6 +295,26 @@ def tq_tensor_cache_step(ctx, q, k_new, v_new, k_ring, v_ring, ring_start, ring_
         _ptr(k_ring), _ptr(v_ring), k_ring.shape[2], _ptr(ring_start), _ptr(ring_len), _ptr(A),
         _ptr(lam), _ptr(eta), _ptr(gate), _ptr(out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)), "tq_tensor_cache_step")
+
+
+def tq_self_index_build(ctx, k, mu, codes, centroids, stream=None):
+    """k fp16 [B, Hkv, T, d] -> mu fp32 [B, Hkv, d], codes uint8 [B, Hkv, T, d/4],
+    centroids fp32 [B, Hkv, d/4, 16, 4] (sign-pattern index of the centred keys)."""
+    _require_cuda(k, mu, codes, centroids)
+    B, Hkv, T, _ = k.shape
+    _check(lib().tq_self_index_build(ctx, _ptr(k), B, Hkv, T, _ptr(mu), _ptr(codes),
+                                     _ptr(centroids), _stream(stream)), "tq_self_index_build")
+
+
+def tq_self_index_scores(ctx, q, codes, centroids, scores, Hkv, stream=None):
+    """q [B, Hq, d]; codes, centroids from tq_self_index_build; scores fp32
+    [B, Hq, T] out: sum over groups of <q_g, centroid[g][code]>."""
+    _require_cuda(q, codes, centroids, scores)
+    B, Hq, _ = q.shape
+    T = codes.shape[2]
+    _check(lib().tq_self_index_scores(ctx, _ptr(q), _dtype_code(q), B, Hq, Hkv, T, _ptr(codes),
+                                      _ptr(centroids), _ptr(scores), _stream(stream)),
+           "tq_self_index_scores")
 
 
 TQ_STAGE1_MSE, TQ_STAGE1_POLAR = 0, 1

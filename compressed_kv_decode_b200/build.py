@@ -8,7 +8,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtq.so")
 SOURCES = ["tq_api.cu", "tq_decode.cu", "tq_compress.cu", "tq_topk.cu", "tq_params.cpp",
            "tq_noalloc.cu", "tq_compress_tc.cu", "tq_monarch.cu",
-           "tq_stage1.cu", "tq_tensor_cache.cu"]
+           "tq_stage1.cu", "tq_tensor_cache.cu", "tq_self_index.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden",

@@ -337,6 +337,28 @@ tq_status tq_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtyp
       A, lambda, eta, gate, out, workspace, ws_bytes, stream));
 }
 
+tq_status tq_self_index_build(const tq_ctx* ctx, const void* k, int B, int Hkv, int T, float* mu,
+                              uint8_t* codes, float* centroids, void* stream) {
+  if (!ctx || !k || !mu || !codes || !centroids || B <= 0 || Hkv <= 0 || T <= 0)
+    return TQ_ERR_INVALID_ARG;
+  if (!tq::aligned(k, 16) || !tq::aligned(codes, 16) || !tq::aligned(centroids, 16))
+    return TQ_ERR_INVALID_ARG;
+  return static_cast<tq_status>(
+      tq::launch_self_index_build(ctx, k, B, Hkv, T, mu, codes, centroids, stream));
+}
+
+tq_status tq_self_index_scores(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                               int Hkv, int T, const uint8_t* codes, const float* centroids,
+                               float* scores, void* stream) {
+  if (!ctx || !q || !codes || !centroids || !scores || B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 ||
+      Hq % Hkv != 0)
+    return TQ_ERR_INVALID_ARG;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (!tq::aligned(codes, 16) || !tq::aligned(centroids, 16)) return TQ_ERR_INVALID_ARG;
+  return static_cast<tq_status>(tq::launch_self_index_scores(ctx, q, q_dtype, B, Hq, Hkv, T, codes,
+                                                             centroids, scores, stream));
+}
+
 size_t tq_stage1_code_bytes(const tq_ctx* ctx, int kind, int bits1, int bits2) {
   if (!ctx) return 0;
   return tq::stage1_code_bytes(ctx->cfg.head_dim, kind, bits1, bits2);

@@ -153,6 +153,11 @@ int launch_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype,
                              int32_t* ring_len, float* A, const float* lambda, const float* eta,
                              const float* gate, float* out, void* ws, size_t ws_bytes,
                              void* stream);
+int launch_self_index_build(const tq_ctx* ctx, const void* k, int B, int Hkv, int T, float* mu,
+                            uint8_t* codes, float* cent, void* stream);
+int launch_self_index_scores(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                             int Hkv, int T, const uint8_t* codes, const float* cent,
+                             float* scores, void* stream);
 size_t stage1_code_bytes(int d, int kind, int b1, int b2);
 int launch_stage1(const tq_ctx* ctx, int kind, int b1, int b2, bool encode, const float* x,
                   const uint8_t* codes_in, uint8_t* codes_out, const uint16_t* norms_in,

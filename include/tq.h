@@ -358,6 +358,31 @@ TQ_API tq_status tq_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype
                                       const float* lambda, const float* eta, const float* gate,
                                       float* out, void* workspace, size_t ws_bytes, void* stream);
 /*
+ * Self-Indexing KV cache, index and compressed-domain scores ("Self-Indexing
+ * KVCache", section "Methodologie: Self-Indexing KVCache", items 1-3).
+ * tq_self_index_build, per (batch, kv head) over its T keys:
+ *  k          device fp16 [B, Hkv, T, d], 16-byte aligned.
+ *  mu         device fp32 [B, Hkv, d] out: the channel mean (fp32 sum / T).
+ *  codes      device uint8 [B, Hkv, T, d/4] out, 16-byte aligned: for group
+ *             g (coordinates 4g .. 4g+3) bit i set where k - mu is positive
+ *             in coordinate 4g + i (zero is not).
+ *  centroids  device fp32 [B, Hkv, d/4, 16, 4] out, 16-byte aligned: the
+ *             mean of the centred subvectors with each index (zero vector for
+ *             an index no token has).  Summed with float atomics: the
+ *             summation order is not fixed.
+ * tq_self_index_scores: for every query head and token, the sum over groups
+ * of <q_g, centroid[g][code]> (a 16-entry table per group), i.e. the dot
+ * product of q with the token's centred reconstruction.
+ *  q          device [B, Hq, d] (F32, F16 or BF16); head h reads kv head
+ *             h / (Hq / Hkv).
+ *  scores     device fp32 [B, Hq, T] out.
+ */
+TQ_API tq_status tq_self_index_build(const tq_ctx* ctx, const void* k, int B, int Hkv, int T,
+                                     float* mu, uint8_t* codes, float* centroids, void* stream);
+TQ_API tq_status tq_self_index_scores(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B,
+                                      int Hq, int Hkv, int T, const uint8_t* codes,
+                                      const float* centroids, float* scores, void* stream);
+/*
  * Stage-1 quantiser variants on rotated vectors, for comparing distortion
  * ("Funktionsweise von TurboQuant": a standard per-coordinate quantiser after
  * the rotation; "PolarQuant: Ein neuer Winkel auf Kompression": coordinate
