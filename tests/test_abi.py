@@ -77,3 +77,35 @@ def test_init_without_device_fails_cleanly():
     cfg = tq.make_config(128, 0)
     st = tq.lib().tq_init_codebook(C.byref(cfg), C.byref(h))
     assert st == tq.TQ_ERR_CUDA and not h.value
+
+
+def test_null_context_on_the_next_row_entries():
+    """The gated decode, Monarch and Tensor Cache steps, the stage-1 variants
+    and the Self-Indexing calls reject a null context (and report no sizes)
+    on the host, before any device call."""
+    L = tq.lib()
+    INV = tq.TQ_ERR_INVALID_ARG
+    assert L.tq_monarch_workspace_bytes(None, 1, 1, 1, 1, 8, 1) == 0
+    assert L.tq_tensor_cache_workspace_bytes(None, 1, 1, 1, 8) == 0
+    assert L.tq_stage1_code_bytes(None, tq.TQ_STAGE1_POLAR, 4, 2) == 0
+    # ctx, q, q_dtype, B, Hq, Hkv, scale, k_hot, v_hot, W_max, hot_start, hot_len, pool,
+    # pool_pages, page_table, max_pages, cold_len, threshold, cold_used, out, workspace,
+    # ws_bytes, stream
+    gated = [None, None, 0, 1, 1, 1, 0.0, None, None, 0, None, None, None, 0, None, 0, None,
+             0.0, None, None, None, 0, None]
+    assert L.tq_decode_attention_gated(*gated) == INV
+    # ctx, q, q_dtype, B, Hq, Hkv, scale, k_new, v_new, k_hot, v_hot, W_max, hot_start,
+    # hot_len, pool, pool_pages, page_table, max_pages, cold_len, threshold, window, E,
+    # cold_used, out, workspace, ws_bytes, stream
+    mon = [None, None, 0, 1, 1, 1, 0.0, None, None, None, None, 8, None, None, None, 1, None, 1,
+           None, 0.0, 4, 2, None, None, None, 0, None]
+    assert L.tq_monarch_step(*mon) == INV
+    # ctx, q, q_dtype, B, Hq, Hkv, scale, k_new, v_new, k_ring, v_ring, W, ring_start,
+    # ring_len, A, lambda, eta, gate, out, workspace, ws_bytes, stream
+    tcs = [None, None, 0, 1, 1, 1, 0.0, None, None, None, None, 8, None, None, None, None, None,
+           None, None, None, 0, None]
+    assert L.tq_tensor_cache_step(*tcs) == INV
+    assert L.tq_stage1_encode(None, 1, 4, 2, None, 1, None, None, None) == INV
+    assert L.tq_stage1_decode(None, 1, 4, 2, None, None, 1, None, None) == INV
+    assert L.tq_self_index_build(None, None, 1, 1, 1, None, None, None, None) == INV
+    assert L.tq_self_index_scores(None, None, 0, 1, 1, 1, 1, None, None, None, None) == INV
