@@ -379,12 +379,15 @@ def measure_tensor_cache(torch, tq, W, workload, steps=256):
 
 
 def measure_self_index(torch, tq, reps=3):
-    """Self-Indexing index build and LUT scores on the 32K decode's key
-    shapes (16 x 8 kv heads x 32768 fp16 keys, d = 128, 32 query heads):
-    kernel times (CUDA events, median of reps) and HBM GB/s over keys read +
-    codes and centroids written (build), codes read + scores written
-    (scores)."""
+    """Self-Indexing on the 32K decode's key shapes (16 x 8 kv heads x 32768
+    fp16 keys and values, d = 128, 32 query heads, top_k = 7.5 % of T):
+    kernel times (CUDA events, median of reps) and GB/s over the algorithmic
+    bytes -- keys read + codes and centroids written (build), codes read +
+    scores written (scores), scores read + picked written (select; its four
+    digit passes re-read the scores from L2), the 64 sinks' and the picked
+    tokens' key and value rows read per query head (attend)."""
     B, Hkv, Hq, T, d = 16, 8, 32, 32768, 128
+    top_k = round(0.075 * T)
     ctx = tq.Context(d, seed=0)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(61)
@@ -394,29 +397,40 @@ def measure_self_index(torch, tq, reps=3):
     codes = torch.empty((B, Hkv, T, d // 4), dtype=torch.uint8, device="cuda")
     cent = torch.empty((B, Hkv, d // 4, 16, 4), device="cuda")
     scores = torch.empty((B, Hq, T), device="cuda")
-    tb, ts = [], []
+    v = torch.randn((B, Hkv, T, d), generator=gen, device="cuda").half()
+    picked = torch.empty((B, Hq, top_k), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, Hq, d), device="cuda")
+    times = {"build": [], "scores": [], "select": [], "attend": []}
     for i in range(reps + 1):
-        for which, lst in (("build", tb), ("scores", ts)):
+        for which, lst in times.items():
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             if which == "build":
                 tq.tq_self_index_build(ctx.handle, k, mu, codes, cent)
-            else:
+            elif which == "scores":
                 tq.tq_self_index_scores(ctx.handle, q, codes, cent, scores, Hkv)
+            elif which == "select":
+                tq.tq_self_index_select(ctx.handle, scores, picked)
+            else:
+                tq.tq_self_index_attend(ctx.handle, q, k, v, picked, out)
             b.record()
             torch.cuda.synchronize()
             if i > 0:
                 lst.append(a.elapsed_time(b))
     ctx.check()
-    mb, ms = statistics.median(tb), statistics.median(ts)
-    by_b = B * Hkv * T * (2 * d + d // 4)
-    by_s = B * Hq * T * (d // 4 + 4)
+    algo = {"build": B * Hkv * T * (2 * d + d // 4),
+            "scores": B * Hq * T * (d // 4 + 4),
+            "select": B * Hq * (T * 4 + top_k * 4),
+            "attend": B * Hq * ((64 + top_k) * 2 * d * 2 + top_k * 4 + d * 2 + d * 4)}
     peak = float(measured_peaks()[0]["hbm_gbs"])
-    return {"workload": "16 x 8 kv heads x 32768 fp16 keys, d=128; 32 query heads",
-            "build_ms": mb, "build_gbs": by_b / (mb / 1e3) / 1e9,
-            "build_hbm_frac": by_b / (mb / 1e3) / 1e9 / peak,
-            "scores_ms": ms, "scores_gbs": by_s / (ms / 1e3) / 1e9,
-            "scores_hbm_frac": by_s / (ms / 1e3) / 1e9 / peak}
+    row = {"workload": "16 x 8 kv heads x 32768 fp16 keys and values, d=128; 32 query "
+                       "heads; top_k = %d (7.5%% of T) + 64 sinks" % top_k}
+    for which, lst in times.items():
+        m = statistics.median(lst)
+        row[which + "_ms"] = m
+        row[which + "_gbs"] = algo[which] / (m / 1e3) / 1e9
+        row[which + "_hbm_frac"] = algo[which] / (m / 1e3) / 1e9 / peak
+    return row
 
 
 def measure_stage1(torch, tq, N=1 << 20, reps=5):

@@ -95,6 +95,11 @@ def lib():
         L.tq_self_index_scores.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, u8p,
                                            f32p, f32p, vp]
         L.tq_self_index_scores.restype = C.c_int
+        L.tq_self_index_select.argtypes = [vp, f32p, C.c_int, C.c_int, C.c_int, C.c_int, i32p, vp]
+        L.tq_self_index_select.restype = C.c_int
+        L.tq_self_index_attend.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, vp,
+                                           vp, i32p, C.c_int, C.c_int, C.c_float, f32p, vp]
+        L.tq_self_index_attend.restype = C.c_int
         L.tq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int,
                                                   C.c_float, vp, vp, C.c_int, i32p, u8p, C.c_int64,
                                                   i32p, C.c_int, i32p, f32p, vp]
@@ -315,6 +320,32 @@ def tq_self_index_scores(ctx, q, codes, centroids, scores, Hkv, stream=None):
     _check(lib().tq_self_index_scores(ctx, _ptr(q), _dtype_code(q), B, Hq, Hkv, T, _ptr(codes),
                                       _ptr(centroids), _ptr(scores), _stream(stream)),
            "tq_self_index_scores")
+
+
+def tq_self_index_select(ctx, scores, picked, n_sink=64, stream=None):
+    """scores fp32 [B, Hq, T] -> picked int32 [B, Hq, top_k]: the best
+    positions after the n_sink sinks in increasing order (ties to the lower
+    position), -1 past the available count."""
+    _require_cuda(scores, picked)
+    T = scores.shape[-1]
+    rows = int(np.prod(scores.shape[:-1]))
+    if tuple(picked.shape[:-1]) != tuple(scores.shape[:-1]):
+        raise ValueError("picked must be [..., top_k] over the rows of scores")
+    _check(lib().tq_self_index_select(ctx, _ptr(scores), rows, T, n_sink, picked.shape[-1],
+                                      _ptr(picked), _stream(stream)), "tq_self_index_select")
+
+
+def tq_self_index_attend(ctx, q, keys, values, picked, out, n_sink=64, scale=0.0, stream=None):
+    """q [B, Hq, d]; keys, values fp16 [B, Hkv, T, d]; picked int32
+    [B, Hq, top_k] -> out fp32 [B, Hq, d]: softmax attention over the sinks
+    and the picked positions."""
+    _require_cuda(q, keys, values, picked, out)
+    B, Hq, _ = q.shape
+    Hkv, T = keys.shape[1], keys.shape[2]
+    _check(lib().tq_self_index_attend(ctx, _ptr(q), _dtype_code(q), B, Hq, Hkv, T, _ptr(keys),
+                                      _ptr(values), _ptr(picked), n_sink, picked.shape[-1],
+                                      float(scale), _ptr(out), _stream(stream)),
+           "tq_self_index_attend")
 
 
 TQ_STAGE1_MSE, TQ_STAGE1_POLAR = 0, 1

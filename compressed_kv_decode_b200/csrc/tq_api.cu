@@ -359,6 +359,38 @@ tq_status tq_self_index_scores(const tq_ctx* ctx, const void* q, tq_dtype q_dtyp
                                                              centroids, scores, stream));
 }
 
+// Tokens the selection returns per row: top_k, or every position after the
+// sinks when there are fewer.
+static int self_index_k_eff(int T, int n_sink, int top_k) {
+  const int cand = T > n_sink ? T - n_sink : 0;
+  return top_k < cand ? top_k : cand;
+}
+
+tq_status tq_self_index_select(const tq_ctx* ctx, const float* scores, int rows, int T,
+                               int n_sink, int top_k, int32_t* picked, void* stream) {
+  if (!ctx || !scores || !picked || rows <= 0 || T < 0 || n_sink < 0 || top_k <= 0)
+    return TQ_ERR_INVALID_ARG;
+  const int lo = n_sink < T ? n_sink : T;
+  return static_cast<tq_status>(tq::launch_self_index_select(
+      scores, rows, T, lo, self_index_k_eff(T, n_sink, top_k), top_k, picked, stream));
+}
+
+tq_status tq_self_index_attend(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
+                               int Hkv, int T, const void* keys, const void* values,
+                               const int32_t* picked, int n_sink, int top_k, float scale,
+                               float* out, void* stream) {
+  if (!ctx || !q || !keys || !values || !picked || !out || B <= 0 || Hq <= 0 || Hkv <= 0 ||
+      Hq % Hkv != 0 || T < 0 || n_sink < 0 || top_k <= 0)
+    return TQ_ERR_INVALID_ARG;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (!tq::aligned(keys, 16) || !tq::aligned(values, 16)) return TQ_ERR_INVALID_ARG;
+  if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(ctx->cfg.head_dim));
+  const int n_s = n_sink < T ? n_sink : T;
+  return static_cast<tq_status>(tq::launch_self_index_attend(
+      ctx, q, q_dtype, B, Hq, Hkv, T, keys, values, picked, top_k,
+      self_index_k_eff(T, n_sink, top_k), n_s, scale, out, stream));
+}
+
 size_t tq_stage1_code_bytes(const tq_ctx* ctx, int kind, int bits1, int bits2) {
   if (!ctx) return 0;
   return tq::stage1_code_bytes(ctx->cfg.head_dim, kind, bits1, bits2);

@@ -383,6 +383,35 @@ TQ_API tq_status tq_self_index_scores(const tq_ctx* ctx, const void* q, tq_dtype
                                       int Hq, int Hkv, int T, const uint8_t* codes,
                                       const float* centroids, float* scores, void* stream);
 /*
+ * Top-k retrieval and sparse attention of the Self-Indexing form ("Self-
+ * Indexing KVCache", Methodologie items 3 and 4): per query head the top_k
+ * positions after the first n_sink tokens by LUT score, then exact softmax
+ * attention over the n_sink sink tokens and those positions with the stored
+ * full-precision keys and values.  k_eff = min(top_k, max(T - n_sink, 0)).
+ * tq_self_index_select:
+ *  scores   device fp32 [rows, T] (rows = B * Hq), not NaN.
+ *  picked   device int32 [rows, top_k] out: the k_eff best positions in
+ *           [n_sink, T), in increasing position order; equal scores go to the
+ *           lower position (-0.0 equals +0.0); entries k_eff.. are -1.
+ * tq_self_index_attend:
+ *  q        device [B, Hq, d] (F32, F16 or BF16); head h reads kv head
+ *           h / (Hq / Hkv).
+ *  keys, values  device fp16 [B, Hkv, T, d], 16-byte aligned.
+ *  picked   device int32 [B * Hq, top_k] as tq_self_index_select writes it;
+ *           the first k_eff entries are read.  An entry outside [0, T) is
+ *           skipped and recorded as TQ_ERR_INVALID_ARG on the context.
+ *  scale    softmax scale; 0 selects 1/sqrt(d).
+ *  out      device fp32 [B, Hq, d] out: sum_j softmax_j(scale <q, k_j>) v_j
+ *           over j in [0, min(n_sink, T)) and the picked positions; zero
+ *           when T = 0.
+ */
+TQ_API tq_status tq_self_index_select(const tq_ctx* ctx, const float* scores, int rows, int T,
+                                      int n_sink, int top_k, int32_t* picked, void* stream);
+TQ_API tq_status tq_self_index_attend(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B,
+                                      int Hq, int Hkv, int T, const void* keys,
+                                      const void* values, const int32_t* picked, int n_sink,
+                                      int top_k, float scale, float* out, void* stream);
+/*
  * Stage-1 quantiser variants on rotated vectors, for comparing distortion
  * ("Funktionsweise von TurboQuant": a standard per-coordinate quantiser after
  * the rotation; "PolarQuant: Ein neuer Winkel auf Kompression": coordinate

@@ -109,3 +109,6 @@ def test_null_context_on_the_next_row_entries():
     assert L.tq_stage1_decode(None, 1, 4, 2, None, None, 1, None, None) == INV
     assert L.tq_self_index_build(None, None, 1, 1, 1, None, None, None, None) == INV
     assert L.tq_self_index_scores(None, None, 0, 1, 1, 1, 1, None, None, None, None) == INV
+    assert L.tq_self_index_select(None, None, 1, 1, 64, 1, None, None) == INV
+    assert L.tq_self_index_attend(None, None, 0, 1, 1, 1, 1, None, None, None, 64, 1, 0.0, None,
+                                  None) == INV
