@@ -11,6 +11,9 @@ independent of any CUDA code.
   torch's scaled_dot_product_attention.
 - Selecting every post-sink token reduces the sparse attention to full
   attention (SDPA); selection ties go to the lower position.
+- Selection equals the first k of a brute-force sort of (-score, position)
+  tuples; sparse attention equals SDPA with a boolean mask over sinks +
+  picked.
 """
 import math
 
@@ -92,3 +95,32 @@ def test_full_selection_is_full_attention_and_ties():
     out0 = S.sparse_attention(q, K, V, [])
     ref0 = _sdpa(q[None], K[:S.N_SINK], V[:S.N_SINK], 1.0 / math.sqrt(d))[0]
     assert np.abs(out0 - ref0).max() < 1e-12
+
+
+def test_select_against_brute_force_order():
+    # the k best of (-score, position) tuples by Python's sort, on integer
+    # scores so that ties are common
+    rng = np.random.default_rng(4)
+    for trial in range(40):
+        T = int(rng.integers(0, 300))
+        n_sink = int(rng.choice([0, 5, 64]))
+        k = int(rng.integers(1, 320))
+        sc = rng.integers(-4, 5, T).astype(np.float64)
+        ranked = sorted(range(n_sink, T), key=lambda t: (-sc[t], t))
+        assert S.select(sc, k, n_sink).tolist() == sorted(ranked[:k])
+
+
+def test_sparse_attention_equals_masked_sdpa():
+    rng = np.random.default_rng(5)
+    T, d = 400, 32
+    K, V = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    q = rng.standard_normal(d)
+    picked = np.sort(rng.choice(np.arange(S.N_SINK, T), 37, replace=False))
+    keep = np.zeros(T, bool)
+    keep[:S.N_SINK] = True
+    keep[picked] = True
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float64))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        t(q)[None, None, None], t(K)[None, None], t(V)[None, None],
+        attn_mask=torch.from_numpy(keep)[None, None, None], scale=0.3)[0, 0, 0].numpy()
+    assert np.abs(S.sparse_attention(q, K, V, picked, scale=0.3) - ref).max() < 1e-12
