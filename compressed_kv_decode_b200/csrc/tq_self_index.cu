@@ -1,9 +1,10 @@
-// Self-Indexing KV cache, index build and compressed-domain scores ("Self-
-// Indexing KVCache", page 2, section "Methodologie: Self-Indexing KVCache",
-// items 1-3): keys are centred by their channel mean, cut into 4-dimensional
-// subvectors whose sign pattern is a 4-bit index, and a codebook of 16
-// centroids per group is built in one pass; a query scores every token by a
-// table of its dot products with the centroids (lookup and add).
+// Self-Indexing KV cache ("Self-Indexing KVCache", section "Methodologie:
+// Self-Indexing KVCache", items 1-4): keys are centred by their channel
+// mean, cut into 4-dimensional subvectors whose sign pattern is a 4-bit
+// index, and a codebook of 16 centroids per group is built in one pass; a
+// query scores every token by a table of its dot products with the centroids
+// (lookup and add), keeps the best tokens after the 64 full-precision sinks,
+// and attends over the sinks and those tokens only.
 //
 //  build   one CTA per (batch, kv head): channel mean (fp32), then every
 //          (token, group) index (one byte each, pattern in the low nibble)
@@ -12,6 +13,10 @@
 //  scores  one CTA per (batch, query head): the d/4 x 16 table in shared
 //          memory, then one token per thread: 4 x 16-byte loads of its d/4
 //          indices and d/4 table lookups.
+//  select  one CTA per (batch, query head): radix select of the top k
+//          scores, ties to the lower position, output in position order.
+//  attend  one CTA per (batch, query head): exact softmax attention over the
+//          sinks and the selected tokens' stored fp16 keys and values.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
