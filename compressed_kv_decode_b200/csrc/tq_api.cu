@@ -384,6 +384,7 @@ tq_status tq_self_index_attend(const tq_ctx* ctx, const void* q, tq_dtype q_dtyp
     return TQ_ERR_INVALID_ARG;
   if (q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
   if (!tq::aligned(keys, 16) || !tq::aligned(values, 16)) return TQ_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
   if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(ctx->cfg.head_dim));
   const int n_s = n_sink < T ? n_sink : T;
   return static_cast<tq_status>(tq::launch_self_index_attend(

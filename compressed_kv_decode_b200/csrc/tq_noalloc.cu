@@ -19,20 +19,45 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
+// Per device: the context the address was looked up in, and the address.  A
+// device reset (or any teardown of the primary context) loads the module
+// again, possibly at another address, so a cached address is reused only
+// while the current context is the one it came from.
+void* g_scratch_ctx[kMaxDevices] = {};
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up on
-// the first call for that device, with that device current).
+// cuCtxGetCurrent from the driver, reached through the runtime (no link to
+// the driver library); null if the driver does not provide it.
+using CtxGetCurrent = int (*)(void**);
+CtxGetCurrent ctx_get_current() {
+  static const CtxGetCurrent fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrent>(nullptr);
+    return reinterpret_cast<CtxGetCurrent>(f);
+  }();
+  return fn;
+}
+
+// Device address of the scratch array on the current device, looked up with
+// that device current on the first call and again whenever the current
+// context is not the one of the cached lookup (or cannot be told).
 tq_status scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return TQ_ERR_UNSUPPORTED;
+  void* cur = nullptr;
+  const CtxGetCurrent get = ctx_get_current();
+  const bool known = get != nullptr && get(&cur) == 0 && cur != nullptr;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (g_scratch_addr[dev] == nullptr || !known || g_scratch_ctx[dev] != cur) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr)
       return TQ_ERR_CUDA;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = known ? cur : nullptr;
   }
   *out = g_scratch_addr[dev];
   return TQ_OK;

@@ -128,8 +128,10 @@ __global__ void __launch_bounds__(256) scores_kernel(const void* q, int q_dtype,
 }
 
 // Ordered key of a score: a larger float gives a larger unsigned key; -0.0
-// and +0.0 share one key (they compare equal).
+// and +0.0 share one key (they compare equal); every NaN gets key 0, below
+// -inf, so NaN scores are picked last (ties among them to the lower position).
 __device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) return 0u;
   const uint32_t u = __float_as_uint(f == 0.0f ? 0.0f : f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }

@@ -290,8 +290,10 @@ TQ_API tq_status tq_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dt
  * workspace (tq_workspace_bytes) exceeds that size is rejected with
  * TQ_ERR_CAPACITY before any launch.
  *  - The first call on a device looks up the array's device address (a
- *    synchronous runtime call, once per device); make that first call before
- *    any stream capture.  The context's device must be the current device.
+ *    synchronous runtime call, once per device and CUDA context: after a
+ *    device reset the next call looks it up again); make that first call
+ *    before any stream capture.  The context's device must be the current
+ *    device.
  *  - All calls share the one array and it keeps the last call's contents
  *    (nothing in it needs to start at zero).  Calls that overlap on the GPU,
  *    from different streams or threads, race on it: serialise them.
@@ -389,10 +391,12 @@ TQ_API tq_status tq_self_index_scores(const tq_ctx* ctx, const void* q, tq_dtype
  * attention over the n_sink sink tokens and those positions with the stored
  * full-precision keys and values.  k_eff = min(top_k, max(T - n_sink, 0)).
  * tq_self_index_select:
- *  scores   device fp32 [rows, T] (rows = B * Hq), not NaN.
+ *  scores   device fp32 [rows, T] (rows = B * Hq).  A NaN score ranks below
+ *           every number, -inf included.
  *  picked   device int32 [rows, top_k] out: the k_eff best positions in
- *           [n_sink, T), in increasing position order; equal scores go to the
- *           lower position (-0.0 equals +0.0); entries k_eff.. are -1.
+ *           [n_sink, T), in increasing position order; equal scores (and NaN
+ *           scores among themselves) go to the lower position (-0.0 equals
+ *           +0.0); entries k_eff.. are -1.
  * tq_self_index_attend:
  *  q        device [B, Hq, d] (F32, F16 or BF16); head h reads kv head
  *           h / (Hq / Hkv).
@@ -400,7 +404,8 @@ TQ_API tq_status tq_self_index_scores(const tq_ctx* ctx, const void* q, tq_dtype
  *  picked   device int32 [B * Hq, top_k] as tq_self_index_select writes it;
  *           the first k_eff entries are read.  An entry outside [0, T) is
  *           skipped and recorded as TQ_ERR_INVALID_ARG on the context.
- *  scale    softmax scale; 0 selects 1/sqrt(d).
+ *  scale    softmax scale; 0 selects 1/sqrt(d); negative, NaN or infinite
+ *           is TQ_ERR_INVALID_ARG.
  *  out      device fp32 [B, Hq, d] out: sum_j softmax_j(scale <q, k_j>) v_j
  *           over j in [0, min(n_sink, T)) and the picked positions; zero
  *           when T = 0.

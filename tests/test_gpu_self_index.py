@@ -101,6 +101,11 @@ def _scores_rows(kind, rows, T, seed):
         return rng.standard_normal((rows, T)).astype(np.float32)
     if kind == "ties":
         return rng.integers(-3, 4, (rows, T)).astype(np.float32)
+    if kind == "nan":  # NaN scores rank below -inf, ties among them to the lower position
+        s = rng.standard_normal((rows, T)).astype(np.float32)
+        s[rng.random((rows, T)) < 0.6] = np.nan
+        s[rng.random((rows, T)) < 0.05] = -np.inf
+        return s
     # zeros of both signs among a few positive and negative values
     s = rng.integers(-1, 2, (rows, T)).astype(np.float32)
     neg0 = (s == 0) & (rng.random((rows, T)) < 0.5)
@@ -110,7 +115,8 @@ def _scores_rows(kind, rows, T, seed):
 
 @pytest.mark.parametrize("kind,T,n_sink,top_k", [
     ("normal", 5000, 64, 300), ("ties", 3000, 64, 1000), ("zeros", 2000, 0, 777),
-    ("normal", 200, 64, 500), ("normal", 50, 64, 10), ("ties", 40000, 64, 3000)])
+    ("normal", 200, 64, 500), ("normal", 50, 64, 10), ("ties", 40000, 64, 3000),
+    ("nan", 3000, 64, 1500)])
 def test_select_matches_oracle(kind, T, n_sink, top_k):
     import torch
     ctx = ctx_for(128)

@@ -17,7 +17,7 @@ from compressed_kv_decode_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def _case(torch, ctx, seed, B, Hkv, G, d, cold, hot, max_pages, qdtype):
+def _case(torch, ctx, seed, B, Hkv, G, d, hot, max_pages, qdtype):
     """Random but valid decode inputs on the device (pages of random records)."""
     dev = "cuda"
     nb = ctx.page_bytes(True)
@@ -58,15 +58,15 @@ def _without_workspace(torch, ctx, c):
 def test_noalloc_matches_workspace_call_twice_in_a_row():
     import torch
     ctx = tq.Context(128, seed=0)
-    big = _case(torch, ctx, 11, B=4, Hkv=8, G=4, d=128, cold=0, hot=64, max_pages=40,
-                qdtype="bfloat16")
-    small = _case(torch, ctx, 21, B=3, Hkv=2, G=8, d=128, cold=0, hot=16, max_pages=3,
-                  qdtype="float16")
+    big = _case(torch, ctx, 11, B=4, Hkv=8, G=4, d=128, hot=64, max_pages=40, qdtype="bfloat16")
+    small = _case(torch, ctx, 21, B=3, Hkv=2, G=8, d=128, hot=16, max_pages=3, qdtype="float16")
     for c in (big, small):
         ref = _with_workspace(torch, ctx, c)
         got = _without_workspace(torch, ctx, c)
         assert tq.tq_get_error(ctx.handle) == tq.TQ_OK
-        assert np.all(np.abs(got - ref) <= 2e-3 + 1e-2 * np.abs(ref))
+        # the same deterministic kernels on the same inputs: equal bit for bit,
+        # so anything left in the shared scratch by the previous call would show
+        assert np.array_equal(got, ref)
     ctx.close()
 
 
