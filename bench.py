@@ -522,10 +522,10 @@ def cpu_baseline(sample_groups=None):
     cores = os.cpu_count() or 1
     n = sample_groups or max(1, min(cfg["B"] * cfg["Hkv"], cores))
     P = O.Params(d, seed=0)
-    nbytes, offs = O.page_layout(d, d, True)
+    nbytes, _ = O.page_layout(d, d, True)
     max_pages = cfg["cold"] // 128
     table = np.arange(n * max_pages, dtype=np.int32).reshape(n, 1, max_pages)
-    pool = W.random_page_bytes(7, n * max_pages, nbytes, offs)
+    pool = W.random_page_bytes(7, n * max_pages, nbytes, O.norm_slots(d, d, True))
     rng = np.random.default_rng(8)
     k_hot = rng.standard_normal((n, 1, cfg["hot"], d)).astype(np.float16).astype(np.float64)
     v_hot = rng.standard_normal((n, 1, cfg["hot"], d)).astype(np.float16).astype(np.float64)

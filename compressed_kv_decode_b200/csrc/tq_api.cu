@@ -16,23 +16,28 @@ PageLayout page_layout(int d, int m, bool with_values) {
   auto up16 = [](size_t x) { return (x + 15) & ~static_cast<size_t>(15); };
   const size_t P = TQ_PAGE_TOKENS;
   PageLayout L{};
+  if (with_values) {
+    const size_t D = static_cast<size_t>(d), M = static_cast<size_t>(m);
+    L.kc = 0;
+    L.kl = 2 * D;
+    L.qs = 4 * D;
+    L.vc = 4 * D + 2 * M;
+    L.kn = 12 * D + 2 * M;
+    L.kg = L.kn + 2;
+    L.vn = L.kn + 64;
+    L.block = L.kn + 96;
+    L.bytes = (P / 16) * L.block;
+    return L;
+  }
   size_t off = 0;
   L.kc = off;
   off = up16(off + P * d / 4);
   L.qs = off;
   off = up16(off + P * m / 8);
-  if (with_values) {
-    L.vc = off;
-    off = up16(off + P * d / 2);
-  }
   L.kn = off;
   off = up16(off + 2 * P);
   L.kg = off;
   off = up16(off + 2 * P);
-  if (with_values) {
-    L.vn = off;
-    off = up16(off + 2 * P);
-  }
   L.bytes = off;
   return L;
 }

@@ -54,6 +54,7 @@ struct Params {
   uint8_t* pool;
   long long pool_pages, page_bytes;
   int off_kc, off_qs, off_vc, off_kn, off_kg, off_vn;
+  int off_kl, blk;  // pages with values: key plane L, block bytes (block layout)
   const int32_t* page_table;
   int max_pages;
   const int32_t* cold_len;
@@ -198,9 +199,12 @@ __global__ void __launch_bounds__(NWARP * 32, 1) compress_kernel(Params p) {
       if (is_key) {
         const float T0 = __fmul_rn(n0, p.kt0), T1 = __fmul_rn(n1, p.kt0);
         const float inv0 = n0 > 0.0f ? 1.0f / n0 : 0.0f, inv1 = n1 > 0.0f ? 1.0f / n1 : 0.0f;
+        // record words (keys-only pages) or plane masks H | L (pages with
+        // values: word w < D/32 of H, word D/32 + w of L, bit j % 32)
         uint32_t kw0[D / 16], kw1[D / 16];
 #pragma unroll
         for (int w = 0; w < D / 16; ++w) kw0[w] = kw1[w] = 0u;
+        const bool planes = p.v != nullptr;
         float gg0 = 0.0f, gg1 = 0.0f;
 #pragma unroll
         for (int t = 0; t < C::NTL; ++t) {
@@ -216,9 +220,17 @@ __global__ void __launch_bounds__(NWARP * 32, 1) compress_kernel(Params p) {
             const float r = (nn > 0.0f) ? fmaf(x, inv, sg ? cpos : -cpos) : 0.0f;
             rr[e] = r;
             const int ei = e & 1;
-            const int sbit = 16 * (t & 1) + 15 - 4 * c - ei;
-            const uint32_t bits = ((nn > 0.0f ? sg : 0u) << sbit) | (mg << (sbit - 2));
-            if (row1) kw1[t >> 1] |= bits; else kw0[t >> 1] |= bits;
+            const uint32_t sgn = nn > 0.0f ? sg : 0u;
+            if (planes) {  // H = 1 - sign, L = sign XOR magnitude, bit j % 32
+              const int j = 8 * t + 2 * c + ei;
+              const uint32_t hb = (1u - sgn) << (j & 31), lb = (sgn ^ mg) << (j & 31);
+              if (row1) { kw1[j >> 5] |= hb; kw1[D / 32 + (j >> 5)] |= lb; }
+              else { kw0[j >> 5] |= hb; kw0[D / 32 + (j >> 5)] |= lb; }
+            } else {
+              const int sbit = 16 * (t & 1) + 15 - 4 * c - ei;
+              const uint32_t bits = (sgn << sbit) | (mg << (sbit - 2));
+              if (row1) kw1[t >> 1] |= bits; else kw0[t >> 1] |= bits;
+            }
             if (row1) gg1 = fmaf(r, r, gg1); else gg0 = fmaf(r, r, gg0);
           }
           // r as fp16 into this warp's rows of the tile (A operand of the sketch)
@@ -237,8 +249,15 @@ __global__ void __launch_bounds__(NWARP * 32, 1) compress_kernel(Params p) {
 #pragma unroll
         for (int w = 0; w < D / 16; ++w) {
           if (w / C::WPT == c) {
-            reinterpret_cast<uint32_t*>(stg + C::STG_KC + r0 * (D / 4))[w] = kw0[w];
-            reinterpret_cast<uint32_t*>(stg + C::STG_KC + r1 * (D / 4))[w] = kw1[w];
+            if (planes) {  // [128][D/32] H masks, then [128][D/32] L masks
+              const int pl = w / (D / 32), ww = w % (D / 32);
+              uint32_t* mk = reinterpret_cast<uint32_t*>(stg + C::STG_KC + pl * (ROWS * D / 8));
+              mk[r0 * (D / 32) + ww] = kw0[w];
+              mk[r1 * (D / 32) + ww] = kw1[w];
+            } else {
+              reinterpret_cast<uint32_t*>(stg + C::STG_KC + r0 * (D / 4))[w] = kw0[w];
+              reinterpret_cast<uint32_t*>(stg + C::STG_KC + r1 * (D / 4))[w] = kw1[w];
+            }
           }
         }
         gg0 += __shfl_xor_sync(0xffffffffu, gg0, 1);
@@ -282,7 +301,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1) compress_kernel(Params p) {
           for (int e = 0; e < 4; ++e) {
             const int ei = e & 1;
             const int within = 8 * (t & 3) + 2 * c + ei;  // index inside its 32-bit word
-            const int bit = 16 * (within >> 4) + 15 - (within & 15);
+            // pages with values: plane mask bit i % 32; keys-only: record bit
+            const int bit = planes ? within : 16 * (within >> 4) + 15 - (within & 15);
             const bool neg = (e < 2 ? n0 : n1) > 0.0f && pk[t][e] < 0.0f;
             if (neg) {
               if (e < 2) qw0[t >> 2] |= 1u << bit; else qw1[t >> 2] |= 1u << bit;
@@ -346,7 +366,16 @@ __global__ void __launch_bounds__(NWARP * 32, 1) compress_kernel(Params p) {
 
     // staging -> page, active slots [s_lo, s_hi) only
     uint8_t* pg = p.pool + static_cast<size_t>(page) * p.page_bytes;
-    {
+    if (p.v) {  // block layout
+      const uint32_t* mk = reinterpret_cast<const uint32_t*>(stg + C::STG_KC);
+      key_planes_out<D>(mk, mk + ROWS * D / 32, reinterpret_cast<const uint32_t*>(stg + C::STG_QS), pg,
+                        p.blk, p.off_kc, p.off_kl, p.off_qs, s_lo, s_hi, tid, blockDim.x);
+      norms_out(reinterpret_cast<const uint16_t*>(stg + C::STG_KN),
+                reinterpret_cast<const uint16_t*>(stg + C::STG_KG),
+                reinterpret_cast<const uint16_t*>(stg + C::STG_VN), pg, p.blk, p.off_kn, p.off_vn,
+                s_lo, s_hi, tid, blockDim.x);
+      vc_copy_out<D>(stg + C::STG_VC, pg, p.blk, p.off_vc, s_lo, s_hi, tid, blockDim.x);
+    } else {  // record layout
       constexpr int KC16 = D / 64;  // uint4 per key row
       for (int i = tid + s_lo * KC16; i < s_hi * KC16; i += blockDim.x)
         reinterpret_cast<uint4*>(pg + p.off_kc)[i] = reinterpret_cast<const uint4*>(stg + C::STG_KC)[i];
@@ -360,10 +389,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) compress_kernel(Params p) {
       for (int i = tid + s_lo; i < s_hi; i += blockDim.x) {
         reinterpret_cast<uint16_t*>(pg + p.off_kn)[i] = reinterpret_cast<const uint16_t*>(stg + C::STG_KN)[i];
         reinterpret_cast<uint16_t*>(pg + p.off_kg)[i] = reinterpret_cast<const uint16_t*>(stg + C::STG_KG)[i];
-        if (p.v)
-          reinterpret_cast<uint16_t*>(pg + p.off_vn)[i] = reinterpret_cast<const uint16_t*>(stg + C::STG_VN)[i];
       }
-      if (p.v) vc_copy_out<D>(stg + C::STG_VC, pg + p.off_vc, s_lo, s_hi, tid, blockDim.x);
     }
     __syncthreads();  // staging reused by the next tile
   }
@@ -413,6 +439,8 @@ int launch_compress(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dt
   p.off_kn = static_cast<int>(L.kn);
   p.off_kg = static_cast<int>(L.kg);
   p.off_vn = static_cast<int>(L.vn);
+  p.off_kl = static_cast<int>(L.kl);
+  p.blk = static_cast<int>(L.block);
   p.page_table = page_table;
   p.max_pages = max_pages;
   p.cold_len = cold_len;

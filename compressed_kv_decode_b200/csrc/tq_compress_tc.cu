@@ -76,7 +76,9 @@ struct Cfg {
   static constexpr int OFF_NV = OFF_NK + 1024;     // float[2][128] value norm^2 halves
   static constexpr int OFF_G = OFF_NV + 1024;      // float[2][128] residual norm^2 halves
   static constexpr int OFF_VS = OFF_G + 1024;      // value-code section staging (64 D bytes)
-  static constexpr int OFF_BAR = OFF_VS + D * 64;  // 5 mbarriers
+  static constexpr int OFF_KM = OFF_VS + D * 64;   // u32 [3][128][D/32] plane masks H, L, QJL
+  static constexpr int OFF_N16 = OFF_KM + 3 * ROWS * D / 8;  // fp16 bits [3][128]: n, gamma, n_v
+  static constexpr int OFF_BAR = OFF_N16 + 3 * ROWS * 2;     // 5 mbarriers
   static constexpr int OFF_TMEM = OFF_BAR + 64;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = (3 * D <= 256) ? 256 : 512;
@@ -89,6 +91,7 @@ struct Params {
   uint8_t* pool;
   long long pool_pages, page_bytes;
   int off_kc, off_qs, off_vc, off_kn, off_kg, off_vn;
+  int off_kl, blk;  // pages with values: key plane L, block bytes (block layout)
   const int32_t* page_table;
   int max_pages;
   const int32_t* cold_len;
@@ -258,7 +261,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     Tile nxt;
     const bool have_next = next_tile(p, tn, nxt);
     const bool page_ok = cur.page >= 0 && cur.page < p.pool_pages;
-    const bool active = row >= cur.s_lo && row < cur.s_hi;
 
     // ---- keys: rotation ------------------------------------------------
     if (!mbar_wait_bounded(bar_full0, par)) { failed = true; break; }
@@ -282,9 +284,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const float n = __half2float(nh);
     const float T0 = __fmul_rn(n, p.kt0);
     const float inv = n > 0.0f ? 1.0f / n : 0.0f;
-    uint32_t kw[C::HALF / 16];
+    // plane masks of this half row (block layout): H = 1 - sign, L = sign XOR
+    // magnitude; bit i % 32 of word i / 32 for column i of the half
+    uint32_t hm[C::HALF / 32], lm[C::HALF / 32];
 #pragma unroll
-    for (int w = 0; w < C::HALF / 16; ++w) kw[w] = 0u;
+    for (int w = 0; w < C::HALF / 32; ++w) hm[w] = lm[w] = 0u;
     float g2 = 0.0f;
 #pragma unroll
     for (int c8 = 0; c8 < C::HALF / 8; ++c8) {
@@ -302,10 +306,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const float r = fmaf(v, inv, neg ? cp : -cp);
           rr[e] = r;
           g2 = fmaf(r, r, g2);
-          const int jj = i & 15, hh = jj >> 3, ii = (jj & 7) >> 1, ee = jj & 1;  // halves are 16-aligned
-          const int sbit = 16 * hh + 15 - 4 * ii - ee;
-          if (neg) kw[i >> 4] |= 1u << sbit;
-          if (big) kw[i >> 4] |= 1u << (sbit - 2);
+          if (!neg) hm[i >> 5] |= 1u << (i & 31);
+          if (neg != big) lm[i >> 5] |= 1u << (i & 31);
         }
         const __half2 pr = __floats2half2_rn(n > 0.0f ? rr[0] : 0.0f, n > 0.0f ? rr[1] : 0.0f);
         rh[e2] = *reinterpret_cast<const uint32_t*>(&pr);
@@ -313,12 +315,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       *reinterpret_cast<uint4*>(smem + C::OFF_R + tc::sw128_offset(row, h * C::HALF + 8 * c8, ROWS)) =
           make_uint4(rh[0], rh[1], rh[2], rh[3]);
     }
-    if (!(n > 0.0f)) {  // zero vector: all codes and the residual norm are 0
+    if (!(n > 0.0f)) {  // zero vector: sign and magnitude 0 (H 1, L 0), residual norm 0
 #pragma unroll
-      for (int w = 0; w < C::HALF / 16; ++w) kw[w] = 0u;
+      for (int w = 0; w < C::HALF / 32; ++w) {
+        hm[w] = 0xFFFFFFFFu;
+        lm[w] = 0u;
+      }
       g2 = 0.0f;
     }
     gp[h * ROWS + row] = g2;
+    uint32_t* km = reinterpret_cast<uint32_t*>(smem + C::OFF_KM);
+    uint16_t* n16 = reinterpret_cast<uint16_t*>(smem + C::OFF_N16);
+#pragma unroll
+    for (int w = 0; w < C::HALF / 32; ++w) {
+      km[row * (D / 32) + h * (C::HALF / 32) + w] = hm[w];
+      km[(ROWS + row) * (D / 32) + h * (C::HALF / 32) + w] = lm[w];
+    }
     fence_proxy_async_smem();  // residual tile visible to the tensor cores
     tc::fence_before_sync();
     __syncthreads();
@@ -344,44 +356,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       nvp[h * ROWS + row] = half_row_sumsq<D, BF>(smem + C::OFF_X1, row, h);
     }
     uint8_t* pg = p.pool + static_cast<size_t>(page_ok ? cur.page : 0) * p.page_bytes;
-    const bool wr = page_ok && active;
-    if (wr) {
-      if constexpr (C::HALF / 16 == 4)
-        *reinterpret_cast<uint4*>(pg + p.off_kc + row * (D / 4) + h * (C::HALF / 4)) =
-            make_uint4(kw[0], kw[1], kw[2], kw[3]);
-      else
-        *reinterpret_cast<uint2*>(pg + p.off_kc + row * (D / 4) + h * (C::HALF / 4)) =
-            make_uint2(kw[0], kw[1]);
-    }
     if (!mbar_wait_bounded(bar_sk, par)) { failed = true; break; }
     tc::fence_after_sync();
     tmem_load_half<D>(t_lane + C::COL_SK + h * C::HALF, x);
     {
-      uint32_t qw[C::HALF / 32];
+      uint32_t qm[C::HALF / 32];  // QJL plane mask: bit i % 32 of word i / 32
 #pragma unroll
-      for (int w = 0; w < C::HALF / 32; ++w) qw[w] = 0u;
+      for (int w = 0; w < C::HALF / 32; ++w) qm[w] = 0u;
 #pragma unroll
-      for (int i = 0; i < C::HALF; ++i) {
-        const int within = i & 31;  // sketch index inside its 32-bit word
-        const int bit = 16 * (within >> 4) + 15 - (within & 15);
-        if (x[i] < 0.0f) qw[i >> 5] |= 1u << bit;
-      }
-      if (!(n > 0.0f)) {  // zero vector
+      for (int i = 0; i < C::HALF; ++i)
+        if (x[i] < 0.0f) qm[i >> 5] |= 1u << (i & 31);
 #pragma unroll
-        for (int w = 0; w < C::HALF / 32; ++w) qw[w] = 0u;
-      }
-      if (wr) {
-        if constexpr (C::HALF / 32 == 2)
-          *reinterpret_cast<uint2*>(pg + p.off_qs + row * (D / 8) + h * (C::HALF / 8)) =
-              make_uint2(qw[0], qw[1]);
-        else
-          *reinterpret_cast<uint32_t*>(pg + p.off_qs + row * (D / 8) + h * (C::HALF / 8)) = qw[0];
-      }
+      for (int w = 0; w < C::HALF / 32; ++w)
+        km[(2 * ROWS + row) * (D / 32) + h * (C::HALF / 32) + w] = (n > 0.0f) ? qm[w] : 0u;
     }
     __syncthreads();  // residual norm halves and value norm halves complete
-    if (wr && h == 0) {
-      reinterpret_cast<__half*>(pg + p.off_kn)[row] = nh;
-      reinterpret_cast<__half*>(pg + p.off_kg)[row] = __float2half_rn(sqrtf(gp[row] + gp[ROWS + row]));
+    if (h == 0) {
+      n16[row] = __half_as_ushort(nh);
+      n16[ROWS + row] = __half_as_ushort(__float2half_rn(sqrtf(gp[row] + gp[ROWS + row])));
     }
     // ---- values ------------------------------------------------------------
     if (p.has_v) {
@@ -429,9 +421,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           vs[vc_pos<D>(h * C::HALF + i, pr)] = static_cast<uint8_t>(lo | (hi << 4));
         }
       }
-      __syncthreads();
-      if (page_ok) vc_copy_out<D>(vs, pg + p.off_vc, cur.s_lo, cur.s_hi, tid, NTHREADS);
-      if (wr && h == 0) reinterpret_cast<__half*>(pg + p.off_vn)[row] = vh;
+      if (h == 0) reinterpret_cast<uint16_t*>(smem + C::OFF_N16)[2 * ROWS + row] = __half_as_ushort(vh);
+    }
+    __syncthreads();  // staged planes, norms and value codes complete
+    if (page_ok) {
+      const uint32_t* kmc = reinterpret_cast<const uint32_t*>(smem + C::OFF_KM);
+      const uint16_t* n16c = reinterpret_cast<const uint16_t*>(smem + C::OFF_N16);
+      key_planes_out<D>(kmc, kmc + ROWS * (D / 32), kmc + 2 * ROWS * (D / 32), pg, p.blk, p.off_kc,
+                        p.off_kl, p.off_qs, cur.s_lo, cur.s_hi, tid, NTHREADS);
+      norms_out(n16c, n16c + ROWS, p.has_v ? n16c + 2 * ROWS : nullptr, pg, p.blk, p.off_kn,
+                p.off_vn, cur.s_lo, cur.s_hi, tid, NTHREADS);
+      if (p.has_v) vc_copy_out<D>(smem + C::OFF_VS, pg, p.blk, p.off_vc, cur.s_lo, cur.s_hi, tid, NTHREADS);
     }
     if (threadIdx.x == 0 && !page_ok) report(p.err, TQ_ERR_CAPACITY);
     tc::fence_before_sync();
@@ -818,6 +818,8 @@ int launch_compress_tc(const tq_ctx* ctx, const void* k, const void* v, bool bf1
   p.off_kn = static_cast<int>(L.kn);
   p.off_kg = static_cast<int>(L.kg);
   p.off_vn = static_cast<int>(L.vn);
+  p.off_kl = static_cast<int>(L.kl);
+  p.blk = static_cast<int>(L.block);
   p.page_table = page_table;
   p.max_pages = max_pages;
   p.cold_len = cold_len;

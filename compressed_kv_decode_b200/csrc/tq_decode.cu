@@ -12,16 +12,19 @@
 //               one extra CTA builds the work schedule (units per segment,
 //               prefix sums, partial-record slots).
 //  2. attention persistent warps, each owning a contiguous range of work
-//               units (64 cold tokens or 16 hot tokens).  A warp streams its
-//               units through a private ring of shared-memory slots filled by
-//               1-D bulk copies (TMA) completing on mbarriers, unpacks the
-//               codes into fp16 tensor-core fragments in registers (the key
-//               code as one plane of +-b / +-a, a / b the fp16 ratio nearest
-//               kc1 / kc0, and the QJL signs as +-gamma), scores them with
-//               m16n8k16 MMAs (tokens on M, q heads x {hi, lo} on N),
-//               keeps an online softmax and accumulates P.V with MMAs (cold
-//               values in the rotated domain).  It writes one partial
-//               (m, l, o) per segment it touched.
+//               units (64 cold tokens = 4 page blocks, or 8 hot tokens).  A
+//               warp streams its units through a private ring of shared-memory
+//               slots, one 1-D bulk copy (TMA) per cold unit, completing on
+//               mbarriers.  Cold keys are scored with 8-bit integer MMAs
+//               (m16n8k32; tokens on M, q heads x {hi, lo} of 16-bit
+//               fixed-point query weights on N): the key planes H, L and the
+//               QJL plane hold 8 tokens per byte, so a lane's operand is its
+//               token's bit of every byte, one AND.  Values are dequantised
+//               through a lane-replicated byte -> fp16 pair table in shared
+//               memory straight into m16n8k16 A fragments.  The warp keeps an
+//               online softmax, accumulates P.V (cold values in the rotated
+//               domain) and writes one partial (m, l, o) per segment it
+//               touched.
 //  3. combine   per (batch, kv head): log-sum-exp merge of the cold partials,
 //               o_cold = Pi^T o_rot, merge with the hot partials, divide.
 #include <cuda_runtime.h>
@@ -36,30 +39,23 @@ namespace tq {
 namespace dec {
 
 constexpr int NW = 12;        // warps per attention CTA
-constexpr int COLD_TOK = 64;  // tokens per cold unit (half a page)
-constexpr int HOT_TOK = 16;   // tokens per hot unit
+constexpr int COLD_TOK = 64;  // tokens per cold unit (4 blocks, half a page)
+constexpr int HOT_TOK = 8;    // tokens per hot unit
 constexpr float NEG_INF = -__builtin_huge_valf();
 
 template <int D, int G>
 struct Cfg {
-  static constexpr int KS = D / 16;              // k-steps per key plane (and QJL, m = D)
+  static constexpr int KS = D / 16;              // k-steps of a hot key row, coordinate tiles of a value
   static constexpr int NT = (2 * G + 7) / 8;     // score n-tiles: G heads x {hi, lo}
   static constexpr int KK = D / 32;              // int8 k-steps per cold plane (m = D)
-  static constexpr int RC = 4 * KK * NT * 2;     // cold B-fragment registers per lane (planes s, m, sm, QJL)
+  static constexpr int RC = 3 * KK * NT * 2;     // cold B-fragment registers per lane (planes H, L, QJL)
   static constexpr int RH = KS * NT * 2;         // hot B-fragment registers per lane
-  static constexpr int WPT = D / 64;             // key code words per lane per token
-  static constexpr int WV = D / 32;              // value words per lane per token pair
-  static constexpr int KC_B = COLD_TOK * D / 4;  // bytes of one unit's sections
-  static constexpr int QS_B = COLD_TOK * D / 8;
-  static constexpr int VC_B = COLD_TOK / 2 * D;
-  static constexpr int OFF_QS = KC_B;
-  static constexpr int OFF_VC = OFF_QS + QS_B;
-  // the page's three norm sections (key, residual, value) are adjacent and
-  // staged whole with one copy
-  static constexpr int OFF_N = OFF_VC + VC_B;
-  static constexpr int NORM_B = 3 * 2 * TQ_PAGE_TOKENS;
-  static constexpr int COLD_B = OFF_N + NORM_B;
-  static constexpr int HROW = 2 * D + 16;  // padded hot row: conflict-free ldmatrix
+  // one 16-token block of a page with values (offsets as the page layout)
+  static constexpr int OFF_H = 0, OFF_L = 2 * D, OFF_Q = 4 * D, OFF_V = 6 * D;
+  static constexpr int OFF_NK = 14 * D, OFF_VN = 14 * D + 64;
+  static constexpr int BLK = 14 * D + 96;
+  static constexpr int COLD_B = 4 * BLK;          // one cold unit: 4 blocks, one copy
+  static constexpr int HROW = 2 * D + 16;         // padded hot row: conflict-free ldmatrix
   static constexpr int HOT_B = 2 * HOT_TOK * HROW;
   static constexpr int SLOT = ((COLD_B > HOT_B ? COLD_B : HOT_B) + 127) / 128 * 128;
   static constexpr int NSLOT = (D == 128) ? 2 : 3;
@@ -94,7 +90,7 @@ struct Params {
   const uint8_t* pool;
   long long pool_pages;
   long long page_bytes;
-  int off_kc, off_qs, off_vc, off_kn, off_kg, off_vn;
+  int blk;  // block bytes of a page with values (block layout)
   const int32_t* page_table;
   const int32_t* cold_len;
   float* out;
@@ -371,13 +367,14 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   __syncthreads();
   matvec_rows2<D, G>(mr, sq, sqr, sqs);  // q_rot = Pi q, q_s = (S Pi) q
   __syncthreads();
-  // Cold keys: four 0/1 operand planes -- sign s, magnitude m, s AND m, QJL
-  // sign b -- against 16-bit fixed-point query weights (int8 hi, lo):
-  //   <q_rot, c_hat> = c0 sum(q_rot) - 2 c0 <q_rot, s> + (c1 - c0) <q_rot, m>
-  //                    - 2 (c1 - c0) <q_rot, s m>
+  // Cold keys: three 0/1 operand planes against 16-bit fixed-point query
+  // weights (int8 hi, lo).  The key code is the index u = 2H + L of its level
+  // in ascending order (-c1, -c0, +c0, +c1), so the level is affine in the two
+  // bits and the QJL term is affine in the sign bits b:
+  //   <q_rot, c_hat> = -c1 sum(q_rot) + (c1 + c0) <q_rot, H> + (c1 - c0) <q_rot, L>
   //   <q_s, 1 - 2 b> = sum(q_s) - 2 <q_s, b>
-  // One fixed-point unit per head for the three key planes, one for the QJL plane.
-  const float ck0 = p.kc0, dk1 = p.kc1 - p.kc0;
+  // One fixed-point unit per head for the two key planes, one for the QJL plane.
+  const float wh = p.kc1 + p.kc0, wl = p.kc1 - p.kc0;
   __shared__ unsigned smr[G], sms[G];
   __shared__ float s_uk[G], s_uq[G];  // reciprocals of the fixed-point units
   if (tid < G) smr[tid] = sms[tid] = 0u;
@@ -415,13 +412,13 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
       }
       if (ln == 0) {
         const float mr = __uint_as_float(smr[wp]), ms = __uint_as_float(sms[wp]);
-        const float uk = mr > 0.0f ? 2.0f * fmaxf(ck0, dk1) * mr / FIX_MAX : 1.0f;
+        const float uk = mr > 0.0f ? wh * mr / FIX_MAX : 1.0f;
         const float uq = ms > 0.0f ? 2.0f * p.alpha * ms / FIX_MAX : 1.0f;
         s_uk[wp] = 1.0f / uk;
         s_uq[wp] = 1.0f / uq;
         float* ds = p.w.desc + static_cast<size_t>(bh) * DESC_N * 8;
         ds[DS_UK * 8 + wp] = p.sl * uk;
-        ds[DS_CK * 8 + wp] = p.sl * ck0 * a;
+        ds[DS_CK * 8 + wp] = -p.sl * p.kc1 * a;
         ds[DS_UQ * 8 + wp] = p.sl * uq;
         ds[DS_CQ * 8 + wp] = p.sl * p.alpha * b2;
         const float f = prescale_for(__uint_as_float(smax[1][wp]));
@@ -432,13 +429,10 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   }
   __syncthreads();
   // cold fragments (m16n8k32, B = [k][n], 4 int8 of k per register):
-  // r = ((plane * KK + kappa) * NT + nt) * 2 + reg, lane = 4 g' + c';
-  // k = 4 c' + j (reg 0) or 4 c' + 16 + j (reg 1) of k-step kappa reads, on the
-  // A side, bit position p of byte j of one of lane c''s packed words:
-  //   key planes: word c' WPT + (2 kappa + reg) / 4, sign position
-  //               p = {7, 6, 3, 2}[(2 kappa + reg) % 4] (magnitude: p - 2)
-  //   QJL plane:  word c' / LPW, p = (c' % LPW) 8 / LPW + 2 kappa + reg
-  constexpr int LPW = 4 / C::KK;  // lanes sharing one QJL word
+  // r = ((plane * KK + kappa) * NT + nt) * 2 + reg, lane = 4 g' + c'; register
+  // reg holds k = 4 c' + j + 16 reg (j = byte), index 32 kappa + k of the plane
+  // (coordinate, or sketch index for the QJL plane), column n = g' = head
+  // 4 nt + g' / 2, part g' % 2 (hi, lo).
   for (int idx = tid; idx < C::RC * 32; idx += blockDim.x) {
     const int r = idx >> 5, lane = idx & 31;
     const int reg = r & 1, nt = (r >> 1) % C::NT, pk = (r >> 1) / C::NT;
@@ -449,21 +443,10 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
     if (h < G) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float qv;
-        if (plane < 3) {
-          const int gam = 2 * kap + reg;
-          const int ps = (gam & 3) == 0 ? 7 : (gam & 3) == 1 ? 6 : (gam & 3) == 2 ? 3 : 2;
-          const int beta = 8 * j + ps, hh = beta >> 4, rem = 15 - (beta & 15);
-          const int coord = 16 * (cc * C::WPT + (gam >> 2)) + 8 * hh + 2 * (rem >> 2) + (rem & 1);
-          const float w = plane == 0 ? -2.0f * ck0 * sqr[h][coord]
-                        : plane == 1 ? dk1 * sqr[h][coord] : -2.0f * dk1 * sqr[h][coord];
-          qv = w * s_uk[h];
-        } else {
-          const int pq = (cc % LPW) * (8 / LPW) + 2 * kap + reg;
-          const int beta = 8 * j + pq, hh = beta >> 4, rr = 15 - (beta & 15);
-          const int si = 32 * (cc / LPW) + 16 * hh + rr;
-          qv = -2.0f * p.alpha * sqs[h][si] * s_uq[h];
-        }
+        const int k = 32 * kap + 4 * cc + j + 16 * reg;
+        const float qv = plane == 0 ? wh * sqr[h][k] * s_uk[h]
+                       : plane == 1 ? wl * sqr[h][k] * s_uk[h]
+                                    : -2.0f * p.alpha * sqs[h][k] * s_uq[h];
         const int q16 = max(-32511, min(32511, __float2int_rn(qv)));
         const int lo = ((q16 + 128) & 255) - 128, hi = (q16 - lo) >> 8;
         val |= static_cast<uint32_t>((part == 0 ? hi : lo) & 0xFF) << (8 * j);
@@ -631,35 +614,27 @@ __device__ __forceinline__ void issue_unit(const Params& p, int sg, int lu, int 
   const int bh = sg >> 1;
   const uint32_t d0 = smem_u32(dst);
   if ((sg & 1) == 0) {
+    // cold: blocks 4 (lu % 2) .. + 3 of the page, contiguous, one copy
     const bool ok = page >= 0 && page < p.pool_pages;
-    if (!ok) {
-      if (lane == 0) {
+    if (lane == 0) {
+      if (!ok) {
         report(p.err, TQ_ERR_CAPACITY);
         mbar_arrive_expect_tx(bar, 0);
+      } else {
+        mbar_arrive_expect_tx(bar, C::COLD_B);
+        bulk_g2s(d0, p.pool + static_cast<size_t>(page) * p.page_bytes + (lu & 1) * C::COLD_B,
+                 C::COLD_B, bar);
       }
-      __syncwarp();
-      return;
     }
-    const int half = lu & 1;
-    const uint8_t* base = p.pool + static_cast<size_t>(page) * p.page_bytes;
-    if (lane == 0) mbar_arrive_expect_tx(bar, C::COLD_B);
     __syncwarp();
-    // the four section copies go out as one instruction, one lane each
-    if (lane < 4) {
-      const uint32_t dst = d0 + (lane == 0 ? 0 : lane == 1 ? C::OFF_QS : lane == 2 ? C::OFF_VC : C::OFF_N);
-      const uint8_t* src = base + (lane == 0 ? p.off_kc + half * C::KC_B
-                                   : lane == 1 ? p.off_qs + half * C::QS_B
-                                   : lane == 2 ? p.off_vc + half * C::VC_B : p.off_kn);
-      const uint32_t bytes = lane == 0 ? C::KC_B : lane == 1 ? C::QS_B : lane == 2 ? C::VC_B : C::NORM_B;
-      bulk_g2s(dst, src, bytes, bar);
-    }
   } else {
+    // hot: K rows then V rows of HOT_TOK ring slots, one row per lane
     const int t0 = lu * HOT_TOK;
     const int rows = min(HOT_TOK, len - t0);
     if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * 2u * (2u * D));
     __syncwarp();
-    const int r = lane & 15, isv = lane >> 4;
-    if (r < rows) {
+    const int r = lane % HOT_TOK, isv = lane / HOT_TOK;
+    if (lane < 2 * HOT_TOK && r < rows) {
       int slot = t0 + r + hot_start_of(p, bh / p.Hkv);
       if (slot >= p.W_max) slot -= p.W_max;
       const __half* src = (isv ? p.v_hot : p.k_hot) +
@@ -679,39 +654,46 @@ __device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1,
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// bit position, inside each byte of a key code word, of the sign bits read by
-// group gam % 4 (the magnitude bits sit two below)
-__host__ __device__ constexpr int sign_pos(int gam) {
-  return (gam & 3) == 0 ? 7 : (gam & 3) == 1 ? 6 : (gam & 3) == 2 ? 3 : 2;
+// d += a * b, m16n8k8, fp16 inputs, fp32 accumulate
+__device__ __forceinline__ void mma_f16_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
 }
 
-// 8 value nibbles of a word (4 coordinates x 2 tokens) -> 4 half2 (token
-// even in the low half), through an fp16 table of the 8 magnitudes
-__device__ __forceinline__ void dequant_values(uint32_t x, uint32_t tl0, uint32_t tl1,
-                                               uint32_t th0, uint32_t th1, uint32_t (&h)[4]) {
-  const uint32_t x4 = x << 4;
-  // magnitude selectors (prmt reads the low 16 bits of its selector)
-  const uint32_t s01 = x & 0x77777777u;
-  const uint32_t s23 = s01 >> 16;
-  const uint32_t lo01 = prmt(tl0, tl1, s01), hi01 = prmt(th0, th1, s01);
-  const uint32_t lo23 = prmt(tl0, tl1, s23), hi23 = prmt(th0, th1, s23);
-  // sign bits of the 8 nibbles as 0x00 / 0xFF bytes (prmt sign replication)
-  const uint32_t m01 = prmt(x, x4, 0x9D8Cu), m23 = prmt(x, x4, 0xBFAEu);
-  const uint32_t hs01 = hi01 | (m01 & 0x80808080u), hs23 = hi23 | (m23 & 0x80808080u);
-  h[0] = prmt(lo01, hs01, 0x5140u);
-  h[1] = prmt(lo01, hs01, 0x7362u);
-  h[2] = prmt(lo23, hs23, 0x5140u);
-  h[3] = prmt(lo23, hs23, 0x7362u);
+__device__ __forceinline__ void ldsm_x1_t(uint32_t addr, uint32_t& r0) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x1.trans.shared.b16 {%0}, [%1];" : "=r"(r0) : "r"(addr));
+}
+
+// Value dequantisation table: entry e (a code byte: two 4-bit codes, the even
+// token's in the low nibble) = fp16 pair (v(e & 15), v(e >> 4)), v(code) =
+// (-1)^(code >> 3) fp16(c[code & 7]).  32 copies, copy L in bank L: lane L
+// reads entry e at byte 128 e + 4 L, so a warp's lookups never conflict.
+__shared__ uint32_t g_vlut[256 * 32];
+
+__device__ __forceinline__ uint32_t vlut(const char* lut, uint32_t off) {
+  return *reinterpret_cast<const uint32_t*>(lut + off);
 }
 
 template <int D, int G>
 __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
-  pdl_wait();  // schedule and query operands come from the prep launch
-  pdl_launch_dependents();
   using C = Cfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
+  // value table (before waiting on the prep launch: it needs only the codebook)
+  for (int i = threadIdx.x; i < 256 * 32; i += NW * 32) {
+    const int e = i >> 5;
+    const float v0 = ((e & 8) ? -1.0f : 1.0f) * p.vc[e & 7];
+    const float v1 = ((e & 128) ? -1.0f : 1.0f) * p.vc[(e >> 4) & 7];
+    const __half2 h2 = __floats2half2_rn(v0, v1);
+    g_vlut[i] = *reinterpret_cast<const uint32_t*>(&h2);
+  }
+  __syncthreads();
+  pdl_wait();  // schedule and query operands come from the prep launch
+  pdl_launch_dependents();
   uint8_t* slots = smem + warp * (C::NSLOT * C::SLOT);
   uint8_t* pbuf = smem + NW * C::NSLOT * C::SLOT + warp * C::PBUF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NW * (C::NSLOT * C::SLOT + C::PBUF)) +
@@ -745,20 +727,21 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
     if (uoff[mid] <= u0) lo = mid; else hi = mid - 1;
   }
   // issue cursor
-  int isg = lo, ilu = u0 - uoff[lo], iend = uoff[lo + 1];
+  int isg = lo, ilu = u0 - uoff[lo], iend = uoff[lo + 1], ilen = slen[lo];
   int iu = u0;
   // the next unit to stage: located (and its page looked up) one unit ahead
   // of its copy, so the page-table load overlaps a unit of compute
   int nx_sg = 0, nx_lu = 0, nx_len = 0, nx_page = -1;
   auto prep_next = [&]() {
-    while (iend <= iu) {  // segment ends are read once per segment
+    while (iend <= iu) {  // segment ends and lengths are read once per segment
       ++isg;
       ilu = 0;
       iend = uoff[isg + 1];
+      ilen = slen[isg];
     }
     nx_sg = isg;
     nx_lu = ilu;
-    nx_len = slen[isg];
+    nx_len = ilen;
     nx_page = ((isg & 1) == 0) ? p.page_table[static_cast<size_t>(isg >> 1) * p.max_pages + (ilu >> 1)] : 0;
   };
   auto fire_next = [&](int slot) {
@@ -773,27 +756,14 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
     fire_next(s);
   }
 
-  // value dequant tables: low and high bytes of fp16(val_c[k])
-  uint32_t tl0 = 0, tl1 = 0, th0 = 0, th1 = 0;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t hb = __half_as_ushort(__float2half_rn(p.vc[k]));
-    if (k < 4) {
-      tl0 |= (hb & 0xFFu) << (8 * k);
-      th0 |= (hb >> 8) << (8 * k);
-    } else {
-      tl1 |= (hb & 0xFFu) << (8 * (k - 4));
-      th1 |= (hb >> 8) << (8 * (k - 4));
-    }
-  }
-
   // consume cursor
-  int sg = lo, lu = u0 - uoff[lo], send = uoff[lo + 1];
-  uint32_t bfr[C::RC];
+  int sg = lo, lu = u0 - uoff[lo], send = uoff[lo + 1], len = slen[lo];
+  uint32_t bfr[C::RC > C::RH ? C::RC : C::RH];
   float dsc[C::NT];                                   // hot: descale
-  float uk[C::NT], ck[C::NT], uq[C::NT], cq[C::NT];  // cold: fixed-point units and constants
+  float uk[C::NT], ck[C::NT], uq[C::NT], cq[C::NT];  // cold: fixed-point units (row scale 2^-g folded in) and constants
   float mrun[C::NT], lrun[C::NT];
   float oacc[C::KS][4];
+  const float rowscale = 1.0f / static_cast<float>(1 << g);  // operand bytes are bit << g
   auto load_segment = [&]() {
     const int bh = sg >> 1, dom = sg & 1;
     if (dom == 0) {
@@ -811,20 +781,19 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
       const int h = c + 4 * nt;
       const bool in = h < G;
       dsc[nt] = in ? ds[DS_HOT * 8 + h] : 0.0f;
-      uk[nt] = in ? ds[DS_UK * 8 + h] : 0.0f;
+      uk[nt] = in ? ds[DS_UK * 8 + h] * rowscale : 0.0f;
       ck[nt] = in ? ds[DS_CK * 8 + h] : 0.0f;
-      uq[nt] = in ? ds[DS_UQ * 8 + h] : 0.0f;
+      uq[nt] = in ? ds[DS_UQ * 8 + h] * rowscale : 0.0f;
       cq[nt] = in ? ds[DS_CQ * 8 + h] : 0.0f;
       mrun[nt] = NEG_INF;
       lrun[nt] = 0.0f;
     }
-    (void)dom;
 #pragma unroll
     for (int i = 0; i < C::KS; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.0f;
   };
   load_segment();
 
-  // online-softmax update for scores sv (log2 domain); returns nothing, rescales oacc
+  // online-softmax update for scores sv (log2 domain); rescales oacc
   auto softmax_update = [&](float* sv, int count_per_nt) {
     float alpha[C::NT];
 #pragma unroll
@@ -874,7 +843,6 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
   };
 
   auto flush_segment = [&]() {
-    const int bh = sg >> 1, dom = sg & 1;
     float lt[C::NT];
 #pragma unroll
     for (int nt = 0; nt < C::NT; ++nt) {
@@ -906,11 +874,12 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         if (h < G) o[h * D + coord] = oacc[i][e];
       }
     }
-    (void)bh;
-    (void)dom;
   };
 
   const uint32_t pb_addr = smem_u32(pbuf);
+  const uint32_t msk = 0x01010101u << g;  // this lane's token in every plane byte
+  const uint32_t l4 = static_cast<uint32_t>(lane) * 4u;
+  const char* lut = reinterpret_cast<const char*>(g_vlut);
   for (int u = u0, k = 0; u < u1; ++u, ++k) {
     if (iu < u1) prep_next();
     const int slot = k % C::NSLOT;
@@ -923,82 +892,61 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         mbar_wait_bounded(smem_u32(&bars[s]), static_cast<uint32_t>((k + s) / C::NSLOT) & 1u);
       return;
     }
-    const int bh = sg >> 1;
-    const int len = slen[sg];
     if ((sg & 1) == 0) {
-      // ---------------- cold unit: 64 tokens ----------------
+      // ---------------- cold unit: 64 tokens, 4 blocks ----------------
       const int page = slot_page[slot];
       const int nv = (page >= 0 && page < p.pool_pages) ? min(COLD_TOK, len - lu * COLD_TOK) : 0;
       float sv[C::NT * 8];
-      const int hoff = (lu & 1) * 2 * COLD_TOK;  // this half page's first norm
-      const __half* kn = reinterpret_cast<const __half*>(sb + C::OFF_N + hoff);
-      const uint16_t* kg = reinterpret_cast<const uint16_t*>(sb + C::OFF_N + 2 * TQ_PAGE_TOKENS + hoff);
-      const __half* vn = reinterpret_cast<const __half*>(sb + C::OFF_N + 4 * TQ_PAGE_TOKENS + hoff);
-      // lane c's QJL word and the first bit position it reads in each byte
-      constexpr int LPW = 4 / C::KK;
-      const int qword = c / LPW, qbase = (c % LPW) * (8 / LPW);
-      constexpr uint32_t M8 = 0x01010101u;
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
-        const int t0 = 16 * mt + g, t1 = t0 + 8;
-        uint32_t kw0[C::WPT], kw1[C::WPT];
-#pragma unroll
-        for (int w = 0; w < C::WPT; ++w) {
-          kw0[w] = *reinterpret_cast<const uint32_t*>(sb + t0 * (D / 4) + 4 * (c * C::WPT + w));
-          kw1[w] = *reinterpret_cast<const uint32_t*>(sb + t1 * (D / 4) + 4 * (c * C::WPT + w));
-        }
-        const uint32_t qw0 = *reinterpret_cast<const uint32_t*>(sb + C::OFF_QS + t0 * (D / 8) + 4 * qword);
-        const uint32_t qw1 = *reinterpret_cast<const uint32_t*>(sb + C::OFF_QS + t1 * (D / 8) + 4 * qword);
-        // integer accumulators: key planes (s, m, s m) and the QJL plane
-        int dk[C::NT][4], dq[C::NT][4];
+        const uint8_t* bp = sb + mt * C::BLK;
+        // integer accumulators: planes H, L (key) and QJL, split in independent chains
+        int ah[C::NT][4], al[C::NT][4], aq0[C::NT][4], aq1[C::NT][4];
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dk[nt][e] = dq[nt][e] = 0;
+          for (int e = 0; e < 4; ++e) ah[nt][e] = al[nt][e] = aq0[nt][e] = aq1[nt][e] = 0;
 #pragma unroll
         for (int kap = 0; kap < C::KK; ++kap) {
-          // A operands: bit p of every byte of a code word, as 0/1 bytes
-          const int ga = 2 * kap, gb = 2 * kap + 1;
-          const int pa = sign_pos(ga), pb = sign_pos(gb);
-          const uint32_t xa0 = kw0[ga >> 2] >> pa, xa1 = kw1[ga >> 2] >> pa;
-          const uint32_t xb0 = kw0[gb >> 2] >> pb, xb1 = kw1[gb >> 2] >> pb;
-          const uint32_t ya0 = kw0[ga >> 2] >> (pa - 2), ya1 = kw1[ga >> 2] >> (pa - 2);
-          const uint32_t yb0 = kw0[gb >> 2] >> (pb - 2), yb1 = kw1[gb >> 2] >> (pb - 2);
+          // words for indices 32 kap + 4c .. (tokens 0-7, 8-15) and 32 kap + 16 + 4c ..
+          const uint4 wh = *reinterpret_cast<const uint4*>(bp + C::OFF_H + (kap * 4 + c) * 16);
+          const uint4 wl = *reinterpret_cast<const uint4*>(bp + C::OFF_L + (kap * 4 + c) * 16);
+          const uint4 wq = *reinterpret_cast<const uint4*>(bp + C::OFF_Q + (kap * 4 + c) * 16);
 #pragma unroll
           for (int nt = 0; nt < C::NT; ++nt) {
-            const uint32_t* bs = bfr + ((0 * C::KK + kap) * C::NT + nt) * 2;
-            const uint32_t* bm = bfr + ((1 * C::KK + kap) * C::NT + nt) * 2;
-            const uint32_t* bsm = bfr + ((2 * C::KK + kap) * C::NT + nt) * 2;
-            imma_u8s8(dk[nt], xa0 & M8, xa1 & M8, xb0 & M8, xb1 & M8, bs[0], bs[1]);
-            imma_u8s8(dk[nt], ya0 & M8, ya1 & M8, yb0 & M8, yb1 & M8, bm[0], bm[1]);
-            imma_u8s8(dk[nt], xa0 & ya0 & M8, xa1 & ya1 & M8, xb0 & yb0 & M8, xb1 & yb1 & M8, bsm[0],
-                      bsm[1]);
+            const uint32_t* bH = bfr + ((0 * C::KK + kap) * C::NT + nt) * 2;
+            const uint32_t* bL = bfr + ((1 * C::KK + kap) * C::NT + nt) * 2;
+            const uint32_t* bQ = bfr + ((2 * C::KK + kap) * C::NT + nt) * 2;
+            imma_u8s8(ah[nt], wh.x & msk, wh.y & msk, wh.z & msk, wh.w & msk, bH[0], bH[1]);
+            imma_u8s8(al[nt], wl.x & msk, wl.y & msk, wl.z & msk, wl.w & msk, bL[0], bL[1]);
+            if (kap & 1)
+              imma_u8s8(aq1[nt], wq.x & msk, wq.y & msk, wq.z & msk, wq.w & msk, bQ[0], bQ[1]);
+            else
+              imma_u8s8(aq0[nt], wq.x & msk, wq.y & msk, wq.z & msk, wq.w & msk, bQ[0], bQ[1]);
           }
         }
-#pragma unroll
-        for (int kap = 0; kap < C::KK; ++kap) {
-          const int pq = qbase + 2 * kap;
-          const uint32_t q0 = (qw0 >> pq) & M8, q1 = (qw1 >> pq) & M8;
-          const uint32_t q2 = (qw0 >> (pq + 1)) & M8, q3 = (qw1 >> (pq + 1)) & M8;
-#pragma unroll
-          for (int nt = 0; nt < C::NT; ++nt) {
-            const uint32_t* bq = bfr + ((3 * C::KK + kap) * C::NT + nt) * 2;
-            imma_u8s8(dq[nt], q0, q1, q2, q3, bq[0], bq[1]);
-          }
-        }
-        const float n0 = __half2float(kn[t0]), n1 = __half2float(kn[t1]);
-        const float gm0 = __half2float(__ushort_as_half(kg[t0])), gm1 = __half2float(__ushort_as_half(kg[t1]));
+        // (n, gamma) of tokens g and g + 8 of the block
+        const uint32_t nk0 = *reinterpret_cast<const uint32_t*>(bp + C::OFF_NK + 4 * g);
+        const uint32_t nk1 = *reinterpret_cast<const uint32_t*>(bp + C::OFF_NK + 4 * (g + 8));
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&nk0));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&nk1));
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt) {
           // columns 2c, 2c+1: the hi and lo bytes of head c's weights
-          const float vk0 = static_cast<float>(dk[nt][0] * 256 + dk[nt][1]);
-          const float vk1 = static_cast<float>(dk[nt][2] * 256 + dk[nt][3]);
-          const float vq0 = static_cast<float>(dq[nt][0] * 256 + dq[nt][1]);
-          const float vq1 = static_cast<float>(dq[nt][2] * 256 + dq[nt][3]);
-          const float v0 = fmaf(gm0, fmaf(uq[nt], vq0, cq[nt]), fmaf(uk[nt], vk0, ck[nt])) * n0;
-          const float v1 = fmaf(gm1, fmaf(uq[nt], vq1, cq[nt]), fmaf(uk[nt], vk1, ck[nt])) * n1;
-          sv[nt * 8 + 2 * mt] = (t0 < nv) ? v0 : NEG_INF;
-          sv[nt * 8 + 2 * mt + 1] = (t1 < nv) ? v1 : NEG_INF;
+          const float vk0 = static_cast<float>((ah[nt][0] + al[nt][0]) * 256 + ah[nt][1] + al[nt][1]);
+          const float vk1 = static_cast<float>((ah[nt][2] + al[nt][2]) * 256 + ah[nt][3] + al[nt][3]);
+          const float vq0 = static_cast<float>((aq0[nt][0] + aq1[nt][0]) * 256 + aq0[nt][1] + aq1[nt][1]);
+          const float vq1 = static_cast<float>((aq0[nt][2] + aq1[nt][2]) * 256 + aq0[nt][3] + aq1[nt][3]);
+          sv[nt * 8 + 2 * mt] = fmaf(f0.y, fmaf(uq[nt], vq0, cq[nt]), fmaf(uk[nt], vk0, ck[nt])) * f0.x;
+          sv[nt * 8 + 2 * mt + 1] = fmaf(f1.y, fmaf(uq[nt], vq1, cq[nt]), fmaf(uk[nt], vk1, ck[nt])) * f1.x;
+        }
+        if (nv < COLD_TOK) {  // tokens past the sequence
+          const int t0 = 16 * mt + g;
+#pragma unroll
+          for (int nt = 0; nt < C::NT; ++nt) {
+            if (t0 >= nv) sv[nt * 8 + 2 * mt] = NEG_INF;
+            if (t0 + 8 >= nv) sv[nt * 8 + 2 * mt + 1] = NEG_INF;
+          }
         }
       }
       softmax_update(sv, 8);
@@ -1006,27 +954,31 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
         const int t0 = 16 * mt + g, t1 = t0 + 8;
-        const float nv0 = __half2float(vn[t0]), nv1 = __half2float(vn[t1]);
+        const __half* vn = reinterpret_cast<const __half*>(sb + mt * C::BLK + C::OFF_VN);
+        const float nv0 = __half2float(vn[g]), nv1 = __half2float(vn[g + 8]);
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt) {
           const int h = c + 4 * nt;
           if (h < G) {
-            const float p0 = (t0 < nv) ? sv[nt * 8 + 2 * mt] * nv0 : 0.0f;
-            const float p1 = (t1 < nv) ? sv[nt * 8 + 2 * mt + 1] * nv1 : 0.0f;
+            float p0 = sv[nt * 8 + 2 * mt] * nv0, p1 = sv[nt * 8 + 2 * mt + 1] * nv1;
+            if (nv < COLD_TOK) {
+              if (t0 >= nv) p0 = 0.0f;
+              if (t1 >= nv) p1 = 0.0f;
+            }
             reinterpret_cast<__half*>(pbuf)[t0 * 8 + h] = __float2half_rn(p0);
             reinterpret_cast<__half*>(pbuf)[t1 * 8 + h] = __float2half_rn(p1);
           }
         }
       }
       __syncwarp();
-      // value codes: the lane's word for coordinate tile i of a 16-token
-      // block dequantises to its A fragment (coordinates x tokens)
-      const uint8_t* vc = sb + C::OFF_VC;
+      // value codes: the lane's word for coordinate tile i of a block
+      // dequantises, byte by byte through the table, to its A fragment
+      // (coordinates x tokens)
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
         uint32_t bp0, bp1;
         ldsm_x2_t(pb_addr + (16 * mt + (lane & 15)) * 16, bp0, bp1);
-        const uint8_t* vb = vc + mt * (8 * D) + lane * 16;
+        const uint8_t* vb = sb + mt * C::BLK + C::OFF_V + lane * 16;
         uint32_t xw[C::KS];
 #pragma unroll
         for (int q4 = 0; q4 < C::KS / 4; ++q4) {
@@ -1035,13 +987,16 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         }
 #pragma unroll
         for (int i = 0; i < C::KS; ++i) {
-          uint32_t h[4];
-          dequant_values(xw[i], tl0, tl1, th0, th1, h);
-          mma_f16(oacc[i], h[0], h[1], h[2], h[3], bp0, bp1);
+          const uint32_t x = xw[i];
+          const uint32_t a0 = vlut(lut, ((x << 7) & 0x7F80u) | l4);
+          const uint32_t a1 = vlut(lut, ((x >> 1) & 0x7F80u) | l4);
+          const uint32_t a2 = vlut(lut, ((x >> 9) & 0x7F80u) | l4);
+          const uint32_t a3 = vlut(lut, ((x >> 17) & 0x7F80u) | l4);
+          mma_f16(oacc[i], a0, a1, a2, a3, bp0, bp1);
         }
       }
     } else {
-      // ---------------- hot unit: 16 tokens ----------------
+      // ---------------- hot unit: 8 tokens ----------------
       const int nv = min(HOT_TOK, len - lu * HOT_TOK);
       const uint8_t* kt = sb;
       uint8_t* vt = sb + HOT_TOK * C::HROW;
@@ -1050,6 +1005,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
           reinterpret_cast<uint32_t*>(vt + nv * C::HROW)[i] = 0u;
         __syncwarp();
       }
+      // scores: tokens on M (rows 8-15 read the V tile and are masked)
       float acc[C::NT][4];
 #pragma unroll
       for (int nt = 0; nt < C::NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
@@ -1064,33 +1020,25 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         for (int nt = 0; nt < C::NT; ++nt)
           mma_f16(acc[nt], a0, a1, a2, a3, bfr[(s * C::NT + nt) * 2], bfr[(s * C::NT + nt) * 2 + 1]);
       }
-      float sv[C::NT * 2];
+      float sv[C::NT];
 #pragma unroll
-      for (int nt = 0; nt < C::NT; ++nt) {
-        sv[nt * 2] = (g < nv) ? (acc[nt][0] + acc[nt][1]) * dsc[nt] : NEG_INF;
-        sv[nt * 2 + 1] = (g + 8 < nv) ? (acc[nt][2] + acc[nt][3]) * dsc[nt] : NEG_INF;
-      }
-      softmax_update(sv, 2);
+      for (int nt = 0; nt < C::NT; ++nt) sv[nt] = (g < nv) ? (acc[nt][0] + acc[nt][1]) * dsc[nt] : NEG_INF;
+      softmax_update(sv, 1);
 #pragma unroll
       for (int nt = 0; nt < C::NT; ++nt) {
         const int h = c + 4 * nt;
-        if (h < G) {
-          reinterpret_cast<__half*>(pbuf)[g * 8 + h] = __float2half_rn(sv[nt * 2]);
-          reinterpret_cast<__half*>(pbuf)[(g + 8) * 8 + h] = __float2half_rn(sv[nt * 2 + 1]);
-        }
+        if (h < G) reinterpret_cast<__half*>(pbuf)[g * 8 + h] = __float2half_rn(sv[nt]);
       }
       __syncwarp();
-      uint32_t bp0, bp1;
-      ldsm_x2_t(pb_addr + (lane & 15) * 16, bp0, bp1);
+      uint32_t bp0;
+      ldsm_x1_t(pb_addr + (lane & 7) * 16, bp0);
       const uint32_t vt_addr = smem_u32(vt);
 #pragma unroll
       for (int i = 0; i < C::KS; ++i) {
-        const int mi = lane >> 3;
-        const int tok = (lane & 7) + (mi >> 1) * 8;
-        const int col = 16 * i + (mi & 1) * 8;
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(vt_addr + tok * C::HROW + col * 2, a0, a1, a2, a3);
-        mma_f16(oacc[i], a0, a1, a2, a3, bp0, bp1);
+        const int col = 16 * i + ((lane >> 3) & 1) * 8;
+        uint32_t a0, a1;
+        ldsm_x2_t(vt_addr + (lane & 7) * C::HROW + col * 2, a0, a1);
+        mma_f16_k8(oacc[i], a0, a1, bp0);
       }
     }
     // all lanes are done with this slot (every value read from it has been
@@ -1104,6 +1052,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         ++sg;
         while (uoff[sg + 1] <= u + 1) ++sg;
         send = uoff[sg + 1];
+        len = slen[sg];
         lu = 0;
         load_segment();
       }
@@ -1346,8 +1295,7 @@ WsLayout ws_layout(int B, int Hkv, int Wtot, int W_max) {
 template <int D, int G>
 int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st) {
   using C = Cfg<D, G>;
-  if (p.off_kg != p.off_kn + 2 * TQ_PAGE_TOKENS || p.off_vn != p.off_kg + 2 * TQ_PAGE_TOKENS)
-    return TQ_ERR_UNSUPPORTED;  // norm sections staged with one copy
+  if (p.blk != C::BLK || p.page_bytes != 8LL * C::BLK) return TQ_ERR_UNSUPPORTED;  // block layout
   const int grid = ctx->num_sms;
   p.Wtot = grid * NW;
   p.S = 2 * p.B * p.Hkv;
@@ -1469,12 +1417,7 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
   p.pool = pool;
   p.pool_pages = pool_pages;
   p.page_bytes = static_cast<long long>(L.bytes);
-  p.off_kc = static_cast<int>(L.kc);
-  p.off_qs = static_cast<int>(L.qs);
-  p.off_vc = static_cast<int>(L.vc);
-  p.off_kn = static_cast<int>(L.kn);
-  p.off_kg = static_cast<int>(L.kg);
-  p.off_vn = static_cast<int>(L.vn);
+  p.blk = static_cast<int>(L.block);
   p.page_table = page_table;
   p.cold_len = cold_len;
   p.out = out;

@@ -172,12 +172,29 @@ __device__ __forceinline__ float load_as_float(const void* p, size_t i, tq_dtype
 
 namespace tq {
 
-// Value-code section of a page: token pair p (slots 2p, 2p+1) of coordinate j
-// is one byte (even slot in the low nibble).  Blocks of 16 tokens (kb) by
-// tiles of 16 coordinates (i): the 32-bit word of lane 4g + c at
-// kb*8D + (i/4)*512 + (4g + c)*16 + (i%4)*4 holds coordinates (g, g+8) x
-// token pairs (c, c+4) of the block -- one m16n8k16 A fragment (rows =
-// coordinates, k = tokens) after dequantisation.
+// ---------------------------------------------------------------------------
+// Pages with values: 8 blocks of 16 token slots.  A block holds the key
+// planes H and L (the key code is the index u = 2H + L of its level in
+// ascending order), the QJL sign plane, the value codes, the (n, gamma) fp16
+// pairs and the value norms; PageLayout gives the offsets inside a block.
+// ---------------------------------------------------------------------------
+
+// Byte, inside a block's plane, of plane index j (coordinate or sketch index)
+// for token t (0..15); the bit is t % 8.  A 32-bit word holds 4 consecutive
+// indices x 8 tokens; word w = 16 (j / 32) + 4 ((j / 4) % 4) + 2 ((j / 16) % 2)
+// + t / 8, so that the four words a lane reads for indices 32k + 4c .. + 3 and
+// 32k + 16 + 4c .. + 3 are adjacent.
+__host__ __device__ __forceinline__ int plane_byte(int j, int t) {
+  return 16 * (4 * (j >> 5) + ((j >> 2) & 3)) + 4 * (2 * ((j >> 4) & 1) + (t >> 3)) + (j & 3);
+}
+
+// Value-code section of a block: token pair p (tokens 2p, 2p+1 of the block)
+// of coordinate j is one byte (even token in the low nibble).  Tiles of 16
+// coordinates (i): the 32-bit word of lane 4g + c at (i/4)*512 + (4g + c)*16 +
+// (i%4)*4 holds coordinates (g, g+8) x token pairs (c, c+4) -- one m16n8k16 A
+// fragment (rows = coordinates, k = tokens) after dequantisation.  A staged
+// page image holds the 8 blocks' sections back to back (vc_pos with the pair
+// index of the page).
 template <int D>
 __host__ __device__ __forceinline__ int vc_pos(int j, int p) {
   const int kb = p >> 3, q = p & 7, c = q & 3, th = q >> 2;
@@ -185,30 +202,90 @@ __host__ __device__ __forceinline__ int vc_pos(int j, int p) {
   return kb * (8 * D) + (i >> 2) * 512 + (4 * g + c) * 16 + (i & 3) * 4 + jh + 2 * th;
 }
 
-// Copy a value-code section staged in shared memory (same layout as the
-// page) to the page, for the active token slots [s_lo, s_hi): 16-byte copies
-// when the whole page is written, else byte copies that keep the nibble of a
-// pair's slot outside the range.
+// Write the key planes H, L and the QJL plane (m = D) of the active slots
+// [s_lo, s_hi) of a page with values, from per-slot masks staged in shared
+// memory: mask[s * (D/32) + j/32] bit j % 32 is the plane bit of index j for
+// slot s.  One 32-bit word (4 indices x 8 tokens) per thread and step; in a
+// word with inactive tokens those tokens' bits keep their stored values.
 template <int D>
-__device__ __forceinline__ void vc_copy_out(const uint8_t* stg, uint8_t* dst, int s_lo, int s_hi,
-                                            int tid, int nthr) {
-  if (s_lo == 0 && s_hi == 128) {
-    for (int i = tid; i < D * 4; i += nthr)
-      reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(stg)[i];
-    return;
-  }
-  const int p_lo = s_lo >> 1, p_hi = (s_hi + 1) >> 1, np = p_hi - p_lo;
-  for (int i = tid; i < D * np; i += nthr) {
-    const int j = i / np, p = p_lo + i % np;
-    const int off = vc_pos<D>(j, p);
-    uint8_t b = stg[off];
-    const bool ev = 2 * p >= s_lo && 2 * p < s_hi;
-    const bool od = 2 * p + 1 >= s_lo && 2 * p + 1 < s_hi;
-    if (!(ev && od)) {
-      const uint8_t keep = ev ? 0xF0 : 0x0F;
-      b = static_cast<uint8_t>((dst[off] & keep) | (b & ~keep));
+__device__ __forceinline__ void key_planes_out(const uint32_t* mh, const uint32_t* ml,
+                                               const uint32_t* mq, uint8_t* pg, int blk,
+                                               int off_h, int off_l, int off_q, int s_lo,
+                                               int s_hi, int tid, int nthr) {
+  constexpr int WPB = D / 2;  // words per plane and block: D indices x 16 tokens / 32
+  const int b_lo = s_lo >> 4, b_hi = (s_hi + 15) >> 4;
+  const int n = (b_hi - b_lo) * 3 * WPB;
+  for (int i = tid; i < n; i += nthr) {
+    const int w = i % WPB, pl = (i / WPB) % 3, kb = b_lo + i / (3 * WPB);
+    const int kap = w >> 4, c = (w >> 2) & 3, r = w & 3;
+    const int s0 = 16 * kb + 8 * (r & 1);      // first slot of the word's 8 tokens
+    const int shift = 16 * (r >> 1) + 4 * c;   // bit of its first index in the mask word
+    const uint32_t* src = pl == 0 ? mh : pl == 1 ? ml : mq;
+    uint32_t out = 0u, act = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int s = s0 + k;
+      const uint32_t nib = (src[s * (D / 32) + kap] >> shift) & 0xFu;
+      out |= ((nib * 0x00204081u) & 0x01010101u) << k;  // bit jj of nib -> bit 8 jj
+      if (s >= s_lo && s < s_hi) act |= 1u << k;
     }
-    dst[off] = b;
+    if (act == 0u) continue;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(pg + kb * blk + (pl == 0 ? off_h : pl == 1 ? off_l : off_q) + 4 * w);
+    if (act != 0xFFu) {
+      const uint32_t m = act * 0x01010101u;
+      out = (*dst & ~m) | (out & m);
+    }
+    *dst = out;
+  }
+}
+
+// Norm fields of the active slots of a page with values: (n, gamma) pairs
+// and (if vn) the value norms, from per-slot fp16 bits staged in shared memory.
+__device__ __forceinline__ void norms_out(const uint16_t* kn, const uint16_t* kg,
+                                          const uint16_t* vn, uint8_t* pg, int blk, int off_kn,
+                                          int off_vn, int s_lo, int s_hi, int tid, int nthr) {
+  for (int s = s_lo + tid; s < s_hi; s += nthr) {
+    uint8_t* bk = pg + (s >> 4) * blk;
+    const int t = s & 15;
+    *reinterpret_cast<uint32_t*>(bk + off_kn + 4 * t) =
+        static_cast<uint32_t>(kn[s]) | (static_cast<uint32_t>(kg[s]) << 16);
+    if (vn) *reinterpret_cast<uint16_t*>(bk + off_vn + 2 * t) = vn[s];
+  }
+}
+
+// Copy a staged value-code image (8 blocks of 8 D bytes, vc_pos layout) to the
+// blocks of a page, for the active slots [s_lo, s_hi): 16-byte copies of the
+// blocks wholly inside the range, byte copies (keeping the nibble of a pair's
+// token outside the range) elsewhere.
+template <int D>
+__device__ __forceinline__ void vc_copy_out(const uint8_t* stg, uint8_t* pg, int blk, int off_vc,
+                                            int s_lo, int s_hi, int tid, int nthr) {
+  constexpr int BV = 8 * D;  // value bytes per block
+  const int f_lo = (s_lo + 15) >> 4, f_hi = s_hi >> 4;  // whole blocks [f_lo, f_hi)
+  for (int i = tid; i < (f_hi - f_lo) * (BV / 16); i += nthr) {
+    const int kb = f_lo + i / (BV / 16), k = i % (BV / 16);
+    reinterpret_cast<uint4*>(pg + kb * blk + off_vc)[k] = reinterpret_cast<const uint4*>(stg + kb * BV)[k];
+  }
+  // the partial blocks at either end
+  for (int e = 0; e < 2; ++e) {
+    const int kb = e == 0 ? (s_lo >> 4) : ((s_hi - 1) >> 4);
+    if (kb >= f_lo && kb < f_hi) continue;
+    if (e == 1 && kb == (s_lo >> 4)) continue;  // one partial block only
+    const int a = max(s_lo, 16 * kb), z = min(s_hi, 16 * kb + 16);
+    const int p_lo = a >> 1, p_hi = (z + 1) >> 1, np = p_hi - p_lo;
+    for (int i = tid; i < D * np; i += nthr) {
+      const int j = i / np, p = p_lo + i % np;
+      const int off = vc_pos<D>(j, p);
+      uint8_t* dst = pg + kb * blk + off_vc + (off - kb * BV);
+      uint8_t b = stg[off];
+      const bool ev = 2 * p >= s_lo && 2 * p < s_hi;
+      const bool od = 2 * p + 1 >= s_lo && 2 * p + 1 < s_hi;
+      if (!(ev && od)) {
+        const uint8_t keep = ev ? 0xF0 : 0x0F;
+        b = static_cast<uint8_t>((*dst & keep) | (b & ~keep));
+      }
+      *dst = b;
+    }
   }
 }
 

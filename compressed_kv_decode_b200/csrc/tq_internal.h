@@ -91,9 +91,13 @@ struct tq_ctx {
 
 namespace tq {
 
-// Page layout (bytes) for head dim d, sketch dim m.
+// Page layout (bytes) for head dim d, sketch dim m.  Keys-only pages (record
+// layout): section offsets kc, qs, kn, kg; block = 0.  Pages with values
+// (block layout, 8 blocks of 16 token slots): offsets inside a block -- kc (key
+// plane H), kl (key plane L), qs, vc, kn (the (n, gamma) pair of token 0), vn
+// (value norm of token 0) -- and the block size.
 struct PageLayout {
-  size_t kc, qs, vc, kn, kg, vn, bytes;
+  size_t kc, kl, qs, vc, kn, kg, vn, block, bytes;
 };
 PageLayout page_layout(int d, int m, bool with_values);
 

@@ -101,15 +101,19 @@ def random_page_table(seed, B, Hkv, max_pages, spare=0):
     return perm.astype(np.int32).reshape(B, Hkv, max_pages), n + spare
 
 
-def random_page_bytes(seed, n_pages, page_bytes, norm_offsets):
+def random_page_bytes(seed, n_pages, page_bytes, norm_slots):
     """Random bytes for pages whose content does not matter, with every fp16
-    norm field set to a finite value in [2, 14) (gamma in [0, 0.5))."""
+    norm field set to a finite value in [2, 14) (gamma in [0, 0.5)).
+    norm_slots: field name (kn, kg, vn) -> byte offsets of the 128 token
+    slots' fp16 fields inside a page."""
     rng = np.random.default_rng(seed)
     pool = rng.integers(0, 256, size=(n_pages, page_bytes), dtype=np.uint8)
     for name, lo, hi in (("kn", 2.0, 14.0), ("kg", 0.0, 0.5), ("vn", 2.0, 14.0)):
-        off = norm_offsets.get(name)
-        if off is None:
+        offs = norm_slots.get(name)
+        if offs is None:
             continue
-        vals = rng.uniform(lo, hi, size=(n_pages, 128)).astype(np.float16)
-        pool[:, off:off + 256] = vals.view(np.uint8).reshape(n_pages, 256)
+        offs = np.asarray(offs, np.int64)
+        vals = rng.uniform(lo, hi, size=(n_pages, len(offs))).astype(np.float16).view(np.uint8)
+        pool[:, offs] = vals[:, 0::2]
+        pool[:, offs + 1] = vals[:, 1::2]
     return pool

@@ -197,9 +197,26 @@ PAGE_TOKENS = 128
 
 
 def page_layout(d, m, with_values=True):
-    offs = (C.c_size_t * 6)()
+    """(page bytes, offsets).  Keys-only pages (record layout): section offsets
+    kc, qs, kn, kg and block = 0.  Pages with values (block layout): offsets
+    inside a 16-token block -- kc (key plane H), kl (plane L), qs, vc, kn and
+    kg (the norm pair of the block's token 0), vn -- and the block size."""
+    offs = (C.c_size_t * 8)()
     nbytes = lib().or_page_layout(d, m, 1 if with_values else 0, offs)
-    return int(nbytes), dict(zip(["kc", "qs", "vc", "kn", "kg", "vn"], [int(o) for o in offs]))
+    return int(nbytes), dict(zip(["kc", "qs", "vc", "kn", "kg", "vn", "block", "kl"],
+                                 [int(o) for o in offs]))
+
+
+def norm_slots(d, m, with_values=True):
+    """Byte offsets inside a page of the fp16 norm fields of the 128 token
+    slots: dict kn, kg (and vn for pages with values) -> int array [128]."""
+    _, L = page_layout(d, m, with_values)
+    s = np.arange(PAGE_TOKENS)
+    if L["block"]:
+        base = (s // 16) * L["block"]
+        t = s % 16
+        return dict(kn=base + L["kn"] + 4 * t, kg=base + L["kg"] + 4 * t, vn=base + L["vn"] + 2 * t)
+    return dict(kn=L["kn"] + 2 * s, kg=L["kg"] + 2 * s)
 
 
 def pack(pool, page_bytes, d, m, with_values, page_id, slot, rec):

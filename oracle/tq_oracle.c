@@ -361,55 +361,86 @@ OR_API int or_lloyd_max(int d, int bits, int max_iter, double* c /* L */, double
 
 /* ------------------------------------------------------------------------ */
 /* Page format (storage layout of the cold tier; 128 token slots per page). */
-/* Sections in order, each starting on a 16-byte boundary:                  */
+/* The format is this library's own (the pages fix none).  Two kinds:       */
+/*                                                                          */
+/* Keys-only pages (a search database): the record layout.  Sections in     */
+/* order, each starting on a 16-byte boundary:                              */
 /*   KC key codes    128 x d/4 bytes   (2-bit codes: sign and magnitude)    */
 /*   QS QJL signs    128 x m/8 bytes                                        */
-/*   VC value codes  64 x d bytes       (4-bit codes; values pages only)    */
 /*   KN key norm     128 x fp16                                             */
 /*   KG residual norm 128 x fp16                                            */
-/*   VN value norm   128 x fp16        (values pages only)                  */
 /* Key code word w (little-endian u32, w < d/16) of a token holds           */
 /* coordinates j = 16w + 8h + r (h in {0,1}, r = 2i + e < 8): sign bit at   */
 /* 16h + 15 - 4i - e, magnitude bit at 16h + 13 - 4i - e.                   */
 /* QJL word w (w < m/32) holds sketch index i = 32w + 16h + r (r < 16) at   */
-/* bit 16h + 15 - r.  Value codes (a code is sign<<3 | magnitude index,      */
-/* 0..7): one byte holds two tokens of one coordinate, the even token in the */
-/* low nibble.  Tokens are grouped in blocks of 16 (kb = slot/16) and        */
-/* coordinates in tiles of 16 (i = j/16); inside a (block, tile) pair, with  */
-/* g = j mod 8, jh = (j mod 16)/8, pair q = (slot mod 16)/2, c = q mod 4,    */
+/* bit 16h + 15 - r.                                                        */
+/*                                                                          */
+/* Pages with values (the decode's cold tier): 8 blocks of 16 token slots   */
+/* (block kb = slot/16, t = slot mod 16), each 12d + 2m + 96 bytes:         */
+/*   KH key plane H  2d bytes   at 0                                        */
+/*   KL key plane L  2d bytes   at 2d                                       */
+/*   QS QJL signs    2m bytes   at 4d                                       */
+/*   VC value codes  8d bytes   at 4d + 2m                                  */
+/*   NK key norm n and residual norm, fp16 pairs (n, gamma) per token, at   */
+/*      12d + 2m + 4t                                                       */
+/*   VN value norm fp16 at 12d + 2m + 64 + 2t                               */
+/* The key code is the index u = 2H + L of the level in ascending order     */
+/* (-c1, -c0, +c0, +c1): H = 1 - sign, L = sign XOR magnitude.  In a plane  */
+/* (index j < d for H and L, sketch index j < m for QS), the bit of token t */
+/* is bit t mod 8 of the byte at                                           */
+/*   16 (4 (j/32) + (j/4) mod 4) + 4 (2 ((j/16) mod 2) + t/8) + j mod 4     */
+/* so that a 32-bit word holds 4 consecutive indices x 8 tokens.            */
+/* Value codes (a code is sign<<3 | magnitude index, 0..7): one byte holds  */
+/* two tokens of one coordinate, the even token in the low nibble.  With    */
+/* i = j/16, g = j mod 8, jh = (j mod 16)/8, pair q = t/2, c = q mod 4,     */
 /* th = q/4, the byte sits at                                               */
-/*   kb*8d + (i/4)*512 + (4g + c)*16 + (i mod 4)*4 + jh + 2*th              */
-/* so that the 32-bit word at (4g + c)*16 + (i mod 4)*4 holds, in its four   */
-/* bytes, coordinates (g, g+8) x token pairs (c, c+4) of the block.          */
+/*   (i/4)*512 + (4g + c)*16 + (i mod 4)*4 + jh + 2*th                      */
+/* of the block's VC section, so that the 32-bit word at (4g + c)*16 +      */
+/* (i mod 4)*4 holds, in its four bytes, coordinates (g, g+8) x token       */
+/* pairs (c, c+4).                                                          */
 /* ------------------------------------------------------------------------ */
 #define PAGE_TOKENS 128
+#define BLOCK_TOKENS 16
 
 typedef struct {
-  size_t kc, qs, vc, kn, kg, vn, bytes;
+  /* record layout: section offsets; block layout: offsets inside a block */
+  size_t kc, kl, qs, vc, kn, kg, vn, block, bytes;
 } or_layout;
 
 static size_t up16(size_t x) { return (x + 15) & ~(size_t)15; }
 
 static or_layout layout_of(int d, int m, int with_values) {
   or_layout L;
+  memset(&L, 0, sizeof(L));
+  if (with_values) {
+    L.kc = 0;
+    L.kl = (size_t)2 * d;
+    L.qs = (size_t)4 * d;
+    L.vc = (size_t)4 * d + (size_t)2 * m;
+    L.kn = (size_t)12 * d + (size_t)2 * m;
+    L.kg = L.kn + 2;
+    L.vn = L.kn + 64;
+    L.block = L.kn + 96;
+    L.bytes = (PAGE_TOKENS / BLOCK_TOKENS) * L.block;
+    return L;
+  }
   size_t off = 0;
   L.kc = off; off = up16(off + (size_t)PAGE_TOKENS * d / 4);
   L.qs = off; off = up16(off + (size_t)PAGE_TOKENS * m / 8);
-  if (with_values) { L.vc = off; off = up16(off + (size_t)PAGE_TOKENS * d / 2); }
-  else L.vc = 0;
   L.kn = off; off = up16(off + 2 * PAGE_TOKENS);
   L.kg = off; off = up16(off + 2 * PAGE_TOKENS);
-  if (with_values) { L.vn = off; off = up16(off + 2 * PAGE_TOKENS); }
-  else L.vn = 0;
   L.bytes = off;
   return L;
 }
 
-OR_API size_t or_page_layout(int d, int m, int with_values, size_t* offs /* 6 or NULL */) {
+/* offs (8 or NULL): kc, qs, vc, kn, kg, vn, block bytes (0: record layout),
+ * kl.  Block layout: kc = KH, kn and kg the fields of token 0 of block 0. */
+OR_API size_t or_page_layout(int d, int m, int with_values, size_t* offs) {
   or_layout L = layout_of(d, m, with_values);
   if (offs) {
     offs[0] = L.kc; offs[1] = L.qs; offs[2] = L.vc;
     offs[3] = L.kn; offs[4] = L.kg; offs[5] = L.vn;
+    offs[6] = L.block; offs[7] = L.kl;
   }
   return L.bytes;
 }
@@ -423,23 +454,32 @@ static void wr32(uint8_t* p, uint32_t v) {
 static uint16_t rd16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
 static void wr16(uint8_t* p, uint16_t v) { p[0] = (uint8_t)v; p[1] = (uint8_t)(v >> 8); }
 
-static int kc_sign_bit(int j) { /* position inside word j/16 */
+static int kc_sign_bit(int j) { /* record layout: position inside word j/16 */
   int h = (j % 16) / 8, r = j % 8, i = r / 2, e = r % 2;
   return 16 * h + 15 - 4 * i - e;
 }
 static int kc_mag_bit(int j) { return kc_sign_bit(j) - 2; }
-static int qs_bit(int i) { /* position inside word i/32 */
+static int qs_bit(int i) { /* record layout: position inside word i/32 */
   int h = (i % 32) / 16, r = i % 16;
   return 16 * h + 15 - r;
 }
 
-/* offset, inside the value-code section, of the byte holding token pair p
- * (slots 2p, 2p+1) of coordinate j */
-static size_t vc_pos(int d, int p, int j) {
-  int kb = p / 8, q = p % 8, c = q % 4, th = q / 4;
+/* block layout: byte of plane index j for token t (bit t mod 8) */
+static size_t plane_byte(int j, int t) {
+  return (size_t)16 * (4 * (j / 32) + (j / 4) % 4) + (size_t)4 * (2 * ((j / 16) % 2) + t / 8) +
+         (size_t)(j % 4);
+}
+static void put_bit(uint8_t* p, int bit, int v) {
+  *p = (uint8_t)(v ? (*p | (1u << bit)) : (*p & ~(1u << bit)));
+}
+
+/* block layout: offset, inside a block's value section, of the byte holding
+ * token t (slot mod 16) of coordinate j */
+static size_t vc_pos(int t, int j) {
+  int q = t / 2, c = q % 4, th = q / 4;
   int i = j / 16, g = j % 8, jh = (j % 16) / 8;
-  return (size_t)kb * 8 * d + (size_t)(i / 4) * 512 + (size_t)(4 * g + c) * 16 +
-         (size_t)(i % 4) * 4 + (size_t)(jh + 2 * th);
+  return (size_t)(i / 4) * 512 + (size_t)(4 * g + c) * 16 + (size_t)(i % 4) * 4 +
+         (size_t)(jh + 2 * th);
 }
 
 /* write one key record into token slot `slot` of page `pg` */
@@ -447,6 +487,18 @@ OR_API void or_pack_key(uint8_t* pg, int d, int m, int with_values, int slot,
                         const int32_t* sign, const int32_t* mag, const int32_t* qbits,
                         double n, double gamma) {
   or_layout L = layout_of(d, m, with_values);
+  if (with_values) {
+    uint8_t* bk = pg + (size_t)(slot / BLOCK_TOKENS) * L.block;
+    int t = slot % BLOCK_TOKENS;
+    for (int j = 0; j < d; ++j) {
+      put_bit(bk + L.kc + plane_byte(j, t), t % 8, !sign[j]);
+      put_bit(bk + L.kl + plane_byte(j, t), t % 8, (sign[j] != 0) != (mag[j] != 0));
+    }
+    for (int i = 0; i < m; ++i) put_bit(bk + L.qs + plane_byte(i, t), t % 8, qbits[i] != 0);
+    wr16(bk + L.kn + 4 * t, f16_bits(or_round_f16(n)));
+    wr16(bk + L.kg + 4 * t, f16_bits(or_round_f16(gamma)));
+    return;
+  }
   uint8_t* kc = pg + L.kc + (size_t)slot * (d / 4);
   for (int w = 0; w < d / 16; ++w) {
     uint32_t word = 0;
@@ -470,6 +522,20 @@ OR_API void or_pack_key(uint8_t* pg, int d, int m, int with_values, int slot,
 OR_API void or_unpack_key(const uint8_t* pg, int d, int m, int with_values, int slot,
                           int32_t* sign, int32_t* mag, int32_t* qbits, double* n, double* gamma) {
   or_layout L = layout_of(d, m, with_values);
+  if (with_values) {
+    const uint8_t* bk = pg + (size_t)(slot / BLOCK_TOKENS) * L.block;
+    int t = slot % BLOCK_TOKENS;
+    for (int j = 0; j < d; ++j) {
+      int h = (bk[L.kc + plane_byte(j, t)] >> (t % 8)) & 1;
+      int l = (bk[L.kl + plane_byte(j, t)] >> (t % 8)) & 1;
+      sign[j] = 1 - h;
+      mag[j] = l ^ sign[j];
+    }
+    for (int i = 0; i < m; ++i) qbits[i] = (bk[L.qs + plane_byte(i, t)] >> (t % 8)) & 1;
+    *n = f16_value(rd16(bk + L.kn + 4 * t));
+    *gamma = f16_value(rd16(bk + L.kg + 4 * t));
+    return;
+  }
   const uint8_t* kc = pg + L.kc + (size_t)slot * (d / 4);
   for (int j = 0; j < d; ++j) {
     uint32_t word = rd32(kc + 4 * (j / 16));
@@ -482,29 +548,28 @@ OR_API void or_unpack_key(const uint8_t* pg, int d, int m, int with_values, int 
   *gamma = f16_value(rd16(pg + L.kg + 2 * slot));
 }
 
-/* value record: code = sign<<3 | magnitude index */
+/* value record (pages with values): code = sign<<3 | magnitude index */
 OR_API void or_pack_value(uint8_t* pg, int d, int m, int slot, const int32_t* code, double n) {
   or_layout L = layout_of(d, m, 1);
-  int p = slot / 2;
-  uint8_t* vc = pg + L.vc;
-  int hi = slot & 1;
+  uint8_t* bk = pg + (size_t)(slot / BLOCK_TOKENS) * L.block;
+  int t = slot % BLOCK_TOKENS, hi = t & 1;
   for (int j = 0; j < d; ++j) {
-    uint8_t* bp = vc + vc_pos(d, p, j);
+    uint8_t* bp = bk + L.vc + vc_pos(t, j);
     uint8_t c = (uint8_t)(code[j] & 0xF);
     *bp = hi ? (uint8_t)((*bp & 0x0F) | (c << 4)) : (uint8_t)((*bp & 0xF0) | c);
   }
-  wr16(pg + L.vn + 2 * slot, f16_bits(or_round_f16(n)));
+  wr16(bk + L.vn + 2 * t, f16_bits(or_round_f16(n)));
 }
 
 OR_API void or_unpack_value(const uint8_t* pg, int d, int m, int slot, int32_t* code, double* n) {
   or_layout L = layout_of(d, m, 1);
-  int p = slot / 2;
-  const uint8_t* vc = pg + L.vc;
+  const uint8_t* bk = pg + (size_t)(slot / BLOCK_TOKENS) * L.block;
+  int t = slot % BLOCK_TOKENS;
   for (int j = 0; j < d; ++j) {
-    uint8_t b = vc[vc_pos(d, p, j)];
-    code[j] = (slot & 1) ? (b >> 4) : (b & 0xF);
+    uint8_t b = bk[L.vc + vc_pos(t, j)];
+    code[j] = (t & 1) ? (b >> 4) : (b & 0xF);
   }
-  *n = f16_value(rd16(pg + L.vn + 2 * slot));
+  *n = f16_value(rd16(bk + L.vn + 2 * t));
 }
 
 /* batched forms: record v goes to page page_id[v], slot slot[v].

@@ -22,10 +22,10 @@ def build(O, P, B, Hq, Hkv, d, cold_len, hot_len, W_max, max_pages, q_dtype="flo
     c.cold_len = np.asarray(cold_len, np.int32)
     c.hot_len = np.asarray(hot_len, np.int32)
     c.W_max, c.max_pages = W_max, max_pages
-    nbytes, offs = O.page_layout(d, d, True)
+    nbytes, _ = O.page_layout(d, d, True)
     c.page_bytes = nbytes
     c.table, n_pages = W.random_page_table(seed + 1, B, Hkv, max_pages, spare=3)
-    c.pool = W.random_page_bytes(seed + 2, n_pages, nbytes, offs)
+    c.pool = W.random_page_bytes(seed + 2, n_pages, nbytes, O.norm_slots(d, d, True))
     chans = W.outlier_channels(seeds[3], Hkv, d, n_out)
     c.k_hot = np.zeros((B, Hkv, max(W_max, 1), d))
     c.v_hot = np.zeros((B, Hkv, max(W_max, 1), d))

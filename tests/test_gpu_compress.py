@@ -345,3 +345,49 @@ def test_compress_then_decode_end_to_end(O):
     diff, qerr = np.concatenate(diff), np.concatenate(qerr)
     assert diff.max() < 2e-2
     assert diff.mean() < 0.1 * qerr.mean(), (diff.mean(), qerr.mean())
+
+
+def test_compress_4m_sampled_records(O):
+    """The full compress workload in the benchmark's launch configuration
+    (8 kv heads x 524288 bf16 vectors, d = 128, x = N(0,1) sigma[h, j], sigma
+    LogNormal(0,1), one call, keys-only pages): 8192 records sampled over all
+    heads and page tiles (first and last page of every head included) match
+    the oracle's encoding of the same input rows within the rotation error."""
+    import torch
+    d, H, T = 128, 8, 524288
+    P = params_for(O, d)
+    ctx = ctx_for(d)
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(21)
+    sigma = torch.exp(torch.randn((H, d), generator=gen, device=dev))
+    x = (torch.randn((1, H, T, d), generator=gen, device=dev) * sigma[None, :, None, :]).to(torch.bfloat16)
+    pages = H * T // 128
+    pool = torch.zeros((pages, ctx.page_bytes(False)), dtype=torch.uint8, device=dev)
+    table = torch.arange(pages, dtype=torch.int32, device=dev).view(1, H, T // 128)
+    cold = torch.zeros(1, dtype=torch.int32, device=dev)
+    tq.tq_compress_append(ctx.handle, x, None, pool, table, cold)
+    torch.cuda.synchronize()
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_OK
+    assert int(cold.item()) == T
+    rng = np.random.default_rng(41)
+    nb = ctx.page_bytes(False)
+    eps = 2.0 ** -8
+    flips = sflips = total = 0
+    for h in range(H):
+        t = np.concatenate([rng.choice(T, 1030, replace=False), [0, 127, T - 128, T - 1]])
+        t = np.unique(t)
+        rows = x[0, h, torch.from_numpy(t).to(dev)].double().cpu().numpy()
+        pg = (h * (T // 128) + t // 128).astype(np.int64)
+        uniq, inv = np.unique(pg, return_inverse=True)
+        sub = pool[torch.from_numpy(uniq).to(dev)].cpu().numpy().reshape(-1)
+        got = O.unpack(sub, nb, d, d, False, inv.astype(np.int32), (t % 128).astype(np.int32))
+        rk = O.encode(P, rows, True)
+        err = (np.abs(rows) @ np.abs(P.pi32).T) * (eps * eps * 2 + 64 * 2.0 ** -24)
+        flips += compare_records(O, P, rows, rk, got, True, err)
+        sflips += check_sketch_raw(P, rk, got, err)
+        total += len(t) * d
+    assert total >= 8192 * d
+    assert sflips <= 0.01 * total
+    print("4M compress, %d sampled records: code differences at decision boundaries %d, "
+          "sketch sign flips near zero %d" % (total // d, flips, sflips))

@@ -13,12 +13,31 @@ D_M = [(64, 64), (128, 128)]
 
 def _golden():
     path = os.path.join(os.path.dirname(__file__), "golden", "page_format_examples.txt")
-    rows = {}
+    rows = []
     for line in open(path):
         if line.strip() and not line.startswith("#"):
             kind, *fields = line.split()
-            rows[kind] = dict(f.split("=") for f in fields)
+            rows.append((kind, dict(f.split("=") for f in fields)))
     return rows
+
+
+def _one(rows, kind):
+    (row,) = [r for k, r in rows if k == kind]
+    return row
+
+
+# The format as the header states it (include/tq.h, tq_page_bytes), typed
+# here from that text: the bit of plane index j for token t of a block, and
+# the value byte of coordinate j for token t of a block.
+def _plane_pos(j, t):
+    return 16 * (4 * (j // 32) + (j // 4) % 4) + 4 * (2 * ((j // 16) % 2) + t // 8) + j % 4, t % 8
+
+
+def _value_pos(j, t):
+    q = t // 2
+    c, th = q % 4, q // 4
+    i, g, jh = j // 16, j % 8, (j % 16) // 8
+    return (i // 4) * 512 + (4 * g + c) * 16 + (i % 4) * 4 + jh + 2 * th
 
 
 @pytest.mark.parametrize("d,m,wv,expect", [(128, 128, 1, 15104), (128, 128, 0, 6656),
@@ -26,10 +45,17 @@ def _golden():
 def test_page_bytes(O, d, m, wv, expect):
     nbytes, offs = O.page_layout(d, m, bool(wv))
     assert nbytes == expect
-    assert all(v % 16 == 0 for v in offs.values())
-    # key codes 2 bits, QJL 1 bit, value codes 4 bits, three fp16 per token
-    assert offs["qs"] - offs["kc"] == 128 * d * 2 // 8
-    assert (offs["vc"] - offs["qs"] if wv else offs["kn"] - offs["qs"]) == 128 * m // 8
+    if wv:  # 8 blocks of 16 slots; 118 (d=128) or 62 (d=64) bytes per token
+        assert offs["block"] * 8 == nbytes and offs["block"] == 16 * (12 * d + 2 * m + 96) // 16
+        assert [offs[k] for k in ("kc", "kl", "qs", "vc", "kn", "vn")] == \
+            [0, 2 * d, 4 * d, 4 * d + 2 * m, 12 * d + 2 * m, 12 * d + 2 * m + 64]
+        assert offs["kg"] == offs["kn"] + 2
+        assert all(offs[k] % 16 == 0 for k in ("kc", "kl", "qs", "vc", "kn", "vn", "block"))
+    else:  # record layout: key codes 2 bits, QJL 1 bit, two fp16 per token
+        assert offs["block"] == 0
+        assert all(v % 16 == 0 for v in offs.values())
+        assert offs["qs"] - offs["kc"] == 128 * d * 2 // 8
+        assert offs["kn"] - offs["qs"] == 128 * m // 8
 
 
 def _empty_records(N, d, m):
@@ -38,52 +64,123 @@ def _empty_records(N, d, m):
                 vcode=z(N, d), vn=np.ones(N))
 
 
-def test_golden_format_examples(O):
+def test_golden_record_layout_examples(O):
+    """Keys-only pages: hand-worked key and QJL words."""
+    g = _golden()
+    d = m = 64
+    nbytes, offs = O.page_layout(d, m, False)
+    pool = np.zeros(nbytes, np.uint8)
+    rec = _empty_records(1, d, m)
+    key, qjl = _one(g, "key"), _one(g, "qjl")
+    for j in map(int, key["sign"].split(",")):
+        rec["sign"][0, j] = 1
+    for j in map(int, key["mag"].split(",")):
+        rec["mag"][0, j] = 1
+    for i in map(int, qjl["bits"].split(",")):
+        rec["qbits"][0, i] = 1
+    O.pack(pool, nbytes, d, m, False, [0], [0], {k: rec[k] for k in ("sign", "mag", "qbits", "n", "gamma")})
+    word = lambda off: int.from_bytes(pool[off:off + 4].tobytes(), "little")
+    assert word(offs["kc"]) == int(key["word0"], 16)
+    assert word(offs["qs"]) == int(qjl["word0"], 16)
+
+
+def test_golden_block_layout_examples(O):
+    """Pages with values: hand-worked plane words, norms and value bytes."""
     g = _golden()
     d = m = 64
     nbytes, offs = O.page_layout(d, m, True)
     pool = np.zeros(nbytes, np.uint8)
-    rec = _empty_records(6, d, m)
-    for j in map(int, g["key"]["sign"].split(",")):
+    b1, b2 = _one(g, "block"), _one(g, "block2")
+    v1, v2 = _one(g, "value"), _one(g, "value2")
+    rec = _empty_records(2, d, m)
+    vrec = _empty_records(4, d, m)
+    ints = lambda s: [int(x) for x in s.split(",")]
+    for j in ints(b1["sign"]):
         rec["sign"][0, j] = 1
-    for j in map(int, g["key"]["mag"].split(",")):
+    for j in ints(b1["mag"]):
         rec["mag"][0, j] = 1
-    for i in map(int, g["qjl"]["bits"].split(",")):
+    for i in ints(b1["qjl"]):
         rec["qbits"][0, i] = 1
-    cj = int(g["value"]["coord"])
-    rec["vcode"][2, cj] = int(g["value"]["slot2"], 16)
-    rec["vcode"][3, cj] = int(g["value"]["slot3"], 16)
-    cj2 = int(g["value2"]["coord"])
-    rec["vcode"][4, cj2] = int(g["value2"]["slot26"], 16)
-    rec["vcode"][5, cj2] = int(g["value2"]["slot27"], 16)
-    O.pack(pool, nbytes, d, m, True, [0] * 6, [0, 1, 2, 3, 26, 27], rec)
+    rec["n"][0], rec["gamma"][0], rec["vn"][0] = float(b1["n"]), float(b1["gamma"]), float(b1["vn"])
+    for j in ints(b2["sign"]):
+        rec["sign"][1, j] = 1
+    cj, cj2 = int(v1["coord"]), int(v2["coord"])
+    vrec["vcode"][0, cj] = int(v1["slot2"], 16)
+    vrec["vcode"][1, cj] = int(v1["slot3"], 16)
+    vrec["vcode"][2, cj2] = int(v2["slot26"], 16)
+    vrec["vcode"][3, cj2] = int(v2["slot27"], 16)
+    O.pack(pool, nbytes, d, m, True, [0] * 2, [int(b1["slot"]), int(b2["slot"])], rec)
+    vpool = np.zeros(nbytes, np.uint8)  # the value examples on a page of their own
+    O.pack(vpool, nbytes, d, m, True, [0] * 4, [2, 3, 26, 27], vrec)
+    sec = {"kh": offs["kc"], "kl": offs["kl"], "qs": offs["qs"], "nk": offs["kn"], "vn": offs["vn"]}
     word = lambda off: int.from_bytes(pool[off:off + 4].tobytes(), "little")
-    assert word(offs["kc"]) == int(g["key"]["word0"], 16)
-    assert word(offs["qs"]) == int(g["qjl"]["word0"], 16)
-    assert pool[offs["vc"] + int(g["value"]["offset"])] == int(g["value"]["byte"], 16)
-    assert pool[offs["vc"] + int(g["value2"]["offset"])] == int(g["value2"]["byte"], 16)
-    assert np.count_nonzero(pool[offs["vc"]:offs["kn"]]) == 2
+    assert int(b1["base"]) == offs["block"] == int(b2["base"])
+    for kind, r in g:
+        if kind in ("block_word", "block_word2"):
+            assert word(offs["block"] + sec[r["section"]] + int(r["off"])) == int(r["word"], 16), r
+        if kind == "block_half":
+            off = offs["block"] + sec[r["section"]] + int(r["off"])
+            assert int.from_bytes(pool[off:off + 2].tobytes(), "little") == int(r["half"], 16)
+    for v in (v1, v2):
+        assert vpool[int(v["block"]) * offs["block"] + offs["vc"] + int(v["offset"])] == int(v["byte"], 16)
+    assert sum(np.count_nonzero(vpool[b * offs["block"] + offs["vc"]:b * offs["block"] + offs["kn"]])
+               for b in range(8)) == 2
+
+
+@pytest.mark.parametrize("d,m", D_M)
+def test_block_plane_positions(O, d, m):
+    """Every (token, index) bit of the H, L and QJL planes lands on the byte
+    and bit the format states, inside its block's plane (each plane a
+    bijection of the block's 16 tokens x d indices onto its 2d bytes)."""
+    nbytes, offs = O.page_layout(d, m, True)
+    blk = offs["block"]
+    for plane, size in (("kc", d), ("kl", d), ("qs", m)):
+        seen = set()
+        for slot in list(range(16, 32)) + [0, 77, 127]:
+            for j in range(size):
+                pool = np.zeros(nbytes, np.uint8)
+                rec = _empty_records(1, d, m)
+                if plane == "kc":    # H = 1 - sign: every sign set except coordinate j
+                    rec["sign"][0] = 1
+                    rec["sign"][0, j] = 0
+                    rec["mag"][0] = 1     # L = 0 everywhere
+                    rec["mag"][0, j] = 0
+                elif plane == "kl":  # L = sign XOR mag: one magnitude bit, no signs
+                    rec["mag"][0, j] = 1
+                else:
+                    rec["qbits"][0, j] = 1
+                O.pack(pool, nbytes, d, m, True, [0], [slot], rec)
+                base = (slot // 16) * blk + offs[plane]
+                sec = pool[base:base + 2 * size]
+                (pos,) = np.nonzero(sec)
+                byte, bit = _plane_pos(j, slot % 16)
+                assert list(pos) == [byte] and sec[byte] == 1 << bit, (plane, slot, j)
+                if 16 <= slot < 32:
+                    seen.add((byte, bit))
+        assert len(seen) == 16 * size
 
 
 @pytest.mark.parametrize("d,m", D_M)
 def test_value_byte_positions(O, d, m):
-    """Every (token pair, coordinate) lands on its own byte of the value
-    section (a bijection onto its 64 d bytes), and all bytes of a 16-token
-    block stay inside that block's 8 d bytes."""
+    """Every (token, coordinate) lands on the byte the format states, in the
+    nibble of its token's parity, inside its block's value section (a
+    bijection onto the block's 8 d bytes)."""
     nbytes, offs = O.page_layout(d, m, True)
+    blk = offs["block"]
     seen = set()
-    for p in range(64):
+    for slot in range(32, 48):
         for j in range(d):
             pool = np.zeros(nbytes, np.uint8)
             rec = _empty_records(1, d, m)
             rec["vcode"][0, j] = 0x9
-            O.pack(pool, nbytes, d, m, True, [0], [2 * p + 1], rec)
-            sec = pool[offs["vc"]: offs["vc"] + 64 * d]
+            O.pack(pool, nbytes, d, m, True, [0], [slot], rec)
+            base = (slot // 16) * blk + offs["vc"]
+            sec = pool[base: base + 8 * d]
             (pos,) = np.nonzero(sec)
-            assert len(pos) == 1 and sec[pos[0]] == 0x90
-            assert pos[0] // (8 * d) == p // 8
-            seen.add(int(pos[0]))
-    assert len(seen) == 64 * d
+            assert list(pos) == [_value_pos(j, slot % 16)]
+            assert sec[pos[0]] == (0x90 if slot & 1 else 0x09)
+            seen.add(int(pos[0]) * 2 + (slot & 1))
+    assert len(seen) == 16 * d
 
 
 @pytest.mark.parametrize("d,m", D_M)

@@ -22,10 +22,12 @@ def _case(torch, ctx, seed, B, Hkv, G, d, hot, max_pages, qdtype):
     dev = "cuda"
     nb = ctx.page_bytes(True)
     table, n_pages = W.random_page_table(seed, B, Hkv, max_pages, spare=1)
-    # norm field offsets of a values page: after KC, QS and VC
-    kc, qs, vc = 128 * d // 4, 128 * d // 8, 128 * d // 2
-    offs = {"kn": kc + qs + vc, "kg": kc + qs + vc + 256, "vn": kc + qs + vc + 512}
-    pool = W.random_page_bytes(seed + 1, n_pages, nb, offs)
+    # fp16 norm fields of a values page: 8 blocks of 16 slots, each block
+    # 14 d + 96 bytes ending in 16 (n, gamma) pairs and 16 value norms
+    blk, s = 14 * d + 96, np.arange(128)
+    kn = (s // 16) * blk + 12 * d + 2 * d + 4 * (s % 16)
+    pool = W.random_page_bytes(seed + 1, n_pages, nb, {"kn": kn, "kg": kn + 2,
+                                                       "vn": (s // 16) * blk + 14 * d + 64 + 2 * (s % 16)})
     rng = np.random.default_rng(seed + 2)
     k_hot = rng.standard_normal((B, Hkv, hot, d)).astype(np.float16)
     v_hot = rng.standard_normal((B, Hkv, hot, d)).astype(np.float16)
