@@ -49,7 +49,8 @@ def parse():
                     help="sequences per GPU (default: the workload's 16); smaller values only "
                          "size profiler captures and are not the benchmark line")
     ap.add_argument("--only", default=None,
-                    choices=["gated", "monarch", "tensor_cache", "stage1", "self_index"],
+                    choices=["gated", "monarch", "tensor_cache", "stage1", "self_index",
+                             "compress", "search"],
                     help="run one extra row alone and print it (sized for profiler captures; "
                          "not the benchmark line)")
     return ap.parse_args()
@@ -176,11 +177,12 @@ def build_state(torch, tq, W, rank, batch=None, workload=WORKLOAD, extra_pages=0
     return st
 
 
-def measure_compress(torch, tq, reps=5):
+def measure_compress(torch, tq, reps=5, T=524288):
     """Compress/append throughput: 8 kv heads x 524288 bf16 vectors (d=128),
-    x = N(0,1) * sigma[h, j], sigma ~ LogNormal(0,1), keys-only pages."""
+    x = N(0,1) * sigma[h, j], sigma ~ LogNormal(0,1), keys-only pages (T
+    smaller only for profiler captures)."""
     dev = torch.device("cuda")
-    H, T, d = 8, 524288, 128
+    H, d = 8, 128
     ctx = tq.Context(d, seed=0)
     gen = torch.Generator(device=dev)
     gen.manual_seed(21)
@@ -206,17 +208,18 @@ def measure_compress(torch, tq, reps=5):
     n = H * T
     bytes_ = n * (2 * d + 52)
     flops = n * 2 * (d * d + d * d)
-    return {"workload": "compress_4m (8 kv heads x 524288 bf16 vectors, d=128, keys-only)",
+    return {"workload": "compress_4m (8 kv heads x %d bf16 vectors, d=128, keys-only)" % T,
             "vectors_per_s": n / (ms / 1e3), "kernel_ms": ms,
             "achieved_gbs": bytes_ / (ms / 1e3) / 1e9, "algorithmic_bytes": bytes_,
             "achieved_tflops": flops / (ms / 1e3) / 1e12, "algorithmic_flops": flops}
 
 
-def measure_search(torch, tq, reps=3):
+def measure_search(torch, tq, reps=3, N=1_000_000):
     """Compressed top-10 search: 10^6 database unit vectors (d=128, bf16
-    input, keys-only pages) and 4096 unit queries."""
+    input, keys-only pages) and 4096 unit queries (N smaller only for
+    profiler captures)."""
     dev = torch.device("cuda")
-    N, Q, d, k = 1_000_000, 4096, 128, 10
+    Q, d, k = 4096, 128, 10
     ctx = tq.Context(d, seed=0)
     gen = torch.Generator(device=dev)
     gen.manual_seed(31)
@@ -537,11 +540,69 @@ def cpu_baseline(sample_groups=None):
     O.attention(P, q, 1, 1.0 / math.sqrt(d), k_hot, v_hot, lens_h, pool.reshape(-1), nbytes,
                 table, lens_c, threads=threads)
     dt = time.perf_counter() - t0
+    t1 = time.perf_counter()  # one thread, one group
+    O.attention(P, q[:1], 1, 1.0 / math.sqrt(d), k_hot[:1], v_hot[:1], lens_h[:1],
+                pool.reshape(-1), nbytes, table[:1], lens_c[:1], threads=1)
+    dt1 = time.perf_counter() - t1
     units = n * (cfg["cold"] + cfg["hot"])
     return {"value": units / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "value_1_thread": (cfg["cold"] + cfg["hot"]) / dt1,
             "sample": "%d of %d (batch, kv head) groups of the 32K decode (%d tokens each), "
-                      "random cold records, %.2f s" % (n, cfg["B"] * cfg["Hkv"],
-                                                       cfg["cold"] + cfg["hot"], dt)}
+                      "random cold records, %.2f s; 1 thread: 1 group, %.2f s"
+                      % (n, cfg["B"] * cfg["Hkv"], cfg["cold"] + cfg["hot"], dt, dt1)}
+
+
+def cpu_baseline_compress(n=1 << 18, n1=1 << 14):
+    """The oracle's encoder (rotation, codes, residual, QJL sketch, keys) on a
+    bounded sample of the compress workload: n of its 4194304 vectors on all
+    host threads, n1 of them on one thread."""
+    import oracle as O
+    from compressed_kv_decode_b200 import workloads as W
+    d, H = 128, 8
+    P = O.Params(d, seed=0)
+    scales = W.compress_scales(21, H, d)
+    x = W.compress_data(22, scales, 524288, rows=(0, 0, n))[0]
+    threads = O.max_threads()
+    t0 = time.perf_counter()
+    O.encode(P, x, True, threads=threads)
+    dt = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    O.encode(P, x[:n1], True, threads=1)
+    dt1 = time.perf_counter() - t1
+    return {"value": n / dt, "unit": "vectors/s", "cores": threads, "kind": "oracle",
+            "value_1_thread": n1 / dt1,
+            "sample": "%d of the 4194304 vectors (head 0), %.2f s; 1 thread: %d vectors, %.2f s"
+                      % (n, dt, n1, dt1)}
+
+
+def cpu_baseline_search(nq=256, nq1=16):
+    """The oracle's search (estimated inner products with every database
+    record, exact top-10) for nq of the 4096 queries against the full 10^6
+    database, which the oracle's encoder writes; nq1 queries on one thread."""
+    import oracle as O
+    from compressed_kv_decode_b200 import workloads as W
+    d, N, k = 128, 1_000_000, 10
+    P = O.Params(d, seed=0)
+    threads = O.max_threads()
+    db = W.unit_vectors(31, N, d)
+    rec = O.encode(P, db, True, threads=threads)
+    nb, _ = O.page_layout(d, d, False)
+    pool = np.zeros(((N + 127) // 128) * nb, np.uint8)
+    idx = np.arange(N)
+    O.pack(pool, nb, d, d, False, idx // 128, idx % 128,
+           {f: rec[f] for f in ("sign", "mag", "qbits", "n", "gamma")})
+    del rec
+    qs = W.unit_vectors(32, 4096, d)
+    t0 = time.perf_counter()
+    O.topk(P, qs[:nq], pool, nb, N, k, threads=threads)
+    dt = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    O.topk(P, qs[:nq1], pool, nb, N, k, threads=1)
+    dt1 = time.perf_counter() - t1
+    return {"value": nq * N / dt, "unit": "query*vectors/s", "cores": threads, "kind": "oracle",
+            "value_1_thread": nq1 * N / dt1,
+            "sample": "%d of the 4096 queries against the full 10^6 database, %.2f s; "
+                      "1 thread: %d queries, %.2f s" % (nq, dt, nq1, dt1)}
 
 
 def run_reference(args, rank, world):
@@ -610,15 +671,16 @@ def run_ours(args, rank, world, local_rank):
     # library on the launching stream around that kernel (K more steps)
     ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
-    for i in range(args.steps):
-        # torch reports only events it recorded itself: record both once; the
-        # library re-records them around the attention kernel
-        ev_k[i][0].record(stream)
-        ev_k[i][1].record(stream)
-        tq.tq_set_profile_events(ctx.handle, ev_k[i][0], ev_k[i][1])
-        decode(tq, st)
-    tq.tq_set_profile_events(ctx.handle, None, None)
-    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk_k:
+        for i in range(args.steps):
+            # torch reports only events it recorded itself: record both once;
+            # the library re-records them around the attention kernel
+            ev_k[i][0].record(stream)
+            ev_k[i][1].record(stream)
+            tq.tq_set_profile_events(ctx.handle, ev_k[i][0], ev_k[i][1])
+            decode(tq, st)
+        tq.tq_set_profile_events(ctx.handle, None, None)
+        torch.cuda.synchronize()
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_k)
 
     # end to end: q from pinned host memory, output back to pinned host memory
@@ -671,8 +733,10 @@ def run_ours(args, rank, world, local_rank):
                                 measure_monarch(torch, tq, W, WORKLOAD, 128)]
         torch.cuda.empty_cache()
         rows["compress"] = measure_compress(torch, tq)
+        rows["compress"]["cpu_baseline"] = cpu_baseline_compress()
         torch.cuda.empty_cache()
         rows["search"] = measure_search(torch, tq)
+        rows["search"]["cpu_baseline"] = cpu_baseline_search()
         torch.cuda.empty_cache()
         rows["stage1"] = measure_stage1(torch, tq)
         torch.cuda.empty_cache()
@@ -701,6 +765,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": 3 * args.steps,
         "step": "one decode call (query prep, split-K attention, combine) replayed from a CUDA graph",
         "clocks": clk.summary(),
+        "clocks_kernel_pass": clk_k.summary(),
         "cpu_baseline": cb,
         "rows": rows,
     }
@@ -721,6 +786,10 @@ def run_only(args):
         res = measure_tensor_cache(torch, tq, W, WORKLOAD, steps=args.steps)
     elif args.only == "self_index":
         res = measure_self_index(torch, tq, reps=max(1, args.steps))
+    elif args.only == "compress":  # --batch b: 8 heads x b * 65536 vectors
+        res = measure_compress(torch, tq, reps=max(1, args.steps), T=65536 * (args.batch or 8))
+    elif args.only == "search":  # --batch b: b * 100000 database vectors
+        res = measure_search(torch, tq, reps=max(1, args.steps), N=100_000 * (args.batch or 10))
     else:
         res = measure_stage1(torch, tq, reps=max(1, args.steps))
     print(json.dumps({"only": args.only, "row": res}), flush=True)

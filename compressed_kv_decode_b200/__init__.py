@@ -111,6 +111,8 @@ def lib():
         L.tq_score_topk.restype = C.c_int
         L.tq_set_profile_events.argtypes = [vp, vp, vp]
         L.tq_set_profile_events.restype = C.c_int
+        L.tq_set_wait_test.argtypes = [vp, C.c_int, C.c_uint64]
+        L.tq_set_wait_test.restype = C.c_int
         L.tq_get_error.argtypes = [vp]
         L.tq_get_error.restype = C.c_int
         L.tq_status_string.argtypes = [C.c_int]
@@ -406,6 +408,12 @@ def tq_set_profile_events(ctx, ev_start, ev_stop):
     a = None if ev_start is None else C.c_void_p(ev_start.cuda_event)
     b = None if ev_stop is None else C.c_void_p(ev_stop.cuda_event)
     _check(lib().tq_set_profile_events(ctx, a, b), "tq_set_profile_events")
+
+
+def tq_set_wait_test(ctx, skip_unit, limit_ns=0):
+    """Testing aid for the bounded waits: skip the copy of cold unit skip_unit
+    (-1: none) and bound every attention wait by limit_ns (0: default)."""
+    _check(lib().tq_set_wait_test(ctx, int(skip_unit), int(limit_ns)), "tq_set_wait_test")
 
 
 def tq_get_error(ctx):

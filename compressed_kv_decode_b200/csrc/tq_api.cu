@@ -4,6 +4,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -43,6 +45,14 @@ PageLayout page_layout(int d, int m, bool with_values) {
 }
 
 namespace {
+
+// NVTX range over one host call (visible in Nsight timelines; the NVTX
+// library is loaded only when a tool injects it, otherwise each push / pop is a
+// no-op check)
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+};
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -87,6 +97,7 @@ tq_status tq_generate_params(const tq_config* cfg, float* rot, float* qjl, float
 }
 
 tq_status tq_init_codebook(const tq_config* cfg, tq_ctx** out) {
+  tq::Range range("tq_init_codebook");
   if (!cfg || !out) return TQ_ERR_INVALID_ARG;
   *out = nullptr;
   if (!tq::config_valid(*cfg)) return TQ_ERR_INVALID_ARG;
@@ -94,6 +105,7 @@ tq_status tq_init_codebook(const tq_config* cfg, tq_ctx** out) {
   tq_ctx* ctx = new (std::nothrow) tq_ctx();
   if (!ctx) return TQ_ERR_OOM;
   ctx->cfg = *cfg;
+  ctx->wait_skip_unit = -1;
   if (!tq::generate_tables(*cfg, ctx->host)) {
     delete ctx;
     return TQ_ERR_INVALID_ARG;
@@ -198,6 +210,7 @@ tq_status tq_compress_append(const tq_ctx* ctx, const void* k, const void* v, tq
                              int flags, int B, int Hkv, int n_new, uint8_t* page_pool,
                              int64_t pool_pages, const int32_t* page_table, int max_pages,
                              int32_t* cold_len, void* stream) {
+  tq::Range range("tq_compress_append");
   if (!ctx || !k || !page_pool || !page_table || !cold_len) return TQ_ERR_INVALID_ARG;
   if (B <= 0 || Hkv <= 0 || n_new < 0 || max_pages <= 0 || pool_pages <= 0)
     return TQ_ERR_INVALID_ARG;
@@ -258,6 +271,7 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype
                               int64_t pool_pages, const int32_t* page_table, int max_pages,
                               const int32_t* cold_len, float* out, void* workspace,
                               size_t ws_bytes, void* stream) {
+  tq::Range range("tq_decode_attention");
   return decode_common(ctx, q, q_dtype, B, Hq, Hkv, scale, k_hot, v_hot, W_max, nullptr, hot_len,
                        page_pool, pool_pages, page_table, max_pages, cold_len, nullptr, out,
                        workspace, ws_bytes, stream);
@@ -428,6 +442,7 @@ size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int Q, int64_t N, int k) {
 tq_status tq_score_topk(const tq_ctx* ctx, const float* queries, int Q, const uint8_t* db_pages,
                         int64_t N, int k, int32_t* out_ids, float* out_scores, void* workspace,
                         size_t ws_bytes, void* stream) {
+  tq::Range range("tq_score_topk");
   if (!ctx || !queries || !db_pages || !out_ids || !out_scores || !workspace)
     return TQ_ERR_INVALID_ARG;
   if (Q <= 0 || N <= 0 || k <= 0) return TQ_ERR_INVALID_ARG;
@@ -444,6 +459,13 @@ tq_status tq_set_profile_events(tq_ctx* ctx, void* ev_start, void* ev_stop) {
   if (!ctx || ((ev_start == nullptr) != (ev_stop == nullptr))) return TQ_ERR_INVALID_ARG;
   ctx->prof_start = ev_start;
   ctx->prof_stop = ev_stop;
+  return TQ_OK;
+}
+
+tq_status tq_set_wait_test(tq_ctx* ctx, int skip_unit, uint64_t limit_ns) {
+  if (!ctx || skip_unit < -1) return TQ_ERR_INVALID_ARG;
+  ctx->wait_skip_unit = skip_unit;
+  ctx->wait_ns = limit_ns;
   return TQ_OK;
 }
 

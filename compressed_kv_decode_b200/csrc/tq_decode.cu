@@ -110,6 +110,10 @@ struct Params {
   int gate_nsplit;     // hot slot ranges of GATE_TOK slots
   int32_t* cold_used;  // [B, Hq] out (gated form), or null
   DecodeFuse fuse;     // combine epilogue (fuse.r null: none)
+  // testing aid for the bounded waits: the cold unit whose copy is armed but
+  // not issued (-1: none), and the bound of every wait of the attention
+  int skip_unit;
+  unsigned long long wait_ns;
 };
 
 __device__ __forceinline__ int* unit_off(const Params& p) { return p.w.sched + 4; }
@@ -608,7 +612,7 @@ __global__ void __launch_bounds__(256) gate_kernel(Params p) {
 // 2. attention
 // ---------------------------------------------------------------------------
 template <int D, int G>
-__device__ __forceinline__ void issue_unit(const Params& p, int sg, int lu, int len, int page,
+__device__ __forceinline__ void issue_unit(const Params& p, int u, int sg, int lu, int len, int page,
                                            uint8_t* dst, uint32_t bar, int lane) {
   using C = Cfg<D, G>;
   const int bh = sg >> 1;
@@ -622,8 +626,9 @@ __device__ __forceinline__ void issue_unit(const Params& p, int sg, int lu, int 
         mbar_arrive_expect_tx(bar, 0);
       } else {
         mbar_arrive_expect_tx(bar, C::COLD_B);
-        bulk_g2s(d0, p.pool + static_cast<size_t>(page) * p.page_bytes + (lu & 1) * C::COLD_B,
-                 C::COLD_B, bar);
+        if (u != p.skip_unit)  // (testing aid: the skipped unit's wait runs out)
+          bulk_g2s(d0, p.pool + static_cast<size_t>(page) * p.page_bytes + (lu & 1) * C::COLD_B,
+                   C::COLD_B, bar);
       }
     }
     __syncwarp();
@@ -746,8 +751,8 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
   };
   auto fire_next = [&](int slot) {
     if (lane == 0) slot_page[slot] = nx_page;
-    issue_unit<D, G>(p, nx_sg, nx_lu, nx_len, nx_page, slots + slot * C::SLOT, smem_u32(&bars[slot]),
-                     lane);
+    issue_unit<D, G>(p, iu, nx_sg, nx_lu, nx_len, nx_page, slots + slot * C::SLOT,
+                     smem_u32(&bars[slot]), lane);
     ++iu;
     ++ilu;
   };
@@ -877,6 +882,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
   };
 
   const uint32_t pb_addr = smem_u32(pbuf);
+  const unsigned long long wait_ns = p.wait_ns ? p.wait_ns : 2000000000ull;
   const uint32_t msk = 0x01010101u << g;  // this lane's token in every plane byte
   const uint32_t l4 = static_cast<uint32_t>(lane) * 4u;
   const char* lut = reinterpret_cast<const char*>(g_vlut);
@@ -885,11 +891,11 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
     const int slot = k % C::NSLOT;
     const uint32_t parity = static_cast<uint32_t>(k / C::NSLOT) & 1u;
     uint8_t* sb = slots + slot * C::SLOT;
-    if (!mbar_wait_bounded(smem_u32(&bars[slot]), parity)) {
+    if (!mbar_wait_bounded(smem_u32(&bars[slot]), parity, wait_ns)) {
       if (lane == 0) report(p.err, TQ_ERR_TIMEOUT);
       // let copies already in flight land before the CTA can exit
       for (int s = 0; s < C::NSLOT; ++s)
-        mbar_wait_bounded(smem_u32(&bars[s]), static_cast<uint32_t>((k + s) / C::NSLOT) & 1u);
+        mbar_wait_bounded(smem_u32(&bars[s]), static_cast<uint32_t>((k + s) / C::NSLOT) & 1u, wait_ns);
       return;
     }
     if ((sg & 1) == 0) {
@@ -900,12 +906,12 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
         const uint8_t* bp = sb + mt * C::BLK;
-        // integer accumulators: planes H, L (key) and QJL, split in independent chains
-        int ah[C::NT][4], al[C::NT][4], aq0[C::NT][4], aq1[C::NT][4];
+        // integer accumulators: key planes H and L, and the QJL plane
+        int ak[C::NT][4], aq[C::NT][4];
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) ah[nt][e] = al[nt][e] = aq0[nt][e] = aq1[nt][e] = 0;
+          for (int e = 0; e < 4; ++e) ak[nt][e] = aq[nt][e] = 0;
 #pragma unroll
         for (int kap = 0; kap < C::KK; ++kap) {
           // words for indices 32 kap + 4c .. (tokens 0-7, 8-15) and 32 kap + 16 + 4c ..
@@ -917,12 +923,9 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
             const uint32_t* bH = bfr + ((0 * C::KK + kap) * C::NT + nt) * 2;
             const uint32_t* bL = bfr + ((1 * C::KK + kap) * C::NT + nt) * 2;
             const uint32_t* bQ = bfr + ((2 * C::KK + kap) * C::NT + nt) * 2;
-            imma_u8s8(ah[nt], wh.x & msk, wh.y & msk, wh.z & msk, wh.w & msk, bH[0], bH[1]);
-            imma_u8s8(al[nt], wl.x & msk, wl.y & msk, wl.z & msk, wl.w & msk, bL[0], bL[1]);
-            if (kap & 1)
-              imma_u8s8(aq1[nt], wq.x & msk, wq.y & msk, wq.z & msk, wq.w & msk, bQ[0], bQ[1]);
-            else
-              imma_u8s8(aq0[nt], wq.x & msk, wq.y & msk, wq.z & msk, wq.w & msk, bQ[0], bQ[1]);
+            imma_u8s8(ak[nt], wh.x & msk, wh.y & msk, wh.z & msk, wh.w & msk, bH[0], bH[1]);
+            imma_u8s8(ak[nt], wl.x & msk, wl.y & msk, wl.z & msk, wl.w & msk, bL[0], bL[1]);
+            imma_u8s8(aq[nt], wq.x & msk, wq.y & msk, wq.z & msk, wq.w & msk, bQ[0], bQ[1]);
           }
         }
         // (n, gamma) of tokens g and g + 8 of the block
@@ -933,10 +936,10 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt) {
           // columns 2c, 2c+1: the hi and lo bytes of head c's weights
-          const float vk0 = static_cast<float>((ah[nt][0] + al[nt][0]) * 256 + ah[nt][1] + al[nt][1]);
-          const float vk1 = static_cast<float>((ah[nt][2] + al[nt][2]) * 256 + ah[nt][3] + al[nt][3]);
-          const float vq0 = static_cast<float>((aq0[nt][0] + aq1[nt][0]) * 256 + aq0[nt][1] + aq1[nt][1]);
-          const float vq1 = static_cast<float>((aq0[nt][2] + aq1[nt][2]) * 256 + aq0[nt][3] + aq1[nt][3]);
+          const float vk0 = static_cast<float>(ak[nt][0] * 256 + ak[nt][1]);
+          const float vk1 = static_cast<float>(ak[nt][2] * 256 + ak[nt][3]);
+          const float vq0 = static_cast<float>(aq[nt][0] * 256 + aq[nt][1]);
+          const float vq1 = static_cast<float>(aq[nt][2] * 256 + aq[nt][3]);
           sv[nt * 8 + 2 * mt] = fmaf(f0.y, fmaf(uq[nt], vq0, cq[nt]), fmaf(uk[nt], vk0, ck[nt])) * f0.x;
           sv[nt * 8 + 2 * mt + 1] = fmaf(f1.y, fmaf(uq[nt], vq1, cq[nt]), fmaf(uk[nt], vk1, ck[nt])) * f1.x;
         }
@@ -1429,6 +1432,8 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
   p.alpha = std::sqrt(3.14159265358979323846f / 2.0f) / static_cast<float>(ctx->cfg.qjl_dim);
   for (int k = 0; k < 8; ++k) p.vc[k] = ctx->cb.val_c[k];
   p.err = ctx->dev.err;
+  p.skip_unit = ctx->wait_skip_unit;
+  p.wait_ns = ctx->wait_ns;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 128) {
     switch (G) {

@@ -87,6 +87,8 @@ struct tq_ctx {
   void* dev_block;  // single allocation holding every device table
   void* prof_start; // optional cudaEvent_t pair around the main kernel
   void* prof_stop;
+  int wait_skip_unit;         // testing aid: cold unit whose copy is not issued (-1: none)
+  unsigned long long wait_ns; // testing aid: bound of the attention's waits (0: default)
 };
 
 namespace tq {

@@ -51,8 +51,9 @@
 extern "C" {
 #endif
 
-/* Version of the cold-page storage format below. */
-#define TQ_LAYOUT_VERSION 1
+/* Version of the cold-page storage format (tq_page_bytes).  2: pages with
+ * values in 16-token blocks with bit-sliced key planes. */
+#define TQ_LAYOUT_VERSION 2
 /* Token slots per cold page. */
 #define TQ_PAGE_TOKENS 128
 
@@ -114,25 +115,45 @@ TQ_API tq_status tq_get_params(const tq_ctx* ctx, float* rot, float* qjl, float*
 /*
  * Bytes of one cold page (TQ_PAGE_TOKENS token slots).  with_values = 1: key
  * and value records (15104 B at d=128, 7936 B at d=64); 0: keys only, as used
- * by a search database (6656 B, 3584 B).  Layout, sections in this order,
- * each starting on a 16-byte boundary:
+ * by a search database (6656 B, 3584 B).  Format version TQ_LAYOUT_VERSION.
+ * Multi-byte fields are little endian; fp16 fields are IEEE binary16.  A key
+ * record is a 2-bit code per coordinate (sign s, magnitude index u of the
+ * level +-key_c[u]), a QJL sign bit per sketch index (1: (S r)_i < 0), the
+ * norm n and the residual norm gamma; a value record is a 4-bit code per
+ * coordinate, s << 3 | u (level +-val_c[u]), and the value norm.  Coordinates
+ * are those of the rotated domain (x_rot = Pi x).
+ *
+ * Pages with values: 8 blocks of 16 token slots (slot = 16 kb + t), each
+ * 12 d + 2 m + 96 bytes (m = qjl_dim):
+ *   KH  at 0            key plane H, 2 d bytes
+ *   KL  at 2 d          key plane L, 2 d bytes
+ *   QS  at 4 d          QJL sign plane, 2 m bytes
+ *   VC  at 4 d + 2 m    value codes, 8 d bytes
+ *   NK  at 12 d + 2 m   per token t, at + 4 t: fp16 n, then fp16 gamma
+ *   VN  at 12 d + 2m + 64   per token t, at + 2 t: fp16 value norm
+ * The key code of a coordinate is the index 2 H + L of its level in ascending
+ * order (-c1, -c0, +c0, +c1): H = 1 - s, L = s XOR u.  In a plane (KH and KL
+ * over coordinates j < d, QS over sketch indices j < m) the bit of token t is
+ * bit t mod 8 of the byte at
+ *     16 (4 (j / 32) + (j / 4) mod 4) + 4 (2 ((j / 16) mod 2) + t / 8) + j mod 4,
+ * so a 32-bit word holds 4 consecutive indices x 8 tokens.  In VC, the byte
+ * of coordinate j for the token pair (2q, 2q + 1) of the block holds the even
+ * token's code in its low nibble and sits at
+ *     (i / 4) 512 + (4 g + c) 16 + (i mod 4) 4 + jh + 2 th,
+ * i = j / 16, g = j mod 8, jh = (j mod 16) / 8, c = q mod 4, th = q / 4 (the
+ * word at (4 g + c) 16 + (i mod 4) 4 holds coordinates (g, g + 8) x token
+ * pairs (c, c + 4)).
+ *
+ * Keys-only pages: sections in this order, each starting on a 16-byte
+ * boundary:
  *   KC  key codes        128 x d/4 B
  *   QS  QJL sign bits    128 x m/8 B
- *   VC  value codes      64 x d B      (values pages only)
  *   KN  key norm n       128 x fp16
  *   KG  residual norm    128 x fp16
- *   VN  value norm       128 x fp16    (values pages only)
- * Key code word w (u32, little endian, w < d/16) of a token holds coordinates
+ * Key code word w (u32, w < d/16) of a token holds coordinates
  * j = 16w + 8h + 2i + e (h, e in {0,1}, i < 4) with the sign bit at
  * 16h + 15 - 4i - e and the magnitude bit at 16h + 13 - 4i - e.  QJL word w
- * (w < m/32) holds sketch index 32w + 16h + r (r < 16) at bit 16h + 15 - r;
- * a set bit means (S r)_i < 0.  Value codes come in token pairs: the byte of
- * coordinate j in pair p holds code(2p, j) in its low nibble and
- * code(2p+1, j) in its high nibble; a code is sign << 3 | magnitude index.
- * The pair's d-byte block is cut in 8 chunks of d/8 bytes and chunk g
- * (coordinates g*d/8 ...) is stored at chunk position (g + 2*(p mod 4)) mod 8,
- * so that four consecutive pairs read chunk-wise hit distinct shared-memory
- * banks.  Coordinates are those of the rotated domain.
+ * (w < m/32) holds sketch index 32w + 16h + r (r < 16) at bit 16h + 15 - r.
  */
 TQ_API size_t tq_page_bytes(const tq_ctx* ctx, int with_values);
 
@@ -466,6 +487,19 @@ TQ_API tq_status tq_stage1_decode(const tq_ctx* ctx, int kind, int bits1, int bi
  * switches it off.  Not thread-safe: set it only while no other thread uses
  * the context. */
 TQ_API tq_status tq_set_profile_events(tq_ctx* ctx, void* ev_start, void* ev_stop);
+
+/* Testing aid for the bounded device waits (no counterpart on the pages).
+ * With skip_unit >= 0, the next decode calls (tq_decode_attention and its
+ * gated, Monarch and no-allocation forms) arm the copy of cold work unit
+ * skip_unit (64 tokens; units are numbered over all (batch, kv head)
+ * segments in order) without issuing it, so the wait for that unit can never
+ * complete; every wait of the attention kernel gives up after limit_ns
+ * nanoseconds (0: the default of 2 s).  The warp that owns the unit records
+ * TQ_ERR_TIMEOUT, lets its other copies land and returns; the call's outputs
+ * are then undefined, the context stays usable.  skip_unit = -1, limit_ns = 0
+ * restores normal operation.  Not thread-safe: set it only while no other
+ * thread uses the context. */
+TQ_API tq_status tq_set_wait_test(tq_ctx* ctx, int skip_unit, uint64_t limit_ns);
 
 /* Read and clear the context's device error word.  Synchronises with the
  * device; call it after the work of interest has completed. */

@@ -662,8 +662,8 @@ OR_API void or_encode(int d, int m, const double* pi, const double* S, const dou
                       int is_key, int32_t* sign, int32_t* mag, int32_t* qbits, double* n,
                       double* gamma, double* xrot_out, int threads) {
 #ifdef _OPENMP
-  if (threads > 0) omp_set_num_threads(threads);
-#pragma omp parallel
+  const int nthreads = threads > 0 ? threads : omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
 #endif
   {
     double* xr = (double*)malloc(sizeof(double) * d);
@@ -869,8 +869,8 @@ OR_API int or_attention_gated(int d, int m, const double* pi, const double* S,
   int G = Hq / Hkv;
   int err = 0;
 #ifdef _OPENMP
-  if (threads > 0) omp_set_num_threads(threads);
-#pragma omp parallel for schedule(dynamic) reduction(| : err)
+  const int nthreads = threads > 0 ? threads : omp_get_max_threads();
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic) reduction(| : err)
 #endif
   for (int s = 0; s < nsel; ++s) {
     int b = sel[2 * s], h = sel[2 * s + 1];
@@ -913,8 +913,8 @@ OR_API void or_topk(int d, int m, const double* pi, const double* S, const doubl
                     const double* queries, int Q, const uint8_t* db, size_t page_bytes, int64_t N,
                     int k, int32_t* out_ids, double* out_scores, int threads) {
 #ifdef _OPENMP
-  if (threads > 0) omp_set_num_threads(threads);
-#pragma omp parallel
+  const int nthreads = threads > 0 ? threads : omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
 #endif
   {
     double* qrot = (double*)malloc(sizeof(double) * d);

@@ -152,3 +152,34 @@ def test_repeat_calls_identical(O):
     a = gpu_out(tq, ctx, c)
     b = gpu_out(tq, ctx, c)
     assert np.array_equal(a, b)
+
+
+def test_bounded_wait_runs_out_and_reports_timeout(O):
+    """The testing hook arms the copy of cold unit 3 without issuing it: the
+    warp that owns the unit gives up after 1 ms, the call reports
+    TQ_ERR_TIMEOUT, the kernel returns (the stream synchronises), and the next
+    normal call on the same context matches the oracle.  No fault, trap or
+    endless wait is involved: the wait is bounded by the hook's limit."""
+    import time
+    cfg = W.DECODE["tinyllama"]
+    P = params_for(O, 64)
+    c = build(O, P, cfg["B"], cfg["Hq"], cfg["Hkv"], 64, [cfg["cold"]], [cfg["hot"]], cfg["hot"],
+              cfg["cold"] // 128, q_dtype=cfg["q_dtype"], seeds=cfg["seeds"], n_out=cfg["n_out"],
+              factor=cfg["factor"])
+    ctx = tq.Context(64, 0)
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_OK
+    tq.tq_set_wait_test(ctx.handle, 3, 1_000_000)
+    try:
+        t0 = time.perf_counter()
+        gpu_out(tq, ctx, c)
+        elapsed = time.perf_counter() - t0
+    finally:
+        tq.tq_set_wait_test(ctx.handle, -1, 0)
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_ERR_TIMEOUT
+    assert elapsed < 30.0
+    got = gpu_out(tq, ctx, c)
+    assert tq.tq_get_error(ctx.handle) == tq.TQ_OK
+    ref = oracle_out(O, P, c)
+    for (b, h), r in ref.items():
+        assert_close(got[b, h * c.G:(h + 1) * c.G], r, what="after the timeout, group %s" % ((b, h),))
+    ctx.close()
