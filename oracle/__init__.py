@@ -68,6 +68,9 @@ def lib():
                                          C.c_int, ip, ip, C.c_int, C.c_int, C.c_double, ip, dp,
                                          C.c_int]
         L.or_attention_gated.restype = C.c_int
+        L.or_cold_logits.argtypes = [C.c_int, C.c_int, dp, dp, dp, C.c_int, dp, C.c_double, u8,
+                                     sz, ip, C.c_int, dp]
+        L.or_cold_logits.restype = None
         L.or_topk.argtypes = [C.c_int, C.c_int, dp, dp, dp, dp, C.c_int, u8, sz, C.c_int64,
                               C.c_int, ip, dp, C.c_int]
         L.or_max_threads.restype = C.c_int
@@ -348,6 +351,23 @@ def attention(params, q, Hkv, scale, k_hot, v_hot, hot_len, pool, page_bytes, pa
                                   out.ctypes.data_as(C.POINTER(C.c_double)), threads)
     assert rc == 0
     return out, groups, opened
+
+
+def cold_logits(params, q, scale, pool, page_bytes, pages, cold_len):
+    """Estimated cold scores of one (batch, kv head) group as the decode
+    attention forms them: q [G, d]; pages: the group's page-table row.
+    Returns [G, cold_len]."""
+    p = params
+    q, qp = _d(np.asarray(q).reshape(-1, p.d))
+    G = q.shape[0]
+    pg, pgp = _i(pages)
+    pi, pip = _d(p.pi32)
+    S, Sp = _d(p.S)
+    kc, kcp = _d(p.kc)
+    out = np.empty((G, int(cold_len)))
+    lib().or_cold_logits(p.d, p.m, pip, Sp, kcp, G, qp, scale, _u8(pool), page_bytes, pgp,
+                         int(cold_len), out.ctypes.data_as(C.POINTER(C.c_double)))
+    return out
 
 
 def topk(params, queries, db_pool, page_bytes, N, k, threads=0):

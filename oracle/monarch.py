@@ -23,14 +23,40 @@ Readings where the pages leave a step open:
   - The new token of a step is appended before attention, so it attends to
     itself (as in standard decoding).
   - The gate is the oracle attention's: per query head, on the raw hot scores.
+  - Attention-weighted promotion with stickiness (section "Wie es
+    funktioniert": tokens with high attention move back to the hot region,
+    with a sticking mechanism against thrashing; section "Vereinfachte
+    Decode-Schleife": cold tokens read in a step are moved to the hot region
+    for the next step; section "Wie man es ausprobiert": promotion threshold
+    0.15, sticky threshold 3).  A cold position's weight in a step is its
+    largest softmax probability over the query heads of the sequence that
+    read the cold tier (a position, not a kv head, moves: all kv heads of a
+    sequence share one hot window).  A weight at or above the threshold
+    counts the step, a weight below it resets the count (consecutive
+    steps); a position whose count reaches the sticky threshold moves back
+    after the step's attention: its decompressed key and value (n Pi^T c_hat,
+    the residual's sketch being no vector, and n_v Pi^T c_hat_v, rounded to
+    fp16) join the hot window of every kv head as its newest tokens, its
+    cold slot is masked (attention skips it from then on) and its count
+    returns to 0.  At most max_per_step positions move per step, in
+    increasing position order, and never more than leave one free ring slot
+    for the next step's token; the others keep their counts.  Eviction runs
+    after promotion.
 
 Parity status: pinned by ``tests/test_oracle_monarch.py`` (window
 invariant, token placement against the appended sequence, attention with a
-shut gate against torch's scaled_dot_product_attention).
+shut gate against torch's scaled_dot_product_attention; the promotion path:
+its attention against the oracle's C attention and against SDPA without the
+masked tokens, counting, moving, masking and the per-step and ring limits).
 """
 import numpy as np
 
-from . import attention, encode, pack, page_layout
+from . import attention, cold_logits, encode, pack, page_layout, unpack
+
+
+def _f16(a):
+    """Round to the nearest fp16 value (ties to even), widened to fp64."""
+    return np.asarray(a, np.float64).astype(np.float16).astype(np.float64)
 
 
 class MonarchCache:
@@ -38,7 +64,9 @@ class MonarchCache:
     values widened to fp64) and cold records in the oracle's page pool."""
 
     def __init__(self, params, B, Hkv, window, evict_block, page_table, cold_len=None,
-                 pool=None, hot_k=None, hot_v=None):
+                 pool=None, hot_k=None, hot_v=None, promotion=None, W_max=None):
+        """promotion: None, or dict(threshold, sticky, max_per_step); W_max:
+        the ring size (needed with promotion)."""
         self.P = params
         self.B, self.Hkv, self.d = B, Hkv, params.d
         self.window, self.E = int(window), int(evict_block)
@@ -51,6 +79,11 @@ class MonarchCache:
                          else np.asarray(cold_len, np.int32).copy())
         # hot[b][h]: list of (k, v) rows, oldest first
         self.hot = [[[] for _ in range(Hkv)] for _ in range(B)]
+        self.promo = promotion
+        self.W_max = W_max
+        cap = self.table.shape[-1] * 128
+        self.cold_mask = np.zeros((B, cap), bool)  # moved back: skipped by attention
+        self.counts = np.zeros((B, cap), np.int32)   # consecutive counted steps
         if hot_k is not None:
             for b in range(B):
                 for h in range(Hkv):
@@ -91,6 +124,85 @@ class MonarchCache:
         opened = None if threshold is None else res[2].reshape(self.B, self.Hkv * G)
         return out, opened
 
+    def _cold_values(self, b, h, cl):
+        """Reconstructed cold values n_v Pi^T c_hat_v [cl, d] of group (b, h)."""
+        t = np.arange(cl)
+        rec = unpack(self.pool, self.page_bytes, self.d, self.P.m, True, self.table[b, h, t // 128],
+                     t % 128)
+        chat = np.where(rec["vcode"] >> 3, -1.0, 1.0) * self.P.vc[rec["vcode"] & 7]
+        return rec["vn"][:, None] * (chat @ self.P.pi32)
+
+    def attend_weights(self, q, scale, threshold=None):
+        """The attention of attend() computed step by step in fp64 (cold scores
+        from the oracle's scorer, values n_v Pi^T c_hat_v, one softmax per query
+        head over its hot tokens and, where its gate opens, the cold tokens not
+        moved back), also returning per sequence the largest weight of every
+        cold position over the query heads that read the cold tier."""
+        B, Hq, d = q.shape
+        G = Hq // self.Hkv
+        out = np.zeros((B, Hq, d))
+        opened = np.zeros((B, Hq), np.int32)
+        wmax = []
+        for b in range(B):
+            cl, hl = int(self.cold_len[b]), self.hot_len(b)
+            live = ~self.cold_mask[b, :cl]
+            w = np.zeros(cl)
+            for h in range(self.Hkv):
+                qg = np.asarray(q[b, h * G:(h + 1) * G], np.float64)
+                kh = np.array([kv[0] for kv in self.hot[b][h]]).reshape(hl, d)
+                vh = np.array([kv[1] for kv in self.hot[b][h]]).reshape(hl, d)
+                raw = qg @ kh.T
+                cs = cold_logits(self.P, qg, scale, self.pool, self.page_bytes, self.table[b, h], cl) \
+                    if cl else np.zeros((G, 0))
+                cv = self._cold_values(b, h, cl) if cl else np.zeros((0, d))
+                for g in range(G):
+                    gmax = raw[g].max() if hl else -np.inf
+                    op = threshold is None or gmax < threshold
+                    opened[b, h * G + g] = op
+                    lc = cs[g][live] if op else np.zeros(0)
+                    logits = np.concatenate([lc, raw[g] * scale])
+                    if len(logits) == 0:
+                        continue
+                    e = np.exp(logits - logits.max())
+                    p = e / e.sum()
+                    out[b, h * G + g] = p @ np.concatenate([cv[live] if op else np.zeros((0, d)), vh])
+                    if op:
+                        wc = np.zeros(cl)
+                        wc[live] = p[:len(lc)]
+                        w = np.maximum(w, wc)
+            wmax.append(w)
+        return out, opened, wmax
+
+    def promote(self, wmax):
+        """Count, then move back the positions whose count reached the sticky
+        threshold (see the module docstring); returns the moved positions per
+        sequence."""
+        pr = self.promo
+        moved = []
+        for b in range(self.B):
+            cl = int(self.cold_len[b])
+            live = ~self.cold_mask[b, :cl]
+            hit = live & (wmax[b] >= pr["threshold"])
+            self.counts[b, :cl] = np.where(hit, np.minimum(self.counts[b, :cl] + 1, 255), 0)
+            cand = np.nonzero(live & (self.counts[b, :cl] >= pr["sticky"]))[0]
+            room = max(0, self.W_max - 1 - self.hot_len(b))
+            chosen = cand[:min(int(pr["max_per_step"]), room)]
+            for h in range(self.Hkv):
+                if len(chosen) == 0:
+                    break
+                rec = unpack(self.pool, self.page_bytes, self.d, self.P.m, True,
+                             self.table[b, h, chosen // 128], chosen % 128)
+                ck = np.where(rec["sign"] == 1, -1.0, 1.0) * self.P.kc[rec["mag"]]
+                cv = np.where(rec["vcode"] >> 3, -1.0, 1.0) * self.P.vc[rec["vcode"] & 7]
+                kd = _f16(rec["n"][:, None] * (ck @ self.P.pi32))
+                vd = _f16(rec["vn"][:, None] * (cv @ self.P.pi32))
+                for i in range(len(chosen)):
+                    self.hot[b][h].append((kd[i], vd[i]))
+            self.cold_mask[b, chosen] = True
+            self.counts[b, chosen] = 0
+            moved.append(chosen)
+        return moved
+
     def evict(self):
         """Move the oldest E hot tokens of every sequence holding at least
         window + E of them to the cold pages; returns how many per sequence."""
@@ -115,8 +227,12 @@ class MonarchCache:
         return moved
 
     def step(self, q, k_new, v_new, scale, threshold=None):
-        """One decode step: append, attend, evict."""
+        """One decode step: append, attend, (promote,) evict."""
         self.append(k_new, v_new)
-        out, opened = self.attend(q, scale, threshold)
+        if self.promo is None:
+            out, opened = self.attend(q, scale, threshold)
+        else:
+            out, opened, wmax = self.attend_weights(q, scale, threshold)
+            self.promote(wmax)
         self.evict()
         return out, opened

@@ -747,6 +747,41 @@ static double key_score(int d, int m, const double* qrot, const double* sq, cons
   return n * (ip + or_qjl_estimate(m, sq, qbits, gamma)) * scale;
 }
 
+/* Estimated scores of the cold tokens of one (batch, kv head) group for G
+ * query heads, exactly as the decode attention forms them (key_score with the
+ * scale applied): q [G, d] (original domain), pages / cold_len as the group's
+ * page table row and length; out [G, cold_len]. */
+OR_API void or_cold_logits(int d, int m, const double* pi, const double* S, const double* kcpos,
+                           int G, const double* q, double scale, const uint8_t* pool,
+                           size_t page_bytes, const int32_t* pages, int cold_len, double* out) {
+  double* qrot = (double*)malloc(sizeof(double) * (size_t)G * d);
+  double* sq = (double*)malloc(sizeof(double) * (size_t)G * m);
+  int32_t* sign = (int32_t*)malloc(sizeof(int32_t) * d);
+  int32_t* mag = (int32_t*)malloc(sizeof(int32_t) * d);
+  int32_t* qb = (int32_t*)malloc(sizeof(int32_t) * m);
+  for (int h = 0; h < G; ++h) {
+    for (int j = 0; j < d; ++j) {
+      double a = 0.0;
+      for (int k = 0; k < d; ++k) a += pi[(size_t)j * d + k] * q[(size_t)h * d + k];
+      qrot[(size_t)h * d + j] = a;
+    }
+    for (int i = 0; i < m; ++i) {
+      double a = 0.0;
+      for (int j = 0; j < d; ++j) a += S[(size_t)i * d + j] * qrot[(size_t)h * d + j];
+      sq[(size_t)h * m + i] = a;
+    }
+  }
+  for (int t = 0; t < cold_len; ++t) {
+    const uint8_t* pg = pool + (size_t)pages[t / PAGE_TOKENS] * page_bytes;
+    double n, gamma;
+    or_unpack_key(pg, d, m, 1, t % PAGE_TOKENS, sign, mag, qb, &n, &gamma);
+    for (int h = 0; h < G; ++h)
+      out[(size_t)h * cold_len + t] = key_score(d, m, qrot + (size_t)h * d, sq + (size_t)h * m,
+                                                 kcpos, sign, mag, qb, n, gamma, scale);
+  }
+  free(qrot); free(sq); free(sign); free(mag); free(qb);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Decode attention over one (batch, kv head) group [MON "Vereinfachte      */
 /* Decode-Schleife": hot scores, cold scores, softmax, aggregation].         */
