@@ -21,12 +21,18 @@ TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
 TQ_INPUT_ROTATED = 1
 TQ_PAGE_TOKENS = 128
 TQ_NOALLOC_SCRATCH_BYTES = 8 << 20
+TQ_PROMOTE_MAX_PER_STEP = 64
 
 
 class TQError(RuntimeError):
     def __init__(self, status, what=""):
         self.status = status
         super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+
+
+class tq_promotion(C.Structure):
+    _fields_ = [("threshold", C.c_float), ("sticky", C.c_int), ("max_per_step", C.c_int),
+                ("cold_mask", C.c_void_p), ("counts", C.c_void_p), ("logits", C.c_void_p)]
 
 
 class tq_config(C.Structure):
@@ -76,6 +82,12 @@ def lib():
                                       C.c_int, i32p, C.c_float, C.c_int, C.c_int, i32p, f32p, vp,
                                       C.c_size_t, vp]
         L.tq_monarch_step.restype = C.c_int
+        L.tq_monarch_step_promote.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, C.c_int,
+                                              C.c_float, vp, vp, vp, vp, C.c_int, i32p, i32p,
+                                              u8p, C.c_int64, i32p, C.c_int, i32p, C.c_float,
+                                              C.c_int, C.c_int, C.POINTER(tq_promotion), i32p,
+                                              f32p, vp, C.c_size_t, vp]
+        L.tq_monarch_step_promote.restype = C.c_int
         L.tq_stage1_code_bytes.argtypes = [vp, C.c_int, C.c_int, C.c_int]
         L.tq_stage1_code_bytes.restype = C.c_size_t
         L.tq_stage1_encode.argtypes = [vp, C.c_int, C.c_int, C.c_int, f32p, C.c_int64, u8p, vp,
@@ -282,6 +294,32 @@ def tq_monarch_step(ctx, q, k_new, v_new, k_hot, v_hot, hot_start, hot_len, page
         float(threshold), int(window), int(evict_block), _ptr(cold_used), _ptr(out),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
         "tq_monarch_step")
+
+
+def tq_monarch_step_promote(ctx, q, k_new, v_new, k_hot, v_hot, hot_start, hot_len, page_pool,
+                            page_table, cold_len, threshold, window, evict_block, promo, out,
+                            workspace, Hkv, scale=0.0, cold_used=None, stream=None):
+    """tq_monarch_step with Monarch's promotion.  promo: dict(threshold,
+    sticky, max_per_step, cold_mask (int32 [B, max_pages * 4]), counts (uint8
+    [B, max_pages * 128]), logits (fp32 [B, Hq, max_pages * 128])), device
+    tensors updated in place; None runs tq_monarch_step."""
+    _require_cuda(q, k_new, v_new, k_hot, v_hot, hot_start, hot_len, page_pool, page_table,
+                  cold_len, out, workspace, cold_used)
+    B, Hq, _ = q.shape
+    W_max = k_hot.shape[2]
+    pr = None
+    if promo is not None:
+        _require_cuda(promo["cold_mask"], promo["counts"], promo["logits"])
+        pr = C.byref(tq_promotion(float(promo["threshold"]), int(promo["sticky"]),
+                                  int(promo["max_per_step"]), _ptr(promo["cold_mask"]),
+                                  _ptr(promo["counts"]), _ptr(promo["logits"])))
+    _check(lib().tq_monarch_step_promote(
+        ctx, _ptr(q), _dtype_code(q), B, Hq, Hkv, float(scale), _ptr(k_new), _ptr(v_new),
+        _ptr(k_hot), _ptr(v_hot), W_max, _ptr(hot_start), _ptr(hot_len), _ptr(page_pool),
+        page_pool.shape[0], _ptr(page_table), page_table.shape[-1], _ptr(cold_len),
+        float(threshold), int(window), int(evict_block), pr, _ptr(cold_used), _ptr(out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+        "tq_monarch_step_promote")
 
 
 def tq_tensor_cache_workspace_bytes(ctx, B, Hq, Hkv, W):

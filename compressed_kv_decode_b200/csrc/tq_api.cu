@@ -303,6 +303,29 @@ tq_status tq_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, in
                           int max_pages, int32_t* cold_len, float threshold, int window,
                           int evict_block, int32_t* cold_used, float* out, void* workspace,
                           size_t ws_bytes, void* stream) {
+  return tq_monarch_step_promote(ctx, q, q_dtype, B, Hq, Hkv, scale, k_new, v_new, k_hot, v_hot,
+                                 W_max, hot_start, hot_len, page_pool, pool_pages, page_table,
+                                 max_pages, cold_len, threshold, window, evict_block, nullptr,
+                                 cold_used, out, workspace, ws_bytes, stream);
+}
+
+tq_status tq_monarch_step_promote(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B,
+                                  int Hq, int Hkv, float scale, const void* k_new,
+                                  const void* v_new, void* k_hot, void* v_hot, int W_max,
+                                  int32_t* hot_start, int32_t* hot_len, uint8_t* page_pool,
+                                  int64_t pool_pages, const int32_t* page_table, int max_pages,
+                                  int32_t* cold_len, float threshold, int window,
+                                  int evict_block, const tq_promotion* promo,
+                                  int32_t* cold_used, float* out, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+  tq::Range range("tq_monarch_step");
+  if (promo) {
+    if (!(promo->threshold > 0.0f) || !std::isfinite(promo->threshold) || promo->sticky < 1 ||
+        promo->max_per_step < 1 || promo->max_per_step > TQ_PROMOTE_MAX_PER_STEP ||
+        !promo->cold_mask || !promo->counts || !promo->logits ||
+        !tq::aligned(promo->cold_mask, 4) || !tq::aligned(promo->logits, 4))
+      return TQ_ERR_INVALID_ARG;
+  }
   if (!ctx || !q || !out || !workspace || !k_hot || !v_hot || !hot_start || !hot_len)
     return TQ_ERR_INVALID_ARG;
   if (!page_pool || !page_table || !cold_len || pool_pages <= 0 || max_pages <= 0)
@@ -325,7 +348,7 @@ tq_status tq_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, in
   return static_cast<tq_status>(tq::launch_monarch_step(
       ctx, q, q_dtype, B, Hq, Hkv, scale, k_new, v_new, k_hot, v_hot, W_max, hot_start, hot_len,
       page_pool, pool_pages, page_table, max_pages, cold_len, threshold, window, evict_block,
-      cold_used, out, workspace, ws_bytes, stream));
+      promo, cold_used, out, workspace, ws_bytes, stream));
 }
 
 size_t tq_tensor_cache_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int W) {

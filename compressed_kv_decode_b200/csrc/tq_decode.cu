@@ -114,6 +114,7 @@ struct Params {
   // not issued (-1: none), and the bound of every wait of the attention
   int skip_unit;
   unsigned long long wait_ns;
+  DecodePromo promo;  // Monarch's promotion (promo.logits null: none)
 };
 
 __device__ __forceinline__ int* unit_off(const Params& p) { return p.w.sched + 4; }
@@ -902,6 +903,14 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
       // ---------------- cold unit: 64 tokens, 4 blocks ----------------
       const int page = slot_page[slot];
       const int nv = (page >= 0 && page < p.pool_pages) ? min(COLD_TOK, len - lu * COLD_TOK) : 0;
+      // tokens of the unit that take part: inside the sequence and not moved
+      // back to the hot window (Monarch's promotion)
+      uint64_t valid = nv >= COLD_TOK ? ~0ull : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
+      const int b_seq = (sg >> 1) / p.Hkv;
+      if (p.promo.cold_mask) {
+        const uint32_t* mw = p.promo.cold_mask + static_cast<size_t>(b_seq) * p.max_pages * 4 + 2 * lu;
+        valid &= ~(static_cast<uint64_t>(mw[0]) | (static_cast<uint64_t>(mw[1]) << 32));
+      }
       float sv[C::NT * 8];
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
@@ -943,12 +952,25 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
           sv[nt * 8 + 2 * mt] = fmaf(f0.y, fmaf(uq[nt], vq0, cq[nt]), fmaf(uk[nt], vk0, ck[nt])) * f0.x;
           sv[nt * 8 + 2 * mt + 1] = fmaf(f1.y, fmaf(uq[nt], vq1, cq[nt]), fmaf(uk[nt], vk1, ck[nt])) * f1.x;
         }
-        if (nv < COLD_TOK) {  // tokens past the sequence
+        if (valid != ~0ull) {  // tokens past the sequence or moved back
           const int t0 = 16 * mt + g;
 #pragma unroll
           for (int nt = 0; nt < C::NT; ++nt) {
-            if (t0 >= nv) sv[nt * 8 + 2 * mt] = NEG_INF;
-            if (t0 + 8 >= nv) sv[nt * 8 + 2 * mt + 1] = NEG_INF;
+            if (!((valid >> t0) & 1ull)) sv[nt * 8 + 2 * mt] = NEG_INF;
+            if (!((valid >> (t0 + 8)) & 1ull)) sv[nt * 8 + 2 * mt + 1] = NEG_INF;
+          }
+        }
+        if (p.promo.logits) {  // every cold logit, for the promotion
+          const int kvh = (sg >> 1) % p.Hkv, cap = p.max_pages * TQ_PAGE_TOKENS;
+          const int pos = lu * COLD_TOK + 16 * mt + g;
+#pragma unroll
+          for (int nt = 0; nt < C::NT; ++nt) {
+            const int h = c + 4 * nt;
+            if (h < G) {
+              float* lg = p.promo.logits + (static_cast<size_t>(b_seq) * p.Hq + kvh * G + h) * cap;
+              lg[pos] = sv[nt * 8 + 2 * mt];
+              lg[pos + 8] = sv[nt * 8 + 2 * mt + 1];
+            }
           }
         }
       }
@@ -964,9 +986,9 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
           const int h = c + 4 * nt;
           if (h < G) {
             float p0 = sv[nt * 8 + 2 * mt] * nv0, p1 = sv[nt * 8 + 2 * mt + 1] * nv1;
-            if (nv < COLD_TOK) {
-              if (t0 >= nv) p0 = 0.0f;
-              if (t1 >= nv) p1 = 0.0f;
+            if (valid != ~0ull) {
+              if (!((valid >> t0) & 1ull)) p0 = 0.0f;
+              if (!((valid >> t1) & 1ull)) p1 = 0.0f;
             }
             reinterpret_cast<__half*>(pbuf)[t0 * 8 + h] = __float2half_rn(p0);
             reinterpret_cast<__half*>(pbuf)[t1 * 8 + h] = __float2half_rn(p1);
@@ -1246,6 +1268,13 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(Params p) {
       res = (den > 0.0f) ? ((fc > 0.0f ? oc * fc : 0.0f) + (fh > 0.0f ? oh * fh : 0.0f)) / den : 0.0f;
     }
     const size_t oi = (static_cast<size_t>(b) * p.Hq + kvh * G + g) * D + j;
+    if (p.promo.lse && j == 0) {  // log-sum-exp of the head's attended tokens (promotion)
+      const float den = (Mx != NINF) ? Lc * ((Lc > 0.0f) ? exp2f(Mc - Mx) : 0.0f) +
+                                           Lh * ((Lh > 0.0f) ? exp2f(Mh - Mx) : 0.0f)
+                                     : 0.0f;
+      p.promo.lse[static_cast<size_t>(b) * p.Hq + kvh * G + g] =
+          (open && den > 0.0f) ? Mx + log2f(den) : __builtin_huge_valf();
+    }
     if (p.fuse.r) {  // out += sigmoid(gate) r
       const float sg = 1.0f / (1.0f + expf(-p.fuse.gate[kvh * G + g]));
       res = fmaf(sg, p.fuse.r[oi], res);
@@ -1393,7 +1422,8 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
                   const int32_t* hot_start, const int32_t* hot_len, const uint8_t* pool,
                   int64_t pool_pages, const int32_t* page_table, int max_pages,
                   const int32_t* cold_len, const DecodeGate* gate, float* out, void* ws,
-                  size_t ws_bytes, void* stream, const DecodeFuse* fuse) {
+                  size_t ws_bytes, void* stream, const DecodeFuse* fuse,
+                  const DecodePromo* promo) {
   const int d = ctx->cfg.head_dim;
   const int G = Hq / Hkv;
   const PageLayout L = page_layout(d, ctx->cfg.qjl_dim, true);
@@ -1412,6 +1442,7 @@ int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int
   p.hot_len = hot_len;
   p.hot_start = hot_start;
   if (fuse) p.fuse = *fuse;
+  if (promo) p.promo = *promo;
   if (gate) {
     p.gated = 1;
     p.gate_thr = gate->threshold;

@@ -124,12 +124,24 @@ struct DecodeFuse {
 };
 
 // Launchers (defined in the .cu files).  Return a tq_status.
+// Inputs and outputs of Monarch's promotion for the decode (all device):
+// cold positions moved back are skipped; the attention writes every cold
+// logit (log2 domain, scale folded in) and the combine the log-sum-exp of each
+// query head over the tokens it attended (+inf where its gate kept it off the
+// cold tier, or where it attended nothing).
+struct DecodePromo {
+  const uint32_t* cold_mask;  // [B][max_pages * 4] bit p % 32 of word p / 32: position p skipped
+  float* logits;              // [B][Hq][max_pages * 128]
+  float* lse;                 // [B][Hq]
+};
+
 int launch_decode(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq, int Hkv,
                   float scale, const void* k_hot, const void* v_hot, int W_max,
                   const int32_t* hot_start, const int32_t* hot_len, const uint8_t* pool,
                   int64_t pool_pages, const int32_t* page_table, int max_pages,
                   const int32_t* cold_len, const DecodeGate* gate, float* out, void* ws,
-                  size_t ws_bytes, void* stream, const DecodeFuse* fuse = nullptr);
+                  size_t ws_bytes, void* stream, const DecodeFuse* fuse = nullptr,
+                  const DecodePromo* promo = nullptr);
 size_t decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_pages, int W_max);
 
 int launch_compress(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype, int flags,
@@ -150,8 +162,8 @@ int launch_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int 
                         void* v_hot, int W_max, int32_t* hot_start, int32_t* hot_len,
                         uint8_t* pool, int64_t pool_pages, const int32_t* page_table,
                         int max_pages, int32_t* cold_len, float threshold, int window,
-                        int evict_block, int32_t* cold_used, float* out, void* ws,
-                        size_t ws_bytes, void* stream);
+                        int evict_block, const tq_promotion* promo, int32_t* cold_used,
+                        float* out, void* ws, size_t ws_bytes, void* stream);
 size_t tensor_cache_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int W);
 int launch_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
                              int Hkv, float scale, const void* k_new, const void* v_new,

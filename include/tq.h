@@ -293,6 +293,56 @@ TQ_API tq_status tq_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dt
                                  float threshold, int window, int evict_block,
                                  int32_t* cold_used, float* out, void* workspace,
                                  size_t ws_bytes, void* stream);
+/*
+ * Monarch's attention-weighted promotion with stickiness ("Monarch v3", section
+ * "Wie es funktioniert": tokens with high attention move back to the hot
+ * region, with a sticking mechanism against thrashing; section "Vereinfachte
+ * Decode-Schleife": cold tokens read in a step move to the hot region for the
+ * next step; section "Wie man es ausprobiert": thresholds 0.15 and 3).
+ * After a step's attention, a cold position's weight is its largest softmax
+ * probability over the query heads of its sequence that read the cold tier.
+ * A weight >= threshold counts the step, a smaller one resets the count (the
+ * count is of consecutive steps).  A position whose count reaches sticky
+ * moves back: its decompressed key and value -- n Pi^T c_hat (the QJL
+ * residual term is an estimator, not a vector) and n_v Pi^T c_hat_v, rounded
+ * to fp16 -- become the newest hot tokens of every kv head of the sequence
+ * (ring slots (hot_start + hot_len) mod W_max, hot_len grows), its cold slot
+ * is masked (the attention skips it from then on), its count returns to 0.
+ * At most max_per_step positions move per sequence and step, in increasing
+ * position order, and never more than leave one ring slot free for the next
+ * step's token; positions left over keep their counts.  Eviction follows.
+ *  threshold     > 0, finite (weights are at most 1)
+ *  sticky        >= 1
+ *  max_per_step  1 .. TQ_PROMOTE_MAX_PER_STEP
+ *  cold_mask     device uint32 [B][max_pages * 4]: bit p % 32 of word p / 32
+ *                set = position p moved back; zero before the first step
+ *  counts        device uint8 [B][max_pages * 128]: consecutive counted
+ *                steps per position; zero before the first step
+ *  logits        device fp32 scratch [B][Hq][max_pages * 128]
+ */
+#define TQ_PROMOTE_MAX_PER_STEP 64
+typedef struct {
+  float threshold;
+  int sticky;
+  int max_per_step;
+  uint32_t* cold_mask;
+  uint8_t* counts;
+  float* logits;
+} tq_promotion;
+
+/* tq_monarch_step with promotion (promo NULL: exactly tq_monarch_step), the
+ * moves taking place between the attention and the eviction.  Same
+ * workspace. */
+TQ_API tq_status tq_monarch_step_promote(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B,
+                                         int Hq, int Hkv, float scale, const void* k_new,
+                                         const void* v_new, void* k_hot, void* v_hot, int W_max,
+                                         int32_t* hot_start, int32_t* hot_len,
+                                         uint8_t* page_pool, int64_t pool_pages,
+                                         const int32_t* page_table, int max_pages,
+                                         int32_t* cold_len, float threshold, int window,
+                                         int evict_block, const tq_promotion* promo,
+                                         int32_t* cold_used, float* out, void* workspace,
+                                         size_t ws_bytes, void* stream);
 /* Largest decode workspace tq_decode_attention_noalloc can serve (8 MiB). */
 #define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 
