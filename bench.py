@@ -49,7 +49,7 @@ def parse():
                     help="sequences per GPU (default: the workload's 16); smaller values only "
                          "size profiler captures and are not the benchmark line")
     ap.add_argument("--only", default=None,
-                    choices=["gated", "monarch", "tensor_cache", "stage1", "self_index",
+                    choices=["gated", "monarch", "promotion", "tensor_cache", "stage1", "self_index",
                              "compress", "search"],
                     help="run one extra row alone and print it (sized for profiler captures; "
                          "not the benchmark line)")
@@ -306,12 +306,17 @@ def measure_gated(torch, tq, st, reps=50):
 
 
 def measure_monarch(torch, tq, W, workload, evict_block, thresholds=(float("inf"), float("-inf")),
-                    steps=256):
+                    steps=256, promotion=None):
     """Monarch decode steps (append, gated attention, eviction) on a decode
     workload: the hot ring holds W_max = the workload's hot length slots,
     window = W_max - E; the timed steps (replayed from a CUDA graph, one step
-    per replay) include every eviction that falls due (one per E steps)."""
-    st = build_state(torch, tq, W, 0, None, workload, extra_pages=(steps + 64) // 128 + 3)
+    per replay) include every eviction that falls due (one per E steps).
+    promotion: None, or dict(threshold, sticky, max_per_step): the steps also
+    count cold weights and move cold tokens back (tq_monarch_step_promote)."""
+    # cold positions the steps can add: one token per step, plus every token
+    # moved back (each can be evicted again into a new cold position)
+    grow = (steps + 64) * (1 + (promotion["max_per_step"] if promotion else 0))
+    st = build_state(torch, tq, W, 0, None, workload, extra_pages=grow // 128 + 3)
     ctx, B, Hq, Hkv, d = st["ctx"], st["B"], st["Hq"], st["Hkv"], st["d"]
     W_max, E = st["hot"], evict_block
     window = W_max - E
@@ -324,21 +329,41 @@ def measure_monarch(torch, tq, W, workload, evict_block, thresholds=(float("inf"
     used = torch.empty((B, Hq), dtype=torch.int32, device=dev)
     res = {"workload": workload, "evict_block": E, "window": window, "hot_slots": W_max,
            "steps": steps}
+    pr = None
+    if promotion is not None:
+        cap = st["table"].shape[-1] * tq.TQ_PAGE_TOKENS
+        pr = dict(promotion, cold_mask=torch.zeros((B, cap // 32), dtype=torch.int32, device=dev),
+                  counts=torch.zeros((B, cap), dtype=torch.uint8, device=dev),
+                  logits=torch.empty((B, Hq, cap), dtype=torch.float32, device=dev))
+        res["promotion"] = dict(promotion)
     for thr in thresholds:
         st["hot_len"].fill_(window)
         hot_start.zero_()
         st["cold_len"].fill_(st["cold"])
+        if pr is not None:
+            pr["cold_mask"].zero_()
+            pr["counts"].zero_()
 
         def step():
-            tq.tq_monarch_step(ctx.handle, st["q"], k_new, v_new, st["k_hot"], st["v_hot"],
-                               hot_start, st["hot_len"], st["pool"], st["table"], st["cold_len"],
-                               thr, window, E, st["out"], ws, Hkv, cold_used=used)
+            if pr is None:
+                tq.tq_monarch_step(ctx.handle, st["q"], k_new, v_new, st["k_hot"], st["v_hot"],
+                                   hot_start, st["hot_len"], st["pool"], st["table"],
+                                   st["cold_len"], thr, window, E, st["out"], ws, Hkv,
+                                   cold_used=used)
+            else:
+                tq.tq_monarch_step_promote(ctx.handle, st["q"], k_new, v_new, st["k_hot"],
+                                           st["v_hot"], hot_start, st["hot_len"], st["pool"],
+                                           st["table"], st["cold_len"], thr, window, E, pr,
+                                           st["out"], ws, Hkv, cold_used=used)
         ms = graph_ms(torch, step, steps)
         ctx.check()
         tokens = B * Hkv * (W_max + st["cold"])
-        res["threshold_%s" % thr] = {"us_per_step": ms * 1e3,
-                                     "kv_tokens_heads_per_s": tokens / (ms / 1e3),
-                                     "heads_reading_cold": float(used.float().mean())}
+        row = {"us_per_step": ms * 1e3, "kv_tokens_heads_per_s": tokens / (ms / 1e3),
+               "heads_reading_cold": float(used.float().mean())}
+        if pr is not None:  # cold positions moved back over every step run (warm-up included)
+            row["moved_back"] = int(sum(bin(int(w) & 0xFFFFFFFF).count("1")
+                                        for w in pr["cold_mask"].flatten().tolist()))
+        res["threshold_%s" % thr] = row
     del st
     torch.cuda.empty_cache()
     return res
@@ -730,7 +755,15 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         rows["monarch_step"] = [measure_monarch(torch, tq, W, "tinyllama", 128),
                                 measure_monarch(torch, tq, W, "tinyllama", 1),
-                                measure_monarch(torch, tq, W, WORKLOAD, 128)]
+                                measure_monarch(torch, tq, W, WORKLOAD, 128),
+                                measure_monarch(torch, tq, W, "tinyllama", 128,
+                                                thresholds=(float("inf"),),
+                                                promotion=dict(threshold=0.15, sticky=3,
+                                                               max_per_step=8)),
+                                measure_monarch(torch, tq, W, "tinyllama", 128,
+                                                thresholds=(float("inf"),),
+                                                promotion=dict(threshold=0.002, sticky=3,
+                                                               max_per_step=8))]
         torch.cuda.empty_cache()
         rows["compress"] = measure_compress(torch, tq)
         rows["compress"]["cpu_baseline"] = cpu_baseline_compress()
@@ -782,6 +815,10 @@ def run_only(args):
         res = measure_gated(torch, tq, st, reps=args.steps)
     elif args.only == "monarch":
         res = measure_monarch(torch, tq, W, "tinyllama", 128, steps=args.steps)
+    elif args.only == "promotion":
+        res = measure_monarch(torch, tq, W, "tinyllama", 128, steps=args.steps,
+                              thresholds=(float("inf"),),
+                              promotion=dict(threshold=0.002, sticky=3, max_per_step=8))
     elif args.only == "tensor_cache":
         res = measure_tensor_cache(torch, tq, W, WORKLOAD, steps=args.steps)
     elif args.only == "self_index":

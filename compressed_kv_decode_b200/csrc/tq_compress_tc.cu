@@ -696,31 +696,44 @@ __global__ void __maxnreg__(96) compress_keys_kernel(const __grid_constant__ CUt
         n = __half2float(nh);
         const float T0 = __fmul_rn(n, p.kt0);
         const float inv = n > 0.0f ? 1.0f / n : 0.0f;
+        // Per coordinate: magnitude index u = [|v| >= n t], residual
+        // r = v / n - c_hat (computed as for n > 0; a zero vector's row is
+        // cleared below).  Key word w: coordinate 16 w + 8 h + 2 i + e has its
+        // sign bit at 16 h + 15 - 4 i - e and its magnitude bit two below, so
+        // the coordinates are taken in the words' bit order (h = 1 first) and
+        // their bits shifted in from the most significant end, one funnel
+        // shift each (the sign bit is the float's).
         uint32_t kw[C::PART / 16];
-#pragma unroll
-        for (int w = 0; w < C::PART / 16; ++w) kw[w] = 0u;
         uint32_t rh[C::PART / 2];
         float g2 = 0.0f;
 #pragma unroll
-        for (int i2 = 0; i2 < C::PART / 2; ++i2) {
-          float rr[2];
+        for (int w = 0; w < C::PART / 16; ++w) {
+          uint32_t acc = 0u;
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            // computed as for n > 0; a zero vector's row is cleared below
-            const int i = 2 * i2 + e;  // column within the part (parts are 16-aligned)
-            const float v = x[i];
-            const bool neg = v < 0.0f, big = fabsf(v) >= T0;
-            const float cp = big ? p.kc1 : p.kc0;
-            const float r = fmaf(v, inv, neg ? cp : -cp);
-            rr[e] = r;
-            g2 = fmaf(r, r, g2);
-            const int jj = i & 15, hh = jj >> 3, ii = (jj & 7) >> 1, ee = jj & 1;
-            const int sbit = 16 * hh + 15 - 4 * ii - ee;
-            if (neg) kw[i >> 4] |= 1u << sbit;
-            if (big) kw[i >> 4] |= 1u << (sbit - 2);
-          }
-          const __half2 pr = __floats2half2_rn(rr[0], rr[1]);
-          rh[i2] = *reinterpret_cast<const uint32_t*>(&pr);
+          for (int hh = 1; hh >= 0; --hh)
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+              const int j = 16 * w + 8 * hh + 2 * ii;
+              float rr[2];
+              uint32_t mb[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const float v = x[j + e];
+                const bool big = fabsf(v) >= T0;
+                // |r| = |v| / n - c_u, with the sign of v (the level's sign)
+                const float m = fmaf(fabsf(v), inv, big ? -p.kc1 : -p.kc0);
+                rr[e] = __uint_as_float(__float_as_uint(m) ^ (__float_as_uint(v) & 0x80000000u));
+                g2 = fmaf(m, m, g2);
+                mb[e] = big ? 0x80000000u : 0u;
+              }
+              const __half2 pr = __floats2half2_rn(rr[0], rr[1]);
+              rh[j / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+              acc = __funnelshift_l(__float_as_uint(x[j]), acc, 1);
+              acc = __funnelshift_l(__float_as_uint(x[j + 1]), acc, 1);
+              acc = __funnelshift_l(mb[0], acc, 1);
+              acc = __funnelshift_l(mb[1], acc, 1);
+            }
+          kw[w] = acc;
         }
         if (!(n > 0.0f)) {  // zero vector: all codes, residual and its norm are 0
 #pragma unroll
@@ -760,12 +773,13 @@ __global__ void __maxnreg__(96) compress_keys_kernel(const __grid_constant__ CUt
           uint8_t* pgp = p.pool + static_cast<size_t>(prev.page) * p.page_bytes;
           // sketch index i of the part sits in its 32-bit word at bit
           // 16 (i / 16 mod 2) + 15 - i mod 16 (a part of 16 fills one half word)
+          // (the float's sign bit, shifted in from the most significant end:
+          // indices 16..31 of the word first, then 0..15)
           uint32_t qw = 0u;
 #pragma unroll
-          for (int i = 0; i < C::PART; ++i) {
-            const int within = i & 31;
-            const int bit = 16 * (within >> 4) + 15 - (within & 15);
-            if (x[i] < 0.0f) qw |= 1u << bit;
+          for (int k2 = 0; k2 < C::PART; ++k2) {
+            const int i = C::PART == 32 ? (k2 + 16) & 31 : k2;
+            qw = __funnelshift_l(__float_as_uint(x[i]), qw, 1);
           }
           if (!(prev_n > 0.0f)) qw = 0u;  // zero vector
           if constexpr (C::PART == 32)

@@ -683,7 +683,8 @@ __device__ __forceinline__ uint32_t vlut(const char* lut, uint32_t off) {
   return *reinterpret_cast<const uint32_t*>(lut + off);
 }
 
-template <int D, int G>
+// PR: the promotion form (moved-back tokens masked, cold logits written).
+template <int D, int G, bool PR>
 __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
   using C = Cfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -906,8 +907,9 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
       // tokens of the unit that take part: inside the sequence and not moved
       // back to the hot window (Monarch's promotion)
       uint64_t valid = nv >= COLD_TOK ? ~0ull : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
-      const int b_seq = (sg >> 1) / p.Hkv;
-      if (p.promo.cold_mask) {
+      int b_seq = 0;
+      if constexpr (PR) {
+        b_seq = (sg >> 1) / p.Hkv;
         const uint32_t* mw = p.promo.cold_mask + static_cast<size_t>(b_seq) * p.max_pages * 4 + 2 * lu;
         valid &= ~(static_cast<uint64_t>(mw[0]) | (static_cast<uint64_t>(mw[1]) << 32));
       }
@@ -960,7 +962,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
             if (!((valid >> (t0 + 8)) & 1ull)) sv[nt * 8 + 2 * mt + 1] = NEG_INF;
           }
         }
-        if (p.promo.logits) {  // every cold logit, for the promotion
+        if constexpr (PR) {  // every cold logit, for the promotion
           const int kvh = (sg >> 1) % p.Hkv, cap = p.max_pages * TQ_PAGE_TOKENS;
           const int pos = lu * COLD_TOK + 16 * mt + g;
 #pragma unroll
@@ -1342,8 +1344,10 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
   p.w.gmax = reinterpret_cast<float*>(base + L.gmax);
   p.w.gmask = reinterpret_cast<int*>(base + L.gmask);
   p.gate_nsplit = gate_splits(p.W_max);
-  static SmemAttr attn_attr;
-  if (!raise_smem_limit(attn_kernel<D, G>, C::SMEM, attn_attr)) return TQ_ERR_CUDA;
+  static SmemAttr attn_attr, attn_attr_pr;
+  auto attn = p.promo.logits ? attn_kernel<D, G, true> : attn_kernel<D, G, false>;
+  if (!raise_smem_limit(attn, C::SMEM, p.promo.logits ? attn_attr_pr : attn_attr))
+    return TQ_ERR_CUDA;
   if (p.gated && p.gate_nsplit > 0) {
     // gate, then prep overlapping it: only prep's schedule CTA waits for the maxima
     gate_kernel<D, G><<<dim3(p.gate_nsplit, p.B * p.Hkv), 256, 0, st>>>(p);
@@ -1372,7 +1376,7 @@ int run(const tq_ctx* ctx, Params& p, void* ws, size_t ws_bytes, cudaStream_t st
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, attn_kernel<D, G>, p) != cudaSuccess) return TQ_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, attn, p) != cudaSuccess) return TQ_ERR_CUDA;
   }
   if (ctx->prof_stop) cudaEventRecord(static_cast<cudaEvent_t>(ctx->prof_stop), st);
   static SmemAttr comb_attr;

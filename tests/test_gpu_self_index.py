@@ -41,7 +41,7 @@ def keys(d, B, Hkv, T, seed):
     return np.float16(K).astype(np.float64)
 
 
-@pytest.mark.parametrize("d,T", [(128, 1000), (64, 777)])
+@pytest.mark.parametrize("d,T", [(128, 1000), (64, 777), (128, 20000), (64, 5)])
 def test_build_matches_oracle(d, T):
     import torch
     ctx = ctx_for(d)
@@ -116,8 +116,11 @@ def _scores_rows(kind, rows, T, seed):
 @pytest.mark.parametrize("kind,T,n_sink,top_k", [
     ("normal", 5000, 64, 300), ("ties", 3000, 64, 1000), ("zeros", 2000, 0, 777),
     ("normal", 200, 64, 500), ("normal", 50, 64, 10), ("ties", 40000, 64, 3000),
-    ("nan", 3000, 64, 1500)])
+    ("nan", 3000, 64, 1500), ("ties", 60000, 64, 5000), ("normal", 70000, 0, 4000)])
 def test_select_matches_oracle(kind, T, n_sink, top_k):
+    """Rows of up to 51200 candidates are staged in shared memory, longer
+    ones re-read from global memory (T = 60000, 70000); rows longer than
+    32768 candidates take more than one ordered pass."""
     import torch
     ctx = ctx_for(128)
     B, Hq = 2, 4
@@ -131,6 +134,21 @@ def test_select_matches_oracle(kind, T, n_sink, top_k):
         ref = S.select(sc[r].astype(np.float64), top_k, n_sink)
         assert np.array_equal(got[r, :len(ref)], ref)
         assert (got[r, len(ref):] == -1).all()
+
+
+def test_select_more_rows_than_sms():
+    """The selection CTAs are persistent over the rows (one per SM): 320 rows."""
+    import torch
+    ctx = ctx_for(64)
+    B, Hq, T, n_sink, top_k = 10, 32, 3000, 64, 225
+    sc = _scores_rows("ties", B * Hq, T, 99)
+    picked = torch.empty((B, Hq, top_k), dtype=torch.int32, device="cuda")
+    tq.tq_self_index_select(ctx.handle, torch.from_numpy(sc).reshape(B, Hq, T).cuda(), picked,
+                            n_sink=n_sink)
+    torch.cuda.synchronize()
+    got = picked.cpu().numpy().reshape(B * Hq, top_k)
+    for r in range(B * Hq):
+        assert np.array_equal(got[r], S.select(sc[r].astype(np.float64), top_k, n_sink))
 
 
 @pytest.mark.parametrize("d,G,qdt,T,top_k", [
