@@ -406,15 +406,15 @@ def measure_tensor_cache(torch, tq, W, workload, steps=256):
             "achieved_gbs": by / (ms / 1e3) / 1e9}
 
 
-def measure_self_index(torch, tq, reps=3):
-    """Self-Indexing on the 32K decode's key shapes (16 x 8 kv heads x 32768
-    fp16 keys and values, d = 128, 32 query heads, top_k = 7.5 % of T):
+def measure_self_index(torch, tq, reps=3, B=16):
+    """Self-Indexing on the 32K decode's key shapes (B = 16 x 8 kv heads x
+    32768 fp16 keys and values, d = 128, 32 query heads, top_k = 7.5 % of T):
     kernel times (CUDA events, median of reps) and GB/s over the algorithmic
     bytes -- keys read + codes and centroids written (build), codes read +
-    scores written (scores), scores read + picked written (select; its four
-    digit passes re-read the scores from L2), the 64 sinks' and the picked
-    tokens' key and value rows read per query head (attend)."""
-    B, Hkv, Hq, T, d = 16, 8, 32, 32768, 128
+    scores written (scores), scores read + picked written (select), the 64
+    sinks' and the picked tokens' key and value rows read per query head
+    (attend).  A smaller B only sizes profiler captures."""
+    Hkv, Hq, T, d = 8, 32, 32768, 128
     top_k = round(0.075 * T)
     ctx = tq.Context(d, seed=0)
     gen = torch.Generator(device="cuda")
@@ -451,8 +451,8 @@ def measure_self_index(torch, tq, reps=3):
             "select": B * Hq * (T * 4 + top_k * 4),
             "attend": B * Hq * ((64 + top_k) * 2 * d * 2 + top_k * 4 + d * 2 + d * 4)}
     peak = float(measured_peaks()[0]["hbm_gbs"])
-    row = {"workload": "16 x 8 kv heads x 32768 fp16 keys and values, d=128; 32 query "
-                       "heads; top_k = %d (7.5%% of T) + 64 sinks" % top_k}
+    row = {"workload": "%d x 8 kv heads x 32768 fp16 keys and values, d=128; 32 query "
+                       "heads; top_k = %d (7.5%% of T) + 64 sinks" % (B, top_k)}
     for which, lst in times.items():
         m = statistics.median(lst)
         row[which + "_ms"] = m
@@ -821,8 +821,8 @@ def run_only(args):
                               promotion=dict(threshold=0.002, sticky=3, max_per_step=8))
     elif args.only == "tensor_cache":
         res = measure_tensor_cache(torch, tq, W, WORKLOAD, steps=args.steps)
-    elif args.only == "self_index":
-        res = measure_self_index(torch, tq, reps=max(1, args.steps))
+    elif args.only == "self_index":  # --batch b: b sequences (default 16)
+        res = measure_self_index(torch, tq, reps=max(1, args.steps), B=args.batch or 16)
     elif args.only == "compress":  # --batch b: 8 heads x b * 65536 vectors
         res = measure_compress(torch, tq, reps=max(1, args.steps), T=65536 * (args.batch or 8))
     elif args.only == "search":  # --batch b: b * 100000 database vectors

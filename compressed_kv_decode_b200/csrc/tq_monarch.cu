@@ -15,11 +15,12 @@
 //   compress    the tensor-core compress/append on the staging tiles, with
 //               the per-sequence counts (sequences with 0 write nothing; CTAs
 //               without a tile leave at once)
-//   promote     (with promotion) one CTA per sequence: per cold position the
-//               largest attention weight over the query heads that read the
-//               cold tier, from the attention's logits and the combine's
-//               log-sum-exp; consecutive counts; positions that reach the
-//               sticky count are masked and their decompressed records
+//   weights     (with promotion) one thread per cold position: its largest
+//               attention weight over the query heads that read the cold
+//               tier, from the attention's logits and the combine's
+//               log-sum-exp; consecutive counts; candidate bits
+//   promote     (with promotion) one CTA per sequence: the first candidates
+//               in position order are masked and their decompressed records
 //               (n Pi^T c_hat for K, n_v Pi^T c_hat_v for V, fp16) appended to
 //               the ring of every kv head
 //   finish      cold_len += n, hot_len -= n, hot_start += n (mod W_max)
@@ -113,6 +114,7 @@ struct PromoParams {
   const float* lse;     // [B][Hq]
   uint32_t* mask;       // [B][cap / 32]
   uint8_t* counts;      // [B][cap]
+  uint32_t* cand;       // [B][cap / 32] workspace: positions whose count reached sticky
   const uint8_t* pool;
   long long pool_pages, page_bytes;
   int blk, off_h, off_l, off_vc, off_nk, off_vn;
@@ -128,102 +130,167 @@ struct PromoParams {
   int* err;
 };
 
-// Promotion (see the launch list above), one CTA per sequence.
-template <int D>
-__global__ void __launch_bounds__(PROMO_THREADS) promote_kernel(PromoParams p) {
-  const int b = blockIdx.x, tid = threadIdx.x;
+// Weights and counts, one thread per cold position (grid: position blocks x
+// sequences): the position's weight is its largest softmax probability over
+// the query heads that read the cold tier (logit and log-sum-exp in base 2;
+// a head that kept off the cold tier has log-sum-exp +inf); a weight at or
+// above the threshold counts the step, a lower one resets the count.  Bit
+// (pos mod 32) of cand word pos / 32: the count reached the sticky value.
+__global__ void __launch_bounds__(PROMO_THREADS) weights_kernel(PromoParams p) {
+  const int b = blockIdx.y, pos = blockIdx.x * PROMO_THREADS + threadIdx.x;
   const int cap = p.max_pages * TQ_PAGE_TOKENS;
-  __shared__ int chosen[PROMO_MAX];
-  __shared__ int s_count, s_hl;
-  __shared__ int wsum[PROMO_THREADS / 32];
-  __shared__ float ck[D], cv[D];
-  const int cl = min(max(p.cold_len[b], 0), cap);
-  const int hl = p.hot_len[b];
-  if (tid == 0) {
-    s_count = 0;
-    s_hl = hl;
-  }
+  extern __shared__ float s_lse[];  // [Hq]
+  for (int h = threadIdx.x; h < p.Hq; h += PROMO_THREADS)
+    s_lse[h] = p.lse[static_cast<size_t>(b) * p.Hq + h];
   __syncthreads();
-  const int limit = min(p.max_per_step, max(0, p.W_max - 1 - hl));
-  uint32_t* mask = p.mask + static_cast<size_t>(b) * (cap / 32);
-  uint8_t* counts = p.counts + static_cast<size_t>(b) * cap;
-  const float* lse = p.lse + static_cast<size_t>(b) * p.Hq;
-  for (int base = 0; base < cl; base += PROMO_THREADS) {
-    const int pos = base + tid;
-    bool cand = false;
-    if (pos < cl && !((mask[pos >> 5] >> (pos & 31)) & 1u)) {
+  const int cl = min(max(p.cold_len[b], 0), cap);
+  bool cand = false;
+  if (pos < cl) {
+    uint32_t* mask = p.mask + static_cast<size_t>(b) * (cap / 32);
+    if (!((mask[pos >> 5] >> (pos & 31)) & 1u)) {
+      const float* lg = p.logits + static_cast<size_t>(b) * p.Hq * cap + pos;
       float w = 0.0f;
+#pragma unroll 8
       for (int h = 0; h < p.Hq; ++h) {
-        const float L = lse[h];
-        if (L < __builtin_huge_valf())  // the head read the cold tier
-          w = fmaxf(w, exp2f(p.logits[(static_cast<size_t>(b) * p.Hq + h) * cap + pos] - L));
+        const float L = s_lse[h];
+        const float x = __ldg(lg + static_cast<size_t>(h) * cap);
+        if (L < __builtin_huge_valf()) w = fmaxf(w, exp2f(x - L));
       }
+      uint8_t* counts = p.counts + static_cast<size_t>(b) * cap;
       const int c = w >= p.thr ? min(counts[pos] + 1, 255) : 0;
       counts[pos] = static_cast<uint8_t>(c);
       cand = c >= p.sticky;
     }
-    // rank of this position among the block's candidates, in position order
-    const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+  }
+  const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+  if ((threadIdx.x & 31) == 0 && pos < cap)
+    p.cand[static_cast<size_t>(b) * (cap / 32) + (pos >> 5)] = bal;
+}
+
+// Promotion of one sequence (one CTA): the first `limit` candidates in
+// position order (limit = min(max_per_step, W_max - 1 - hot_len)) are masked,
+// their counts reset, and their decompressed records, n Pi^T c_hat (K) and
+// n_v Pi^T c_hat_v (V) rounded to fp16, appended to the ring of every kv head;
+// hot_len grows by their number.  Pi is staged in shared memory, and the
+// (position, kv head) pairs are decompressed in batches, every thread taking
+// outputs of every pair of the batch.
+template <int D>
+__global__ void __launch_bounds__(PROMO_THREADS) promote_kernel(PromoParams p) {
+  constexpr int PB = 8;  // (position, kv head) pairs per batch
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int cap = p.max_pages * TQ_PAGE_TOKENS;
+  extern __shared__ float s_rot[];  // [D][D]
+  __shared__ int chosen[PROMO_MAX];
+  __shared__ int wsum[PROMO_THREADS / 32];
+  __shared__ float lev[PB][2][D];   // key and value levels of the batch's pairs
+  __shared__ float nrm[PB][2];
+  __shared__ int s_count;
+  const int cl = min(max(p.cold_len[b], 0), cap);
+  const int hl = p.hot_len[b];
+  const int limit = min(p.max_per_step, max(0, p.W_max - 1 - hl));
+  if (tid == 0) s_count = 0;
+  __syncthreads();
+  // the first `limit` candidates, in position order (one word per thread)
+  const uint32_t* cw = p.cand + static_cast<size_t>(b) * (cap / 32);
+  const int nwords = (cl + 31) / 32;
+  for (int w0 = 0; w0 < nwords && s_count < limit; w0 += PROMO_THREADS) {
+    const int w = w0 + tid;
+    uint32_t bits = 0u;
+    if (w < nwords) {
+      bits = cw[w];
+      if (32 * w + 32 > cl) bits &= (cl - 32 * w >= 32) ? ~0u : ((1u << (cl - 32 * w)) - 1u);
+    }
+    const int n = __popc(bits);
+    // exclusive prefix of n over the block's threads
+    int incl = n;
     const int lane = tid & 31, warp = tid >> 5;
-    if (lane == 0) wsum[warp] = __popc(bal);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int w = 0; w < PROMO_THREADS / 32; ++w) {
-      if (w < warp) before += wsum[w];
-      total += wsum[w];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
     }
-    const int rank = s_count + before + __popc(bal & ((1u << lane) - 1u));
-    if (cand && rank < limit) {
-      chosen[rank] = pos;
-      counts[pos] = 0;
-      atomicOr(&mask[pos >> 5], 1u << (pos & 31));
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = s_count;
+    for (int q = 0; q < warp; ++q) before += wsum[q];
+    before += incl - n;
+    while (bits && before < limit) {
+      const int j = __ffs(static_cast<int>(bits)) - 1;
+      bits &= bits - 1u;
+      chosen[before++] = 32 * w + j;
     }
     __syncthreads();
-    if (tid == 0) s_count = min(limit, s_count + total);
+    if (tid == 0) {
+      int tot = 0;
+      for (int q = 0; q < PROMO_THREADS / 32; ++q) tot += wsum[q];
+      s_count = min(limit, s_count + tot);
+    }
     __syncthreads();
   }
   const int n = s_count;
+  if (n == 0) return;
+  uint32_t* mask = p.mask + static_cast<size_t>(b) * (cap / 32);
+  uint8_t* counts = p.counts + static_cast<size_t>(b) * cap;
+  for (int i = tid; i < n; i += PROMO_THREADS) {
+    const int pos = chosen[i];
+    counts[pos] = 0;
+    atomicOr(&mask[pos >> 5], 1u << (pos & 31));
+  }
+  for (int i = tid; i < D * D; i += PROMO_THREADS) s_rot[i] = p.rot[i];
   int start = p.hot_start[b];
   if (start < 0 || start >= p.W_max) start = 0;
-  // decompress each moved position into the ring of every kv head
-  for (int i = 0; i < n; ++i) {
-    const int pos = chosen[i];
-    int slot = start + hl + i;
-    while (slot >= p.W_max) slot -= p.W_max;
-    for (int kvh = 0; kvh < p.Hkv; ++kvh) {
+  const int npair = n * p.Hkv;
+  for (int pb0 = 0; pb0 < npair; pb0 += PB) {
+    const int nb = min(PB, npair - pb0);
+    __syncthreads();  // s_rot staged; the previous batch's levels consumed
+    // levels of the batch's pairs: pair = i * Hkv + kvh
+    for (int e = tid; e < nb * D; e += PROMO_THREADS) {
+      const int q = e / D, j = e % D;
+      const int pr = pb0 + q, i = pr / p.Hkv, kvh = pr % p.Hkv;
+      const int pos = chosen[i];
       const int bh = b * p.Hkv + kvh;
       const int page = p.page_table[static_cast<size_t>(bh) * p.max_pages + pos / TQ_PAGE_TOKENS];
       const bool ok = page >= 0 && page < p.pool_pages;
-      if (!ok && tid == 0) report(p.err, TQ_ERR_CAPACITY);
+      if (!ok && j == 0) report(p.err, TQ_ERR_CAPACITY);
       const int s16 = pos % TQ_PAGE_TOKENS, t = s16 & 15;
       const uint8_t* bk = p.pool + static_cast<size_t>(ok ? page : 0) * p.page_bytes + (s16 >> 4) * p.blk;
-      for (int j = tid; j < D; j += PROMO_THREADS) {
-        const int byte = plane_byte(j, t);
-        const int hb = (bk[p.off_h + byte] >> (t & 7)) & 1, lb = (bk[p.off_l + byte] >> (t & 7)) & 1;
-        // level index 2H + L of (-c1, -c0, +c0, +c1)
-        const float lev = hb ? (lb ? p.kc1 : p.kc0) : (lb ? -p.kc0 : -p.kc1);
-        ck[j] = ok ? lev : 0.0f;
-        const int vb = bk[p.off_vc + (vc_pos<D>(j, t >> 1) & (8 * D - 1))];
-        const int code = (t & 1) ? (vb >> 4) : (vb & 15);
-        cv[j] = ok ? ((code & 8) ? -p.vc[code & 7] : p.vc[code & 7]) : 0.0f;
+      const int byte = plane_byte(j, t);
+      const int hb = (bk[p.off_h + byte] >> (t & 7)) & 1, lb = (bk[p.off_l + byte] >> (t & 7)) & 1;
+      // level index 2H + L of (-c1, -c0, +c0, +c1)
+      lev[q][0][j] = ok ? (hb ? (lb ? p.kc1 : p.kc0) : (lb ? -p.kc0 : -p.kc1)) : 0.0f;
+      const int vb = bk[p.off_vc + (vc_pos<D>(j, t >> 1) & (8 * D - 1))];
+      const int code = (t & 1) ? (vb >> 4) : (vb & 15);
+      lev[q][1][j] = ok ? ((code & 8) ? -p.vc[code & 7] : p.vc[code & 7]) : 0.0f;
+      if (j == 0) {
+        nrm[q][0] = ok ? __low2float(*reinterpret_cast<const __half2*>(bk + p.off_nk + 4 * t)) : 0.0f;
+        nrm[q][1] = ok ? __half2float(*reinterpret_cast<const __half*>(bk + p.off_vn + 2 * t)) : 0.0f;
       }
-      __syncthreads();
-      const __half2 nn = *reinterpret_cast<const __half2*>(bk + p.off_nk + 4 * t);
-      const float nk = ok ? __low2float(nn) : 0.0f;
-      const float nv = ok ? __half2float(*reinterpret_cast<const __half*>(bk + p.off_vn + 2 * t)) : 0.0f;
-      for (int o = tid; o < 2 * D; o += PROMO_THREADS) {
-        const int isv = o >= D, oo = isv ? o - D : o;
-        const float* cc = isv ? cv : ck;
-        float acc = 0.0f;
-        for (int j = 0; j < D; ++j) acc = fmaf(p.rot[j * D + oo], cc[j], acc);  // (Pi^T c)[oo]
-        const size_t dst = (static_cast<size_t>(bh) * p.W_max + slot) * D + oo;
-        if (isv) p.v_hot[dst] = __float2half_rn(nv * acc);
-        else p.k_hot[dst] = __float2half_rn(nk * acc);
+    }
+    __syncthreads();
+    // outputs (Pi^T c)[o] = sum_j Pi[j][o] c[j]: thread = output coordinate
+    // and K / V, over every pair of the batch
+    for (int e = tid; e < 2 * D; e += PROMO_THREADS) {
+      const int isv = e >= D, o = isv ? e - D : e;
+      float acc[PB];
+#pragma unroll
+      for (int q = 0; q < PB; ++q) acc[q] = 0.0f;
+      for (int j = 0; j < D; ++j) {
+        const float r = s_rot[j * D + o];
+#pragma unroll
+        for (int q = 0; q < PB; ++q) acc[q] = fmaf(r, lev[q][isv][j], acc[q]);
       }
-      __syncthreads();
+      for (int q = 0; q < nb; ++q) {
+        const int pr = pb0 + q, i = pr / p.Hkv, kvh = pr % p.Hkv;
+        int slot = start + hl + i;
+        while (slot >= p.W_max) slot -= p.W_max;
+        const size_t dst = ((static_cast<size_t>(b) * p.Hkv + kvh) * p.W_max + slot) * D + o;
+        const __half hv = __float2half_rn(nrm[q][isv] * acc[q]);
+        if (isv) p.v_hot[dst] = hv;
+        else p.k_hot[dst] = hv;
+      }
     }
   }
-  if (tid == 0) p.hot_len[b] = s_hl + n;
+  if (tid == 0) p.hot_len[b] = hl + n;
 }
 
 }  // namespace mon
@@ -234,7 +301,8 @@ size_t monarch_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int ma
   if (dec == 0 || evict_block <= 0) return 0;
   const size_t stage = static_cast<size_t>(B) * Hkv * evict_block * ctx->cfg.head_dim * 2;
   return mon::align256(dec) + 2 * mon::align256(stage) + mon::align256(sizeof(int32_t) * B) +
-         mon::align256(sizeof(float) * B * Hq);  // per-head log-sum-exp (promotion)
+         mon::align256(sizeof(float) * B * Hq) +  // per-head log-sum-exp (promotion)
+         mon::align256(sizeof(uint32_t) * B * max_pages * (TQ_PAGE_TOKENS / 32));  // candidates
 }
 
 int launch_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq, int Hkv,
@@ -254,6 +322,8 @@ int launch_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int 
   int32_t* n_evict = reinterpret_cast<int32_t*>(v_stage + mon::align256(stage));
   float* lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(n_evict) +
                                         mon::align256(sizeof(int32_t) * B));
+  uint32_t* cand = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(lse) +
+                                               mon::align256(sizeof(float) * B * Hq));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int row_chunks = d / 8;
   if (k_new) {
@@ -309,10 +379,19 @@ int launch_monarch_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int 
     pp.kc1 = ctx->cb.key_c[1];
     for (int i = 0; i < 8; ++i) pp.vc[i] = ctx->cb.val_c[i];
     pp.err = ctx->dev.err;
-    if (d == 128)
-      mon::promote_kernel<128><<<B, mon::PROMO_THREADS, 0, st>>>(pp);
-    else
-      mon::promote_kernel<64><<<B, mon::PROMO_THREADS, 0, st>>>(pp);
+    pp.cand = cand;
+    const int cap = max_pages * TQ_PAGE_TOKENS;
+    mon::weights_kernel<<<dim3((cap + mon::PROMO_THREADS - 1) / mon::PROMO_THREADS, B),
+                          mon::PROMO_THREADS, sizeof(float) * Hq, st>>>(pp);
+    if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
+    const int rot_bytes = static_cast<int>(sizeof(float)) * d * d;
+    static SmemAttr promo_attr;
+    if (d == 128) {
+      if (!raise_smem_limit(mon::promote_kernel<128>, rot_bytes, promo_attr)) return TQ_ERR_CUDA;
+      mon::promote_kernel<128><<<B, mon::PROMO_THREADS, rot_bytes, st>>>(pp);
+    } else {
+      mon::promote_kernel<64><<<B, mon::PROMO_THREADS, rot_bytes, st>>>(pp);
+    }
     if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
   }
   mon::gather_kernel<<<B * Hkv, 256, 0, st>>>(
