@@ -13,10 +13,13 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtq.so")
+# TQ_LIB=debug selects the range-checked build (libtq_debug.so, compiled with
+# TQ_DEBUG: every checked index outside its array records TQ_ERR_RANGE and the
+# access is skipped)
+LIB_PATH = os.path.join(_HERE, "libtq_debug.so" if os.environ.get("TQ_LIB") == "debug" else "libtq.so")
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA = 0, 1, 2, 3
-TQ_ERR_OOM, TQ_ERR_CAPACITY, TQ_ERR_TIMEOUT = 4, 5, 6
+TQ_ERR_OOM, TQ_ERR_CAPACITY, TQ_ERR_TIMEOUT, TQ_ERR_RANGE = 4, 5, 6, 7
 TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
 TQ_INPUT_ROTATED = 1
 TQ_PAGE_TOKENS = 128
@@ -49,7 +52,7 @@ def lib():
     if _lib is None:
         if not os.path.exists(LIB_PATH) or os.environ.get("TQ_REBUILD"):
             from . import build as _build
-            _build.build()
+            _build.build(debug=LIB_PATH.endswith("_debug.so"))
         L = C.CDLL(LIB_PATH)
         vp, i32p, f32p, u8p = C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p
         L.tq_generate_params.argtypes = [C.POINTER(tq_config)] + [C.c_void_p] * 6

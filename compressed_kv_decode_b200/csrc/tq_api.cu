@@ -75,6 +75,7 @@ const char* tq_status_string(tq_status s) {
     case TQ_ERR_OOM: return "out of device memory";
     case TQ_ERR_CAPACITY: return "capacity exceeded (page table, pool or window)";
     case TQ_ERR_TIMEOUT: return "bounded wait timed out";
+    case TQ_ERR_RANGE: return "index out of range (range-checked build)";
   }
   return "unknown status";
 }
@@ -414,7 +415,7 @@ tq_status tq_self_index_select(const tq_ctx* ctx, const float* scores, int rows,
     return TQ_ERR_INVALID_ARG;
   const int lo = n_sink < T ? n_sink : T;
   return static_cast<tq_status>(tq::launch_self_index_select(
-      scores, rows, T, lo, self_index_k_eff(T, n_sink, top_k), top_k, picked, stream));
+      ctx, scores, rows, T, lo, self_index_k_eff(T, n_sink, top_k), top_k, picked, stream));
 }
 
 tq_status tq_self_index_attend(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,

@@ -748,7 +748,8 @@ __global__ void __maxnreg__(96) compress_keys_kernel(const __grid_constant__ CUt
         else
           tc::st8(t_lane + C::COL_RES0 + b * (D / 2) + q * (C::PART / 2), rh);
         gp[(b * NPART + q) * ROWS + row] = g2;
-        if (wr) {
+        if (wr && TQ_IN_RANGE(p.err, p.off_kc + row * (D / 4) + (q + 1) * (C::PART / 4) - 1,
+                              p.page_bytes)) {
           if constexpr (C::PART / 16 == 2)
             *reinterpret_cast<uint2*>(pg + p.off_kc + row * (D / 4) + q * (C::PART / 4)) =
                 make_uint2(kw[0], kw[1]);
@@ -769,7 +770,8 @@ __global__ void __maxnreg__(96) compress_keys_kernel(const __grid_constant__ CUt
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_skfree);
         const bool page_ok = prev.page >= 0 && prev.page < p.pool_pages;
-        if (!failed && page_ok && row >= prev.s_lo && row < prev.s_hi) {
+        if (!failed && page_ok && row >= prev.s_lo && row < prev.s_hi &&
+            TQ_IN_RANGE(p.err, p.off_qs + row * (D / 8) + (q + 1) * (C::PART / 8) - 1, p.page_bytes)) {
           uint8_t* pgp = p.pool + static_cast<size_t>(prev.page) * p.page_bytes;
           // sketch index i of the part sits in its 32-bit word at bit
           // 16 (i / 16 mod 2) + 15 - i mod 16 (a part of 16 fills one half word)

@@ -860,6 +860,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
       lt[nt] = l;
     }
     const int first = warp_of(uoff[sg], U, Weff);
+    if (!TQ_IN_RANGE(p.err, soff[sg] + (gw - first), p.Wtot + p.S)) return;  // partial record
     float* rec = p.w.part + static_cast<size_t>(soff[sg] + (gw - first)) * G * (D + 2);
     if (g == 0) {
 #pragma unroll
@@ -970,8 +971,10 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
             const int h = c + 4 * nt;
             if (h < G) {
               float* lg = p.promo.logits + (static_cast<size_t>(b_seq) * p.Hq + kvh * G + h) * cap;
-              lg[pos] = sv[nt * 8 + 2 * mt];
-              lg[pos + 8] = sv[nt * 8 + 2 * mt + 1];
+              if (TQ_IN_RANGE(p.err, pos + 8, cap)) {
+                lg[pos] = sv[nt * 8 + 2 * mt];
+                lg[pos + 8] = sv[nt * 8 + 2 * mt + 1];
+              }
             }
           }
         }
@@ -1281,7 +1284,7 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(Params p) {
       const float sg = 1.0f / (1.0f + expf(-p.fuse.gate[kvh * G + g]));
       res = fmaf(sg, p.fuse.r[oi], res);
     }
-    p.out[oi] = res;
+    if (TQ_IN_RANGE(p.err, oi, static_cast<long long>(p.B) * p.Hq * D)) p.out[oi] = res;
     if (j == 0 && p.gated && p.cold_used)
       p.cold_used[static_cast<size_t>(b) * p.Hq + kvh * G + g] = open;
   }

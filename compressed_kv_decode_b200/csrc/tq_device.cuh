@@ -16,6 +16,22 @@ __device__ __forceinline__ void report(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// Range check of the debug build (compiled with TQ_DEBUG): true when
+// 0 <= i < n; otherwise TQ_ERR_RANGE goes to the error word and the result
+// is false, so that the caller skips the access (no trap, no assert).  In
+// the release build it is the constant true.
+#ifdef TQ_DEBUG
+__device__ __forceinline__ bool in_range(int* err, long long i, long long n) {
+  if (i >= 0 && i < n) return true;
+  report(err, TQ_ERR_RANGE);
+  return false;
+}
+#define TQ_IN_RANGE(err, i, n) \
+  ::tq::in_range((err), static_cast<long long>(i), static_cast<long long>(n))
+#else
+#define TQ_IN_RANGE(err, i, n) true
+#endif
+
 // ---- shared-memory address ----------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -176,8 +176,8 @@ int launch_self_index_build(const tq_ctx* ctx, const void* k, int B, int Hkv, in
 int launch_self_index_scores(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
                              int Hkv, int T, const uint8_t* codes, const float* cent,
                              float* scores, void* stream);
-int launch_self_index_select(const float* scores, int rows, int T, int lo, int k_eff, int k_cap,
-                             int32_t* picked, void* stream);
+int launch_self_index_select(const tq_ctx* ctx, const float* scores, int rows, int T, int lo,
+                             int k_eff, int k_cap, int32_t* picked, void* stream);
 int launch_self_index_attend(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int B, int Hq,
                              int Hkv, int T, const void* keys, const void* values,
                              const int32_t* picked, int k_cap, int k_eff, int n_s, float scale,

@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(256) append_kernel(const uint4* __restrict__ k
   }
   int slot = start + len;
   if (slot >= W_max) slot -= W_max;
+  if (!TQ_IN_RANGE(err, slot, W_max)) return;  // (the whole block)
   const int per = Hkv * row_chunks;  // 16-byte chunks of one sequence's new K (or V)
   for (int i = threadIdx.x; i < 2 * per; i += blockDim.x) {
     const int isv = i >= per, c = isv ? i - per : i;
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(PROMO_THREADS) promote_kernel(PromoParams p) {
     for (int e = tid; e < nb * D; e += PROMO_THREADS) {
       const int q = e / D, j = e % D;
       const int pr = pb0 + q, i = pr / p.Hkv, kvh = pr % p.Hkv;
-      const int pos = chosen[i];
+      const int pos = TQ_IN_RANGE(p.err, chosen[i], cap) ? chosen[i] : 0;
       const int bh = b * p.Hkv + kvh;
       const int page = p.page_table[static_cast<size_t>(bh) * p.max_pages + pos / TQ_PAGE_TOKENS];
       const bool ok = page >= 0 && page < p.pool_pages;
@@ -285,6 +286,7 @@ __global__ void __launch_bounds__(PROMO_THREADS) promote_kernel(PromoParams p) {
         while (slot >= p.W_max) slot -= p.W_max;
         const size_t dst = ((static_cast<size_t>(b) * p.Hkv + kvh) * p.W_max + slot) * D + o;
         const __half hv = __float2half_rn(nrm[q][isv] * acc[q]);
+        if (!TQ_IN_RANGE(p.err, i, PROMO_MAX)) continue;
         if (isv) p.v_hot[dst] = hv;
         else p.k_hot[dst] = hv;
       }

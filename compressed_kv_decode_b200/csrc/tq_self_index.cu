@@ -47,13 +47,14 @@ constexpr int BUILD_SMEM = 160 * 1024;
 // Index build for one (batch, kv head) per cluster of CS CTAs, CTA r taking
 // the tokens [T r / CS, T (r + 1) / CS):
 //   1. per-channel partial sums of its tokens (16-byte loads, 8 channels per
-//      thread, eight rows in flight, then a fixed-order reduction over the
+//      thread, sixteen rows in flight, then a fixed-order reduction over the
 //      token phases);
 //   2. cluster barrier; every CTA adds the CS partials in rank order from
 //      distributed shared memory, so all CTAs hold the same fp32 mean;
 //   3. its tokens' (token, group) sign patterns, written as bytes; lane g of
-//      a lane group takes group g and adds the centred subvector to its own
-//      table entry (no atomics: every entry has one writer);
+//      a lane group takes group g and adds the subvector to its own table
+//      entry (no atomics: every entry has one writer); the mean is taken off
+//      the sums once per entry at the end;
 //   4. the CTA's tables added entry by entry in a fixed order; cluster
 //      barrier; CTA r reduces a slice of the (group, pattern) entries over
 //      the CS CTAs in rank order and writes the centroids.
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(BUILD_THREADS, 1) build_kernel(const __half* _
   constexpr int NWARP = BUILD_THREADS / 32;
   constexpr int NCOPY = NWARP * TPW;                // private tables
   constexpr int TSTEP = NCOPY;                      // tokens per CTA per index round
-  constexpr int U = 8;                              // rows in flight per thread
+  constexpr int U = 16;                             // rows in flight per thread
   constexpr int NE = 16 * NG;                       // (pattern, group) entries
   static_assert(NCOPY * NE * 20 <= BUILD_SMEM, "tables");
   static_assert(PH * D * 4 <= BUILD_SMEM, "mean partials");
@@ -138,7 +139,10 @@ __global__ void __launch_bounds__(BUILD_THREADS, 1) build_kernel(const __half* _
     if (r == 0) mu[static_cast<size_t>(bh) * D + tid] = m;
   }
   __syncthreads();
-  // 3. sign patterns and the lane's table: lane = (token of the warp, group g)
+  // 3. sign patterns and the lane's table: lane = (token of the warp, group g).
+  // The pattern compares the raw key with the mean (the sign of the fp32
+  // difference is that of the exact one); the table sums the raw subvectors,
+  // and n mu is taken off once per entry at the end.
   {
     const int warp = tid >> 5, lane = tid & 31;
     const int sub = lane / NG, g = lane % NG;
@@ -146,30 +150,28 @@ __global__ void __launch_bounds__(BUILD_THREADS, 1) build_kernel(const __half* _
     float4* my_sum = csum + static_cast<size_t>(copy) * NE + g;  // + 16-entry stride NG
     float* my_cnt = ccnt + static_cast<size_t>(copy) * NE + g;
     const float m0 = smu[4 * g], m1 = smu[4 * g + 1], m2 = smu[4 * g + 2], m3 = smu[4 * g + 3];
-    uint8_t* cb = codes + static_cast<size_t>(bh) * T * NG + g;
-    for (int t = t0 + copy; t < t1; t += U * TSTEP) {
+    const int t_first = t0 + copy;
+    uint8_t* cbp = codes + (static_cast<size_t>(bh) * T + t_first) * NG + g;
+    const __half* kp = kb + static_cast<size_t>(t_first) * D + 4 * g;
+    for (int t = t_first; t < t1; t += U * TSTEP, cbp += U * TSTEP * NG, kp += U * TSTEP * D) {
       uint2 raw[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int tt = t + u * TSTEP;
-        raw[u] = tt < t1 ? *reinterpret_cast<const uint2*>(kb + static_cast<size_t>(tt) * D + 4 * g)
-                         : make_uint2(0u, 0u);
-      }
+      for (int u = 0; u < U; ++u)
+        raw[u] = t + u * TSTEP < t1 ? *reinterpret_cast<const uint2*>(kp + u * TSTEP * D)
+                                    : make_uint2(0u, 0u);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const int tt = t + u * TSTEP;
-        if (tt >= t1) break;
+        if (t + u * TSTEP >= t1) break;
         const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw[u].x));
         const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw[u].y));
-        const float c0 = a.x - m0, c1 = a.y - m1, c2 = b.x - m2, c3 = b.y - m3;
-        const int pt = (c0 > 0.0f ? 1 : 0) | (c1 > 0.0f ? 2 : 0) | (c2 > 0.0f ? 4 : 0) |
-                       (c3 > 0.0f ? 8 : 0);
-        cb[static_cast<size_t>(tt) * NG] = static_cast<uint8_t>(pt);
+        const int pt = (a.x > m0 ? 1 : 0) | (a.y > m1 ? 2 : 0) | (b.x > m2 ? 4 : 0) |
+                       (b.y > m3 ? 8 : 0);
+        cbp[u * TSTEP * NG] = static_cast<uint8_t>(pt);
         float4 sv = my_sum[pt * NG];
-        sv.x += c0;
-        sv.y += c1;
-        sv.z += c2;
-        sv.w += c3;
+        sv.x += a.x;
+        sv.y += a.y;
+        sv.z += b.x;
+        sv.w += b.y;
         my_sum[pt * NG] = sv;
         my_cnt[pt * NG] += 1.0f;
       }
@@ -206,12 +208,13 @@ __global__ void __launch_bounds__(BUILD_THREADS, 1) build_kernel(const __half* _
         sv.w += o.w;
       }
       // entry e = (pattern pt, group g); centroids are stored [group][pattern][4]
+      // (the tables hold raw sums: the centred mean is sum / n - mu)
       const int pt = e / NG, g = e % NG;
       float* out = cent + ((static_cast<size_t>(bh) * NG + g) * 16 + pt) * 4;
-      out[0] = n > 0.0f ? sv.x / n : 0.0f;
-      out[1] = n > 0.0f ? sv.y / n : 0.0f;
-      out[2] = n > 0.0f ? sv.z / n : 0.0f;
-      out[3] = n > 0.0f ? sv.w / n : 0.0f;
+      out[0] = n > 0.0f ? sv.x / n - smu[4 * g] : 0.0f;
+      out[1] = n > 0.0f ? sv.y / n - smu[4 * g + 1] : 0.0f;
+      out[2] = n > 0.0f ? sv.z / n - smu[4 * g + 2] : 0.0f;
+      out[3] = n > 0.0f ? sv.w / n - smu[4 * g + 3] : 0.0f;
     }
   }
   cluster.sync();  // no CTA leaves while another still reads its shared memory
@@ -642,8 +645,9 @@ int launch_self_index_scores(const tq_ctx* ctx, const void* q, tq_dtype q_dtype,
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
-int launch_self_index_select(const float* scores, int rows, int T, int lo, int k_eff, int k_cap,
-                            int32_t* picked, void* stream) {
+int launch_self_index_select(const tq_ctx* ctx, const float* scores, int rows, int T, int lo,
+                            int k_eff, int k_cap, int32_t* picked, void* stream) {
+  (void)ctx;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   static std::mutex mu;
   static int sms[64] = {};

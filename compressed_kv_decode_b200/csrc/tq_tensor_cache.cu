@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(256) update_kernel(const void* q, int q_dtype,
   const bool evict = len == W;
   int slot = evict ? start : start + len;
   if (slot >= W) slot -= W;
-  const size_t row = (static_cast<size_t>(bh) * W + slot) * D;
+  const size_t row = (static_cast<size_t>(bh) * W + (TQ_IN_RANGE(err, slot, W) ? slot : 0)) * D;
   if (tid < D) {
     sk[tid] = evict ? __half2float(k_ring[row + tid]) : 0.0f;
     sv[tid] = evict ? __half2float(v_ring[row + tid]) : 0.0f;

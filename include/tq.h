@@ -64,7 +64,10 @@ typedef enum {
   TQ_ERR_CUDA = 3,
   TQ_ERR_OOM = 4,
   TQ_ERR_CAPACITY = 5, /* device: a sequence outgrew its page table or pool */
-  TQ_ERR_TIMEOUT = 6   /* device: a bounded wait on a copy ran out */
+  TQ_ERR_TIMEOUT = 6,  /* device: a bounded wait on a copy ran out */
+  TQ_ERR_RANGE = 7     /* device, range-checked build (libtq_debug.so) only: a
+                          computed index fell outside its array; the access
+                          was skipped */
 } tq_status;
 
 typedef enum { TQ_F32 = 0, TQ_F16 = 1, TQ_BF16 = 2 } tq_dtype;

@@ -27,8 +27,19 @@ def test_exports_every_declared_symbol():
         assert hasattr(L, n), n
 
 
+def test_range_checked_build_exports_every_declared_symbol():
+    """libtq_debug.so (the same sources compiled with TQ_DEBUG) is built
+    in-tree beside libtq.so and exports the same entry points."""
+    from compressed_kv_decode_b200 import build
+    path = build.build(debug=True)
+    assert path.endswith("libtq_debug.so") and os.path.exists(path)
+    L = C.CDLL(path)
+    for n in _declared():
+        assert hasattr(L, n), n
+
+
 def test_status_strings():
-    for s in range(7):
+    for s in range(8):
         assert tq.status_string(s) and "unknown" not in tq.status_string(s)
     assert "unknown" in tq.status_string(99)
 

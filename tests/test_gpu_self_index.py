@@ -118,7 +118,7 @@ def _scores_rows(kind, rows, T, seed):
     ("normal", 200, 64, 500), ("normal", 50, 64, 10), ("ties", 40000, 64, 3000),
     ("nan", 3000, 64, 1500), ("ties", 60000, 64, 5000), ("normal", 70000, 0, 4000)])
 def test_select_matches_oracle(kind, T, n_sink, top_k):
-    """Rows of up to 51200 candidates are staged in shared memory, longer
+    """Rows of up to 50176 candidates are staged in shared memory, longer
     ones re-read from global memory (T = 60000, 70000); rows longer than
     32768 candidates take more than one ordered pass."""
     import torch
