@@ -231,3 +231,114 @@ def test_promotion_arguments_rejected(O):
                                        z(B, Hq, d), ws, Hkv)
         assert e.value.status == tq.TQ_ERR_INVALID_ARG
     ctx.close()
+
+
+def test_tinyllama_shape_promotion(O):
+    """The promotion step at the TinyLlama decode shape the benchmark times
+    (B = 1, 32 q / 4 kv heads, d = 64, 1024 cold tokens written by the
+    oracle's packer, 384 hot tokens in a 512-slot ring, E = 128; K, V with
+    4 outlier channels x10): the same query every step, the threshold placed
+    in the widest gap of the oracle's first-step weights among the largest
+    ones (so no decision lies near it), sticky 2, up to 8 moves per step.
+    Masks, counts, lengths and ring start exact after every step; outputs
+    within the decode tolerance; moved-back rows within one fp16 unit."""
+    import copy
+    import torch
+    from compressed_kv_decode_b200 import workloads as W
+    cfg = W.DECODE["tinyllama"]
+    B, Hq, Hkv, d = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"]
+    G = Hq // Hkv
+    n_cold, n_hot, W_max, E = 1024, 384, 512, 128
+    window = W_max - E
+    steps = 6
+    P = O.Params(d, seed=0)
+    ctx = tq.Context(d, 0)
+    sk, sv, sq, so = cfg["seeds"]
+    chans = W.outlier_channels(so, Hkv, d, cfg["n_out"])
+    T = n_cold + n_hot + steps
+    max_pages = (n_cold + steps + 127) // 128 + 1
+    table, n_pages = W.random_page_table(5, B, Hkv, max_pages)
+    nb, _ = O.page_layout(d, d, True)
+    pool = np.zeros(n_pages * nb, np.uint8)
+    seqs = []
+    hot_k = [[None] * Hkv]
+    hot_v = [[None] * Hkv]
+    for h in range(Hkv):
+        K, V = W.kv_sequence(sk, sv, 0, h, T, d, chans[h], cfg["factor"])
+        K, V = f16(K), f16(V)
+        seqs.append((K, V))
+        t = np.arange(n_cold)
+        kr, vr = O.encode(P, K[:n_cold], True), O.encode(P, V[:n_cold], False)
+        O.pack(pool, nb, d, d, True, table[0, h, t // 128], t % 128,
+               dict(sign=kr["sign"], mag=kr["mag"], qbits=kr["qbits"], n=kr["n"],
+                    gamma=kr["gamma"], vcode=vr["vcode"], vn=vr["vn"]))
+        hot_k[0][h] = list(K[n_cold:n_cold + n_hot])
+        hot_v[0][h] = list(V[n_cold:n_cold + n_hot])
+    q = W.queries(sq, B, Hq, d, cfg["q_dtype"])
+    scale = 1.0 / math.sqrt(d)
+    new_k = [np.stack([seqs[h][0][n_cold + n_hot + s] for h in range(Hkv)])[None] for s in range(steps)]
+    new_v = [np.stack([seqs[h][1][n_cold + n_hot + s] for h in range(Hkv)])[None] for s in range(steps)]
+    base = MonarchCache(P, B, Hkv, window, E, table, cold_len=[n_cold], pool=pool, hot_k=hot_k,
+                        hot_v=hot_v, promotion=dict(threshold=1.0, sticky=2, max_per_step=8),
+                        W_max=W_max)
+    probe = copy.deepcopy(base)
+    probe.append(new_k[0], new_v[0])
+    _, _, wmax = probe.attend_weights(q, scale)
+    w = np.sort(wmax[0])[::-1][:40]
+    gaps = w[:-1] / np.maximum(w[1:], 1e-30)
+    i = int(np.argmax(gaps[4:])) + 4  # at least five positions above the threshold
+    assert gaps[i] > 1.3, gaps
+    thr = float(np.sqrt(w[i] * w[i + 1]))
+    promo = dict(threshold=thr, sticky=2, max_per_step=8)
+    cache = copy.deepcopy(base)
+    cache.promo = promo
+    dev = "cuda"
+    kr_ = np.full((B, Hkv, W_max, d), np.nan)
+    vr_ = np.full((B, Hkv, W_max, d), np.nan)
+    for h in range(Hkv):
+        kr_[0, h, :n_hot] = np.stack(hot_k[0][h])
+        vr_[0, h, :n_hot] = np.stack(hot_v[0][h])
+    k_hot = torch.from_numpy(kr_).half().to(dev)
+    v_hot = torch.from_numpy(vr_).half().to(dev)
+    hs = torch.zeros(B, dtype=torch.int32, device=dev)
+    hl = torch.full((B,), n_hot, dtype=torch.int32, device=dev)
+    cl = torch.full((B,), n_cold, dtype=torch.int32, device=dev)
+    gpool = torch.from_numpy(pool.reshape(n_pages, nb).copy()).to(dev)
+    tbl = torch.from_numpy(table).to(dev)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    used = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+    ws = torch.empty(tq.tq_monarch_workspace_bytes(ctx.handle, B, Hq, Hkv, max_pages, W_max, E),
+                     dtype=torch.uint8, device=dev)
+    cap = max_pages * 128
+    gpromo = dict(promo, cold_mask=torch.zeros((B, cap // 32), dtype=torch.int32, device=dev),
+                  counts=torch.zeros((B, cap), dtype=torch.uint8, device=dev),
+                  logits=torch.empty((B, Hq, cap), dtype=torch.float32, device=dev))
+    qd = torch.from_numpy(q).to(torch.float16).to(dev)
+    n_moved = 0
+    for s in range(steps):
+        hot_before = cache.hot_len(0)
+        ref, opened = cache.step(q, new_k[s], new_v[s], scale, np.inf)
+        tq.tq_monarch_step_promote(ctx.handle, qd, torch.from_numpy(new_k[s]).half().to(dev),
+                                   torch.from_numpy(new_v[s]).half().to(dev), k_hot, v_hot, hs, hl,
+                                   gpool, tbl, cl, float("inf"), window, E, gpromo, out, ws, Hkv,
+                                   cold_used=used)
+        torch.cuda.synchronize()
+        assert tq.tq_get_error(ctx.handle) == tq.TQ_OK
+        gm = gpromo["cold_mask"].cpu().numpy().view(np.uint32)
+        bits = np.unpackbits(gm[0].view(np.uint8), bitorder="little").astype(bool)
+        assert np.array_equal(bits, cache.cold_mask[0]), "moved-back mask, step %d" % s
+        assert np.array_equal(gpromo["counts"].cpu().numpy()[0].astype(np.int32), cache.counts[0])
+        assert hl.item() == cache.hot_len(0) and cl.item() == cache.cold_len[0] and hs.item() == 0
+        got = out.cpu().numpy().astype(np.float64)
+        for hq in range(Hq):
+            assert_close(got[0, hq], ref[0, hq], what="step %d head %d" % (s, hq))
+        moved = cache.hot_len(0) - hot_before - 1
+        kg = k_hot.float().cpu().numpy()
+        for h in range(Hkv):
+            for i in range(hot_before + 1, cache.hot_len(0)):
+                kk, vv = cache.hot[0][h][i]
+                for g_, w_ in ((kg[0, h, i], kk), (v_hot.float().cpu().numpy()[0, h, i], vv)):
+                    ulp = np.abs(np.spacing(np.float16(w_)).astype(np.float64))
+                    assert np.all(np.abs(g_ - w_) <= ulp), "moved-back row, step %d" % s
+        n_moved += moved
+    assert n_moved >= 5
