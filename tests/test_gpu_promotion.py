@@ -10,7 +10,8 @@ seeded tokens and queries (8 u + noise on most steps, -8 u on some, so that
 counts also reset).  Per step: ring start and lengths exact; the moved-back
 mask and the per-position counts exact; attention within 2e-3 + 1e-2 |ref|.
 The moved-back rows are n Pi^T c_hat rounded to fp16 on both sides (fp32 on
-the GPU, fp64 in the oracle): equal within one fp16 unit in the last place.
+the GPU, fp64 in the oracle): equal within one fp16 unit in the last place
+plus the fp32 sum's rounding error (moved_row_tol).
 Without eviction every hot row is compared; with eviction the evicted rows
 are compressed by each side, so outputs are compared only before the first
 eviction that takes a moved-back row."""
@@ -29,6 +30,18 @@ pytestmark = pytest.mark.gpu
 
 def f16(a):
     return np.float16(a).astype(np.float64)
+
+
+def moved_row_tol(row):
+    """Tolerance of a moved-back row, n Pi^T c_hat rounded to fp16, GPU
+    (fp32 sums of d products) against the oracle (fp64): one fp16 unit in the
+    last place, plus the fp32 accumulation's error, at most d * 2^-24 times
+    the sum of the products' magnitudes, which is taken as 2^-17 (d <= 128)
+    times the row's largest element (the products are of the order of the
+    row's entries; an entry that cancels to near zero keeps this absolute
+    error)."""
+    row = np.asarray(row, np.float64)
+    return np.abs(np.spacing(np.float16(row)).astype(np.float64)) + 2.0 ** -17 * np.abs(row).max()
 
 
 def run(O, d, G, steps, window, E, W_max, attractors, promo, mode="open", seed=3, n_cold=300,
@@ -163,8 +176,7 @@ def run(O, d, G, steps, window, E, W_max, attractors, promo, mode="open", seed=3
                         kk, vv = cache.hot[b][h][i]
                         if i in moved_rows[b]:
                             for g_, w_ in ((kg[b, h, slot], kk), (vg[b, h, slot], vv)):
-                                ulp = np.abs(np.spacing(np.float16(w_)).astype(np.float64))
-                                assert np.all(np.abs(g_ - w_) <= ulp), "moved-back row"
+                                assert np.all(np.abs(g_ - w_) <= moved_row_tol(w_)), "moved-back row"
                         else:
                             assert np.array_equal(kg[b, h, slot], kk)
                             assert np.array_equal(vg[b, h, slot], vv)
@@ -241,7 +253,7 @@ def test_tinyllama_shape_promotion(O):
     in the widest gap of the oracle's first-step weights among the largest
     ones (so no decision lies near it), sticky 2, up to 8 moves per step.
     Masks, counts, lengths and ring start exact after every step; outputs
-    within the decode tolerance; moved-back rows within one fp16 unit."""
+    within the decode tolerance; moved-back rows within moved_row_tol."""
     import copy
     import torch
     from compressed_kv_decode_b200 import workloads as W
@@ -338,7 +350,6 @@ def test_tinyllama_shape_promotion(O):
             for i in range(hot_before + 1, cache.hot_len(0)):
                 kk, vv = cache.hot[0][h][i]
                 for g_, w_ in ((kg[0, h, i], kk), (v_hot.float().cpu().numpy()[0, h, i], vv)):
-                    ulp = np.abs(np.spacing(np.float16(w_)).astype(np.float64))
-                    assert np.all(np.abs(g_ - w_) <= ulp), "moved-back row, step %d" % s
+                    assert np.all(np.abs(g_ - w_) <= moved_row_tol(w_)), "moved-back row, step %d" % s
         n_moved += moved
     assert n_moved >= 5
