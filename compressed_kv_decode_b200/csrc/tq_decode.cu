@@ -357,12 +357,29 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
     return;
   }
   const int bh = blockIdx.x, b = bh / p.Hkv, kvh = bh % p.Hkv;
+  if (p.fuse.k_new) {  // the step's token into its ring slot (the attention waits for this launch)
+    const int len = p.hot_len[b];
+    if (len > 0 && len <= p.W_max) {
+      int slot = hot_start_of(p, b) + len - 1;
+      if (slot >= p.W_max) slot -= p.W_max;
+      const size_t row = (static_cast<size_t>(bh) * p.W_max + slot) * D;
+      const __half* kn = static_cast<const __half*>(p.fuse.k_new) + static_cast<size_t>(bh) * D;
+      const __half* vn = static_cast<const __half*>(p.fuse.v_new) + static_cast<size_t>(bh) * D;
+      for (int i = threadIdx.x; i < 2 * D; i += blockDim.x) {
+        if (i < D) static_cast<__half*>(p.fuse.k_ring)[row + i] = kn[i];
+        else static_cast<__half*>(p.fuse.v_ring)[row + i - D] = vn[i - D];
+      }
+    }
+  }
   __shared__ __align__(16) float sq[G][D], sqr[G][D], sqs[G][D];
   __shared__ unsigned smax[2][G];
   __shared__ float sfac[2][G];
   const int tid = threadIdx.x;
+  // without cold pages (a call over the hot window alone) only the hot
+  // operands are needed: no rotation of the query
+  const bool cold = p.max_pages > 0;
   MatRows<D> mr;
-  matvec_prefetch<D>(p.rot, p.sp, mr);  // Pi and S Pi rows do not wait for the query
+  if (cold) matvec_prefetch<D>(p.rot, p.sp, mr);  // Pi and S Pi rows do not wait for the query
   if (tid < 2 * G) smax[tid / G][tid % G] = 0u;
   for (int i = tid; i < G * D; i += blockDim.x) {
     const int g = i / D, j = i % D;
@@ -370,7 +387,7 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
                              static_cast<tq_dtype>(p.q_dtype));
   }
   __syncthreads();
-  matvec_rows2<D, G>(mr, sq, sqr, sqs);  // q_rot = Pi q, q_s = (S Pi) q
+  if (cold) matvec_rows2<D, G>(mr, sq, sqr, sqs);  // q_rot = Pi q, q_s = (S Pi) q
   __syncthreads();
   // Cold keys: three 0/1 operand planes against 16-bit fixed-point query
   // weights (int8 hi, lo).  The key code is the index u = 2H + L of its level
@@ -388,7 +405,8 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   // warp reduction leaves one shared-memory atomic per warp and quantity
   for (int i = tid; i < G * D; i += blockDim.x) {
     const int g = i / D, j = i % D;
-    float a = fabsf(sqr[g][j]), c = fabsf(sqs[g][j]), e = fabsf(p.sl * sq[g][j]);
+    float a = cold ? fabsf(sqr[g][j]) : 0.0f, c = cold ? fabsf(sqs[g][j]) : 0.0f;
+    float e = fabsf(p.sl * sq[g][j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
@@ -407,7 +425,7 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
     const int wp = tid >> 5, ln = tid & 31;
     if (wp < G) {
       float a = 0.0f, b2 = 0.0f;
-      for (int j = ln; j < D; j += 32) {
+      for (int j = ln; j < D && cold; j += 32) {
         a += sqr[wp][j];
         b2 += sqs[wp][j];
       }
@@ -438,7 +456,7 @@ __global__ void __launch_bounds__(256) prep_kernel(Params p) {
   // reg holds k = 4 c' + j + 16 reg (j = byte), index 32 kappa + k of the plane
   // (coordinate, or sketch index for the QJL plane), column n = g' = head
   // 4 nt + g' / 2, part g' % 2 (hi, lo).
-  for (int idx = tid; idx < C::RC * 32; idx += blockDim.x) {
+  for (int idx = tid; idx < C::RC * 32 && cold; idx += blockDim.x) {
     const int r = idx >> 5, lane = idx & 31;
     const int reg = r & 1, nt = (r >> 1) % C::NT, pk = (r >> 1) / C::NT;
     const int plane = pk / C::KK, kap = pk % C::KK;
@@ -1144,8 +1162,9 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(Params p) {
   __shared__ float red[COMB_THREADS / 32][G];
   __shared__ float sM[2][G], sL[2][G];
   // Pi does not depend on the attention launch: stage it first, overlapping
-  // the tail of that launch
-  {
+  // the tail of that launch (a call without cold pages has no rotated sums)
+  const bool cold = p.max_pages > 0;
+  if (cold) {
     constexpr int PER = D * D / 4 / COMB_THREADS;
 #pragma unroll
     for (int i = 0; i < PER; ++i)
@@ -1258,8 +1277,10 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(Params p) {
   for (int g = sl; g < G; g += NSL) {
     const float* so = ssum + g * D;  // cold sums (domain 0)
     float oc = 0.0f;
+    if (cold) {
 #pragma unroll 16
-    for (int i = 0; i < D; ++i) oc = fmaf(spi[i * D + j], so[i], oc);
+      for (int i = 0; i < D; ++i) oc = fmaf(spi[i * D + j], so[i], oc);
+    }
     const float oh = ssum[(G + g) * D + j];
     const bool open = (mask >> g) & 1;
     const float Mc = sM[0][g], Mh = sM[1][g];

@@ -111,9 +111,12 @@ struct DecodeGate {
   int32_t* cold_used;
 };
 
-// Optional epilogue of the decode's combine: out += sigmoid(gate[h]) r (the
-// Tensor Cache memory read), and the ring start and length of the step copied
-// back to the caller's arrays.
+// Optional parts of a decode call that steps a ring (Tensor Cache): the prep
+// launch writes the step's token (fp16 rows of [B, Hkv, D]) into ring slot
+// (hot_start + hot_len - 1) mod W_max of its (batch, kv head) before the
+// attention reads the ring; the combine's epilogue adds sigmoid(gate[h]) r
+// (the memory read) and copies the ring start and length of the step back to
+// the caller's arrays.
 struct DecodeFuse {
   const float* r;         // [B, Hq, D]
   const float* gate;      // [Hq]
@@ -121,6 +124,10 @@ struct DecodeFuse {
   const int32_t* src_len;  // [B]
   int32_t* dst_start;
   int32_t* dst_len;  // [B]
+  const void* k_new;
+  const void* v_new;  // fp16 [B, Hkv, D], or null: no token to write
+  void* k_ring;
+  void* v_ring;  // fp16 [B, Hkv, W_max, D]
 };
 
 // Launchers (defined in the .cu files).  Return a tq_status.

@@ -6,16 +6,17 @@
 //   A <- lambda A + eta (k (x) v),   r = q A,   y = y_local + sigmoid(g) r.
 //
 // Launches, all on the caller's stream:
-//   update   one CTA per (sequence, kv head): the step's token enters the
-//            ring; when the ring is full the token it overwrites is first
-//            written into A; then r = q A (the updated A) for the group's
+//   update   D / 32 CTAs per (sequence, kv head), each 32 columns of A:
+//            when the ring is full the token the step's token will overwrite
+//            is written into A; then r = q A (the updated A) for the group's
 //            query heads.  One pass over A: read, update, write, and the
-//            partial products of the read.  The new ring start and length go
-//            to the workspace (the caller's arrays are read by every head).
+//            products of the read.  The new ring start and length go to the
+//            workspace (the caller's arrays are read by every CTA).
 //   decode   the split-K attention over the ring alone (prep, attention,
-//            combine), with the ring start and length of this step; the
-//            combine's epilogue adds sigmoid(g) r and writes the new ring
-//            start and length back
+//            combine), with the ring start and length of this step: prep
+//            writes the step's token into its slot (after every update CTA
+//            has read the token it replaces), the combine's epilogue adds
+//            sigmoid(g) r and writes the new ring start and length back
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -28,66 +29,65 @@
 namespace tq {
 namespace tcache {
 
+// Columns of A per update CTA: a (sequence, kv head) takes D / UPD_COLS CTAs,
+// each the whole read r_j = sum_i q_i A[i][j] of its columns (no reduction
+// across CTAs).
+constexpr int UPD_COLS = 32;
+
 template <int D, int G>
 __global__ void __launch_bounds__(256) update_kernel(const void* q, int q_dtype, int Hq, int Hkv,
-                                                     const __half* __restrict__ k_new,
-                                                     const __half* __restrict__ v_new,
-                                                     __half* k_ring, __half* v_ring, int W,
-                                                     const int32_t* ring_start,
+                                                     const __half* k_ring, const __half* v_ring,
+                                                     int W, const int32_t* ring_start,
                                                      const int32_t* ring_len, float* A,
                                                      const float* lambda, const float* eta,
                                                      float* r_out, int32_t* new_start,
                                                      int32_t* new_len, int* err) {
-  constexpr int NR = 256 / D;  // row phases
-  const int bh = blockIdx.x, b = bh / Hkv, kvh = bh % Hkv;
-  const int tid = threadIdx.x, j = tid % D, rp = tid / D;
-  __shared__ float sk[D], sv[D];
+  constexpr int NSPLIT = D / UPD_COLS;
+  constexpr int NR = 256 / UPD_COLS;  // row phases
+  constexpr int RPT = D / NR;         // rows per thread
+  const int bh = blockIdx.x / NSPLIT, cs = blockIdx.x % NSPLIT;
+  const int b = bh / Hkv, kvh = bh % Hkv;
+  const int tid = threadIdx.x, jl = tid % UPD_COLS, rp = tid / UPD_COLS;
+  const int j = cs * UPD_COLS + jl;
+  __shared__ float sk[D];
   __shared__ float sq[G][D];
-  __shared__ float part[NR][G][D];
+  __shared__ float part[NR][G][UPD_COLS];
   const int len = ring_len[b], start = ring_start[b];
   const bool ok = len >= 0 && len <= W && start >= 0 && start < W;
+  const bool lead = cs == 0 && kvh == 0 && tid == 0;  // one writer of the sequence's ring state
   if (!ok) {
     if (tid == 0) report(err, TQ_ERR_CAPACITY);
-    if (tid == 0 && kvh == 0) {
+    if (lead) {
       new_start[b] = 0;
       new_len[b] = 0;
     }
-    for (int i = tid; i < G * D; i += blockDim.x)
-      r_out[(static_cast<size_t>(b) * Hq + kvh * G + i / D) * D + i % D] = 0.0f;
+    if (tid < G * UPD_COLS)
+      r_out[(static_cast<size_t>(b) * Hq + kvh * G + tid / UPD_COLS) * D + cs * UPD_COLS +
+            tid % UPD_COLS] = 0.0f;
     return;
   }
+  // a full ring evicts its oldest token, whose slot the step's token takes
+  // (written by the decode's prep launch, after this one)
   const bool evict = len == W;
-  int slot = evict ? start : start + len;
-  if (slot >= W) slot -= W;
-  const size_t row = (static_cast<size_t>(bh) * W + (TQ_IN_RANGE(err, slot, W) ? slot : 0)) * D;
-  if (tid < D) {
-    sk[tid] = evict ? __half2float(k_ring[row + tid]) : 0.0f;
-    sv[tid] = evict ? __half2float(v_ring[row + tid]) : 0.0f;
-  }
+  const size_t row = (static_cast<size_t>(bh) * W + (TQ_IN_RANGE(err, start, W) ? start : 0)) * D;
+  if (tid < D) sk[tid] = evict ? __half2float(k_ring[row + tid]) : 0.0f;
   for (int i = tid; i < G * D; i += blockDim.x)
     sq[i / D][i % D] = load_as_float(q, (static_cast<size_t>(b) * Hq + kvh * G) * D + i,
                                      static_cast<tq_dtype>(q_dtype));
-  __syncthreads();  // the evicted row is read before the new token overwrites it
-  if (tid < D) {
-    k_ring[row + tid] = k_new[static_cast<size_t>(bh) * D + tid];
-    v_ring[row + tid] = v_new[static_cast<size_t>(bh) * D + tid];
-  }
-  if (tid == 0 && kvh == 0) {
+  if (lead) {
     new_start[b] = evict ? (start + 1 == W ? 0 : start + 1) : start;
     new_len[b] = evict ? W : len + 1;
   }
+  const float lam = lambda[kvh], et = eta[kvh];
+  const float evj = evict ? et * __half2float(v_ring[row + j]) : 0.0f;
   // A[i][j], i = key coordinate: this thread takes column j, rows rp, rp + NR,
-  // ...; all of its D / NR values are loaded before any arithmetic (the
-  // kernel has one CTA per group, so memory parallelism comes from here)
-  constexpr int RPT = D / NR;  // rows per thread
+  // ...; all of its values are loaded before any arithmetic
   float* Ab = A + static_cast<size_t>(bh) * D * D;
   float av[RPT];
 #pragma unroll
   for (int m = 0; m < RPT; ++m) av[m] = Ab[static_cast<size_t>(rp + NR * m) * D + j];
-  // a barrier keeps the compiler from sinking the loads past the stores below
+  // (the barrier also keeps the compiler from sinking the loads past the stores below)
   __syncthreads();
-  const float lam = lambda[kvh], et = eta[kvh];
-  const float evj = evict ? et * sv[j] : 0.0f;
   float acc[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) acc[g] = 0.0f;
@@ -103,14 +103,14 @@ __global__ void __launch_bounds__(256) update_kernel(const void* q, int q_dtype,
     for (int g = 0; g < G; ++g) acc[g] = fmaf(sq[g][i], a, acc[g]);
   }
 #pragma unroll
-  for (int g = 0; g < G; ++g) part[rp][g][j] = acc[g];
+  for (int g = 0; g < G; ++g) part[rp][g][jl] = acc[g];
   __syncthreads();
-  for (int i = tid; i < G * D; i += blockDim.x) {
-    const int g = i / D, jj = i % D;
+  for (int i = tid; i < G * UPD_COLS; i += blockDim.x) {
+    const int g = i / UPD_COLS, jj = i % UPD_COLS;
     float s = 0.0f;
 #pragma unroll
     for (int k = 0; k < NR; ++k) s += part[k][g][jj];
-    r_out[(static_cast<size_t>(b) * Hq + kvh * G + g) * D + jj] = s;
+    r_out[(static_cast<size_t>(b) * Hq + kvh * G + g) * D + cs * UPD_COLS + jj] = s;
   }
 }
 
@@ -143,15 +143,12 @@ int launch_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype,
   int32_t* nl = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ns) +
                                            tcache::align256(sizeof(int32_t) * B));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const __half* kn = static_cast<const __half*>(k_new);
-  const __half* vn = static_cast<const __half*>(v_new);
-  __half* kr = static_cast<__half*>(k_ring);
-  __half* vr = static_cast<__half*>(v_ring);
+  const __half* kr = static_cast<const __half*>(k_ring);
+  const __half* vr = static_cast<const __half*>(v_ring);
   const int qd = static_cast<int>(q_dtype);
 #define TQ_TC_LAUNCH(DD, GG)                                                                      \
-  tcache::update_kernel<DD, GG><<<B * Hkv, 256, 0, st>>>(q, qd, Hq, Hkv, kn, vn, kr, vr, W,       \
-                                                        ring_start, ring_len, A, lambda, eta, r,  \
-                                                        ns, nl, ctx->dev.err)
+  tcache::update_kernel<DD, GG><<<B * Hkv * (DD / tcache::UPD_COLS), 256, 0, st>>>(               \
+      q, qd, Hq, Hkv, kr, vr, W, ring_start, ring_len, A, lambda, eta, r, ns, nl, ctx->dev.err)
   if (d == 128) {
     switch (G) {
       case 1: TQ_TC_LAUNCH(128, 1); break;
@@ -173,8 +170,9 @@ int launch_tensor_cache_step(const tq_ctx* ctx, const void* q, tq_dtype q_dtype,
   }
 #undef TQ_TC_LAUNCH
   if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
-  // the combine adds sigmoid(g) r and writes the ring start and length back
-  const DecodeFuse fz{r, gate, ns, nl, ring_start, ring_len};
+  // prep writes the step's token into the ring; the combine adds sigmoid(g) r
+  // and writes the ring start and length back
+  const DecodeFuse fz{r, gate, ns, nl, ring_start, ring_len, k_new, v_new, k_ring, v_ring};
   return launch_decode(ctx, q, q_dtype, B, Hq, Hkv, scale, k_ring, v_ring, W, ns, nl, nullptr, 0,
                        nullptr, 0, nullptr, nullptr, out, ws, dec, stream, &fz);
 }
