@@ -158,7 +158,7 @@ __device__ __forceinline__ uint32_t level_code(float re, float ro, const float* 
 }
 
 template <int D, int B1, int B2>
-__global__ void __launch_bounds__(WARPS * 32, 1) polar_encode_kernel(const float* __restrict__ x,
+__global__ void __launch_bounds__(WARPS * 32, 4) polar_encode_kernel(const float* __restrict__ x,
                                                                   long long N,
                                                                   int code_bytes,
                                                                   uint8_t* __restrict__ codes,

@@ -521,7 +521,8 @@ TQ_API tq_status tq_self_index_attend(const tq_ctx* ctx, const void* q, tq_dtype
  *  x_rot   device fp32 [N, d] rotated vectors, 16-byte aligned.
  *  codes   device uint8 [N, tq_stage1_code_bytes(...)], 4-byte aligned (a
  *          record is a whole number of 32-bit words); norms device fp16 [N].
- *  x_hat   device fp32 [N, d] reconstruction in the rotated domain.
+ *  x_hat   device fp32 [N, d] reconstruction in the rotated domain, 16-byte
+ *          aligned.
  * Unsupported bit counts give TQ_ERR_UNSUPPORTED (and a code size of 0).
  */
 typedef enum { TQ_STAGE1_MSE = 0, TQ_STAGE1_POLAR = 1 } tq_stage1_kind;
