@@ -40,7 +40,7 @@ namespace dec {
 
 constexpr int NW = 12;        // warps per attention CTA
 constexpr int COLD_TOK = 64;  // tokens per cold unit (4 blocks, half a page)
-constexpr int HOT_TOK = 8;    // tokens per hot unit
+constexpr int HOT_TOK = 13;   // tokens per hot unit (K, V and a zero row fill a cold unit's slot)
 constexpr float NEG_INF = -__builtin_huge_valf();
 
 template <int D, int G>
@@ -60,7 +60,10 @@ struct Cfg {
   static constexpr int SLOT = ((COLD_B > HOT_B ? COLD_B : HOT_B) + 127) / 128 * 128;
   static constexpr int NSLOT = (D == 128) ? 2 : 3;
   static constexpr int PBUF = COLD_TOK * 16;  // fp16 P' tile [64 tokens][8 heads]
-  static constexpr int SMEM = NW * (NSLOT * SLOT + PBUF) + NW * NSLOT * 8 + NW * NSLOT * 4;
+  // one zero row (read for token rows past a hot unit), never written by copies
+  static constexpr int OFF_ZERO = (NW * (NSLOT * SLOT + PBUF) + NW * NSLOT * 8 + NW * NSLOT * 4 + 15) / 16 * 16;
+  static constexpr int SMEM = OFF_ZERO + HROW;
+  static_assert(HOT_TOK <= 16 && HOT_B <= COLD_B, "a hot unit fills at most a cold unit's slot");
 };
 
 constexpr int DESC_N = 6;
@@ -678,19 +681,6 @@ __device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1,
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// d += a * b, m16n8k8, fp16 inputs, fp32 accumulate
-__device__ __forceinline__ void mma_f16_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(b0));
-}
-
-__device__ __forceinline__ void ldsm_x1_t(uint32_t addr, uint32_t& r0) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x1.trans.shared.b16 {%0}, [%1];" : "=r"(r0) : "r"(addr));
-}
-
 // Value dequantisation table: entry e (a code byte: two 4-bit codes, the even
 // token's in the low nibble) = fp16 pair (v(e & 15), v(e >> 4)), v(code) =
 // (-1)^(code >> 3) fp16(c[code & 7]).  32 copies, copy L in bank L: lane L
@@ -716,6 +706,8 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
     const __half2 h2 = __floats2half2_rn(v0, v1);
     g_vlut[i] = *reinterpret_cast<const uint32_t*>(&h2);
   }
+  for (int i = threadIdx.x; i < C::HROW / 4; i += NW * 32)
+    reinterpret_cast<uint32_t*>(smem + C::OFF_ZERO)[i] = 0u;
   __syncthreads();
   pdl_wait();  // schedule and query operands come from the prep launch
   pdl_launch_dependents();
@@ -903,6 +895,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
   };
 
   const uint32_t pb_addr = smem_u32(pbuf);
+  const uint32_t zr_addr = smem_u32(smem + C::OFF_ZERO);
   const unsigned long long wait_ns = p.wait_ns ? p.wait_ns : 2000000000ull;
   const uint32_t msk = 0x01010101u << g;  // this lane's token in every plane byte
   const uint32_t l4 = static_cast<uint32_t>(lane) * 4u;
@@ -1044,49 +1037,55 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         }
       }
     } else {
-      // ---------------- hot unit: 8 tokens ----------------
+      // ---------------- hot unit: HOT_TOK tokens ----------------
+      // K rows then V rows; the MMAs read 16 token rows, and rows at or past
+      // nv (not copied, or past the unit) read the CTA's zero row
       const int nv = min(HOT_TOK, len - lu * HOT_TOK);
-      const uint8_t* kt = sb;
-      uint8_t* vt = sb + HOT_TOK * C::HROW;
-      if (nv < HOT_TOK) {  // rows past the window were not copied: zero them
-        for (int i = lane; i < (HOT_TOK - nv) * (C::HROW / 4); i += 32)
-          reinterpret_cast<uint32_t*>(vt + nv * C::HROW)[i] = 0u;
-        __syncwarp();
-      }
-      // scores: tokens on M (rows 8-15 read the V tile and are masked)
+      const uint32_t kt_addr = smem_u32(sb), vt_addr = kt_addr + HOT_TOK * C::HROW;
+      // scores: tokens on M; rows at or past nv are masked
       float acc[C::NT][4];
 #pragma unroll
       for (int nt = 0; nt < C::NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-      const uint32_t kt_addr = smem_u32(kt);
+      const int krow = (lane & 7) + ((lane >> 3) & 1) * 8;
+      const uint32_t krow_addr = krow < nv ? kt_addr + krow * C::HROW : zr_addr;
 #pragma unroll
       for (int s = 0; s < C::KS; ++s) {
-        const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
         const int col = 16 * s + (lane >> 4) * 8;
         uint32_t a0, a1, a2, a3;
-        ldsm_x4(kt_addr + row * C::HROW + col * 2, a0, a1, a2, a3);
+        ldsm_x4(krow_addr + col * 2, a0, a1, a2, a3);
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt)
           mma_f16(acc[nt], a0, a1, a2, a3, bfr[(s * C::NT + nt) * 2], bfr[(s * C::NT + nt) * 2 + 1]);
       }
-      float sv[C::NT];
+      // accumulator columns 2c, 2c + 1: the hi and lo parts of head c
+      float sv[C::NT * 2];
 #pragma unroll
-      for (int nt = 0; nt < C::NT; ++nt) sv[nt] = (g < nv) ? (acc[nt][0] + acc[nt][1]) * dsc[nt] : NEG_INF;
-      softmax_update(sv, 1);
+      for (int nt = 0; nt < C::NT; ++nt) {
+        sv[nt * 2] = (g < nv) ? (acc[nt][0] + acc[nt][1]) * dsc[nt] : NEG_INF;
+        sv[nt * 2 + 1] = (g + 8 < nv) ? (acc[nt][2] + acc[nt][3]) * dsc[nt] : NEG_INF;
+      }
+      softmax_update(sv, 2);
 #pragma unroll
       for (int nt = 0; nt < C::NT; ++nt) {
         const int h = c + 4 * nt;
-        if (h < G) reinterpret_cast<__half*>(pbuf)[g * 8 + h] = __float2half_rn(sv[nt]);
+        if (h < G) {
+          reinterpret_cast<__half*>(pbuf)[g * 8 + h] = __float2half_rn(sv[nt * 2]);
+          reinterpret_cast<__half*>(pbuf)[(g + 8) * 8 + h] = __float2half_rn(sv[nt * 2 + 1]);
+        }
       }
       __syncwarp();
-      uint32_t bp0;
-      ldsm_x1_t(pb_addr + (lane & 7) * 16, bp0);
-      const uint32_t vt_addr = smem_u32(vt);
+      // P V over 16 token rows: A = V^T (coordinates x tokens) by transposed
+      // loads of the V rows, B = the P' tile
+      uint32_t bp0, bp1;
+      ldsm_x2_t(pb_addr + (lane & 15) * 16, bp0, bp1);
+      const int vrow = (lane & 7) + ((lane >> 4) & 1) * 8;
+      const uint32_t vrow_addr = vrow < nv ? vt_addr + vrow * C::HROW : zr_addr;
 #pragma unroll
       for (int i = 0; i < C::KS; ++i) {
         const int col = 16 * i + ((lane >> 3) & 1) * 8;
-        uint32_t a0, a1;
-        ldsm_x2_t(vt_addr + (lane & 7) * C::HROW + col * 2, a0, a1);
-        mma_f16_k8(oacc[i], a0, a1, bp0);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(vrow_addr + col * 2, a0, a1, a2, a3);
+        mma_f16(oacc[i], a0, a1, a2, a3, bp0, bp1);
       }
     }
     // all lanes are done with this slot (every value read from it has been
