@@ -929,12 +929,13 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
         const uint8_t* bp = sb + mt * C::BLK;
-        // integer accumulators: key planes H and L, and the QJL plane
-        int ak[C::NT][4], aq[C::NT][4];
+        // integer accumulators: key planes H and L (two chains, added
+        // exactly at the end), and the QJL plane
+        int ak[C::NT][4], al[C::NT][4], aq[C::NT][4];
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) ak[nt][e] = aq[nt][e] = 0;
+          for (int e = 0; e < 4; ++e) ak[nt][e] = al[nt][e] = aq[nt][e] = 0;
 #pragma unroll
         for (int kap = 0; kap < C::KK; ++kap) {
           // words for indices 32 kap + 4c .. (tokens 0-7, 8-15) and 32 kap + 16 + 4c ..
@@ -947,10 +948,14 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
             const uint32_t* bL = bfr + ((1 * C::KK + kap) * C::NT + nt) * 2;
             const uint32_t* bQ = bfr + ((2 * C::KK + kap) * C::NT + nt) * 2;
             imma_u8s8(ak[nt], wh.x & msk, wh.y & msk, wh.z & msk, wh.w & msk, bH[0], bH[1]);
-            imma_u8s8(ak[nt], wl.x & msk, wl.y & msk, wl.z & msk, wl.w & msk, bL[0], bL[1]);
+            imma_u8s8(al[nt], wl.x & msk, wl.y & msk, wl.z & msk, wl.w & msk, bL[0], bL[1]);
             imma_u8s8(aq[nt], wq.x & msk, wq.y & msk, wq.z & msk, wq.w & msk, bQ[0], bQ[1]);
           }
         }
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) ak[nt][e] += al[nt][e];
         // (n, gamma) of tokens g and g + 8 of the block
         const uint32_t nk0 = *reinterpret_cast<const uint32_t*>(bp + C::OFF_NK + 4 * g);
         const uint32_t nk1 = *reinterpret_cast<const uint32_t*>(bp + C::OFF_NK + 4 * (g + 8));
@@ -1043,9 +1048,12 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
       const int nv = min(HOT_TOK, len - lu * HOT_TOK);
       const uint32_t kt_addr = smem_u32(sb), vt_addr = kt_addr + HOT_TOK * C::HROW;
       // scores: tokens on M; rows at or past nv are masked
-      float acc[C::NT][4];
+      // (two accumulator chains, even and odd k-steps, summed at the end)
+      float acc[C::NT][4], acc2[C::NT][4];
 #pragma unroll
-      for (int nt = 0; nt < C::NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+      for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = acc2[nt][e] = 0.0f;
       const int krow = (lane & 7) + ((lane >> 3) & 1) * 8;
       const uint32_t krow_addr = krow < nv ? kt_addr + krow * C::HROW : zr_addr;
 #pragma unroll
@@ -1054,9 +1062,16 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         uint32_t a0, a1, a2, a3;
         ldsm_x4(krow_addr + col * 2, a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < C::NT; ++nt)
-          mma_f16(acc[nt], a0, a1, a2, a3, bfr[(s * C::NT + nt) * 2], bfr[(s * C::NT + nt) * 2 + 1]);
+        for (int nt = 0; nt < C::NT; ++nt) {
+          const uint32_t b0 = bfr[(s * C::NT + nt) * 2], b1 = bfr[(s * C::NT + nt) * 2 + 1];
+          if (s & 1) mma_f16(acc2[nt], a0, a1, a2, a3, b0, b1);
+          else mma_f16(acc[nt], a0, a1, a2, a3, b0, b1);
+        }
       }
+#pragma unroll
+      for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] += acc2[nt][e];
       // accumulator columns 2c, 2c + 1: the hi and lo parts of head c
       float sv[C::NT * 2];
 #pragma unroll
