@@ -69,9 +69,20 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
 
 
+def source_sha(source):
+    """Hash of a CUDA source's code: comments and whitespace removed, so a
+    comment edit keeps a capture valid and any code change voids it."""
+    import re
+    with open(os.path.join(ROOT, source)) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()[:16]
+
+
 def kernel_traffic(kernel, source):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current source of the kernel; else None."""
+    the current code of the kernel's source; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -79,9 +90,7 @@ def kernel_traffic(kernel, source):
         rec = json.load(f).get(kernel)
     if not rec:
         return None
-    with open(os.path.join(ROOT, source), "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()[:16]
-    return rec["bytes_per_launch"] if rec.get("src_sha") == sha else None
+    return rec["bytes_per_launch"] if rec.get("src_sha") == source_sha(source) else None
 
 
 class ClockSampler:

@@ -7,15 +7,17 @@
 //
 // Three launches:
 //  1. prep      one CTA per (batch, kv head): q_rot = Pi q, q_s = S q_rot, the
-//               constants of the estimator folded in, split into fp16 hi/lo
-//               and laid out as the tensor-core B fragments each lane needs;
-//               one extra CTA builds the work schedule (units per segment,
-//               prefix sums, partial-record slots).
+//               constants of the estimator folded in, split into fixed-point
+//               (cold) and fp16 hi/lo (hot) parts and laid out as the
+//               tensor-core B fragments each lane needs (the cold ones only
+//               when the call has cold pages); one extra CTA builds the work
+//               schedule (units per segment, prefix sums, partial-record
+//               slots).
 //  2. attention persistent warps, each owning a contiguous range of work
-//               units (64 cold tokens = 4 page blocks, or 8 hot tokens).  A
+//               units (64 cold tokens = 4 page blocks, or 13 hot tokens).  A
 //               warp streams its units through a private ring of shared-memory
-//               slots, one 1-D bulk copy (TMA) per cold unit, completing on
-//               mbarriers.  Cold keys are scored with 8-bit integer MMAs
+//               slots, one 1-D bulk copy (TMA) per cold unit and one per hot
+//               row, completing on mbarriers.  Cold keys are scored with 8-bit integer MMAs
 //               (m16n8k32; tokens on M, q heads x {hi, lo} of 16-bit
 //               fixed-point query weights on N): the key planes H, L and the
 //               QJL plane hold 8 tokens per byte, so a lane's operand is its
