@@ -92,6 +92,19 @@ def test_ragged_lengths(O, d, G, qdt):
     check_case(O, c, d, what="ragged d=%d G=%d" % (d, G))
 
 
+@pytest.mark.parametrize("d,G", [(128, 4), (64, 8), (128, 1)])
+def test_hot_window_only(O, d, G):
+    """No cold pages (max_pages = 0: prep and combine skip the query
+    rotation); hot lengths around the 13-token hot unit (1, 12, 13, 14, 26,
+    40), NaN in the slots past hot_len."""
+    P = params_for(O, d)
+    Hkv = 2
+    hot = [1, 12, 13, 14, 26, 40]
+    c = build(O, P, len(hot), G * Hkv, Hkv, d, [0] * len(hot), hot, 48, 0, q_dtype="bfloat16",
+              n_out=2, factor=4.0, seed=3 * d + G)
+    check_case(O, c, d, what="hot only d=%d G=%d" % (d, G))
+
+
 def test_empty_sequence_gives_zeros(O):
     P = params_for(O, 128)
     c = build(O, P, 2, 8, 2, 128, [0, 200], [0, 5], 16, 2)

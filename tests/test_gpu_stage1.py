@@ -67,7 +67,8 @@ def distortion(x, xh, seed=9):
 
 
 @pytest.mark.parametrize("d,b1,b2", [(128, 4, 2), (64, 4, 2), (128, 3, 3), (128, 5, 1),
-                                     (64, 2, 2)])
+                                     (64, 2, 2), (128, 2, 1), (128, 5, 3), (64, 5, 3),
+                                     (64, 3, 1)])
 def test_polar_bit_exact(O, d, b1, b2):
     ctx = ctx_for(d)
     x = inputs(d, 2000, d + 10 * b1 + b2)
@@ -83,7 +84,7 @@ def test_polar_bit_exact(O, d, b1, b2):
     assert abs(g[0] - o[0]) <= 1e-3 * o[0] and abs(g[1] - o[1]) <= 1e-3 * o[1]
 
 
-@pytest.mark.parametrize("d,bits", [(128, 2), (128, 3), (128, 4), (64, 3)])
+@pytest.mark.parametrize("d,bits", [(128, 2), (128, 3), (128, 4), (64, 2), (64, 3), (64, 4)])
 def test_mse_codes_and_reconstruction(O, d, bits):
     ctx = ctx_for(d)
     P = O.Params(d, seed=0)
