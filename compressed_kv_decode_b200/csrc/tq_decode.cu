@@ -689,6 +689,14 @@ __device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1,
 // reads entry e at byte 128 e + 4 L, so a warp's lookups never conflict.
 __shared__ uint32_t g_vlut[256 * 32];
 
+// 2^x by the hardware approximation; results below 2^-126 flush to zero,
+// which a softmax weight next to its running maximum (weight 1) can take
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t vlut(const char* lut, uint32_t off) {
   return *reinterpret_cast<const uint32_t*>(lut + off);
 }
@@ -828,9 +836,9 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
         alpha[nt] = 1.0f;
         for (int i = 0; i < count_per_nt; ++i) sv[nt * count_per_nt + i] = 0.0f;
       } else {
-        alpha[nt] = exp2f(mrun[nt] - mnew);
+        alpha[nt] = ex2_ftz(mrun[nt] - mnew);
         for (int i = 0; i < count_per_nt; ++i) {
-          const float e = exp2f(sv[nt * count_per_nt + i] - mnew);
+          const float e = ex2_ftz(sv[nt * count_per_nt + i] - mnew);
           sv[nt * count_per_nt + i] = e;
           ps += e;
         }
@@ -1033,13 +1041,15 @@ __global__ void __launch_bounds__(NW * 32, 1) attn_kernel(Params p) {
           const uint4 v = *reinterpret_cast<const uint4*>(vb + 512 * q4);
           xw[4 * q4] = v.x; xw[4 * q4 + 1] = v.y; xw[4 * q4 + 2] = v.z; xw[4 * q4 + 3] = v.w;
         }
+        // table address of code byte j: 128 * byte + 4 lane, one 4-way byte
+        // dot product with a weight of 128 on byte j (sum < 2^15, exact)
 #pragma unroll
         for (int i = 0; i < C::KS; ++i) {
           const uint32_t x = xw[i];
-          const uint32_t a0 = vlut(lut, ((x << 7) & 0x7F80u) | l4);
-          const uint32_t a1 = vlut(lut, ((x >> 1) & 0x7F80u) | l4);
-          const uint32_t a2 = vlut(lut, ((x >> 9) & 0x7F80u) | l4);
-          const uint32_t a3 = vlut(lut, ((x >> 17) & 0x7F80u) | l4);
+          const uint32_t a0 = vlut(lut, __dp4a(x, 0x00000080u, l4));
+          const uint32_t a1 = vlut(lut, __dp4a(x, 0x00008000u, l4));
+          const uint32_t a2 = vlut(lut, __dp4a(x, 0x00800000u, l4));
+          const uint32_t a3 = vlut(lut, __dp4a(x, 0x80000000u, l4));
           mma_f16(oacc[i], a0, a1, a2, a3, bp0, bp1);
         }
       }
@@ -1293,9 +1303,13 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(Params p) {
   for (int g = sl; g < G; g += NSL) {
     const float* so = ssum + g * D;  // cold sums (domain 0)
     float oc = 0.0f;
-    if (cold) {
+    if (cold) {  // four partial sums: a quarter of the dependent chain each
+      float o4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 16
-      for (int i = 0; i < D; ++i) oc = fmaf(spi[i * D + j], so[i], oc);
+      for (int i = 0; i < D; i += 4)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o4[k] = fmaf(spi[(i + k) * D + j], so[i + k], o4[k]);
+      oc = (o4[0] + o4[1]) + (o4[2] + o4[3]);
     }
     const float oh = ssum[(G + g) * D + j];
     const bool open = (mask >> g) & 1;
