@@ -23,7 +23,8 @@
 //               QJL plane hold 8 tokens per byte, so a lane's operand is its
 //               token's bit of every byte, one AND.  Values are dequantised
 //               through a lane-replicated byte -> fp16 pair table in shared
-//               memory straight into m16n8k16 A fragments.  The warp keeps an
+//               memory (each address one byte dot product) straight into
+//               m16n8k16 A fragments.  The warp keeps an
 //               online softmax, accumulates P.V (cold values in the rotated
 //               domain) and writes one partial (m, l, o) per segment it
 //               touched.
