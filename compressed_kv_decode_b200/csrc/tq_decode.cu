@@ -24,10 +24,9 @@
 //               token's bit of every byte, one AND.  Values are dequantised
 //               through a lane-replicated byte -> fp16 pair table in shared
 //               memory (each address one byte dot product) straight into
-//               m16n8k16 A fragments.  The warp keeps an
-//               online softmax, accumulates P.V (cold values in the rotated
-//               domain) and writes one partial (m, l, o) per segment it
-//               touched.
+//               m16n8k16 A fragments.  The warp keeps an online softmax,
+//               accumulates P.V (cold values in the rotated domain) and
+//               writes one partial (m, l, o) per segment it touched.
 //  3. combine   per (batch, kv head): log-sum-exp merge of the cold partials,
 //               o_cold = Pi^T o_rot, merge with the hot partials, divide.
 #include <cuda_runtime.h>
